@@ -1,0 +1,235 @@
+"""Oracle: the TurboQuant hot path in plain fp64 NumPy (test infrastructure only).
+
+Write half (``quantize``), per row x in R^d:
+  1. n = ||x||; a row with n < 1e-10 is stored as all zeros
+     [0h-n0.github.io "ICLR 2026論文解説: TurboQuant", section "Step 1:
+     PolarQuant" (normalise onto the unit sphere, keep the norm) and section
+     "実装のポイント" (norm storage); the 1e-10 zero rule is the one in that
+     page's encoder sketch];
+  2. y = R (x / n), R = H_d D / sqrt(d)   [same page, "Step 1: PolarQuant"];
+  3. code_i = #{k : t_k < y_i}, yhat = c[code]   [Qiita TurboQuant explainer
+     (qiita.com/kai_kou), "Stage 1: PolarQuant", step 3 Lloyd-Max];
+  4. r = y - yhat, rho = ||r||; p = S r; bit_j = 1 iff p_j < 0  [Qiita
+     explainer, "Stage 2: QJL"; ai.spot.hk "Google TurboQuant", section
+     "無偏內積估計" (b-1 bits of MSE quantizer, then 1-bit QJL on the residual)];
+  5. store codes, sign bits, norm = n and rnorm = n * rho (fp32).
+
+Read half:
+  logit(q, k) = norm * <R q, yhat> + rnorm * sqrt(pi/2) / m * <S R q, z>,
+  z_j = +1 - 2 bit_j   [Qiita explainer, "Stage 2: QJL", the estimator
+  <q,k> ~ <q,k_mse> + ||residual|| sqrt(pi/2)/m <S q, sign(S residual)>];
+  dequant (PROD) x~ = R^T (norm * yhat + sqrt(pi/2)/m * rnorm * S^T z)
+  [ai.spot.hk, "無偏內積估計": E<y, Q^-1(Q(x))> = <y, x>];
+  dequant (MSE)  x~ = norm * R^T yhat  [Qiita explainer, "APIの構成"
+  (values compressed by the MSE stage alone)].
+
+Readings (each listed in the design doc):
+  * the residual lives in the rotated, unit-normalised domain, and rnorm is
+    stored in the original units (n * rho);
+  * y_i exactly on a threshold goes to the lower cell; p_j = 0 counts as
+    positive (bit 0); bit 1 means negative, as in the 0h-n0 encoder sketch;
+  * codes are an LSB-first bitstream per row, code i in bits [B i, B i + B);
+    sign j is bit (j mod 8) of byte j // 8;
+  * the logit carries no 1/sqrt(d) softmax scale.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+SQRT_HALF_PI = math.sqrt(math.pi / 2.0)
+ZERO_NORM = 1e-10
+
+
+# --------------------------------------------------------------------------
+# Rotation
+# --------------------------------------------------------------------------
+def sylvester_hadamard(d: int) -> np.ndarray:
+    """H_1 = [1], H_2d = [[H_d, H_d], [H_d, -H_d]]  [0h-n0 explainer,
+    "Step 1: PolarQuant", recursive Hadamard definition]."""
+    H = np.ones((1, 1))
+    base = np.array([[1.0, 1.0], [1.0, -1.0]])
+    while H.shape[0] < d:
+        H = np.kron(base, H)
+    return H
+
+
+def rotation_matrix(D: np.ndarray) -> np.ndarray:
+    """Dense R = H_d diag(D) / sqrt(d)."""
+    d = D.shape[0]
+    return sylvester_hadamard(d) * D.astype(np.float64)[None, :] / math.sqrt(d)
+
+
+def fwht(v: np.ndarray) -> np.ndarray:
+    """Unnormalised fast Walsh-Hadamard transform along the last axis, the
+    butterfly (a, b) -> (a + b, a - b) at strides 1, 2, 4, ...  [0h-n0
+    explainer, "実装のポイント" (butterfly structure, O(d log d))].
+    Equal to v @ H_d (H_d symmetric)."""
+    v = np.array(v, dtype=np.float64, copy=True)
+    d = v.shape[-1]
+    h = 1
+    while h < d:
+        w = v.reshape(v.shape[:-1] + (d // (2 * h), 2, h))
+        a = w[..., 0, :].copy()
+        b = w[..., 1, :].copy()
+        w[..., 0, :] = a + b
+        w[..., 1, :] = a - b
+        h *= 2
+    return v
+
+
+def rotate(v: np.ndarray, P) -> np.ndarray:
+    """Row-wise R v (v has rows of length d)."""
+    return np.asarray(v, dtype=np.float64) @ P.R.T
+
+
+def rotate_inverse(v: np.ndarray, P) -> np.ndarray:
+    """Row-wise R^T v."""
+    return np.asarray(v, dtype=np.float64) @ P.R
+
+
+# --------------------------------------------------------------------------
+# Packing
+# --------------------------------------------------------------------------
+def packed_sizes(d: int, b: int, m: int):
+    """Bytes per row: codes d (b-1) / 8, signs m / 8, plus two fp32 norms."""
+    return d * (b - 1) // 8, m // 8
+
+
+def pack_codes(codes: np.ndarray, B: int) -> np.ndarray:
+    """LSB-first bitstream: bit B*i + j of the row is bit j of code i."""
+    codes = np.asarray(codes, dtype=np.int64)
+    N, d = codes.shape
+    bits = ((codes[:, :, None] >> np.arange(B)[None, None, :]) & 1).astype(np.uint8)
+    return np.packbits(bits.reshape(N, d * B), axis=1, bitorder="little")
+
+
+def unpack_codes(packed: np.ndarray, d: int, B: int) -> np.ndarray:
+    bits = np.unpackbits(np.asarray(packed, dtype=np.uint8), axis=1, bitorder="little")
+    bits = bits[:, : d * B].reshape(-1, d, B).astype(np.int64)
+    return np.sum(bits << np.arange(B)[None, None, :], axis=2)
+
+
+def pack_signs(bits: np.ndarray) -> np.ndarray:
+    """Sign j is bit (j mod 8) of byte j // 8; bit 1 means negative."""
+    return np.packbits(np.asarray(bits, dtype=np.uint8), axis=1, bitorder="little")
+
+
+def unpack_signs(packed: np.ndarray, m: int) -> np.ndarray:
+    bits = np.unpackbits(np.asarray(packed, dtype=np.uint8), axis=1, bitorder="little")
+    return bits[:, :m].astype(np.int64)
+
+
+# --------------------------------------------------------------------------
+# Write half
+# --------------------------------------------------------------------------
+def bucketize(y: np.ndarray, thresholds: np.ndarray) -> np.ndarray:
+    """code = number of thresholds strictly below y (ties go to the lower cell)."""
+    return np.sum(y[..., None] > thresholds, axis=-1)
+
+
+def quantize(x: np.ndarray, P, *, keep_intermediates: bool = False, codes_override=None):
+    """TurboQuant_prod write half for rows x (N, d), values exactly as the
+    kernel reads them (bf16 or fp32 inputs widened to fp64).
+
+    Returns a dict with packed ``codes`` (N, d B / 8) u8, ``signs`` (N, m / 8)
+    u8, ``norm`` and ``rnorm`` (N,) fp32; with ``keep_intermediates`` also the
+    fp64 ``y``, ``code``, ``p``, ``bits``, ``n`` and ``rho``.
+
+    ``codes_override`` lets a test fix the codes of some rows (values chosen
+    by the test, e.g. the other side of a threshold within the tie band) to
+    see what the residual stage gives for them; it is never fed kernel output.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    N = x.shape[0]
+    n = np.sqrt(np.sum(x * x, axis=1))
+    zero = n < ZERO_NORM
+    safe = np.where(zero, 1.0, n)
+    u = x / safe[:, None]
+    y = rotate(u, P)
+    code = bucketize(y, P.thresholds) if codes_override is None else np.asarray(codes_override)
+    yhat = P.centroids[code]
+    r = y - yhat
+    rho = np.sqrt(np.sum(r * r, axis=1))
+    p = r @ P.S.T
+    bits = (p < 0).astype(np.int64)
+    code = np.where(zero[:, None], 0, code)
+    bits = np.where(zero[:, None], 0, bits)
+    out = {
+        "codes": pack_codes(code, P.B),
+        "signs": pack_signs(bits),
+        "norm": np.where(zero, 0.0, n).astype(np.float32),
+        "rnorm": np.where(zero, 0.0, n * rho).astype(np.float32),
+    }
+    if keep_intermediates:
+        out.update(y=y, code=code, p=p, bits=bits, n=n, rho=rho, zero=zero)
+    return out
+
+
+# --------------------------------------------------------------------------
+# Read half
+# --------------------------------------------------------------------------
+def decode(packed: dict, P):
+    """yhat (N, d) from the codes and z (N, m) in {+1, -1} from the signs."""
+    code = unpack_codes(packed["codes"], P.d, P.B)
+    yhat = P.centroids[code]
+    z = 1.0 - 2.0 * unpack_signs(packed["signs"], P.m)
+    return yhat, z
+
+
+def qjl_correction(sq: np.ndarray, z: np.ndarray, rnorm, m: int) -> np.ndarray:
+    """||residual|| * sqrt(pi/2) / m * <S q, sign(S residual)>, for every
+    (query row of ``sq``, key row of ``z``) pair; z_j = +-1."""
+    return (np.asarray(rnorm, dtype=np.float64) * (SQRT_HALF_PI / m)) * (sq @ z.T)
+
+
+def query_prep(q: np.ndarray, P):
+    """q_rot = R q and sq = S q_rot, once per query."""
+    q_rot = rotate(q, P)
+    return q_rot, q_rot @ P.S.T
+
+
+def logits(q: np.ndarray, packed: dict, P, n_sets: int, g: int, n_keys: int) -> np.ndarray:
+    """Estimated <q, k> for every query of a set against every key of that set.
+
+    q: (n_sets * g, d) rows, query j of set s at row s * g + j.
+    packed: rows of set s at [s * n_keys, (s + 1) * n_keys).
+    Returns (n_sets, g, n_keys) fp64."""
+    yhat, z = decode(packed, P)
+    norm = np.asarray(packed["norm"], dtype=np.float64)
+    rnorm = np.asarray(packed["rnorm"], dtype=np.float64)
+    q_rot, sq = query_prep(np.asarray(q, dtype=np.float64).reshape(n_sets * g, P.d), P)
+    out = np.empty((n_sets, g, n_keys))
+    for s in range(n_sets):
+        ks = slice(s * n_keys, (s + 1) * n_keys)
+        qs = slice(s * g, (s + 1) * g)
+        mse = q_rot[qs] @ yhat[ks].T
+        out[s] = norm[ks][None, :] * mse + qjl_correction(sq[qs], z[ks], rnorm[ks], P.m)
+    return out
+
+
+DEQUANT_PROD = 0
+DEQUANT_MSE = 1
+
+
+def dequant(packed: dict, P, mode: int = DEQUANT_PROD) -> np.ndarray:
+    """Reconstructed rows (N, d) fp64.
+    PROD: R^T (norm * yhat + sqrt(pi/2)/m * rnorm * S^T z).
+    MSE:  R^T (norm * yhat)."""
+    yhat, z = decode(packed, P)
+    norm = np.asarray(packed["norm"], dtype=np.float64)
+    rnorm = np.asarray(packed["rnorm"], dtype=np.float64)
+    v = norm[:, None] * yhat
+    if mode == DEQUANT_PROD:
+        v = v + (SQRT_HALF_PI / P.m) * rnorm[:, None] * (z @ P.S)
+    return rotate_inverse(v, P)
+
+
+def topk(scores: np.ndarray, k: int):
+    """Per row, the k largest scores, larger first, equal scores by lower
+    index first.  Returns (idx int32, val)."""
+    scores = np.asarray(scores)
+    order = np.argsort(-scores, axis=1, kind="stable")[:, :k]
+    return order.astype(np.int32), np.take_along_axis(scores, order, axis=1)
