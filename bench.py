@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""TurboQuant hot-path benchmark on B200.
+
+One step = one pass of the whole hot path over one batch of the long-context
+decode workload at d = 128, b = 3 (2-bit Lloyd-Max + 1-bit QJL, m = 128):
+batch 8 x 8 KV heads x 131072 tokens of bf16 K and V (per-channel log-uniform
+scales), 32 query heads (GQA 4):
+
+    tq_quantize(K)  tq_quantize(V)  tq_logits(Q, packed K)  tq_dequant(packed V)
+
+`value` is compressed-key logits per second of the whole step (all ranks);
+per-kernel times, the quantize rows/s and the bf16 unquantized-key baseline
+kernel on the same shapes are reported beside it.  Inputs (2.1 GB per K/V
+tensor) are larger than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_vector_15_b200 import inputs  # noqa: E402
+
+WORKLOADS = {
+    # long-context decode at the headline bit width (the metric's d = 128, b = 3)
+    "decode-128k-b3": dict(batch=8, ctx=131072, b=3, m=128, kv_heads=8, q_heads=32, d=128),
+    "decode-128k-b4": dict(batch=8, ctx=131072, b=4, m=128, kv_heads=8, q_heads=32, d=128),
+    "decode-8k-b3": dict(batch=1, ctx=8192, b=3, m=128, kv_heads=8, q_heads=32, d=128),
+}
+METRIC = "compressed-key logits/s and % HBM roofline (d=128,b=3); quantize rows/s"
+UNIT = "logits/s"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(ws, v: float) -> float:
+    if ws == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline): a bounded sample of the workload
+# ---------------------------------------------------------------------------
+def oracle_sample_step(cfg, n_keys: int):
+    """One step of the hot path on the oracle for 1 (batch, kv head) set and
+    n_keys tokens: quantize K and V rows, logits for the set's g queries,
+    dequant V.  Returns (logits computed, seconds)."""
+    from oracle import params as op
+    from oracle import turboquant as ot
+    K, V, Q = inputs.decode(cfg["batch"], cfg["ctx"], kv_heads=cfg["kv_heads"], q_heads=cfg["q_heads"])
+    g = cfg["q_heads"] // cfg["kv_heads"]
+    k = K.as_f32(K.rows(0, n_keys)).astype(np.float64)
+    v = V.as_f32(V.rows(0, n_keys)).astype(np.float64)
+    q = Q.as_f32(Q.rows(0, g)).astype(np.float64)
+    P = op.Params(cfg["d"], cfg["b"], cfg["m"], seed=0)
+    t0 = time.perf_counter()
+    pk = ot.quantize(k, P)
+    pv = ot.quantize(v, P)
+    ot.logits(q, pk, P, 1, g, n_keys)
+    ot.dequant(pv, P, ot.DEQUANT_PROD)
+    return g * n_keys, time.perf_counter() - t0
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, cfg, ws, rank):
+    if rank != 0:
+        return
+    n_keys = 8192
+    for _ in range(args.warmup):
+        oracle_sample_step(cfg, n_keys)
+    total_units, total_t = 0, 0.0
+    for _ in range(args.steps):
+        u, t = oracle_sample_step(cfg, n_keys)
+        total_units += u
+        total_t += t
+    value = total_units / total_t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, **cfg},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": f"1 (batch, kv head) set x {n_keys} tokens per step: quantize K and V, "
+                                   f"logits for its 4 query heads, PROD dequant of V"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# CUDA path
+# ---------------------------------------------------------------------------
+def run_ours(args, cfg, ws, rank, local):
+    import torch
+    from kv_cache_vector_15_b200 import tq
+
+    d, b, m = cfg["d"], cfg["b"], cfg["m"]
+    n_sets = cfg["batch"] * cfg["kv_heads"]
+    g = cfg["q_heads"] // cfg["kv_heads"]
+    n_keys = cfg["ctx"]
+    N = n_sets * n_keys
+    dev = torch.device("cuda", local)
+    T = tq.TurboQuant(d, b, m, seed=0)
+
+    # seeded inputs, drawn on the host into pinned buffers (also the e2e source)
+    K, V, Q = inputs.decode(cfg["batch"], cfg["ctx"], kv_heads=cfg["kv_heads"], q_heads=cfg["q_heads"])
+    hK = torch.empty((N, d), dtype=torch.bfloat16, pin_memory=True)
+    hV = torch.empty((N, d), dtype=torch.bfloat16, pin_memory=True)
+    hQ = torch.empty((n_sets * g, d), dtype=torch.bfloat16, pin_memory=True)
+    K.fill(hK.view(torch.int16).numpy().view(np.uint16))
+    V.fill(hV.view(torch.int16).numpy().view(np.uint16))
+    Q.fill(hQ.view(torch.int16).numpy().view(np.uint16))
+    dK, dV, dQ = hK.to(dev), hV.to(dev), hQ.to(dev)
+    pK, pV = T.empty_packed(N, dev), T.empty_packed(N, dev)
+    logits = torch.empty((n_sets, g, n_keys), dtype=torch.float32, device=dev)
+    vhat = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
+    wbytes = T.workspace_bytes(n_sets, g)
+    work = torch.empty(max(wbytes, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        T.quantize(dK, pK, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        T.quantize(dV, pV, stream=stream)
+        if ev:
+            ev[2].record(stream)
+        T.logits(dQ, pK, n_sets, g, n_keys, out=logits, workspace=work, stream=stream)
+        if ev:
+            ev[3].record(stream)
+        T.dequant(pV, N, out=vhat, stream=stream)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(ws)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    launches0 = tq.launch_count()
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize(dev)
+        barrier(ws)
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(ws)
+    launches = tq.launch_count() - launches0
+    elapsed_ms = max_over_ranks(ws, start.elapsed_time(end))
+    ms_step = elapsed_ms / args.steps
+    per = {"quantize_K": [], "quantize_V": [], "logits": [], "dequant": []}
+    for e in evs:
+        per["quantize_K"].append(e[0].elapsed_time(e[1]))
+        per["quantize_V"].append(e[1].elapsed_time(e[2]))
+        per["logits"].append(e[2].elapsed_time(e[3]))
+        per["dequant"].append(e[3].elapsed_time(e[4]))
+    avg = {k: sum(v) / len(v) for k, v in per.items()}
+    n_logits = n_sets * g * n_keys
+    value = ws * n_logits / (ms_step * 1e-3)
+
+    hbm, hbm_kind = peaks()
+    P = T.row_bytes
+    alg = {  # algorithmic bytes per launch
+        "quantize": N * (2 * d + P),
+        "logits": N * (P + 4 * g),
+        "dequant": N * (P + 2 * d),
+    }
+    q_ms = (avg["quantize_K"] + avg["quantize_V"]) / 2
+    kern = {
+        "quantize": {"ms": q_ms, "launches_per_step": 2, "bytes": alg["quantize"]},
+        "logits": {"ms": avg["logits"], "launches_per_step": 2, "bytes": alg["logits"]},
+        "dequant": {"ms": avg["dequant"], "launches_per_step": 1, "bytes": alg["dequant"]},
+    }
+    for k, v in kern.items():
+        v["gbs"] = v["bytes"] / (v["ms"] * 1e-3) / 1e9
+        v["frac_hbm"] = v["gbs"] / hbm
+    dominant = max(kern, key=lambda k: kern[k]["ms"] * (2 if k == "quantize" else 1))
+    dk = kern[dominant]
+
+    # bf16 unquantized-key logits on the same shapes (comparison point)
+    bf16_out = torch.empty_like(logits)
+    for _ in range(3):
+        tq.logits_bf16(dQ, dK, n_sets, g, n_keys, out=bf16_out, stream=stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    e0.record(stream)
+    for _ in range(reps):
+        tq.logits_bf16(dQ, dK, n_sets, g, n_keys, out=bf16_out, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    bf16_ms = e0.elapsed_time(e1) / reps
+    bf16_bytes = N * (2 * d + 4 * g)
+
+    # end to end through the public API with host buffers
+    hL = torch.empty((n_sets, g, n_keys), dtype=torch.float32, pin_memory=True)
+    hVh = torch.empty((N, d), dtype=torch.bfloat16, pin_memory=True)
+
+    def e2e_step():
+        dK.copy_(hK, non_blocking=True)
+        dV.copy_(hV, non_blocking=True)
+        dQ.copy_(hQ, non_blocking=True)
+        step()
+        hL.copy_(logits, non_blocking=True)
+        hVh.copy_(vhat, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(ws)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(ws, e0.elapsed_time(e1)) / e2e_steps
+    h2d = (hK.numel() + hV.numel() + hQ.numel()) * 2
+    d2h = hL.numel() * 4 + hVh.numel() * 2
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if ws == 1 and not args.no_cpu_baseline:
+            n_keys_cpu = 16384
+            units, secs = oracle_sample_step(cfg, n_keys_cpu)
+            cpu = {"value": units / secs, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                   "sample": f"1 (batch, kv head) set x {n_keys_cpu} tokens: quantize K and V, logits for its "
+                             f"{g} query heads, PROD dequant of V ({secs:.1f} s)"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": args.workload, "batch": cfg["batch"], "kv_heads": cfg["kv_heads"],
+                       "q_heads": cfg["q_heads"], "ctx": cfg["ctx"], "d": d, "b": b, "m": m,
+                       "parallelism": f"dp{ws} (independent (batch, kv head) sets per rank)",
+                       "l2": "inputs larger than L2 (K, V 2.1 GB each); no flush"},
+            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dk["gbs"], "peak": hbm,
+                         "unit": "GB/s", "frac": dk["frac_hbm"], "traffic": None,
+                         "peak_kind": hbm_kind},
+            "quantize_rows_per_s": ws * N / (q_ms * 1e-3),
+            "kernels": {k: {"ms_per_launch": v["ms"], "algorithmic_GBps": v["gbs"], "frac_hbm": v["frac_hbm"],
+                            "bytes_per_launch": v["bytes"]} for k, v in kern.items()},
+            "bf16_key_logits_baseline": {"ms": bf16_ms, "algorithmic_GBps": bf16_bytes / (bf16_ms * 1e-3) / 1e9,
+                                         "tq_logits_speedup": bf16_ms / avg["logits"]},
+            "cpu_baseline": cpu,
+            "e2e": {"value": ws * n_logits / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    T.close()
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="decode-128k-b3", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, cfg, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        return
+    ws, rank, local = dist_setup()
+    try:
+        run_ours(args, cfg, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,175 @@
+/*
+ * tq.h -- C ABI of libtq, the TurboQuant KV-cache / vector quantization hot
+ * path for NVIDIA B200 (sm_100a).
+ *
+ * TurboQuant compresses a row x in R^d in two stages and reads the result
+ * back without decompressing it:
+ *
+ *   write half (tq_quantize)
+ *     n = ||x||, u = x / n                       -- 0h-n0.github.io "ICLR 2026論文解説:
+ *                                                   TurboQuant", section "Step 1: PolarQuant"
+ *     y = R u, R = H_d D / sqrt(d)               -- same section (randomized Hadamard
+ *                                                   transform, Rademacher D)
+ *     code_i = #{k : t_k < y_i}, yhat = c[code]  -- Qiita TurboQuant explainer, section
+ *                                                   "Stage 1: PolarQuant" (Lloyd-Max)
+ *     r = y - yhat; bit_j = [ (S r)_j < 0 ]      -- Qiita explainer, section "Stage 2: QJL";
+ *                                                   ai.spot.hk "Google TurboQuant", section
+ *                                                   "無偏內積估計" ((b-1)-bit MSE + 1-bit QJL)
+ *     store codes, sign bits, norm = n, rnorm = n ||r||
+ *
+ *   read half
+ *     tq_logits:  <q,k> ~ norm <R q, yhat> + rnorm sqrt(pi/2)/m <S R q, z>,  z_j = 1 - 2 bit_j
+ *                 -- Qiita explainer, "Stage 2: QJL" (the estimator formula)
+ *     tq_dequant: x~ = R^T (norm yhat + sqrt(pi/2)/m rnorm S^T z)   (PROD, unbiased:
+ *                 ai.spot.hk "無偏內積估計") or x~ = norm R^T yhat (MSE, Qiita "APIの構成")
+ *
+ * Conventions for every call
+ *   - Tensor pointers are DEVICE pointers owned by the caller, unless a
+ *     parameter says "host".  The library never frees them.
+ *   - Compute calls are asynchronous on the CUDA stream passed as `stream`
+ *     (a cudaStream_t; NULL = legacy default stream) and allocate nothing.
+ *   - Arguments are checked on the host before any launch.  A failed check
+ *     returns a status and launches nothing; tq_last_error() then gives a
+ *     one-line reason (thread-local, valid until the next call on the thread).
+ *   - n_rows == 0 (or n_keys == 0, n_sets == 0) is a no-op returning TQ_OK.
+ *   - Inputs must be finite and ||x||^2 must be finite in fp32; the output
+ *     for other inputs is unspecified (no fault: every access stays in bounds).
+ *   - A tq_ctx is immutable after tq_init; one context may be used from
+ *     several host threads and streams at once.  It belongs to the device
+ *     that was current at tq_init; calls must be made with that device current.
+ *
+ * Packed row format (all little-endian, one array per field, row r at r * bytes):
+ *   codes  d (b-1) / 8 bytes: LSB-first bitstream, code i in bits [B i, B i + B), B = b - 1
+ *   signs  m / 8 bytes: sign j is bit (j mod 8) of byte j / 8; 1 = negative projection
+ *   norm   fp32 n;  rnorm fp32 n * ||r||.   A row with n < 1e-10 is stored as all zeros.
+ * At d = 128, m = 128 a row takes 40 / 56 / 72 bytes for b = 2 / 3 / 4.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or enum */
+  TQ_ERR_UNSUPPORTED = 2,  /* valid request outside what this build implements */
+  TQ_ERR_NOMEM = 3,        /* device or host allocation failed (tq_init only) */
+  TQ_ERR_CUDA = 4          /* a CUDA runtime call or launch failed; see tq_last_error() */
+} tq_status;
+
+typedef enum { TQ_BF16 = 0, TQ_F32 = 1 } tq_dtype;
+typedef enum { TQ_DEQUANT_PROD = 0, TQ_DEQUANT_MSE = 1 } tq_dequant_mode;
+
+typedef struct tq_ctx tq_ctx;
+
+/* Caller-owned device arrays of one packed batch (row r at codes + r*codes_bytes
+ * etc.).  codes and signs must be 16-byte aligned; norm and rnorm 4-byte aligned. */
+typedef struct {
+  uint8_t* codes;
+  uint8_t* signs;
+  float* norm;
+  float* rnorm;
+} tq_packed;
+
+/* ---------------------------------------------------------------- setup -- */
+
+/* Derive the method's fixed parameters on the host, without any CUDA call.
+ *   d     power of two in [32, 4096]; b in [2, 5] (b-1 MSE bits + 1 QJL bit);
+ *   m     multiple of 32 in [32, 4096]; seed any 64-bit value.
+ * Outputs (host arrays, any may be NULL):
+ *   centroids[2^(b-1)] ascending fp32 Lloyd-Max levels for one rotated coordinate,
+ *   thresholds[2^(b-1)-1] fp32 midpoints,
+ *   D[d] int8 +-1 (Rademacher diagonal), S_bits[m*d] binary16 bit patterns of
+ *   the Gaussian projection, row-major (row j = projection j).
+ * The codebook is the Lloyd-Max fixed point for the exact law of a coordinate
+ * of a uniform unit vector, f_d(x) ~ (1-x^2)^((d-3)/2) (ai.spot.hk,
+ * "隨機旋轉與Beta分佈": rotated coordinates follow one Beta law).  D and S come
+ * from SplitMix64 used as a counter generator (stream 0: D, stream 1: S,
+ * Box-Muller, rounded once to binary16). */
+tq_status tq_host_params(int d, int b, int m, uint64_t seed, float* centroids, float* thresholds,
+                         int8_t* D, uint16_t* S_bits);
+
+/* Create a context on the current device: derives the parameters as above
+ * and uploads them (the only host->device copy of parameters).  Requires a
+ * compute capability 10.x device.  *out receives the context. */
+tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out);
+
+/* Free a context's device memory.  The caller must make sure no work that
+ * uses it is still in flight.  NULL is accepted. */
+tq_status tq_destroy(tq_ctx* ctx);
+
+/* Bytes per array for n_rows packed rows (norm and rnorm take 4 * n_rows each). */
+tq_status tq_packed_sizes(const tq_ctx* ctx, int64_t n_rows, size_t* codes_bytes, size_t* signs_bytes);
+
+/* Host copies of the context's parameters (formats as tq_host_params; any may be NULL). */
+tq_status tq_get_params(const tq_ctx* ctx, float* centroids, float* thresholds, int8_t* D, uint16_t* S_bits);
+
+/* ---------------------------------------------------------- write half -- */
+
+/* Quantize n_rows rows of x (row r at x + r * ld_x elements, dtype bf16 or
+ * fp32, ld_x >= d, x and ld_x * element size 16-byte aligned) into `out`.
+ * Per row: norm, rotation, Lloyd-Max codes, QJL signs of the residual,
+ * residual norm (write half above).  One launch. */
+tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
+                      tq_packed out, void* stream);
+
+/* ----------------------------------------------------------- read half -- */
+
+/* Device workspace that tq_logits needs for n_sets * g queries (bytes; 0 when
+ * the call needs none, in which case workspace may be NULL). */
+size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g);
+
+/* Estimated logits of queries against packed keys (estimator above; no
+ * 1/sqrt(d) softmax scale).
+ *   q     [n_sets, g, d] bf16 or fp32 (query j of set s at row s*g + j), 16-byte aligned;
+ *   keys  packed rows, set s at rows [s*n_keys, (s+1)*n_keys);
+ *   out   [n_sets, g, n_keys] fp32.
+ * For grouped-query attention a set is one (batch, kv head) pair and g the
+ * number of query heads sharing it; for vector search n_sets = 1 and g the
+ * number of queries.  g in [1, 4096].  workspace: device memory of at least
+ * tq_logits_workspace_bytes(ctx, n_sets, g) bytes, 16-byte aligned, not used
+ * concurrently by another call. */
+tq_status tq_logits(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
+                    tq_packed keys, int64_t n_keys, float* out, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/* Reconstruct n_rows packed rows into out [n_rows, d] (bf16 or fp32,
+ * contiguous, 16-byte aligned).  mode PROD adds the QJL term (unbiased),
+ * MSE uses the codes alone. */
+tq_status tq_dequant(const tq_ctx* ctx, tq_packed in, int64_t n_rows, void* out, tq_dtype out_dtype,
+                     tq_dequant_mode mode, void* stream);
+
+/* Per row of scores [rows, cols] fp32, the k largest values, larger first,
+ * equal values by lower column index first.  idx [rows, k] int32 and
+ * val [rows, k] fp32 (val may be NULL).  k in [1, 64], k <= cols. */
+tq_status tq_topk(const float* scores, int64_t rows, int64_t cols, int k, int32_t* idx, float* val,
+                  void* stream);
+
+/* ------------------------------------------------------------ baseline -- */
+
+/* Plain unquantized-key logits, the comparison point for tq_logits:
+ * out[s, j, t] = <q[s, j], k[s, t]> with bf16 q [n_sets, g, d], bf16 keys
+ * [n_sets, n_keys, d] (contiguous, 16-byte aligned), fp32 accumulation,
+ * fp32 out [n_sets, g, n_keys].  d in {64, 128, 256}, g in [1, 8], n_sets <= 65535. */
+tq_status tq_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, int d,
+                         float* out, void* stream);
+
+/* ----------------------------------------------------------- reporting -- */
+
+const char* tq_status_str(tq_status s);
+/* One-line reason for the last non-OK status returned on this host thread. */
+const char* tq_last_error(void);
+/* Number of kernel launches this library has issued in this process (all
+ * threads), for launch accounting in benchmarks. */
+uint64_t tq_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

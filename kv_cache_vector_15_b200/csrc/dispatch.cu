@@ -1,0 +1,22 @@
+// Kernel selection: the d = 128 hot-path kernels where they apply, the
+// general kernels everywhere else.
+#include "tq_internal.h"
+
+namespace tq {
+
+int launch_quantize(const KParams& P, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x, const Packed& out,
+                    void* stream) {
+  return launch_quantize_generic(P, x, x_is_bf16, n_rows, ld_x, out, stream);
+}
+
+int launch_logits(const KParams& P, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
+                  float* out, void* stream) {
+  return launch_logits_generic(P, qp, n_sets, g, keys, n_keys, out, stream);
+}
+
+int launch_dequant(const KParams& P, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
+                   void* stream) {
+  return launch_dequant_generic(P, in, n_rows, out, out_is_bf16, prod, stream);
+}
+
+}  // namespace tq

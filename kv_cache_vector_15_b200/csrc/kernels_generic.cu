@@ -1,0 +1,744 @@
+// General CUDA-core kernels of libtq: every (d, b, m) the C ABI accepts.
+//
+// These are the reference-shaped kernels for all supported shapes:
+//   k_quantize_warp  write half, one warp per row (norm, RHT, Lloyd-Max codes,
+//                    residual, QJL projection and signs, packing)
+//   k_qprep_warp     q_rot = R q and sq = S q_rot for each query
+//   k_logits_rowkey  small query groups: one thread per key, all g queries
+//   k_logits_tiled   large query groups: register-tiled (keys x queries) dot
+//                    products over the combined d + m dimension
+//   k_dequant_warp   PROD / MSE reconstruction, one warp per row
+//   k_topk_row       per-row top-k, one CTA per row
+//   k_logits_bf16    plain bf16-key logits (the comparison baseline)
+// The d = 128 hot-path kernels live in kernels_d128.cu.
+//
+// Method references (page title, section):
+//   rotation R = H_d D / sqrt(d): 0h-n0.github.io "ICLR 2026論文解説: TurboQuant",
+//     "Step 1: PolarQuant"; butterfly FWHT: same page, "実装のポイント";
+//   Lloyd-Max codes: Qiita TurboQuant explainer, "Stage 1: PolarQuant";
+//   QJL signs and the logit estimator: Qiita explainer, "Stage 2: QJL";
+//   (b-1)+1 bit split and unbiased dequantization: ai.spot.hk "Google
+//     TurboQuant", "無偏內積估計".
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "tq_internal.h"
+
+namespace tq {
+
+namespace {
+
+constexpr int kWarps = 8;           // warps per CTA in the warp-per-row kernels
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+
+template <bool BF16>
+__device__ __forceinline__ float load_elem(const void* base, int64_t idx) {
+  if (BF16) {
+    uint16_t u = __ldg(reinterpret_cast<const uint16_t*>(base) + idx);
+    return __uint_as_float(static_cast<uint32_t>(u) << 16);
+  } else {
+    return __ldg(reinterpret_cast<const float*>(base) + idx);
+  }
+}
+
+// Walsh-Hadamard butterflies over a warp-distributed vector: lane l holds
+// elements l*E .. l*E+E-1.  Produces H_d v (Sylvester order), unnormalised.
+template <int E>
+__device__ __forceinline__ void warp_fwht(float (&v)[E], int lane, int d) {
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if ((e & h) == 0) {
+        float a = v[e], b = v[e + h];
+        v[e] = a + b;
+        v[e + h] = a - b;
+      }
+    }
+  }
+  for (int h = E; h < d; h <<= 1) {
+    const int lm = h / E;
+    const bool upper = (lane & lm) != 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      float p = __shfl_xor_sync(0xffffffffu, v[e], lm);
+      v[e] = upper ? (p - v[e]) : (v[e] + p);
+    }
+  }
+}
+
+template <int E>
+__device__ __forceinline__ void apply_D(float (&v)[E], const uint32_t* Dmask, int lane) {
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = lane * E + e;
+    const uint32_t bit = (__ldg(Dmask + (i >> 5)) >> (i & 31)) & 1u;
+    v[e] = bit ? -v[e] : v[e];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// write half
+// ---------------------------------------------------------------------------
+template <int E, bool BF16>
+__global__ void __launch_bounds__(kWarps * 32)
+k_quantize_warp(const KParams P, const void* __restrict__ x, int64_t n_rows, int64_t ld, const Packed out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int d = P.d, m = P.m, B = P.B;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  float* rs = reinterpret_cast<float*>(smem_raw) + wib * d;                       // residual
+  uint8_t* cs = smem_raw + static_cast<size_t>(kWarps) * d * 4 + wib * d;         // codes
+  __shared__ float thr[kMaxLevels], lut[kMaxLevels];
+  if (threadIdx.x < kMaxLevels) { thr[threadIdx.x] = P.t[threadIdx.x]; lut[threadIdx.x] = P.c[threadIdx.x]; }
+  __syncthreads();
+
+  const int nwords_codes = d * B / 32, nwords_signs = m / 32;
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + wib; row < n_rows;
+       row += static_cast<int64_t>(gridDim.x) * kWarps) {
+    uint32_t* codes_out = reinterpret_cast<uint32_t*>(out.codes + row * P.codes_bytes);
+    uint32_t* signs_out = reinterpret_cast<uint32_t*>(out.signs + row * P.signs_bytes);
+    float v[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] = load_elem<BF16>(x, row * ld + lane * E + e);
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) ss = fmaf(v[e], v[e], ss);
+    ss = warp_sum(ss);
+    const float n = sqrtf(ss);
+    if (!(n >= kZeroNorm)) {                   // zero row (or a non-finite norm)
+      for (int w = lane; w < nwords_codes; w += 32) codes_out[w] = 0u;
+      for (int w = lane; w < nwords_signs; w += 32) signs_out[w] = 0u;
+      if (lane == 0) { out.norm[row] = 0.f; out.rnorm[row] = 0.f; }
+      continue;
+    }
+    apply_D<E>(v, P.Dmask, lane);
+    warp_fwht<E>(v, lane, d);
+    const float inv_n = 1.0f / n;
+    float r2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float y = (v[e] * inv_n) * P.inv_sqrt_d;
+      int code = 0;
+      for (int k = 0; k < P.L - 1; ++k) code += (y > thr[k]) ? 1 : 0;
+      const float r = y - lut[code];
+      rs[lane * E + e] = r;
+      cs[lane * E + e] = static_cast<uint8_t>(code);
+      r2 = fmaf(r, r, r2);
+    }
+    r2 = warp_sum(r2);
+    __syncwarp();
+    // codes: output word w holds stream bits [32w, 32w + 32)
+    for (int w = lane; w < nwords_codes; w += 32) {
+      uint32_t acc = 0;
+      const int i0 = (32 * w) / B, i1 = (32 * w + 31) / B;
+      for (int i = i0; i <= i1 && i < d; ++i) {
+        const int sh = B * i - 32 * w;
+        const uint32_t c = cs[i];
+        acc |= sh >= 0 ? (c << sh) : (c >> (-sh));
+      }
+      codes_out[w] = acc;
+    }
+    // QJL: p_j = sum_i S[j][i] r_i, bit j = [p_j < 0]; lane handles j = 32 t + lane
+    for (int t = 0; t < nwords_signs; ++t) {
+      const int j = 32 * t + lane;
+      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+      for (int i = 0; i < d; i += 4) {
+        p0 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i) * m + j)), rs[i], p0);
+        p1 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i + 1) * m + j)), rs[i + 1], p1);
+        p2 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i + 2) * m + j)), rs[i + 2], p2);
+        p3 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i + 3) * m + j)), rs[i + 3], p3);
+      }
+      const float p = (p0 + p1) + (p2 + p3);
+      const uint32_t bits = __ballot_sync(0xffffffffu, p < 0.f);
+      if (lane == 0) signs_out[t] = bits;
+    }
+    if (lane == 0) { out.norm[row] = n; out.rnorm[row] = n * sqrtf(r2); }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// query prep: qp[row] = [R q (d floats) | S R q (m floats)]
+// ---------------------------------------------------------------------------
+template <int E, bool BF16>
+__global__ void __launch_bounds__(kWarps * 32)
+k_qprep_warp(const KParams P, const void* __restrict__ q, int64_t n_q, float* __restrict__ qp) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int d = P.d, m = P.m;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  float* qs = reinterpret_cast<float*>(smem_raw) + wib * d;
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + wib; row < n_q;
+       row += static_cast<int64_t>(gridDim.x) * kWarps) {
+    float v[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] = load_elem<BF16>(q, row * d + lane * E + e);
+    apply_D<E>(v, P.Dmask, lane);
+    warp_fwht<E>(v, lane, d);
+    float* dst = qp + row * (d + m);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float y = v[e] * P.inv_sqrt_d;
+      qs[lane * E + e] = y;
+      dst[lane * E + e] = y;
+    }
+    __syncwarp();
+    for (int j = lane; j < m; j += 32) {
+      float a0 = 0.f, a1 = 0.f;
+      for (int i = 0; i < d; i += 2) {
+        a0 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i) * m + j)), qs[i], a0);
+        a1 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i + 1) * m + j)), qs[i + 1], a1);
+      }
+      dst[d + j] = a0 + a1;
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// logits, small g: one thread per key, all g queries of its set
+// ---------------------------------------------------------------------------
+template <int B, int G>
+__global__ void __launch_bounds__(256)
+k_logits_rowkey(const KParams P, const float* __restrict__ qp, int64_t n_keys, const Packed keys,
+                float* __restrict__ out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* qs = reinterpret_cast<float*>(smem_raw);        // [G][d + m]
+  __shared__ float lut[kMaxLevels];
+  const int d = P.d, m = P.m, dm = d + m;
+  const int64_t set = blockIdx.y;
+  for (int i = threadIdx.x; i < G * dm; i += blockDim.x) qs[i] = qp[(set * G) * dm + i];
+  if (threadIdx.x < kMaxLevels) lut[threadIdx.x] = P.c[threadIdx.x];
+  __syncthreads();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= n_keys) return;
+  const int64_t row = set * n_keys + t;
+  const uint32_t* cw = reinterpret_cast<const uint32_t*>(keys.codes + row * P.codes_bytes);
+  const uint32_t* sw = reinterpret_cast<const uint32_t*>(keys.signs + row * P.signs_bytes);
+  float am[G], aq[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) { am[g] = 0.f; aq[g] = 0.f; }
+  constexpr uint32_t mask = (1u << B) - 1u;
+  for (int c = 0; c < d / 32; ++c) {
+    uint32_t w[B + 1];
+#pragma unroll
+    for (int b = 0; b < B; ++b) w[b] = __ldg(cw + c * B + b);
+    w[B] = 0u;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int bit = B * i, wi = bit >> 5, sh = bit & 31;
+      uint32_t code = w[wi] >> sh;
+      if (sh + B > 32) code |= w[wi + 1] << (32 - sh);
+      const float yv = lut[code & mask];
+#pragma unroll
+      for (int g = 0; g < G; ++g) am[g] = fmaf(qs[g * dm + c * 32 + i], yv, am[g]);
+    }
+  }
+  for (int c = 0; c < m / 32; ++c) {
+    const uint32_t s = __ldg(sw + c);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const bool neg = (s >> j) & 1u;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float v = qs[g * dm + d + c * 32 + j];
+        aq[g] += neg ? -v : v;
+      }
+    }
+  }
+  const float nrm = keys.norm[row], rn = keys.rnorm[row] * P.qjl_scale;
+#pragma unroll
+  for (int g = 0; g < G; ++g) out[(set * G + g) * n_keys + t] = nrm * am[g] + rn * aq[g];
+}
+
+// ---------------------------------------------------------------------------
+// logits, large g: 64 keys x 32 queries per CTA, 4 x 2 outputs per thread.
+// The combined dimension d + m is walked in chunks of 32; each chunk of key
+// values is decoded once per CTA into shared memory as norm*c[code] (MSE
+// coordinates) or rnorm*sqrt(pi/2)/m*z (QJL coordinates).
+// ---------------------------------------------------------------------------
+constexpr int TK = 64, TQ = 32, KC = 32;
+
+__global__ void __launch_bounds__(256)
+k_logits_tiled(const KParams P, const float* __restrict__ qp, int g, int64_t n_keys, const Packed keys,
+               float* __restrict__ out) {
+  __shared__ float Ks[KC][TK + 4];
+  __shared__ float Qs[KC][TQ + 4];
+  __shared__ float lut[kMaxLevels];
+  const int d = P.d, m = P.m, dm = d + m, B = P.B;
+  const int64_t set = blockIdx.z;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * TK;
+  const int q0 = blockIdx.y * TQ;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  if (threadIdx.x < kMaxLevels) lut[threadIdx.x] = P.c[threadIdx.x];
+  float acc[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+  // the key this thread decodes in each chunk and its scales
+  const int dk = threadIdx.x & (TK - 1), dc0 = (threadIdx.x >> 6) * 8;
+  const int64_t krow = set * n_keys + k0 + dk;
+  const bool kvalid = (k0 + dk) < n_keys;
+  float knorm = 0.f, krn = 0.f;
+  if (kvalid) { knorm = keys.norm[krow]; krn = keys.rnorm[krow] * P.qjl_scale; }
+  __syncthreads();
+  for (int kk = 0; kk < dm; kk += KC) {
+    // decode 8 coordinates of key dk
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = kk + dc0 + u;
+      float val = 0.f;
+      if (kvalid) {
+        if (c < d) {
+          const int bit = B * c, by = bit >> 3, sh = bit & 7;
+          const uint8_t* cb = keys.codes + krow * P.codes_bytes;
+          uint32_t win = cb[by];
+          if (sh + B > 8) win |= static_cast<uint32_t>(cb[by + 1]) << 8;
+          val = knorm * lut[(win >> sh) & ((1u << B) - 1u)];
+        } else {
+          const int j = c - d;
+          const uint8_t sb = keys.signs[krow * P.signs_bytes + (j >> 3)];
+          val = ((sb >> (j & 7)) & 1u) ? -krn : krn;
+        }
+      }
+      Ks[dc0 + u][dk] = val;
+    }
+    // stage 32 queries x 32 coordinates
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = threadIdx.x + u * 256;         // 0..1023
+      const int qq = e >> 5, c = e & 31;
+      const int qi = q0 + qq;
+      Qs[c][qq] = (qi < g) ? qp[(set * g + qi) * dm + kk + c] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < KC; ++c) {
+      float a[4], b[2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = Ks[c][tx * 4 + i];
+      b[0] = Qs[c][ty * 2];
+      b[1] = Qs[c][ty * 2 + 1];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[i][0] = fmaf(a[i], b[0], acc[i][0]);
+        acc[i][1] = fmaf(a[i], b[1], acc[i][1]);
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int qi = q0 + ty * 2 + j;
+    if (qi >= g) continue;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t kt = k0 + tx * 4 + i;
+      if (kt < n_keys) out[(set * g + qi) * n_keys + kt] = acc[i][j];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dequant: x~ = R^T (norm yhat [+ sqrt(pi/2)/m rnorm S^T z])
+// ---------------------------------------------------------------------------
+template <int E, bool BF16OUT>
+__global__ void __launch_bounds__(kWarps * 32)
+k_dequant_warp(const KParams P, const Packed in, int64_t n_rows, void* __restrict__ outv, int prod) {
+  const int d = P.d, m = P.m, B = P.B;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  __shared__ float lut[kMaxLevels];
+  if (threadIdx.x < kMaxLevels) lut[threadIdx.x] = P.c[threadIdx.x];
+  __syncthreads();
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + wib; row < n_rows;
+       row += static_cast<int64_t>(gridDim.x) * kWarps) {
+    const uint8_t* cb = in.codes + row * P.codes_bytes;
+    const uint32_t* sw = reinterpret_cast<const uint32_t*>(in.signs + row * P.signs_bytes);
+    const float nrm = in.norm[row], rn = in.rnorm[row];
+    float v[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int i = lane * E + e;
+      const int bit = B * i, by = bit >> 3, sh = bit & 7;
+      uint32_t win = cb[by];
+      if (sh + B > 8) win |= static_cast<uint32_t>(cb[by + 1]) << 8;
+      v[e] = nrm * lut[(win >> sh) & ((1u << B) - 1u)];
+    }
+    if (prod && rn != 0.f) {
+      float acc[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = 0.f;
+      for (int c = 0; c < m / 32; ++c) {
+        const uint32_t s = __ldg(sw + c);
+        for (int jj = 0; jj < 32; ++jj) {
+          const int j = c * 32 + jj;
+          const bool neg = (s >> jj) & 1u;
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float sv = half_bits_to_float(__ldg(P.S + static_cast<int64_t>(j) * d + lane * E + e));
+            acc[e] += neg ? -sv : sv;
+          }
+        }
+      }
+      const float s = P.qjl_scale * rn;
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[e] = fmaf(s, acc[e], v[e]);
+    }
+    warp_fwht<E>(v, lane, d);
+    apply_D<E>(v, P.Dmask, lane);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float o = v[e] * P.inv_sqrt_d;
+      const int64_t idx = row * d + lane * E + e;
+      if (BF16OUT) reinterpret_cast<__nv_bfloat16*>(outv)[idx] = __float2bfloat16_rn(o);
+      else reinterpret_cast<float*>(outv)[idx] = o;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// top-k per row: larger first, equal values by lower index first
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+constexpr int kTopkThreads = 256;
+
+__global__ void __launch_bounds__(kTopkThreads)
+k_topk_row(const float* __restrict__ scores, int64_t cols, int k, int32_t* __restrict__ idx,
+           float* __restrict__ val) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* cv = reinterpret_cast<float*>(smem_raw);                 // [threads][k]
+  int* ci = reinterpret_cast<int*>(cv + kTopkThreads * k);        // [threads][k]
+  __shared__ float wv[kTopkThreads / 32];
+  __shared__ int wi[kTopkThreads / 32], wt[kTopkThreads / 32];
+  __shared__ int win_thread;
+  const int64_t row = blockIdx.x;
+  const float* s = scores + row * cols;
+  float* myv = cv + threadIdx.x * k;
+  int* myi = ci + threadIdx.x * k;
+  int cnt = 0;
+  for (int64_t c = threadIdx.x; c < cols; c += kTopkThreads) {
+    const float x = s[c];
+    const int xi = static_cast<int>(c);
+    if (cnt == k && !better(x, xi, myv[k - 1], myi[k - 1])) continue;
+    int p = cnt < k ? cnt : k - 1;
+    while (p > 0 && better(x, xi, myv[p - 1], myi[p - 1])) { myv[p] = myv[p - 1]; myi[p] = myi[p - 1]; --p; }
+    myv[p] = x; myi[p] = xi;
+    if (cnt < k) ++cnt;
+  }
+  int head = 0;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int r = 0; r < k; ++r) {
+    float bv = head < cnt ? myv[head] : -INFINITY;
+    int bi = head < cnt ? myi[head] : INT32_MAX;
+    int bt = head < cnt ? static_cast<int>(threadIdx.x) : -1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      int ot = __shfl_xor_sync(0xffffffffu, bt, o);
+      if (ot >= 0 && (bt < 0 || better(ov, oi, bv, bi))) { bv = ov; bi = oi; bt = ot; }
+    }
+    if (lane == 0) { wv[w] = bv; wi[w] = bi; wt[w] = bt; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float xv = wv[0]; int xi = wi[0], xt = wt[0];
+      for (int q = 1; q < kTopkThreads / 32; ++q)
+        if (wt[q] >= 0 && (xt < 0 || better(wv[q], wi[q], xv, xi))) { xv = wv[q]; xi = wi[q]; xt = wt[q]; }
+      idx[row * k + r] = xi;
+      if (val) val[row * k + r] = xv;
+      win_thread = xt;
+    }
+    __syncthreads();
+    if (static_cast<int>(threadIdx.x) == win_thread) ++head;
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bf16 unquantized-key logits: 8 lanes per key, fp32 accumulation
+// ---------------------------------------------------------------------------
+template <int DL, int G>     // DL = d / 8 elements per lane
+__global__ void __launch_bounds__(256)
+k_logits_bf16(const uint16_t* __restrict__ q, const uint16_t* __restrict__ keys, int64_t n_keys,
+              float* __restrict__ out) {
+  const int d = DL * 8;
+  const int sub = threadIdx.x & 7;
+  const int64_t set = blockIdx.y;
+  float qr[G][DL];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < DL; ++e)
+      qr[g][e] = __uint_as_float(static_cast<uint32_t>(__ldg(q + (set * G + g) * d + sub * DL + e)) << 16);
+  const int64_t keys_per_iter = static_cast<int64_t>(gridDim.x) * (blockDim.x / 8);
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 8) + (threadIdx.x >> 3); t < n_keys;
+       t += keys_per_iter) {
+    const uint4* kp = reinterpret_cast<const uint4*>(keys + (set * n_keys + t) * d + sub * DL);
+    float acc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g] = 0.f;
+#pragma unroll
+    for (int v = 0; v < DL / 8; ++v) {
+      const uint4 u = __ldg(kp + v);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float lo = __uint_as_float(w[h] << 16), hi = __uint_as_float(w[h] & 0xffff0000u);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          acc[g] = fmaf(qr[g][v * 8 + 2 * h], lo, acc[g]);
+          acc[g] = fmaf(qr[g][v * 8 + 2 * h + 1], hi, acc[g]);
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float a = acc[g];
+      a += __shfl_xor_sync(0xffffffffu, a, 1);
+      a += __shfl_xor_sync(0xffffffffu, a, 2);
+      a += __shfl_xor_sync(0xffffffffu, a, 4);
+      if (sub == g) out[(set * G + g) * n_keys + t] = a;
+    }
+  }
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <typename F>
+int set_smem(F* kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return 0;
+  return static_cast<int>(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(bytes)));
+}
+
+int grid_rows(int64_t n_rows) {
+  int64_t want = (n_rows + kWarps - 1) / kWarps;
+  int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+  return static_cast<int>(want < cap ? want : cap);
+}
+
+template <int E>
+int launch_quantize_E(const KParams& P, const void* x, int bf16, int64_t n_rows, int64_t ld, const Packed& out,
+                      cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(kWarps) * P.d * 5;
+  int g = grid_rows(n_rows);
+  int err;
+  if (bf16) {
+    if ((err = set_smem(k_quantize_warp<E, true>, smem))) return err;
+    k_quantize_warp<E, true><<<g, kWarps * 32, smem, s>>>(P, x, n_rows, ld, out);
+  } else {
+    if ((err = set_smem(k_quantize_warp<E, false>, smem))) return err;
+    k_quantize_warp<E, false><<<g, kWarps * 32, smem, s>>>(P, x, n_rows, ld, out);
+  }
+  count_launch();
+  return static_cast<int>(cudaGetLastError());
+}
+
+template <int E>
+int launch_qprep_E(const KParams& P, const void* q, int bf16, int64_t n_q, float* qp, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(kWarps) * P.d * 4;
+  int g = grid_rows(n_q);
+  int err;
+  if (bf16) {
+    if ((err = set_smem(k_qprep_warp<E, true>, smem))) return err;
+    k_qprep_warp<E, true><<<g, kWarps * 32, smem, s>>>(P, q, n_q, qp);
+  } else {
+    if ((err = set_smem(k_qprep_warp<E, false>, smem))) return err;
+    k_qprep_warp<E, false><<<g, kWarps * 32, smem, s>>>(P, q, n_q, qp);
+  }
+  count_launch();
+  return static_cast<int>(cudaGetLastError());
+}
+
+template <int E>
+int launch_dequant_E(const KParams& P, const Packed& in, int64_t n_rows, void* out, int bf16, int prod,
+                     cudaStream_t s) {
+  int g = grid_rows(n_rows);
+  if (bf16) k_dequant_warp<E, true><<<g, kWarps * 32, 0, s>>>(P, in, n_rows, out, prod);
+  else k_dequant_warp<E, false><<<g, kWarps * 32, 0, s>>>(P, in, n_rows, out, prod);
+  count_launch();
+  return static_cast<int>(cudaGetLastError());
+}
+
+template <int B, int G>
+int launch_rowkey(const KParams& P, const float* qp, int64_t n_sets, int64_t n_keys, const Packed& keys, float* out,
+                  cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(G) * (P.d + P.m) * 4;
+  int err;
+  if ((err = set_smem(k_logits_rowkey<B, G>, smem))) return err;
+  for (int64_t s0 = 0; s0 < n_sets; s0 += 65535) {
+    const int64_t ns = n_sets - s0 < 65535 ? n_sets - s0 : 65535;
+    dim3 grid(static_cast<unsigned>((n_keys + 255) / 256), static_cast<unsigned>(ns));
+    const Packed kk{keys.codes + s0 * n_keys * P.codes_bytes, keys.signs + s0 * n_keys * P.signs_bytes,
+                    keys.norm + s0 * n_keys, keys.rnorm + s0 * n_keys};
+    k_logits_rowkey<B, G><<<grid, 256, smem, s>>>(P, qp + s0 * G * (P.d + P.m), n_keys, kk, out + s0 * G * n_keys);
+    count_launch();
+  }
+  return static_cast<int>(cudaGetLastError());
+}
+
+template <int B>
+int launch_rowkey_B(const KParams& P, const float* qp, int64_t n_sets, int g, int64_t n_keys, const Packed& keys,
+                    float* out, cudaStream_t s) {
+  switch (g) {
+    case 1: return launch_rowkey<B, 1>(P, qp, n_sets, n_keys, keys, out, s);
+    case 2: return launch_rowkey<B, 2>(P, qp, n_sets, n_keys, keys, out, s);
+    case 3: return launch_rowkey<B, 3>(P, qp, n_sets, n_keys, keys, out, s);
+    case 4: return launch_rowkey<B, 4>(P, qp, n_sets, n_keys, keys, out, s);
+    case 5: return launch_rowkey<B, 5>(P, qp, n_sets, n_keys, keys, out, s);
+    case 6: return launch_rowkey<B, 6>(P, qp, n_sets, n_keys, keys, out, s);
+    case 7: return launch_rowkey<B, 7>(P, qp, n_sets, n_keys, keys, out, s);
+    default: return launch_rowkey<B, 8>(P, qp, n_sets, n_keys, keys, out, s);
+  }
+}
+
+template <int DL>
+int launch_bf16_DL(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, float* out,
+                   cudaStream_t s) {
+  const int64_t blocks_per_set_want = (n_keys + 31) / 32;
+  int64_t cap = (static_cast<int64_t>(sm_count()) * 8 + n_sets - 1) / n_sets;
+  if (cap < 1) cap = 1;
+  dim3 grid(static_cast<unsigned>(blocks_per_set_want < cap ? blocks_per_set_want : cap),
+            static_cast<unsigned>(n_sets));
+  const uint16_t* qq = static_cast<const uint16_t*>(q);
+  const uint16_t* kk = static_cast<const uint16_t*>(keys);
+  switch (g) {
+    case 1: k_logits_bf16<DL, 1><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
+    case 2: k_logits_bf16<DL, 2><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
+    case 3: k_logits_bf16<DL, 3><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
+    case 4: k_logits_bf16<DL, 4><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
+    case 5: k_logits_bf16<DL, 5><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
+    case 6: k_logits_bf16<DL, 6><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
+    case 7: k_logits_bf16<DL, 7><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
+    default: k_logits_bf16<DL, 8><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
+  }
+  count_launch();
+  return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace
+
+const char* cuda_error_string(int err) { return cudaGetErrorString(static_cast<cudaError_t>(err)); }
+
+int launch_quantize_generic(const KParams& P, const void* x, int bf16, int64_t n_rows, int64_t ld,
+                            const Packed& out, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+#define CALL(E) launch_quantize_E<E>(P, x, bf16, n_rows, ld, out, s)
+  switch (P.d / 32) {
+    case 1: return CALL(1);
+    case 2: return CALL(2);
+    case 4: return CALL(4);
+    case 8: return CALL(8);
+    case 16: return CALL(16);
+    case 32: return CALL(32);
+    case 64: return CALL(64);
+    case 128: return CALL(128);
+  }
+#undef CALL
+  return static_cast<int>(cudaErrorInvalidValue);
+}
+
+int launch_qprep(const KParams& P, const void* q, int bf16, int64_t n_q, float* qp, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+#define CALL(E) launch_qprep_E<E>(P, q, bf16, n_q, qp, s)
+  switch (P.d / 32) {
+    case 1: return CALL(1);
+    case 2: return CALL(2);
+    case 4: return CALL(4);
+    case 8: return CALL(8);
+    case 16: return CALL(16);
+    case 32: return CALL(32);
+    case 64: return CALL(64);
+    case 128: return CALL(128);
+  }
+#undef CALL
+  return static_cast<int>(cudaErrorInvalidValue);
+}
+
+int launch_logits_generic(const KParams& P, const float* qp, int64_t n_sets, int g, const Packed& keys,
+                          int64_t n_keys, float* out, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t rowkey_smem = static_cast<size_t>(g) * (P.d + P.m) * 4;
+  if (g <= 8 && rowkey_smem <= 200 * 1024) {
+    switch (P.B) {
+      case 1: return launch_rowkey_B<1>(P, qp, n_sets, g, n_keys, keys, out, s);
+      case 2: return launch_rowkey_B<2>(P, qp, n_sets, g, n_keys, keys, out, s);
+      case 3: return launch_rowkey_B<3>(P, qp, n_sets, g, n_keys, keys, out, s);
+      default: return launch_rowkey_B<4>(P, qp, n_sets, g, n_keys, keys, out, s);
+    }
+  }
+  for (int64_t s0 = 0; s0 < n_sets; s0 += 65535) {
+    const int64_t ns = n_sets - s0 < 65535 ? n_sets - s0 : 65535;
+    dim3 grid(static_cast<unsigned>((n_keys + TK - 1) / TK), static_cast<unsigned>((g + TQ - 1) / TQ),
+              static_cast<unsigned>(ns));
+    const Packed kk{keys.codes + s0 * n_keys * P.codes_bytes, keys.signs + s0 * n_keys * P.signs_bytes,
+                    keys.norm + s0 * n_keys, keys.rnorm + s0 * n_keys};
+    k_logits_tiled<<<grid, 256, 0, s>>>(P, qp + s0 * g * (P.d + P.m), g, n_keys, kk, out + s0 * g * n_keys);
+    count_launch();
+  }
+  return static_cast<int>(cudaGetLastError());
+}
+
+int launch_dequant_generic(const KParams& P, const Packed& in, int64_t n_rows, void* out, int bf16, int prod,
+                           void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+#define CALL(E) launch_dequant_E<E>(P, in, n_rows, out, bf16, prod, s)
+  switch (P.d / 32) {
+    case 1: return CALL(1);
+    case 2: return CALL(2);
+    case 4: return CALL(4);
+    case 8: return CALL(8);
+    case 16: return CALL(16);
+    case 32: return CALL(32);
+    case 64: return CALL(64);
+    case 128: return CALL(128);
+  }
+#undef CALL
+  return static_cast<int>(cudaErrorInvalidValue);
+}
+
+int launch_topk(const float* scores, int64_t rows, int64_t cols, int k, int32_t* idx, float* val, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t smem = static_cast<size_t>(kTopkThreads) * k * 8;
+  int err;
+  if ((err = set_smem(k_topk_row, smem))) return err;
+  for (int64_t r0 = 0; r0 < rows; r0 += 65535) {
+    const int64_t nr = rows - r0 < 65535 ? rows - r0 : 65535;
+    k_topk_row<<<static_cast<unsigned>(nr), kTopkThreads, smem, s>>>(scores + r0 * cols, cols, k, idx + r0 * k,
+                                                                    val ? val + r0 * k : nullptr);
+    count_launch();
+  }
+  return static_cast<int>(cudaGetLastError());
+}
+
+int launch_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, int d, float* out,
+                       void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return launch_bf16_DL<8>(q, keys, n_sets, g, n_keys, out, s);
+    case 128: return launch_bf16_DL<16>(q, keys, n_sets, g, n_keys, out, s);
+    case 256: return launch_bf16_DL<32>(q, keys, n_sets, g, n_keys, out, s);
+  }
+  return static_cast<int>(cudaErrorInvalidValue);
+}
+
+}  // namespace tq

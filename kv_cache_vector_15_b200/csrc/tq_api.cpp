@@ -1,0 +1,263 @@
+// C ABI of libtq: argument checks, context set-up and kernel dispatch.
+// Every compute entry point validates its arguments on the host and launches
+// nothing when a check fails; see include/tq.h for the contract.
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "tq_internal.h"
+
+namespace tq {
+
+static thread_local std::string g_last_error;
+static std::atomic<uint64_t> g_launches{0};
+
+tq_status fail(tq_status s, const std::string& why) {
+  g_last_error = why;
+  return s;
+}
+
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+tq_status check_dims(int d, int b, int m) {
+  if (d < 32 || d > 4096 || (d & (d - 1)))
+    return fail(TQ_ERR_INVALID_ARG, "d must be a power of two in [32, 4096]");
+  if (b < 2 || b > 5) return fail(TQ_ERR_INVALID_ARG, "b must be in [2, 5]");
+  if (m < 32 || m > 4096 || (m % 32)) return fail(TQ_ERR_INVALID_ARG, "m must be a multiple of 32 in [32, 4096]");
+  return TQ_OK;
+}
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static tq_status cuda_fail(int err, const char* what) {
+  return fail(TQ_ERR_CUDA, std::string(what) + ": " + cuda_error_string(err));
+}
+
+static tq_status check_ctx(const tq_ctx* ctx) {
+  if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(TQ_ERR_CUDA, "cudaGetDevice failed");
+  if (dev != ctx->device) return fail(TQ_ERR_INVALID_ARG, "the current device is not the context's device");
+  return TQ_OK;
+}
+
+static tq_status check_packed(const tq_ctx* ctx, const tq_packed& p) {
+  if (!p.codes || !p.signs || !p.norm || !p.rnorm) return fail(TQ_ERR_INVALID_ARG, "a packed pointer is NULL");
+  if (!aligned(p.codes, 16) || !aligned(p.signs, 16))
+    return fail(TQ_ERR_INVALID_ARG, "packed codes/signs must be 16-byte aligned");
+  if (!aligned(p.norm, 4) || !aligned(p.rnorm, 4))
+    return fail(TQ_ERR_INVALID_ARG, "packed norm/rnorm must be 4-byte aligned");
+  (void)ctx;
+  return TQ_OK;
+}
+
+static Packed to_internal(const tq_packed& p) { return Packed{p.codes, p.signs, p.norm, p.rnorm}; }
+
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" {
+
+const char* tq_status_str(tq_status s) {
+  switch (s) {
+    case TQ_OK: return "TQ_OK";
+    case TQ_ERR_INVALID_ARG: return "TQ_ERR_INVALID_ARG";
+    case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED";
+    case TQ_ERR_NOMEM: return "TQ_ERR_NOMEM";
+    case TQ_ERR_CUDA: return "TQ_ERR_CUDA";
+  }
+  return "TQ_ERR_UNKNOWN";
+}
+
+const char* tq_last_error(void) { return g_last_error.c_str(); }
+
+uint64_t tq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
+  if (!out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  tq_status st = check_dims(d, b, m);
+  if (st != TQ_OK) return st;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0;
+  e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  if (major != 10) return fail(TQ_ERR_UNSUPPORTED, "libtq is built for sm_100a (compute capability 10.x)");
+
+  tq_ctx* ctx = new (std::nothrow) tq_ctx();
+  if (!ctx) return fail(TQ_ERR_NOMEM, "host allocation failed");
+  ctx->d = d; ctx->b = b; ctx->m = m; ctx->seed = seed; ctx->device = dev;
+  const int B = b - 1, L = 1 << B;
+  ctx->centroids.resize(L);
+  ctx->thresholds.resize(L - 1);
+  ctx->D.resize(d);
+  ctx->S_bits.resize(static_cast<size_t>(m) * d);
+  tq_host_params(d, b, m, seed, ctx->centroids.data(), ctx->thresholds.data(), ctx->D.data(), ctx->S_bits.data());
+
+  // device block, 256-byte aligned parts: Dmask (d/32 words) | S [m][d] | St [d][m]
+  auto round256 = [](size_t v) { return (v + 255) / 256 * 256; };
+  const size_t n_mask = static_cast<size_t>(d) / 32;
+  const size_t sz_S = static_cast<size_t>(m) * d * sizeof(uint16_t);
+  const size_t off_mask = 0;
+  const size_t off_S2 = round256(n_mask * 4);
+  const size_t off_St = off_S2 + round256(sz_S);
+  const size_t total = off_St + round256(sz_S);
+  void* blk = nullptr;
+  e = cudaMalloc(&blk, total);
+  if (e != cudaSuccess) { delete ctx; return fail(TQ_ERR_NOMEM, std::string("cudaMalloc: ") + cudaGetErrorString(e)); }
+  ctx->dev_block = blk;
+
+  std::vector<uint8_t> host(total, 0);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(host.data() + off_mask);
+  for (int i = 0; i < d; ++i)
+    if (ctx->D[i] < 0) mask[i / 32] |= (1u << (i % 32));
+  std::memcpy(host.data() + off_S2, ctx->S_bits.data(), sz_S);
+  uint16_t* St = reinterpret_cast<uint16_t*>(host.data() + off_St);
+  for (int j = 0; j < m; ++j)
+    for (int i = 0; i < d; ++i) St[static_cast<size_t>(i) * m + j] = ctx->S_bits[static_cast<size_t>(j) * d + i];
+  e = cudaMemcpy(blk, host.data(), total, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) { cudaFree(blk); delete ctx; return cuda_fail(e, "cudaMemcpy"); }
+
+  KParams& kp = ctx->kp;
+  std::memset(&kp, 0, sizeof(kp));
+  kp.d = d; kp.m = m; kp.B = B; kp.L = L;
+  kp.codes_bytes = d * B / 8;
+  kp.signs_bytes = m / 8;
+  kp.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  kp.qjl_scale = static_cast<float>(std::sqrt(std::acos(-1.0) / 2.0) / m);
+  for (int i = 0; i < L; ++i) kp.c[i] = ctx->centroids[i];
+  for (int i = 0; i < L - 1; ++i) kp.t[i] = ctx->thresholds[i];
+  kp.Dmask = reinterpret_cast<const uint32_t*>(static_cast<uint8_t*>(blk) + off_mask);
+  kp.S = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(blk) + off_S2);
+  kp.St = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(blk) + off_St);
+  *out = ctx;
+  return TQ_OK;
+}
+
+tq_status tq_destroy(tq_ctx* ctx) {
+  if (!ctx) return TQ_OK;
+  cudaError_t e = cudaSuccess;
+  if (ctx->dev_block) e = cudaFree(ctx->dev_block);
+  delete ctx;
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFree");
+  return TQ_OK;
+}
+
+tq_status tq_packed_sizes(const tq_ctx* ctx, int64_t n_rows, size_t* codes_bytes, size_t* signs_bytes) {
+  if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (n_rows < 0) return fail(TQ_ERR_INVALID_ARG, "n_rows < 0");
+  if (codes_bytes) *codes_bytes = static_cast<size_t>(n_rows) * ctx->kp.codes_bytes;
+  if (signs_bytes) *signs_bytes = static_cast<size_t>(n_rows) * ctx->kp.signs_bytes;
+  return TQ_OK;
+}
+
+tq_status tq_get_params(const tq_ctx* ctx, float* centroids, float* thresholds, int8_t* D, uint16_t* S_bits) {
+  if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (centroids) std::memcpy(centroids, ctx->centroids.data(), ctx->centroids.size() * sizeof(float));
+  if (thresholds) std::memcpy(thresholds, ctx->thresholds.data(), ctx->thresholds.size() * sizeof(float));
+  if (D) std::memcpy(D, ctx->D.data(), ctx->D.size());
+  if (S_bits) std::memcpy(S_bits, ctx->S_bits.data(), ctx->S_bits.size() * sizeof(uint16_t));
+  return TQ_OK;
+}
+
+tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
+                      tq_packed out, void* stream) {
+  tq_status st = check_ctx(ctx);
+  if (st != TQ_OK) return st;
+  if (n_rows < 0) return fail(TQ_ERR_INVALID_ARG, "n_rows < 0");
+  if (x_dtype != TQ_BF16 && x_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "x_dtype must be TQ_BF16 or TQ_F32");
+  if (n_rows == 0) return TQ_OK;
+  if (!x) return fail(TQ_ERR_INVALID_ARG, "x is NULL");
+  const size_t esz = x_dtype == TQ_BF16 ? 2 : 4;
+  if (ld_x < ctx->d) return fail(TQ_ERR_INVALID_ARG, "ld_x < d");
+  if (!aligned(x, 16) || (static_cast<size_t>(ld_x) * esz) % 16)
+    return fail(TQ_ERR_INVALID_ARG, "x and its row stride must be 16-byte aligned");
+  if ((st = check_packed(ctx, out)) != TQ_OK) return st;
+  int err = launch_quantize(ctx->kp, x, x_dtype == TQ_BF16, n_rows, ld_x, to_internal(out), stream);
+  if (err) return cuda_fail(err, "tq_quantize launch");
+  return TQ_OK;
+}
+
+size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g) {
+  if (!ctx || n_sets <= 0 || g <= 0) return 0;
+  return static_cast<size_t>(n_sets) * g * (ctx->d + ctx->m) * sizeof(float);
+}
+
+tq_status tq_logits(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g, tq_packed keys,
+                    int64_t n_keys, float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  tq_status st = check_ctx(ctx);
+  if (st != TQ_OK) return st;
+  if (n_sets < 0 || n_keys < 0) return fail(TQ_ERR_INVALID_ARG, "n_sets and n_keys must be >= 0");
+  if (g < 1 || g > 4096) return fail(TQ_ERR_INVALID_ARG, "g must be in [1, 4096]");
+  if (q_dtype != TQ_BF16 && q_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "q_dtype must be TQ_BF16 or TQ_F32");
+  if (n_sets == 0 || n_keys == 0) return TQ_OK;
+  if (!q || !out) return fail(TQ_ERR_INVALID_ARG, "q or out is NULL");
+  if (!aligned(q, 16) || !aligned(out, 4)) return fail(TQ_ERR_INVALID_ARG, "q must be 16-byte and out 4-byte aligned");
+  if ((st = check_packed(ctx, keys)) != TQ_OK) return st;
+  const size_t need = tq_logits_workspace_bytes(ctx, n_sets, g);
+  if (need) {
+    if (!workspace || workspace_bytes < need) return fail(TQ_ERR_INVALID_ARG, "workspace missing or too small");
+    if (!aligned(workspace, 16)) return fail(TQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  }
+  float* qp = static_cast<float*>(workspace);
+  int err = launch_qprep(ctx->kp, q, q_dtype == TQ_BF16, n_sets * g, qp, stream);
+  if (err) return cuda_fail(err, "tq_logits query-prep launch");
+  err = launch_logits(ctx->kp, qp, n_sets, g, to_internal(keys), n_keys, out, stream);
+  if (err) return cuda_fail(err, "tq_logits launch");
+  return TQ_OK;
+}
+
+tq_status tq_dequant(const tq_ctx* ctx, tq_packed in, int64_t n_rows, void* out, tq_dtype out_dtype,
+                     tq_dequant_mode mode, void* stream) {
+  tq_status st = check_ctx(ctx);
+  if (st != TQ_OK) return st;
+  if (n_rows < 0) return fail(TQ_ERR_INVALID_ARG, "n_rows < 0");
+  if (out_dtype != TQ_BF16 && out_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "out_dtype must be TQ_BF16 or TQ_F32");
+  if (mode != TQ_DEQUANT_PROD && mode != TQ_DEQUANT_MSE) return fail(TQ_ERR_INVALID_ARG, "bad dequant mode");
+  if (n_rows == 0) return TQ_OK;
+  if (!out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
+  if (!aligned(out, 16)) return fail(TQ_ERR_INVALID_ARG, "out must be 16-byte aligned");
+  if ((st = check_packed(ctx, in)) != TQ_OK) return st;
+  int err = launch_dequant(ctx->kp, to_internal(in), n_rows, out, out_dtype == TQ_BF16, mode == TQ_DEQUANT_PROD, stream);
+  if (err) return cuda_fail(err, "tq_dequant launch");
+  return TQ_OK;
+}
+
+tq_status tq_topk(const float* scores, int64_t rows, int64_t cols, int k, int32_t* idx, float* val, void* stream) {
+  if (rows < 0 || cols < 0) return fail(TQ_ERR_INVALID_ARG, "rows and cols must be >= 0");
+  if (k < 1 || k > 64) return fail(TQ_ERR_INVALID_ARG, "k must be in [1, 64]");
+  if (rows == 0) return TQ_OK;
+  if (k > cols) return fail(TQ_ERR_INVALID_ARG, "k > cols");
+  if (cols > INT32_MAX) return fail(TQ_ERR_UNSUPPORTED, "cols must fit in int32");
+  if (!scores || !idx) return fail(TQ_ERR_INVALID_ARG, "scores or idx is NULL");
+  if (!aligned(scores, 4) || !aligned(idx, 4) || (val && !aligned(val, 4)))
+    return fail(TQ_ERR_INVALID_ARG, "scores/idx/val must be 4-byte aligned");
+  int err = launch_topk(scores, rows, cols, k, idx, val, stream);
+  if (err) return cuda_fail(err, "tq_topk launch");
+  return TQ_OK;
+}
+
+tq_status tq_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, int d, float* out,
+                         void* stream) {
+  if (n_sets < 0 || n_keys < 0) return fail(TQ_ERR_INVALID_ARG, "n_sets and n_keys must be >= 0");
+  if (g < 1 || g > 8) return fail(TQ_ERR_INVALID_ARG, "g must be in [1, 8]");
+  if (d != 64 && d != 128 && d != 256) return fail(TQ_ERR_INVALID_ARG, "d must be 64, 128 or 256");
+  if (n_sets == 0 || n_keys == 0) return TQ_OK;
+  if (n_sets > 65535) return fail(TQ_ERR_UNSUPPORTED, "n_sets must be <= 65535");
+  if (!q || !keys || !out) return fail(TQ_ERR_INVALID_ARG, "a pointer is NULL");
+  if (!aligned(q, 16) || !aligned(keys, 16) || !aligned(out, 4))
+    return fail(TQ_ERR_INVALID_ARG, "q and keys must be 16-byte aligned, out 4-byte");
+  int err = launch_logits_bf16(q, keys, n_sets, g, n_keys, d, out, stream);
+  if (err) return cuda_fail(err, "tq_logits_bf16 launch");
+  return TQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,77 @@
+// Internal declarations shared by the C-ABI layer (tq_api.cpp), the host
+// parameter code and the CUDA kernels.  Not part of the public interface.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+constexpr int kMaxLevels = 16;      // 2^(b-1) for b <= 5
+constexpr float kZeroNorm = 1e-10f; // rows with ||x|| below this are stored as zeros
+
+// Everything a kernel needs about one parameter set, passed by value.
+struct KParams {
+  int d, m, B, L;
+  int codes_bytes, signs_bytes;       // per row
+  float inv_sqrt_d;                   // 1/sqrt(d), fp32
+  float qjl_scale;                    // sqrt(pi/2) / m, fp32
+  float c[kMaxLevels];                // centroids, ascending
+  float t[kMaxLevels];                // thresholds (L-1 used)
+  const uint32_t* Dmask;              // d/32 words, bit i set iff D_i = -1
+  const uint16_t* S;                  // [m][d] binary16
+  const uint16_t* St;                 // [d][m] binary16 (transpose)
+};
+
+struct Packed {
+  uint8_t* codes;
+  uint8_t* signs;
+  float* norm;
+  float* rnorm;
+};
+
+tq_status check_dims(int d, int b, int m);
+tq_status fail(tq_status s, const std::string& why);   // records tq_last_error()
+void count_launch(int n = 1);
+
+// host_params.cpp
+uint16_t double_to_half_bits(double v);
+void rademacher(int d, uint64_t seed, int8_t* D);
+void gaussian_projection_half(int m, int d, uint64_t seed, uint16_t* S_bits);
+void lloyd_max(int d, int bits_mse, std::vector<double>& centroids, std::vector<double>& thresholds);
+
+// kernels (return cudaError_t as int; 0 = success).  launch_* choose between
+// the d = 128 hot-path kernels and the general ones (*_generic).
+int launch_quantize_generic(const KParams& P, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x,
+                            const Packed& out, void* stream);
+int launch_logits_generic(const KParams& P, const float* qp, int64_t n_sets, int g, const Packed& keys,
+                          int64_t n_keys, float* out, void* stream);
+int launch_dequant_generic(const KParams& P, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
+                           void* stream);
+int launch_quantize(const KParams& P, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x,
+                    const Packed& out, void* stream);
+int launch_qprep(const KParams& P, const void* q, int q_is_bf16, int64_t n_queries, float* qp, void* stream);
+int launch_logits(const KParams& P, const float* qp, int64_t n_sets, int g, const Packed& keys,
+                  int64_t n_keys, float* out, void* stream);
+int launch_dequant(const KParams& P, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
+                   void* stream);
+int launch_topk(const float* scores, int64_t rows, int64_t cols, int k, int32_t* idx, float* val, void* stream);
+int launch_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, int d, float* out,
+                       void* stream);
+const char* cuda_error_string(int err);
+
+}  // namespace tq
+
+struct tq_ctx {
+  int d, b, m;
+  uint64_t seed;
+  int device;
+  std::vector<float> centroids, thresholds;
+  std::vector<int8_t> D;
+  std::vector<uint16_t> S_bits;
+  void* dev_block;                    // one allocation holding everything below
+  tq::KParams kp;
+};

@@ -35,10 +35,13 @@ BLOCK = 65536
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round fp32 to bf16 (nearest, ties to even); returns uint16 bits."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return u.astype(np.uint16)
+    """Round finite fp32 to bf16 (nearest, ties to even); returns uint16 bits."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u >> np.uint32(16)) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u                      # finite inputs: no wrap below the NaN range
+    r >>= np.uint32(16)
+    return r.astype(np.uint16)
 
 
 def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -136,6 +139,22 @@ class RowTensor:
 
     def all(self) -> np.ndarray:
         return self.rows(0, self.n_rows)
+
+    def fill(self, out: np.ndarray, threads: int = 0) -> np.ndarray:
+        """Write all rows into ``out`` (uint16 for bf16, fp32 otherwise, shape
+        [n_rows, d]) block by block on a thread pool; same values as all()."""
+        import concurrent.futures as cf
+        import os
+        nblk = (self.n_rows + BLOCK - 1) // BLOCK
+        threads = threads or min(32, os.cpu_count() or 1)
+
+        def one(k):
+            lo, hi = k * BLOCK, min(self.n_rows, (k + 1) * BLOCK)
+            out[lo:hi] = self.rows(lo, hi)
+
+        with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(one, range(nblk)))
+        return out
 
     def as_f32(self, rows: np.ndarray) -> np.ndarray:
         return bf16_to_f32(rows) if self.dtype == "bf16" else rows

@@ -81,13 +81,14 @@ def fwht(v: np.ndarray) -> np.ndarray:
 
 
 def rotate(v: np.ndarray, P) -> np.ndarray:
-    """Row-wise R v (v has rows of length d)."""
-    return np.asarray(v, dtype=np.float64) @ P.R.T
+    """Row-wise R v = H_d (D v) / sqrt(d) (v has rows of length d), by the
+    butterfly; equal to the dense P.R @ v (pinned in the tests)."""
+    return fwht(np.asarray(v, dtype=np.float64) * P.D) / math.sqrt(P.d)
 
 
 def rotate_inverse(v: np.ndarray, P) -> np.ndarray:
-    """Row-wise R^T v."""
-    return np.asarray(v, dtype=np.float64) @ P.R
+    """Row-wise R^T v = D (H_d v) / sqrt(d)."""
+    return fwht(np.asarray(v, dtype=np.float64)) * P.D / math.sqrt(P.d)
 
 
 # --------------------------------------------------------------------------

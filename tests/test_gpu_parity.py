@@ -1,0 +1,176 @@
+"""GPU parity: every entry point of the C ABI against the fp64 oracle, on the
+same seeded inputs, element by element.  Sizes span several tiles and a
+ragged tail; edge rows (zero, tiny, huge, one-hot, constant) are mixed in.
+
+The read-half kernels are fed packed rows produced by the oracle, so both
+sides compute on byte-identical inputs; the write half is compared with the
+boundary-band rule in tests/parity.py.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+from kv_cache_vector_15_b200 import inputs
+from oracle import params as op
+from oracle import turboquant as ot
+from tests import parity
+
+torch = pytest.importorskip("torch")
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+
+@pytest.fixture(scope="module")
+def tq():
+    from kv_cache_vector_15_b200 import tq as _tq
+    return _tq
+
+
+def edge_rows(d, rng):
+    rows = [np.zeros(d), np.full(d, 0.5), np.eye(1, d, 3)[0] * 7.0, rng.standard_normal(d) * 1e-8,
+            rng.standard_normal(d) * 3e3, np.concatenate([np.ones(2), np.zeros(d - 2)])]
+    return np.stack(rows)
+
+
+def make_rows(d, n, dtype, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((n, d)) * rng.uniform(0.1, 10, size=(n, 1))
+    x[: 6] = edge_rows(d, rng)
+    x = x.astype(np.float32)
+    if dtype == "bf16":
+        bits = inputs.bf16_bits(x)
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16), inputs.bf16_to_f32(bits)
+    return torch.from_numpy(x), x
+
+
+CASES = [(32, 2, 32), (64, 3, 64), (128, 2, 128), (128, 3, 128), (128, 4, 128), (128, 5, 128),
+         (256, 3, 96), (512, 4, 256), (1024, 4, 1024), (2048, 2, 64), (4096, 3, 128)]
+
+
+@pytest.mark.parametrize("d,b,m", CASES)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_quantize_parity(tq, d, b, m, dtype):
+    n = 1531 if d <= 1024 else 301
+    xt, x = make_rows(d, n, dtype, seed=d * 10 + b)
+    P = op.Params(d, b, m, seed=0)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    got = T.quantize(xt.cuda()).to_numpy()
+    torch.cuda.synchronize()
+    want = ot.quantize(x, P, keep_intermediates=True)
+    rep = parity.compare_quantize(P, got, want)
+    parity.assert_quantize_ok(rep)
+
+
+def test_quantize_strided_rows(tq):
+    d, b, m = 128, 3, 128
+    xt, x = make_rows(d, 777, "bf16", seed=5)
+    wide = torch.zeros((777, 200), dtype=torch.bfloat16)
+    wide[:, :d] = xt
+    P = op.Params(d, b, m, seed=0)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    got = T.quantize(wide.cuda()[:, :d]).to_numpy()
+    parity.assert_quantize_ok(parity.compare_quantize(P, got, ot.quantize(x, P, keep_intermediates=True)))
+
+
+@pytest.mark.parametrize("d,b,m,n_sets,g,n_keys", [
+    (128, 3, 128, 3, 4, 1000), (128, 4, 128, 2, 1, 4097), (128, 2, 128, 5, 8, 333), (64, 5, 64, 2, 3, 700),
+    (128, 3, 128, 2, 16, 1500), (256, 3, 128, 1, 40, 900), (1024, 4, 1024, 1, 37, 600), (32, 2, 32, 4, 5, 129)])
+@pytest.mark.parametrize("qdtype", ["bf16", "f32"])
+def test_logits_parity_on_oracle_packed_keys(tq, d, b, m, n_sets, g, n_keys, qdtype):
+    P = op.Params(d, b, m, seed=0)
+    rng = np.random.default_rng(d + g)
+    k = rng.standard_normal((n_sets * n_keys, d)) * rng.uniform(0.1, 10, size=(n_sets * n_keys, 1))
+    k[:3] = edge_rows(d, rng)[:3]
+    pk = ot.quantize(k, P)
+    qt, q = make_rows(d, n_sets * g, qdtype, seed=7 + g)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    got = T.logits(qt.cuda(), tq.Packed.from_numpy(pk), n_sets, g, n_keys).cpu().numpy()
+    want = ot.logits(q, pk, P, n_sets, g, n_keys)
+    tol = parity.logit_tolerance(q, np.linalg.norm(k, axis=1), n_sets, g, n_keys)
+    err = np.abs(got - want)
+    assert np.all(err <= tol + 1e-30), float(np.max(err / (tol + 1e-30)))
+
+
+@pytest.mark.parametrize("d,b,m", [(128, 3, 128), (128, 4, 128), (64, 2, 96), (1024, 4, 1024)])
+def test_end_to_end_quantize_then_logits(tq, d, b, m):
+    """GPU quantize -> GPU logits against oracle quantize -> oracle logits.
+    Keys whose packed bytes differ (boundary-band cases) are counted, not compared."""
+    n_sets, g, n_keys = 2, 4, 1200
+    P = op.Params(d, b, m, seed=0)
+    kt, k = make_rows(d, n_sets * n_keys, "bf16", seed=11)
+    qt, q = make_rows(d, n_sets * g, "bf16", seed=12)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    pg = T.quantize(kt.cuda())
+    got = T.logits(qt.cuda(), pg, n_sets, g, n_keys).cpu().numpy()
+    po = ot.quantize(k, P)
+    want = ot.logits(q, po, P, n_sets, g, n_keys)
+    png = pg.to_numpy()
+    same = (np.all(png["codes"] == po["codes"], axis=1) & np.all(png["signs"] == po["signs"], axis=1))
+    assert np.mean(~same) <= 1e-3
+    tol = parity.logit_tolerance(q, np.linalg.norm(k, axis=1), n_sets, g, n_keys)
+    ok = (np.abs(got - want) <= tol + 1e-30) | ~same.reshape(n_sets, 1, n_keys)
+    assert ok.all()
+
+
+@pytest.mark.parametrize("d,b,m", [(128, 3, 128), (128, 4, 128), (128, 2, 128), (64, 5, 32), (1024, 4, 1024),
+                                   (4096, 3, 64)])
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_dequant_parity_on_oracle_packed_rows(tq, d, b, m, mode, out):
+    P = op.Params(d, b, m, seed=0)
+    rng = np.random.default_rng(d * 3 + b)
+    n = 1029 if d <= 1024 else 130
+    x = rng.standard_normal((n, d)) * rng.uniform(0.1, 10, size=(n, 1))
+    x[:6] = edge_rows(d, rng)
+    pk = ot.quantize(x, P)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    dt = torch.bfloat16 if out == "bf16" else torch.float32
+    got = T.dequant(tq.Packed.from_numpy(pk), out_dtype=dt, mode=mode).float().cpu().numpy()
+    want = ot.dequant(pk, P, mode)
+    parity.assert_dequant_ok(got, want, out == "bf16")
+
+
+@pytest.mark.parametrize("rows,cols,k", [(7, 1000, 10), (3, 5, 5), (64, 100003, 10), (5, 4096, 64), (2, 77, 1)])
+def test_topk_parity_with_ties(tq, rows, cols, k):
+    rng = np.random.default_rng(rows * cols + k)
+    s = rng.standard_normal((rows, cols)).astype(np.float32)
+    s[:, ::7] = np.round(s[:, ::7] * 2) / 2          # many exact ties
+    s[0, :] = 1.0                                   # an all-equal row
+    idx, val = tq.topk(torch.from_numpy(s).cuda(), k)
+    wi, wv = ot.topk(s, k)
+    assert np.array_equal(idx.cpu().numpy(), wi)
+    assert np.array_equal(val.cpu().numpy(), wv)
+
+
+@pytest.mark.parametrize("d,g", [(128, 4), (64, 1), (256, 8), (128, 3)])
+def test_bf16_baseline_logits(tq, d, g):
+    n_sets, n_keys = 3, 2049
+    kt, k = make_rows(d, n_sets * n_keys, "bf16", seed=d + g)
+    qt, q = make_rows(d, n_sets * g, "bf16", seed=d * g)
+    got = tq.logits_bf16(qt.cuda(), kt.cuda(), n_sets, g, n_keys).cpu().numpy()
+    want = np.einsum("sgd,snd->sgn", q.reshape(n_sets, g, d).astype(np.float64),
+                     k.reshape(n_sets, n_keys, d).astype(np.float64))
+    bound = np.einsum("sgd,snd->sgn", np.abs(q.reshape(n_sets, g, d)), np.abs(k.reshape(n_sets, n_keys, d)))
+    assert np.all(np.abs(got - want) <= d * 2.0 ** -24 * bound + 1e-30)
+
+
+def test_gpu_api_errors_and_empty_calls(tq):
+    T = tq.TurboQuant(128, 3, 128)
+    x = torch.zeros((0, 128), dtype=torch.bfloat16, device="cuda")
+    p = T.quantize(x)                              # n = 0: no-op
+    assert p.n_rows == 0
+    xb = torch.zeros((10, 129), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(tq.TQError) as e:
+        T.quantize(xb[:, 1:])                      # misaligned base pointer
+    assert e.value.status == tq.TQ_ERR_INVALID_ARG
+    with pytest.raises(tq.TQError):
+        T.quantize(torch.zeros((10, 100), dtype=torch.float32, device="cuda"))   # ld < d is caught below
+    with pytest.raises(tq.TQError):
+        T.logits(torch.zeros((4, 128), device="cuda"), T.empty_packed(8), 1, 0, 8)  # g = 0
+    before = tq.launch_count()
+    with pytest.raises(tq.TQError):
+        T.logits(torch.zeros((4, 128), device="cuda"), T.empty_packed(8), 1, 4, 8,
+                 workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert tq.launch_count() == before
