@@ -162,6 +162,10 @@ tq_status tq_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g,
 /* ----------------------------------------------------------- reporting -- */
 
 const char* tq_status_str(tq_status s);
+/* Wait for `stream`, then report whether any kernel of this context timed out
+ * in one of its bounded device-side waits since the last check (TQ_ERR_CUDA,
+ * outputs of that call invalid) and clear the record.  Blocking. */
+tq_status tq_sync_status(const tq_ctx* ctx, void* stream);
 /* One-line reason for the last non-OK status returned on this host thread. */
 const char* tq_last_error(void);
 /* Number of kernel launches this library has issued in this process (all

@@ -4,9 +4,11 @@
 
 namespace tq {
 
-int launch_quantize(const KParams& P, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x, const Packed& out,
+int launch_quantize(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x, const Packed& out,
                     void* stream) {
-  return launch_quantize_generic(P, x, x_is_bf16, n_rows, ld_x, out, stream);
+  if (quantize_d128_applies(ctx, n_rows))
+    return launch_quantize_d128(ctx, x, x_is_bf16, n_rows, ld_x, out, stream);
+  return launch_quantize_generic(ctx.kp, x, x_is_bf16, n_rows, ld_x, out, stream);
 }
 
 int launch_logits(const KParams& P, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,

@@ -4,8 +4,10 @@
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <string>
@@ -58,6 +60,12 @@ static tq_status check_packed(const tq_ctx* ctx, const tq_packed& p) {
 
 static Packed to_internal(const tq_packed& p) { return Packed{p.codes, p.signs, p.norm, p.rnorm}; }
 
+static double half_bits_to_double(uint16_t h) {
+  const int sign = (h >> 15) & 1, e = (h >> 10) & 31, f = h & 1023;
+  double v = e == 0 ? std::ldexp(static_cast<double>(f), -24) : std::ldexp(static_cast<double>(1024 + f), e - 25);
+  return sign ? -v : v;
+}
+
 }  // namespace tq
 
 using namespace tq;
@@ -76,6 +84,23 @@ const char* tq_status_str(tq_status s) {
 }
 
 const char* tq_last_error(void) { return g_last_error.c_str(); }
+
+tq_status tq_sync_status(const tq_ctx* ctx, void* stream) {
+  tq_status st = check_ctx(ctx);
+  if (st != TQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int word = 0;
+  e = cudaMemcpy(&word, ctx->kp.err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+  if (word) {
+    const int zero = 0;
+    cudaMemcpy(ctx->kp.err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    return fail(TQ_ERR_CUDA, "a kernel wait ran out of time (code " + std::to_string(word) + "); outputs are invalid");
+  }
+  return TQ_OK;
+}
 
 uint64_t tq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -102,12 +127,13 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
   ctx->S_bits.resize(static_cast<size_t>(m) * d);
   tq_host_params(d, b, m, seed, ctx->centroids.data(), ctx->thresholds.data(), ctx->D.data(), ctx->S_bits.data());
 
-  // device block, 256-byte aligned parts: Dmask (d/32 words) | S [m][d] | St [d][m]
+  // device block, 256-byte aligned parts: error word | Dmask (d/32 words) | S [m][d] | St [d][m]
   auto round256 = [](size_t v) { return (v + 255) / 256 * 256; };
   const size_t n_mask = static_cast<size_t>(d) / 32;
   const size_t sz_S = static_cast<size_t>(m) * d * sizeof(uint16_t);
-  const size_t off_mask = 0;
-  const size_t off_S2 = round256(n_mask * 4);
+  const size_t off_err = 0;
+  const size_t off_mask = 256;
+  const size_t off_S2 = off_mask + round256(n_mask * 4);
   const size_t off_St = off_S2 + round256(sz_S);
   const size_t total = off_St + round256(sz_S);
   void* blk = nullptr;
@@ -138,6 +164,28 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
   kp.Dmask = reinterpret_cast<const uint32_t*>(static_cast<uint8_t*>(blk) + off_mask);
   kp.S = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(blk) + off_S2);
   kp.St = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(blk) + off_St);
+  kp.err = reinterpret_cast<int*>(static_cast<uint8_t*>(blk) + off_err);
+
+  int nsm = 0;
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  ctx->num_sms = nsm > 0 ? nsm : 148;
+  const char* kern = std::getenv("TQ_KERNELS");
+  ctx->use_tc = !(kern && std::strcmp(kern, "generic") == 0);
+  // projection error bound coefficient: 4 * 18 * 2^-22 * max_j ||S_j||
+  // and max_j ||S_j||_1 * 2^-25 / 64 for binary16 underflow of the scaled residual
+  double smax = 0.0, s1max = 0.0;
+  for (int j = 0; j < m; ++j) {
+    double acc = 0.0, acc1 = 0.0;
+    for (int i = 0; i < d; ++i) {
+      const double v = half_bits_to_double(ctx->S_bits[static_cast<size_t>(j) * d + i]);
+      acc += v * v;
+      acc1 += std::fabs(v);
+    }
+    smax = std::max(smax, std::sqrt(acc));
+    s1max = std::max(s1max, acc1);
+  }
+  ctx->qjl_eps_scale = static_cast<float>(4.0 * 18.0 * std::ldexp(1.0, -22) * smax);
+  ctx->qjl_eps_abs = static_cast<float>(2.0 * s1max * std::ldexp(1.0, -25) / 64.0);
   *out = ctx;
   return TQ_OK;
 }
@@ -181,7 +229,7 @@ tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_
   if (!aligned(x, 16) || (static_cast<size_t>(ld_x) * esz) % 16)
     return fail(TQ_ERR_INVALID_ARG, "x and its row stride must be 16-byte aligned");
   if ((st = check_packed(ctx, out)) != TQ_OK) return st;
-  int err = launch_quantize(ctx->kp, x, x_dtype == TQ_BF16, n_rows, ld_x, to_internal(out), stream);
+  int err = launch_quantize(*ctx, x, x_dtype == TQ_BF16, n_rows, ld_x, to_internal(out), stream);
   if (err) return cuda_fail(err, "tq_quantize launch");
   return TQ_OK;
 }

@@ -24,6 +24,7 @@ struct KParams {
   const uint32_t* Dmask;              // d/32 words, bit i set iff D_i = -1
   const uint16_t* S;                  // [m][d] binary16
   const uint16_t* St;                 // [d][m] binary16 (transpose)
+  int* err;                           // device error word (a bounded wait ran out)
 };
 
 struct Packed {
@@ -51,7 +52,7 @@ int launch_logits_generic(const KParams& P, const float* qp, int64_t n_sets, int
                           int64_t n_keys, float* out, void* stream);
 int launch_dequant_generic(const KParams& P, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
                            void* stream);
-int launch_quantize(const KParams& P, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x,
+int launch_quantize(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x,
                     const Packed& out, void* stream);
 int launch_qprep(const KParams& P, const void* q, int q_is_bf16, int64_t n_queries, float* qp, void* stream);
 int launch_logits(const KParams& P, const float* qp, int64_t n_sets, int g, const Packed& keys,
@@ -65,10 +66,23 @@ const char* cuda_error_string(int err);
 
 }  // namespace tq
 
+struct tq_ctx;
+
+namespace tq {
+// d = 128 hot-path kernels (quantize_d128.cu, ...)
+bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows);
+int launch_quantize_d128(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
+                         const Packed& out, void* stream);
+}  // namespace tq
+
 struct tq_ctx {
   int d, b, m;
   uint64_t seed;
   int device;
+  int num_sms;
+  bool use_tc;                        // hot-path (tensor-core) kernels enabled
+  float qjl_eps_scale;                // projection error bound coefficients (quantize_d128.cu)
+  float qjl_eps_abs;
   std::vector<float> centroids, thresholds;
   std::vector<int8_t> D;
   std::vector<uint16_t> S_bits;

@@ -29,7 +29,7 @@ TQ_DEQUANT_PROD, TQ_DEQUANT_MSE = 0, 1
 SYMBOLS = [
     "tq_host_params", "tq_init", "tq_destroy", "tq_packed_sizes", "tq_get_params", "tq_quantize",
     "tq_logits_workspace_bytes", "tq_logits", "tq_dequant", "tq_topk", "tq_logits_bf16",
-    "tq_status_str", "tq_last_error", "tq_launch_count",
+    "tq_status_str", "tq_sync_status", "tq_last_error", "tq_launch_count",
 ]
 
 
@@ -52,6 +52,7 @@ _sig = {
     "tq_topk": (_i32, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "tq_logits_bf16": (_i32, [_vp, _vp, _i64, _i32, _i64, _i32, _vp, _vp]),
     "tq_status_str": (ctypes.c_char_p, [_i32]),
+    "tq_sync_status": (_i32, [_vp, _vp]),
     "tq_last_error": (ctypes.c_char_p, []),
     "tq_launch_count": (_u64, []),
 }
@@ -196,6 +197,10 @@ class TurboQuant:
         _check(_lib.tq_quantize(self._h, _ptr(x), _dtype_code(x), n, x.stride(0), out.c(), _stream(stream)),
                "tq_quantize")
         return out
+
+    def sync_status(self, stream=None):
+        """Wait for the stream and raise if a kernel's bounded wait ran out."""
+        _check(_lib.tq_sync_status(self._h, _stream(stream)), "tq_sync_status")
 
     def workspace_bytes(self, n_sets: int, g: int) -> int:
         return int(_lib.tq_logits_workspace_bytes(self._h, n_sets, g))

@@ -28,6 +28,21 @@ def tq():
     return _tq
 
 
+def make_ctx(tq, d, b, m, kernels="auto"):
+    """A context whose compute calls use the hot-path kernels ("auto") or the
+    general CUDA-core kernels ("generic"); the choice is fixed at creation."""
+    import os
+    old = os.environ.pop("TQ_KERNELS", None)
+    if kernels == "generic":
+        os.environ["TQ_KERNELS"] = "generic"
+    try:
+        return tq.TurboQuant(d, b, m, seed=0)
+    finally:
+        os.environ.pop("TQ_KERNELS", None)
+        if old is not None:
+            os.environ["TQ_KERNELS"] = old
+
+
 def edge_rows(d, rng):
     rows = [np.zeros(d), np.full(d, 0.5), np.eye(1, d, 3)[0] * 7.0, rng.standard_normal(d) * 1e-8,
             rng.standard_normal(d) * 3e3, np.concatenate([np.ones(2), np.zeros(d - 2)])]
@@ -37,7 +52,8 @@ def edge_rows(d, rng):
 def make_rows(d, n, dtype, seed):
     rng = np.random.default_rng(seed)
     x = rng.standard_normal((n, d)) * rng.uniform(0.1, 10, size=(n, 1))
-    x[: 6] = edge_rows(d, rng)
+    e = edge_rows(d, rng)
+    x[: min(6, n)] = e[: min(6, n)]
     x = x.astype(np.float32)
     if dtype == "bf16":
         bits = inputs.bf16_bits(x)
@@ -49,15 +65,45 @@ CASES = [(32, 2, 32), (64, 3, 64), (128, 2, 128), (128, 3, 128), (128, 4, 128), 
          (256, 3, 96), (512, 4, 256), (1024, 4, 1024), (2048, 2, 64), (4096, 3, 128)]
 
 
+@pytest.mark.parametrize("b", [2, 3, 4, 5])
+def test_quantize_d128_tensor_core_small_first(tq, b):
+    """The tcgen05 write half on a handful of rows (one partial tile)."""
+    d, m = 128, 128
+    xt, x = make_rows(d, 37, "bf16", seed=b)
+    P = op.Params(d, b, m, seed=0)
+    T = make_ctx(tq, d, b, m)
+    got = T.quantize(xt.cuda()).to_numpy()
+    T.sync_status()
+    parity.assert_quantize_ok(parity.compare_quantize(P, got, ot.quantize(x, P, keep_intermediates=True)))
+
+
+@pytest.mark.parametrize("b", [2, 3, 4, 5])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_quantize_d128_many_tiles(tq, b, dtype):
+    """Enough rows that every CTA loops over several tiles (phase flips of
+    every barrier), with a ragged last tile."""
+    d, m, n = 128, 128, 100003
+    xt, x = make_rows(d, n, dtype, seed=100 + b)
+    P = op.Params(d, b, m, seed=0)
+    T = make_ctx(tq, d, b, m)
+    got = T.quantize(xt.cuda()).to_numpy()
+    T.sync_status()
+    rep = parity.compare_quantize(P, got, ot.quantize(x, P, keep_intermediates=True))
+    parity.assert_quantize_ok(rep)
+
+
 @pytest.mark.parametrize("d,b,m", CASES)
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_quantize_parity(tq, d, b, m, dtype):
+@pytest.mark.parametrize("kernels", ["auto", "generic"])
+def test_quantize_parity(tq, d, b, m, dtype, kernels):
+    if kernels == "generic" and d != 128:
+        pytest.skip("shapes other than d = 128 always use the general kernels")
     n = 1531 if d <= 1024 else 301
     xt, x = make_rows(d, n, dtype, seed=d * 10 + b)
     P = op.Params(d, b, m, seed=0)
-    T = tq.TurboQuant(d, b, m, seed=0)
+    T = make_ctx(tq, d, b, m, kernels)
     got = T.quantize(xt.cuda()).to_numpy()
-    torch.cuda.synchronize()
+    T.sync_status()
     want = ot.quantize(x, P, keep_intermediates=True)
     rep = parity.compare_quantize(P, got, want)
     parity.assert_quantize_ok(rep)
