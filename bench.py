@@ -40,6 +40,8 @@ WORKLOADS = {
     "decode-128k-b3": dict(batch=8, ctx=131072, b=3, m=128, kv_heads=8, q_heads=32, d=128),
     "decode-128k-b4": dict(batch=8, ctx=131072, b=4, m=128, kv_heads=8, q_heads=32, d=128),
     "decode-8k-b3": dict(batch=1, ctx=8192, b=3, m=128, kv_heads=8, q_heads=32, d=128),
+    # a 1M-row case (268 MB per tensor, above L2) for profiler captures
+    "decode-2x64k-b3": dict(batch=2, ctx=65536, b=3, m=128, kv_heads=8, q_heads=32, d=128),
 }
 METRIC = "compressed-key logits/s and % HBM roofline (d=128,b=3); quantize rows/s"
 UNIT = "logits/s"

@@ -1,0 +1,344 @@
+// Read half, value reconstruction at d = 128, m = 128 on sm_100a.
+//
+//   PROD: x~ = R^T (norm yhat + sqrt(pi/2)/m rnorm S^T z)   ai.spot.hk "Google
+//         TurboQuant", "無偏內積估計" (unbiased inverse of the quantizer)
+//   MSE:  x~ = R^T (norm yhat)                              Qiita TurboQuant
+//         explainer, "APIの構成" (values through the MSE stage alone)
+//   R^T = D H_d / sqrt(d)                                   0h-n0.github.io "ICLR
+//         2026論文解説: TurboQuant", "Step 1: PolarQuant"
+//
+// One thread per row (two warpgroups of 128 rows, persistent CTAs).  S^T z is
+// a 128 x 128 x 128 tensor-core product per tile: with z_j = 1 - 2 b_j,
+// S^T z = colsum(S) - 2 S^T b, and the sign bits b go into TMEM as binary16
+// values {0, 2^-14} (two shifts and a mask per pair of bits; S b is exact
+// in the MMA, the 2^14 comes back out as an exact scaling).  The centroid
+// decode, the inverse Walsh-Hadamard transform, D, 1/sqrt(d) and the output
+// rounding run in registers; the finished tile is written back by a TMA
+// tensor store from a swizzled shared-memory stage.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+
+#include "sm100.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128, kM = 128, kTile = 128, kWG = 2, kThreads = kWG * 128;
+constexpr long long kWaitCycles = 2000000000ll;
+constexpr uint32_t kTmemCols = 512;     // per warpgroup: 128 D columns + 64 A columns (in 256)
+
+struct DequantD128Args {
+  float D[kD];                          // Rademacher signs as +-1.0f
+  float colsum[kD];                     // sum_j S[j][i]
+  int* err;
+};
+
+template <bool BF16OUT>
+struct OutStage {
+  static constexpr int kColsPerBox = BF16OUT ? 64 : 32;
+  static constexpr int kBoxes = kD / kColsPerBox;
+  static constexpr int kBytes = kBoxes * kTile * 128;     // 32 KB or 64 KB
+};
+
+template <bool BF16OUT>
+constexpr size_t dequant_smem_bytes() {
+  return 1024 + 32768 /*St*/ + kWG * OutStage<BF16OUT>::kBytes + 128;
+}
+
+__device__ __forceinline__ void tma_store_2d(const void* tmap, const void* smem_src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(tmap), "r"(smem_u32(smem_src)), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+template <int B, bool PROD, bool BF16OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P, const DequantD128Args X,
+                  const Packed in, int64_t n_rows) {
+  constexpr int L = 1 << B;
+  constexpr int kStage = OutStage<BF16OUT>::kBytes;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sSt = smem;                                   // B operand: St (N = i, K = j), swizzled
+  uint8_t* sOut = smem + 32768;
+  uint64_t* mdone = reinterpret_cast<uint64_t*>(sOut + kWG * kStage);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kWG);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* lut = reinterpret_cast<float*>(tmem_slot + 2);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
+  if (tid == 0) {
+    for (int i = 0; i < kWG; ++i) mbar_init(&mdone[i], 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (tid < L) lut[tid] = P.c[tid];
+  if (PROD) {
+    // B operand row i (output coordinate), K position kappa holds S[j(kappa)][i]
+    // in the order the sign bits are laid out in TMEM (see the A construction):
+    // column c = kappa / 2 holds bits (c % 16) and (c % 16) + 16 of sign word
+    // c / 16, so j(kappa) = 32 (c / 16) + (c % 16) + 16 (kappa % 2).
+    uint16_t* sSt16 = reinterpret_cast<uint16_t*>(sSt);
+    for (int e = tid; e < kD * kM; e += kThreads) {
+      const int i = e >> 7, kappa = e & 127;
+      const int c = kappa >> 1, j = 32 * (c >> 4) + (c & 15) + 16 * (kappa & 1);
+      const int kb = kappa >> 6, chunk = (kappa & 63) >> 3, within = kappa & 7;
+      sSt16[(kb * 16384 + i * 128 + ((chunk ^ (i & 7)) << 4)) / 2 + within] = P.St[i * kM + j];
+    }
+    fence_proxy_async_smem();
+  }
+  if (PROD && warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = PROD ? *tmem_slot : 0u;
+
+  const int wg = warp >> 2, wl = warp & 3;
+  const bool leader = (wl == 0 && lane == 0);
+  const int trow = wl * 32 + lane;
+  const uint32_t lane_base = static_cast<uint32_t>(wl * 32) << 16;
+  const uint32_t t_acc = tmem + lane_base + wg * 256;
+  const uint32_t t_a = t_acc + 128;
+  uint8_t* stage = sOut + wg * kStage;
+  const float inv_sqrt_d = 0.08838834764831845f;
+  const float qjl = P.qjl_scale;
+  const int64_t t_first = blockIdx.x + static_cast<int64_t>(wg) * gridDim.x;
+  const int64_t t_step = static_cast<int64_t>(kWG) * gridDim.x;
+  bool store_pending = false;
+  int mine = 0;
+  for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
+    const int64_t row = t * kTile + trow;
+    const bool valid = row < n_rows;
+    // ---- packed row -------------------------------------------------------------
+    uint32_t cw[B * 4];
+    uint4 sg = make_uint4(0u, 0u, 0u, 0u);
+    float nrm = 0.f, rn = 0.f;
+    if (valid) {
+      const uint4* cp = reinterpret_cast<const uint4*>(in.codes + row * (B * 16));
+#pragma unroll
+      for (int q = 0; q < B; ++q) {
+        const uint4 u = __ldg(cp + q);
+        cw[4 * q] = u.x; cw[4 * q + 1] = u.y; cw[4 * q + 2] = u.z; cw[4 * q + 3] = u.w;
+      }
+      if (PROD) sg = __ldg(reinterpret_cast<const uint4*>(in.signs + row * 16));
+      nrm = __ldg(in.norm + row);
+      rn = __ldg(in.rnorm + row);
+    } else {
+#pragma unroll
+      for (int w = 0; w < B * 4; ++w) cw[w] = 0u;
+    }
+    if (PROD) {
+      // sign bits -> binary16 {0, 2^-14}: column k of sign word w holds bits
+      // (k, k + 16) of the word, i.e. projections 32 w + k and 32 w + k + 16
+      const uint32_t sw[4] = {sg.x, sg.y, sg.z, sg.w};
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t a[32];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const uint32_t s = sw[half * 2 + q];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const uint32_t sh = (k <= 10) ? (s << (10 - k)) : (s >> (k - 10));
+            a[q * 16 + k] = sh & 0x04000400u;
+          }
+        }
+        tmem_st32(t_a + half * 32, a);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      if (named_bar_sync_or(1 + wg, 128, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
+      if (leader) {
+        tc_fence_after();
+        const uint32_t sbase = smem_u32(sSt);
+        const uint32_t idesc = idesc_f16_f32(kTile, kD);
+        const uint32_t d_tmem = tmem + wg * 256;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t bdesc = smem_desc_sw128(sbase + (k >> 2) * 16384 + (k & 3) * 32, 1024);
+          mma_f16_ts(d_tmem, d_tmem + 128 + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&mdone[wg]);
+      }
+    }
+    // ---- norm * yhat while the MMA runs ------------------------------------------
+    float v[kD];
+#pragma unroll
+    for (int e = 0; e < kD; ++e) {
+      const int bit = B * e, wi = bit >> 5, sh = bit & 31;
+      uint32_t code = cw[wi] >> sh;
+      if (sh + B > 32) code |= cw[wi + 1] << (32 - sh);
+      code &= (1u << B) - 1u;
+      float c;
+      if constexpr (B == 1) {
+        c = code ? P.c[1] : -P.c[1];
+      } else if constexpr (B == 2) {
+        const float mag = ((code == 0u) || (code == 3u)) ? P.c[3] : P.c[2];
+        c = (code & 2u) ? mag : -mag;
+      } else {
+        c = lut[code];
+      }
+      v[e] = nrm * c;
+    }
+    if (PROD) {
+      if (!mbar_wait(&mdone[wg], mine & 1, kWaitCycles)) { if (X.err) atomicCAS(X.err, 0, 5); atomicExch(abort_flag, 1); }
+      tc_fence_after();
+      // sum_j z_j S[j][i] = colsum_i - 2 * 2^14 * acc_i
+      const float w = qjl * rn;
+      const float w2 = -2.0f * 16384.0f * w;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t acc[32];
+        tmem_ld32(t_acc + c * 32, acc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const int i = c * 32 + k;
+          v[i] = fmaf(w2, __uint_as_float(acc[k]), fmaf(w, X.colsum[i], v[i]));
+        }
+      }
+      tc_fence_before();
+    }
+    // ---- inverse rotation: D H v / sqrt(d) -----------------------------------------
+#pragma unroll
+    for (int h = 2; h < kD; h <<= 1) {
+#pragma unroll
+      for (int e = 0; e < kD; e += 2) {
+        if ((e & h) == 0) {
+          const float2 a = make_float2(v[e], v[e + 1]), b = make_float2(v[e + h], v[e + h + 1]);
+          const float2 sum = __fadd2_rn(a, b);
+          const float2 dif = __ffma2_rn(b, make_float2(-1.f, -1.f), a);
+          v[e] = sum.x; v[e + 1] = sum.y; v[e + h] = dif.x; v[e + h + 1] = dif.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < kD; e += 2) {
+      const float a = v[e], b = v[e + 1];
+      v[e] = a + b;
+      v[e + 1] = a - b;
+    }
+    // ---- stage the row (swizzled for the TMA store) and write the tile ---------------
+    if (leader && store_pending) bulk_wait_read0();         // previous tile's store has read the stage
+    named_bar_sync(1 + wg, 128);
+    if (BF16OUT) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        uint32_t wv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = c * 8 + 2 * u;
+          const __nv_bfloat162 p = __floats2bfloat162_rn(v[e] * (X.D[e] * inv_sqrt_d),
+                                                         v[e + 1] * (X.D[e + 1] * inv_sqrt_d));
+          wv[u] = *reinterpret_cast<const uint32_t*>(&p);
+        }
+        const int bx = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4*>(stage + bx * (kTile * 128) + trow * 128 + ((cc ^ (trow & 7)) << 4)) =
+            make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        float4 o;
+        o.x = v[c * 4 + 0] * (X.D[c * 4 + 0] * inv_sqrt_d);
+        o.y = v[c * 4 + 1] * (X.D[c * 4 + 1] * inv_sqrt_d);
+        o.z = v[c * 4 + 2] * (X.D[c * 4 + 2] * inv_sqrt_d);
+        o.w = v[c * 4 + 3] * (X.D[c * 4 + 3] * inv_sqrt_d);
+        const int bx = c >> 3, cc = c & 7;
+        *reinterpret_cast<float4*>(stage + bx * (kTile * 128) + trow * 128 + ((cc ^ (trow & 7)) << 4)) = o;
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1 + wg, 128);
+    if (leader) {
+#pragma unroll
+      for (int bx = 0; bx < OutStage<BF16OUT>::kBoxes; ++bx)
+        tma_store_2d(&tmap_out, stage + bx * (kTile * 128), bx * OutStage<BF16OUT>::kColsPerBox,
+                     static_cast<int>(t * kTile));
+      bulk_commit();
+      store_pending = true;
+    }
+  }
+  if (leader && store_pending) bulk_wait0();               // all our stores have landed
+  __syncthreads();
+  if (PROD && warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int B, bool PROD, bool BF16OUT>
+int launch(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, cudaStream_t s) {
+  const KParams& P = ctx.kp;
+  auto encode = tensor_map_encoder();
+  if (!encode) return static_cast<int>(cudaErrorNotSupported);
+  CUtensorMap tmap;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(n_rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * (BF16OUT ? 2 : 4)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(OutStage<BF16OUT>::kColsPerBox), static_cast<cuuint32_t>(kTile)};
+  const cuuint32_t estr[2] = {1, 1};
+  if (encode(&tmap, BF16OUT ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, out, dims,
+             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return static_cast<int>(cudaErrorInvalidValue);
+  DequantD128Args X;
+  for (int i = 0; i < kD; ++i) {
+    X.D[i] = static_cast<float>(ctx.D[i]);
+    X.colsum[i] = ctx.colsum_d128[i];
+  }
+  X.err = P.err;
+  const size_t smem = dequant_smem_bytes<BF16OUT>();
+  cudaError_t e = cudaFuncSetAttribute(k_dequant_d128_tc<B, PROD, BF16OUT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return static_cast<int>(e);
+  const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
+  const int grid = static_cast<int>(n_tiles < ctx.num_sms ? n_tiles : ctx.num_sms);
+  k_dequant_d128_tc<B, PROD, BF16OUT><<<grid, kThreads, smem, s>>>(tmap, P, X, in, n_rows);
+  count_launch();
+  return static_cast<int>(cudaGetLastError());
+}
+
+template <int B>
+int launch_B(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int bf16, int prod, cudaStream_t s) {
+  if (prod) return bf16 ? launch<B, true, true>(ctx, in, n_rows, out, s) : launch<B, true, false>(ctx, in, n_rows, out, s);
+  return bf16 ? launch<B, false, true>(ctx, in, n_rows, out, s) : launch<B, false, false>(ctx, in, n_rows, out, s);
+}
+
+}  // namespace
+
+bool dequant_d128_applies(const tq_ctx& ctx, int64_t n_rows) {
+  const KParams& P = ctx.kp;
+  return P.d == kD && P.m == kM && P.B >= 1 && P.B <= 4 && n_rows > 0 && n_rows < (int64_t(1) << 31) &&
+         ctx.use_tc && tensor_map_encoder() != nullptr;
+}
+
+int launch_dequant_d128(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
+                        void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (ctx.kp.B) {
+    case 1: return launch_B<1>(ctx, in, n_rows, out, out_is_bf16, prod, s);
+    case 2: return launch_B<2>(ctx, in, n_rows, out, out_is_bf16, prod, s);
+    case 3: return launch_B<3>(ctx, in, n_rows, out, out_is_bf16, prod, s);
+    default: return launch_B<4>(ctx, in, n_rows, out, out_is_bf16, prod, s);
+  }
+}
+
+}  // namespace tq

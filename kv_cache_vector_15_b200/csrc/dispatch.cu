@@ -16,9 +16,11 @@ int launch_logits(const KParams& P, const float* qp, int64_t n_sets, int g, cons
   return launch_logits_generic(P, qp, n_sets, g, keys, n_keys, out, stream);
 }
 
-int launch_dequant(const KParams& P, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
+int launch_dequant(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
                    void* stream) {
-  return launch_dequant_generic(P, in, n_rows, out, out_is_bf16, prod, stream);
+  if (dequant_d128_applies(ctx, n_rows))
+    return launch_dequant_d128(ctx, in, n_rows, out, out_is_bf16, prod, stream);
+  return launch_dequant_generic(ctx.kp, in, n_rows, out, out_is_bf16, prod, stream);
 }
 
 }  // namespace tq

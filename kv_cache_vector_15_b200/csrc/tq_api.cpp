@@ -186,6 +186,14 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
   }
   ctx->qjl_eps_scale = static_cast<float>(4.0 * 18.0 * std::ldexp(1.0, -22) * smax);
   ctx->qjl_eps_abs = static_cast<float>(2.0 * s1max * std::ldexp(1.0, -25) / 64.0);
+  for (int i = 0; i < 128; ++i) ctx->colsum_d128[i] = 0.f;
+  if (d == 128) {
+    for (int i = 0; i < d; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < m; ++j) acc += half_bits_to_double(ctx->S_bits[static_cast<size_t>(j) * d + i]);
+      ctx->colsum_d128[i] = static_cast<float>(acc);
+    }
+  }
   *out = ctx;
   return TQ_OK;
 }
@@ -274,7 +282,7 @@ tq_status tq_dequant(const tq_ctx* ctx, tq_packed in, int64_t n_rows, void* out,
   if (!out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
   if (!aligned(out, 16)) return fail(TQ_ERR_INVALID_ARG, "out must be 16-byte aligned");
   if ((st = check_packed(ctx, in)) != TQ_OK) return st;
-  int err = launch_dequant(ctx->kp, to_internal(in), n_rows, out, out_dtype == TQ_BF16, mode == TQ_DEQUANT_PROD, stream);
+  int err = launch_dequant(*ctx, to_internal(in), n_rows, out, out_dtype == TQ_BF16, mode == TQ_DEQUANT_PROD, stream);
   if (err) return cuda_fail(err, "tq_dequant launch");
   return TQ_OK;
 }

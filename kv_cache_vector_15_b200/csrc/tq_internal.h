@@ -57,7 +57,7 @@ int launch_quantize(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_r
 int launch_qprep(const KParams& P, const void* q, int q_is_bf16, int64_t n_queries, float* qp, void* stream);
 int launch_logits(const KParams& P, const float* qp, int64_t n_sets, int g, const Packed& keys,
                   int64_t n_keys, float* out, void* stream);
-int launch_dequant(const KParams& P, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
+int launch_dequant(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
                    void* stream);
 int launch_topk(const float* scores, int64_t rows, int64_t cols, int k, int32_t* idx, float* val, void* stream);
 int launch_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, int d, float* out,
@@ -73,6 +73,9 @@ namespace tq {
 bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows);
 int launch_quantize_d128(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
                          const Packed& out, void* stream);
+bool dequant_d128_applies(const tq_ctx& ctx, int64_t n_rows);
+int launch_dequant_d128(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
+                        void* stream);
 }  // namespace tq
 
 struct tq_ctx {
@@ -83,6 +86,7 @@ struct tq_ctx {
   bool use_tc;                        // hot-path (tensor-core) kernels enabled
   float qjl_eps_scale;                // projection error bound coefficients (quantize_d128.cu)
   float qjl_eps_abs;
+  float colsum_d128[128];             // sum_j S[j][i] (d = 128 only)
   std::vector<float> centroids, thresholds;
   std::vector<int8_t> D;
   std::vector<uint16_t> S_bits;
