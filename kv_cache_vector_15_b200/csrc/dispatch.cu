@@ -11,9 +11,11 @@ int launch_quantize(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_r
   return launch_quantize_generic(ctx.kp, x, x_is_bf16, n_rows, ld_x, out, stream);
 }
 
-int launch_logits(const KParams& P, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
+int launch_logits(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
                   float* out, void* stream) {
-  return launch_logits_generic(P, qp, n_sets, g, keys, n_keys, out, stream);
+  if (logits_d128_applies(ctx, n_sets, g, n_keys))
+    return launch_logits_d128(ctx, qp, n_sets, g, keys, n_keys, out, stream);
+  return launch_logits_generic(ctx.kp, qp, n_sets, g, keys, n_keys, out, stream);
 }
 
 int launch_dequant(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,

@@ -1,0 +1,358 @@
+// Read half, estimated attention logits from packed keys at d = 128, m = 128,
+// b = 2 or 3 (1- or 2-bit codes), on the tcgen05 tensor cores.
+//
+//   logit(q, k) = norm <R q, yhat> + rnorm sqrt(pi/2)/m <S R q, z>
+//   -- Qiita TurboQuant explainer, "Stage 2: QJL" (the estimator), with
+//      q_rot = R q and sq = S q_rot prepared once per query.
+//
+// Both inner products are linear in the stored bits.  For 1- and 2-bit
+// symmetric Lloyd-Max codebooks the centroid is affine in the code bits,
+//   B = 2: c[code] = -c3 + (c3 - c2) b0 + (c3 + c2) b1,   B = 1: c = -c1 + 2 c1 b0,
+// and z_j = 1 - 2 bit_j, so for each key
+//   <q_rot, yhat> = const_q + sum_(bits) weight(bit) q_rot[coord(bit)] * bit
+//   <sq, z>       = sum_j sq_j - 2 sum_j sq_j bit_j.
+// Each key's bits become an unsigned 8-bit row of 0/1 values in TMEM (two
+// integer ops per four bits, taken straight from the packed words), and one
+// integer MMA (kind::i8, exact int32 accumulation) per 128-key tile multiplies
+// them with the set's queries, which sit in shared memory as three signed
+// 8-bit limbs of a fixed-point value per (bit, query).  The epilogue recombines
+// the limbs, adds the constants and applies norm and rnorm.
+//
+// Work split: persistent CTAs of four warpgroups; each warpgroup walks a
+// contiguous range of 128-key tiles (so the set, and with it the query operand
+// it builds in its own shared-memory slot, changes rarely), one thread per key.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "sm100.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128, kM = 128, kTile = 128, kWG = 4, kThreads = kWG * 128;
+constexpr long long kWaitCycles = 2000000000ll;
+constexpr uint32_t kTmemCols = 512;          // per warpgroup: 96 A columns + 32 D columns (in 128)
+
+__host__ __device__ constexpr uint32_t idesc_i8(uint32_t M, uint32_t N) {
+  return (2u << 4)              // D format: S32
+         | (0u << 7)            // A: unsigned 8-bit
+         | (1u << 10)           // B: signed 8-bit
+         | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <int B>
+struct Shape {
+  static constexpr int kCodeWords = B * 4;                  // 32-bit words of codes per key
+  static constexpr int kAWords = 8 * (kCodeWords + 4);      // 0/1 bytes, four per TMEM column
+  static constexpr int kK = 4 * kAWords;                    // K of the MMA (bytes)
+  static constexpr int kKBlocks = kK / 128;                 // 128-byte swizzle atoms along K
+  static constexpr int kKSteps = kK / 32;
+};
+
+struct LogitsArgs {
+  float wbit[2];                  // weight of code bit 0 / 1 in the centroid
+  float cconst;                   // centroid constant term
+  int* err;
+};
+
+template <int B, int G, int NG>
+__global__ void __launch_bounds__(kThreads, 1)
+k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ qp, int64_t n_sets,
+                 int64_t n_keys, const Packed keys, float* __restrict__ out) {
+  using S = Shape<B>;
+  constexpr int N = 2 * NG;
+  constexpr int kBBytes = S::kKBlocks * N * 128;            // query operand per warpgroup
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wg = warp >> 2, wl = warp & 3;
+  uint8_t* sB = smem + wg * kBBytes;
+  float* sScal = reinterpret_cast<float*>(smem + kWG * kBBytes) + wg * 64;   // per-warpgroup scalars
+  uint64_t* mdone = reinterpret_cast<uint64_t*>(smem + kWG * kBBytes + kWG * 64 * 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kWG);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  if (tid == 0) {
+    for (int i = 0; i < kWG; ++i) mbar_init(&mdone[i], 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool leader = (wl == 0 && lane == 0);
+  const int trow = wl * 32 + lane;
+  const uint32_t t_base = tmem + (static_cast<uint32_t>(wl * 32) << 16) + wg * 128;   // this thread's lane
+  const uint32_t t_a = t_base, t_d = t_base + S::kAWords;
+
+  // contiguous tile range of this warpgroup
+  const int64_t tiles_per_set = (n_keys + kTile - 1) / kTile;
+  const int64_t n_tiles = tiles_per_set * n_sets;
+  const int64_t n_wg = static_cast<int64_t>(gridDim.x) * kWG;
+  const int64_t wid = static_cast<int64_t>(blockIdx.x) * kWG + wg;
+  const int64_t t0 = n_tiles * wid / n_wg, t1 = n_tiles * (wid + 1) / n_wg;
+  int64_t cur_set = -1;
+  int mine = 0;
+  for (int64_t t = t0; t < t1; ++t, ++mine) {
+    const int64_t set = t / tiles_per_set;
+    const int64_t key = (t % tiles_per_set) * kTile + trow;
+    if (set != cur_set) {
+      // ---- build the query operand of this set --------------------------------
+      cur_set = set;
+      named_bar_sync(1 + wg, 128);                      // previous tile's MMA inputs no longer in use
+      // thread trow owns coordinate/projection trow; per query maxima for scaling
+      float* sMax = sScal;                              // [0..G): mse max, [G..2G): qjl max
+      if (trow < 2 * G) sMax[trow] = 0.f;
+      named_bar_sync(1 + wg, 128);
+      const float* qs = qp + set * G * (kD + kM);
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        float a = fabsf(qs[q * (kD + kM) + trow]);
+        float b = fabsf(qs[q * (kD + kM) + kD + trow]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+          b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
+        }
+        if (lane == 0) {
+          atomicMax(reinterpret_cast<int*>(&sMax[q]), __float_as_int(a));
+          atomicMax(reinterpret_cast<int*>(&sMax[G + q]), __float_as_int(b));
+        }
+      }
+      named_bar_sync(1 + wg, 128);
+      // fixed-point scales: |value| * 2^F <= 2^22
+      float scale[2 * G];
+      const float wmax = fmaxf(fabsf(X.wbit[0]), B == 2 ? fabsf(X.wbit[1]) : 0.f);
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        const float vm = sMax[q] * wmax, vq = sMax[G + q] * 2.f;
+        int e1 = 0, e2 = 0;
+        frexpf(vm > 0.f ? vm : 1.f, &e1);
+        frexpf(vq > 0.f ? vq : 1.f, &e2);
+        scale[q] = ldexpf(1.f, 22 - e1);
+        scale[G + q] = ldexpf(1.f, 22 - e2);
+      }
+      // operand bytes: K position kappa (byte t of A column o) of this thread
+#pragma unroll
+      for (int r = 0; r < S::kK / 128; ++r) {
+        const int kappa = trow + 128 * r;
+        const int o = kappa >> 2, tb = kappa & 3;
+        int8_t limb[N];
+#pragma unroll
+        for (int n = 0; n < N; ++n) limb[n] = 0;
+        if (o < 8 * S::kCodeWords) {
+          const int c = o >> 3, k = o & 7;
+          const int s = 32 * c + k + 8 * tb;          // bit position in the code stream
+          const int coord = s / B, plane = s % B;
+          const float w = X.wbit[plane];
+#pragma unroll
+          for (int q = 0; q < G; ++q) {
+            const int v = __float2int_rn(w * qs[q * (kD + kM) + coord] * scale[q]);
+            const int l0 = static_cast<int8_t>(v & 0xff);
+            const int r1 = (v - l0) >> 8;
+            const int l1 = static_cast<int8_t>(r1 & 0xff);
+            const int l2 = (r1 - l1) >> 8;
+            limb[3 * q] = static_cast<int8_t>(l0);
+            limb[3 * q + 1] = static_cast<int8_t>(l1);
+            limb[3 * q + 2] = static_cast<int8_t>(l2);
+          }
+        } else {
+          const int c = (o - 8 * S::kCodeWords) >> 3, k = o & 7;
+          const int j = 32 * c + k + 8 * tb;           // projection
+#pragma unroll
+          for (int q = 0; q < G; ++q) {
+            const int v = __float2int_rn(-2.f * qs[q * (kD + kM) + kD + j] * scale[G + q]);
+            const int l0 = static_cast<int8_t>(v & 0xff);
+            const int r1 = (v - l0) >> 8;
+            const int l1 = static_cast<int8_t>(r1 & 0xff);
+            const int l2 = (r1 - l1) >> 8;
+            limb[NG + 3 * q] = static_cast<int8_t>(l0);
+            limb[NG + 3 * q + 1] = static_cast<int8_t>(l1);
+            limb[NG + 3 * q + 2] = static_cast<int8_t>(l2);
+          }
+        }
+        const int kb = kappa >> 7, chunk = (kappa & 127) >> 4, within = kappa & 15;
+#pragma unroll
+        for (int n = 0; n < N; ++n)
+          sB[kb * (N * 128) + n * 128 + ((chunk ^ (n & 7)) << 4) + within] = static_cast<uint8_t>(limb[n]);
+      }
+      // per-query constants: c_const * sum q_rot, sum sq, and the inverse scales
+      named_bar_sync(1 + wg, 128);
+      if (trow < 2 * G) {
+        const int q = trow % G;
+        const bool isq = trow >= G;
+        float acc = 0.f;
+        for (int i = 0; i < 128; ++i) acc += qs[q * (kD + kM) + (isq ? kD : 0) + i];
+        sScal[2 * G + trow] = isq ? acc : X.cconst * acc;
+        sScal[4 * G + trow] = 1.f / scale[trow];
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1 + wg, 128);
+    }
+    // ---- decode this thread's key into TMEM ------------------------------------------
+    const bool valid = key < n_keys;
+    const int64_t row = set * n_keys + key;
+    uint32_t cw[S::kCodeWords], sw[4];
+    float nrm = 0.f, rn = 0.f;
+    if (valid) {
+      const uint4* cp = reinterpret_cast<const uint4*>(keys.codes + row * (B * 16));
+#pragma unroll
+      for (int q = 0; q < B; ++q) {
+        const uint4 u = __ldg(cp + q);
+        cw[4 * q] = u.x; cw[4 * q + 1] = u.y; cw[4 * q + 2] = u.z; cw[4 * q + 3] = u.w;
+      }
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(keys.signs + row * 16));
+      sw[0] = u.x; sw[1] = u.y; sw[2] = u.z; sw[3] = u.w;
+      nrm = __ldg(keys.norm + row);
+      rn = __ldg(keys.rnorm + row) * P.qjl_scale;
+    } else {
+#pragma unroll
+      for (int w = 0; w < S::kCodeWords; ++w) cw[w] = 0u;
+      sw[0] = sw[1] = sw[2] = sw[3] = 0u;
+    }
+    {
+      uint32_t a[32];
+      int n = 0, col = 0;
+#pragma unroll
+      for (int c = 0; c < S::kCodeWords + 4; ++c) {
+        const uint32_t w = c < S::kCodeWords ? cw[c] : sw[c - S::kCodeWords];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          a[n++] = (w >> k) & 0x01010101u;
+          if (n == 32) {
+            tmem_st32(t_a + col, a);
+            col += 32;
+            n = 0;
+          }
+        }
+      }
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    if (named_bar_sync_or(1 + wg, 128, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
+    if (leader) {
+      tc_fence_after();
+      const uint32_t sbase = smem_u32(sB);
+      const uint32_t idesc = idesc_i8(kTile, N);
+      const uint32_t d_tmem = tmem + wg * 128 + S::kAWords;
+#pragma unroll
+      for (int k = 0; k < S::kKSteps; ++k) {
+        const uint64_t bdesc = smem_desc_sw128(sbase + (k >> 2) * (N * 128) + (k & 3) * 32, 1024);
+        mma_i8_ts(d_tmem, tmem + wg * 128 + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
+      }
+      mma_commit(&mdone[wg]);
+    }
+    if (!mbar_wait(&mdone[wg], mine & 1, kWaitCycles)) {
+      if (X.err) atomicCAS(X.err, 0, 6);
+      atomicExch(abort_flag, 1);
+    }
+    tc_fence_after();
+    // ---- epilogue: recombine limbs, constants, norms ----------------------------------
+    uint32_t acc[32];
+    tmem_ld32(t_d, acc);
+    tmem_wait_ld();
+    tc_fence_before();
+    if (valid) {
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        const int mse_i = static_cast<int>(acc[3 * q]) + (static_cast<int>(acc[3 * q + 1]) << 8) +
+                          (static_cast<int>(acc[3 * q + 2]) << 16);
+        const int qjl_i = static_cast<int>(acc[NG + 3 * q]) + (static_cast<int>(acc[NG + 3 * q + 1]) << 8) +
+                          (static_cast<int>(acc[NG + 3 * q + 2]) << 16);
+        const float mse = fmaf(static_cast<float>(mse_i), sScal[4 * G + q], sScal[2 * G + q]);
+        const float qjl = fmaf(static_cast<float>(qjl_i), sScal[4 * G + G + q], sScal[2 * G + G + q]);
+        out[(set * G + q) * n_keys + key] = fmaf(nrm, mse, rn * qjl);
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int B, int G>
+int launch_G(const tq_ctx& ctx, const float* qp, int64_t n_sets, int64_t n_keys, const Packed& keys, float* out,
+             cudaStream_t s) {
+  constexpr int NG = (3 * G <= 16) ? 16 : 32;
+  using Sh = Shape<B>;
+  const KParams& P = ctx.kp;
+  LogitsArgs X;
+  if (B == 2) {
+    X.wbit[0] = P.c[3] - P.c[2];
+    X.wbit[1] = P.c[3] + P.c[2];
+    X.cconst = -P.c[3];
+  } else {
+    X.wbit[0] = 2.f * P.c[1];
+    X.wbit[1] = 0.f;
+    X.cconst = -P.c[1];
+  }
+  X.err = P.err;
+  const size_t smem = 1024 + static_cast<size_t>(kWG) * Sh::kKBlocks * (2 * NG) * 128 + kWG * 64 * 4 + 64;
+  cudaError_t e = cudaFuncSetAttribute(k_logits_d128_i8<B, G, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return static_cast<int>(e);
+  const int64_t n_tiles = ((n_keys + kTile - 1) / kTile) * n_sets;
+  int64_t grid = (n_tiles + kWG - 1) / kWG;
+  if (grid > ctx.num_sms) grid = ctx.num_sms;
+  k_logits_d128_i8<B, G, NG><<<static_cast<int>(grid), kThreads, smem, s>>>(P, X, qp, n_sets, n_keys, keys, out);
+  count_launch();
+  return static_cast<int>(cudaGetLastError());
+}
+
+template <int B>
+int launch_B(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, int64_t n_keys, const Packed& keys, float* out,
+             cudaStream_t s) {
+  switch (g) {
+    case 1: return launch_G<B, 1>(ctx, qp, n_sets, n_keys, keys, out, s);
+    case 2: return launch_G<B, 2>(ctx, qp, n_sets, n_keys, keys, out, s);
+    case 3: return launch_G<B, 3>(ctx, qp, n_sets, n_keys, keys, out, s);
+    case 4: return launch_G<B, 4>(ctx, qp, n_sets, n_keys, keys, out, s);
+    case 5: return launch_G<B, 5>(ctx, qp, n_sets, n_keys, keys, out, s);
+    case 6: return launch_G<B, 6>(ctx, qp, n_sets, n_keys, keys, out, s);
+    case 7: return launch_G<B, 7>(ctx, qp, n_sets, n_keys, keys, out, s);
+    default: return launch_G<B, 8>(ctx, qp, n_sets, n_keys, keys, out, s);
+  }
+}
+
+}  // namespace
+
+bool logits_d128_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys) {
+  const KParams& P = ctx.kp;
+  // the A operand and the accumulator share a 128-column TMEM slice per warpgroup
+  const int a_cols = 8 * (P.B * 4 + 4), n_cols = (3 * g <= 16) ? 32 : 64;
+  return P.d == kD && P.m == kM && (P.B == 1 || P.B == 2) && g >= 1 && g <= 8 && a_cols + n_cols <= 128 &&
+         n_keys > 0 && n_sets > 0 && ctx.use_tc;
+}
+
+int launch_logits_d128(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
+                       float* out, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (ctx.kp.B == 1) return launch_B<1>(ctx, qp, n_sets, g, n_keys, keys, out, s);
+  return launch_B<2>(ctx, qp, n_sets, g, n_keys, keys, out, s);
+}
+
+}  // namespace tq

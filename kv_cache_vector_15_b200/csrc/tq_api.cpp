@@ -266,7 +266,7 @@ tq_status tq_logits(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t 
   float* qp = static_cast<float*>(workspace);
   int err = launch_qprep(ctx->kp, q, q_dtype == TQ_BF16, n_sets * g, qp, stream);
   if (err) return cuda_fail(err, "tq_logits query-prep launch");
-  err = launch_logits(ctx->kp, qp, n_sets, g, to_internal(keys), n_keys, out, stream);
+  err = launch_logits(*ctx, qp, n_sets, g, to_internal(keys), n_keys, out, stream);
   if (err) return cuda_fail(err, "tq_logits launch");
   return TQ_OK;
 }

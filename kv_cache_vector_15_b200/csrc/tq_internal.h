@@ -55,7 +55,7 @@ int launch_dequant_generic(const KParams& P, const Packed& in, int64_t n_rows, v
 int launch_quantize(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x,
                     const Packed& out, void* stream);
 int launch_qprep(const KParams& P, const void* q, int q_is_bf16, int64_t n_queries, float* qp, void* stream);
-int launch_logits(const KParams& P, const float* qp, int64_t n_sets, int g, const Packed& keys,
+int launch_logits(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys,
                   int64_t n_keys, float* out, void* stream);
 int launch_dequant(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
                    void* stream);
@@ -74,6 +74,9 @@ bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows);
 int launch_quantize_d128(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
                          const Packed& out, void* stream);
 bool dequant_d128_applies(const tq_ctx& ctx, int64_t n_rows);
+bool logits_d128_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys);
+int launch_logits_d128(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
+                       float* out, void* stream);
 int launch_dequant_d128(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
                         void* stream);
 }  // namespace tq

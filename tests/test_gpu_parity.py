@@ -139,6 +139,26 @@ def test_logits_parity_on_oracle_packed_keys(tq, d, b, m, n_sets, g, n_keys, qdt
     assert np.all(err <= tol + 1e-30), float(np.max(err / (tol + 1e-30)))
 
 
+@pytest.mark.parametrize("b,g", [(3, 4), (2, 8), (3, 5), (3, 1)])
+@pytest.mark.parametrize("kernels", ["auto", "generic"])
+def test_logits_d128_many_tiles_and_sets(tq, b, g, kernels):
+    """Several 128-key tiles per warpgroup, sets changing inside a warpgroup's
+    tile range, ragged last tile of every set."""
+    d, m, n_sets, n_keys = 128, 128, 7, 20001
+    P = op.Params(d, b, m, seed=0)
+    rng = np.random.default_rng(b * 10 + g)
+    k = rng.standard_normal((n_sets * n_keys, d)) * rng.uniform(0.1, 10, size=(n_sets * n_keys, 1))
+    pk = ot.quantize(k, P)
+    qt, q = make_rows(d, n_sets * g, "bf16", seed=3 + g)
+    T = make_ctx(tq, d, b, m, kernels)
+    got = T.logits(qt.cuda(), tq.Packed.from_numpy(pk), n_sets, g, n_keys).cpu().numpy()
+    T.sync_status()
+    want = ot.logits(q, pk, P, n_sets, g, n_keys)
+    tol = parity.logit_tolerance(q, np.linalg.norm(k, axis=1), n_sets, g, n_keys)
+    err = np.abs(got - want)
+    assert np.all(err <= tol + 1e-30), float(np.max(err / (tol + 1e-30)))
+
+
 @pytest.mark.parametrize("d,b,m", [(128, 3, 128), (128, 4, 128), (64, 2, 96), (1024, 4, 1024)])
 def test_end_to_end_quantize_then_logits(tq, d, b, m):
     """GPU quantize -> GPU logits against oracle quantize -> oracle logits.
@@ -160,14 +180,14 @@ def test_end_to_end_quantize_then_logits(tq, d, b, m):
     assert ok.all()
 
 
-@pytest.mark.parametrize("d,b,m", [(128, 3, 128), (128, 4, 128), (128, 2, 128), (64, 5, 32), (1024, 4, 1024),
-                                   (4096, 3, 64)])
+@pytest.mark.parametrize("d,b,m,n", [(128, 3, 128, 1029), (128, 4, 128, 1029), (128, 2, 128, 1029),
+                                     (64, 5, 32, 1029), (1024, 4, 1024, 1029), (4096, 3, 64, 130),
+                                     (128, 3, 128, 77777), (128, 5, 128, 40001)])
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
-def test_dequant_parity_on_oracle_packed_rows(tq, d, b, m, mode, out):
+def test_dequant_parity_on_oracle_packed_rows(tq, d, b, m, n, mode, out):
     P = op.Params(d, b, m, seed=0)
     rng = np.random.default_rng(d * 3 + b)
-    n = 1029 if d <= 1024 else 130
     x = rng.standard_normal((n, d)) * rng.uniform(0.1, 10, size=(n, 1))
     x[:6] = edge_rows(d, rng)
     pk = ot.quantize(x, P)
