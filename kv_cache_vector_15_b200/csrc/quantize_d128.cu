@@ -84,13 +84,15 @@ struct XStage {
   static constexpr int kColsPerBox = BF16IN ? 64 : 32;    // 128 bytes of a row per box
   static constexpr int kBoxes = kD / kColsPerBox;
   static constexpr int kBytes = kBoxes * kTile * 128;     // 32 KB (bf16) or 64 KB (fp32)
+  static constexpr int kStages = BF16IN ? 2 : 1;          // per warpgroup (shared memory budget)
 };
 
 constexpr int kSmemS = 32768;        // S as the MMA B operand (128 x 128 fp16, swizzled)
 
 template <bool BF16IN>
 constexpr size_t quant_smem_bytes() {
-  return 1024 /*alignment slack*/ + kSmemS + 2 * kWG * XStage<BF16IN>::kBytes + 256 /*barriers etc*/;
+  return 1024 /*alignment slack*/ + kSmemS + XStage<BF16IN>::kStages * kWG * XStage<BF16IN>::kBytes +
+         256 /*barriers etc*/;
 }
 
 __device__ __forceinline__ void flag_error(int* err, int* abort_flag, int code) {
@@ -120,11 +122,12 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
                    int64_t n_rows, const Packed out) {
   constexpr int L = 1 << B;
   constexpr int kStage = XStage<BF16IN>::kBytes;
+  constexpr int NS = XStage<BF16IN>::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sS = smem;
-  uint8_t* sX = smem + kSmemS;                                   // [warpgroup][2 buffers] stages
-  uint64_t* full = reinterpret_cast<uint64_t*>(sX + 2 * kWG * kStage);   // [warpgroup][2]
+  uint8_t* sX = smem + kSmemS;                                   // [warpgroup][NS buffers] stages
+  uint64_t* full = reinterpret_cast<uint64_t*>(sX + NS * kWG * kStage);  // [warpgroup][2]
   uint64_t* mdone = full + 2 * kWG;                              // [warpgroup]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kWG);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
@@ -164,7 +167,7 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
   const uint32_t t_acc = tmem + lane_base + wg * 256;            // projections, 128 columns
   const uint32_t t_a = t_acc + 128;                              // residual hi | lo, 128 columns
   const float sqrt_d = 11.313708498984761f;                      // sqrt(128)
-  uint8_t* stages = sX + wg * 2 * kStage;
+  uint8_t* stages = sX + wg * NS * kStage;
   uint64_t* wfull = full + 2 * wg;
   const int64_t t_first = blockIdx.x + static_cast<int64_t>(wg) * gridDim.x;
   const int64_t t_step = static_cast<int64_t>(kWG) * gridDim.x;
@@ -180,7 +183,7 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
   if (leader) {
     prefetch_tmap(&tmap);
     if (t_first < n_tiles) { issue_load(t_first, 0); ++issued[0]; }
-    if (t_first + t_step < n_tiles) { issue_load(t_first + t_step, 1); ++issued[1]; }
+    if (NS == 2 && t_first + t_step < n_tiles) { issue_load(t_first + t_step, 1); ++issued[1]; }
   }
 
   RowState<B> prev;
@@ -273,8 +276,8 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
   };
 
   for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
-    const int buf = mine & 1;
-    if (mbar_wait(&wfull[buf], (mine >> 1) & 1, kWaitCycles)) {
+    const int buf = mine % NS;
+    if (mbar_wait(&wfull[buf], (mine / NS) & 1, kWaitCycles)) {
       if (leader) ++waited[buf];
     } else {
       flag_error(X.err, abort_flag, 2);
@@ -437,7 +440,7 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
         mma_f16_ts(d_tmem, d_tmem + 128 + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
       }
       mma_commit(&mdone[wg]);
-      if (t + 2 * t_step < n_tiles) { issue_load(t + 2 * t_step, buf); ++issued[buf]; }
+      if (t + NS * t_step < n_tiles) { issue_load(t + NS * t_step, buf); ++issued[buf]; }
     }
     prev = cur;
     have_prev = true;
