@@ -124,27 +124,39 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
   const int64_t t_step = static_cast<int64_t>(kWG) * gridDim.x;
   bool store_pending = false;
   int mine = 0;
-  for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
-    const int64_t row = t * kTile + trow;
-    const bool valid = row < n_rows;
-    // ---- packed row -------------------------------------------------------------
-    uint32_t cw[B * 4];
-    uint4 sg = make_uint4(0u, 0u, 0u, 0u);
-    float nrm = 0.f, rn = 0.f;
-    if (valid) {
+  // packed row of this thread for the next tile, loaded one tile ahead
+  uint32_t ncw[B * 4];
+  uint4 nsg = make_uint4(0u, 0u, 0u, 0u);
+  float nnrm = 0.f, nrn = 0.f;
+  auto load_packed = [&](int64_t tile) {
+    const int64_t row = tile * kTile + trow;
+    if (tile < n_tiles && row < n_rows) {
       const uint4* cp = reinterpret_cast<const uint4*>(in.codes + row * (B * 16));
 #pragma unroll
       for (int q = 0; q < B; ++q) {
         const uint4 u = __ldg(cp + q);
-        cw[4 * q] = u.x; cw[4 * q + 1] = u.y; cw[4 * q + 2] = u.z; cw[4 * q + 3] = u.w;
+        ncw[4 * q] = u.x; ncw[4 * q + 1] = u.y; ncw[4 * q + 2] = u.z; ncw[4 * q + 3] = u.w;
       }
-      if (PROD) sg = __ldg(reinterpret_cast<const uint4*>(in.signs + row * 16));
-      nrm = __ldg(in.norm + row);
-      rn = __ldg(in.rnorm + row);
+      if (PROD) nsg = __ldg(reinterpret_cast<const uint4*>(in.signs + row * 16));
+      nnrm = __ldg(in.norm + row);
+      nrn = __ldg(in.rnorm + row);
     } else {
 #pragma unroll
-      for (int w = 0; w < B * 4; ++w) cw[w] = 0u;
+      for (int w = 0; w < B * 4; ++w) ncw[w] = 0u;
+      nsg = make_uint4(0u, 0u, 0u, 0u);
+      nnrm = 0.f;
+      nrn = 0.f;
     }
+  };
+  load_packed(t_first);
+  for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
+    // ---- this tile's packed row (loaded during the previous tile) ---------------
+    uint32_t cw[B * 4];
+#pragma unroll
+    for (int w = 0; w < B * 4; ++w) cw[w] = ncw[w];
+    const uint4 sg = nsg;
+    const float nrm = nnrm, rn = nrn;
+    load_packed(t + t_step);
     if (PROD) {
       // sign bits -> binary16 {0, 2^-14}: column k of sign word w holds bits
       // (k, k + 16) of the word, i.e. projections 32 w + k and 32 w + k + 16

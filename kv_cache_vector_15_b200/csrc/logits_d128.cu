@@ -270,9 +270,17 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
     }
     tc_fence_after();
     // ---- epilogue: recombine limbs, constants, norms ----------------------------------
-    uint32_t acc[32];
-    tmem_ld32(t_d, acc);
-    tmem_wait_ld();
+    uint32_t acc[N];
+    {
+      uint32_t part[32];
+#pragma unroll
+      for (int c = 0; c < N / 32; ++c) {
+        tmem_ld32(t_d + 32 * c, part);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) acc[32 * c + k] = part[k];
+      }
+    }
     tc_fence_before();
     if (valid) {
 #pragma unroll
