@@ -63,10 +63,10 @@ using namespace sm100;
 constexpr int kD = 128;              // row length
 constexpr int kM = 128;              // projections
 constexpr int kTile = 128;           // rows per tile = MMA M
-constexpr int kWG = 2;               // compute warpgroups
-constexpr int kThreads = kWG * 128;
+constexpr int kPairs = 2;            // warpgroup pairs per CTA, one 128-row tile each in flight
+constexpr int kThreads = kPairs * 256;
 constexpr long long kWaitCycles = 2000000000ll;   // ~1 s at 2 GHz
-constexpr uint32_t kTmemCols = 512;  // per warpgroup: 128 accumulator + 128 A columns, x2
+constexpr uint32_t kTmemCols = 512;  // per pair: 128 accumulator + 128 A columns, x2
 
 struct QuantD128Args {
   uint32_t Dsign[kD];                // Rademacher signs as fp32 sign-bit masks (0 or 0x80000000)
@@ -91,8 +91,8 @@ constexpr int kSmemS = 32768;        // S as the MMA B operand (128 x 128 fp16, 
 
 template <bool BF16IN>
 constexpr size_t quant_smem_bytes() {
-  return 1024 /*alignment slack*/ + kSmemS + XStage<BF16IN>::kStages * kWG * XStage<BF16IN>::kBytes +
-         256 /*barriers etc*/;
+  return 1024 /*alignment slack*/ + kSmemS + XStage<BF16IN>::kStages * kPairs * XStage<BF16IN>::kBytes +
+         2 * kPairs * 2 * kTile * 4 /*partial sums*/ + 256 /*barriers etc*/;
 }
 
 __device__ __forceinline__ void flag_error(int* err, int* abort_flag, int code) {
@@ -106,16 +106,10 @@ __device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi) 
   hi = __uint_as_float(w & 0xffff0000u);
 }
 
-// State a warpgroup thread carries from a tile's first half (rotation, codes,
-// residual into TMEM) to its second half (signs from the MMA, stores).
-template <int B>
-struct RowState {
-  uint32_t cw[B * 4];                // packed codes
-  float n, rho;
-  int64_t row;
-  bool zero, valid;
-};
-
+// Two warpgroups ("halves") share every 128-row tile: thread t of warp w in
+// half h owns coordinates [64 h, 64 h + 64) of row 32 (w % 4) + t, which is
+// also the row's TMEM lane, so both halves of a row meet in the same lane.
+// Two such pairs run per CTA (512 threads, 16 warps per SM).
 template <int B, bool BF16IN>
 __global__ void __launch_bounds__(kThreads, 1)
 k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, const QuantD128Args X,
@@ -123,13 +117,15 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
   constexpr int L = 1 << B;
   constexpr int kStage = XStage<BF16IN>::kBytes;
   constexpr int NS = XStage<BF16IN>::kStages;
+  constexpr int kH = kD / 2;                                     // coordinates per thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sS = smem;
-  uint8_t* sX = smem + kSmemS;                                   // [warpgroup][NS buffers] stages
-  uint64_t* full = reinterpret_cast<uint64_t*>(sX + NS * kWG * kStage);  // [warpgroup][2]
-  uint64_t* mdone = full + 2 * kWG;                              // [warpgroup]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kWG);
+  uint8_t* sX = smem + kSmemS;                                   // [pair][NS] stages
+  float* sPart = reinterpret_cast<float*>(sX + NS * kPairs * kStage);   // [2 sums][pair][half][row] partials
+  uint64_t* full = reinterpret_cast<uint64_t*>(sPart + 2 * kPairs * 2 * kTile);   // [pair][2]
+  uint64_t* mdone = full + 2 * kPairs;                           // [pair]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kPairs);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   float* lut = reinterpret_cast<float*>(tmem_slot + 2);          // L centroids (scaled by 64)
 
@@ -137,8 +133,8 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
 
   if (tid == 0) {
-    for (int i = 0; i < 2 * kWG; ++i) mbar_init(&full[i], 1);
-    for (int i = 0; i < kWG; ++i) mbar_init(&mdone[i], 1);
+    for (int i = 0; i < 2 * kPairs; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < kPairs; ++i) mbar_init(&mdone[i], 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -160,48 +156,219 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int wg = warp >> 2, wl = warp & 3;
-  const bool leader = (wl == 0 && lane == 0);                    // issues this warpgroup's TMA and MMAs
-  const int trow = wl * 32 + lane;                               // row in tile == TMEM lane
-  const uint32_t lane_base = static_cast<uint32_t>(wl * 32) << 16;
-  const uint32_t t_acc = tmem + lane_base + wg * 256;            // projections, 128 columns
+  const int wgi = warp >> 2, pair = wgi >> 1, half = wgi & 1, lb = warp & 3;
+  const bool leader = (half == 0 && lb == 0 && lane == 0);       // issues this pair's TMA and MMAs
+  const int trow = lb * 32 + lane;                               // row in tile == TMEM lane
+  const uint32_t lane_base = static_cast<uint32_t>(lb * 32) << 16;
+  const uint32_t t_acc = tmem + lane_base + pair * 256;          // projections, 128 columns
   const uint32_t t_a = t_acc + 128;                              // residual hi | lo, 128 columns
+  const uint32_t bar_id = 1 + pair;                              // named barrier of the pair (256 threads)
   const float sqrt_d = 11.313708498984761f;                      // sqrt(128)
-  uint8_t* stages = sX + wg * NS * kStage;
-  uint64_t* wfull = full + 2 * wg;
-  const int64_t t_first = blockIdx.x + static_cast<int64_t>(wg) * gridDim.x;
-  const int64_t t_step = static_cast<int64_t>(kWG) * gridDim.x;
+  uint8_t* stages = sX + pair * NS * kStage;
+  uint64_t* pfull = full + 2 * pair;
+  float* myN2 = sPart + (pair * 2 + half) * kTile;               // partial ||x||^2
+  const float* otN2 = sPart + (pair * 2 + (half ^ 1)) * kTile;
+  float* myR2 = sPart + kPairs * 2 * kTile + (pair * 2 + half) * kTile;   // partial ||r||^2
+  const float* otR2 = sPart + kPairs * 2 * kTile + (pair * 2 + (half ^ 1)) * kTile;
+  const int64_t t_first = blockIdx.x + static_cast<int64_t>(pair) * gridDim.x;
+  const int64_t t_step = static_cast<int64_t>(kPairs) * gridDim.x;
   auto issue_load = [&](int64_t tile, int buf) {
-    mbar_arrive_expect_tx(&wfull[buf], kStage);
+    mbar_arrive_expect_tx(&pfull[buf], kStage);
 #pragma unroll
     for (int bx = 0; bx < XStage<BF16IN>::kBoxes; ++bx)
-      tma_load_2d(stages + buf * kStage + bx * (kTile * 128), &tmap, &wfull[buf],
+      tma_load_2d(stages + buf * kStage + bx * (kTile * 128), &tmap, &pfull[buf],
                   bx * XStage<BF16IN>::kColsPerBox, static_cast<int>(tile * kTile));
   };
-  // loads in flight (leader only): fill count per buffer issued vs waited
-  int issued[2] = {0, 0}, waited[2] = {0, 0};
+  int issued[2] = {0, 0}, waited[2] = {0, 0};                    // leader's TMA bookkeeping
   if (leader) {
     prefetch_tmap(&tmap);
     if (t_first < n_tiles) { issue_load(t_first, 0); ++issued[0]; }
     if (NS == 2 && t_first + t_step < n_tiles) { issue_load(t_first + t_step, 1); ++issued[1]; }
   }
 
-  RowState<B> prev;
-  bool have_prev = false;
   int mine = 0;
-  bool aborted = false;
+  for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
+    const int buf = mine % NS;
+    if (mbar_wait(&pfull[buf], (mine / NS) & 1, kWaitCycles)) {
+      if (leader) ++waited[buf];
+    } else {
+      flag_error(X.err, abort_flag, 2);
+    }
+    const uint8_t* stage = stages + buf * kStage;
 
-  // second half of a tile: signs from the accumulator (exact recomputation of
-  // the projections within the error bound of zero), then the stores
-  auto finish = [&](const RowState<B>& st, int tile_no) {
-    if (!mbar_wait(&mdone[wg], tile_no & 1, kWaitCycles)) flag_error(X.err, abort_flag, 3);
-    tc_fence_after();
-    const float eps = kResScale * fmaf(X.eps_scale, st.rho, X.eps_abs);   // in the MMA's (scaled) units
-    uint32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0, f0 = 0, f1 = 0, f2 = 0, f3 = 0;
+    // ---- my half row, D folded into the widening -------------------------------
+    float v[kH];
+    if (BF16IN) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {                  // 16 projections at a time
+      for (int cc = 0; cc < 8; ++cc) {                           // box `half` holds my 64 columns
+        const uint4 w = *reinterpret_cast<const uint4*>(stage + half * (kTile * 128) + trow * 128 +
+                                                        ((cc ^ (trow & 7)) << 4));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = cc * 8 + 2 * u;
+          v[e] = __uint_as_float((ws[u] << 16) ^ X.Dsign[half * kH + e]);
+          v[e + 1] = __uint_as_float((ws[u] & 0xffff0000u) ^ X.Dsign[half * kH + e + 1]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {                             // boxes 2 half, 2 half + 1
+        const int bx = 2 * half + (c >> 3), cc = c & 7;
+        const uint4 w = *reinterpret_cast<const uint4*>(stage + bx * (kTile * 128) + trow * 128 +
+                                                        ((cc ^ (trow & 7)) << 4));
+        v[c * 4 + 0] = __uint_as_float(w.x ^ X.Dsign[half * kH + c * 4 + 0]);
+        v[c * 4 + 1] = __uint_as_float(w.y ^ X.Dsign[half * kH + c * 4 + 1]);
+        v[c * 4 + 2] = __uint_as_float(w.z ^ X.Dsign[half * kH + c * 4 + 2]);
+        v[c * 4 + 3] = __uint_as_float(w.w ^ X.Dsign[half * kH + c * 4 + 3]);
+      }
+    }
+    // partial norm (sign flips do not change it)
+    {
+      float2 a2 = make_float2(0.f, 0.f), b2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int e = 0; e < kH; e += 4) {
+        const float2 a = make_float2(v[e], v[e + 1]), b = make_float2(v[e + 2], v[e + 3]);
+        a2 = __ffma2_rn(a, a, a2);
+        b2 = __ffma2_rn(b, b, b2);
+      }
+      myN2[trow] = (a2.x + a2.y) + (b2.x + b2.y);
+    }
+    // Walsh-Hadamard within my 64 coordinates (strides 2..32 packed, then 1)
+#pragma unroll
+    for (int h = 2; h < kH; h <<= 1) {
+#pragma unroll
+      for (int e = 0; e < kH; e += 2) {
+        if ((e & h) == 0) {
+          const float2 a = make_float2(v[e], v[e + 1]), b = make_float2(v[e + h], v[e + h + 1]);
+          const float2 sum = __fadd2_rn(a, b);
+          const float2 dif = __ffma2_rn(b, make_float2(-1.f, -1.f), a);
+          v[e] = sum.x; v[e + 1] = sum.y; v[e + h] = dif.x; v[e + h + 1] = dif.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < kH; e += 2) {
+      const float a = v[e], b = v[e + 1];
+      v[e] = a + b;
+      v[e + 1] = a - b;
+    }
+    // stride-64 stage across the halves, through this row's TMEM lane: my
+    // values go to columns [64 half, 64 half + 64) of the (idle) accumulator
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t w[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) w[k] = __float_as_uint(v[c * 16 + k]);
+      tmem_st16(t_acc + half * 64 + c * 16, w);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    named_bar_sync(bar_id, 256);                                  // #1: both halves in TMEM; stage read
+    tc_fence_after();
+    if (leader && t + NS * t_step < n_tiles) { issue_load(t + NS * t_step, buf); ++issued[buf]; }
+    const float n = sqrtf(myN2[trow] + otN2[trow]);
+    const bool zero_row = !(n >= kZeroNorm);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t w[16];
+      tmem_ld16(t_acc + (half ^ 1) * 64 + c * 16, w);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float o = __uint_as_float(w[k]);
+        v[c * 16 + k] = half == 0 ? v[c * 16 + k] + o : o - v[c * 16 + k];
+      }
+    }
+
+    // ---- Lloyd-Max codes and the residual (x 64) ----------------------------------
+    // v holds y' = n sqrt(d) y; compare against per-row scaled thresholds; the
+    // residual in unit-normalised units times 64 is r64 = y' sc64 - 64 c[code].
+    const float nsd = zero_row ? 1.f : n * sqrt_d;
+    const float sc64 = zero_row ? 0.f : kResScale / nsd;
+    float tq[L - 1];
+#pragma unroll
+    for (int k = 0; k < L - 1; ++k) tq[k] = P.t[k] * nsd;
+    uint32_t cw[B * 2];                                          // codes of my 64 coordinates
+#pragma unroll
+    for (int w = 0; w < B * 2; ++w) cw[w] = 0u;
+    float2 r2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {                             // 32 coordinates, then their hi | lo words
+#pragma unroll
+      for (int e = ch * 32; e < ch * 32 + 32; ++e) {
+        const float y = v[e];
+        uint32_t code;
+        float cval;
+        {
+          code = 0u;
+#pragma unroll
+          for (int lev = B - 1; lev >= 0; --lev) {
+            const int base = (1 << lev) - 1;
+            float thr = tq[base];
+#pragma unroll
+            for (int k = 1; k < (1 << (B - 1 - lev)); ++k)
+              if (code == static_cast<uint32_t>(k << (lev + 1))) thr = tq[base + (k << (lev + 1))];
+            if (y > thr) code |= (1u << lev);
+          }
+          cval = lut[code];
+        }
+        const float r = zero_row ? 0.f : fmaf(y, sc64, -cval);
+        v[e] = r;
+        if (e & 1) r2.y = fmaf(r, r, r2.y); else r2.x = fmaf(r, r, r2.x);
+        const int bit = B * e, wi = bit >> 5, sh = bit & 31;   // my 64 codes start word aligned
+        cw[wi] |= code << sh;
+        if (sh + B > 32) cw[wi + 1] |= code >> (32 - sh);
+      }
+      uint32_t hw[16], lw[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int e = ch * 32 + 2 * k;
+        const __half2 h = __floats2half2_rn(v[e], v[e + 1]);
+        const float2 hf = __half22float2(h);
+        const __half2 l = __floats2half2_rn(v[e] - hf.x, v[e + 1] - hf.y);
+        hw[k] = *reinterpret_cast<const uint32_t*>(&h);
+        lw[k] = *reinterpret_cast<const uint32_t*>(&l);
+      }
+      tmem_st16(t_a + half * 32 + ch * 16, hw);
+      tmem_st16(t_a + 64 + half * 32 + ch * 16, lw);
+    }
+    if (zero_row) {
+#pragma unroll
+      for (int w = 0; w < B * 2; ++w) cw[w] = 0u;
+    }
+    myR2[trow] = r2.x + r2.y;
+    tmem_wait_st();
+    tc_fence_before();
+    // #2: A complete, exchange reads done; ORs everyone's view of the abort
+    // flag so every thread of the pair takes the same decision
+    if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
+    const float rho = zero_row ? 0.f : sqrtf(myR2[trow] + otR2[trow]) * (1.0f / kResScale);
+
+    // ---- projection on the tensor cores: P = [hi | lo] [S ; S]^T ---------------------
+    if (leader) {
+      tc_fence_after();
+      const uint32_t sbase = smem_u32(sS);
+      const uint32_t idesc = idesc_f16_f32(kTile, kM);
+      const uint32_t d_tmem = tmem + pair * 256;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int kk = k & 7;                                      // K step within S (16 columns each)
+        const uint64_t bdesc = smem_desc_sw128(sbase + (kk >> 2) * 16384 + (kk & 3) * 32, 1024);
+        mma_f16_ts(d_tmem, d_tmem + 128 + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
+      }
+      mma_commit(&mdone[pair]);
+    }
+    if (!mbar_wait(&mdone[pair], mine & 1, kWaitCycles)) flag_error(X.err, abort_flag, 3);
+    tc_fence_after();
+
+    // ---- my 64 signs, exact recomputation within the error bound of zero ------------
+    const float eps = kResScale * fmaf(X.eps_scale, rho, X.eps_abs);   // in the MMA's (scaled) units
+    uint32_t s0 = 0, s1 = 0, f0 = 0, f1 = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
       uint32_t p[16];
-      tmem_ld16(t_acc + c * 16, p);
+      tmem_ld16(t_acc + half * 64 + c * 16, p);
       tmem_wait_ld();
       uint32_t bits = 0u, flags = 0u;
 #pragma unroll
@@ -211,35 +378,29 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
       }
       const int sh = (c & 1) * 16;
       if ((c >> 1) == 0) { s0 |= bits << sh; f0 |= flags << sh; }
-      if ((c >> 1) == 1) { s1 |= bits << sh; f1 |= flags << sh; }
-      if ((c >> 1) == 2) { s2 |= bits << sh; f2 |= flags << sh; }
-      if ((c >> 1) == 3) { s3 |= bits << sh; f3 |= flags << sh; }
+      else { s1 |= bits << sh; f1 |= flags << sh; }
     }
-    // Recompute flagged projections in fp32 from hi + lo, one flagged j per
-    // lane per pass; the TMEM reads are warp-collective, so every lane runs
-    // max-over-lanes passes.
-    const int nflag = __popc(f0) + __popc(f1) + __popc(f2) + __popc(f3);
+    const int nflag = __popc(f0) + __popc(f1);
     const int passes = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(nflag));
     for (int q = 0; q < passes; ++q) {
-      int j = -1;
-      if (q < nflag) {                           // the lowest remaining flagged projection
-        if (f3) j = 96 + __ffs(f3) - 1;
-        if (f2) j = 64 + __ffs(f2) - 1;
+      int j = -1;                                                  // local index in [0, 64)
+      if (q < nflag) {
         if (f1) j = 32 + __ffs(f1) - 1;
         if (f0) j = __ffs(f0) - 1;
       }
+      const int jg = half * 64 + (j < 0 ? 0 : j);                  // projection index
       float acc = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {              // 16 residual pairs (32 entries) at a time
-        uint32_t ah[16], al[16];
-        tmem_ld16(t_a + c * 16, ah);
-        tmem_ld16(t_a + 64 + c * 16, al);
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {                                // 8 residual pairs (16 entries) at a time
+        uint32_t ah[8], al[8];
+        tmem_ld8(t_a + c * 8, ah);
+        tmem_ld8(t_a + 64 + c * 8, al);
         tmem_wait_ld();
         if (j >= 0) {
 #pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {                      // 16-byte chunks of S row j: 8 entries
-            const int chunk = c * 4 + qq, kb = chunk >> 3, cc = chunk & 7;
-            const uint4 sv = *reinterpret_cast<const uint4*>(sS + kb * 16384 + j * 128 + ((cc ^ (j & 7)) << 4));
+          for (int qq = 0; qq < 2; ++qq) {                         // 16-byte chunks of S row jg: 8 entries
+            const int chunk = c * 2 + qq, kb = chunk >> 3, cc = chunk & 7;
+            const uint4 sv = *reinterpret_cast<const uint4*>(sS + kb * 16384 + jg * 128 + ((cc ^ (jg & 7)) << 4));
             const uint32_t sws[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -255,203 +416,41 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
       }
       if (j >= 0) {
         const uint32_t m = 1u << (j & 31), nb = acc < 0.f ? m : 0u;
-        const int c = j >> 5;
-        if (c == 0) { s0 = (s0 & ~m) | nb; f0 &= ~m; }
-        if (c == 1) { s1 = (s1 & ~m) | nb; f1 &= ~m; }
-        if (c == 2) { s2 = (s2 & ~m) | nb; f2 &= ~m; }
-        if (c == 3) { s3 = (s3 & ~m) | nb; f3 &= ~m; }
+        if (j < 32) { s0 = (s0 & ~m) | nb; f0 &= ~m; }
+        else { s1 = (s1 & ~m) | nb; f1 &= ~m; }
       }
     }
-    if (st.zero || st.rho == 0.f) s0 = s1 = s2 = s3 = 0u;
+    if (zero_row || rho == 0.f) s0 = s1 = 0u;
     tc_fence_before();
-    if (st.valid) {
-      uint4* co = reinterpret_cast<uint4*>(out.codes + st.row * (B * 16));
-#pragma unroll
-      for (int q = 0; q < B; ++q)
-        co[q] = make_uint4(st.cw[4 * q], st.cw[4 * q + 1], st.cw[4 * q + 2], st.cw[4 * q + 3]);
-      *reinterpret_cast<uint4*>(out.signs + st.row * 16) = make_uint4(s0, s1, s2, s3);
-      out.norm[st.row] = st.zero ? 0.f : st.n;
-      out.rnorm[st.row] = st.zero ? 0.f : st.n * st.rho;
-    }
-  };
 
-  for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
-    const int buf = mine % NS;
-    if (mbar_wait(&wfull[buf], (mine / NS) & 1, kWaitCycles)) {
-      if (leader) ++waited[buf];
-    } else {
-      flag_error(X.err, abort_flag, 2);
-    }
-    const uint8_t* stage = stages + buf * kStage;
-    RowState<B> cur;
-    cur.row = t * kTile + trow;
-    cur.valid = cur.row < n_rows;
-
-    // ---- this thread's row, D folded into the bf16 -> fp32 widening ----------
-    float v[kD];
-    if (BF16IN) {
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int bx = c >> 3, cc = c & 7;
-        const uint4 w = *reinterpret_cast<const uint4*>(stage + bx * (kTile * 128) + trow * 128 +
-                                                        ((cc ^ (trow & 7)) << 4));
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int e = c * 8 + 2 * u;
-          v[e] = __uint_as_float((ws[u] << 16) ^ X.Dsign[e]);
-          v[e + 1] = __uint_as_float((ws[u] & 0xffff0000u) ^ X.Dsign[e + 1]);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int bx = c >> 3, cc = c & 7;
-        const uint4 w = *reinterpret_cast<const uint4*>(stage + bx * (kTile * 128) + trow * 128 +
-                                                        ((cc ^ (trow & 7)) << 4));
-        v[c * 4 + 0] = __uint_as_float(w.x ^ X.Dsign[c * 4 + 0]);
-        v[c * 4 + 1] = __uint_as_float(w.y ^ X.Dsign[c * 4 + 1]);
-        v[c * 4 + 2] = __uint_as_float(w.z ^ X.Dsign[c * 4 + 2]);
-        v[c * 4 + 3] = __uint_as_float(w.w ^ X.Dsign[c * 4 + 3]);
-      }
-    }
-
-    // ---- norm (sign flips do not change it), Walsh-Hadamard (unnormalised) ----
-    float2 ssa = make_float2(0.f, 0.f), ssb = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int e = 0; e < kD; e += 4) {
-      const float2 a = make_float2(v[e], v[e + 1]), b = make_float2(v[e + 2], v[e + 3]);
-      ssa = __ffma2_rn(a, a, ssa);
-      ssb = __ffma2_rn(b, b, ssb);
-    }
-    cur.n = sqrtf((ssa.x + ssa.y) + (ssb.x + ssb.y));
-    cur.zero = !(cur.n >= kZeroNorm);
-#pragma unroll
-    for (int h = 2; h < kD; h <<= 1) {
-#pragma unroll
-      for (int e = 0; e < kD; e += 2) {
-        if ((e & h) == 0) {
-          const float2 a = make_float2(v[e], v[e + 1]), b = make_float2(v[e + h], v[e + h + 1]);
-          const float2 sum = __fadd2_rn(a, b);
-          const float2 dif = __ffma2_rn(b, make_float2(-1.f, -1.f), a);
-          v[e] = sum.x; v[e + 1] = sum.y; v[e + h] = dif.x; v[e + h + 1] = dif.y;
-        }
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < kD; e += 2) {
-      const float a = v[e], b = v[e + 1];
-      v[e] = a + b;
-      v[e + 1] = a - b;
-    }
-
-    // ---- Lloyd-Max codes and the residual (x 64) ----------------------------------
-    // v holds y' = n sqrt(d) y; compare against per-row scaled thresholds; the
-    // residual in unit-normalised units times 64 is r64 = y' sc64 - 64 c[code].
-    const float nsd = cur.zero ? 1.f : cur.n * sqrt_d;
-    const float sc64 = cur.zero ? 0.f : kResScale / nsd;
-    float tq[L - 1];
-#pragma unroll
-    for (int k = 0; k < L - 1; ++k) tq[k] = P.t[k] * nsd;
-#pragma unroll
-    for (int w = 0; w < B * 4; ++w) cur.cw[w] = 0u;
-    float2 r2 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int e = 0; e < kD; ++e) {
-      const float y = v[e];
-      uint32_t code;
-      float cval;
+    // ---- stores: my half of the codes and signs; norms from half 0 ------------------
+    const int64_t row = t * kTile + trow;
+    if (row < n_rows) {
+      uint32_t* co = reinterpret_cast<uint32_t*>(out.codes + row * (B * 16) + half * (B * 8));
       if constexpr (B == 1) {
-        const bool up = y > 0.f;
-        code = up ? 1u : 0u;
-        cval = up ? lut[1] : -lut[1];
+        *reinterpret_cast<uint2*>(co) = make_uint2(cw[0], cw[1]);
       } else if constexpr (B == 2) {
-        // symmetric 4-level codebook: t = (-tau, 0, tau), c = (-c3, -c2, c2, c3).
-        // Outer cell by |y| > tau (y exactly equal to -tau, a boundary tie, would
-        // take the inner cell; such a coordinate lies in the tie band).
-        const bool up = y > 0.f, outer = fabsf(y) > tq[2];
-        code = (up ? 2u : 0u) | ((up == outer) ? 1u : 0u);
-        const float mag = outer ? lut[3] : lut[2];
-        cval = up ? mag : -mag;
+        *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      } else if constexpr (B == 3) {
+        *reinterpret_cast<uint2*>(co) = make_uint2(cw[0], cw[1]);
+        *reinterpret_cast<uint4*>(co + 2) = make_uint4(cw[2], cw[3], cw[4], cw[5]);
       } else {
-        code = 0u;
-#pragma unroll
-        for (int lev = B - 1; lev >= 0; --lev) {
-          const int base = (1 << lev) - 1;
-          float thr = tq[base];
-#pragma unroll
-          for (int k = 1; k < (1 << (B - 1 - lev)); ++k)
-            if (code == static_cast<uint32_t>(k << (lev + 1))) thr = tq[base + (k << (lev + 1))];
-          if (y > thr) code |= (1u << lev);
-        }
-        cval = lut[code];
+        *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint4*>(co + 4) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
       }
-      const float r = fmaf(y, sc64, -cval);
-      v[e] = r;
-      if (e & 1) r2.y = fmaf(r, r, r2.y); else r2.x = fmaf(r, r, r2.x);
-      const int bit = B * e, wi = bit >> 5, sh = bit & 31;
-      cur.cw[wi] |= code << sh;
-      if (sh + B > 32) cur.cw[wi + 1] |= code >> (32 - sh);
-    }
-    cur.rho = sqrtf(r2.x + r2.y) * (1.0f / kResScale);
-    if (cur.zero) {
-      cur.rho = 0.f;
-#pragma unroll
-      for (int w = 0; w < B * 4; ++w) cur.cw[w] = 0u;
-#pragma unroll
-      for (int e = 0; e < kD; ++e) v[e] = 0.f;
-    }
-
-    // ---- previous tile's signs and stores, now that its MMA has had time ---------
-    if (have_prev) finish(prev, mine - 1);
-
-    // ---- residual -> TMEM as binary16 hi | lo (A operand) --------------------------
-#pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
-      uint32_t hw[16], lw[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int e = ch * 32 + 2 * k;
-        const __half2 h = __floats2half2_rn(v[e], v[e + 1]);
-        const float2 hf = __half22float2(h);
-        const __half2 l = __floats2half2_rn(v[e] - hf.x, v[e + 1] - hf.y);
-        hw[k] = *reinterpret_cast<const uint32_t*>(&h);
-        lw[k] = *reinterpret_cast<const uint32_t*>(&l);
+      *reinterpret_cast<uint2*>(out.signs + row * 16 + half * 8) = make_uint2(s0, s1);
+      if (half == 0) {
+        out.norm[row] = zero_row ? 0.f : n;
+        out.rnorm[row] = zero_row ? 0.f : n * rho;
       }
-      tmem_st16(t_a + ch * 16, hw);
-      tmem_st16(t_a + 64 + ch * 16, lw);
     }
-    tmem_wait_st();
-    tc_fence_before();
-    // barrier over the warpgroup that also ORs everyone's view of the abort
-    // flag, so the decision to stop is the same in every thread
-    if (named_bar_sync_or(1 + wg, 128, *reinterpret_cast<volatile int*>(abort_flag) != 0)) { aborted = true; break; }
-
-    // ---- projection on the tensor cores: P = [hi | lo] [S ; S]^T; refill the stage --
-    if (leader) {
-      tc_fence_after();
-      const uint32_t sbase = smem_u32(sS);
-      const uint32_t idesc = idesc_f16_f32(kTile, kM);
-      const uint32_t d_tmem = tmem + wg * 256;
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int kk = k & 7;                                      // K step within S (16 columns each)
-        const uint64_t bdesc = smem_desc_sw128(sbase + (kk >> 2) * 16384 + (kk & 3) * 32, 1024);
-        mma_f16_ts(d_tmem, d_tmem + 128 + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
-      }
-      mma_commit(&mdone[wg]);
-      if (t + NS * t_step < n_tiles) { issue_load(t + NS * t_step, buf); ++issued[buf]; }
-    }
-    prev = cur;
-    have_prev = true;
   }
-  if (have_prev && !aborted) finish(prev, mine - 1);
 
   // ---- teardown: no TMA load of ours may still be in flight ----------------------
   if (leader) {
     for (int b2 = 0; b2 < 2; ++b2)
       while (waited[b2] < issued[b2]) {
-        if (!mbar_wait(&wfull[b2], waited[b2] & 1, kWaitCycles)) { flag_error(X.err, abort_flag, 4); break; }
+        if (!mbar_wait(&pfull[b2], waited[b2] & 1, kWaitCycles)) { flag_error(X.err, abort_flag, 4); break; }
         ++waited[b2];
       }
   }
