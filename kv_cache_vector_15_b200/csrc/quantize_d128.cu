@@ -432,8 +432,15 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
       } else if constexpr (B == 2) {
         *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
       } else if constexpr (B == 3) {
-        *reinterpret_cast<uint2*>(co) = make_uint2(cw[0], cw[1]);
-        *reinterpret_cast<uint4*>(co + 2) = make_uint4(cw[2], cw[3], cw[4], cw[5]);
+        // 24 bytes per half: half 0 at row offset 0 (16 + 8), half 1 at 24 (8 + 16),
+        // so that each 16-byte store stays 16-byte aligned
+        if (half == 0) {
+          *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          *reinterpret_cast<uint2*>(co + 4) = make_uint2(cw[4], cw[5]);
+        } else {
+          *reinterpret_cast<uint2*>(co) = make_uint2(cw[0], cw[1]);
+          *reinterpret_cast<uint4*>(co + 2) = make_uint4(cw[2], cw[3], cw[4], cw[5]);
+        }
       } else {
         *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
         *reinterpret_cast<uint4*>(co + 4) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
