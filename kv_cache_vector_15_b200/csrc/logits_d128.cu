@@ -115,9 +115,44 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
   const int64_t t0 = n_tiles * wid / n_wg, t1 = n_tiles * (wid + 1) / n_wg;
   int64_t cur_set = -1;
   int mine = 0;
+  // packed key of this thread for the next tile, loaded one tile ahead
+  uint32_t ncw[S::kCodeWords], nsw[4];
+  float nnrm = 0.f, nrn = 0.f;
+  auto load_key = [&](int64_t tile) {
+    const int64_t set = tile / tiles_per_set;
+    const int64_t key = (tile % tiles_per_set) * kTile + trow;
+    if (tile < t1 && key < n_keys) {
+      const int64_t row = set * n_keys + key;
+      const uint4* cp = reinterpret_cast<const uint4*>(keys.codes + row * (B * 16));
+#pragma unroll
+      for (int q = 0; q < B; ++q) {
+        const uint4 u = __ldg(cp + q);
+        ncw[4 * q] = u.x; ncw[4 * q + 1] = u.y; ncw[4 * q + 2] = u.z; ncw[4 * q + 3] = u.w;
+      }
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(keys.signs + row * 16));
+      nsw[0] = u.x; nsw[1] = u.y; nsw[2] = u.z; nsw[3] = u.w;
+      nnrm = __ldg(keys.norm + row);
+      nrn = __ldg(keys.rnorm + row);
+    } else {
+#pragma unroll
+      for (int w = 0; w < S::kCodeWords; ++w) ncw[w] = 0u;
+      nsw[0] = nsw[1] = nsw[2] = nsw[3] = 0u;
+      nnrm = 0.f;
+      nrn = 0.f;
+    }
+  };
+  load_key(t0);
   for (int64_t t = t0; t < t1; ++t, ++mine) {
     const int64_t set = t / tiles_per_set;
     const int64_t key = (t % tiles_per_set) * kTile + trow;
+    const bool valid = key < n_keys;
+    uint32_t cw[S::kCodeWords], sw[4];
+#pragma unroll
+    for (int w = 0; w < S::kCodeWords; ++w) cw[w] = ncw[w];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) sw[w] = nsw[w];
+    const float nrm = nnrm, rn = nrn * P.qjl_scale;
+    load_key(t + 1);
     if (set != cur_set) {
       // ---- build the query operand of this set --------------------------------
       cur_set = set;
@@ -212,26 +247,6 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
       named_bar_sync(1 + wg, 128);
     }
     // ---- decode this thread's key into TMEM ------------------------------------------
-    const bool valid = key < n_keys;
-    const int64_t row = set * n_keys + key;
-    uint32_t cw[S::kCodeWords], sw[4];
-    float nrm = 0.f, rn = 0.f;
-    if (valid) {
-      const uint4* cp = reinterpret_cast<const uint4*>(keys.codes + row * (B * 16));
-#pragma unroll
-      for (int q = 0; q < B; ++q) {
-        const uint4 u = __ldg(cp + q);
-        cw[4 * q] = u.x; cw[4 * q + 1] = u.y; cw[4 * q + 2] = u.z; cw[4 * q + 3] = u.w;
-      }
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(keys.signs + row * 16));
-      sw[0] = u.x; sw[1] = u.y; sw[2] = u.z; sw[3] = u.w;
-      nrm = __ldg(keys.norm + row);
-      rn = __ldg(keys.rnorm + row) * P.qjl_scale;
-    } else {
-#pragma unroll
-      for (int w = 0; w < S::kCodeWords; ++w) cw[w] = 0u;
-      sw[0] = sw[1] = sw[2] = sw[3] = 0u;
-    }
     {
       uint32_t a[32];
       int n = 0, col = 0;
