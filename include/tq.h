@@ -138,6 +138,22 @@ tq_status tq_logits(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t 
                     tq_packed keys, int64_t n_keys, float* out, void* workspace, size_t workspace_bytes,
                     void* stream);
 
+/* tq_logits without a caller-provided workspace, for callers that cannot
+ * allocate device memory where they make the call (a component that does not
+ * own the device memory pool, a plug-in barred from the CUDA allocator, a
+ * latency-critical path that must not risk the synchronization an allocation
+ * can cause).  The pages describe no such call: it is an interface
+ * convenience of this library.  Same arguments and results as tq_logits; the
+ * per-query operands go to a 4 MiB scratch array compiled into the library
+ * (held on every device that loads it until the process exits), so
+ * n_sets * g * (d + m) * 4 must be at most 4 MiB (else TQ_ERR_UNSUPPORTED, no
+ * launch).  Allocates nothing.  The first call on each device looks up the
+ * array's device address (make it before any stream capture).  All calls
+ * share the array: calls that may overlap on the GPU race and must be
+ * serialized by the caller. */
+tq_status tq_logits_noalloc(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
+                            tq_packed keys, int64_t n_keys, float* out, void* stream);
+
 /* Reconstruct n_rows packed rows into out [n_rows, d] (bf16 or fp32,
  * contiguous, 16-byte aligned).  mode PROD adds the QJL term (unbiased),
  * MSE uses the codes alone. */

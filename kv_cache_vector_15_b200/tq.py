@@ -28,7 +28,7 @@ TQ_DEQUANT_PROD, TQ_DEQUANT_MSE = 0, 1
 # exported symbols, in header order
 SYMBOLS = [
     "tq_host_params", "tq_init", "tq_destroy", "tq_packed_sizes", "tq_get_params", "tq_quantize",
-    "tq_logits_workspace_bytes", "tq_logits", "tq_dequant", "tq_topk", "tq_logits_bf16",
+    "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_dequant", "tq_topk", "tq_logits_bf16",
     "tq_status_str", "tq_sync_status", "tq_last_error", "tq_launch_count",
 ]
 
@@ -48,6 +48,7 @@ _sig = {
     "tq_quantize": (_i32, [_vp, _vp, _i32, _i64, _i64, _Packed, _vp]),
     "tq_logits_workspace_bytes": (_sz, [_vp, _i64, _i32]),
     "tq_logits": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _i64, _vp, _vp, _sz, _vp]),
+    "tq_logits_noalloc": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _i64, _vp, _vp]),
     "tq_dequant": (_i32, [_vp, _Packed, _i64, _vp, _i32, _i32, _vp]),
     "tq_topk": (_i32, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "tq_logits_bf16": (_i32, [_vp, _vp, _i64, _i32, _i64, _i32, _vp, _vp]),
@@ -217,6 +218,13 @@ class TurboQuant:
         wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
         _check(_lib.tq_logits(self._h, _ptr(q), _dtype_code(q), n_sets, g, keys.c(), n_keys, _ptr(out),
                               _ptr(workspace), wbytes, _stream(stream)), "tq_logits")
+        return out
+
+    def logits_noalloc(self, q, keys: Packed, n_sets: int, g: int, n_keys: int, out, stream=None):
+        """tq_logits with the library's built-in scratch instead of a workspace;
+        allocates nothing on the device (``out`` must be provided)."""
+        _check(_lib.tq_logits_noalloc(self._h, _ptr(q), _dtype_code(q), n_sets, g, keys.c(), n_keys, _ptr(out),
+                                      _stream(stream)), "tq_logits_noalloc")
         return out
 
     def dequant(self, packed: Packed, n_rows: int | None = None, out_dtype=None, mode: int = TQ_DEQUANT_PROD,
