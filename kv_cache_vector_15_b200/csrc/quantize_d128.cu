@@ -299,7 +299,7 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
       for (int e = ch * 32; e < ch * 32 + 32; ++e) {
         const float y = v[e];
         uint32_t code;
-        float cval;
+        float r;
         {
           code = 0u;
 #pragma unroll
@@ -311,9 +311,9 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
               if (code == static_cast<uint32_t>(k << (lev + 1))) thr = tq[base + (k << (lev + 1))];
             if (y > thr) code |= (1u << lev);
           }
-          cval = lut[code];
+          r = fmaf(y, sc64, -lut[code]);
         }
-        const float r = zero_row ? 0.f : fmaf(y, sc64, -cval);
+        if (zero_row) r = 0.f;
         v[e] = r;
         if (e & 1) r2.y = fmaf(r, r, r2.y); else r2.x = fmaf(r, r, r2.x);
         const int bit = B * e, wi = bit >> 5, sh = bit & 31;   // my 64 codes start word aligned
@@ -365,20 +365,37 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
     // ---- my 64 signs, exact recomputation within the error bound of zero ------------
     const float eps = kResScale * fmaf(X.eps_scale, rho, X.eps_abs);   // in the MMA's (scaled) units
     uint32_t s0 = 0, s1 = 0, f0 = 0, f1 = 0;
+    float pmin = INFINITY;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t p[16];
       tmem_ld16(t_acc + half * 64 + c * 16, p);
       tmem_wait_ld();
-      uint32_t bits = 0u, flags = 0u;
+      uint32_t bits = 0u;
 #pragma unroll
       for (int j = 15; j >= 0; --j) {
         bits = (bits << 1) | (p[j] >> 31);
-        flags = (flags << 1) | (fabsf(__uint_as_float(p[j])) < eps ? 1u : 0u);
+        pmin = fminf(pmin, fabsf(__uint_as_float(p[j])));
       }
-      const int sh = (c & 1) * 16;
-      if ((c >> 1) == 0) { s0 |= bits << sh; f0 |= flags << sh; }
-      else { s1 |= bits << sh; f1 |= flags << sh; }
+      if (c == 0) s0 = bits;
+      if (c == 1) s0 |= bits << 16;
+      if (c == 2) s1 = bits;
+      if (c == 3) s1 |= bits << 16;
+    }
+    if (pmin < eps) {                        // rare: find which projections are within the bound
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t p[16];
+        tmem_ld16(t_acc + half * 64 + c * 16, p);
+        tmem_wait_ld();
+        uint32_t flags = 0u;
+#pragma unroll
+        for (int j = 15; j >= 0; --j) flags = (flags << 1) | (fabsf(__uint_as_float(p[j])) < eps ? 1u : 0u);
+        if (c == 0) f0 = flags;
+        if (c == 1) f0 |= flags << 16;
+        if (c == 2) f1 = flags;
+        if (c == 3) f1 |= flags << 16;
+      }
     }
     const int nflag = __popc(f0) + __popc(f1);
     const int passes = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(nflag));
