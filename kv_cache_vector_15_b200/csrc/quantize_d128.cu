@@ -382,7 +382,9 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
       if (c == 2) s1 = bits;
       if (c == 3) s1 |= bits << 16;
     }
-    if (pmin < eps) {                        // rare: find which projections are within the bound
+    // rare: find which projections are within the bound.  The TMEM loads are
+    // warp-collective, so the whole warp takes this branch when any lane needs it.
+    if (__any_sync(0xffffffffu, pmin < eps)) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t p[16];
