@@ -47,6 +47,26 @@ METRIC = "compressed-key logits/s and % HBM roofline (d=128,b=3); quantize rows/
 UNIT = "logits/s"
 
 
+KERNEL_OF = {"quantize": "k_quantize_d128_tc", "logits": "k_logits_d128_i8", "dequant": "k_dequant_d128_tc"}
+
+
+def captured_traffic(kernel: str, units: int):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture summary
+    (profiles/traffic.json), scaled by the units one launch processes -- or
+    None when there is no capture or the kernel's source changed since."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    entry = json.load(open(p)).get(KERNEL_OF.get(kernel, ""), None)
+    if not entry:
+        return None
+    src = os.path.join(ROOT, entry["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != entry["source_sha256"]:
+        return None
+    return entry["dram_bytes_per_unit"] * units
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -351,8 +371,8 @@ def run_ours(args, cfg, ws, rank, local):
                        "parallelism": f"dp{ws} (independent (batch, kv head) sets per rank)",
                        "l2": "inputs larger than L2 (K, V 2.1 GB each); no flush"},
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dk["gbs"], "peak": hbm,
-                         "unit": "GB/s", "frac": dk["frac_hbm"], "traffic": None,
-                         "peak_kind": hbm_kind},
+                         "unit": "GB/s", "frac": dk["frac_hbm"], "traffic": captured_traffic(dominant, N),
+                         "algorithmic_bytes": dk["bytes"], "peak_kind": hbm_kind},
             "quantize_rows_per_s": ws * N / (q_ms * 1e-3),
             "kernels": {k: {"ms_per_launch": v["ms"], "algorithmic_GBps": v["gbs"], "frac_hbm": v["frac_hbm"],
                             "bytes_per_launch": v["bytes"]} for k, v in kern.items()},
