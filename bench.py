@@ -33,6 +33,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from kv_cache_vector_15_b200 import dist as dist_util  # noqa: E402
 from kv_cache_vector_15_b200 import inputs  # noqa: E402
 
 WORKLOADS = {
@@ -148,19 +149,12 @@ def dist_setup():
 
 
 def barrier(ws):
-    if ws > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    dist_util.barrier(ws)
 
 
 def max_over_ranks(ws, v: float) -> float:
-    if ws == 1:
-        return v
     import torch
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return dist_util.max_over_ranks(ws, v, device=torch.device("cuda", torch.cuda.current_device()))
 
 
 # ---------------------------------------------------------------------------
@@ -226,7 +220,9 @@ def run_ours(args, cfg, ws, rank, local):
     from kv_cache_vector_15_b200 import tq
 
     d, b, m = cfg["d"], cfg["b"], cfg["m"]
-    n_sets = cfg["batch"] * cfg["kv_heads"]
+    # this rank's sequences of a global batch of ws * batch (weak scaling)
+    sh = dist_util.decode_shard(cfg["batch"], ws, rank, cfg["kv_heads"], cfg["q_heads"], cfg["ctx"])
+    n_sets = sh.n_sets
     g = cfg["q_heads"] // cfg["kv_heads"]
     n_keys = cfg["ctx"]
     N = n_sets * n_keys
@@ -234,13 +230,13 @@ def run_ours(args, cfg, ws, rank, local):
     T = tq.TurboQuant(d, b, m, seed=0)
 
     # seeded inputs, drawn on the host into pinned buffers (also the e2e source)
-    K, V, Q = inputs.decode(cfg["batch"], cfg["ctx"], kv_heads=cfg["kv_heads"], q_heads=cfg["q_heads"])
+    K, V, Q = inputs.decode(sh.global_batch, cfg["ctx"], kv_heads=cfg["kv_heads"], q_heads=cfg["q_heads"])
     hK = torch.empty((N, d), dtype=torch.bfloat16, pin_memory=True)
     hV = torch.empty((N, d), dtype=torch.bfloat16, pin_memory=True)
     hQ = torch.empty((n_sets * g, d), dtype=torch.bfloat16, pin_memory=True)
-    K.fill(hK.view(torch.int16).numpy().view(np.uint16))
-    V.fill(hV.view(torch.int16).numpy().view(np.uint16))
-    Q.fill(hQ.view(torch.int16).numpy().view(np.uint16))
+    K.fill(hK.view(torch.int16).numpy().view(np.uint16), start=sh.kv_rows[0])
+    V.fill(hV.view(torch.int16).numpy().view(np.uint16), start=sh.kv_rows[0])
+    Q.fill(hQ.view(torch.int16).numpy().view(np.uint16), start=sh.q_rows[0])
     dK, dV, dQ = hK.to(dev), hV.to(dev), hQ.to(dev)
     pK, pV = T.empty_packed(N, dev), T.empty_packed(N, dev)
     logits = torch.empty((n_sets, g, n_keys), dtype=torch.float32, device=dev)
@@ -293,7 +289,9 @@ def run_ours(args, cfg, ws, rank, local):
         per["dequant"].append(e[3].elapsed_time(e[4]))
     avg = {k: sum(v) / len(v) for k, v in per.items()}
     n_logits = n_sets * g * n_keys
-    value = ws * n_logits / (ms_step * 1e-3)
+    total_logits = dist_util.sum_over_ranks(ws, n_logits, device=dev)
+    total_rows = dist_util.sum_over_ranks(ws, N, device=dev)
+    value = total_logits / (ms_step * 1e-3)
 
     hbm, hbm_kind = peaks()
     P = T.row_bytes
@@ -366,20 +364,22 @@ def run_ours(args, cfg, ws, rank, local):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": args.workload, "batch": cfg["batch"], "kv_heads": cfg["kv_heads"],
+            "config": {"workload": args.workload, "batch": cfg["batch"], "global_batch": sh.global_batch,
+                       "kv_heads": cfg["kv_heads"],
                        "q_heads": cfg["q_heads"], "ctx": cfg["ctx"], "d": d, "b": b, "m": m,
-                       "parallelism": f"dp{ws} (independent (batch, kv head) sets per rank)",
+                       "parallelism": f"dp{ws} (each rank owns {cfg['batch']} sequences of the global batch; "
+                                      "no data-path collective)",
                        "l2": "inputs larger than L2 (K, V 2.1 GB each); no flush"},
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dk["gbs"], "peak": hbm,
                          "unit": "GB/s", "frac": dk["frac_hbm"], "traffic": captured_traffic(dominant, N),
                          "algorithmic_bytes": dk["bytes"], "peak_kind": hbm_kind},
-            "quantize_rows_per_s": ws * N / (q_ms * 1e-3),
+            "quantize_rows_per_s": total_rows / (q_ms * 1e-3),
             "kernels": {k: {"ms_per_launch": v["ms"], "algorithmic_GBps": v["gbs"], "frac_hbm": v["frac_hbm"],
                             "bytes_per_launch": v["bytes"]} for k, v in kern.items()},
             "bf16_key_logits_baseline": {"ms": bf16_ms, "algorithmic_GBps": bf16_bytes / (bf16_ms * 1e-3) / 1e9,
                                          "tq_logits_speedup": bf16_ms / avg["logits"]},
             "cpu_baseline": cpu,
-            "e2e": {"value": ws * n_logits / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": total_logits / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches,
             "clocks": clk.summary(),

@@ -140,20 +140,26 @@ class RowTensor:
     def all(self) -> np.ndarray:
         return self.rows(0, self.n_rows)
 
-    def fill(self, out: np.ndarray, threads: int = 0) -> np.ndarray:
-        """Write all rows into ``out`` (uint16 for bf16, fp32 otherwise, shape
-        [n_rows, d]) block by block on a thread pool; same values as all()."""
+    def fill(self, out: np.ndarray, threads: int = 0, start: int = 0) -> np.ndarray:
+        """Write rows [start, start + len(out)) into ``out`` (uint16 for bf16,
+        fp32 otherwise) block by block on a thread pool; the same values as
+        rows(start, start + len(out)).  With start = 0 and len(out) = n_rows
+        this is all()."""
         import concurrent.futures as cf
         import os
-        nblk = (self.n_rows + BLOCK - 1) // BLOCK
+        stop = start + out.shape[0]
+        if start < 0 or stop > self.n_rows:
+            raise ValueError(f"rows [{start}, {stop}) outside [0, {self.n_rows})")
         threads = threads or min(32, os.cpu_count() or 1)
+        cuts = list(range(start, stop, BLOCK)) if start % BLOCK == 0 else \
+            [start] + list(range((start // BLOCK + 1) * BLOCK, stop, BLOCK))
 
-        def one(k):
-            lo, hi = k * BLOCK, min(self.n_rows, (k + 1) * BLOCK)
-            out[lo:hi] = self.rows(lo, hi)
+        def one(lo):
+            hi = min(stop, (lo // BLOCK + 1) * BLOCK)
+            out[lo - start:hi - start] = self.rows(lo, hi)
 
         with cf.ThreadPoolExecutor(max_workers=threads) as ex:
-            list(ex.map(one, range(nblk)))
+            list(ex.map(one, cuts))
         return out
 
     def as_f32(self, rows: np.ndarray) -> np.ndarray:
