@@ -487,8 +487,343 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
   }
 }
 
+// bf16 rows: the rotation itself on the tensor cores.  y' = H D x is a
+// 128 x 128 x 128 product per tile with the x tile straight from its TMA stage
+// (the 128-byte-swizzled layout the TMA writes is the MMA's K-major operand
+// layout) and B = D H as bf16 +-1 values (exact products, fp32 accumulation),
+// so no widening, no butterflies and no cross-thread exchange run on the CUDA
+// cores.  Each thread reads its row's 128 rotated values from TMEM (the norm
+// is ||y'|| / sqrt(d)), keeps its 64, and the rest follows the fp32 kernel:
+// codes, residual hi | lo into TMEM, the projection MMA, signs, stores.
+template <int B>
+__global__ void __launch_bounds__(kThreads, 1)
+k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, const QuantD128Args X,
+                       int64_t n_rows, const Packed out) {
+  constexpr int L = 1 << B;
+  constexpr int kStage = XStage<true>::kBytes;                  // 32 KB: two 64-column boxes
+  constexpr int NS = 2;
+  constexpr int kH = kD / 2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sS = smem;                                            // projection B operand
+  uint8_t* sHD = smem + kSmemS;                                  // rotation B operand (D H, bf16 +-1)
+  uint8_t* sX = sHD + kSmemS;                                    // [pair][NS] stages
+  float* sR2 = reinterpret_cast<float*>(sX + NS * kPairs * kStage);      // [pair][half][row] partial ||r||^2
+  uint64_t* full = reinterpret_cast<uint64_t*>(sR2 + kPairs * 2 * kTile);   // [pair][2]
+  uint64_t* ydone = full + 2 * kPairs;                           // [pair]
+  uint64_t* mdone = ydone + kPairs;                              // [pair]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kPairs);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* lut = reinterpret_cast<float*>(tmem_slot + 2);          // L centroids (scaled by 64)
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
+  if (tid == 0) {
+    for (int i = 0; i < 2 * kPairs; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < kPairs; ++i) { mbar_init(&ydone[i], 1); mbar_init(&mdone[i], 1); }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (tid < L) lut[tid] = P.c[tid] * kResScale;
+  for (int e = tid; e < kM * 16; e += kThreads) {
+    const int j = e >> 4, c = e & 15, kb = c >> 3, cc = c & 7;
+    const uint4 v = *reinterpret_cast<const uint4*>(P.S + j * kD + c * 8);
+    *reinterpret_cast<uint4*>(sS + kb * 16384 + j * 128 + ((cc ^ (j & 7)) << 4)) = v;
+  }
+  // (D H)[n][k] = H[n][k] D_k = (-1)^popcount(n & k) D_k, as bf16 +-1.0, same swizzled layout
+  uint16_t* hd16 = reinterpret_cast<uint16_t*>(sHD);
+  for (int e = tid; e < kD * kD; e += kThreads) {
+    const int n = e >> 7, k = e & 127;
+    const bool neg = ((__popc(n & k) & 1) != 0) != (X.Dsign[k] != 0u);
+    const int kb = k >> 6, chunk = (k & 63) >> 3, within = k & 7;
+    hd16[(kb * 16384 + n * 128 + ((chunk ^ (n & 7)) << 4)) / 2 + within] = neg ? 0xBF80u : 0x3F80u;
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int wgi = warp >> 2, pair = wgi >> 1, half = wgi & 1, lb = warp & 3;
+  const bool leader = (half == 0 && lb == 0 && lane == 0);
+  const int trow = lb * 32 + lane;
+  const uint32_t lane_base = static_cast<uint32_t>(lb * 32) << 16;
+  const uint32_t t_acc = tmem + lane_base + pair * 256;          // y', then the projections
+  const uint32_t t_a = t_acc + 128;                              // residual hi | lo
+  const uint32_t bar_id = 1 + pair;
+  uint8_t* stages = sX + pair * NS * kStage;
+  uint64_t* pfull = full + 2 * pair;
+  float* myR2 = sR2 + (pair * 2 + half) * kTile;
+  const float* otR2 = sR2 + (pair * 2 + (half ^ 1)) * kTile;
+  const int64_t t_first = blockIdx.x + static_cast<int64_t>(pair) * gridDim.x;
+  const int64_t t_step = static_cast<int64_t>(kPairs) * gridDim.x;
+  auto issue_load = [&](int64_t tile, int buf) {
+    mbar_arrive_expect_tx(&pfull[buf], kStage);
+#pragma unroll
+    for (int bx = 0; bx < 2; ++bx)
+      tma_load_2d(stages + buf * kStage + bx * (kTile * 128), &tmap, &pfull[buf], bx * 64,
+                  static_cast<int>(tile * kTile));
+  };
+  int issued[2] = {0, 0}, waited[2] = {0, 0};
+  if (leader) {
+    prefetch_tmap(&tmap);
+    if (t_first < n_tiles) { issue_load(t_first, 0); ++issued[0]; }
+    if (t_first + t_step < n_tiles) { issue_load(t_first + t_step, 1); ++issued[1]; }
+  }
+
+  int mine = 0;
+  for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
+    const int buf = mine & 1;
+    // #A: the previous tile's accumulator reads are done (and a uniform abort check)
+    if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
+    if (leader) {
+      if (mbar_wait(&pfull[buf], (mine >> 1) & 1, kWaitCycles)) ++waited[buf];
+      else flag_error(X.err, abort_flag, 2);
+      tc_fence_after();
+      const uint32_t xbase = smem_u32(stages + buf * kStage), hbase = smem_u32(sHD);
+      const uint32_t idesc = idesc_bf16_f32(kTile, kD);
+      const uint32_t d_tmem = tmem + pair * 256;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+        mma_f16_ss(d_tmem, smem_desc_sw128(xbase + off, 1024), smem_desc_sw128(hbase + off, 1024), idesc,
+                   k > 0 ? 1u : 0u);
+      }
+      mma_commit(&ydone[pair]);
+    }
+    if (!mbar_wait(&ydone[pair], mine & 1, kWaitCycles)) flag_error(X.err, abort_flag, 5);
+    tc_fence_after();
+    // the stage has been read by the rotation MMA: refill it two tiles ahead
+    if (leader && t + NS * t_step < n_tiles) { issue_load(t + NS * t_step, buf); ++issued[buf]; }
+
+    // ---- the row's rotated values: all 128 for the norm, my 64 kept ----------------
+    float v[kH];
+    float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {                                // the other half: squares only
+      uint32_t w[16];
+      tmem_ld16(t_acc + (half ^ 1) * 64 + c * 16, w);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 16; k += 2) {
+        const float2 a = make_float2(__uint_as_float(w[k]), __uint_as_float(w[k + 1]));
+        ss2 = __ffma2_rn(a, a, ss2);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {                                // my half, kept
+      uint32_t w[16];
+      tmem_ld16(t_acc + half * 64 + c * 16, w);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 16; k += 2) {
+        const float2 a = make_float2(__uint_as_float(w[k]), __uint_as_float(w[k + 1]));
+        ss2 = __ffma2_rn(a, a, ss2);
+        v[c * 16 + k] = a.x;
+        v[c * 16 + k + 1] = a.y;
+      }
+    }
+    const float nsd = sqrtf(ss2.x + ss2.y);                      // ||H D x|| = sqrt(d) ||x||
+    const float n = nsd * 0.08838834764831845f;                  // / sqrt(128)
+    const bool zero_row = !(n >= kZeroNorm);
+    const float nsd_t = zero_row ? 1.f : nsd;
+    const float sc64 = zero_row ? 0.f : kResScale / nsd_t;
+    float tq[L - 1];
+#pragma unroll
+    for (int k = 0; k < L - 1; ++k) tq[k] = P.t[k] * nsd_t;
+    uint32_t cw[B * 2];
+#pragma unroll
+    for (int w = 0; w < B * 2; ++w) cw[w] = 0u;
+    float2 r2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+      for (int e = ch * 32; e < ch * 32 + 32; ++e) {
+        const float y = v[e];
+        uint32_t code = 0u;
+#pragma unroll
+        for (int lev = B - 1; lev >= 0; --lev) {
+          const int base = (1 << lev) - 1;
+          float thr = tq[base];
+#pragma unroll
+          for (int k = 1; k < (1 << (B - 1 - lev)); ++k)
+            if (code == static_cast<uint32_t>(k << (lev + 1))) thr = tq[base + (k << (lev + 1))];
+          if (y > thr) code |= (1u << lev);
+        }
+        float r = fmaf(y, sc64, -lut[code]);
+        if (zero_row) r = 0.f;
+        v[e] = r;
+        if (e & 1) r2.y = fmaf(r, r, r2.y); else r2.x = fmaf(r, r, r2.x);
+        const int bit = B * e, wi = bit >> 5, sh = bit & 31;
+        cw[wi] |= code << sh;
+        if (sh + B > 32) cw[wi + 1] |= code >> (32 - sh);
+      }
+      uint32_t hw[16], lw[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int e = ch * 32 + 2 * k;
+        const __half2 h = __floats2half2_rn(v[e], v[e + 1]);
+        const float2 hf = __half22float2(h);
+        const __half2 l = __floats2half2_rn(v[e] - hf.x, v[e + 1] - hf.y);
+        hw[k] = *reinterpret_cast<const uint32_t*>(&h);
+        lw[k] = *reinterpret_cast<const uint32_t*>(&l);
+      }
+      tmem_st16(t_a + half * 32 + ch * 16, hw);
+      tmem_st16(t_a + 64 + half * 32 + ch * 16, lw);
+    }
+    if (zero_row) {
+#pragma unroll
+      for (int w = 0; w < B * 2; ++w) cw[w] = 0u;
+    }
+    myR2[trow] = r2.x + r2.y;
+    tmem_wait_st();
+    tc_fence_before();
+    // #B: A complete and every y' read done (the projection overwrites them)
+    if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
+    const float rho = zero_row ? 0.f : sqrtf(myR2[trow] + otR2[trow]) * (1.0f / kResScale);
+    if (leader) {
+      tc_fence_after();
+      const uint32_t sbase = smem_u32(sS);
+      const uint32_t idesc = idesc_f16_f32(kTile, kM);
+      const uint32_t d_tmem = tmem + pair * 256;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int kk = k & 7;
+        const uint64_t bdesc = smem_desc_sw128(sbase + (kk >> 2) * 16384 + (kk & 3) * 32, 1024);
+        mma_f16_ts(d_tmem, d_tmem + 128 + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
+      }
+      mma_commit(&mdone[pair]);
+    }
+    if (!mbar_wait(&mdone[pair], mine & 1, kWaitCycles)) flag_error(X.err, abort_flag, 3);
+    tc_fence_after();
+
+    // ---- my 64 signs, exact recomputation within the error bound of zero ------------
+    const float eps = kResScale * fmaf(X.eps_scale, rho, X.eps_abs);
+    uint32_t s0 = 0, s1 = 0, f0 = 0, f1 = 0;
+    float pmin = INFINITY;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t p[16];
+      tmem_ld16(t_acc + half * 64 + c * 16, p);
+      tmem_wait_ld();
+      uint32_t bits = 0u;
+#pragma unroll
+      for (int j = 15; j >= 0; --j) {
+        bits = (bits << 1) | (p[j] >> 31);
+        pmin = fminf(pmin, fabsf(__uint_as_float(p[j])));
+      }
+      if (c == 0) s0 = bits;
+      if (c == 1) s0 |= bits << 16;
+      if (c == 2) s1 = bits;
+      if (c == 3) s1 |= bits << 16;
+    }
+    if (__any_sync(0xffffffffu, pmin < eps)) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t p[16];
+        tmem_ld16(t_acc + half * 64 + c * 16, p);
+        tmem_wait_ld();
+        uint32_t flags = 0u;
+#pragma unroll
+        for (int j = 15; j >= 0; --j) flags = (flags << 1) | (fabsf(__uint_as_float(p[j])) < eps ? 1u : 0u);
+        if (c == 0) f0 = flags;
+        if (c == 1) f0 |= flags << 16;
+        if (c == 2) f1 = flags;
+        if (c == 3) f1 |= flags << 16;
+      }
+    }
+    const int nflag = __popc(f0) + __popc(f1);
+    const int passes = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(nflag));
+    for (int q = 0; q < passes; ++q) {
+      int j = -1;
+      if (q < nflag) {
+        if (f1) j = 32 + __ffs(f1) - 1;
+        if (f0) j = __ffs(f0) - 1;
+      }
+      const int jg = half * 64 + (j < 0 ? 0 : j);
+      float acc = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t ah[8], al[8];
+        tmem_ld8(t_a + c * 8, ah);
+        tmem_ld8(t_a + 64 + c * 8, al);
+        tmem_wait_ld();
+        if (j >= 0) {
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            const int chunk = c * 2 + qq, kb = chunk >> 3, cc = chunk & 7;
+            const uint4 sv = *reinterpret_cast<const uint4*>(sS + kb * 16384 + jg * 128 + ((cc ^ (jg & 7)) << 4));
+            const uint32_t sws[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int w = qq * 4 + u;
+              const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sws[u]));
+              const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&ah[w]));
+              const float2 lf = __half22float2(*reinterpret_cast<const __half2*>(&al[w]));
+              acc = fmaf(sf.x, hf.x + lf.x, acc);
+              acc = fmaf(sf.y, hf.y + lf.y, acc);
+            }
+          }
+        }
+      }
+      if (j >= 0) {
+        const uint32_t m = 1u << (j & 31), nb = acc < 0.f ? m : 0u;
+        if (j < 32) { s0 = (s0 & ~m) | nb; f0 &= ~m; }
+        else { s1 = (s1 & ~m) | nb; f1 &= ~m; }
+      }
+    }
+    if (zero_row || rho == 0.f) s0 = s1 = 0u;
+    tc_fence_before();
+    const int64_t row = t * kTile + trow;
+    if (row < n_rows) {
+      uint32_t* co = reinterpret_cast<uint32_t*>(out.codes + row * (B * 16) + half * (B * 8));
+      if constexpr (B == 1) {
+        *reinterpret_cast<uint2*>(co) = make_uint2(cw[0], cw[1]);
+      } else if constexpr (B == 2) {
+        *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      } else if constexpr (B == 3) {
+        if (half == 0) {
+          *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          *reinterpret_cast<uint2*>(co + 4) = make_uint2(cw[4], cw[5]);
+        } else {
+          *reinterpret_cast<uint2*>(co) = make_uint2(cw[0], cw[1]);
+          *reinterpret_cast<uint4*>(co + 2) = make_uint4(cw[2], cw[3], cw[4], cw[5]);
+        }
+      } else {
+        *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint4*>(co + 4) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      }
+      *reinterpret_cast<uint2*>(out.signs + row * 16 + half * 8) = make_uint2(s0, s1);
+      if (half == 0) {
+        out.norm[row] = zero_row ? 0.f : n;
+        out.rnorm[row] = zero_row ? 0.f : n * rho;
+      }
+    }
+  }
+  if (leader) {
+    for (int b2 = 0; b2 < 2; ++b2)
+      while (waited[b2] < issued[b2]) {
+        if (!mbar_wait(&pfull[b2], waited[b2] & 1, kWaitCycles)) { flag_error(X.err, abort_flag, 4); break; }
+        ++waited[b2];
+      }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // -------------------------------------------------------------------------- host
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() { return tensor_map_encoder(); }
+
+constexpr size_t quant_rot_smem_bytes() {
+  return 1024 + 2 * kSmemS + 2 * kPairs * XStage<true>::kBytes + kPairs * 2 * kTile * 4 + 256;
+}
 
 template <int B, bool BF16IN>
 int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, const Packed& out, cudaStream_t s) {
@@ -510,12 +845,21 @@ int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, cons
   X.eps_scale = ctx.qjl_eps_scale;
   X.eps_abs = ctx.qjl_eps_abs;
   X.err = P.err;
+  const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
+  const int grid = static_cast<int>(n_tiles < ctx.num_sms ? n_tiles : ctx.num_sms);
+  if (BF16IN) {
+    const size_t smem = quant_rot_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(k_quantize_d128_rot_tc<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+    k_quantize_d128_rot_tc<B><<<grid, kThreads, smem, s>>>(tmap, P, X, n_rows, out);
+    count_launch();
+    return static_cast<int>(cudaGetLastError());
+  }
   const size_t smem = quant_smem_bytes<BF16IN>();
   cudaError_t e = cudaFuncSetAttribute(k_quantize_d128_tc<B, BF16IN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return static_cast<int>(e);
-  const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
-  const int grid = static_cast<int>(n_tiles < ctx.num_sms ? n_tiles : ctx.num_sms);
   k_quantize_d128_tc<B, BF16IN><<<grid, kThreads, smem, s>>>(tmap, P, X, n_rows, out);
   count_launch();
   return static_cast<int>(cudaGetLastError());
