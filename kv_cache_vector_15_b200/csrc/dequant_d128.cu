@@ -7,14 +7,18 @@
 //   R^T = D H_d / sqrt(d)                                   0h-n0.github.io "ICLR
 //         2026論文解説: TurboQuant", "Step 1: PolarQuant"
 //
-// One thread per row (two warpgroups of 128 rows, persistent CTAs).  S^T z is
-// a 128 x 128 x 128 tensor-core product per tile: with z_j = 1 - 2 b_j,
-// S^T z = colsum(S) - 2 S^T b, and the sign bits b go into TMEM as binary16
-// values {0, 2^-14} (two shifts and a mask per pair of bits; S b is exact
-// in the MMA, the 2^14 comes back out as an exact scaling).  The centroid
-// decode, the inverse Walsh-Hadamard transform, D, 1/sqrt(d) and the output
-// rounding run in registers; the finished tile is written back by a TMA
-// tensor store from a swizzled shared-memory stage.
+// Both products run on the tcgen05 tensor cores, one 128-row tile at a time:
+//   1. S^T z (PROD): the sign bits go into TMEM as binary16 z_j 2^-14 (one
+//      shift and one mask per pair of bits), B = S^T (binary16, exact), so the
+//      fp32 sums are S^T z scaled by an exact 2^-14.
+//   2. the inverse rotation: each thread forms v = yhat + sqrt(pi/2)/m
+//      (rnorm / norm) S^T z for its 64 coordinates (unit-norm domain, x64),
+//      splits it into binary16 hi + lo in TMEM, and one MMA with
+//      B = [D H; D H] (exact +-1 entries, K = 256) gives D H v in fp32;
+//      norm / sqrt(d) / 64 scales the result.
+// The CUDA cores are left with the centroid decode, one FMA per coordinate,
+// the split and the output rounding; the finished tile leaves through a
+// swizzled shared-memory stage and a TMA tensor store.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -38,11 +42,11 @@ using namespace sm100;
 
 constexpr int kD = 128, kM = 128, kTile = 128, kPairs = 2, kThreads = kPairs * 256;
 constexpr long long kWaitCycles = 2000000000ll;
-constexpr uint32_t kTmemCols = 512;     // per pair: 128 D columns + 64 A columns (in 256)
+constexpr uint32_t kTmemCols = 512;     // per pair: 128 D columns + 128 A columns
+constexpr float kUnit = 64.0f;          // scale of the unit-norm domain the rotation runs in
 
 struct DequantD128Args {
-  float Dscale[kD];                     // D_i / sqrt(d)
-  float colsum[kD];                     // sum_j S[j][i]
+  uint32_t Dneg[kD / 32];               // bit i of word i / 32: D_i = -1
   int* err;
 };
 
@@ -55,7 +59,7 @@ struct OutStage {
 
 template <bool BF16OUT>
 constexpr size_t dequant_smem_bytes() {
-  return 1024 + 32768 /*St*/ + kPairs * OutStage<BF16OUT>::kBytes + 128;
+  return 1024 + 32768 /*St*/ + 32768 /*D H*/ + kPairs * OutStage<BF16OUT>::kBytes + 128;
 }
 
 __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* smem_src, int x, int y) {
@@ -67,10 +71,9 @@ __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Two warpgroups ("halves") share every 128-row tile: thread t of warp w in
-// half h owns output coordinates [64 h, 64 h + 64) of row 32 (w % 4) + t (the
-// row's TMEM lane).  Two such pairs run per CTA (512 threads).  The inverse
-// rotation starts with its stride-64 butterfly (the stages of H commute),
-// exchanged through the row's TMEM lane, then runs six stages in registers.
+// half h owns coordinates [64 h, 64 h + 64) of row 32 (w % 4) + t (the row's
+// TMEM lane), on the way in (code decode, S^T z) and on the way out (the
+// rotated output columns).  Two such pairs run per CTA (512 threads).
 template <int B, bool PROD, bool BF16OUT>
 __global__ void __launch_bounds__(kThreads, 1)
 k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P, const DequantD128Args X,
@@ -80,21 +83,23 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
   constexpr int kH = kD / 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sSt = smem;                                   // B operand: St (N = i, K = j), swizzled
-  uint8_t* sOut = smem + 32768;                          // [pair] output stages
-  uint64_t* mdone = reinterpret_cast<uint64_t*>(sOut + kPairs * kStage);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kPairs);
+  uint8_t* sSt = smem;                                   // B of the S^T z product (N = i, K = j), swizzled
+  uint8_t* sDH = smem + 32768;                           // B of the rotation (N = n, K = k), swizzled
+  uint8_t* sOut = smem + 65536;                          // [pair] output stages
+  uint64_t* m1 = reinterpret_cast<uint64_t*>(sOut + kPairs * kStage);   // [pair] S^T z done
+  uint64_t* m2 = m1 + kPairs;                                            // [pair] rotation done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(m2 + kPairs);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   float* lut = reinterpret_cast<float*>(tmem_slot + 2);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
   if (tid == 0) {
-    for (int i = 0; i < kPairs; ++i) mbar_init(&mdone[i], 1);
+    for (int i = 0; i < kPairs; ++i) { mbar_init(&m1[i], 1); mbar_init(&m2[i], 1); }
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (tid < L) lut[tid] = P.c[tid];
+  if (tid < L) lut[tid] = P.c[tid] * kUnit;
   if (PROD) {
     // B operand row i (output coordinate), K position kappa holds S[j(kappa)][i]
     // in the order the sign bits are laid out in TMEM (see the A construction):
@@ -107,8 +112,18 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
       const int kb = kappa >> 6, chunk = (kappa & 63) >> 3, within = kappa & 7;
       sSt16[(kb * 16384 + i * 128 + ((chunk ^ (i & 7)) << 4)) / 2 + within] = P.St[i * kM + j];
     }
-    fence_proxy_async_smem();
   }
+  {
+    // (D H)[n][k] = D_n (-1)^popcount(n & k), binary16 +-1, same swizzled layout
+    uint16_t* h16 = reinterpret_cast<uint16_t*>(sDH);
+    for (int e = tid; e < kD * kD; e += kThreads) {
+      const int n = e >> 7, k = e & 127;
+      const bool neg = ((__popc(n & k) & 1) != 0) != (((X.Dneg[n >> 5] >> (n & 31)) & 1u) != 0);
+      const int kb = k >> 6, chunk = (k & 63) >> 3, within = k & 7;
+      h16[(kb * 16384 + n * 128 + ((chunk ^ (n & 7)) << 4)) / 2 + within] = neg ? 0xBC00u : 0x3C00u;
+    }
+  }
+  fence_proxy_async_smem();
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -122,12 +137,12 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
   const bool leader = (half == 0 && lb == 0 && lane == 0);
   const int trow = lb * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>(lb * 32) << 16;
-  const uint32_t t_acc = tmem + lane_base + pair * 256;   // S^T b (128 columns), then the exchange
-  const uint32_t t_a = t_acc + 128;                       // sign bits as binary16 (64 columns)
+  const uint32_t t_acc = tmem + lane_base + pair * 256;   // S^T z, then the rotated row (128 columns)
+  const uint32_t t_a = t_acc + 128;                       // sign bits (64 columns), then v hi | lo (128)
   const uint32_t bar_id = 1 + pair;
   uint8_t* stage = sOut + pair * kStage;
   const float inv_sqrt_d = 0.08838834764831845f;
-  const float qjl = P.qjl_scale;
+  const float qjl = P.qjl_scale * 16384.0f * kUnit;       // S^T z = 2^14 * acc, in unit-norm x kUnit
   const int64_t t_first = blockIdx.x + static_cast<int64_t>(pair) * gridDim.x;
   const int64_t t_step = static_cast<int64_t>(kPairs) * gridDim.x;
   bool store_pending = false;
@@ -182,25 +197,27 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
 #pragma unroll
     for (int w = 0; w < B * 2; ++w) cw[w] = ncw[w];
     const uint32_t sg0 = nsg0, sg1 = nsg1;
-    const float nrm = nnrm, rn = nrn;
+    // v in the unit-norm domain times kUnit (binary16 hi | lo stay clear of
+    // underflow and overflow whatever the row's norm); norm / sqrt(d) / kUnit
+    // is applied to the rotated output
+    const float wq = nnrm > 0.f ? (nrn / nnrm) * qjl : 0.f;
+    const float oscale = nnrm * (inv_sqrt_d / kUnit);
     load_packed(t + t_step);
     if (PROD) {
-      // sign bits -> binary16 {0, 2^-14}: column k of sign word w holds bits
-      // (k, k + 16) of the word, i.e. projections 32 w + k and 32 w + k + 16;
-      // half h writes the columns of sign words 2h and 2h + 1
+      // z_j 2^-14 as binary16: column k of sign word w holds bits (k, k + 16)
+      // of the word, i.e. projections 32 w + k and 32 w + k + 16, moved to the
+      // sign bits (15, 31) of the pair; half h writes sign words 2h and 2h + 1
       uint32_t a[32];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         const uint32_t sgw = q == 0 ? sg0 : sg1;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const uint32_t sh = (k <= 10) ? (sgw << (10 - k)) : (sgw >> (k - 10));
-          a[q * 16 + k] = sh & 0x04000400u;
-        }
+        for (int k = 0; k < 16; ++k) a[q * 16 + k] = ((sgw << (15 - k)) & 0x80008000u) | 0x04000400u;
       }
       tmem_st32(t_a + half * 32, a);
       tmem_wait_st();
       tc_fence_before();
+      // #1: the sign operand is complete, and the previous tile's outputs are read
       if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
       if (leader) {
         tc_fence_after();
@@ -212,10 +229,10 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
           const uint64_t bdesc = smem_desc_sw128(sbase + (k >> 2) * 16384 + (k & 3) * 32, 1024);
           mma_f16_ts(d_tmem, d_tmem + 128 + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
         }
-        mma_commit(&mdone[pair]);
+        mma_commit(&m1[pair]);
       }
     }
-    // ---- norm * yhat of my coordinates while the MMA runs -------------------------
+    // ---- yhat of my coordinates while the MMA runs ----------------------------------
     float v[kH];
 #pragma unroll
     for (int e = 0; e < kH; ++e) {
@@ -223,73 +240,68 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
       uint32_t code = cw[wi] >> sh;
       if (sh + B > 32) code |= cw[wi + 1] << (32 - sh);
       code &= (1u << B) - 1u;
-      v[e] = nrm * lut[code];
+      v[e] = lut[code];
     }
     if (PROD) {
-      if (!mbar_wait(&mdone[pair], mine & 1, kWaitCycles)) {
+      if (!mbar_wait(&m1[pair], mine & 1, kWaitCycles)) {
         if (X.err) atomicCAS(X.err, 0, 5);
         atomicExch(abort_flag, 1);
       }
       tc_fence_after();
-      // sum_j z_j S[j][i] = colsum_i - 2 * 2^14 * acc_i
-      const float w = qjl * rn;
-      const float w2 = -2.0f * 16384.0f * w;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t acc[16];
-        tmem_ld16(t_acc + half * 64 + c * 16, acc);
+      for (int g2 = 0; g2 < 2; ++g2) {
+        uint32_t acc[2][16];
+        tmem_ld16(t_acc + half * 64 + g2 * 32, acc[0]);
+        tmem_ld16(t_acc + half * 64 + g2 * 32 + 16, acc[1]);
         tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int e = c * 16 + k;
-          v[e] = fmaf(w2, __uint_as_float(acc[k]), fmaf(w, X.colsum[half * kH + e], v[e]));
-        }
+        for (int k = 0; k < 32; ++k) v[g2 * 32 + k] = fmaf(wq, __uint_as_float(acc[k >> 4][k & 15]), v[g2 * 32 + k]);
       }
     }
-    // ---- stride-64 butterfly across the halves through the TMEM lane ----------------
+    // ---- v = hi + lo (binary16) into TMEM: the rotation's A operand ------------------
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t w16[16];
+    for (int ch = 0; ch < 2; ++ch) {
+      uint32_t hw[16], lw[16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) w16[k] = __float_as_uint(v[c * 16 + k]);
-      tmem_st16(t_acc + half * 64 + c * 16, w16);
+      for (int k = 0; k < 16; ++k) {
+        const int e = ch * 32 + 2 * k;
+        const __half2 h = __floats2half2_rn(v[e], v[e + 1]);
+        const float2 hf = __half22float2(h);
+        const __half2 l = __floats2half2_rn(v[e] - hf.x, v[e + 1] - hf.y);
+        hw[k] = *reinterpret_cast<const uint32_t*>(&h);
+        lw[k] = *reinterpret_cast<const uint32_t*>(&l);
+      }
+      tmem_st16(t_a + half * 32 + ch * 16, hw);
+      tmem_st16(t_a + 64 + half * 32 + ch * 16, lw);
     }
     tmem_wait_st();
     tc_fence_before();
-    named_bar_sync(bar_id, 256);
-    tc_fence_after();
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t w16[16];
-      tmem_ld16(t_acc + (half ^ 1) * 64 + c * 16, w16);
-      tmem_wait_ld();
+    // #2: v complete in TMEM and every S^T z read done (the rotation overwrites them)
+    if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
+    if (leader) {
+      tc_fence_after();
+      const uint32_t sbase = smem_u32(sDH);
+      const uint32_t idesc = idesc_f16_f32(kTile, kD);
+      const uint32_t d_tmem = tmem + pair * 256;
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
-        const float o = __uint_as_float(w16[k]);
-        v[c * 16 + k] = half == 0 ? v[c * 16 + k] + o : o - v[c * 16 + k];
+        const int kk = k & 7;
+        const uint64_t bdesc = smem_desc_sw128(sbase + (kk >> 2) * 16384 + (kk & 3) * 32, 1024);
+        mma_f16_ts(d_tmem, d_tmem + 128 + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
       }
+      mma_commit(&m2[pair]);
     }
+    if (!mbar_wait(&m2[pair], mine & 1, kWaitCycles)) {
+      if (X.err) atomicCAS(X.err, 0, 8);
+      atomicExch(abort_flag, 1);
+    }
+    tc_fence_after();
+    // ---- my 64 output columns, staged (swizzled) for the TMA store --------------------
+    uint32_t o[4][16];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld16(t_acc + half * 64 + c * 16, o[c]);
+    tmem_wait_ld();
     tc_fence_before();
-    // ---- six in-register stages --------------------------------------------------------
-#pragma unroll
-    for (int h = 2; h < kH; h <<= 1) {
-#pragma unroll
-      for (int e = 0; e < kH; e += 2) {
-        if ((e & h) == 0) {
-          const float2 a = make_float2(v[e], v[e + 1]), b = make_float2(v[e + h], v[e + h + 1]);
-          const float2 sum = __fadd2_rn(a, b);
-          const float2 dif = __ffma2_rn(b, make_float2(-1.f, -1.f), a);
-          v[e] = sum.x; v[e + 1] = sum.y; v[e + h] = dif.x; v[e + h + 1] = dif.y;
-        }
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < kH; e += 2) {
-      const float a = v[e], b = v[e + 1];
-      v[e] = a + b;
-      v[e + 1] = a - b;
-    }
-    // ---- stage my half row (swizzled for the TMA store) and write the tile -----------
     if (leader && store_pending) bulk_wait_read0();         // previous tile's store has read the stage
     named_bar_sync(bar_id, 256);
     if (BF16OUT) {
@@ -299,9 +311,9 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int e = cc * 8 + 2 * u;
-          const __nv_bfloat162 p = __floats2bfloat162_rn(v[e] * X.Dscale[half * kH + e],
-                                                         v[e + 1] * X.Dscale[half * kH + e + 1]);
-          wv[u] = *reinterpret_cast<const uint32_t*>(&p);
+          const __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(o[e >> 4][e & 15]) * oscale,
+                                                          __uint_as_float(o[(e + 1) >> 4][(e + 1) & 15]) * oscale);
+          wv[u] = *reinterpret_cast<const uint32_t*>(&p2);
         }
         *reinterpret_cast<uint4*>(stage + half * (kTile * 128) + trow * 128 + ((cc ^ (trow & 7)) << 4)) =
             make_uint4(wv[0], wv[1], wv[2], wv[3]);
@@ -310,13 +322,12 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
 #pragma unroll
       for (int c = 0; c < 16; ++c) {                        // boxes 2 half, 2 half + 1
         const int e = c * 4;
-        float4 o;
-        o.x = v[e + 0] * X.Dscale[half * kH + e + 0];
-        o.y = v[e + 1] * X.Dscale[half * kH + e + 1];
-        o.z = v[e + 2] * X.Dscale[half * kH + e + 2];
-        o.w = v[e + 3] * X.Dscale[half * kH + e + 3];
+        const float4 w4 = make_float4(__uint_as_float(o[e >> 4][e & 15]) * oscale,
+                                      __uint_as_float(o[e >> 4][(e & 15) + 1]) * oscale,
+                                      __uint_as_float(o[e >> 4][(e & 15) + 2]) * oscale,
+                                      __uint_as_float(o[e >> 4][(e & 15) + 3]) * oscale);
         const int bx = 2 * half + (c >> 3), cc = c & 7;
-        *reinterpret_cast<float4*>(stage + bx * (kTile * 128) + trow * 128 + ((cc ^ (trow & 7)) << 4)) = o;
+        *reinterpret_cast<float4*>(stage + bx * (kTile * 128) + trow * 128 + ((cc ^ (trow & 7)) << 4)) = w4;
       }
     }
     fence_proxy_async_smem();
@@ -353,10 +364,9 @@ int launch(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, cudaS
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return static_cast<int>(cudaErrorInvalidValue);
   DequantD128Args X;
-  for (int i = 0; i < kD; ++i) {
-    X.Dscale[i] = static_cast<float>(ctx.D[i] / std::sqrt(128.0));
-    X.colsum[i] = ctx.colsum_d128[i];
-  }
+  for (int w = 0; w < kD / 32; ++w) X.Dneg[w] = 0u;
+  for (int i = 0; i < kD; ++i)
+    if (ctx.D[i] < 0) X.Dneg[i >> 5] |= 1u << (i & 31);
   X.err = P.err;
   const size_t smem = dequant_smem_bytes<BF16OUT>();
   cudaError_t e = cudaFuncSetAttribute(k_dequant_d128_tc<B, PROD, BF16OUT>,

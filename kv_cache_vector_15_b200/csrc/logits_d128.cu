@@ -60,11 +60,15 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
 template <int B>
 struct Shape {
   static constexpr int kCodeWords = B * 4;                  // 32-bit words of codes per key
+  static constexpr int kCodeBytes = B * 16;
   static constexpr int kAWords = 8 * (kCodeWords + 4);      // 0/1 bytes, four per TMEM column
   static constexpr int kK = 4 * kAWords;                    // K of the MMA (bytes)
   static constexpr int kKBlocks = kK / 128;                 // 128-byte swizzle atoms along K
   static constexpr int kKSteps = kK / 32;
+  static constexpr int kStageBytes = kTile * (kCodeBytes + 16);   // one tile's codes | signs
 };
+
+constexpr int kStages = 4;                   // packed tiles in flight per warpgroup
 
 struct LogitsArgs {
   float wbit[2];                  // weight of code bit 0 / 1 in the centroid
@@ -84,12 +88,16 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wg = warp >> 2, wl = warp & 3;
   uint8_t* sB = smem + wg * kBBytes;
-  float* sScal = reinterpret_cast<float*>(smem + kWG * kBBytes) + wg * 64;   // per-warpgroup scalars
-  uint64_t* mdone = reinterpret_cast<uint64_t*>(smem + kWG * kBBytes + kWG * 64 * 4);
+  uint8_t* stages = smem + kWG * kBBytes + wg * kStages * S::kStageBytes;
+  float* sScal = reinterpret_cast<float*>(smem + kWG * (kBBytes + kStages * S::kStageBytes)) + wg * 64;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWG * (kBBytes + kStages * S::kStageBytes) + kWG * 64 * 4);
+  uint64_t* full = bars + wg * kStages;                     // [wg][stage]
+  uint64_t* mdone = bars + kWG * kStages;                   // [wg]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kWG);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   if (tid == 0) {
+    for (int i = 0; i < kWG * kStages; ++i) mbar_init(&bars[i], 1);
     for (int i = 0; i < kWG; ++i) mbar_init(&mdone[i], 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -107,52 +115,53 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
   const uint32_t t_base = tmem + (static_cast<uint32_t>(wl * 32) << 16) + wg * 128;   // this thread's lane
   const uint32_t t_a = t_base, t_d = t_base + S::kAWords;
 
-  // contiguous tile range of this warpgroup
+  // contiguous tile range of this warpgroup; (set, key tile) advance incrementally
   const int64_t tiles_per_set = (n_keys + kTile - 1) / kTile;
   const int64_t n_tiles = tiles_per_set * n_sets;
   const int64_t n_wg = static_cast<int64_t>(gridDim.x) * kWG;
   const int64_t wid = static_cast<int64_t>(blockIdx.x) * kWG + wg;
   const int64_t t0 = n_tiles * wid / n_wg, t1 = n_tiles * (wid + 1) / n_wg;
-  int64_t cur_set = -1;
-  int mine = 0;
-  // packed key of this thread for the next tile, loaded one tile ahead
-  uint32_t ncw[S::kCodeWords], nsw[4];
+  const int64_t n_mine = t1 - t0;
+  int64_t set = t0 / tiles_per_set, kt = t0 - (t0 / tiles_per_set) * tiles_per_set;
+
+  // producer (the warpgroup's leader): bulk copies of a tile's codes and signs
+  int64_t p_set = set, p_kt = kt, issued = 0, consumed = 0;
+  auto issue = [&](int stage) {
+    const int64_t row0 = p_set * n_keys + p_kt * kTile;
+    const int64_t left = n_keys - p_kt * kTile;
+    const uint32_t valid = static_cast<uint32_t>(left < kTile ? left : kTile);
+    uint8_t* st = stages + stage * S::kStageBytes;
+    mbar_arrive_expect_tx(&full[stage], valid * (S::kCodeBytes + 16));
+    bulk_load(st, keys.codes + row0 * S::kCodeBytes, valid * S::kCodeBytes, &full[stage]);
+    bulk_load(st + kTile * S::kCodeBytes, keys.signs + row0 * 16, valid * 16, &full[stage]);
+    if (++p_kt == tiles_per_set) { p_kt = 0; ++p_set; }
+    ++issued;
+  };
+  if (leader)
+    for (int i = 0; i < kStages && i < n_mine; ++i) issue(i);
+
+  // norms of this thread's key, loaded one tile ahead
   float nnrm = 0.f, nrn = 0.f;
-  auto load_key = [&](int64_t tile) {
-    const int64_t set = tile / tiles_per_set;
-    const int64_t key = (tile % tiles_per_set) * kTile + trow;
-    if (tile < t1 && key < n_keys) {
-      const int64_t row = set * n_keys + key;
-      const uint4* cp = reinterpret_cast<const uint4*>(keys.codes + row * (B * 16));
-#pragma unroll
-      for (int q = 0; q < B; ++q) {
-        const uint4 u = __ldg(cp + q);
-        ncw[4 * q] = u.x; ncw[4 * q + 1] = u.y; ncw[4 * q + 2] = u.z; ncw[4 * q + 3] = u.w;
-      }
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(keys.signs + row * 16));
-      nsw[0] = u.x; nsw[1] = u.y; nsw[2] = u.z; nsw[3] = u.w;
-      nnrm = __ldg(keys.norm + row);
-      nrn = __ldg(keys.rnorm + row);
-    } else {
-#pragma unroll
-      for (int w = 0; w < S::kCodeWords; ++w) ncw[w] = 0u;
-      nsw[0] = nsw[1] = nsw[2] = nsw[3] = 0u;
-      nnrm = 0.f;
-      nrn = 0.f;
+  auto load_norms = [&](int64_t s_, int64_t kt_) {
+    const int64_t key = kt_ * kTile + trow;
+    nnrm = nrn = 0.f;
+    if (key < n_keys) {
+      nnrm = __ldg(keys.norm + s_ * n_keys + key);
+      nrn = __ldg(keys.rnorm + s_ * n_keys + key);
     }
   };
-  load_key(t0);
-  for (int64_t t = t0; t < t1; ++t, ++mine) {
-    const int64_t set = t / tiles_per_set;
-    const int64_t key = (t % tiles_per_set) * kTile + trow;
+  if (n_mine > 0) load_norms(set, kt);
+
+  int64_t cur_set = -1;
+  for (int64_t i = 0; i < n_mine; ++i) {
+    const int stage = static_cast<int>(i % kStages);
+    const uint32_t parity = static_cast<uint32_t>((i / kStages) & 1);
+    const int64_t key = kt * kTile + trow;
     const bool valid = key < n_keys;
-    uint32_t cw[S::kCodeWords], sw[4];
-#pragma unroll
-    for (int w = 0; w < S::kCodeWords; ++w) cw[w] = ncw[w];
-#pragma unroll
-    for (int w = 0; w < 4; ++w) sw[w] = nsw[w];
     const float nrm = nnrm, rn = nrn * P.qjl_scale;
-    load_key(t + 1);
+    int64_t nset = set, nkt = kt + 1;
+    if (nkt == tiles_per_set) { nkt = 0; ++nset; }
+    if (i + 1 < n_mine) load_norms(nset, nkt);
     if (set != cur_set) {
       // ---- build the query operand of this set --------------------------------
       cur_set = set;
@@ -239,23 +248,43 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
         const int q = trow % G;
         const bool isq = trow >= G;
         float acc = 0.f;
-        for (int i = 0; i < 128; ++i) acc += qs[q * (kD + kM) + (isq ? kD : 0) + i];
+        for (int i2 = 0; i2 < 128; ++i2) acc += qs[q * (kD + kM) + (isq ? kD : 0) + i2];
         sScal[2 * G + trow] = isq ? acc : X.cconst * acc;
         sScal[4 * G + trow] = 1.f / scale[trow];
       }
       fence_proxy_async_smem();
       named_bar_sync(1 + wg, 128);
     }
-    // ---- decode this thread's key into TMEM ------------------------------------------
+    // ---- this thread's key from the stage, decoded into TMEM -----------------------
+    if (mbar_wait(&full[stage], parity, kWaitCycles)) {
+      if (leader) ++consumed;
+    } else {
+      if (X.err) atomicCAS(X.err, 0, 7);
+      atomicExch(abort_flag, 1);
+    }
     {
+      uint32_t cw[S::kCodeWords + 4];
+      const uint8_t* st = stages + stage * S::kStageBytes;
+      if (valid) {
+#pragma unroll
+        for (int q = 0; q < B; ++q) {
+          const uint4 u = *reinterpret_cast<const uint4*>(st + trow * S::kCodeBytes + 16 * q);
+          cw[4 * q] = u.x; cw[4 * q + 1] = u.y; cw[4 * q + 2] = u.z; cw[4 * q + 3] = u.w;
+        }
+        const uint4 u = *reinterpret_cast<const uint4*>(st + kTile * S::kCodeBytes + trow * 16);
+        cw[S::kCodeWords] = u.x; cw[S::kCodeWords + 1] = u.y;
+        cw[S::kCodeWords + 2] = u.z; cw[S::kCodeWords + 3] = u.w;
+      } else {
+#pragma unroll
+        for (int w = 0; w < S::kCodeWords + 4; ++w) cw[w] = 0u;
+      }
       uint32_t a[32];
       int n = 0, col = 0;
 #pragma unroll
       for (int c = 0; c < S::kCodeWords + 4; ++c) {
-        const uint32_t w = c < S::kCodeWords ? cw[c] : sw[c - S::kCodeWords];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          a[n++] = (w >> k) & 0x01010101u;
+          a[n++] = (cw[c] >> k) & 0x01010101u;
           if (n == 32) {
             tmem_st32(t_a + col, a);
             col += 32;
@@ -266,8 +295,10 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
     }
     tmem_wait_st();
     tc_fence_before();
+    // every thread has read its key from the stage and written its TMEM row
     if (named_bar_sync_or(1 + wg, 128, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
     if (leader) {
+      if (issued < n_mine) issue(stage);
       tc_fence_after();
       const uint32_t sbase = smem_u32(sB);
       const uint32_t idesc = idesc_i8(kTile, N);
@@ -279,7 +310,7 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
       }
       mma_commit(&mdone[wg]);
     }
-    if (!mbar_wait(&mdone[wg], mine & 1, kWaitCycles)) {
+    if (!mbar_wait(&mdone[wg], static_cast<uint32_t>(i & 1), kWaitCycles)) {
       if (X.err) atomicCAS(X.err, 0, 6);
       atomicExch(abort_flag, 1);
     }
@@ -298,6 +329,7 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
     }
     tc_fence_before();
     if (valid) {
+      float* o = out + set * G * n_keys + key;
 #pragma unroll
       for (int q = 0; q < G; ++q) {
         const int mse_i = static_cast<int>(acc[3 * q]) + (static_cast<int>(acc[3 * q + 1]) << 8) +
@@ -306,8 +338,17 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
                           (static_cast<int>(acc[NG + 3 * q + 2]) << 16);
         const float mse = fmaf(static_cast<float>(mse_i), sScal[4 * G + q], sScal[2 * G + q]);
         const float qjl = fmaf(static_cast<float>(qjl_i), sScal[4 * G + G + q], sScal[2 * G + G + q]);
-        out[(set * G + q) * n_keys + key] = fmaf(nrm, mse, rn * qjl);
+        o[q * n_keys] = fmaf(nrm, mse, rn * qjl);
       }
+    }
+    set = nset;
+    kt = nkt;
+  }
+  if (leader) {
+    // copies still in flight (only after an abort): let them land before exit
+    for (; consumed < issued; ++consumed) {
+      const int64_t j = consumed;
+      if (!mbar_wait(&full[j % kStages], static_cast<uint32_t>((j / kStages) & 1), kWaitCycles)) break;
     }
   }
   __syncthreads();
@@ -334,7 +375,8 @@ int launch_G(const tq_ctx& ctx, const float* qp, int64_t n_sets, int64_t n_keys,
     X.cconst = -P.c[1];
   }
   X.err = P.err;
-  const size_t smem = 1024 + static_cast<size_t>(kWG) * Sh::kKBlocks * (2 * NG) * 128 + kWG * 64 * 4 + 64;
+  const size_t smem = 1024 + static_cast<size_t>(kWG) * (Sh::kKBlocks * (2 * NG) * 128 + kStages * Sh::kStageBytes) +
+                      kWG * 64 * 4 + (kWG * kStages + kWG) * 8 + 16;
   cudaError_t e = cudaFuncSetAttribute(k_logits_d128_i8<B, G, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return static_cast<int>(e);
