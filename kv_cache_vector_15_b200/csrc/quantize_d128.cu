@@ -22,8 +22,8 @@
 // (|r - hi - lo| <= 2^-22 |r| + 2^-25) and the MMA accumulates S hi + S lo
 // (K = 256) in fp32.  A sign is taken from the tensor-core sum only where
 // |p_j| exceeds a bound on that sum's error, eps = eps_scale ||r|| + eps_abs
-// with eps_scale = 4 * 18 * 2^-22 * max_j ||S_j||_2 (18 = 16 accumulation
-// steps + the split + slack, times 4 for margin) and eps_abs =
+// with eps_scale = 16 * 2^-22 * max_j ||S_j||_2 (the split's 2^-22 plus 16
+// accumulation steps of at most 2^-23 each, with margin) and eps_abs =
 // max_j ||S_j||_1 * 2^-25 / 64 (binary16 underflow); the rare projections
 // below it are recomputed in fp32 on the CUDA cores from hi + lo.
 //
@@ -514,7 +514,8 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
   uint64_t* mdone = ydone + kPairs;                              // [pair]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kPairs);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  float* lut = reinterpret_cast<float*>(tmem_slot + 2);          // L centroids (scaled by 64)
+  float* lut = reinterpret_cast<float*>(tmem_slot + 2);          // L centroids (scaled by 64), then L zeros
+  int* loads_issued = reinterpret_cast<int*>(lut + 2 * L);       // [pair][stage]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
@@ -524,7 +525,7 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (tid < L) lut[tid] = P.c[tid] * kResScale;
+  if (tid < 2 * L) lut[tid] = tid < L ? P.c[tid] * kResScale : 0.f;
   for (int e = tid; e < kM * 16; e += kThreads) {
     const int j = e >> 4, c = e & 15, kb = c >> 3, cc = c & 7;
     const uint4 v = *reinterpret_cast<const uint4*>(P.S + j * kD + c * 8);
@@ -549,7 +550,8 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
   const uint32_t tmem = *tmem_slot;
 
   const int wgi = warp >> 2, pair = wgi >> 1, half = wgi & 1, lb = warp & 3;
-  const bool leader = (half == 0 && lb == 0 && lane == 0);
+  const bool leader = (half == 0 && lb == 0 && lane == 0);       // waits for stages, issues MMAs
+  const bool loader = (half == 1 && lb == 0 && lane == 0);       // issues the stage loads (TMA)
   const int trow = lb * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>(lb * 32) << 16;
   const uint32_t t_acc = tmem + lane_base + pair * 256;          // y', then the projections
@@ -569,7 +571,7 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
                   static_cast<int>(tile * kTile));
   };
   int issued[2] = {0, 0}, waited[2] = {0, 0};
-  if (leader) {
+  if (loader) {
     prefetch_tmap(&tmap);
     if (t_first < n_tiles) { issue_load(t_first, 0); ++issued[0]; }
     if (t_first + t_step < n_tiles) { issue_load(t_first + t_step, 1); ++issued[1]; }
@@ -597,41 +599,39 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
     }
     if (!mbar_wait(&ydone[pair], mine & 1, kWaitCycles)) flag_error(X.err, abort_flag, 5);
     tc_fence_after();
-    // the stage has been read by the rotation MMA: refill it two tiles ahead
-    if (leader && t + NS * t_step < n_tiles) { issue_load(t + NS * t_step, buf); ++issued[buf]; }
 
     // ---- the row's rotated values: all 128 for the norm, my 64 kept ----------------
-    float v[kH];
+    // (four loads in flight per wait: the other half's columns, then my own)
+    uint32_t u[kH];
     float2 ss2 = make_float2(0.f, 0.f);
+    {
+      uint32_t w[4][16];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {                                // the other half: squares only
-      uint32_t w[16];
-      tmem_ld16(t_acc + (half ^ 1) * 64 + c * 16, w);
+      for (int c = 0; c < 4; ++c) tmem_ld16(t_acc + (half ^ 1) * 64 + c * 16, w[c]);
       tmem_wait_ld();
 #pragma unroll
-      for (int k = 0; k < 16; k += 2) {
-        const float2 a = make_float2(__uint_as_float(w[k]), __uint_as_float(w[k + 1]));
-        ss2 = __ffma2_rn(a, a, ss2);
-      }
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int k = 0; k < 16; k += 2) {
+          const float2 a = make_float2(__uint_as_float(w[c][k]), __uint_as_float(w[c][k + 1]));
+          ss2 = __ffma2_rn(a, a, ss2);
+        }
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {                                // my half, kept
-      uint32_t w[16];
-      tmem_ld16(t_acc + half * 64 + c * 16, w);
-      tmem_wait_ld();
+    for (int c = 0; c < 4; ++c) tmem_ld16(t_acc + half * 64 + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&u[c * 16]));
+    tmem_wait_ld();
 #pragma unroll
-      for (int k = 0; k < 16; k += 2) {
-        const float2 a = make_float2(__uint_as_float(w[k]), __uint_as_float(w[k + 1]));
-        ss2 = __ffma2_rn(a, a, ss2);
-        v[c * 16 + k] = a.x;
-        v[c * 16 + k + 1] = a.y;
-      }
+    for (int k = 0; k < kH; k += 2) {
+      const float2 a = make_float2(__uint_as_float(u[k]), __uint_as_float(u[k + 1]));
+      ss2 = __ffma2_rn(a, a, ss2);
     }
     const float nsd = sqrtf(ss2.x + ss2.y);                      // ||H D x|| = sqrt(d) ||x||
     const float n = nsd * 0.08838834764831845f;                  // / sqrt(128)
     const bool zero_row = !(n >= kZeroNorm);
     const float nsd_t = zero_row ? 1.f : nsd;
     const float sc64 = zero_row ? 0.f : kResScale / nsd_t;
+    // a zero row reads an all-zero table: y = 0, scale 0, residual 0
+    const float* tab = zero_row ? lut + L : lut;
     float tq[L - 1];
 #pragma unroll
     for (int k = 0; k < L - 1; ++k) tq[k] = P.t[k] * nsd_t;
@@ -641,36 +641,35 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
     float2 r2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int ch = 0; ch < 2; ++ch) {
-#pragma unroll
-      for (int e = ch * 32; e < ch * 32 + 32; ++e) {
-        const float y = v[e];
-        uint32_t code = 0u;
-#pragma unroll
-        for (int lev = B - 1; lev >= 0; --lev) {
-          const int base = (1 << lev) - 1;
-          float thr = tq[base];
-#pragma unroll
-          for (int k = 1; k < (1 << (B - 1 - lev)); ++k)
-            if (code == static_cast<uint32_t>(k << (lev + 1))) thr = tq[base + (k << (lev + 1))];
-          if (y > thr) code |= (1u << lev);
-        }
-        float r = fmaf(y, sc64, -lut[code]);
-        if (zero_row) r = 0.f;
-        v[e] = r;
-        if (e & 1) r2.y = fmaf(r, r, r2.y); else r2.x = fmaf(r, r, r2.x);
-        const int bit = B * e, wi = bit >> 5, sh = bit & 31;
-        cw[wi] |= code << sh;
-        if (sh + B > 32) cw[wi + 1] |= code >> (32 - sh);
-      }
       uint32_t hw[16], lw[16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int e = ch * 32 + 2 * k;
-        const __half2 h = __floats2half2_rn(v[e], v[e + 1]);
+      for (int e = ch * 32; e < ch * 32 + 32; e += 2) {
+        float rr[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const float y = __uint_as_float(u[e + q]);
+          uint32_t code = 0u;
+#pragma unroll
+          for (int lev = B - 1; lev >= 0; --lev) {
+            const int base = (1 << lev) - 1;
+            float thr = tq[base];
+#pragma unroll
+            for (int k = 1; k < (1 << (B - 1 - lev)); ++k)
+              if (code == static_cast<uint32_t>(k << (lev + 1))) thr = tq[base + (k << (lev + 1))];
+            if (y > thr) code |= (1u << lev);
+          }
+          rr[q] = fmaf(y, sc64, -tab[code]);
+          const int bit = B * (e + q), wi = bit >> 5, sh = bit & 31;
+          cw[wi] |= code << sh;
+          if (sh + B > 32) cw[wi + 1] |= code >> (32 - sh);
+        }
+        const float2 rv = make_float2(rr[0], rr[1]);
+        r2 = __ffma2_rn(rv, rv, r2);
+        const __half2 h = __floats2half2_rn(rr[0], rr[1]);
         const float2 hf = __half22float2(h);
-        const __half2 l = __floats2half2_rn(v[e] - hf.x, v[e + 1] - hf.y);
-        hw[k] = *reinterpret_cast<const uint32_t*>(&h);
-        lw[k] = *reinterpret_cast<const uint32_t*>(&l);
+        const __half2 l = __floats2half2_rn(rr[0] - hf.x, rr[1] - hf.y);
+        hw[(e - ch * 32) >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+        lw[(e - ch * 32) >> 1] = *reinterpret_cast<const uint32_t*>(&l);
       }
       tmem_st16(t_a + half * 32 + ch * 16, hw);
       tmem_st16(t_a + 64 + half * 32 + ch * 16, lw);
@@ -705,21 +704,24 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
     const float eps = kResScale * fmaf(X.eps_scale, rho, X.eps_abs);
     uint32_t s0 = 0, s1 = 0, f0 = 0, f1 = 0;
     float pmin = INFINITY;
+    {
+      uint32_t p[4][16];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t p[16];
-      tmem_ld16(t_acc + half * 64 + c * 16, p);
+      for (int c = 0; c < 4; ++c) tmem_ld16(t_acc + half * 64 + c * 16, p[c]);
       tmem_wait_ld();
-      uint32_t bits = 0u;
 #pragma unroll
-      for (int j = 15; j >= 0; --j) {
-        bits = (bits << 1) | (p[j] >> 31);
-        pmin = fminf(pmin, fabsf(__uint_as_float(p[j])));
+      for (int c = 0; c < 4; ++c) {
+        uint32_t bits = 0u;
+#pragma unroll
+        for (int j = 15; j >= 0; --j) {
+          bits = (bits << 1) | (p[c][j] >> 31);
+          pmin = fminf(pmin, fabsf(__uint_as_float(p[c][j])));
+        }
+        if (c == 0) s0 = bits;
+        if (c == 1) s0 |= bits << 16;
+        if (c == 2) s1 = bits;
+        if (c == 3) s1 |= bits << 16;
       }
-      if (c == 0) s0 = bits;
-      if (c == 1) s0 |= bits << 16;
-      if (c == 2) s1 = bits;
-      if (c == 3) s1 |= bits << 16;
     }
     if (__any_sync(0xffffffffu, pmin < eps)) {
 #pragma unroll
@@ -746,26 +748,26 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
       }
       const int jg = half * 64 + (j < 0 ? 0 : j);
       float acc = 0.f;
+      // S_j . hi, then S_j . lo: 32 columns per load batch, one wait each
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t ah[8], al[8];
-        tmem_ld8(t_a + c * 8, ah);
-        tmem_ld8(t_a + 64 + c * 8, al);
+      for (int part = 0; part < 4; ++part) {
+        uint32_t a[2][16];
+        tmem_ld16(t_a + part * 32, a[0]);
+        tmem_ld16(t_a + part * 32 + 16, a[1]);
         tmem_wait_ld();
         if (j >= 0) {
 #pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            const int chunk = c * 2 + qq, kb = chunk >> 3, cc = chunk & 7;
+          for (int ch = 0; ch < 8; ++ch) {
+            const int chunk = (part & 1) * 8 + ch, kb = chunk >> 3, cc = chunk & 7;
             const uint4 sv = *reinterpret_cast<const uint4*>(sS + kb * 16384 + jg * 128 + ((cc ^ (jg & 7)) << 4));
             const uint32_t sws[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              const int w = qq * 4 + u;
+              const int w = ch * 4 + u;                              // column part * 32 + w
               const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sws[u]));
-              const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&ah[w]));
-              const float2 lf = __half22float2(*reinterpret_cast<const __half2*>(&al[w]));
-              acc = fmaf(sf.x, hf.x + lf.x, acc);
-              acc = fmaf(sf.y, hf.y + lf.y, acc);
+              const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&a[w >> 4][w & 15]));
+              acc = fmaf(sf.x, hf.x, acc);
+              acc = fmaf(sf.y, hf.y, acc);
             }
           }
         }
@@ -803,8 +805,17 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
         out.rnorm[row] = zero_row ? 0.f : n * rho;
       }
     }
+    // the stage was read by this tile's rotation MMA: refill it two tiles ahead
+    // (a TMA issue can hold its thread for a while, so it comes from a warp of
+    // the other half than the one that issues the MMAs)
+    if (loader && t + NS * t_step < n_tiles) { issue_load(t + NS * t_step, buf); ++issued[buf]; }
   }
+  // let every issued stage load land before the shared memory is released
+  if (loader) { loads_issued[2 * pair] = issued[0]; loads_issued[2 * pair + 1] = issued[1]; }
+  __syncthreads();
   if (leader) {
+    issued[0] = loads_issued[2 * pair];
+    issued[1] = loads_issued[2 * pair + 1];
     for (int b2 = 0; b2 < 2; ++b2)
       while (waited[b2] < issued[b2]) {
         if (!mbar_wait(&pfull[b2], waited[b2] & 1, kWaitCycles)) { flag_error(X.err, abort_flag, 4); break; }
