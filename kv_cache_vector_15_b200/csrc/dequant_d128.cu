@@ -134,7 +134,8 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
   const uint32_t tmem = *tmem_slot;
 
   const int wgi = warp >> 2, pair = wgi >> 1, half = wgi & 1, lb = warp & 3;
-  const bool leader = (half == 0 && lb == 0 && lane == 0);
+  const bool leader = (half == 0 && lb == 0 && lane == 0);        // issues the pair's MMAs
+  const bool storer = (half == 1 && lb == 0 && lane == 0);        // issues the pair's TMA stores
   const int trow = lb * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>(lb * 32) << 16;
   const uint32_t t_acc = tmem + lane_base + pair * 256;   // S^T z, then the rotated row (128 columns)
@@ -302,7 +303,7 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
     for (int c = 0; c < 4; ++c) tmem_ld16(t_acc + half * 64 + c * 16, o[c]);
     tmem_wait_ld();
     tc_fence_before();
-    if (leader && store_pending) bulk_wait_read0();         // previous tile's store has read the stage
+    if (storer && store_pending) bulk_wait_read0();         // previous tile's store has read the stage
     named_bar_sync(bar_id, 256);
     if (BF16OUT) {
 #pragma unroll
@@ -332,7 +333,7 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
     }
     fence_proxy_async_smem();
     named_bar_sync(bar_id, 256);
-    if (leader) {
+    if (storer) {
 #pragma unroll
       for (int bx = 0; bx < OutStage<BF16OUT>::kBoxes; ++bx)
         tma_store_2d(&tmap_out, stage + bx * (kTile * 128), bx * OutStage<BF16OUT>::kColsPerBox,
@@ -341,7 +342,7 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
       store_pending = true;
     }
   }
-  if (leader && store_pending) bulk_wait0();               // all our stores have landed
+  if (storer && store_pending) bulk_wait0();               // all our stores have landed
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
