@@ -59,7 +59,7 @@ struct OutStage {
 
 template <bool BF16OUT>
 constexpr size_t dequant_smem_bytes() {
-  return 1024 + 32768 /*St*/ + 32768 /*D H*/ + kPairs * OutStage<BF16OUT>::kBytes + 128;
+  return 1024 + 32768 /*St*/ + 32768 /*D H*/ + kPairs * OutStage<BF16OUT>::kBytes + 512;
 }
 
 __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* smem_src, int x, int y) {
@@ -90,7 +90,8 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
   uint64_t* m2 = m1 + kPairs;                                            // [pair] rotation done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(m2 + kPairs);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  float* lut = reinterpret_cast<float*>(tmem_slot + 2);
+  float* lut = reinterpret_cast<float*>(tmem_slot + 2);                 // L centroids x kUnit
+  float2* lut2 = reinterpret_cast<float2*>(lut + 16);                   // 2-bit codes: pairs (4 bits)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
@@ -100,6 +101,7 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
     mbar_fence_init();
   }
   if (tid < L) lut[tid] = P.c[tid] * kUnit;
+  if (B == 2 && tid < 16) lut2[tid] = make_float2(P.c[tid & 3] * kUnit, P.c[tid >> 2] * kUnit);
   if (PROD) {
     // B operand row i (output coordinate), K position kappa holds S[j(kappa)][i]
     // in the order the sign bits are laid out in TMEM (see the A construction):
@@ -235,13 +237,22 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
     }
     // ---- yhat of my coordinates while the MMA runs ----------------------------------
     float v[kH];
+    if constexpr (B == 2) {
 #pragma unroll
-    for (int e = 0; e < kH; ++e) {
-      const int bit = B * e, wi = bit >> 5, sh = bit & 31;
-      uint32_t code = cw[wi] >> sh;
-      if (sh + B > 32) code |= cw[wi + 1] << (32 - sh);
-      code &= (1u << B) - 1u;
-      v[e] = lut[code];
+      for (int e = 0; e < kH; e += 2) {                    // two codes per lookup
+        const float2 c2 = lut2[(cw[e >> 4] >> ((2 * e) & 31)) & 15u];
+        v[e] = c2.x;
+        v[e + 1] = c2.y;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < kH; ++e) {
+        const int bit = B * e, wi = bit >> 5, sh = bit & 31;
+        uint32_t code = cw[wi] >> sh;
+        if (sh + B > 32) code |= cw[wi + 1] << (32 - sh);
+        code &= (1u << B) - 1u;
+        v[e] = lut[code];
+      }
     }
     if (PROD) {
       if (!mbar_wait(&m1[pair], mine & 1, kWaitCycles)) {

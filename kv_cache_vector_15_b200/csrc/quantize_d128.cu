@@ -639,29 +639,56 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
 #pragma unroll
     for (int w = 0; w < B * 2; ++w) cw[w] = 0u;
     float2 r2 = make_float2(0.f, 0.f);
+    // 2-bit codes: bit 1 = [y > t1], bit 0 = [y > (bit 1 ? t2 : t0)], each the
+    // sign of an exact difference (t - y < 0 iff y > t; t - t = +0), funnel-
+    // shifted into the packed word from the word's last code down
+    float cc[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (B == 2) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) cc[k] = tab[k];
+    }
 #pragma unroll
     for (int ch = 0; ch < 2; ++ch) {
       uint32_t hw[16], lw[16];
+      float rb[32];
+      if constexpr (B == 2) {
+#pragma unroll
+        for (int e = ch * 32 + 31; e >= ch * 32; --e) {
+          const float y = __uint_as_float(u[e]);
+          const float d1 = tq[1] - y;
+          const bool b1 = d1 < 0.f;
+          const float d0 = (b1 ? tq[2] : tq[0]) - y;
+          const bool b0 = d0 < 0.f;
+          cw[e >> 4] = __funnelshift_l(__float_as_uint(d1), cw[e >> 4], 1);
+          cw[e >> 4] = __funnelshift_l(__float_as_uint(d0), cw[e >> 4], 1);
+          const float c = b1 ? (b0 ? cc[3] : cc[2]) : (b0 ? cc[1] : cc[0]);
+          rb[e - ch * 32] = fmaf(y, sc64, -c);
+        }
+      }
 #pragma unroll
       for (int e = ch * 32; e < ch * 32 + 32; e += 2) {
         float rr[2];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          const float y = __uint_as_float(u[e + q]);
-          uint32_t code = 0u;
+          if constexpr (B == 2) {
+            rr[q] = rb[e + q - ch * 32];
+          } else {
+            const float y = __uint_as_float(u[e + q]);
+            uint32_t code = 0u;
 #pragma unroll
-          for (int lev = B - 1; lev >= 0; --lev) {
-            const int base = (1 << lev) - 1;
-            float thr = tq[base];
+            for (int lev = B - 1; lev >= 0; --lev) {
+              const int base = (1 << lev) - 1;
+              float thr = tq[base];
 #pragma unroll
-            for (int k = 1; k < (1 << (B - 1 - lev)); ++k)
-              if (code == static_cast<uint32_t>(k << (lev + 1))) thr = tq[base + (k << (lev + 1))];
-            if (y > thr) code |= (1u << lev);
+              for (int k = 1; k < (1 << (B - 1 - lev)); ++k)
+                if (code == static_cast<uint32_t>(k << (lev + 1))) thr = tq[base + (k << (lev + 1))];
+              if (y > thr) code |= (1u << lev);
+            }
+            rr[q] = fmaf(y, sc64, -tab[code]);
+            const int bit = B * (e + q), wi = bit >> 5, sh = bit & 31;
+            cw[wi] |= code << sh;
+            if (sh + B > 32) cw[wi + 1] |= code >> (32 - sh);
           }
-          rr[q] = fmaf(y, sc64, -tab[code]);
-          const int bit = B * (e + q), wi = bit >> 5, sh = bit & 31;
-          cw[wi] |= code << sh;
-          if (sh + B > 32) cw[wi + 1] |= code >> (32 - sh);
         }
         const float2 rv = make_float2(rr[0], rr[1]);
         r2 = __ffma2_rn(rv, rv, r2);
