@@ -7,8 +7,13 @@
 //
 // Both inner products are linear in the stored bits.  For 1- and 2-bit
 // symmetric Lloyd-Max codebooks the centroid is affine in the code bits,
-//   B = 2: c[code] = -c3 + (c3 - c2) b0 + (c3 + c2) b1,   B = 1: c = -c1 + 2 c1 b0,
-// and z_j = 1 - 2 bit_j, so for each key
+//   B = 2: c[code] = -c3 + (c3 - c2) b0 + (c3 + c2) b1,   B = 1: c = -c1 + 2 c1 b0.
+// A symmetric 3-bit codebook is an odd function of x_i = 2 b_i - 1 (the
+// mirror code complements every bit), so it is a0 x0 + a1 x1 + a2 x2 +
+// a3 x0 x1 x2 exactly, and x0 x1 x2 = 2 p - 1 with p = b0 ^ b1 ^ b2:
+//   B = 3: c[code] = sum_i 2 a_i b_i + 2 a3 p - (a0 + a1 + a2 + a3),
+// one more bit plane (the per-code parity) next to the three code planes.
+// z_j = 1 - 2 bit_j, so for each key
 //   <q_rot, yhat> = const_q + sum_(bits) weight(bit) q_rot[coord(bit)] * bit
 //   <sq, z>       = sum_j sq_j - 2 sum_j sq_j bit_j.
 // Each key's bits become an unsigned 8-bit row of 0/1 values in TMEM (two
@@ -18,13 +23,17 @@
 // 8-bit limbs of a fixed-point value per (bit, query).  The epilogue recombines
 // the limbs, adds the constants and applies norm and rnorm.
 //
-// Work split: persistent CTAs of four warpgroups; each warpgroup walks a
-// contiguous range of 128-key tiles (so the set, and with it the query operand
-// it builds in its own shared-memory slot, changes rarely), one thread per key.
+// Work split: persistent CTAs of four warpgroups (two for 3-bit codes, whose
+// wider operand takes 160 of a warpgroup's TMEM columns); each warpgroup walks
+// a contiguous range of 128-key tiles (so the set, and with it the query
+// operand it builds in its own shared-memory slot, changes rarely), one thread
+// per key.
 
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <cmath>
 #include <cstdint>
 
 #include "sm100.cuh"
@@ -36,9 +45,9 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kD = 128, kM = 128, kTile = 128, kWG = 4, kThreads = kWG * 128;
+constexpr int kD = 128, kM = 128, kTile = 128;
 constexpr long long kWaitCycles = 2000000000ll;
-constexpr uint32_t kTmemCols = 512;          // per warpgroup: 96 A columns + 32 D columns (in 128)
+constexpr uint32_t kTmemCols = 512;          // split evenly between the warpgroups (A columns, then D)
 
 __host__ __device__ constexpr uint32_t idesc_i8(uint32_t M, uint32_t N) {
   return (2u << 4)              // D format: S32
@@ -60,8 +69,12 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
 template <int B>
 struct Shape {
   static constexpr int kCodeWords = B * 4;                  // 32-bit words of codes per key
+  static constexpr int kParWords = B == 3 ? 4 : 0;          // per-code parity bits (3-bit codes)
   static constexpr int kCodeBytes = B * 16;
-  static constexpr int kAWords = 8 * (kCodeWords + 4);      // 0/1 bytes, four per TMEM column
+  static constexpr int kWG = B == 3 ? 2 : 4;                // warpgroups per CTA
+  static constexpr int kThreads = kWG * 128;
+  static constexpr uint32_t kColsPerWG = kTmemCols / kWG;
+  static constexpr int kAWords = 8 * (kCodeWords + kParWords + 4);   // 0/1 bytes, four per TMEM column
   static constexpr int kK = 4 * kAWords;                    // K of the MMA (bytes)
   static constexpr int kKBlocks = kK / 128;                 // 128-byte swizzle atoms along K
   static constexpr int kKSteps = kK / 32;
@@ -71,16 +84,37 @@ struct Shape {
 constexpr int kStages = 4;                   // packed tiles in flight per warpgroup
 
 struct LogitsArgs {
-  float wbit[2];                  // weight of code bit 0 / 1 in the centroid
+  float wbit[3];                  // weight of code bit 0 / 1 / 2 in the centroid
+  float wpar;                     // weight of the code's parity bit (3-bit codes)
   float cconst;                   // centroid constant term
   int* err;
 };
 
+// Every third bit of x (bits 0, 3, ..., 30) packed into bits 0..10.
+__device__ __forceinline__ uint32_t every_third_bit(uint32_t x) {
+  x &= 0x49249249u;
+  x = (x | (x >> 2)) & 0xC30C30C3u;
+  x = (x | (x >> 4)) & 0x0F00F00Fu;
+  x = (x | (x >> 8)) & 0xFF0000FFu;
+  x = (x | (x >> 16)) & 0x0000FFFFu;
+  return x;
+}
+
+// Parity of each of the 32 3-bit codes held in three consecutive stream words
+// (code i in bits 3i .. 3i + 2 of w0 | w1 << 32 | w2 << 64), bit i of the result.
+__device__ __forceinline__ uint32_t code_parities(uint32_t w0, uint32_t w1, uint32_t w2) {
+  const uint32_t x0 = w0 ^ __funnelshift_r(w0, w1, 1) ^ __funnelshift_r(w0, w1, 2);
+  const uint32_t x1 = w1 ^ __funnelshift_r(w1, w2, 1) ^ __funnelshift_r(w1, w2, 2);
+  const uint32_t x2 = w2 ^ (w2 >> 1) ^ (w2 >> 2);
+  return every_third_bit(x0) | (every_third_bit(x1 >> 1) << 11) | ((every_third_bit(x2 >> 2) & 0x3FFu) << 22);
+}
+
 template <int B, int G, int NG>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Shape<B>::kThreads, 1)
 k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ qp, int64_t n_sets,
                  int64_t n_keys, const Packed keys, float* __restrict__ out) {
   using S = Shape<B>;
+  constexpr int kWG = S::kWG;
   constexpr int N = 2 * NG;
   constexpr int kBBytes = S::kKBlocks * N * 128;            // query operand per warpgroup
   extern __shared__ uint8_t smem_raw[];
@@ -112,7 +146,7 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
   const uint32_t tmem = *tmem_slot;
   const bool leader = (wl == 0 && lane == 0);
   const int trow = wl * 32 + lane;
-  const uint32_t t_base = tmem + (static_cast<uint32_t>(wl * 32) << 16) + wg * 128;   // this thread's lane
+  const uint32_t t_base = tmem + (static_cast<uint32_t>(wl * 32) << 16) + wg * S::kColsPerWG;   // my lane
   const uint32_t t_a = t_base, t_d = t_base + S::kAWords;
 
   // contiguous tile range of this warpgroup; (set, key tile) advance incrementally
@@ -188,7 +222,9 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
       named_bar_sync(1 + wg, 128);
       // fixed-point scales: |value| * 2^F <= 2^22
       float scale[2 * G];
-      const float wmax = fmaxf(fabsf(X.wbit[0]), B == 2 ? fabsf(X.wbit[1]) : 0.f);
+      float wmax = fabsf(X.wbit[0]);
+      if (B >= 2) wmax = fmaxf(wmax, fabsf(X.wbit[1]));
+      if (B == 3) wmax = fmaxf(wmax, fmaxf(fabsf(X.wbit[2]), fabsf(X.wpar)));
 #pragma unroll
       for (int q = 0; q < G; ++q) {
         const float vm = sMax[q] * wmax, vq = sMax[G + q] * 2.f;
@@ -206,11 +242,19 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
         int8_t limb[N];
 #pragma unroll
         for (int n = 0; n < N; ++n) limb[n] = 0;
-        if (o < 8 * S::kCodeWords) {
-          const int c = o >> 3, k = o & 7;
-          const int s = 32 * c + k + 8 * tb;          // bit position in the code stream
-          const int coord = s / B, plane = s % B;
-          const float w = X.wbit[plane];
+        if (o < 8 * (S::kCodeWords + S::kParWords)) {
+          int coord;
+          float w;
+          if (o < 8 * S::kCodeWords) {
+            const int c = o >> 3, k = o & 7;
+            const int s = 32 * c + k + 8 * tb;        // bit position in the code stream
+            coord = s / B;
+            w = X.wbit[s % B];
+          } else {
+            const int c = (o - 8 * S::kCodeWords) >> 3, k = o & 7;
+            coord = 32 * c + k + 8 * tb;              // parity bit of this code
+            w = X.wpar;
+          }
 #pragma unroll
           for (int q = 0; q < G; ++q) {
             const int v = __float2int_rn(w * qs[q * (kD + kM) + coord] * scale[q]);
@@ -223,7 +267,7 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
             limb[3 * q + 2] = static_cast<int8_t>(l2);
           }
         } else {
-          const int c = (o - 8 * S::kCodeWords) >> 3, k = o & 7;
+          const int c = (o - 8 * (S::kCodeWords + S::kParWords)) >> 3, k = o & 7;
           const int j = 32 * c + k + 8 * tb;           // projection
 #pragma unroll
           for (int q = 0; q < G; ++q) {
@@ -263,7 +307,7 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
       atomicExch(abort_flag, 1);
     }
     {
-      uint32_t cw[S::kCodeWords + 4];
+      uint32_t cw[S::kCodeWords + S::kParWords + 4];
       const uint8_t* st = stages + stage * S::kStageBytes;
       if (valid) {
 #pragma unroll
@@ -272,16 +316,21 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
           cw[4 * q] = u.x; cw[4 * q + 1] = u.y; cw[4 * q + 2] = u.z; cw[4 * q + 3] = u.w;
         }
         const uint4 u = *reinterpret_cast<const uint4*>(st + kTile * S::kCodeBytes + trow * 16);
-        cw[S::kCodeWords] = u.x; cw[S::kCodeWords + 1] = u.y;
-        cw[S::kCodeWords + 2] = u.z; cw[S::kCodeWords + 3] = u.w;
+        constexpr int so = S::kCodeWords + S::kParWords;
+        cw[so] = u.x; cw[so + 1] = u.y; cw[so + 2] = u.z; cw[so + 3] = u.w;
+        if constexpr (B == 3) {
+#pragma unroll
+          for (int g2 = 0; g2 < 4; ++g2)
+            cw[S::kCodeWords + g2] = code_parities(cw[3 * g2], cw[3 * g2 + 1], cw[3 * g2 + 2]);
+        }
       } else {
 #pragma unroll
-        for (int w = 0; w < S::kCodeWords + 4; ++w) cw[w] = 0u;
+        for (int w = 0; w < S::kCodeWords + S::kParWords + 4; ++w) cw[w] = 0u;
       }
       uint32_t a[32];
       int n = 0, col = 0;
 #pragma unroll
-      for (int c = 0; c < S::kCodeWords + 4; ++c) {
+      for (int c = 0; c < S::kCodeWords + S::kParWords + 4; ++c) {
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           a[n++] = (cw[c] >> k) & 0x01010101u;
@@ -302,11 +351,11 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
       tc_fence_after();
       const uint32_t sbase = smem_u32(sB);
       const uint32_t idesc = idesc_i8(kTile, N);
-      const uint32_t d_tmem = tmem + wg * 128 + S::kAWords;
+      const uint32_t d_tmem = tmem + wg * S::kColsPerWG + S::kAWords;
 #pragma unroll
       for (int k = 0; k < S::kKSteps; ++k) {
         const uint64_t bdesc = smem_desc_sw128(sbase + (k >> 2) * (N * 128) + (k & 3) * 32, 1024);
-        mma_i8_ts(d_tmem, tmem + wg * 128 + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
+        mma_i8_ts(d_tmem, tmem + wg * S::kColsPerWG + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
       }
       mma_commit(&mdone[wg]);
     }
@@ -358,14 +407,47 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
   }
 }
 
+// The 3-bit codebook as an odd function of x_i = 2 b_i - 1: coefficients of
+// x0, x1, x2 and x0 x1 x2 (a Walsh transform of the eight centroids), and the
+// largest deviation of that fit from the centroids (zero for a symmetric book).
+double odd_fit3(const float* c, double a[4]) {
+  for (int i = 0; i < 4; ++i) a[i] = 0.0;
+  for (int k = 0; k < 8; ++k) {
+    const double x0 = 2.0 * (k & 1) - 1.0, x1 = 2.0 * ((k >> 1) & 1) - 1.0, x2 = 2.0 * ((k >> 2) & 1) - 1.0;
+    a[0] += c[k] * x0 / 8.0;
+    a[1] += c[k] * x1 / 8.0;
+    a[2] += c[k] * x2 / 8.0;
+    a[3] += c[k] * x0 * x1 * x2 / 8.0;
+  }
+  double worst = 0.0, cmax = 0.0;
+  for (int k = 0; k < 8; ++k) {
+    const double x0 = 2.0 * (k & 1) - 1.0, x1 = 2.0 * ((k >> 1) & 1) - 1.0, x2 = 2.0 * ((k >> 2) & 1) - 1.0;
+    const double f = a[0] * x0 + a[1] * x1 + a[2] * x2 + a[3] * x0 * x1 * x2;
+    worst = std::max(worst, std::fabs(f - c[k]));
+    cmax = std::max(cmax, std::fabs(static_cast<double>(c[k])));
+  }
+  return cmax > 0.0 ? worst / cmax : worst;
+}
+
 template <int B, int G>
 int launch_G(const tq_ctx& ctx, const float* qp, int64_t n_sets, int64_t n_keys, const Packed& keys, float* out,
              cudaStream_t s) {
   constexpr int NG = (3 * G <= 16) ? 16 : 32;
   using Sh = Shape<B>;
+  constexpr int kWG = Sh::kWG;
   const KParams& P = ctx.kp;
   LogitsArgs X;
-  if (B == 2) {
+  X.wbit[2] = 0.f;
+  X.wpar = 0.f;
+  if (B == 3) {
+    double a[4];
+    odd_fit3(P.c, a);
+    X.wbit[0] = static_cast<float>(2.0 * a[0]);
+    X.wbit[1] = static_cast<float>(2.0 * a[1]);
+    X.wbit[2] = static_cast<float>(2.0 * a[2]);
+    X.wpar = static_cast<float>(2.0 * a[3]);
+    X.cconst = static_cast<float>(-(a[0] + a[1] + a[2] + a[3]));
+  } else if (B == 2) {
     X.wbit[0] = P.c[3] - P.c[2];
     X.wbit[1] = P.c[3] + P.c[2];
     X.cconst = -P.c[3];
@@ -383,7 +465,7 @@ int launch_G(const tq_ctx& ctx, const float* qp, int64_t n_sets, int64_t n_keys,
   const int64_t n_tiles = ((n_keys + kTile - 1) / kTile) * n_sets;
   int64_t grid = (n_tiles + kWG - 1) / kWG;
   if (grid > ctx.num_sms) grid = ctx.num_sms;
-  k_logits_d128_i8<B, G, NG><<<static_cast<int>(grid), kThreads, smem, s>>>(P, X, qp, n_sets, n_keys, keys, out);
+  k_logits_d128_i8<B, G, NG><<<static_cast<int>(grid), Sh::kThreads, smem, s>>>(P, X, qp, n_sets, n_keys, keys, out);
   count_launch();
   return static_cast<int>(cudaGetLastError());
 }
@@ -407,17 +489,26 @@ int launch_B(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, int64_t 
 
 bool logits_d128_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys) {
   const KParams& P = ctx.kp;
-  // the A operand and the accumulator share a 128-column TMEM slice per warpgroup
-  const int a_cols = 8 * (P.B * 4 + 4), n_cols = (3 * g <= 16) ? 32 : 64;
-  return P.d == kD && P.m == kM && (P.B == 1 || P.B == 2) && g >= 1 && g <= 8 && a_cols + n_cols <= 128 &&
-         n_keys > 0 && n_sets > 0 && ctx.use_tc;
+  if (!(P.d == kD && P.m == kM && P.B >= 1 && P.B <= 3 && g >= 1 && g <= 8 && n_keys > 0 && n_sets > 0 &&
+        ctx.use_tc))
+    return false;
+  // the A operand and the accumulator share a warpgroup's TMEM columns
+  const int a_cols = 8 * (P.B * 4 + (P.B == 3 ? 4 : 0) + 4), n_cols = (3 * g <= 16) ? 32 : 64;
+  const int cols = P.B == 3 ? 256 : 128;
+  if (a_cols + n_cols > cols) return false;
+  if (P.B == 3) {                       // the bit-plane form needs a symmetric codebook
+    double a[4];
+    if (odd_fit3(P.c, a) > 1e-6) return false;
+  }
+  return true;
 }
 
 int launch_logits_d128(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
                        float* out, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (ctx.kp.B == 1) return launch_B<1>(ctx, qp, n_sets, g, n_keys, keys, out, s);
-  return launch_B<2>(ctx, qp, n_sets, g, n_keys, keys, out, s);
+  if (ctx.kp.B == 2) return launch_B<2>(ctx, qp, n_sets, g, n_keys, keys, out, s);
+  return launch_B<3>(ctx, qp, n_sets, g, n_keys, keys, out, s);
 }
 
 }  // namespace tq

@@ -139,7 +139,7 @@ def test_logits_parity_on_oracle_packed_keys(tq, d, b, m, n_sets, g, n_keys, qdt
     assert np.all(err <= tol + 1e-30), float(np.max(err / (tol + 1e-30)))
 
 
-@pytest.mark.parametrize("b,g", [(3, 4), (2, 8), (3, 5), (3, 1)])
+@pytest.mark.parametrize("b,g", [(3, 4), (2, 8), (3, 5), (3, 1), (4, 4), (4, 8), (4, 1)])
 @pytest.mark.parametrize("kernels", ["auto", "generic"])
 def test_logits_d128_many_tiles_and_sets(tq, b, g, kernels):
     """Several 128-key tiles per warpgroup, sets changing inside a warpgroup's
