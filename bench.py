@@ -44,6 +44,15 @@ WORKLOADS = {
     # a 1M-row case (268 MB per tensor, above L2) for profiler captures
     "decode-2x64k-b3": dict(batch=2, ctx=65536, b=3, m=128, kv_heads=8, q_heads=32, d=128),
 }
+# secondary workloads, each with its own metric (not the headline line)
+AUX_WORKLOADS = {
+    # prefill write path: quantize K and V of 32 layers x 8 heads x 32768 tokens
+    "prefill-b2": dict(kind="prefill", b=2, m=128, d=128),
+    "prefill-b3": dict(kind="prefill", b=3, m=128, d=128),
+    "prefill-b4": dict(kind="prefill", b=4, m=128, d=128),
+    # vector search: 1e6 x 1024 fp32 database, 1024 queries, b = 4, m = 1024, top-10
+    "vsearch": dict(kind="vsearch", b=4, m=1024, d=1024),
+}
 METRIC = "compressed-key logits/s and % HBM roofline (d=128,b=3); quantize rows/s"
 UNIT = "logits/s"
 
@@ -331,23 +340,58 @@ def run_ours(args, cfg, ws, rank, local):
     bf16_ms = e0.elapsed_time(e1) / reps
     bf16_bytes = N * (2 * d + 4 * g)
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: every step uploads K,
+    # V and q from pinned host memory and downloads the logits and V-hat,
+    # pipelined over this rank's sequences -- sequence i+1 uploads on one copy
+    # stream and sequence i-1's results download on another while sequence i
+    # is computed (PCIe is full duplex)
     hL = torch.empty((n_sets, g, n_keys), dtype=torch.float32, pin_memory=True)
     hVh = torch.empty((N, d), dtype=torch.bfloat16, pin_memory=True)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    nseq = sh.batch
+    kv_per, q_per, sets_per = cfg["kv_heads"] * n_keys, cfg["q_heads"], cfg["kv_heads"]
+    computed = [None] * nseq          # per sequence: its compute finished (inputs free)
+    downloaded = [None] * nseq        # per sequence: its results are on the host (outputs free)
 
     def e2e_step():
-        dK.copy_(hK, non_blocking=True)
-        dV.copy_(hV, non_blocking=True)
-        dQ.copy_(hQ, non_blocking=True)
-        step()
-        hL.copy_(logits, non_blocking=True)
-        hVh.copy_(vhat, non_blocking=True)
+        for i in range(nseq):
+            r0, r1 = i * kv_per, (i + 1) * kv_per
+            q0, q1 = i * q_per, (i + 1) * q_per
+            s0, s1 = i * sets_per, (i + 1) * sets_per
+            if computed[i] is not None:
+                s_in.wait_event(computed[i])
+            with torch.cuda.stream(s_in):
+                dK[r0:r1].copy_(hK[r0:r1], non_blocking=True)
+                dV[r0:r1].copy_(hV[r0:r1], non_blocking=True)
+                dQ[q0:q1].copy_(hQ[q0:q1], non_blocking=True)
+            up = torch.cuda.Event()
+            up.record(s_in)
+            stream.wait_event(up)
+            if downloaded[i] is not None:
+                stream.wait_event(downloaded[i])
+            pk, pv = pK.rows(r0, r1), pV.rows(r0, r1)
+            T.quantize(dK[r0:r1], pk, stream=stream)
+            T.quantize(dV[r0:r1], pv, stream=stream)
+            T.logits(dQ[q0:q1], pk, sets_per, g, n_keys, out=logits[s0:s1], workspace=work, stream=stream)
+            T.dequant(pv, kv_per, out=vhat[r0:r1], stream=stream)
+            done = torch.cuda.Event()
+            done.record(stream)
+            computed[i] = done
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                hL[s0:s1].copy_(logits[s0:s1], non_blocking=True)
+                hVh[r0:r1].copy_(vhat[r0:r1], non_blocking=True)
+            dn = torch.cuda.Event()
+            dn.record(s_out)
+            downloaded[i] = dn
+        stream.wait_stream(s_out)
 
     e2e_steps = max(1, min(args.steps, 5))
     e2e_step()
     torch.cuda.synchronize(dev)
     barrier(ws)
     e0.record(stream)
+    s_in.wait_stream(stream)          # no upload starts before the timed region
     for _ in range(e2e_steps):
         e2e_step()
     e1.record(stream)
@@ -394,17 +438,109 @@ def run_ours(args, cfg, ws, rank, local):
     return line
 
 
+# ---------------------------------------------------------------------------
+# Secondary workloads (prefill write path, vector search): CUDA path only
+# ---------------------------------------------------------------------------
+def run_aux(args, cfg, ws, rank, local):
+    import torch
+    from kv_cache_vector_15_b200 import tq
+
+    d, b, m = cfg["d"], cfg["b"], cfg["m"]
+    dev = torch.device("cuda", local)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    stream = torch.cuda.current_stream(dev)
+    hbm, hbm_kind = peaks()
+    P = T.row_bytes
+    if cfg["kind"] == "prefill":
+        K, V = inputs.prefill()
+        N = K.n_rows
+        lo, hi = dist_util.shard(N, ws, rank)          # each rank quantizes its slice of the rows
+        n = hi - lo
+        hK = torch.empty((n, d), dtype=torch.bfloat16)
+        hV = torch.empty((n, d), dtype=torch.bfloat16)
+        K.fill(hK.view(torch.int16).numpy().view(np.uint16), start=lo)
+        V.fill(hV.view(torch.int16).numpy().view(np.uint16), start=lo)
+        dK, dV = hK.to(dev), hV.to(dev)
+        del hK, hV
+        pK, pV = T.empty_packed(n, dev), T.empty_packed(n, dev)
+
+        def step():
+            T.quantize(dK, pK, stream=stream)
+            T.quantize(dV, pV, stream=stream)
+        units, unit, metric = 2 * n, "rows/s", f"tq_quantize rows/s, prefill write path (b={b})"
+        alg = 2 * n * (2 * d + P)
+        kern = "quantize"
+    else:
+        db, qs = inputs.vector_search()
+        nq, ndb = qs.n_rows, db.n_rows
+        hdb = torch.empty((ndb, d), dtype=torch.float32)
+        db.fill(hdb.numpy())
+        ddb = hdb.to(dev)
+        del hdb
+        dq = torch.from_numpy(qs.all()).to(dev)
+        pk = T.empty_packed(ndb, dev)
+        scores = torch.empty((1, nq, ndb), dtype=torch.float32, device=dev)
+        work = torch.empty(max(T.workspace_bytes(1, nq), 16), dtype=torch.uint8, device=dev)
+
+        def step():
+            T.quantize(ddb, pk, stream=stream)
+            T.logits(dq, pk, 1, nq, ndb, out=scores, workspace=work, stream=stream)
+            tq.topk(scores[0], 10, stream=stream)
+        units, unit, metric = nq * ndb, "IP estimates/s", "vector search: quantize DB, all-pairs IP estimates, top-10"
+        alg = ndb * (4 * d + P) + ndb * P + 2 * nq * ndb * 4
+        kern = "step"
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(ws)
+    launches0 = tq.launch_count()
+    with ClockSampler(local) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(ws)
+    ms = max_over_ranks(ws, e0.elapsed_time(e1)) / args.steps
+    total = dist_util.sum_over_ranks(ws, units, device=dev)
+    if rank == 0:
+        gbs = alg / (ms * 1e-3) / 1e9
+        print(json.dumps({
+            "metric": metric, "value": total / (ms * 1e-3), "unit": unit, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": args.workload, "d": d, "b": b, "m": m, "l2": "inputs larger than L2; no flush"},
+            "roofline": {"bound": "hbm", "kernel": kern, "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm, "traffic": None, "algorithmic_bytes": alg, "peak_kind": hbm_kind},
+            "gpu_launches": tq.launch_count() - launches0, "clocks": clk.summary()}), flush=True)
+    T.close()
+
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="decode-128k-b3", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="decode-128k-b3", choices=sorted(WORKLOADS) + sorted(AUX_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload in AUX_WORKLOADS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the headline workload only"}))
+            return
+        ws, rank, local = dist_setup()
+        try:
+            run_aux(args, AUX_WORKLOADS[args.workload], ws, rank, local)
+        finally:
+            if ws > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
     cfg = WORKLOADS[args.workload]
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))

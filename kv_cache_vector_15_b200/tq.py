@@ -131,6 +131,10 @@ class Packed:
     def nbytes(self) -> int:
         return sum(int(t.numel() * t.element_size()) for t in (self.codes, self.signs, self.norm, self.rnorm))
 
+    def rows(self, start: int, stop: int) -> "Packed":
+        """Rows [start, stop) as views of the same storage."""
+        return Packed(self.codes[start:stop], self.signs[start:stop], self.norm[start:stop], self.rnorm[start:stop])
+
     def to_numpy(self) -> dict:
         return {k: getattr(self, k).cpu().numpy() for k in ("codes", "signs", "norm", "rnorm")}
 
