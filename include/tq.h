@@ -57,7 +57,7 @@ extern "C" {
 typedef enum {
   TQ_OK = 0,
   TQ_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or enum */
-  TQ_ERR_UNSUPPORTED = 2,  /* valid request outside what this build implements */
+  TQ_ERR_UNSUPPORTED = 2,  /* valid request outside what this library implements */
   TQ_ERR_NOMEM = 3,        /* device or host allocation failed (tq_init only) */
   TQ_ERR_CUDA = 4          /* a CUDA runtime call or launch failed; see tq_last_error() */
 } tq_status;

@@ -18,7 +18,7 @@ Everything here is written for a reader to check by eye against the pages:
 
 Parity status per function is stated in each docstring; the pins live in
 ``tests/test_oracle_*.py``.  Nothing here is "parity unpinned" except the
-exact values of D and S, which are this build's choice of generator and are
+exact values of D and S, which depend on the chosen generator and are
 pinned only by their published generator definitions (SplitMix64, Box-Muller)
 and by their statistics.
 """

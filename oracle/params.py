@@ -15,7 +15,7 @@ Three things are drawn or fitted once per ``(d, b, m, seed)``:
   壓縮 6 倍", section "隨機旋轉與Beta分佈" (each rotated coordinate follows a
   concentrated Beta law and one scalar quantizer serves all coordinates)].
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * Random numbers come from SplitMix64 (Steele, Lea & Flood 2014; Vigna's
   public-domain definition) used counter-style: output(seed, stream, i) is the

@@ -21,9 +21,10 @@ Read half:
   dequant (PROD) x~ = R^T (norm * yhat + sqrt(pi/2)/m * rnorm * S^T z)
   [ai.spot.hk, "無偏內積估計": E<y, Q^-1(Q(x))> = <y, x>];
   dequant (MSE)  x~ = norm * R^T yhat  [Qiita explainer, "APIの構成"
-  (values compressed by the MSE stage alone)].
+  (values compressed by the MSE stage alone)];
+  attention: softmax over keys of scale * logit, times the dequantized values.
 
-Readings (each listed in the design doc):
+Readings taken where the pages are silent:
   * the residual lives in the rotated, unit-normalised domain, and rnorm is
     stored in the original units (n * rho);
   * y_i exactly on a threshold goes to the lower cell; p_j = 0 counts as
@@ -226,6 +227,29 @@ def dequant(packed: dict, P, mode: int = DEQUANT_PROD) -> np.ndarray:
     if mode == DEQUANT_PROD:
         v = v + (SQRT_HALF_PI / P.m) * rnorm[:, None] * (z @ P.S)
     return rotate_inverse(v, P)
+
+
+def attention(q: np.ndarray, keys: dict, values: dict, P, n_sets: int, g: int, n_keys: int, scale: float,
+              mode: int = DEQUANT_PROD, logits_in=None) -> np.ndarray:
+    """Decode attention read from packed keys and values: for query j of set s,
+    softmax over the set's keys of scale * logit, times the dequantized values
+    of the same keys.  [Qiita explainer, "APIの構成": attention scores taken
+    from the compressed keys (asymmetric_attention_scores) and values kept in
+    compressed form; the weighted sum of values is ordinary attention.]
+
+    logits_in: (n_sets, g, n_keys) logits to use instead of the estimator's
+    own (so a caller can evaluate the softmax and the value sum on given
+    scores).  Returns (n_sets, g, d) fp64."""
+    s = logits(q, keys, P, n_sets, g, n_keys) if logits_in is None else np.asarray(logits_in, dtype=np.float64)
+    z = scale * s.reshape(n_sets, g, n_keys)
+    z = z - z.max(axis=-1, keepdims=True)
+    w = np.exp(z)
+    w /= w.sum(axis=-1, keepdims=True)
+    xv = dequant(values, P, mode).reshape(n_sets, n_keys, P.d)
+    out = np.empty((n_sets, g, P.d))
+    for st in range(n_sets):
+        out[st] = w[st] @ xv[st]
+    return out
 
 
 def topk(scores: np.ndarray, k: int):

@@ -274,3 +274,57 @@ def test_topk_brute_force_with_ties():
         want = sorted(range(s.shape[1]), key=lambda j: (-s[r, j], j))[:10]
         assert list(idx[r]) == want
         assert np.array_equal(val[r], s[r, want])
+
+
+# ---------------------------------------------------------------------------
+# attention from packed keys and values: pinned by what softmax-weighted
+# averaging must do, independent of the formula's own arithmetic
+# ---------------------------------------------------------------------------
+def _packed_pair(d=32, b=3, m=32, n=7, seed=3):
+    P = op.Params(d, b, m, seed=0)
+    rng = np.random.default_rng(seed)
+    k = rng.standard_normal((n, d)) * 2.0
+    v = rng.standard_normal((n, d))
+    return P, ot.quantize(k, P), ot.quantize(v, P), rng
+
+
+def test_attention_single_key_returns_that_value():
+    P, pk, pv, rng = _packed_pair(n=1)
+    q = rng.standard_normal((3, P.d))
+    out = ot.attention(q, pk, pv, P, 1, 3, 1, scale=0.7)
+    xv = ot.dequant(pv, P)
+    assert np.allclose(out[0], np.repeat(xv, 3, axis=0), rtol=0, atol=1e-12)
+
+
+def test_attention_equal_scores_average_the_values():
+    P, pk, pv, rng = _packed_pair(n=9)
+    q = rng.standard_normal((2, P.d))
+    out = ot.attention(q, pk, pv, P, 1, 2, 9, scale=1.0, logits_in=np.zeros((1, 2, 9)))
+    for mode in (ot.DEQUANT_PROD, ot.DEQUANT_MSE):
+        o = ot.attention(q, pk, pv, P, 1, 2, 9, scale=1.0, mode=mode, logits_in=np.full((1, 2, 9), 3.5))
+        assert np.allclose(o[0], ot.dequant(pv, P, mode).mean(axis=0)[None, :], atol=1e-12)
+    assert np.allclose(out[0][0], out[0][1])
+
+
+def test_attention_large_scale_selects_the_top_key():
+    P, pk, pv, rng = _packed_pair(n=6)
+    s = np.array([[[0.1, 2.0, -1.0, 1.9, 0.0, 0.5]]])
+    o = ot.attention(rng.standard_normal((1, P.d)), pk, pv, P, 1, 1, 6, scale=1e4, logits_in=s)
+    assert np.allclose(o[0, 0], ot.dequant(pv, P)[1], atol=1e-9)
+
+
+def test_attention_is_invariant_to_key_order_and_weights_sum_to_one():
+    P, pk, pv, rng = _packed_pair(n=8)
+    q = rng.standard_normal((1, P.d))
+    perm = rng.permutation(8)
+    pk2 = {k: v[perm] for k, v in pk.items()}
+    pv2 = {k: v[perm] for k, v in pv.items()}
+    a = ot.attention(q, pk, pv, P, 1, 1, 8, scale=0.3)
+    b = ot.attention(q, pk2, pv2, P, 1, 1, 8, scale=0.3)
+    assert np.allclose(a, b, atol=1e-12)
+    # against softmax weights built by hand from the estimator's logits
+    s = ot.logits(q, pk, P, 1, 1, 8)[0, 0]
+    w = np.exp(0.3 * (s - s.max()))
+    w /= w.sum()
+    assert abs(w.sum() - 1.0) < 1e-15
+    assert np.allclose(a[0, 0], w @ ot.dequant(pv, P), atol=1e-12)
