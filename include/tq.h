@@ -154,6 +154,30 @@ tq_status tq_logits(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t 
 tq_status tq_logits_noalloc(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
                             tq_packed keys, int64_t n_keys, float* out, void* stream);
 
+/* Device workspace that tq_attention needs (bytes; 0 for an empty call):
+ * query operands, the logits and per-chunk partial sums. */
+size_t tq_attention_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g, int64_t n_keys);
+
+/* Decode attention read from packed keys and values (Qiita TurboQuant
+ * explainer, "APIの構成": attention scores from the compressed keys, values
+ * kept compressed):
+ *   out[s*g + j] = sum_k softmax_k(scale * logit(q_{s,j}, key_{s,k})) * dequant(value_{s,k})
+ * with the logit estimator of tq_logits and dequant in `mode` (PROD or MSE).
+ * The weighted sum is formed in the rotated domain and rotated back once per
+ * query; no value row is reconstructed in memory.
+ * q [n_sets * g, d] bf16/fp32 (16-byte aligned); keys and values: rows of set
+ * s at [s * n_keys, (s + 1) * n_keys) of each packed array (caller-owned
+ * device pointers, as for tq_logits); out [n_sets * g, d] fp32; scale is the
+ * softmax scale (1/sqrt(d) for the usual attention), finite; g in [1, 8];
+ * d + m <= 2048; n_keys >= 1 when n_sets > 0.  workspace: device buffer of at
+ * least tq_attention_workspace_bytes(ctx, n_sets, g, n_keys) bytes, 16-byte
+ * aligned, used only by this call's kernels on `stream`.  Arguments are checked
+ * before any launch (TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED, nothing
+ * launched).  Launches qprep, logits and two attention kernels on `stream`. */
+tq_status tq_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
+                       tq_packed keys, tq_packed values, int64_t n_keys, float scale, tq_dequant_mode mode,
+                       float* out, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Reconstruct n_rows packed rows into out [n_rows, d] (bf16 or fp32,
  * contiguous, 16-byte aligned).  mode PROD adds the QJL term (unbiased),
  * MSE uses the codes alone. */

@@ -1,0 +1,292 @@
+// Decode attention straight from packed keys and values.
+//
+//   out[s][j] = sum_k softmax_k(scale * logit(q_sj, k_sk)) * dequant(v_sk)
+//
+// Attention scores come from the compressed keys (the logit estimator,
+// tq_logits) and the values stay compressed: Qiita TurboQuant explainer,
+// "APIの構成" (asymmetric_attention_scores on compressed keys, values kept by
+// the MSE compressor).  Because dequantization is linear in what a packed row
+// stores,
+//   dequant(v) = R^T (norm yhat + sqrt(pi/2)/m rnorm S^T z)        (PROD)
+// (ai.spot.hk "Google TurboQuant", "無偏內積估計"), the softmax-weighted sum of
+// values is taken in the rotated domain and rotated back once per query:
+//   out = R^T (a + sqrt(pi/2)/m S^T b),  a = sum_k w_k norm_k yhat_k,
+//                                        b = sum_k w_k rnorm_k z_k,
+// so no value row is ever reconstructed in memory.
+//
+// Kernels (after qprep + logits into the workspace):
+//   k_attn_chunk     one CTA per (key chunk, set): the chunk's softmax maximum
+//                    and normaliser per query, and its partial a, b (weights
+//                    exp(scale (s - max_chunk))), one thread per coordinate /
+//                    projection slot; the chunk's packed rows pass through
+//                    shared memory 32 keys at a time
+//   k_attn_finalize  one CTA per (set, query): combines the chunks (the usual
+//                    rescaling by exp(max_chunk - max)), adds sqrt(pi/2)/m S^T b,
+//                    rotates back (FWHT in shared memory, D, 1/sqrt(d))
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "tq_internal.h"
+
+namespace tq {
+
+namespace {
+
+constexpr int kAttnThreads = 256;
+constexpr int kAttnBatch = 32;            // keys staged in shared memory at a time
+constexpr float kLog2e = 1.4426950408889634f;
+
+// partial record per (set, query, chunk): [max (log2 units), normaliser, a (d), b (m)]
+__host__ __device__ inline int64_t partial_floats(int d, int m) { return 2 + d + m; }
+
+template <int G, int SLOTS>
+__global__ void __launch_bounds__(kAttnThreads)
+k_attn_chunk(const KParams P, const float* __restrict__ logits, const Packed values, int64_t n_keys, int chunk,
+             float scale_log2, int prod, float* __restrict__ partial) {
+  const int d = P.d, m = P.m, B = P.B;
+  const int set = blockIdx.y, c = blockIdx.x, n_chunks = gridDim.x;
+  const int64_t k0 = static_cast<int64_t>(c) * chunk;
+  const int64_t k1 = k0 + chunk < n_keys ? k0 + chunk : n_keys;
+  const int tid = threadIdx.x;
+  const int cw32 = P.codes_bytes / 4, sw32 = P.signs_bytes / 4;   // words per packed row
+  extern __shared__ __align__(16) uint32_t sm[];
+  uint32_t* sCodes = sm;                                        // [batch][cw32 + 1]
+  uint32_t* sSigns = sCodes + kAttnBatch * (cw32 + 1);          // [batch][sw32]
+  float* sNorm = reinterpret_cast<float*>(sSigns + kAttnBatch * sw32);   // [batch]
+  float* sRn = sNorm + kAttnBatch;                              // [batch]
+  float* sW = sRn + kAttnBatch;                                 // [batch][G]
+  float* sMax = sW + kAttnBatch * G;                            // [G]
+  float* sRed = sMax + G;                                       // [kAttnThreads / 32][G]
+  __shared__ float lut[kMaxLevels];
+  if (tid < kMaxLevels) lut[tid] = P.c[tid];
+
+  const float* lg = logits + static_cast<int64_t>(set) * G * n_keys;
+  // ---- the chunk's maximum of scale * logit per query (log2 units) -------------
+  float mx[G];
+#pragma unroll
+  for (int q = 0; q < G; ++q) mx[q] = -INFINITY;
+  for (int64_t k = k0 + tid; k < k1; k += kAttnThreads)
+#pragma unroll
+    for (int q = 0; q < G; ++q) mx[q] = fmaxf(mx[q], lg[q * n_keys + k] * scale_log2);
+#pragma unroll
+  for (int q = 0; q < G; ++q) {
+    float v = mx[q];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if ((tid & 31) == 0) sRed[(tid >> 5) * G + q] = v;
+  }
+  __syncthreads();
+  if (tid < G) {
+    float v = -INFINITY;
+    for (int w = 0; w < kAttnThreads / 32; ++w) v = fmaxf(v, sRed[w * G + tid]);
+    sMax[tid] = v;
+  }
+  __syncthreads();
+  float cm[G];
+#pragma unroll
+  for (int q = 0; q < G; ++q) cm[q] = sMax[q];
+
+  // ---- weighted sums: thread slot x = s * 256 + tid is coordinate x (x < d) or
+  // projection x - d (PROD only) --------------------------------------------------
+  float acc[SLOTS][G];
+#pragma unroll
+  for (int s = 0; s < SLOTS; ++s)
+#pragma unroll
+    for (int q = 0; q < G; ++q) acc[s][q] = 0.f;
+  float lsum = 0.f;                                            // thread tid < batch*G: its (key, query)
+  const int nx = d + (prod ? m : 0);
+  const uint32_t mask = (1u << B) - 1u;
+  for (int64_t kb = k0; kb < k1; kb += kAttnBatch) {
+    const int nb = static_cast<int>(k1 - kb < kAttnBatch ? k1 - kb : kAttnBatch);
+    __syncthreads();                                            // previous batch consumed
+    const int64_t row0 = static_cast<int64_t>(set) * n_keys + kb;
+    for (int e = tid; e < nb * cw32; e += kAttnThreads) {
+      const int r = e / cw32, w = e - r * cw32;
+      sCodes[r * (cw32 + 1) + w] = __ldg(reinterpret_cast<const uint32_t*>(values.codes) + (row0 + r) * cw32 + w);
+    }
+    for (int r = tid; r < nb; r += kAttnThreads) sCodes[r * (cw32 + 1) + cw32] = 0u;
+    if (prod)
+      for (int e = tid; e < nb * sw32; e += kAttnThreads) {
+        const int r = e / sw32, w = e - r * sw32;
+        sSigns[r * sw32 + w] = __ldg(reinterpret_cast<const uint32_t*>(values.signs) + (row0 + r) * sw32 + w);
+      }
+    for (int r = tid; r < nb; r += kAttnThreads) {
+      sNorm[r] = __ldg(values.norm + row0 + r);
+      sRn[r] = __ldg(values.rnorm + row0 + r);
+    }
+    for (int e = tid; e < nb * G; e += kAttnThreads) {
+      const int r = e / G, q = e - r * G;
+      const float w = exp2f(lg[q * n_keys + kb + r] * scale_log2 - cm[q]);
+      sW[r * G + q] = w;
+      lsum += w;                                                // (e == tid: one (key, query) per thread)
+    }
+    __syncthreads();
+#pragma unroll
+    for (int s = 0; s < SLOTS; ++s) {
+      const int x = s * kAttnThreads + tid;
+      if (x < d) {
+        const int bit = B * x, wi = bit >> 5, sh = bit & 31;
+        for (int r = 0; r < nb; ++r) {
+          const uint32_t* cr = sCodes + r * (cw32 + 1);
+          const uint32_t lo = cr[wi], hi = cr[wi + 1];
+          const uint32_t code = static_cast<uint32_t>(((static_cast<uint64_t>(hi) << 32) | lo) >> sh) & mask;
+          const float v = sNorm[r] * lut[code];
+#pragma unroll
+          for (int q = 0; q < G; ++q) acc[s][q] = fmaf(sW[r * G + q], v, acc[s][q]);
+        }
+      } else if (x < nx) {
+        const int j = x - d;
+        for (int r = 0; r < nb; ++r) {
+          const uint32_t bitv = (sSigns[r * sw32 + (j >> 5)] >> (j & 31)) & 1u;
+          const float v = bitv ? -sRn[r] : sRn[r];
+#pragma unroll
+          for (int q = 0; q < G; ++q) acc[s][q] = fmaf(sW[r * G + q], v, acc[s][q]);
+        }
+      }
+    }
+  }
+  // ---- the chunk's normaliser per query and the partial record -----------------
+  // thread tid accumulated (key tid / G, query tid % G) of every batch
+  __syncthreads();
+  float* sL = sRed;                                             // [kAttnThreads]
+  sL[tid] = lsum;
+  __syncthreads();
+  float* rec = partial + ((static_cast<int64_t>(set) * G) * n_chunks + c) * partial_floats(d, m);
+  const int64_t qstride = static_cast<int64_t>(n_chunks) * partial_floats(d, m);
+  if (tid < G) {
+    float l = 0.f;
+    for (int t = tid; t < kAttnBatch * G && t < kAttnThreads; t += G) l += sL[t];
+    rec[tid * qstride + 0] = cm[tid];
+    rec[tid * qstride + 1] = l;
+  }
+#pragma unroll
+  for (int s = 0; s < SLOTS; ++s) {
+    const int x = s * kAttnThreads + tid;
+    if (x < nx)
+#pragma unroll
+      for (int q = 0; q < G; ++q) rec[q * qstride + 2 + x] = acc[s][q];
+  }
+}
+
+__global__ void __launch_bounds__(kAttnThreads)
+k_attn_finalize(const KParams P, const float* __restrict__ partial, int n_chunks, int prod, float* __restrict__ out) {
+  const int d = P.d, m = P.m, tid = threadIdx.x;
+  const int64_t rowq = blockIdx.x;                              // set * g + query
+  const int64_t pf = partial_floats(d, m);
+  const float* rec = partial + rowq * n_chunks * pf;
+  extern __shared__ __align__(16) float fs[];
+  float* sa = fs;                                               // [d]
+  float* sb = fs + d;                                           // [m]
+  __shared__ float sM, sLn;
+  if (tid == 0) {
+    float mx = -INFINITY;
+    for (int c = 0; c < n_chunks; ++c) mx = fmaxf(mx, rec[c * pf]);
+    float l = 0.f;
+    for (int c = 0; c < n_chunks; ++c) l += rec[c * pf + 1] * exp2f(rec[c * pf] - mx);
+    sM = mx;
+    sLn = l;
+  }
+  __syncthreads();
+  const float mx = sM, inv_l = 1.f / sLn;
+  const int nx = d + (prod ? m : 0);
+  for (int x = tid; x < nx; x += kAttnThreads) {
+    float v = 0.f;
+    for (int c = 0; c < n_chunks; ++c) v = fmaf(rec[c * pf + 2 + x], exp2f(rec[c * pf] - mx), v);
+    v *= inv_l;
+    if (x < d) sa[x] = v;
+    else sb[x - d] = v;
+  }
+  __syncthreads();
+  if (prod) {
+    // a += sqrt(pi/2)/m S^T b   (S^T row i is contiguous in P.St)
+    for (int i = tid; i < d; i += kAttnThreads) {
+      const __half* st = reinterpret_cast<const __half*>(P.St) + static_cast<int64_t>(i) * m;
+      float acc = 0.f;
+      for (int j = 0; j < m; ++j) acc = fmaf(__half2float(st[j]), sb[j], acc);
+      sa[i] = fmaf(P.qjl_scale, acc, sa[i]);
+    }
+    __syncthreads();
+  }
+  // R^T a = D (H a) / sqrt(d): Walsh-Hadamard butterflies in shared memory
+  for (int h = 1; h < d; h <<= 1) {
+    for (int p = tid; p < d / 2; p += kAttnThreads) {
+      const int i = (p / h) * 2 * h + (p % h), j = i + h;
+      const float u = sa[i], w = sa[j];
+      sa[i] = u + w;
+      sa[j] = u - w;
+    }
+    __syncthreads();
+  }
+  for (int i = tid; i < d; i += kAttnThreads) {
+    const bool neg = (P.Dmask[i >> 5] >> (i & 31)) & 1u;
+    const float v = sa[i] * P.inv_sqrt_d;
+    out[rowq * d + i] = neg ? -v : v;
+  }
+}
+
+template <int G, int SLOTS>
+int launch_chunk(const KParams& P, const float* logits, const Packed& values, int64_t n_sets, int64_t n_keys,
+                 int chunk, int n_chunks, float scale_log2, int prod, float* partial, cudaStream_t s) {
+  const int cw32 = P.codes_bytes / 4, sw32 = P.signs_bytes / 4;
+  const size_t smem = (static_cast<size_t>(kAttnBatch) * (cw32 + 1) + kAttnBatch * sw32 + 2 * kAttnBatch +
+                       kAttnBatch * G + G + kAttnThreads) * 4;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_attn_chunk<G, SLOTS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  dim3 grid(static_cast<unsigned>(n_chunks), static_cast<unsigned>(n_sets));
+  k_attn_chunk<G, SLOTS><<<grid, kAttnThreads, smem, s>>>(P, logits, values, n_keys, chunk, scale_log2, prod, partial);
+  count_launch();
+  return static_cast<int>(cudaGetLastError());
+}
+
+template <int G>
+int launch_chunk_g(const KParams& P, const float* logits, const Packed& values, int64_t n_sets, int64_t n_keys,
+                   int chunk, int n_chunks, float scale_log2, int prod, float* partial, cudaStream_t s) {
+  const int nx = P.d + (prod ? P.m : 0);
+  const int slots = (nx + kAttnThreads - 1) / kAttnThreads;
+  if (slots <= 1) return launch_chunk<G, 1>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s);
+  if (slots <= 2) return launch_chunk<G, 2>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s);
+  if (slots <= 4) return launch_chunk<G, 4>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s);
+  return launch_chunk<G, 8>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s);
+}
+
+}  // namespace
+
+int attention_chunk_keys() { return 2048; }
+
+size_t attention_partial_bytes(const KParams& P, int64_t n_sets, int g, int64_t n_keys) {
+  const int64_t n_chunks = (n_keys + attention_chunk_keys() - 1) / attention_chunk_keys();
+  return static_cast<size_t>(n_sets) * g * n_chunks * partial_floats(P.d, P.m) * sizeof(float);
+}
+
+int launch_attention_tail(const KParams& P, const float* logits, const Packed& values, int64_t n_sets, int g,
+                          int64_t n_keys, float scale, int prod, float* partial, float* out, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int chunk = attention_chunk_keys();
+  const int n_chunks = static_cast<int>((n_keys + chunk - 1) / chunk);
+  const float scale_log2 = scale * kLog2e;
+  int err = 0;
+  switch (g) {
+    case 1: err = launch_chunk_g<1>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s); break;
+    case 2: err = launch_chunk_g<2>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s); break;
+    case 3: err = launch_chunk_g<3>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s); break;
+    case 4: err = launch_chunk_g<4>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s); break;
+    case 5: err = launch_chunk_g<5>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s); break;
+    case 6: err = launch_chunk_g<6>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s); break;
+    case 7: err = launch_chunk_g<7>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s); break;
+    default: err = launch_chunk_g<8>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s); break;
+  }
+  if (err) return err;
+  const size_t smem = static_cast<size_t>(P.d + P.m) * sizeof(float);
+  k_attn_finalize<<<static_cast<unsigned>(n_sets * g), kAttnThreads, smem, s>>>(P, partial, n_chunks, prod, out);
+  count_launch();
+  return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace tq

@@ -275,6 +275,52 @@ tq_status tq_logits(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t 
   return TQ_OK;
 }
 
+static size_t round16(size_t v) { return (v + 15) & ~static_cast<size_t>(15); }
+
+size_t tq_attention_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g, int64_t n_keys) {
+  if (!ctx || n_sets <= 0 || g <= 0 || n_keys <= 0) return 0;
+  return round16(tq_logits_workspace_bytes(ctx, n_sets, g)) +
+         round16(static_cast<size_t>(n_sets) * g * n_keys * sizeof(float)) +
+         round16(attention_partial_bytes(ctx->kp, n_sets, g, n_keys));
+}
+
+tq_status tq_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g, tq_packed keys,
+                       tq_packed values, int64_t n_keys, float scale, tq_dequant_mode mode, float* out,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  tq_status st = check_ctx(ctx);
+  if (st != TQ_OK) return st;
+  if (n_sets < 0 || n_keys < 0) return fail(TQ_ERR_INVALID_ARG, "n_sets and n_keys must be >= 0");
+  if (g < 1 || g > 8) return fail(TQ_ERR_INVALID_ARG, "g must be in [1, 8]");
+  if (q_dtype != TQ_BF16 && q_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "q_dtype must be TQ_BF16 or TQ_F32");
+  if (mode != TQ_DEQUANT_PROD && mode != TQ_DEQUANT_MSE) return fail(TQ_ERR_INVALID_ARG, "bad dequant mode");
+  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale must be finite");
+  if (ctx->d + ctx->m > 2048) return fail(TQ_ERR_UNSUPPORTED, "tq_attention needs d + m <= 2048");
+  if (n_sets == 0) return TQ_OK;
+  if (n_keys == 0) return fail(TQ_ERR_INVALID_ARG, "n_keys must be >= 1 (softmax over no keys)");
+  if (n_sets > 65535) return fail(TQ_ERR_UNSUPPORTED, "n_sets must be <= 65535");
+  if (n_keys > (int64_t(1) << 31) - 4096) return fail(TQ_ERR_UNSUPPORTED, "n_keys too large");
+  if (!q || !out) return fail(TQ_ERR_INVALID_ARG, "q or out is NULL");
+  if (!aligned(q, 16) || !aligned(out, 4)) return fail(TQ_ERR_INVALID_ARG, "q must be 16-byte and out 4-byte aligned");
+  if ((st = check_packed(ctx, keys)) != TQ_OK) return st;
+  if ((st = check_packed(ctx, values)) != TQ_OK) return st;
+  const size_t need = tq_attention_workspace_bytes(ctx, n_sets, g, n_keys);
+  if (!workspace || workspace_bytes < need) return fail(TQ_ERR_INVALID_ARG, "workspace missing or too small");
+  if (!aligned(workspace, 16)) return fail(TQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  float* qp = reinterpret_cast<float*>(w);
+  float* lg = reinterpret_cast<float*>(w + round16(tq_logits_workspace_bytes(ctx, n_sets, g)));
+  float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(lg) +
+                                         round16(static_cast<size_t>(n_sets) * g * n_keys * sizeof(float)));
+  int err = launch_qprep(ctx->kp, q, q_dtype == TQ_BF16, n_sets * g, qp, stream);
+  if (err) return cuda_fail(err, "tq_attention query-prep launch");
+  err = launch_logits(*ctx, qp, n_sets, g, to_internal(keys), n_keys, lg, stream);
+  if (err) return cuda_fail(err, "tq_attention logits launch");
+  err = launch_attention_tail(ctx->kp, lg, to_internal(values), n_sets, g, n_keys, scale,
+                              mode == TQ_DEQUANT_PROD ? 1 : 0, part, out, stream);
+  if (err) return cuda_fail(err, "tq_attention launch");
+  return TQ_OK;
+}
+
 tq_status tq_dequant(const tq_ctx* ctx, tq_packed in, int64_t n_rows, void* out, tq_dtype out_dtype,
                      tq_dequant_mode mode, void* stream) {
   tq_status st = check_ctx(ctx);

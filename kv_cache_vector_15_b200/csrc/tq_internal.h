@@ -59,6 +59,10 @@ int launch_logits(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, con
                   int64_t n_keys, float* out, void* stream);
 int launch_dequant(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
                    void* stream);
+// attention.cu: the softmax-weighted value sums after the logits are in place
+size_t attention_partial_bytes(const KParams& P, int64_t n_sets, int g, int64_t n_keys);
+int launch_attention_tail(const KParams& P, const float* logits, const Packed& values, int64_t n_sets, int g,
+                          int64_t n_keys, float scale, int prod, float* partial, float* out, void* stream);
 int launch_topk(const float* scores, int64_t rows, int64_t cols, int k, int32_t* idx, float* val, void* stream);
 int launch_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, int d, float* out,
                        void* stream);

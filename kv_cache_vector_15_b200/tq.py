@@ -9,6 +9,7 @@ there is no fallback path.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from dataclasses import dataclass
 
@@ -29,7 +30,8 @@ TQ_DEQUANT_PROD, TQ_DEQUANT_MSE = 0, 1
 SYMBOLS = [
     "tq_host_params", "tq_init", "tq_destroy", "tq_packed_sizes", "tq_get_params", "tq_quantize",
     "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_dequant", "tq_topk", "tq_logits_bf16",
-    "tq_status_str", "tq_sync_status", "tq_last_error", "tq_launch_count",
+    "tq_status_str", "tq_sync_status", "tq_last_error", "tq_launch_count", "tq_attention_workspace_bytes",
+    "tq_attention",
 ]
 
 
@@ -50,6 +52,9 @@ _sig = {
     "tq_logits": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _i64, _vp, _vp, _sz, _vp]),
     "tq_logits_noalloc": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _i64, _vp, _vp]),
     "tq_dequant": (_i32, [_vp, _Packed, _i64, _vp, _i32, _i32, _vp]),
+    "tq_attention_workspace_bytes": (_sz, [_vp, _i64, _i32, _i64]),
+    "tq_attention": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _Packed, _i64, ctypes.c_float, _i32, _vp, _vp, _sz,
+                            _vp]),
     "tq_topk": (_i32, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "tq_logits_bf16": (_i32, [_vp, _vp, _i64, _i32, _i64, _i32, _vp, _vp]),
     "tq_status_str": (ctypes.c_char_p, [_i32]),
@@ -239,6 +244,29 @@ class TurboQuant:
             out = torch.empty((n, self.d), dtype=out_dtype or torch.bfloat16, device=packed.norm.device)
         _check(_lib.tq_dequant(self._h, packed.c(), n, _ptr(out), _dtype_code(out), mode, _stream(stream)),
                "tq_dequant")
+        return out
+
+
+    def attention_workspace_bytes(self, n_sets: int, g: int, n_keys: int) -> int:
+        return int(_lib.tq_attention_workspace_bytes(self._h, n_sets, g, n_keys))
+
+    def attention(self, q, keys: Packed, values: Packed, n_sets: int, g: int, n_keys: int, scale: float | None = None,
+                  mode: int = TQ_DEQUANT_PROD, out=None, workspace=None, stream=None):
+        """Decode attention from packed keys and values: [n_sets*g, d] fp32
+        (softmax over each set's keys of scale * logit, times the dequantized
+        values; scale defaults to 1/sqrt(d))."""
+        import torch
+        if scale is None:
+            scale = 1.0 / math.sqrt(self.d)
+        if out is None:
+            out = torch.empty((n_sets * g, self.d), dtype=torch.float32, device=q.device)
+        need = self.attention_workspace_bytes(n_sets, g, n_keys)
+        if need and workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        _check(_lib.tq_attention(self._h, _ptr(q), _dtype_code(q), n_sets, g, keys.c(), values.c(), n_keys,
+                                 float(scale), mode, _ptr(out), _ptr(workspace), wbytes, _stream(stream)),
+               "tq_attention")
         return out
 
 

@@ -73,6 +73,9 @@ def test_host_calls_validate_before_any_launch():
     assert tq.call_status("tq_logits_bf16", None, None, 1, 9, 10, 128, None, None) == tq.TQ_ERR_INVALID_ARG
     assert tq.call_status("tq_logits_bf16", None, None, 1, 4, 10, 96, None, None) == tq.TQ_ERR_INVALID_ARG
     assert tq.call_status("tq_logits_bf16", None, None, 0, 4, 10, 128, None, None) == tq.TQ_OK
+    assert tq.call_status("tq_attention", None, None, 0, 1, 4, P, P, 10, ctypes.c_float(0.1), 0, None, None, 0,
+                          None) == tq.TQ_ERR_INVALID_ARG
+    assert tq._lib.tq_attention_workspace_bytes(None, 1, 4, 10) == 0
     assert tq.launch_count() == before
 
 

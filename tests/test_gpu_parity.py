@@ -240,3 +240,61 @@ def test_gpu_api_errors_and_empty_calls(tq):
         T.logits(torch.zeros((4, 128), device="cuda"), T.empty_packed(8), 1, 4, 8,
                  workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
     assert tq.launch_count() == before
+
+
+@pytest.mark.parametrize("d,b,m,n_sets,g,n_keys", [
+    (128, 3, 128, 3, 4, 5000), (128, 4, 128, 2, 8, 2049), (128, 2, 128, 2, 1, 77), (64, 3, 96, 2, 3, 4100),
+    (256, 4, 128, 1, 5, 1500), (1024, 4, 1024, 1, 2, 300)])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_attention_parity(tq, d, b, m, n_sets, g, n_keys, mode):
+    """Attention from packed keys and values against the oracle's softmax and
+    dequantized value sum, driven by the kernel's own logits (the logits have
+    their own parity test): what is compared is the softmax, the weighted sum
+    in the rotated domain, the QJL term and the rotation back."""
+    P = op.Params(d, b, m, seed=0)
+    rng = np.random.default_rng(d + b + g)
+    k = rng.standard_normal((n_sets * n_keys, d)) * rng.uniform(0.5, 2, size=(n_sets * n_keys, 1))
+    v = rng.standard_normal((n_sets * n_keys, d)) * rng.uniform(0.1, 10, size=(n_sets * n_keys, 1))
+    v[:4] = edge_rows(d, rng)[:4]
+    pk, pv = ot.quantize(k, P), ot.quantize(v, P)
+    qt, q = make_rows(d, n_sets * g, "bf16", seed=9)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    keys, vals = tq.Packed.from_numpy(pk), tq.Packed.from_numpy(pv)
+    scale = 1.0 / np.sqrt(d)
+    got = T.attention(qt.cuda(), keys, vals, n_sets, g, n_keys, scale=scale, mode=mode).cpu().numpy()
+    lg = T.logits(qt.cuda(), keys, n_sets, g, n_keys).cpu().numpy()
+    T.sync_status()
+    want = ot.attention(q, pk, pv, P, n_sets, g, n_keys, scale, mode=mode, logits_in=lg).reshape(n_sets * g, d)
+    # the output is a convex combination of dequantized rows: compare on the scale of those rows
+    xv = ot.dequant(pv, P, mode).reshape(n_sets, n_keys, d)
+    vscale = np.repeat(np.abs(xv).max(axis=(1, 2)), g)[:, None]
+    assert np.all(np.abs(got - want) <= 1e-4 * vscale + 1e-30), float(np.max(np.abs(got - want) / vscale))
+
+
+def test_attention_matches_logits_softmax_on_full_oracle(tq):
+    """End to end against the oracle's own logits: agreement within what the
+    logit tolerance lets the softmax move."""
+    d, b, m, n_sets, g, n_keys = 128, 3, 128, 2, 4, 3000
+    P = op.Params(d, b, m, seed=0)
+    rng = np.random.default_rng(21)
+    k = rng.standard_normal((n_sets * n_keys, d)) * 0.3
+    v = rng.standard_normal((n_sets * n_keys, d))
+    pk, pv = ot.quantize(k, P), ot.quantize(v, P)
+    qt, q = make_rows(d, n_sets * g, "bf16", seed=22)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    got = T.attention(qt.cuda(), tq.Packed.from_numpy(pk), tq.Packed.from_numpy(pv), n_sets, g, n_keys).cpu().numpy()
+    want = ot.attention(q, pk, pv, P, n_sets, g, n_keys, 1.0 / np.sqrt(d)).reshape(n_sets * g, d)
+    vmax = np.abs(ot.dequant(pv, P)).max()
+    assert np.max(np.abs(got - want)) <= 1e-3 * vmax
+
+
+def test_attention_argument_errors(tq):
+    T = tq.TurboQuant(128, 3, 128, seed=0)
+    q = torch.zeros((4, 128), dtype=torch.bfloat16, device="cuda")
+    pk = T.empty_packed(10, "cuda")
+    with pytest.raises(tq.TQError):
+        T.attention(q, pk, pk, 1, 9, 10)                 # g > 8
+    with pytest.raises(tq.TQError):
+        T.attention(q, pk, pk, 1, 4, 0)                  # no keys
+    out = torch.empty((0, 128), dtype=torch.float32, device="cuda")
+    T.attention(q, pk, pk, 0, 4, 10, out=out)            # no sets: no-op
