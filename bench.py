@@ -340,6 +340,36 @@ def run_ours(args, cfg, ws, rank, local):
     bf16_ms = e0.elapsed_time(e1) / reps
     bf16_bytes = N * (2 * d + 4 * g)
 
+    # decode attention from the compressed cache (softmax over the estimated
+    # logits, value sum in the rotated domain) and torch's bf16 SDPA on the same
+    # shapes as a reference point (a library kernel, not part of the path)
+    attn_out = torch.empty((n_sets * g, d), dtype=torch.float32, device=dev)
+    attn_ws = torch.empty(max(T.attention_workspace_bytes(n_sets, g, n_keys), 16), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        T.attention(dQ, pK, pV, n_sets, g, n_keys, out=attn_out, workspace=attn_ws, stream=stream)
+    e0.record(stream)
+    for _ in range(reps):
+        T.attention(dQ, pK, pV, n_sets, g, n_keys, out=attn_out, workspace=attn_ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    attn_ms = e0.elapsed_time(e1) / reps
+    sdpa_ms = None
+    try:
+        import torch.nn.functional as F
+        qh = dQ.view(sh.batch, cfg["q_heads"], 1, d)
+        kh = dK.view(sh.batch, cfg["kv_heads"], n_keys, d)
+        vh = dV.view(sh.batch, cfg["kv_heads"], n_keys, d)
+        for _ in range(3):
+            F.scaled_dot_product_attention(qh, kh, vh, enable_gqa=True)
+        e0.record(stream)
+        for _ in range(reps):
+            F.scaled_dot_product_attention(qh, kh, vh, enable_gqa=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        sdpa_ms = e0.elapsed_time(e1) / reps
+    except Exception:                     # the reference point is optional
+        sdpa_ms = None
+
     # end to end through the public API with host buffers: every step uploads K,
     # V and q from pinned host memory and downloads the logits and V-hat,
     # pipelined over this rank's sequences -- sequence i+1 uploads on one copy
@@ -427,6 +457,8 @@ def run_ours(args, cfg, ws, rank, local):
                             "bytes_per_launch": v["bytes"]} for k, v in kern.items()},
             "bf16_key_logits_baseline": {"ms": bf16_ms, "algorithmic_GBps": bf16_bytes / (bf16_ms * 1e-3) / 1e9,
                                          "tq_logits_speedup": bf16_ms / avg["logits"]},
+            "attention": {"ms": attn_ms, "packed_GBps": N * 2 * P / (attn_ms * 1e-3) / 1e9,
+                          "torch_sdpa_bf16_ms": sdpa_ms},
             "cpu_baseline": cpu,
             "e2e": {"value": total_logits / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

@@ -56,10 +56,10 @@ k_attn_chunk(const KParams P, const float* __restrict__ logits, const Packed val
   extern __shared__ __align__(16) uint32_t sm[];
   uint32_t* sCodes = sm;                                        // [batch][cw32 + 1]
   uint32_t* sSigns = sCodes + kAttnBatch * (cw32 + 1);          // [batch][sw32]
-  float* sNorm = reinterpret_cast<float*>(sSigns + kAttnBatch * sw32);   // [batch]
-  float* sRn = sNorm + kAttnBatch;                              // [batch]
-  float* sW = sRn + kAttnBatch;                                 // [batch][G]
-  float* sMax = sW + kAttnBatch * G;                            // [G]
+  constexpr int GP = (G + 3) / 4 * 4;                           // weights per key, padded for float4 loads
+  float* sWn = reinterpret_cast<float*>(sSigns + kAttnBatch * sw32);     // [batch][GP] weight * norm
+  float* sWr = sWn + kAttnBatch * GP;                           // [batch][GP] weight * rnorm
+  float* sMax = sWr + kAttnBatch * GP;                          // [G]
   float* sRed = sMax + G;                                       // [kAttnThreads / 32][G]
   __shared__ float lut[kMaxLevels];
   if (tid < kMaxLevels) lut[tid] = P.c[tid];
@@ -114,15 +114,12 @@ k_attn_chunk(const KParams P, const float* __restrict__ logits, const Packed val
         const int r = e / sw32, w = e - r * sw32;
         sSigns[r * sw32 + w] = __ldg(reinterpret_cast<const uint32_t*>(values.signs) + (row0 + r) * sw32 + w);
       }
-    for (int r = tid; r < nb; r += kAttnThreads) {
-      sNorm[r] = __ldg(values.norm + row0 + r);
-      sRn[r] = __ldg(values.rnorm + row0 + r);
-    }
-    for (int e = tid; e < nb * G; e += kAttnThreads) {
+    for (int e = tid; e < nb * G; e += kAttnThreads) {        // (e == tid: one (key, query) per thread)
       const int r = e / G, q = e - r * G;
       const float w = exp2f(lg[q * n_keys + kb + r] * scale_log2 - cm[q]);
-      sW[r * G + q] = w;
-      lsum += w;                                                // (e == tid: one (key, query) per thread)
+      sWn[r * GP + q] = w * __ldg(values.norm + row0 + r);
+      sWr[r * GP + q] = w * __ldg(values.rnorm + row0 + r);
+      lsum += w;
     }
     __syncthreads();
 #pragma unroll
@@ -130,21 +127,35 @@ k_attn_chunk(const KParams P, const float* __restrict__ logits, const Packed val
       const int x = s * kAttnThreads + tid;
       if (x < d) {
         const int bit = B * x, wi = bit >> 5, sh = bit & 31;
+        const bool one_word = (32 % B) == 0;                    // codes never straddle two words
         for (int r = 0; r < nb; ++r) {
           const uint32_t* cr = sCodes + r * (cw32 + 1);
-          const uint32_t lo = cr[wi], hi = cr[wi + 1];
-          const uint32_t code = static_cast<uint32_t>(((static_cast<uint64_t>(hi) << 32) | lo) >> sh) & mask;
-          const float v = sNorm[r] * lut[code];
+          uint32_t code;
+          if (one_word) code = (cr[wi] >> sh) & mask;
+          else code = static_cast<uint32_t>(((static_cast<uint64_t>(cr[wi + 1]) << 32) | cr[wi]) >> sh) & mask;
+          const float v = lut[code];
 #pragma unroll
-          for (int q = 0; q < G; ++q) acc[s][q] = fmaf(sW[r * G + q], v, acc[s][q]);
+          for (int q4 = 0; q4 < GP; q4 += 4) {
+            const float4 w = *reinterpret_cast<const float4*>(sWn + r * GP + q4);
+            if (q4 + 0 < G) acc[s][q4 + 0] = fmaf(w.x, v, acc[s][q4 + 0]);
+            if (q4 + 1 < G) acc[s][q4 + 1] = fmaf(w.y, v, acc[s][q4 + 1]);
+            if (q4 + 2 < G) acc[s][q4 + 2] = fmaf(w.z, v, acc[s][q4 + 2]);
+            if (q4 + 3 < G) acc[s][q4 + 3] = fmaf(w.w, v, acc[s][q4 + 3]);
+          }
         }
       } else if (x < nx) {
         const int j = x - d;
         for (int r = 0; r < nb; ++r) {
           const uint32_t bitv = (sSigns[r * sw32 + (j >> 5)] >> (j & 31)) & 1u;
-          const float v = bitv ? -sRn[r] : sRn[r];
+          const float z = bitv ? -1.f : 1.f;
 #pragma unroll
-          for (int q = 0; q < G; ++q) acc[s][q] = fmaf(sW[r * G + q], v, acc[s][q]);
+          for (int q4 = 0; q4 < GP; q4 += 4) {
+            const float4 w = *reinterpret_cast<const float4*>(sWr + r * GP + q4);
+            if (q4 + 0 < G) acc[s][q4 + 0] = fmaf(w.x, z, acc[s][q4 + 0]);
+            if (q4 + 1 < G) acc[s][q4 + 1] = fmaf(w.y, z, acc[s][q4 + 1]);
+            if (q4 + 2 < G) acc[s][q4 + 2] = fmaf(w.z, z, acc[s][q4 + 2]);
+            if (q4 + 3 < G) acc[s][q4 + 3] = fmaf(w.w, z, acc[s][q4 + 3]);
+          }
         }
       }
     }
@@ -232,8 +243,9 @@ template <int G, int SLOTS>
 int launch_chunk(const KParams& P, const float* logits, const Packed& values, int64_t n_sets, int64_t n_keys,
                  int chunk, int n_chunks, float scale_log2, int prod, float* partial, cudaStream_t s) {
   const int cw32 = P.codes_bytes / 4, sw32 = P.signs_bytes / 4;
-  const size_t smem = (static_cast<size_t>(kAttnBatch) * (cw32 + 1) + kAttnBatch * sw32 + 2 * kAttnBatch +
-                       kAttnBatch * G + G + kAttnThreads) * 4;
+  constexpr int GP = (G + 3) / 4 * 4;
+  const size_t smem = (static_cast<size_t>(kAttnBatch) * (cw32 + 1) + kAttnBatch * sw32 + 2 * kAttnBatch * GP + G +
+                       kAttnThreads) * 4;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k_attn_chunk<G, SLOTS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
