@@ -52,6 +52,9 @@ AUX_WORKLOADS = {
     "prefill-b4": dict(kind="prefill", b=4, m=128, d=128),
     # vector search: 1e6 x 1024 fp32 database, 1024 queries, b = 4, m = 1024, top-10
     "vsearch": dict(kind="vsearch", b=4, m=1024, d=1024),
+    # decode-time append: one new token of a 32-layer x 8-KV-head model (256 K rows
+    # and 256 V rows) scattered into a paged packed cache, latency per token
+    "append-b3": dict(kind="append", b=3, m=128, d=128),
 }
 METRIC = "compressed-key logits/s and % HBM roofline (d=128,b=3); quantize rows/s"
 UNIT = "logits/s"
@@ -473,6 +476,33 @@ def run_ours(args, cfg, ws, rank, local):
 # ---------------------------------------------------------------------------
 # Secondary workloads (prefill write path, vector search): CUDA path only
 # ---------------------------------------------------------------------------
+def append_graph_ms(torch, T, dev, stream, dk, dv, slots, cK, cV, steps):
+    """The append step replayed from a CUDA graph (no per-launch host cost);
+    None if the capture is not possible here."""
+    try:
+        gs = torch.cuda.Stream(dev)
+        gs.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gs):
+            T.quantize_scatter(dk, slots, cK, stream=gs)
+            T.quantize_scatter(dv, slots, cV, stream=gs)
+        stream.wait_stream(gs)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / steps
+        del g
+        return ms
+    except Exception:
+        return None
+
+
 def run_aux(args, cfg, ws, rank, local):
     import torch
     from kv_cache_vector_15_b200 import tq
@@ -502,6 +532,24 @@ def run_aux(args, cfg, ws, rank, local):
         units, unit, metric = 2 * n, "rows/s", f"tq_quantize rows/s, prefill write path (b={b})"
         alg = 2 * n * (2 * d + P)
         kern = "quantize"
+    elif cfg["kind"] == "append":
+        n_tok_rows, cache_rows = 256, 256 * 8192
+        K, V = inputs.prefill(layers=32, heads=8, ctx=1)            # one token: 256 rows each
+        hk = torch.empty((n_tok_rows, d), dtype=torch.bfloat16)
+        hv = torch.empty((n_tok_rows, d), dtype=torch.bfloat16)
+        K.fill(hk.view(torch.int16).numpy().view(np.uint16))
+        V.fill(hv.view(torch.int16).numpy().view(np.uint16))
+        dk, dv = hk.to(dev), hv.to(dev)
+        cK, cV = T.empty_packed(cache_rows, dev), T.empty_packed(cache_rows, dev)
+        # token position 4000 of every (layer, head) page of 8192 slots
+        slots = torch.arange(n_tok_rows, dtype=torch.int64, device=dev) * 8192 + 4000
+
+        def step():
+            T.quantize_scatter(dk, slots, cK, stream=stream)
+            T.quantize_scatter(dv, slots, cV, stream=stream)
+        units, unit, metric = 1, "tokens/s", "decode-time append: one token's K and V rows (32 layers x 8 heads) into a paged packed cache"
+        alg = 2 * n_tok_rows * (2 * d + P)
+        kern = "step"
     else:
         db, qs = inputs.vector_search()
         nq, ndb = qs.n_rows, db.n_rows
@@ -536,6 +584,9 @@ def run_aux(args, cfg, ws, rank, local):
         barrier(ws)
     ms = max_over_ranks(ws, e0.elapsed_time(e1)) / args.steps
     total = dist_util.sum_over_ranks(ws, units, device=dev)
+    graph_ms = None
+    if cfg["kind"] == "append":
+        graph_ms = append_graph_ms(torch, T, dev, stream, dk, dv, slots, cK, cV, args.steps)
     if rank == 0:
         gbs = alg / (ms * 1e-3) / 1e9
         print(json.dumps({
@@ -545,6 +596,7 @@ def run_aux(args, cfg, ws, rank, local):
             "config": {"workload": args.workload, "d": d, "b": b, "m": m, "l2": "inputs larger than L2; no flush"},
             "roofline": {"bound": "hbm", "kernel": kern, "achieved": gbs, "peak": hbm, "unit": "GB/s",
                          "frac": gbs / hbm, "traffic": None, "algorithmic_bytes": alg, "peak_kind": hbm_kind},
+            "cuda_graph_ms_per_step": graph_ms,
             "gpu_launches": tq.launch_count() - launches0, "clocks": clk.summary()}), flush=True)
     T.close()
 

@@ -120,6 +120,19 @@ tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_
 
 /* ----------------------------------------------------------- read half -- */
 
+/* Decode-time append into a paged cache: quantize n_rows rows of x (as
+ * tq_quantize) and write input row i to packed row dest_rows[i] of `cache`,
+ * a packed array of n_cache_rows rows (write-phase compression of the newly
+ * generated tokens: Qiita TurboQuant explainer, "APIの構成", the KV-cache
+ * wrapper).  dest_rows: device int64 array of n_rows indices (8-byte
+ * aligned); rows not named are left untouched; an index outside
+ * [0, n_cache_rows) is not written and makes the next tq_sync_status report
+ * TQ_ERR_INVALID_ARG (checked on the device, no fault).  Indices should be distinct (two rows sent to one
+ * slot race).  Runs one warp per row, sized for a handful of tokens
+ * (32 .. 256 rows): latency, not throughput. */
+tq_status tq_quantize_scatter(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
+                              const int64_t* dest_rows, int64_t n_cache_rows, tq_packed cache, void* stream);
+
 /* Device workspace that tq_logits needs for n_sets * g queries (bytes; 0 when
  * the call needs none, in which case workspace may be NULL). */
 size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g);
@@ -204,7 +217,8 @@ tq_status tq_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g,
 const char* tq_status_str(tq_status s);
 /* Wait for `stream`, then report whether any kernel of this context timed out
  * in one of its bounded device-side waits since the last check (TQ_ERR_CUDA,
- * outputs of that call invalid) and clear the record.  Blocking. */
+ * outputs of that call invalid), or met an out-of-range destination row in
+ * tq_quantize_scatter (TQ_ERR_INVALID_ARG), and clear the record.  Blocking. */
 tq_status tq_sync_status(const tq_ctx* ctx, void* stream);
 /* One-line reason for the last non-OK status returned on this host thread. */
 const char* tq_last_error(void);

@@ -91,9 +91,12 @@ __device__ __forceinline__ void apply_D(float (&v)[E], const uint32_t* Dmask, in
 // ---------------------------------------------------------------------------
 // write half
 // ---------------------------------------------------------------------------
+// dest: when not null, input row i goes to packed row dest[i] (a paged cache);
+// an index outside [0, n_dest) is not written and sets the error word (7).
 template <int E, bool BF16>
 __global__ void __launch_bounds__(kWarps * 32)
-k_quantize_warp(const KParams P, const void* __restrict__ x, int64_t n_rows, int64_t ld, const Packed out) {
+k_quantize_warp(const KParams P, const void* __restrict__ x, int64_t n_rows, int64_t ld, const Packed out,
+                const int64_t* __restrict__ dest, int64_t n_dest) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int d = P.d, m = P.m, B = P.B;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -106,8 +109,16 @@ k_quantize_warp(const KParams P, const void* __restrict__ x, int64_t n_rows, int
   const int nwords_codes = d * B / 32, nwords_signs = m / 32;
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + wib; row < n_rows;
        row += static_cast<int64_t>(gridDim.x) * kWarps) {
-    uint32_t* codes_out = reinterpret_cast<uint32_t*>(out.codes + row * P.codes_bytes);
-    uint32_t* signs_out = reinterpret_cast<uint32_t*>(out.signs + row * P.signs_bytes);
+    int64_t orow = row;
+    if (dest) {
+      orow = __ldg(dest + row);
+      if (orow < 0 || orow >= n_dest) {                      // warp-uniform: skip the row, flag it
+        if (lane == 0 && P.err) atomicCAS(P.err, 0, 7);
+        continue;
+      }
+    }
+    uint32_t* codes_out = reinterpret_cast<uint32_t*>(out.codes + orow * P.codes_bytes);
+    uint32_t* signs_out = reinterpret_cast<uint32_t*>(out.signs + orow * P.signs_bytes);
     float v[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) v[e] = load_elem<BF16>(x, row * ld + lane * E + e);
@@ -119,7 +130,7 @@ k_quantize_warp(const KParams P, const void* __restrict__ x, int64_t n_rows, int
     if (!(n >= kZeroNorm)) {                   // zero row (or a non-finite norm)
       for (int w = lane; w < nwords_codes; w += 32) codes_out[w] = 0u;
       for (int w = lane; w < nwords_signs; w += 32) signs_out[w] = 0u;
-      if (lane == 0) { out.norm[row] = 0.f; out.rnorm[row] = 0.f; }
+      if (lane == 0) { out.norm[orow] = 0.f; out.rnorm[orow] = 0.f; }
       continue;
     }
     apply_D<E>(v, P.Dmask, lane);
@@ -153,6 +164,7 @@ k_quantize_warp(const KParams P, const void* __restrict__ x, int64_t n_rows, int
     for (int t = 0; t < nwords_signs; ++t) {
       const int j = 32 * t + lane;
       float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll 8
       for (int i = 0; i < d; i += 4) {
         p0 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i) * m + j)), rs[i], p0);
         p1 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i + 1) * m + j)), rs[i + 1], p1);
@@ -163,7 +175,7 @@ k_quantize_warp(const KParams P, const void* __restrict__ x, int64_t n_rows, int
       const uint32_t bits = __ballot_sync(0xffffffffu, p < 0.f);
       if (lane == 0) signs_out[t] = bits;
     }
-    if (lane == 0) { out.norm[row] = n; out.rnorm[row] = n * sqrtf(r2); }
+    if (lane == 0) { out.norm[orow] = n; out.rnorm[orow] = n * sqrtf(r2); }
     __syncwarp();
   }
 }
@@ -195,6 +207,7 @@ k_qprep_warp(const KParams P, const void* __restrict__ q, int64_t n_q, float* __
     __syncwarp();
     for (int j = lane; j < m; j += 32) {
       float a0 = 0.f, a1 = 0.f;
+#pragma unroll 16
       for (int i = 0; i < d; i += 2) {
         a0 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i) * m + j)), qs[i], a0);
         a1 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i + 1) * m + j)), qs[i + 1], a1);
@@ -538,16 +551,16 @@ int grid_rows(int64_t n_rows) {
 
 template <int E>
 int launch_quantize_E(const KParams& P, const void* x, int bf16, int64_t n_rows, int64_t ld, const Packed& out,
-                      cudaStream_t s) {
+                      cudaStream_t s, const int64_t* dest = nullptr, int64_t n_dest = 0) {
   const size_t smem = static_cast<size_t>(kWarps) * P.d * 5;
   int g = grid_rows(n_rows);
   int err;
   if (bf16) {
     if ((err = set_smem(k_quantize_warp<E, true>, smem))) return err;
-    k_quantize_warp<E, true><<<g, kWarps * 32, smem, s>>>(P, x, n_rows, ld, out);
+    k_quantize_warp<E, true><<<g, kWarps * 32, smem, s>>>(P, x, n_rows, ld, out, dest, n_dest);
   } else {
     if ((err = set_smem(k_quantize_warp<E, false>, smem))) return err;
-    k_quantize_warp<E, false><<<g, kWarps * 32, smem, s>>>(P, x, n_rows, ld, out);
+    k_quantize_warp<E, false><<<g, kWarps * 32, smem, s>>>(P, x, n_rows, ld, out, dest, n_dest);
   }
   count_launch();
   return static_cast<int>(cudaGetLastError());
@@ -643,6 +656,24 @@ int launch_quantize_generic(const KParams& P, const void* x, int bf16, int64_t n
                             const Packed& out, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 #define CALL(E) launch_quantize_E<E>(P, x, bf16, n_rows, ld, out, s)
+  switch (P.d / 32) {
+    case 1: return CALL(1);
+    case 2: return CALL(2);
+    case 4: return CALL(4);
+    case 8: return CALL(8);
+    case 16: return CALL(16);
+    case 32: return CALL(32);
+    case 64: return CALL(64);
+    case 128: return CALL(128);
+  }
+#undef CALL
+  return static_cast<int>(cudaErrorInvalidValue);
+}
+
+int launch_quantize_scatter(const KParams& P, const void* x, int bf16, int64_t n_rows, int64_t ld,
+                            const int64_t* dest, int64_t n_dest, const Packed& out, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+#define CALL(E) launch_quantize_E<E>(P, x, bf16, n_rows, ld, out, s, dest, n_dest)
   switch (P.d / 32) {
     case 1: return CALL(1);
     case 2: return CALL(2);

@@ -97,6 +97,8 @@ tq_status tq_sync_status(const tq_ctx* ctx, void* stream) {
   if (word) {
     const int zero = 0;
     cudaMemcpy(ctx->kp.err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (word == 7) return fail(TQ_ERR_INVALID_ARG, "tq_quantize_scatter: a destination row index was out of range "
+                                                   "(that row was not written)");
     return fail(TQ_ERR_CUDA, "a kernel wait ran out of time (code " + std::to_string(word) + "); outputs are invalid");
   }
   return TQ_OK;
@@ -243,6 +245,26 @@ tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_
   if ((st = check_packed(ctx, out)) != TQ_OK) return st;
   int err = launch_quantize(*ctx, x, x_dtype == TQ_BF16, n_rows, ld_x, to_internal(out), stream);
   if (err) return cuda_fail(err, "tq_quantize launch");
+  return TQ_OK;
+}
+
+tq_status tq_quantize_scatter(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
+                              const int64_t* dest_rows, int64_t n_cache_rows, tq_packed cache, void* stream) {
+  tq_status st = check_ctx(ctx);
+  if (st != TQ_OK) return st;
+  if (n_rows < 0 || n_cache_rows < 0) return fail(TQ_ERR_INVALID_ARG, "n_rows and n_cache_rows must be >= 0");
+  if (x_dtype != TQ_BF16 && x_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "x_dtype must be TQ_BF16 or TQ_F32");
+  if (n_rows == 0) return TQ_OK;
+  if (!x || !dest_rows) return fail(TQ_ERR_INVALID_ARG, "x or dest_rows is NULL");
+  const size_t esz = x_dtype == TQ_BF16 ? 2 : 4;
+  if (ld_x < ctx->d) return fail(TQ_ERR_INVALID_ARG, "ld_x < d");
+  if (!aligned(x, 16) || (static_cast<size_t>(ld_x) * esz) % 16)
+    return fail(TQ_ERR_INVALID_ARG, "x and its row stride must be 16-byte aligned");
+  if (!aligned(dest_rows, 8)) return fail(TQ_ERR_INVALID_ARG, "dest_rows must be 8-byte aligned");
+  if ((st = check_packed(ctx, cache)) != TQ_OK) return st;
+  int err = launch_quantize_scatter(ctx->kp, x, x_dtype == TQ_BF16, n_rows, ld_x, dest_rows, n_cache_rows,
+                                    to_internal(cache), stream);
+  if (err) return cuda_fail(err, "tq_quantize_scatter launch");
   return TQ_OK;
 }
 

@@ -54,6 +54,8 @@ int launch_dequant_generic(const KParams& P, const Packed& in, int64_t n_rows, v
                            void* stream);
 int launch_quantize(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x,
                     const Packed& out, void* stream);
+int launch_quantize_scatter(const KParams& P, const void* x, int bf16, int64_t n_rows, int64_t ld,
+                            const int64_t* dest, int64_t n_dest, const Packed& out, void* stream);
 int launch_qprep(const KParams& P, const void* q, int q_is_bf16, int64_t n_queries, float* qp, void* stream);
 int launch_logits(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys,
                   int64_t n_keys, float* out, void* stream);

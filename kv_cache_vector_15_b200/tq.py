@@ -31,7 +31,7 @@ SYMBOLS = [
     "tq_host_params", "tq_init", "tq_destroy", "tq_packed_sizes", "tq_get_params", "tq_quantize",
     "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_dequant", "tq_topk", "tq_logits_bf16",
     "tq_status_str", "tq_sync_status", "tq_last_error", "tq_launch_count", "tq_attention_workspace_bytes",
-    "tq_attention",
+    "tq_attention", "tq_quantize_scatter",
 ]
 
 
@@ -48,6 +48,7 @@ _sig = {
     "tq_packed_sizes": (_i32, [_vp, _i64, ctypes.POINTER(_sz), ctypes.POINTER(_sz)]),
     "tq_get_params": (_i32, [_vp, _vp, _vp, _vp, _vp]),
     "tq_quantize": (_i32, [_vp, _vp, _i32, _i64, _i64, _Packed, _vp]),
+    "tq_quantize_scatter": (_i32, [_vp, _vp, _i32, _i64, _i64, _vp, _i64, _Packed, _vp]),
     "tq_logits_workspace_bytes": (_sz, [_vp, _i64, _i32]),
     "tq_logits": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _i64, _vp, _vp, _sz, _vp]),
     "tq_logits_noalloc": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _i64, _vp, _vp]),
@@ -246,6 +247,16 @@ class TurboQuant:
                "tq_dequant")
         return out
 
+
+    def quantize_scatter(self, x, dest_rows, cache: Packed, stream=None) -> Packed:
+        """Append: row i of x [N, d] (bf16/fp32 CUDA tensor) goes to packed row
+        dest_rows[i] (int64 CUDA tensor) of ``cache``."""
+        import torch
+        assert x.dim() == 2 and x.stride(1) == 1
+        assert dest_rows.dtype == torch.int64 and dest_rows.is_contiguous() and dest_rows.numel() == x.shape[0]
+        _check(_lib.tq_quantize_scatter(self._h, _ptr(x), _dtype_code(x), x.shape[0], x.stride(0), _ptr(dest_rows),
+                                        cache.n_rows, cache.c(), _stream(stream)), "tq_quantize_scatter")
+        return cache
 
     def attention_workspace_bytes(self, n_sets: int, g: int, n_keys: int) -> int:
         return int(_lib.tq_attention_workspace_bytes(self._h, n_sets, g, n_keys))

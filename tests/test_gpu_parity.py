@@ -298,3 +298,42 @@ def test_attention_argument_errors(tq):
         T.attention(q, pk, pk, 1, 4, 0)                  # no keys
     out = torch.empty((0, 128), dtype=torch.float32, device="cuda")
     T.attention(q, pk, pk, 0, 4, 10, out=out)            # no sets: no-op
+
+
+@pytest.mark.parametrize("d,b,m,n", [(128, 3, 128, 256), (128, 4, 128, 32), (64, 2, 96, 77), (1024, 4, 1024, 9)])
+def test_quantize_scatter_into_paged_cache(tq, d, b, m, n):
+    """Append n new rows into a 1000-row packed cache at scattered slots: the
+    slots hold what the oracle packs for those rows, every other slot keeps
+    its previous contents byte for byte."""
+    P = op.Params(d, b, m, seed=0)
+    xt, x = make_rows(d, n, "bf16", seed=d + n)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    cache = T.empty_packed(1000, "cuda")
+    for f in ("codes", "signs"):
+        getattr(cache, f).fill_(0xA5)
+    cache.norm.fill_(-1.0)
+    cache.rnorm.fill_(-2.0)
+    before = cache.to_numpy()
+    slots = np.random.default_rng(n).choice(1000, size=n, replace=False)
+    T.quantize_scatter(xt.cuda(), torch.from_numpy(slots.astype(np.int64)).cuda(), cache)
+    T.sync_status()
+    after = cache.to_numpy()
+    want = ot.quantize(x, P, keep_intermediates=True)
+    got = {k: after[k][slots] for k in ("codes", "signs", "norm", "rnorm")}
+    parity.assert_quantize_ok(parity.compare_quantize(P, got, want))
+    untouched = np.setdiff1d(np.arange(1000), slots)
+    for k in ("codes", "signs", "norm", "rnorm"):
+        assert np.array_equal(after[k][untouched], before[k][untouched]), k
+
+
+def test_quantize_scatter_rejects_out_of_range_slot(tq):
+    T = tq.TurboQuant(128, 3, 128, seed=0)
+    cache = T.empty_packed(10, "cuda")
+    cache.norm.fill_(-1.0)
+    x = torch.ones((2, 128), dtype=torch.bfloat16, device="cuda")
+    T.quantize_scatter(x, torch.tensor([3, 10], dtype=torch.int64, device="cuda"), cache)
+    with pytest.raises(tq.TQError):
+        T.sync_status()
+    norm = cache.norm.cpu().numpy()
+    assert norm[3] > 0 and np.all(np.delete(norm, 3) == -1.0)
+    T.sync_status()                                      # the record was cleared
