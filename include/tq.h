@@ -79,12 +79,18 @@ typedef struct {
 /* ---------------------------------------------------------------- setup -- */
 
 /* Derive the method's fixed parameters on the host, without any CUDA call.
- *   d     power of two in [32, 4096]; b in [2, 5] (b-1 MSE bits + 1 QJL bit);
+ *   d     row length in [32, 4096]; b in [2, 5] (b-1 MSE bits + 1 QJL bit);
  *   m     multiple of 32 in [32, 4096]; seed any 64-bit value.
+ * A d that is not a power of two is zero-padded to D' = the next power of two
+ * (0h-n0 "ICLR 2026論文解説: TurboQuant", "実装のポイント": the randomized
+ * Hadamard rotation needs a power-of-two length); every parameter, and the
+ * packed format, is that of D' (D' = d otherwise).  Rows and queries keep d
+ * elements on the way in, dequantized rows and attention outputs have d on
+ * the way out.
  * Outputs (host arrays, any may be NULL):
  *   centroids[2^(b-1)] ascending fp32 Lloyd-Max levels for one rotated coordinate,
  *   thresholds[2^(b-1)-1] fp32 midpoints,
- *   D[d] int8 +-1 (Rademacher diagonal), S_bits[m*d] binary16 bit patterns of
+ *   D[D'] int8 +-1 (Rademacher diagonal), S_bits[m*D'] binary16 bit patterns of
  *   the Gaussian projection, row-major (row j = projection j).
  * The codebook is the Lloyd-Max fixed point for the exact law of a coordinate
  * of a uniform unit vector, f_d(x) ~ (1-x^2)^((d-3)/2) (ai.spot.hk,
@@ -112,7 +118,8 @@ tq_status tq_get_params(const tq_ctx* ctx, float* centroids, float* thresholds, 
 /* ---------------------------------------------------------- write half -- */
 
 /* Quantize n_rows rows of x (row r at x + r * ld_x elements, dtype bf16 or
- * fp32, ld_x >= d, x and ld_x * element size 16-byte aligned) into `out`.
+ * fp32, ld_x >= d; x and ld_x * element size 16-byte aligned when d is a
+ * power of two, x aligned to its element size otherwise) into `out`.
  * Per row: norm, rotation, Lloyd-Max codes, QJL signs of the residual,
  * residual norm (write half above).  One launch. */
 tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,

@@ -128,6 +128,7 @@ k_attn_chunk(const KParams P, const float* __restrict__ logits, const Packed val
       if (x < d) {
         const int bit = B * x, wi = bit >> 5, sh = bit & 31;
         const bool one_word = (32 % B) == 0;                    // codes never straddle two words
+#pragma unroll 8
         for (int r = 0; r < nb; ++r) {
           const uint32_t* cr = sCodes + r * (cw32 + 1);
           uint32_t code;
@@ -145,6 +146,7 @@ k_attn_chunk(const KParams P, const float* __restrict__ logits, const Packed val
         }
       } else if (x < nx) {
         const int j = x - d;
+#pragma unroll 8
         for (int r = 0; r < nb; ++r) {
           const uint32_t bitv = (sSigns[r * sw32 + (j >> 5)] >> (j & 31)) & 1u;
           const float z = bitv ? -1.f : 1.f;
@@ -232,10 +234,10 @@ k_attn_finalize(const KParams P, const float* __restrict__ partial, int n_chunks
     }
     __syncthreads();
   }
-  for (int i = tid; i < d; i += kAttnThreads) {
+  for (int i = tid; i < P.d_in; i += kAttnThreads) {         // the caller's coordinates only
     const bool neg = (P.Dmask[i >> 5] >> (i & 31)) & 1u;
     const float v = sa[i] * P.inv_sqrt_d;
-    out[rowq * d + i] = neg ? -v : v;
+    out[rowq * P.d_in + i] = neg ? -v : v;
   }
 }
 

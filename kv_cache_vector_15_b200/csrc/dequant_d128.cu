@@ -400,6 +400,7 @@ int launch_B(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int
 }  // namespace
 
 bool dequant_d128_applies(const tq_ctx& ctx, int64_t n_rows) {
+  if (ctx.d_in != ctx.d) return false;                   // padded rows use the general kernel
   const KParams& P = ctx.kp;
   return P.d == kD && P.m == kM && P.B >= 1 && P.B <= 4 && n_rows > 0 && n_rows < (int64_t(1) << 31) &&
          ctx.use_tc && tensor_map_encoder() != nullptr;

@@ -150,6 +150,7 @@ extern "C" tq_status tq_host_params(int d, int b, int m, uint64_t seed, float* c
                                     int8_t* D, uint16_t* S_bits) {
   tq_status st = tq::check_dims(d, b, m);
   if (st != TQ_OK) return st;
+  d = tq::padded_dim(d);                      // parameters of the padded dimension
   if (centroids || thresholds) {
     std::vector<double> c, t;
     tq::lloyd_max(d, b - 1, c, t);

@@ -121,7 +121,10 @@ k_quantize_warp(const KParams P, const void* __restrict__ x, int64_t n_rows, int
     uint32_t* signs_out = reinterpret_cast<uint32_t*>(out.signs + orow * P.signs_bytes);
     float v[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) v[e] = load_elem<BF16>(x, row * ld + lane * E + e);
+    for (int e = 0; e < E; ++e) {
+      const int col = lane * E + e;                          // zero padding beyond the caller's row
+      v[e] = col < P.d_in ? load_elem<BF16>(x, row * ld + col) : 0.f;
+    }
     float ss = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) ss = fmaf(v[e], v[e], ss);
@@ -194,7 +197,10 @@ k_qprep_warp(const KParams P, const void* __restrict__ q, int64_t n_q, float* __
        row += static_cast<int64_t>(gridDim.x) * kWarps) {
     float v[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) v[e] = load_elem<BF16>(q, row * d + lane * E + e);
+    for (int e = 0; e < E; ++e) {
+      const int col = lane * E + e;                          // queries are zero-padded like keys
+      v[e] = col < P.d_in ? load_elem<BF16>(q, row * P.d_in + col) : 0.f;
+    }
     apply_D<E>(v, P.Dmask, lane);
     warp_fwht<E>(v, lane, d);
     float* dst = qp + row * (d + m);
@@ -409,9 +415,12 @@ k_dequant_warp(const KParams P, const Packed in, int64_t n_rows, void* __restric
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const float o = v[e] * P.inv_sqrt_d;
-      const int64_t idx = row * d + lane * E + e;
-      if (BF16OUT) reinterpret_cast<__nv_bfloat16*>(outv)[idx] = __float2bfloat16_rn(o);
-      else reinterpret_cast<float*>(outv)[idx] = o;
+      const int col = lane * E + e;                          // the caller's coordinates only
+      const int64_t idx = row * P.d_in + col;
+      if (col < P.d_in) {
+        if (BF16OUT) reinterpret_cast<__nv_bfloat16*>(outv)[idx] = __float2bfloat16_rn(o);
+        else reinterpret_cast<float*>(outv)[idx] = o;
+      }
     }
   }
 }

@@ -1,6 +1,6 @@
 // Write half at d = 128, m = 128 on sm_100a: TMA-staged rows, the
-// randomized Hadamard rotation and Lloyd-Max bucketing in registers (one
-// thread per row), and the QJL projection S r on the tcgen05 tensor cores.
+// randomized Hadamard rotation, Lloyd-Max bucketing, and the QJL projection
+// S r on the tcgen05 tensor cores.
 //
 // Method (page title, section):
 //   n = ||x||, y = H_d D x / (n sqrt(d))      0h-n0.github.io "ICLR 2026論文解説:
@@ -9,13 +9,19 @@
 //                                             "Stage 1: PolarQuant" (Lloyd-Max)
 //   bit_j = [ (S r)_j < 0 ], rnorm = n ||r||    Qiita explainer, "Stage 2: QJL"
 //
-// CTA layout (persistent, one CTA per SM): two warpgroups, each with its own
-// stage buffer.  Warpgroup w handles every other 128-row tile; thread t of the
-// warpgroup owns row t of the tile, which is also TMEM lane t, so the
-// projection result comes back to the thread that owns the row.  As soon as
-// all its threads have read a tile into registers, the warpgroup's first
-// thread issues the TMA load of its next tile into the same stage, so the
-// load overlaps the rest of the tile's work.
+// CTA layout (persistent, one CTA per SM): two pairs of warpgroups, each pair
+// on one 128-row tile at a time; thread t of warp w in half h of a pair owns
+// coordinates [64h, 64h + 64) (and projections [64h, 64h + 64)) of row
+// 32 (w % 4) + t, which is also the row's TMEM lane, so tensor-core results
+// come back to the threads that own the row.  Rows arrive by TMA, a tile or
+// two ahead.  Two kernels:
+//   k_quantize_d128_rot_tc  bf16 rows: the rotation itself is an MMA whose A
+//                           operand is the TMA stage and B = D H (+-1), then
+//                           codes / residual on the CUDA cores, then the
+//                           projection MMA;
+//   k_quantize_d128_tc      fp32 rows: the rotation in registers (five FWHT
+//                           stages, the stride-64 stage through the TMEM lane),
+//                           then the same codes and projection MMA.
 //
 // Projection precision: S is binary16 by definition (exact in the MMA).  The
 // residual, scaled by 64, is split r = hi + lo into two binary16 parts
@@ -98,12 +104,6 @@ constexpr size_t quant_smem_bytes() {
 __device__ __forceinline__ void flag_error(int* err, int* abort_flag, int code) {
   if (err) atomicCAS(err, 0, code);
   atomicExch(abort_flag, 1);
-}
-
-// bf16 pair in one 32-bit word -> two floats (exact)
-__device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi) {
-  lo = __uint_as_float(w << 16);
-  hi = __uint_as_float(w & 0xffff0000u);
 }
 
 // Two warpgroups ("halves") share every 128-row tile: thread t of warp w in
@@ -885,20 +885,19 @@ int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, cons
   X.err = P.err;
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
   const int grid = static_cast<int>(n_tiles < ctx.num_sms ? n_tiles : ctx.num_sms);
-  if (BF16IN) {
+  if constexpr (BF16IN) {                // bf16 rows: the rotation on the tensor cores
     const size_t smem = quant_rot_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(k_quantize_d128_rot_tc<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
     k_quantize_d128_rot_tc<B><<<grid, kThreads, smem, s>>>(tmap, P, X, n_rows, out);
-    count_launch();
-    return static_cast<int>(cudaGetLastError());
+  } else {                                // fp32 rows: the rotation in registers
+    const size_t smem = quant_smem_bytes<false>();
+    cudaError_t e = cudaFuncSetAttribute(k_quantize_d128_tc<B, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+    k_quantize_d128_tc<B, false><<<grid, kThreads, smem, s>>>(tmap, P, X, n_rows, out);
   }
-  const size_t smem = quant_smem_bytes<BF16IN>();
-  cudaError_t e = cudaFuncSetAttribute(k_quantize_d128_tc<B, BF16IN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return static_cast<int>(e);
-  k_quantize_d128_tc<B, BF16IN><<<grid, kThreads, smem, s>>>(tmap, P, X, n_rows, out);
   count_launch();
   return static_cast<int>(cudaGetLastError());
 }
@@ -906,6 +905,7 @@ int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, cons
 }  // namespace
 
 bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows) {
+  if (ctx.d_in != ctx.d) return false;                   // padded rows use the general kernel
   const KParams& P = ctx.kp;
   return P.d == kD && P.m == kM && P.B >= 1 && P.B <= 4 && n_rows > 0 && n_rows < (int64_t(1) << 31) &&
          ctx.use_tc && get_encode() != nullptr;

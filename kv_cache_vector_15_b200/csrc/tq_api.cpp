@@ -26,9 +26,14 @@ tq_status fail(tq_status s, const std::string& why) {
 
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
+int padded_dim(int d) {
+  int p = 1;
+  while (p < d) p <<= 1;
+  return p;
+}
+
 tq_status check_dims(int d, int b, int m) {
-  if (d < 32 || d > 4096 || (d & (d - 1)))
-    return fail(TQ_ERR_INVALID_ARG, "d must be a power of two in [32, 4096]");
+  if (d < 32 || d > 4096) return fail(TQ_ERR_INVALID_ARG, "d must be in [32, 4096]");
   if (b < 2 || b > 5) return fail(TQ_ERR_INVALID_ARG, "b must be in [2, 5]");
   if (m < 32 || m > 4096 || (m % 32)) return fail(TQ_ERR_INVALID_ARG, "m must be a multiple of 32 in [32, 4096]");
   return TQ_OK;
@@ -121,6 +126,11 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
 
   tq_ctx* ctx = new (std::nothrow) tq_ctx();
   if (!ctx) return fail(TQ_ERR_NOMEM, "host allocation failed");
+  // a row length that is not a power of two is zero-padded to the next one
+  // (0h-n0 "ICLR 2026論文解説: TurboQuant", "実装のポイント"): the rotation, the
+  // codebook, D, S and the packed format are those of the padded dimension
+  ctx->d_in = d;
+  d = padded_dim(d);
   ctx->d = d; ctx->b = b; ctx->m = m; ctx->seed = seed; ctx->device = dev;
   const int B = b - 1, L = 1 << B;
   ctx->centroids.resize(L);
@@ -157,6 +167,7 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
   KParams& kp = ctx->kp;
   std::memset(&kp, 0, sizeof(kp));
   kp.d = d; kp.m = m; kp.B = B; kp.L = L;
+  kp.d_in = ctx->d_in;
   kp.codes_bytes = d * B / 8;
   kp.signs_bytes = m / 8;
   kp.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
@@ -239,9 +250,13 @@ tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_
   if (n_rows == 0) return TQ_OK;
   if (!x) return fail(TQ_ERR_INVALID_ARG, "x is NULL");
   const size_t esz = x_dtype == TQ_BF16 ? 2 : 4;
-  if (ld_x < ctx->d) return fail(TQ_ERR_INVALID_ARG, "ld_x < d");
-  if (!aligned(x, 16) || (static_cast<size_t>(ld_x) * esz) % 16)
-    return fail(TQ_ERR_INVALID_ARG, "x and its row stride must be 16-byte aligned");
+  if (ld_x < ctx->d_in) return fail(TQ_ERR_INVALID_ARG, "ld_x < d");
+  if (ctx->d_in == ctx->d) {
+    if (!aligned(x, 16) || (static_cast<size_t>(ld_x) * esz) % 16)
+      return fail(TQ_ERR_INVALID_ARG, "x and its row stride must be 16-byte aligned");
+  } else if (!aligned(x, esz)) {        // padded rows are read element by element
+    return fail(TQ_ERR_INVALID_ARG, "x must be aligned to its element size");
+  }
   if ((st = check_packed(ctx, out)) != TQ_OK) return st;
   int err = launch_quantize(*ctx, x, x_dtype == TQ_BF16, n_rows, ld_x, to_internal(out), stream);
   if (err) return cuda_fail(err, "tq_quantize launch");
@@ -257,9 +272,8 @@ tq_status tq_quantize_scatter(const tq_ctx* ctx, const void* x, tq_dtype x_dtype
   if (n_rows == 0) return TQ_OK;
   if (!x || !dest_rows) return fail(TQ_ERR_INVALID_ARG, "x or dest_rows is NULL");
   const size_t esz = x_dtype == TQ_BF16 ? 2 : 4;
-  if (ld_x < ctx->d) return fail(TQ_ERR_INVALID_ARG, "ld_x < d");
-  if (!aligned(x, 16) || (static_cast<size_t>(ld_x) * esz) % 16)
-    return fail(TQ_ERR_INVALID_ARG, "x and its row stride must be 16-byte aligned");
+  if (ld_x < ctx->d_in) return fail(TQ_ERR_INVALID_ARG, "ld_x < d");
+  if (!aligned(x, esz)) return fail(TQ_ERR_INVALID_ARG, "x must be aligned to its element size");
   if (!aligned(dest_rows, 8)) return fail(TQ_ERR_INVALID_ARG, "dest_rows must be 8-byte aligned");
   if ((st = check_packed(ctx, cache)) != TQ_OK) return st;
   int err = launch_quantize_scatter(ctx->kp, x, x_dtype == TQ_BF16, n_rows, ld_x, dest_rows, n_cache_rows,

@@ -15,7 +15,8 @@ constexpr float kZeroNorm = 1e-10f; // rows with ||x|| below this are stored as 
 
 // Everything a kernel needs about one parameter set, passed by value.
 struct KParams {
-  int d, m, B, L;
+  int d, m, B, L;                     // d: the rotation dimension (a power of two)
+  int d_in;                           // the caller's row length (<= d; rows are zero-padded to d)
   int codes_bytes, signs_bytes;       // per row
   float inv_sqrt_d;                   // 1/sqrt(d), fp32
   float qjl_scale;                    // sqrt(pi/2) / m, fp32
@@ -35,6 +36,7 @@ struct Packed {
 };
 
 tq_status check_dims(int d, int b, int m);
+int padded_dim(int d);                // the next power of two >= d
 tq_status fail(tq_status s, const std::string& why);   // records tq_last_error()
 void count_launch(int n = 1);
 
@@ -88,7 +90,8 @@ int launch_dequant_d128(const tq_ctx& ctx, const Packed& in, int64_t n_rows, voi
 }  // namespace tq
 
 struct tq_ctx {
-  int d, b, m;
+  int d, b, m;                        // d: padded (power-of-two) dimension
+  int d_in;                           // the caller's row length
   uint64_t seed;
   int device;
   int num_sms;

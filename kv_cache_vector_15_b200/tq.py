@@ -88,15 +88,17 @@ def launch_count() -> int:
 
 def host_params(d: int, b: int, m: int, seed: int = 0):
     """Parameters derived on the host (no CUDA): centroids, thresholds (fp32),
-    D (int8), S (binary16 as numpy float16, [m, d])."""
+    D (int8), S (binary16 as numpy float16, [m, d']), where d' is d padded to
+    the next power of two."""
     L = 1 << (b - 1)
+    dp = 1 << (d - 1).bit_length() if d > 0 else 0
     c = np.zeros(L, np.float32)
     t = np.zeros(L - 1, np.float32)
-    D = np.zeros(d, np.int8)
-    S = np.zeros(m * d, np.uint16)
+    D = np.zeros(max(dp, 1), np.int8)
+    S = np.zeros(max(m * dp, 1), np.uint16)
     _check(_lib.tq_host_params(d, b, m, seed & (2**64 - 1), c.ctypes.data, t.ctypes.data, D.ctypes.data,
                                S.ctypes.data), "tq_host_params")
-    return c, t, D, S.view(np.float16).reshape(m, d)
+    return c, t, D, S.view(np.float16).reshape(m, dp)
 
 
 def _ptr(t) -> int:
@@ -156,6 +158,8 @@ class TurboQuant:
 
     def __init__(self, d: int, b: int, m: int, seed: int = 0):
         self.d, self.b, self.m, self.seed = d, b, m, seed
+        # rows of a length that is not a power of two are zero-padded to the next one
+        self.d_pad = 1 << (d - 1).bit_length()
         h = _vp()
         _check(_lib.tq_init(d, b, m, seed & (2**64 - 1), ctypes.byref(h)), "tq_init")
         self._h = h
@@ -186,11 +190,11 @@ class TurboQuant:
         L = 1 << (self.b - 1)
         c = np.zeros(L, np.float32)
         t = np.zeros(L - 1, np.float32)
-        D = np.zeros(self.d, np.int8)
-        S = np.zeros(self.m * self.d, np.uint16)
+        D = np.zeros(self.d_pad, np.int8)
+        S = np.zeros(self.m * self.d_pad, np.uint16)
         _check(_lib.tq_get_params(self._h, c.ctypes.data, t.ctypes.data, D.ctypes.data, S.ctypes.data),
                "tq_get_params")
-        return c, t, D, S.view(np.float16).reshape(self.m, self.d)
+        return c, t, D, S.view(np.float16).reshape(self.m, self.d_pad)
 
     def empty_packed(self, n_rows: int, device="cuda") -> Packed:
         import torch

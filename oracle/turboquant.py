@@ -31,7 +31,11 @@ Readings taken where the pages are silent:
     positive (bit 0); bit 1 means negative, as in the 0h-n0 encoder sketch;
   * codes are an LSB-first bitstream per row, code i in bits [B i, B i + B);
     sign j is bit (j mod 8) of byte j // 8;
-  * the logit carries no 1/sqrt(d) softmax scale.
+  * the logit carries no 1/sqrt(d) softmax scale;
+  * a row length d that is not a power of two is zero-padded to the next
+    power of two (``padded_dim``, ``pad_rows``); every parameter and the
+    packed format are those of the padded length, and reconstructed rows are
+    read back in their first d coordinates.
 """
 
 from __future__ import annotations
@@ -95,6 +99,22 @@ def rotate_inverse(v: np.ndarray, P) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Packing
 # --------------------------------------------------------------------------
+def padded_dim(d: int) -> int:
+    """The power of two a row of length d is zero-padded to before the
+    rotation [0h-n0 "ICLR 2026論文解説: TurboQuant", "実装のポイント": RHT needs
+    a power-of-two dimension; pad with zeros up to the nearest one above]."""
+    p = 1
+    while p < d:
+        p *= 2
+    return p
+
+
+def pad_rows(x: np.ndarray, d_pad: int) -> np.ndarray:
+    """Rows of x (..., d) with d_pad - d zero coordinates appended."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.concatenate([x, np.zeros(x.shape[:-1] + (d_pad - x.shape[-1],))], axis=-1)
+
+
 def packed_sizes(d: int, b: int, m: int):
     """Bytes per row: codes d (b-1) / 8, signs m / 8, plus two fp32 norms."""
     return d * (b - 1) // 8, m // 8

@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 
 from oracle import params as op
+from oracle import turboquant as ot
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -38,10 +39,13 @@ def test_library_exports_every_declared_symbol():
 
 
 @pytest.mark.parametrize("d,b,m,seed", [(32, 2, 32, 0), (128, 2, 128, 0), (128, 3, 128, 0), (128, 4, 128, 7),
-                                        (256, 5, 96, 3), (1024, 4, 1024, 0), (4096, 3, 64, 11)])
+                                        (256, 5, 96, 3), (1024, 4, 1024, 0), (4096, 3, 64, 11), (100, 3, 128, 0),
+                                        (3072, 4, 128, 5)])
 def test_host_params_equal_oracle(d, b, m, seed):
+    """A d that is not a power of two gets the parameters of the padded length."""
     tq = _lib()
     c, t, D, S = tq.host_params(d, b, m, seed)
+    d = ot.padded_dim(d)
     P = op.Params(d, b, m, seed)
     assert np.array_equal(D, P.D)
     assert np.array_equal(S.astype(np.float64), P.S)           # binary16 bit-exact
@@ -50,7 +54,7 @@ def test_host_params_equal_oracle(d, b, m, seed):
     assert np.max(np.abs(c.astype(np.float64) - P.centroids64)) < 1e-7 / np.sqrt(d) * 4
 
 
-@pytest.mark.parametrize("d,b,m", [(16, 3, 128), (100, 3, 128), (8192, 3, 128), (128, 1, 128), (128, 6, 128),
+@pytest.mark.parametrize("d,b,m", [(16, 3, 128), (31, 3, 128), (8192, 3, 128), (128, 1, 128), (128, 6, 128),
                                    (128, 3, 100), (128, 3, 0), (128, 3, 8192)])
 def test_bad_dims_rejected(d, b, m):
     tq = _lib()

@@ -337,3 +337,47 @@ def test_quantize_scatter_rejects_out_of_range_slot(tq):
     norm = cache.norm.cpu().numpy()
     assert norm[3] > 0 and np.all(np.delete(norm, 3) == -1.0)
     T.sync_status()                                      # the record was cleared
+
+
+@pytest.mark.parametrize("d,b,m", [(96, 3, 128), (100, 4, 128), (200, 3, 64), (3072, 4, 128)])
+def test_padded_dimension_end_to_end(tq, d, b, m):
+    """A row length that is not a power of two: the library pads rows and
+    queries with zeros to the next power of two, and dequant / attention give
+    back the first d coordinates -- compared with the oracle on explicitly
+    padded inputs."""
+    dp = ot.padded_dim(d)
+    P = op.Params(dp, b, m, seed=0)
+    n_sets, g, n_keys = 2, 3, 700
+    # random rows only: the structured edge rows put whole groups of rotated
+    # coordinates within 1e-6 of a threshold once padded (exempt, but counted)
+    rng = np.random.default_rng(d)
+    xs = (rng.standard_normal((n_sets * n_keys, d)) * rng.uniform(0.1, 10, size=(n_sets * n_keys, 1)))
+    bits = inputs.bf16_bits(xs.astype(np.float32))
+    xt = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    x = inputs.bf16_to_f32(bits)
+    qt, q = make_rows(d, n_sets * g, "bf16", seed=d + 1)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    pk = T.quantize(xt.cuda())
+    got = pk.to_numpy()
+    T.sync_status()
+    want = ot.quantize(ot.pad_rows(x, dp), P, keep_intermediates=True)
+    parity.assert_quantize_ok(parity.compare_quantize(P, got, want))
+    po = {k: want[k] for k in ("codes", "signs", "norm", "rnorm")}
+    keys = tq.Packed.from_numpy(po)
+    lg = T.logits(qt.cuda(), keys, n_sets, g, n_keys).cpu().numpy()
+    lw = ot.logits(ot.pad_rows(q, dp), po, P, n_sets, g, n_keys)
+    tol = parity.logit_tolerance(q, np.linalg.norm(x, axis=1), n_sets, g, n_keys)
+    assert np.all(np.abs(lg - lw) <= tol + 1e-30)
+    dq = T.dequant(keys, out_dtype=torch.float32).cpu().numpy()
+    assert dq.shape == (n_sets * n_keys, d)
+    parity.assert_dequant_ok(dq, ot.dequant(po, P)[:, :d], bf16=False)
+    if dp + m > 2048:                                    # beyond tq_attention's shapes
+        with pytest.raises(tq.TQError):
+            T.attention(qt.cuda(), keys, keys, n_sets, g, n_keys)
+        return
+    att = T.attention(qt.cuda(), keys, keys, n_sets, g, n_keys).cpu().numpy()
+    aw = ot.attention(ot.pad_rows(q, dp), po, po, P, n_sets, g, n_keys, 1.0 / np.sqrt(d), logits_in=lg)
+    aw = aw.reshape(n_sets * g, dp)[:, :d]
+    vscale = np.abs(ot.dequant(po, P)).max()
+    assert att.shape == (n_sets * g, d)
+    assert np.max(np.abs(att - aw)) <= 1e-4 * vscale

@@ -328,3 +328,17 @@ def test_attention_is_invariant_to_key_order_and_weights_sum_to_one():
     w /= w.sum()
     assert abs(w.sum() - 1.0) < 1e-15
     assert np.allclose(a[0, 0], w @ ot.dequant(pv, P), atol=1e-12)
+
+
+def test_padding_to_a_power_of_two():
+    """Zero padding changes neither the norm nor any inner product, and the
+    padded rotation keeps the padded vector's length: the padded quantizer sees
+    the same geometry as the original row."""
+    assert [ot.padded_dim(d) for d in (32, 33, 96, 100, 128, 3072, 4096)] == [32, 64, 128, 128, 128, 4096, 4096]
+    rng = np.random.default_rng(1)
+    x, y = rng.standard_normal((2, 100))
+    px, py = ot.pad_rows(x, 128), ot.pad_rows(y, 128)
+    assert px.shape == (128,) and np.all(px[100:] == 0) and np.array_equal(px[:100], x)
+    assert np.isclose(px @ py, x @ y, rtol=1e-14)
+    P = op.Params(128, 3, 128, seed=0)
+    assert np.isclose(np.linalg.norm(ot.rotate(px[None, :], P)), np.linalg.norm(x), rtol=1e-13)
