@@ -93,92 +93,119 @@ __device__ __forceinline__ void apply_D(float (&v)[E], const uint32_t* Dmask, in
 // ---------------------------------------------------------------------------
 // dest: when not null, input row i goes to packed row dest[i] (a paged cache);
 // an index outside [0, n_dest) is not written and sets the error word (7).
-template <int E, bool BF16>
+// Each warp takes R rows at a time and projects them together, so that every
+// S^T element read from L2 feeds R multiply-adds (R = 1 for a handful of rows,
+// where latency matters more than L2 traffic).
+template <int E, bool BF16, int R>
 __global__ void __launch_bounds__(kWarps * 32)
 k_quantize_warp(const KParams P, const void* __restrict__ x, int64_t n_rows, int64_t ld, const Packed out,
                 const int64_t* __restrict__ dest, int64_t n_dest) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int d = P.d, m = P.m, B = P.B;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  float* rs = reinterpret_cast<float*>(smem_raw) + wib * d;                       // residual
-  uint8_t* cs = smem_raw + static_cast<size_t>(kWarps) * d * 4 + wib * d;         // codes
+  float* rs = reinterpret_cast<float*>(smem_raw) + static_cast<size_t>(wib) * R * d;        // [R][d] residuals
+  uint8_t* cs = smem_raw + static_cast<size_t>(kWarps) * R * d * 4 + static_cast<size_t>(wib) * d;   // codes
   __shared__ float thr[kMaxLevels], lut[kMaxLevels];
   if (threadIdx.x < kMaxLevels) { thr[threadIdx.x] = P.t[threadIdx.x]; lut[threadIdx.x] = P.c[threadIdx.x]; }
   __syncthreads();
 
   const int nwords_codes = d * B / 32, nwords_signs = m / 32;
-  for (int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + wib; row < n_rows;
-       row += static_cast<int64_t>(gridDim.x) * kWarps) {
-    int64_t orow = row;
-    if (dest) {
-      orow = __ldg(dest + row);
-      if (orow < 0 || orow >= n_dest) {                      // warp-uniform: skip the row, flag it
-        if (lane == 0 && P.err) atomicCAS(P.err, 0, 7);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarps;
+  for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * kWarps + wib; row0 < n_rows; row0 += stride * R) {
+    int64_t orows[R];
+    bool live[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t row = row0 + r * stride;
+      live[r] = false;
+      orows[r] = row;
+      if (row >= n_rows) continue;                             // warp-uniform
+      int64_t orow = row;
+      if (dest) {
+        orow = __ldg(dest + row);
+        if (orow < 0 || orow >= n_dest) {                      // warp-uniform: skip the row, flag it
+          if (lane == 0 && P.err) atomicCAS(P.err, 0, 7);
+          continue;
+        }
+      }
+      orows[r] = orow;
+      uint32_t* codes_out = reinterpret_cast<uint32_t*>(out.codes + orow * P.codes_bytes);
+      uint32_t* signs_out = reinterpret_cast<uint32_t*>(out.signs + orow * P.signs_bytes);
+      float v[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int col = lane * E + e;                          // zero padding beyond the caller's row
+        v[e] = col < P.d_in ? load_elem<BF16>(x, row * ld + col) : 0.f;
+      }
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) ss = fmaf(v[e], v[e], ss);
+      ss = warp_sum(ss);
+      const float n = sqrtf(ss);
+      if (!(n >= kZeroNorm)) {                   // zero row (or a non-finite norm)
+        for (int w = lane; w < nwords_codes; w += 32) codes_out[w] = 0u;
+        for (int w = lane; w < nwords_signs; w += 32) signs_out[w] = 0u;
+        if (lane == 0) { out.norm[orow] = 0.f; out.rnorm[orow] = 0.f; }
         continue;
       }
-    }
-    uint32_t* codes_out = reinterpret_cast<uint32_t*>(out.codes + orow * P.codes_bytes);
-    uint32_t* signs_out = reinterpret_cast<uint32_t*>(out.signs + orow * P.signs_bytes);
-    float v[E];
+      apply_D<E>(v, P.Dmask, lane);
+      warp_fwht<E>(v, lane, d);
+      const float inv_n = 1.0f / n;
+      float r2 = 0.f;
+      float* rr = rs + r * d;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int col = lane * E + e;                          // zero padding beyond the caller's row
-      v[e] = col < P.d_in ? load_elem<BF16>(x, row * ld + col) : 0.f;
-    }
-    float ss = 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) ss = fmaf(v[e], v[e], ss);
-    ss = warp_sum(ss);
-    const float n = sqrtf(ss);
-    if (!(n >= kZeroNorm)) {                   // zero row (or a non-finite norm)
-      for (int w = lane; w < nwords_codes; w += 32) codes_out[w] = 0u;
-      for (int w = lane; w < nwords_signs; w += 32) signs_out[w] = 0u;
-      if (lane == 0) { out.norm[orow] = 0.f; out.rnorm[orow] = 0.f; }
-      continue;
-    }
-    apply_D<E>(v, P.Dmask, lane);
-    warp_fwht<E>(v, lane, d);
-    const float inv_n = 1.0f / n;
-    float r2 = 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const float y = (v[e] * inv_n) * P.inv_sqrt_d;
-      int code = 0;
-      for (int k = 0; k < P.L - 1; ++k) code += (y > thr[k]) ? 1 : 0;
-      const float r = y - lut[code];
-      rs[lane * E + e] = r;
-      cs[lane * E + e] = static_cast<uint8_t>(code);
-      r2 = fmaf(r, r, r2);
-    }
-    r2 = warp_sum(r2);
-    __syncwarp();
-    // codes: output word w holds stream bits [32w, 32w + 32)
-    for (int w = lane; w < nwords_codes; w += 32) {
-      uint32_t acc = 0;
-      const int i0 = (32 * w) / B, i1 = (32 * w + 31) / B;
-      for (int i = i0; i <= i1 && i < d; ++i) {
-        const int sh = B * i - 32 * w;
-        const uint32_t c = cs[i];
-        acc |= sh >= 0 ? (c << sh) : (c >> (-sh));
+      for (int e = 0; e < E; ++e) {
+        const float y = (v[e] * inv_n) * P.inv_sqrt_d;
+        int code = 0;
+        for (int k = 0; k < P.L - 1; ++k) code += (y > thr[k]) ? 1 : 0;
+        const float res = y - lut[code];
+        rr[lane * E + e] = res;
+        cs[lane * E + e] = static_cast<uint8_t>(code);
+        r2 = fmaf(res, res, r2);
       }
-      codes_out[w] = acc;
+      r2 = warp_sum(r2);
+      __syncwarp();
+      // codes: output word w holds stream bits [32w, 32w + 32)
+      for (int w = lane; w < nwords_codes; w += 32) {
+        uint32_t acc = 0;
+        const int i0 = (32 * w) / B, i1 = (32 * w + 31) / B;
+        for (int i = i0; i <= i1 && i < d; ++i) {
+          const int sh = B * i - 32 * w;
+          const uint32_t c = cs[i];
+          acc |= sh >= 0 ? (c << sh) : (c >> (-sh));
+        }
+        codes_out[w] = acc;
+      }
+      if (lane == 0) { out.norm[orow] = n; out.rnorm[orow] = n * sqrtf(r2); }
+      live[r] = true;
+      __syncwarp();
     }
-    // QJL: p_j = sum_i S[j][i] r_i, bit j = [p_j < 0]; lane handles j = 32 t + lane
+    // QJL: p_j = sum_i S[j][i] r_i, bit j = [p_j < 0]; lane handles j = 32 t + lane,
+    // for the R rows at once (rows that are not live compute on stale data and
+    // store nothing)
     for (int t = 0; t < nwords_signs; ++t) {
       const int j = 32 * t + lane;
-      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < d; i += 4) {
-        p0 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i) * m + j)), rs[i], p0);
-        p1 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i + 1) * m + j)), rs[i + 1], p1);
-        p2 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i + 2) * m + j)), rs[i + 2], p2);
-        p3 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i + 3) * m + j)), rs[i + 3], p3);
+      float p[R][2];
+#pragma unroll
+      for (int r = 0; r < R; ++r) p[r][0] = p[r][1] = 0.f;
+#pragma unroll (R == 1 ? 16 : 4)
+      for (int i = 0; i < d; i += 2) {
+        const float s0 = half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i) * m + j));
+        const float s1 = half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i + 1) * m + j));
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const float2 rv = *reinterpret_cast<const float2*>(rs + r * d + i);
+          p[r][0] = fmaf(s0, rv.x, p[r][0]);
+          p[r][1] = fmaf(s1, rv.y, p[r][1]);
+        }
       }
-      const float p = (p0 + p1) + (p2 + p3);
-      const uint32_t bits = __ballot_sync(0xffffffffu, p < 0.f);
-      if (lane == 0) signs_out[t] = bits;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const uint32_t bits = __ballot_sync(0xffffffffu, (p[r][0] + p[r][1]) < 0.f);
+        if (live[r] && lane == 0)
+          reinterpret_cast<uint32_t*>(out.signs + orows[r] * P.signs_bytes)[t] = bits;
+      }
     }
-    if (lane == 0) { out.norm[orow] = n; out.rnorm[orow] = n * sqrtf(r2); }
     __syncwarp();
   }
 }
@@ -281,35 +308,45 @@ k_logits_rowkey(const KParams P, const float* __restrict__ qp, int64_t n_keys, c
 }
 
 // ---------------------------------------------------------------------------
-// logits, large g: 64 keys x 32 queries per CTA, 4 x 2 outputs per thread.
-// The combined dimension d + m is walked in chunks of 32; each chunk of key
+// logits, large g: 128 keys x 128 queries per CTA, 8 x 8 outputs per thread
+// (register tiling: four shared-memory vector loads feed 64 FMAs).  The
+// combined dimension d + m is walked in chunks of 16; each chunk of key
 // values is decoded once per CTA into shared memory as norm*c[code] (MSE
 // coordinates) or rnorm*sqrt(pi/2)/m*z (QJL coordinates).
 // ---------------------------------------------------------------------------
-constexpr int TK = 64, TQ = 32, KC = 32;
+constexpr int TK = 128, TQ = 128, KC = 16;
 
 __global__ void __launch_bounds__(256)
 k_logits_tiled(const KParams P, const float* __restrict__ qp, int g, int64_t n_keys, const Packed keys,
                float* __restrict__ out) {
-  __shared__ float Ks[KC][TK + 4];
-  __shared__ float Qs[KC][TQ + 4];
+  __shared__ __align__(16) float Ks[KC][TK];
+  __shared__ __align__(16) float Qs[KC][TQ];
   __shared__ float lut[kMaxLevels];
   const int d = P.d, m = P.m, dm = d + m, B = P.B;
   const int64_t set = blockIdx.z;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * TK;
   const int q0 = blockIdx.y * TQ;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  if (threadIdx.x < kMaxLevels) lut[threadIdx.x] = P.c[threadIdx.x];
-  float acc[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-  // the key this thread decodes in each chunk and its scales
-  const int dk = threadIdx.x & (TK - 1), dc0 = (threadIdx.x >> 6) * 8;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  if (tid < kMaxLevels) lut[tid] = P.c[tid];
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  // the key this thread decodes (8 coordinates of each chunk) and its scales
+  const int dk = tid & (TK - 1), dc0 = (tid >> 7) * 8;
   const int64_t krow = set * n_keys + k0 + dk;
   const bool kvalid = (k0 + dk) < n_keys;
   float knorm = 0.f, krn = 0.f;
   if (kvalid) { knorm = keys.norm[krow]; krn = keys.rnorm[krow] * P.qjl_scale; }
+  const uint8_t* cb = keys.codes + krow * P.codes_bytes;
+  const uint8_t* sbp = keys.signs + krow * P.signs_bytes;
+  // the query this thread stages (8 coordinates of each chunk)
+  const int ql = tid & (TQ - 1);
+  const bool qvalid = q0 + ql < g;
+  const float* qrow = qp + (set * g + q0 + ql) * dm;
   __syncthreads();
   for (int kk = 0; kk < dm; kk += KC) {
-    // decode 8 coordinates of key dk
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int c = kk + dc0 + u;
@@ -317,50 +354,50 @@ k_logits_tiled(const KParams P, const float* __restrict__ qp, int g, int64_t n_k
       if (kvalid) {
         if (c < d) {
           const int bit = B * c, by = bit >> 3, sh = bit & 7;
-          const uint8_t* cb = keys.codes + krow * P.codes_bytes;
           uint32_t win = cb[by];
           if (sh + B > 8) win |= static_cast<uint32_t>(cb[by + 1]) << 8;
           val = knorm * lut[(win >> sh) & ((1u << B) - 1u)];
         } else {
           const int j = c - d;
-          const uint8_t sb = keys.signs[krow * P.signs_bytes + (j >> 3)];
-          val = ((sb >> (j & 7)) & 1u) ? -krn : krn;
+          val = ((sbp[j >> 3] >> (j & 7)) & 1u) ? -krn : krn;
         }
       }
       Ks[dc0 + u][dk] = val;
     }
-    // stage 32 queries x 32 coordinates
+    if (qvalid) {
+      const float4 a = *reinterpret_cast<const float4*>(qrow + kk + dc0);
+      const float4 b = *reinterpret_cast<const float4*>(qrow + kk + dc0 + 4);
+      Qs[dc0 + 0][ql] = a.x; Qs[dc0 + 1][ql] = a.y; Qs[dc0 + 2][ql] = a.z; Qs[dc0 + 3][ql] = a.w;
+      Qs[dc0 + 4][ql] = b.x; Qs[dc0 + 5][ql] = b.y; Qs[dc0 + 6][ql] = b.z; Qs[dc0 + 7][ql] = b.w;
+    } else {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int e = threadIdx.x + u * 256;         // 0..1023
-      const int qq = e >> 5, c = e & 31;
-      const int qi = q0 + qq;
-      Qs[c][qq] = (qi < g) ? qp[(set * g + qi) * dm + kk + c] : 0.f;
+      for (int u = 0; u < 8; ++u) Qs[dc0 + u][ql] = 0.f;
     }
     __syncthreads();
-#pragma unroll 8
+#pragma unroll
     for (int c = 0; c < KC; ++c) {
-      float a[4], b[2];
+      const float4 ka = *reinterpret_cast<const float4*>(&Ks[c][tx * 4]);
+      const float4 kb = *reinterpret_cast<const float4*>(&Ks[c][64 + tx * 4]);
+      const float4 qa = *reinterpret_cast<const float4*>(&Qs[c][ty * 4]);
+      const float4 qb = *reinterpret_cast<const float4*>(&Qs[c][64 + ty * 4]);
+      const float kv[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+      const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = Ks[c][tx * 4 + i];
-      b[0] = Qs[c][ty * 2];
-      b[1] = Qs[c][ty * 2 + 1];
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[i][0] = fmaf(a[i], b[0], acc[i][0]);
-        acc[i][1] = fmaf(a[i], b[1], acc[i][1]);
-      }
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(kv[i], qv[j], acc[i][j]);
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int qi = q0 + ty * 2 + j;
+  for (int j = 0; j < 8; ++j) {
+    const int qi = q0 + (j < 4 ? ty * 4 + j : 64 + ty * 4 + (j - 4));
     if (qi >= g) continue;
+    float* orow = out + (set * g + qi) * n_keys;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int64_t kt = k0 + tx * 4 + i;
-      if (kt < n_keys) out[(set * g + qi) * n_keys + kt] = acc[i][j];
+    for (int i = 0; i < 8; ++i) {
+      const int64_t kt = k0 + (i < 4 ? tx * 4 + i : 64 + tx * 4 + (i - 4));
+      if (kt < n_keys) orow[kt] = acc[i][j];
     }
   }
 }
@@ -558,19 +595,28 @@ int grid_rows(int64_t n_rows) {
   return static_cast<int>(want < cap ? want : cap);
 }
 
+template <int E, bool BF16, int R>
+int launch_quantize_ER(const KParams& P, const void* x, int64_t n_rows, int64_t ld, const Packed& out,
+                       cudaStream_t s, const int64_t* dest, int64_t n_dest) {
+  const size_t smem = static_cast<size_t>(kWarps) * P.d * (4 * R + 1);
+  const int g = grid_rows((n_rows + R - 1) / R);
+  int err;
+  if ((err = set_smem(k_quantize_warp<E, BF16, R>, smem))) return err;
+  k_quantize_warp<E, BF16, R><<<g, kWarps * 32, smem, s>>>(P, x, n_rows, ld, out, dest, n_dest);
+  return 0;
+}
+
 template <int E>
 int launch_quantize_E(const KParams& P, const void* x, int bf16, int64_t n_rows, int64_t ld, const Packed& out,
                       cudaStream_t s, const int64_t* dest = nullptr, int64_t n_dest = 0) {
-  const size_t smem = static_cast<size_t>(kWarps) * P.d * 5;
-  int g = grid_rows(n_rows);
+  // four rows per warp when there are many rows and their residuals fit
+  const bool four = n_rows >= 65536 && P.d <= 1024;
   int err;
-  if (bf16) {
-    if ((err = set_smem(k_quantize_warp<E, true>, smem))) return err;
-    k_quantize_warp<E, true><<<g, kWarps * 32, smem, s>>>(P, x, n_rows, ld, out, dest, n_dest);
-  } else {
-    if ((err = set_smem(k_quantize_warp<E, false>, smem))) return err;
-    k_quantize_warp<E, false><<<g, kWarps * 32, smem, s>>>(P, x, n_rows, ld, out, dest, n_dest);
-  }
+  if (bf16) err = four ? launch_quantize_ER<E, true, 4>(P, x, n_rows, ld, out, s, dest, n_dest)
+                       : launch_quantize_ER<E, true, 1>(P, x, n_rows, ld, out, s, dest, n_dest);
+  else err = four ? launch_quantize_ER<E, false, 4>(P, x, n_rows, ld, out, s, dest, n_dest)
+                  : launch_quantize_ER<E, false, 1>(P, x, n_rows, ld, out, s, dest, n_dest);
+  if (err) return err;
   count_launch();
   return static_cast<int>(cudaGetLastError());
 }

@@ -501,7 +501,7 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
                        int64_t n_rows, const Packed out) {
   constexpr int L = 1 << B;
   constexpr int kStage = XStage<true>::kBytes;                  // 32 KB: two 64-column boxes
-  constexpr int NS = 2;
+  constexpr int NS = XStage<true>::kStages;                     // two stages per pair
   constexpr int kH = kD / 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
