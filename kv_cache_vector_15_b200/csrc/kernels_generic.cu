@@ -33,6 +33,7 @@ namespace tq {
 namespace {
 
 constexpr int kWarps = 8;           // warps per CTA in the warp-per-row kernels
+constexpr size_t kQprepStBytes = 64 * 1024;   // S^T staged in shared memory up to this size
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -132,10 +133,15 @@ k_quantize_warp(const KParams P, const void* __restrict__ x, int64_t n_rows, int
       uint32_t* codes_out = reinterpret_cast<uint32_t*>(out.codes + orow * P.codes_bytes);
       uint32_t* signs_out = reinterpret_cast<uint32_t*>(out.signs + orow * P.signs_bytes);
       float v[E];
+      if (P.d_in != d) {
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const int col = lane * E + e;                          // zero padding beyond the caller's row
-        v[e] = col < P.d_in ? load_elem<BF16>(x, row * ld + col) : 0.f;
+        for (int e = 0; e < E; ++e) {
+          const int col = lane * E + e;                        // zero padding beyond the caller's row
+          v[e] = col < P.d_in ? load_elem<BF16>(x, row * ld + col) : 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[e] = load_elem<BF16>(x, row * ld + lane * E + e);
       }
       float ss = 0.f;
 #pragma unroll
@@ -220,13 +226,30 @@ k_qprep_warp(const KParams P, const void* __restrict__ q, int64_t n_q, float* __
   const int d = P.d, m = P.m;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   float* qs = reinterpret_cast<float*>(smem_raw) + wib * d;
+  // S^T in shared memory when it is small (all warps of the CTA share it),
+  // else read from L2
+  const bool st_smem = static_cast<size_t>(d) * m * 2 <= kQprepStBytes;
+  uint16_t* sst = reinterpret_cast<uint16_t*>(smem_raw + static_cast<size_t>(kWarps) * d * 4);
+  if (st_smem) {
+    const int n16 = d * m / 8;                                 // 16-byte pieces
+    for (int e = threadIdx.x; e < n16; e += kWarps * 32)
+      reinterpret_cast<uint4*>(sst)[e] = __ldg(reinterpret_cast<const uint4*>(P.St) + e);
+    __syncthreads();
+  }
+  const uint16_t* st = st_smem ? sst : P.St;
+  const bool padded = P.d_in != d;
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + wib; row < n_q;
        row += static_cast<int64_t>(gridDim.x) * kWarps) {
     float v[E];
+    if (padded) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int col = lane * E + e;                          // queries are zero-padded like keys
-      v[e] = col < P.d_in ? load_elem<BF16>(q, row * P.d_in + col) : 0.f;
+      for (int e = 0; e < E; ++e) {
+        const int col = lane * E + e;                          // queries are zero-padded like keys
+        v[e] = col < P.d_in ? load_elem<BF16>(q, row * P.d_in + col) : 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[e] = load_elem<BF16>(q, row * d + lane * E + e);
     }
     apply_D<E>(v, P.Dmask, lane);
     warp_fwht<E>(v, lane, d);
@@ -242,8 +265,8 @@ k_qprep_warp(const KParams P, const void* __restrict__ q, int64_t n_q, float* __
       float a0 = 0.f, a1 = 0.f;
 #pragma unroll 16
       for (int i = 0; i < d; i += 2) {
-        a0 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i) * m + j)), qs[i], a0);
-        a1 = fmaf(half_bits_to_float(__ldg(P.St + static_cast<int64_t>(i + 1) * m + j)), qs[i + 1], a1);
+        a0 = fmaf(half_bits_to_float(st[static_cast<int64_t>(i) * m + j]), qs[i], a0);
+        a1 = fmaf(half_bits_to_float(st[static_cast<int64_t>(i + 1) * m + j]), qs[i + 1], a1);
       }
       dst[d + j] = a0 + a1;
     }
@@ -623,7 +646,8 @@ int launch_quantize_E(const KParams& P, const void* x, int bf16, int64_t n_rows,
 
 template <int E>
 int launch_qprep_E(const KParams& P, const void* q, int bf16, int64_t n_q, float* qp, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(kWarps) * P.d * 4;
+  const size_t st_bytes = static_cast<size_t>(P.d) * P.m * 2;
+  const size_t smem = static_cast<size_t>(kWarps) * P.d * 4 + (st_bytes <= kQprepStBytes ? st_bytes : 0);
   int g = grid_rows(n_q);
   int err;
   if (bf16) {

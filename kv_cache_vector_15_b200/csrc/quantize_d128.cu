@@ -577,26 +577,30 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
     if (t_first + t_step < n_tiles) { issue_load(t_first + t_step, 1); ++issued[1]; }
   }
 
+  // the rotation MMA of this pair's k-th tile (leader only): waits for its stage
+  auto issue_rotation = [&](int k) {
+    const int b = k & 1;
+    if (mbar_wait(&pfull[b], (k >> 1) & 1, kWaitCycles)) ++waited[b];
+    else flag_error(X.err, abort_flag, 2);
+    tc_fence_after();
+    const uint32_t xbase = smem_u32(stages + b * kStage), hbase = smem_u32(sHD);
+    const uint32_t idesc = idesc_bf16_f32(kTile, kD);
+    const uint32_t d_tmem = tmem + pair * 256;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+      mma_f16_ss(d_tmem, smem_desc_sw128(xbase + off, 1024), smem_desc_sw128(hbase + off, 1024), idesc,
+                 kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&ydone[pair]);
+  };
+  // each tile's rotation is issued as soon as the previous tile's accumulator
+  // has been read (below), so it runs under that tile's stores
+  if (leader && t_first < n_tiles) issue_rotation(0);
+
   int mine = 0;
   for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
     const int buf = mine & 1;
-    // #A: the previous tile's accumulator reads are done (and a uniform abort check)
-    if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
-    if (leader) {
-      if (mbar_wait(&pfull[buf], (mine >> 1) & 1, kWaitCycles)) ++waited[buf];
-      else flag_error(X.err, abort_flag, 2);
-      tc_fence_after();
-      const uint32_t xbase = smem_u32(stages + buf * kStage), hbase = smem_u32(sHD);
-      const uint32_t idesc = idesc_bf16_f32(kTile, kD);
-      const uint32_t d_tmem = tmem + pair * 256;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-        mma_f16_ss(d_tmem, smem_desc_sw128(xbase + off, 1024), smem_desc_sw128(hbase + off, 1024), idesc,
-                   k > 0 ? 1u : 0u);
-      }
-      mma_commit(&ydone[pair]);
-    }
     if (!mbar_wait(&ydone[pair], mine & 1, kWaitCycles)) flag_error(X.err, abort_flag, 5);
     tc_fence_after();
 
@@ -807,6 +811,10 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
     }
     if (zero_row || rho == 0.f) s0 = s1 = 0u;
     tc_fence_before();
+    // #A: every read of this tile's accumulator and operand columns is done
+    // (and a uniform abort check): the next tile's rotation may start
+    if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
+    if (leader && t + t_step < n_tiles) issue_rotation(mine + 1);
     const int64_t row = t * kTile + trow;
     if (row < n_rows) {
       uint32_t* co = reinterpret_cast<uint32_t*>(out.codes + row * (B * 16) + half * (B * 8));
