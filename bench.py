@@ -52,6 +52,8 @@ AUX_WORKLOADS = {
     "prefill-b4": dict(kind="prefill", b=4, m=128, d=128),
     # vector search: 1e6 x 1024 fp32 database, 1024 queries, b = 4, m = 1024, top-10
     "vsearch": dict(kind="vsearch", b=4, m=1024, d=1024),
+    # the same on a 131072-row database (0.5 GB, above L2) for profiler captures
+    "vsearch-128k": dict(kind="vsearch", b=4, m=1024, d=1024, n=131072),
     # decode-time append: one new token of a 32-layer x 8-KV-head model (256 K rows
     # and 256 V rows) scattered into a paged packed cache, latency per token
     "append-b3": dict(kind="append", b=3, m=128, d=128),
@@ -88,6 +90,17 @@ def peaks():
     return 6650.0, "fallback"
 
 
+def tensor_peak():
+    """Dense fp16/bf16 tensor peak (TFLOP/s) for a kernel timed inside a long
+    step: the sustained measurement, else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        if "bf16_tflops_sustained" in j:
+            return float(j["bf16_tflops_sustained"]), "measured (sustained)"
+    return 1400.0, "fallback (sustained)"
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason sampling during the timed region."""
 
@@ -109,6 +122,13 @@ class ClockSampler:
                  "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
+        # wait for the first sample: nvidia-smi's start-up (driver queries) must
+        # not overlap the timed region, where it can delay kernel launches
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < 5.0:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
         time.sleep(0.3)
         return self
 
@@ -551,7 +571,7 @@ def run_aux(args, cfg, ws, rank, local):
         alg = 2 * n_tok_rows * (2 * d + P)
         kern = "step"
     else:
-        db, qs = inputs.vector_search()
+        db, qs = inputs.vector_search(n=cfg.get("n", 1_000_000))
         nq, ndb = qs.n_rows, db.n_rows
         hdb = torch.empty((ndb, d), dtype=torch.float32)
         db.fill(hdb.numpy())
@@ -562,10 +582,21 @@ def run_aux(args, cfg, ws, rank, local):
         scores = torch.empty((1, nq, ndb), dtype=torch.float32, device=dev)
         work = torch.empty(max(T.workspace_bytes(1, nq), 16), dtype=torch.uint8, device=dev)
 
-        def step():
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        split = {"quantize": 0.0, "logits": 0.0, "topk": 0.0}
+
+        def step(timed=False):
+            if timed: ev[0].record(stream)
             T.quantize(ddb, pk, stream=stream)
+            if timed: ev[1].record(stream)
             T.logits(dq, pk, 1, nq, ndb, out=scores, workspace=work, stream=stream)
+            if timed: ev[2].record(stream)
             tq.topk(scores[0], 10, stream=stream)
+            if timed:
+                ev[3].record(stream)
+                ev[3].synchronize()
+                for i, k in enumerate(split):
+                    split[k] += ev[i].elapsed_time(ev[i + 1])
         units, unit, metric = nq * ndb, "IP estimates/s", "vector search: quantize DB, all-pairs IP estimates, top-10"
         alg = ndb * (4 * d + P) + ndb * P + 2 * nq * ndb * 4
         kern = "step"
@@ -584,20 +615,37 @@ def run_aux(args, cfg, ws, rank, local):
         barrier(ws)
     ms = max_over_ranks(ws, e0.elapsed_time(e1)) / args.steps
     total = dist_util.sum_over_ranks(ws, units, device=dev)
+    launches = tq.launch_count() - launches0
     graph_ms = None
     if cfg["kind"] == "append":
         graph_ms = append_graph_ms(torch, T, dev, stream, dk, dv, slots, cK, cV, args.steps)
+    gbs = alg / (ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": kern, "achieved": gbs, "peak": hbm, "unit": "GB/s",
+            "frac": gbs / hbm, "traffic": None, "algorithmic_bytes": alg, "peak_kind": hbm_kind}
+    phases = None
+    if cfg["kind"] == "vsearch":
+        # per-phase device times in separate steps (events between the calls),
+        # outside the timed region; the estimates are a dense contraction:
+        # 2 nq ndb (d + m) algorithmic flops (the fp16 hi/lo form executes
+        # 2 nq ndb (3 d + 2 m)), against the sustained tensor peak
+        for _ in range(args.steps):
+            step(timed=True)
+        phases = {k: v / args.steps for k, v in split.items()}
+        tf, tf_kind = tensor_peak()
+        flops = 2.0 * nq * ndb * (d + m)
+        ach = flops / (phases["logits"] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "logits (estimates, incl. key / query operand prep)", "achieved": ach,
+                "peak": tf, "unit": "TFLOP/s", "frac": ach / tf, "traffic": None, "algorithmic_flops": flops,
+                "executed_flops": 2.0 * nq * ndb * (3 * d + 2 * m), "peak_kind": tf_kind}
     if rank == 0:
-        gbs = alg / (ms * 1e-3) / 1e9
         print(json.dumps({
             "metric": metric, "value": total / (ms * 1e-3), "unit": unit, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": args.workload, "d": d, "b": b, "m": m, "l2": "inputs larger than L2; no flush"},
-            "roofline": {"bound": "hbm", "kernel": kern, "achieved": gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": gbs / hbm, "traffic": None, "algorithmic_bytes": alg, "peak_kind": hbm_kind},
+            "roofline": roof, "phases_ms": phases,
             "cuda_graph_ms_per_step": graph_ms,
-            "gpu_launches": tq.launch_count() - launches0, "clocks": clk.summary()}), flush=True)
+            "gpu_launches": launches, "clocks": clk.summary()}), flush=True)
     T.close()
 
 

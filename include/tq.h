@@ -27,7 +27,12 @@
  *   - Tensor pointers are DEVICE pointers owned by the caller, unless a
  *     parameter says "host".  The library never frees them.
  *   - Compute calls are asynchronous on the CUDA stream passed as `stream`
- *     (a cudaStream_t; NULL = legacy default stream) and allocate nothing.
+ *     (a cudaStream_t; NULL = legacy default stream) and allocate nothing,
+ *     except tq_quantize and tq_logits on wide rows (d >= 256, at least 4096
+ *     rows or keys), which take stream-ordered scratch on `stream` from a
+ *     memory pool the context owns (cudaMallocFromPoolAsync / cudaFreeAsync;
+ *     the pool keeps the memory between calls and is released by tq_destroy);
+ *     a failed scratch allocation returns TQ_ERR_CUDA.
  *   - Arguments are checked on the host before any launch.  A failed check
  *     returns a status and launches nothing; tq_last_error() then gives a
  *     one-line reason (thread-local, valid until the next call on the thread).
@@ -121,7 +126,11 @@ tq_status tq_get_params(const tq_ctx* ctx, float* centroids, float* thresholds, 
  * fp32, ld_x >= d; x and ld_x * element size 16-byte aligned when d is a
  * power of two, x aligned to its element size otherwise) into `out`.
  * Per row: norm, rotation, Lloyd-Max codes, QJL signs of the residual,
- * residual norm (write half above).  One launch. */
+ * residual norm (write half above).  One launch at d = 128 and for small
+ * batches.  Wide rows (d >= 256, n_rows >= 4096) run per 18944-row chunk: a
+ * CUDA-core kernel (norm, rotation, codes, residual halves), a tensor-core
+ * GEMM for the projections and their signs, and a fix-up of the rare
+ * projections inside the GEMM's error bound (recomputed in fp64). */
 tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
                       tq_packed out, void* stream);
 
@@ -153,7 +162,9 @@ size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g);
  * number of query heads sharing it; for vector search n_sets = 1 and g the
  * number of queries.  g in [1, 4096].  workspace: device memory of at least
  * tq_logits_workspace_bytes(ctx, n_sets, g) bytes, 16-byte aligned, not used
- * concurrently by another call. */
+ * concurrently by another call.  With d >= 256, m a multiple of 64, g >= 64
+ * and n_keys >= 4096 the estimates run as a tensor-core GEMM over keys
+ * decoded into binary16 operands, 18944 keys at a time. */
 tq_status tq_logits(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
                     tq_packed keys, int64_t n_keys, float* out, void* workspace, size_t workspace_bytes,
                     void* stream);
@@ -224,7 +235,9 @@ tq_status tq_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g,
 const char* tq_status_str(tq_status s);
 /* Wait for `stream`, then report whether any kernel of this context timed out
  * in one of its bounded device-side waits since the last check (TQ_ERR_CUDA,
- * outputs of that call invalid), or met an out-of-range destination row in
+ * outputs of that call invalid), found more projections inside the wide-row
+ * GEMM's error bound than its fix-up list holds (TQ_ERR_CUDA, some signs not
+ * recomputed), or met an out-of-range destination row in
  * tq_quantize_scatter (TQ_ERR_INVALID_ARG), and clear the record.  Blocking. */
 tq_status tq_sync_status(const tq_ctx* ctx, void* stream);
 /* One-line reason for the last non-OK status returned on this host thread. */

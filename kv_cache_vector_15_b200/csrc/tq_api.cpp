@@ -65,7 +65,7 @@ static tq_status check_packed(const tq_ctx* ctx, const tq_packed& p) {
 
 static Packed to_internal(const tq_packed& p) { return Packed{p.codes, p.signs, p.norm, p.rnorm}; }
 
-static double half_bits_to_double(uint16_t h) {
+double half_bits_to_double(uint16_t h) {
   const int sign = (h >> 15) & 1, e = (h >> 10) & 31, f = h & 1023;
   double v = e == 0 ? std::ldexp(static_cast<double>(f), -24) : std::ldexp(static_cast<double>(1024 + f), e - 25);
   return sign ? -v : v;
@@ -104,6 +104,8 @@ tq_status tq_sync_status(const tq_ctx* ctx, void* stream) {
     cudaMemcpy(ctx->kp.err, &zero, sizeof(int), cudaMemcpyHostToDevice);
     if (word == 7) return fail(TQ_ERR_INVALID_ARG, "tq_quantize_scatter: a destination row index was out of range "
                                                    "(that row was not written)");
+    if (word == 8) return fail(TQ_ERR_CUDA, "tq_quantize: more projections than expected fell inside the tensor-core "
+                                            "error bound; some sign bits were not recomputed");
     return fail(TQ_ERR_CUDA, "a kernel wait ran out of time (code " + std::to_string(word) + "); outputs are invalid");
   }
   return TQ_OK;
@@ -139,7 +141,8 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
   ctx->S_bits.resize(static_cast<size_t>(m) * d);
   tq_host_params(d, b, m, seed, ctx->centroids.data(), ctx->thresholds.data(), ctx->D.data(), ctx->S_bits.data());
 
-  // device block, 256-byte aligned parts: error word | Dmask (d/32 words) | S [m][d] | St [d][m]
+  // device block, 256-byte aligned parts: error word | Dmask (d/32 words) | S [m][d] | St [d][m] |
+  // ||S_j||_2 [m]
   auto round256 = [](size_t v) { return (v + 255) / 256 * 256; };
   const size_t n_mask = static_cast<size_t>(d) / 32;
   const size_t sz_S = static_cast<size_t>(m) * d * sizeof(uint16_t);
@@ -147,7 +150,8 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
   const size_t off_mask = 256;
   const size_t off_S2 = off_mask + round256(n_mask * 4);
   const size_t off_St = off_S2 + round256(sz_S);
-  const size_t total = off_St + round256(sz_S);
+  const size_t off_sn = off_St + round256(sz_S);
+  const size_t total = off_sn + round256(static_cast<size_t>(m) * 4);
   void* blk = nullptr;
   e = cudaMalloc(&blk, total);
   if (e != cudaSuccess) { delete ctx; return fail(TQ_ERR_NOMEM, std::string("cudaMalloc: ") + cudaGetErrorString(e)); }
@@ -161,6 +165,19 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
   uint16_t* St = reinterpret_cast<uint16_t*>(host.data() + off_St);
   for (int j = 0; j < m; ++j)
     for (int i = 0; i < d; ++i) St[static_cast<size_t>(i) * m + j] = ctx->S_bits[static_cast<size_t>(j) * d + i];
+  float* snorm = reinterpret_cast<float*>(host.data() + off_sn);
+  double smax = 0.0, s1max = 0.0;                      // max_j ||S_j||_2 and max_j ||S_j||_1
+  for (int j = 0; j < m; ++j) {
+    double acc = 0.0, acc1 = 0.0;
+    for (int i = 0; i < d; ++i) {
+      const double v = half_bits_to_double(ctx->S_bits[static_cast<size_t>(j) * d + i]);
+      acc += v * v;
+      acc1 += std::fabs(v);
+    }
+    snorm[j] = static_cast<float>(std::sqrt(acc) * (1.0 + 1e-6));   // rounded up
+    smax = std::max(smax, std::sqrt(acc));
+    s1max = std::max(s1max, acc1);
+  }
   e = cudaMemcpy(blk, host.data(), total, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) { cudaFree(blk); delete ctx; return cuda_fail(e, "cudaMemcpy"); }
 
@@ -190,17 +207,8 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
   // a further margin; the tensor-core error measured over 10^6 projections
   // peaks at 1.7 * 2^-22 ||S_j|| ||r||), plus max_j ||S_j||_1 * 2^-25 / 64 for
   // binary16 underflow of the scaled residual
-  double smax = 0.0, s1max = 0.0;
-  for (int j = 0; j < m; ++j) {
-    double acc = 0.0, acc1 = 0.0;
-    for (int i = 0; i < d; ++i) {
-      const double v = half_bits_to_double(ctx->S_bits[static_cast<size_t>(j) * d + i]);
-      acc += v * v;
-      acc1 += std::fabs(v);
-    }
-    smax = std::max(smax, std::sqrt(acc));
-    s1max = std::max(s1max, acc1);
-  }
+  ctx->s1max = s1max;
+  ctx->snorm_dev = reinterpret_cast<const float*>(static_cast<uint8_t*>(blk) + off_sn);
   ctx->qjl_eps_scale = static_cast<float>(16.0 * std::ldexp(1.0, -22) * smax);
   ctx->qjl_eps_abs = static_cast<float>(2.0 * s1max * std::ldexp(1.0, -25) / 64.0);
   for (int i = 0; i < 128; ++i) ctx->colsum_d128[i] = 0.f;
@@ -211,6 +219,23 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
       ctx->colsum_d128[i] = static_cast<float>(acc);
     }
   }
+  // wide rows: a memory pool for the stream-ordered scratch of the tensor-core
+  // paths, kept (not released to the device) between calls
+  ctx->pool = nullptr;
+  if (d >= 256) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) == cudaSuccess) {
+      uint64_t keep = UINT64_MAX;
+      cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+      ctx->pool = pool;
+    } else {
+      cudaGetLastError();                              // the general kernels serve instead
+    }
+  }
   *out = ctx;
   return TQ_OK;
 }
@@ -218,6 +243,8 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
 tq_status tq_destroy(tq_ctx* ctx) {
   if (!ctx) return TQ_OK;
   cudaError_t e = cudaSuccess;
+  // a pool whose stream-ordered frees are still queued is released once they complete
+  if (ctx->pool) cudaMemPoolDestroy(static_cast<cudaMemPool_t>(ctx->pool));
   if (ctx->dev_block) e = cudaFree(ctx->dev_block);
   delete ctx;
   if (e != cudaSuccess) return cuda_fail(e, "cudaFree");

@@ -42,6 +42,7 @@ void count_launch(int n = 1);
 
 // host_params.cpp
 uint16_t double_to_half_bits(double v);
+double half_bits_to_double(uint16_t h);         // (tq_api.cpp) finite values only
 void rademacher(int d, uint64_t seed, int8_t* D);
 void gaussian_projection_half(int m, int d, uint64_t seed, uint16_t* S_bits);
 void lloyd_max(int d, int bits_mse, std::vector<double>& centroids, std::vector<double>& thresholds);
@@ -87,6 +88,13 @@ int launch_logits_d128(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g
                        float* out, void* stream);
 int launch_dequant_d128(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
                         void* stream);
+// wide rows (d >= 256): tensor-core QJL projection and estimates (wide_tc.cu)
+bool wide_quantize_applies(const tq_ctx& ctx, int64_t n_rows);
+int launch_quantize_wide(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
+                         const Packed& out, void* stream);
+bool wide_logits_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys);
+int launch_logits_wide(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
+                       float* out, void* stream);
 }  // namespace tq
 
 struct tq_ctx {
@@ -102,6 +110,9 @@ struct tq_ctx {
   std::vector<float> centroids, thresholds;
   std::vector<int8_t> D;
   std::vector<uint16_t> S_bits;
+  double s1max;                       // max_j ||S_j||_1
+  const float* snorm_dev;             // [m] ||S_j||_2 on the device (in dev_block)
+  void* pool;                         // cudaMemPool_t for stream-ordered scratch (wide rows), or null
   void* dev_block;                    // one allocation holding everything below
   tq::KParams kp;
 };

@@ -386,11 +386,12 @@ def test_padded_dimension_end_to_end(tq, d, b, m):
 @pytest.mark.parametrize("d,b,m,dtype", [(256, 3, 128, "bf16"), (64, 4, 96, "f32"), (1024, 2, 64, "bf16")])
 def test_quantize_general_kernel_many_rows(tq, d, b, m, dtype):
     """The general write half with four rows per warp (taken from 65536 rows
-    on): every row of a ragged last group, and the edge rows."""
+    on): every row of a ragged last group, and the edge rows.  (With the
+    hot-path kernels on, these shapes take the wide-row tensor-core path.)"""
     n = 70001
     xt, x = make_rows(d, n, dtype, seed=d + b)
     P = op.Params(d, b, m, seed=0)
-    T = tq.TurboQuant(d, b, m, seed=0)
+    T = make_ctx(tq, d, b, m, "generic")
     got = T.quantize(xt.cuda()).to_numpy()
     T.sync_status()
     parity.assert_quantize_ok(parity.compare_quantize(P, got, ot.quantize(x, P, keep_intermediates=True)))

@@ -1,0 +1,90 @@
+"""GPU parity of the wide-row tensor-core paths (d >= 256, many rows): the
+QJL projection of the write half as an fp16 GEMM with a listed fp64 fix-up of
+the projections inside its error bound, and the all-pairs estimates as an
+fp16 GEMM over decoded keys and split queries.
+
+Row counts span more than one 18944-row chunk (148 tiles of 128 rows) and end
+in a ragged tile; query counts end in a ragged 256-column tile.  Codes, signs,
+norms and estimates follow the oracle rules of tests/parity.py.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import params as op
+from oracle import turboquant as ot
+from tests import parity
+from tests.test_gpu_parity import edge_rows, make_ctx, make_rows
+
+torch = pytest.importorskip("torch")
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+CHUNK = 148 * 128
+
+
+@pytest.fixture(scope="module")
+def tq():
+    from kv_cache_vector_15_b200 import tq as _tq
+    return _tq
+
+
+@pytest.mark.parametrize("d,b,m,dtype,n", [
+    (256, 3, 256, "f32", 2 * CHUNK + 1001),
+    (256, 2, 96, "bf16", CHUNK + 77),
+    (512, 4, 128, "bf16", 4096),
+    (1024, 4, 1024, "f32", CHUNK + 777),
+    (2048, 3, 64, "bf16", 5000),
+])
+def test_wide_quantize_parity(tq, d, b, m, dtype, n):
+    xt, x = make_rows(d, n, dtype, seed=d + 7 * b + m)
+    P = op.Params(d, b, m, seed=0)
+    T = make_ctx(tq, d, b, m)
+    got = T.quantize(xt.cuda()).to_numpy()
+    T.sync_status()
+    rep = parity.compare_quantize(P, got, ot.quantize(x, P, keep_intermediates=True))
+    parity.assert_quantize_ok(rep)
+
+
+@pytest.mark.parametrize("d,b,m,n_sets,g,n_keys,qdtype", [
+    (256, 3, 256, 2, 300, CHUNK + 513, "f32"),
+    (512, 2, 128, 3, 64, 5000, "bf16"),
+    (1024, 4, 1024, 1, 1024, 4500, "f32"),
+    (256, 5, 64, 1, 257, 4096, "bf16"),
+])
+def test_wide_logits_parity(tq, d, b, m, n_sets, g, n_keys, qdtype):
+    P = op.Params(d, b, m, seed=0)
+    rng = np.random.default_rng(d + g + b)
+    k = rng.standard_normal((n_sets * n_keys, d)) * rng.uniform(0.1, 10, size=(n_sets * n_keys, 1))
+    k[:3] = edge_rows(d, rng)[:3]
+    pk = ot.quantize(k, P)
+    qt, q = make_rows(d, n_sets * g, qdtype, seed=3 * g + b)
+    T = make_ctx(tq, d, b, m)
+    got = T.logits(qt.cuda(), tq.Packed.from_numpy(pk), n_sets, g, n_keys).cpu().numpy()
+    T.sync_status()
+    want = ot.logits(q, pk, P, n_sets, g, n_keys)
+    tol = parity.logit_tolerance(q, np.linalg.norm(k, axis=1), n_sets, g, n_keys)
+    err = np.abs(got - want)
+    assert np.all(err <= tol + 1e-30), float(np.max(err / (tol + 1e-30)))
+
+
+def test_wide_quantize_then_logits_end_to_end(tq):
+    """GPU quantize -> GPU estimates on the wide paths against the oracle's
+    quantize -> estimates; keys whose packed bytes differ (boundary band) are
+    counted, not compared."""
+    d, b, m, g, n_keys = 1024, 4, 1024, 300, 6000
+    P = op.Params(d, b, m, seed=0)
+    kt, k = make_rows(d, n_keys, "f32", seed=21)
+    qt, q = make_rows(d, g, "f32", seed=22)
+    T = make_ctx(tq, d, b, m)
+    pg = T.quantize(kt.cuda())
+    got = T.logits(qt.cuda(), pg, 1, g, n_keys).cpu().numpy()
+    T.sync_status()
+    po = ot.quantize(k, P)
+    want = ot.logits(q, po, P, 1, g, n_keys)
+    png = pg.to_numpy()
+    same = np.all(png["codes"] == po["codes"], axis=1) & np.all(png["signs"] == po["signs"], axis=1)
+    assert np.mean(~same) <= 1e-2
+    tol = parity.logit_tolerance(q, np.linalg.norm(k, axis=1), 1, g, n_keys)
+    ok = (np.abs(got - want) <= tol + 1e-30) | ~same.reshape(1, 1, n_keys)
+    assert ok.all()
