@@ -377,11 +377,11 @@ k_quantize_residual_warp(const KParams P, const void* __restrict__ x, int64_t n_
     // butterflies at distance 1 .. 16 across lanes, then 32 .. d/2 within a lane
 #pragma unroll
     for (int h = 1; h < 32; h <<= 1) {
-      const bool upper = (lane & h) != 0;
+      const float sgn = (lane & h) ? -1.f : 1.f;       // upper lane: partner - own; lower: own + partner
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         const float p = __shfl_xor_sync(0xffffffffu, v[e], h);
-        v[e] = upper ? (p - v[e]) : (v[e] + p);
+        v[e] = fmaf(sgn, v[e], p);                     // exact sign flip, one rounding: as p -/+ v
       }
     }
 #pragma unroll
@@ -660,6 +660,7 @@ bool wide_logits_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_key
 }
 
 int64_t wide_chunk_rows() { return static_cast<int64_t>(kChunkTiles) * kTM; }
+
 
 int launch_quantize_wide(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
                          const Packed& out, void* stream) {
