@@ -54,6 +54,11 @@ AUX_WORKLOADS = {
     "vsearch": dict(kind="vsearch", b=4, m=1024, d=1024),
     # the same on a 131072-row database (0.5 GB, above L2) for profiler captures
     "vsearch-128k": dict(kind="vsearch", b=4, m=1024, d=1024, n=131072),
+    # fractional bit widths: the long-context decode step with each row's 128
+    # channels split 64 / 64 between two instances (2.5 bits: b = 3 / 2;
+    # 3.5 bits: b = 4 / 3)
+    "decode-128k-2.5bit": dict(kind="split", d=128, d_hi=64, b_hi=3, b_lo=2, b=2.5, m=64),
+    "decode-128k-3.5bit": dict(kind="split", d=128, d_hi=64, b_hi=4, b_lo=3, b=3.5, m=64),
     # decode-time append: one new token of a 32-layer x 8-KV-head model (256 K rows
     # and 256 V rows) scattered into a paged packed cache, latency per token
     "append-b3": dict(kind="append", b=3, m=128, d=128),
@@ -529,11 +534,46 @@ def run_aux(args, cfg, ws, rank, local):
 
     d, b, m = cfg["d"], cfg["b"], cfg["m"]
     dev = torch.device("cuda", local)
-    T = tq.TurboQuant(d, b, m, seed=0)
+    if cfg["kind"] == "split":
+        T = tq.TurboQuantSplit(d, cfg["d_hi"], cfg["b_hi"], cfg["b_lo"], seed=0)
+        P = T.row_bytes
+    else:
+        T = tq.TurboQuant(d, b, m, seed=0)
+        P = T.row_bytes
     stream = torch.cuda.current_stream(dev)
     hbm, hbm_kind = peaks()
-    P = T.row_bytes
-    if cfg["kind"] == "prefill":
+    if cfg["kind"] == "split":
+        # the long-context decode step (8 x 8 x 131072 keys and values, GQA 4)
+        # on the split format; each rank takes its slice of the batch
+        batch, ctx, kvh, qh = 8, 131072, 8, 32
+        g = qh // kvh
+        b0, b1 = dist_util.shard(batch, ws, rank)
+        n_sets, n_keys = (b1 - b0) * kvh, ctx
+        N = n_sets * n_keys
+        K, V, Q = inputs.decode(batch, ctx, kv_heads=kvh, q_heads=qh)
+        hK = torch.empty((N, d), dtype=torch.bfloat16)
+        hV = torch.empty((N, d), dtype=torch.bfloat16)
+        hQ = torch.empty((n_sets * g, d), dtype=torch.bfloat16)
+        K.fill(hK.view(torch.int16).numpy().view(np.uint16), start=b0 * kvh * ctx)
+        V.fill(hV.view(torch.int16).numpy().view(np.uint16), start=b0 * kvh * ctx)
+        Q.fill(hQ.view(torch.int16).numpy().view(np.uint16), start=b0 * qh)
+        dK, dV, dQ = hK.to(dev), hV.to(dev), hQ.to(dev)
+        del hK, hV
+        pK, pV = T.empty_packed(N, dev), T.empty_packed(N, dev)
+        lg = torch.empty((n_sets, g, n_keys), dtype=torch.float32, device=dev)
+        vhat = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
+        work = torch.empty(max(T.logits_workspace_bytes(n_sets, g, n_keys), 16), dtype=torch.uint8, device=dev)
+
+        def step():
+            T.quantize(dK, pK, stream=stream)
+            T.quantize(dV, pV, stream=stream)
+            T.logits(dQ, pK, n_sets, g, n_keys, out=lg, workspace=work, stream=stream)
+            T.dequant(pV, N, out=vhat, stream=stream)
+        units, unit = n_sets * g * n_keys, "logits/s"
+        metric = f"compressed-key logits/s, long-context decode step at {b} bits (64 + 64 channel split)"
+        alg = 2 * N * (2 * d + P) + N * (P + 4 * g) + N * (P + 2 * d)
+        kern = "step"
+    elif cfg["kind"] == "prefill":
         K, V = inputs.prefill()
         N = K.n_rows
         lo, hi = dist_util.shard(N, ws, rank)          # each rank quantizes its slice of the rows
@@ -579,26 +619,28 @@ def run_aux(args, cfg, ws, rank, local):
         del hdb
         dq = torch.from_numpy(qs.all()).to(dev)
         pk = T.empty_packed(ndb, dev)
-        scores = torch.empty((1, nq, ndb), dtype=torch.float32, device=dev)
-        work = torch.empty(max(T.workspace_bytes(1, nq), 16), dtype=torch.uint8, device=dev)
-
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        split = {"quantize": 0.0, "logits": 0.0, "topk": 0.0}
+        kq = 10
+        idx = torch.empty((nq, kq), dtype=torch.int32, device=dev)
+        val = torch.empty((nq, kq), dtype=torch.float32, device=dev)
+        work = torch.empty(max(T.search_workspace_bytes(nq, ndb, kq), 16), dtype=torch.uint8, device=dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        split = {"quantize": 0.0, "search": 0.0}
 
         def step(timed=False):
+            # quantize the database, then every query's top-10 by estimated
+            # inner product (estimates on the tensor cores, top-k fused into
+            # their epilogue)
             if timed: ev[0].record(stream)
             T.quantize(ddb, pk, stream=stream)
             if timed: ev[1].record(stream)
-            T.logits(dq, pk, 1, nq, ndb, out=scores, workspace=work, stream=stream)
-            if timed: ev[2].record(stream)
-            tq.topk(scores[0], 10, stream=stream)
+            T.search(dq, pk, ndb, kq, idx=idx, val=val, workspace=work, stream=stream)
             if timed:
-                ev[3].record(stream)
-                ev[3].synchronize()
+                ev[2].record(stream)
+                ev[2].synchronize()
                 for i, k in enumerate(split):
                     split[k] += ev[i].elapsed_time(ev[i + 1])
         units, unit, metric = nq * ndb, "IP estimates/s", "vector search: quantize DB, all-pairs IP estimates, top-10"
-        alg = ndb * (4 * d + P) + ndb * P + 2 * nq * ndb * 4
+        alg = ndb * (4 * d + P) + ndb * P + nq * kq * 8
         kern = "step"
     for _ in range(args.warmup):
         step()
@@ -633,8 +675,8 @@ def run_aux(args, cfg, ws, rank, local):
         phases = {k: v / args.steps for k, v in split.items()}
         tf, tf_kind = tensor_peak()
         flops = 2.0 * nq * ndb * (d + m)
-        ach = flops / (phases["logits"] * 1e-3) / 1e12
-        roof = {"bound": "tensor", "kernel": "logits (estimates, incl. key / query operand prep)", "achieved": ach,
+        ach = flops / (phases["search"] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "search (estimates incl. key / query operands, fused top-10)", "achieved": ach,
                 "peak": tf, "unit": "TFLOP/s", "frac": ach / tf, "traffic": None, "algorithmic_flops": flops,
                 "executed_flops": 2.0 * nq * ndb * (3 * d + 2 * m), "peak_kind": tf_kind}
     if rank == 0:

@@ -215,6 +215,25 @@ tq_status tq_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64
 tq_status tq_dequant(const tq_ctx* ctx, tq_packed in, int64_t n_rows, void* out, tq_dtype out_dtype,
                      tq_dequant_mode mode, void* stream);
 
+/* Vector search: for each of n_q queries, the k packed rows (of n_keys) with
+ * the largest estimated inner product (the tq_logits estimator with
+ * n_sets = 1, g = n_q), larger first, equal estimates by lower row index:
+ * exactly tq_topk over the scores tq_logits would write, without writing
+ * them when the wide-row path applies (d >= 256, m a multiple of 64,
+ * n_q >= 64, n_keys >= 4096): there the estimates GEMM keeps the k largest
+ * of every 128-key tile per query (Google Research blog "TurboQuant:
+ * Redefining AI efficiency with extreme compression", vector search; the
+ * top-k is the search's answer).  Elsewhere the scores go through the
+ * workspace.
+ *   q    [n_q, d] bf16 or fp32, 16-byte aligned; n_q in [0, 4096];
+ *   idx  [n_q, k] int32 row indices; val [n_q, k] fp32 estimates (may be NULL);
+ *   k in [1, 16], k <= n_keys < 2^31;
+ *   workspace: device memory of at least tq_search_workspace_bytes(ctx, n_q,
+ *   n_keys, k) bytes, 16-byte aligned, not used concurrently by another call. */
+size_t tq_search_workspace_bytes(const tq_ctx* ctx, int64_t n_q, int64_t n_keys, int k);
+tq_status tq_search(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_q, tq_packed keys, int64_t n_keys,
+                    int k, int32_t* idx, float* val, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Per row of scores [rows, cols] fp32, the k largest values, larger first,
  * equal values by lower column index first.  idx [rows, k] int32 and
  * val [rows, k] fp32 (val may be NULL).  k in [1, 64], k <= cols. */
@@ -229,6 +248,39 @@ tq_status tq_topk(const float* scores, int64_t rows, int64_t cols, int k, int32_
  * fp32 out [n_sets, g, n_keys].  d in {64, 128, 256}, g in [1, 8], n_sets <= 65535. */
 tq_status tq_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, int d,
                          float* out, void* stream);
+
+/* ------------------------------------------- fractional bit widths -- */
+
+/* A channel split: channels [0, d_hi) of each row are one TurboQuant
+ * instance with b_hi bits per coordinate, channels [d_hi, d) another with
+ * b_lo bits (m = each part's dimension; seeds seed and seed + 1), for
+ * (d_hi b_hi + (d - d_hi) b_lo) / d bits per coordinate: 2.5 bits at
+ * d = 128 as 64 channels at b = 3 and 64 at b = 2, 3.5 bits as 64 at 4 and
+ * 64 at 3.  The pages report 2.5- and 3.5-bit results without the split rule
+ * (inlevel9 "TurboQuantのメモリ圧縮と半導体需要", "TurboQuantが実際に行っていること");
+ * this is the library's reading: the estimate of <q, k> is the sum of the
+ * two parts' estimates (inner products add over disjoint channels, so it
+ * stays unbiased), and the caller picks the channels that get the higher
+ * width by ordering them first.  d_hi and d - d_hi: multiples of 32, >= 32.
+ * The part contexts (tq_split_part) give packed sizes and parameters; each
+ * part has its own packed arrays. */
+typedef struct tq_split tq_split;
+tq_status tq_split_init(int d, int d_hi, int b_hi, int b_lo, uint64_t seed, tq_split** out);
+tq_status tq_split_destroy(tq_split* sp);
+/* part 0 (channels [0, d_hi)) or 1 (channels [d_hi, d)); owned by sp */
+tq_status tq_split_part(const tq_split* sp, int part, const tq_ctx** out);
+/* x [n_rows, ld_x >= d] as tq_quantize; each part's columns into its packed rows. */
+tq_status tq_split_quantize(const tq_split* sp, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
+                            tq_packed out_hi, tq_packed out_lo, void* stream);
+size_t tq_split_logits_workspace_bytes(const tq_split* sp, int64_t n_sets, int g, int64_t n_keys);
+/* As tq_logits, with q [n_sets, g, d] and each part's packed keys; out is the
+ * sum of the two parts' estimates. */
+tq_status tq_split_logits(const tq_split* sp, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
+                          tq_packed keys_hi, tq_packed keys_lo, int64_t n_keys, float* out, void* workspace,
+                          size_t workspace_bytes, void* stream);
+/* Reconstructed rows [n_rows, d] (each part's columns from its packed rows). */
+tq_status tq_split_dequant(const tq_split* sp, tq_packed in_hi, tq_packed in_lo, int64_t n_rows, void* out,
+                           tq_dtype out_dtype, tq_dequant_mode mode, void* stream);
 
 /* ----------------------------------------------------------- reporting -- */
 

@@ -245,11 +245,11 @@ k_qprep_warp(const KParams P, const void* __restrict__ q, int64_t n_q, float* __
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         const int col = lane * E + e;                          // queries are zero-padded like keys
-        v[e] = col < P.d_in ? load_elem<BF16>(q, row * P.d_in + col) : 0.f;
+        v[e] = col < P.d_in ? load_elem<BF16>(q, row * P.ld_q + col) : 0.f;
       }
     } else {
 #pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = load_elem<BF16>(q, row * d + lane * E + e);
+      for (int e = 0; e < E; ++e) v[e] = load_elem<BF16>(q, row * P.ld_q + lane * E + e);
     }
     apply_D<E>(v, P.Dmask, lane);
     warp_fwht<E>(v, lane, d);
@@ -476,13 +476,20 @@ k_dequant_warp(const KParams P, const Packed in, int64_t n_rows, void* __restric
     for (int e = 0; e < E; ++e) {
       const float o = v[e] * P.inv_sqrt_d;
       const int col = lane * E + e;                          // the caller's coordinates only
-      const int64_t idx = row * P.d_in + col;
+      const int64_t idx = row * P.ld_out + col;
       if (col < P.d_in) {
         if (BF16OUT) reinterpret_cast<__nv_bfloat16*>(outv)[idx] = __float2bfloat16_rn(o);
         else reinterpret_cast<float*>(outv)[idx] = o;
       }
     }
   }
+}
+
+// out += in, elementwise (the two halves of a channel split's logits)
+__global__ void __launch_bounds__(256) k_add_f32(float* __restrict__ out, const float* __restrict__ in, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] += in[i];
 }
 
 // ---------------------------------------------------------------------------
@@ -837,6 +844,14 @@ int launch_topk(const float* scores, int64_t rows, int64_t cols, int k, int32_t*
                                                                     val ? val + r0 * k : nullptr);
     count_launch();
   }
+  return static_cast<int>(cudaGetLastError());
+}
+
+int launch_add(float* out, const float* in, int64_t n, void* stream) {
+  if (n <= 0) return 0;
+  const int64_t want = (n + 255) / 256, cap = static_cast<int64_t>(sm_count()) * 8;
+  k_add_f32<<<static_cast<unsigned>(want < cap ? want : cap), 256, 0, static_cast<cudaStream_t>(stream)>>>(out, in, n);
+  count_launch();
   return static_cast<int>(cudaGetLastError());
 }
 

@@ -185,6 +185,7 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
   std::memset(&kp, 0, sizeof(kp));
   kp.d = d; kp.m = m; kp.B = B; kp.L = L;
   kp.d_in = ctx->d_in;
+  kp.ld_q = kp.ld_out = ctx->d_in;
   kp.codes_bytes = d * B / 8;
   kp.signs_bytes = m / 8;
   kp.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
@@ -339,6 +340,49 @@ tq_status tq_logits(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t 
 }
 
 static size_t round16(size_t v) { return (v + 15) & ~static_cast<size_t>(15); }
+
+size_t tq_search_workspace_bytes(const tq_ctx* ctx, int64_t n_q, int64_t n_keys, int k) {
+  if (!ctx || n_q <= 0 || n_keys <= 0 || k <= 0) return 0;
+  const size_t qp = round16(static_cast<size_t>(n_q) * (ctx->d + ctx->m) * sizeof(float));
+  if (wide_search_applies(*ctx, n_q, n_keys, k)) return qp + wide_search_partial_bytes(n_q, n_keys, k);
+  return qp + round16(static_cast<size_t>(n_q) * n_keys * sizeof(float));
+}
+
+tq_status tq_search(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_q, tq_packed keys, int64_t n_keys,
+                    int k, int32_t* idx, float* val, void* workspace, size_t workspace_bytes, void* stream) {
+  tq_status st = check_ctx(ctx);
+  if (st != TQ_OK) return st;
+  if (n_q < 0 || n_keys < 0) return fail(TQ_ERR_INVALID_ARG, "n_q and n_keys must be >= 0");
+  if (n_q > 4096) return fail(TQ_ERR_INVALID_ARG, "n_q must be in [0, 4096]");
+  if (k < 1 || k > 16) return fail(TQ_ERR_INVALID_ARG, "k must be in [1, 16]");
+  if (q_dtype != TQ_BF16 && q_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "q_dtype must be TQ_BF16 or TQ_F32");
+  if (n_q == 0) return TQ_OK;
+  if (k > n_keys) return fail(TQ_ERR_INVALID_ARG, "k > n_keys");
+  if (n_keys > INT32_MAX) return fail(TQ_ERR_UNSUPPORTED, "n_keys must fit in int32");
+  if (!q || !idx) return fail(TQ_ERR_INVALID_ARG, "q or idx is NULL");
+  if (!aligned(q, 16) || !aligned(idx, 4) || (val && !aligned(val, 4)))
+    return fail(TQ_ERR_INVALID_ARG, "q must be 16-byte and idx/val 4-byte aligned");
+  if ((st = check_packed(ctx, keys)) != TQ_OK) return st;
+  const size_t need = tq_search_workspace_bytes(ctx, n_q, n_keys, k);
+  if (!workspace || workspace_bytes < need) return fail(TQ_ERR_INVALID_ARG, "workspace missing or too small");
+  if (!aligned(workspace, 16)) return fail(TQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  float* qp = reinterpret_cast<float*>(w);
+  void* rest = w + round16(static_cast<size_t>(n_q) * (ctx->d + ctx->m) * sizeof(float));
+  int err = launch_qprep(ctx->kp, q, q_dtype == TQ_BF16, n_q, qp, stream);
+  if (err) return cuda_fail(err, "tq_search query-prep launch");
+  if (wide_search_applies(*ctx, n_q, n_keys, k)) {
+    err = launch_search_wide(*ctx, qp, n_q, to_internal(keys), n_keys, k, idx, val, rest, stream);
+    if (err) return cuda_fail(err, "tq_search launch");
+    return TQ_OK;
+  }
+  float* scores = static_cast<float*>(rest);         // [n_q, n_keys], then the top-k of each row
+  err = launch_logits(*ctx, qp, 1, static_cast<int>(n_q), to_internal(keys), n_keys, scores, stream);
+  if (err) return cuda_fail(err, "tq_search logits launch");
+  err = launch_topk(scores, n_q, n_keys, k, idx, val, stream);
+  if (err) return cuda_fail(err, "tq_search top-k launch");
+  return TQ_OK;
+}
 
 size_t tq_attention_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g, int64_t n_keys) {
   if (!ctx || n_sets <= 0 || g <= 0 || n_keys <= 0) return 0;

@@ -17,6 +17,9 @@ constexpr float kZeroNorm = 1e-10f; // rows with ||x|| below this are stored as 
 struct KParams {
   int d, m, B, L;                     // d: the rotation dimension (a power of two)
   int d_in;                           // the caller's row length (<= d; rows are zero-padded to d)
+  int64_t ld_q, ld_out;               // row strides (elements) of the queries the query prep reads and of
+                                      // the rows the general dequant writes: d_in, unless a caller's
+                                      // view of wider rows (a channel split) says otherwise
   int codes_bytes, signs_bytes;       // per row
   float inv_sqrt_d;                   // 1/sqrt(d), fp32
   float qjl_scale;                    // sqrt(pi/2) / m, fp32
@@ -69,6 +72,7 @@ size_t attention_partial_bytes(const KParams& P, int64_t n_sets, int g, int64_t 
 int launch_attention_tail(const KParams& P, const float* logits, const Packed& values, int64_t n_sets, int g,
                           int64_t n_keys, float scale, int prod, float* partial, float* out, void* stream);
 int launch_topk(const float* scores, int64_t rows, int64_t cols, int k, int32_t* idx, float* val, void* stream);
+int launch_add(float* out, const float* in, int64_t n, void* stream);    // out += in, elementwise
 int launch_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, int d, float* out,
                        void* stream);
 const char* cuda_error_string(int err);
@@ -95,6 +99,11 @@ int launch_quantize_wide(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_
 bool wide_logits_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys);
 int launch_logits_wide(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
                        float* out, void* stream);
+// vector search with the top-k fused into the estimates' epilogue
+bool wide_search_applies(const tq_ctx& ctx, int64_t n_q, int64_t n_keys, int k);
+size_t wide_search_partial_bytes(int64_t n_q, int64_t n_keys, int k);
+int launch_search_wide(const tq_ctx& ctx, const float* qp, int64_t n_q, const Packed& keys, int64_t n_keys, int k,
+                       int32_t* idx, float* val, void* part, void* stream);
 }  // namespace tq
 
 struct tq_ctx {

@@ -91,20 +91,33 @@ struct SignEpi {
   uint32_t fix_cap;
 };
 
-// epilogue of the read half: estimates of one (set, chunk of keys)
+// epilogue of the read half: estimates of one (set, chunk of keys), written
+// out (kScores) or reduced to the k largest per (query, 128-key tile) (kTopk)
 struct LogitEpi {
-  float* out;                            // out[q * ld_out + key0 + key] for this set
+  float* out;                            // kScores: out[q * ld_out + key0 + key] for this set
   int64_t ld_out, key0;
   const float* norm;                     // the chunk's first key
   const float* rnorm;
   const float* qscale;                   // [n_q][2] for this set's queries
+  int k;                                 // kTopk: candidates per (query, tile), <= kMaxSearchK
+  float* pval;                           // kTopk: [n_q][ld_part], tile t at [t k, t k + k)
+  int32_t* pidx;
+  int64_t ld_part;
 };
+
+enum { kSigns = 0, kScores = 1, kTopk = 2 };
+constexpr int kMaxSearchK = 16;
+constexpr int kEstLd = kTM + 1;          // padded row of the [query][key] estimate tile in shared memory
+
+__device__ __forceinline__ const float* sE_col(const uint8_t* base, int col) {
+  return reinterpret_cast<const float*>(base) + col * kEstLd;
+}
 
 __device__ __forceinline__ void set_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
-template <int NACC, bool LOGITS, class Epi>
+template <int NACC, int MODE, class Epi>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_wide_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, const GemmPlan plan,
                int64_t n_rows, int n_cols, const Epi E, int* err) {
@@ -138,7 +151,7 @@ k_gemm_wide_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
     tmem_relinquish();
   }
   for (int c = threadIdx.x; c < kTN; c += kThreads) {
-    if constexpr (LOGITS) {
+    if constexpr (MODE != kSigns) {
       const int q = col0 + c;
       s_col[2 * c] = q < n_cols ? E.qscale[2 * q] : 0.f;
       s_col[2 * c + 1] = q < n_cols ? E.qscale[2 * q + 1] : 0.f;
@@ -218,9 +231,12 @@ k_gemm_wide_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
     const int64_t row = row0 + rl;
     const bool valid = row < n_rows;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    if constexpr (LOGITS) {
+    if constexpr (MODE != kSigns) {
       const float nrm = valid ? E.norm[row] : 0.f, rn = valid ? E.rnorm[row] : 0.f;
       float* orow = E.out + E.key0 + row;
+      // kTopk: the tile's estimates go to shared memory as [query][key] over the
+      // stage buffers (every load has landed and every MMA has completed)
+      float* sE = reinterpret_cast<float*>(base);
       for (int c = 0; c < kTN / 32; ++c) {
         const int q0 = col0 + c * 32;
         if (q0 >= n_cols) break;                     // uniform over the CTA
@@ -228,15 +244,15 @@ k_gemm_wide_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
         tmem_ld32(taddr + c * 32, a0);
         tmem_ld32(taddr + 256 + c * 32, a1);
         tmem_wait_ld();
-        if (valid) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int q = q0 + i;
-            if (q < n_cols) {
-              const float v = nrm * (__uint_as_float(a0[i]) * s_col[2 * (c * 32 + i)]) +
-                              rn * (__uint_as_float(a1[i]) * s_col[2 * (c * 32 + i) + 1]);
-              orow[static_cast<int64_t>(q) * E.ld_out] = v;
-            }
+        for (int i = 0; i < 32; ++i) {
+          const int q = q0 + i;
+          const float v = nrm * (__uint_as_float(a0[i]) * s_col[2 * (c * 32 + i)]) +
+                          rn * (__uint_as_float(a1[i]) * s_col[2 * (c * 32 + i) + 1]);
+          if constexpr (MODE == kScores) {
+            if (valid && q < n_cols) orow[static_cast<int64_t>(q) * E.ld_out] = v;
+          } else {
+            sE[(c * 32 + i) * kEstLd + rl] = v;
           }
         }
       }
@@ -270,7 +286,55 @@ k_gemm_wide_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
     }
   }
 
-  if constexpr (!LOGITS) {                      // the tile's list joins the global one (one reservation)
+  if constexpr (MODE == kTopk) {
+    // per query column: the k largest estimates of the tile's keys, larger
+    // first, equal values by lower key index.  The list is a 16-slot register
+    // insertion network (compile-time slots; an element moves in only where it
+    // is strictly larger, so an equal later key never displaces an earlier
+    // one); the first k slots are the answer, -inf where the tile has fewer
+    // keys
+    __syncthreads();
+    if (!bad) {
+      const int K = E.k;
+      const int64_t tile = (E.key0 + row0) / kTM;
+      const int nr = static_cast<int>(n_rows - row0 < kTM ? n_rows - row0 : kTM);
+      for (int col = threadIdx.x; col < kTN; col += kThreads) {
+        const int q = col0 + col;
+        if (q >= n_cols) continue;
+        float tv[kMaxSearchK];
+        int32_t ti[kMaxSearchK];
+#pragma unroll
+        for (int u = 0; u < kMaxSearchK; ++u) { tv[u] = -INFINITY; ti[u] = INT32_MAX; }
+        float kth = -INFINITY;                           // slot K - 1
+        const float* e = sE_col(base, col);
+        for (int r = 0; r < nr; ++r) {
+          float x = e[r];
+          if (!(x > kth)) continue;
+          int32_t xi = static_cast<int32_t>(E.key0 + row0 + r);
+#pragma unroll
+          for (int u = 0; u < kMaxSearchK; ++u) {
+            const bool take = x > tv[u];
+            const float pv = tv[u];
+            const int32_t pi = ti[u];
+            tv[u] = take ? x : pv;
+            ti[u] = take ? xi : pi;
+            x = take ? pv : x;
+            xi = take ? pi : xi;
+          }
+#pragma unroll
+          for (int u = 0; u < kMaxSearchK; ++u)
+            if (u == K - 1) kth = tv[u];
+        }
+        float* pv = E.pval + static_cast<int64_t>(q) * E.ld_part + tile * K;
+        int32_t* pi = E.pidx + static_cast<int64_t>(q) * E.ld_part + tile * K;
+#pragma unroll
+        for (int u = 0; u < kMaxSearchK; ++u)
+          if (u < K) { pv[u] = tv[u]; pi[u] = ti[u]; }
+      }
+    }
+  }
+
+  if constexpr (MODE == kSigns) {               // the tile's list joins the global one (one reservation)
     __syncthreads();
     __shared__ uint32_t s_base;
     const uint32_t nloc = min(*s_nfix, static_cast<uint32_t>(kLocalFix));
@@ -593,19 +657,19 @@ int make_map(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows, int 
   return r == CUDA_SUCCESS ? 0 : static_cast<int>(cudaErrorInvalidValue);
 }
 
-template <int NACC, bool LOGITS, class Epi>
+template <int NACC, int MODE, class Epi>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPlan& plan, int64_t n_rows, int n_cols,
                 const Epi& E, int* err, cudaStream_t s) {
   const size_t smem = gemm_smem_bytes();
   static bool attr_set = false;                        // once per instantiation (host-side cost per launch)
   if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(k_gemm_wide_tc<NACC, LOGITS, Epi>,
+    const cudaError_t e = cudaFuncSetAttribute(k_gemm_wide_tc<NACC, MODE, Epi>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
     attr_set = true;
   }
   const dim3 grid(static_cast<unsigned>((n_cols + kTN - 1) / kTN), static_cast<unsigned>((n_rows + kTM - 1) / kTM));
-  k_gemm_wide_tc<NACC, LOGITS, Epi><<<grid, kThreads, smem, s>>>(ta, tb, plan, n_rows, n_cols, E, err);
+  k_gemm_wide_tc<NACC, MODE, Epi><<<grid, kThreads, smem, s>>>(ta, tb, plan, n_rows, n_cols, E, err);
   count_launch();
   return static_cast<int>(cudaGetLastError());
 }
@@ -720,7 +784,7 @@ int launch_quantize_wide(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_
     }
     if (err) return err;
     Ep.signs = reinterpret_cast<uint32_t*>(po.signs);
-    if ((err = launch_gemm<1, false>(ta, tb, plan, nr, m, Ep, P.err, s))) return err;
+    if ((err = launch_gemm<1, kSigns>(ta, tb, plan, nr, m, Ep, P.err, s))) return err;
     k_qjl_fixup<<<ctx.num_sms * 8, 256, 0, s>>>(P, A.res, fix, nfix, fix_cap, Ep.signs, m / 32);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return static_cast<int>(e);
@@ -728,10 +792,14 @@ int launch_quantize_wide(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_
   return 0;
 }
 
-int launch_logits_wide(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys,
-                       int64_t n_keys, float* out, void* stream) {
+namespace {
+
+// estimates of every query of a set against every key of that set, per
+// 18944-key chunk: key operand, then the GEMM with the MODE epilogue
+template <int MODE>
+int run_estimates(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
+                  const LogitEpi& tmpl, cudaStream_t s) {
   const KParams& P = ctx.kp;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int d = P.d, m = P.m;
   const int64_t n_q = n_sets * g;
   const int64_t chunk = wide_chunk_rows();
@@ -782,17 +850,68 @@ int launch_logits_wide(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g
                       keys.rnorm + row};
       k_key_operand<<<grid_warps(nk, ctx.num_sms), 256, 0, s>>>(P, kk, nk, K, a);
       count_launch();
-      LogitEpi Ep;
-      Ep.out = out + set * g * n_keys;
+      LogitEpi Ep = tmpl;
+      if (MODE == kScores) Ep.out = tmpl.out + set * g * n_keys;
       Ep.ld_out = n_keys;
       Ep.key0 = k0;
       Ep.norm = kk.norm;
       Ep.rnorm = kk.rnorm;
       Ep.qscale = qscale + 2 * set * g;
-      if ((err = launch_gemm<2, true>(ta, tb, plan, nk, g, Ep, P.err, s))) return err;
+      if ((err = launch_gemm<2, MODE>(ta, tb, plan, nk, g, Ep, P.err, s))) return err;
     }
   }
   return 0;
+}
+
+// idx[q][r] = pidx[q][pos[q][r]]: the key index of each chosen candidate
+__global__ void k_gather_idx(const int32_t* __restrict__ pidx, int64_t ld_part, const int32_t* __restrict__ pos,
+                             int64_t n, int k, int32_t* __restrict__ idx) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= n) return;
+  const int64_t q = t / k;
+  idx[t] = pidx[q * ld_part + pos[t]];
+}
+
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+}  // namespace
+
+int launch_logits_wide(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys,
+                       int64_t n_keys, float* out, void* stream) {
+  LogitEpi t{};
+  t.out = out;
+  return run_estimates<kScores>(ctx, qp, n_sets, g, keys, n_keys, t, static_cast<cudaStream_t>(stream));
+}
+
+bool wide_search_applies(const tq_ctx& ctx, int64_t n_q, int64_t n_keys, int k) {
+  return wide_applies(ctx) && ctx.kp.m % 64 == 0 && n_q >= 64 && n_keys >= 4096 && k >= 1 && k <= kMaxSearchK;
+}
+
+size_t wide_search_partial_bytes(int64_t n_q, int64_t n_keys, int k) {
+  const int64_t L = (n_keys + kTM - 1) / kTM * k;
+  return 2 * round256(static_cast<size_t>(n_q) * L * 4) + round256(static_cast<size_t>(n_q) * k * 4);
+}
+
+int launch_search_wide(const tq_ctx& ctx, const float* qp, int64_t n_q, const Packed& keys, int64_t n_keys, int k,
+                       int32_t* idx, float* val, void* part, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t L = (n_keys + kTM - 1) / kTM * k;
+  uint8_t* pb = static_cast<uint8_t*>(part);
+  float* pval = reinterpret_cast<float*>(pb);
+  int32_t* pidx = reinterpret_cast<int32_t*>(pb + round256(static_cast<size_t>(n_q) * L * 4));
+  int32_t* pos = reinterpret_cast<int32_t*>(pb + 2 * round256(static_cast<size_t>(n_q) * L * 4));
+  LogitEpi t{};
+  t.k = k;
+  t.pval = pval;
+  t.pidx = pidx;
+  t.ld_part = L;
+  int err = run_estimates<kTopk>(ctx, qp, 1, static_cast<int>(n_q), keys, n_keys, t, s);
+  if (err) return err;
+  if ((err = launch_topk(pval, n_q, L, k, pos, val, stream))) return err;
+  const int64_t n = n_q * k;
+  k_gather_idx<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(pidx, L, pos, n, k, idx);
+  count_launch();
+  return static_cast<int>(cudaGetLastError());
 }
 
 }  // namespace tq

@@ -31,7 +31,9 @@ SYMBOLS = [
     "tq_host_params", "tq_init", "tq_destroy", "tq_packed_sizes", "tq_get_params", "tq_quantize",
     "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_dequant", "tq_topk", "tq_logits_bf16",
     "tq_status_str", "tq_sync_status", "tq_last_error", "tq_launch_count", "tq_attention_workspace_bytes",
-    "tq_attention", "tq_quantize_scatter",
+    "tq_attention", "tq_quantize_scatter", "tq_search_workspace_bytes", "tq_search", "tq_split_init",
+    "tq_split_destroy", "tq_split_part", "tq_split_quantize", "tq_split_logits_workspace_bytes", "tq_split_logits",
+    "tq_split_dequant",
 ]
 
 
@@ -56,6 +58,15 @@ _sig = {
     "tq_attention_workspace_bytes": (_sz, [_vp, _i64, _i32, _i64]),
     "tq_attention": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _Packed, _i64, ctypes.c_float, _i32, _vp, _vp, _sz,
                             _vp]),
+    "tq_search_workspace_bytes": (_sz, [_vp, _i64, _i64, _i32]),
+    "tq_search": (_i32, [_vp, _vp, _i32, _i64, _Packed, _i64, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "tq_split_init": (_i32, [_i32, _i32, _i32, _i32, _u64, ctypes.POINTER(_vp)]),
+    "tq_split_destroy": (_i32, [_vp]),
+    "tq_split_part": (_i32, [_vp, _i32, ctypes.POINTER(_vp)]),
+    "tq_split_quantize": (_i32, [_vp, _vp, _i32, _i64, _i64, _Packed, _Packed, _vp]),
+    "tq_split_logits_workspace_bytes": (_sz, [_vp, _i64, _i32, _i64]),
+    "tq_split_logits": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _Packed, _i64, _vp, _vp, _sz, _vp]),
+    "tq_split_dequant": (_i32, [_vp, _Packed, _Packed, _i64, _vp, _i32, _i32, _vp]),
     "tq_topk": (_i32, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "tq_logits_bf16": (_i32, [_vp, _vp, _i64, _i32, _i64, _i32, _vp, _vp]),
     "tq_status_str": (ctypes.c_char_p, [_i32]),
@@ -262,6 +273,27 @@ class TurboQuant:
                                         cache.n_rows, cache.c(), _stream(stream)), "tq_quantize_scatter")
         return cache
 
+    def search_workspace_bytes(self, n_q: int, n_keys: int, k: int) -> int:
+        return int(_lib.tq_search_workspace_bytes(self._h, n_q, n_keys, k))
+
+    def search(self, q, keys: Packed, n_keys: int, k: int, idx=None, val=None, workspace=None, stream=None):
+        """Vector search: per query of q [n_q, d], the k packed rows with the
+        largest estimate (larger first, ties to the lower row); returns
+        (idx [n_q, k] int32, val [n_q, k] fp32)."""
+        import torch
+        n_q = q.shape[0]
+        if idx is None:
+            idx = torch.empty((n_q, k), dtype=torch.int32, device=q.device)
+        if val is None:
+            val = torch.empty((n_q, k), dtype=torch.float32, device=q.device)
+        need = self.search_workspace_bytes(n_q, n_keys, k)
+        if need and workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        _check(_lib.tq_search(self._h, _ptr(q), _dtype_code(q), n_q, keys.c(), n_keys, k, _ptr(idx), _ptr(val),
+                              _ptr(workspace), wbytes, _stream(stream)), "tq_search")
+        return idx, val
+
     def attention_workspace_bytes(self, n_sets: int, g: int, n_keys: int) -> int:
         return int(_lib.tq_attention_workspace_bytes(self._h, n_sets, g, n_keys))
 
@@ -282,6 +314,91 @@ class TurboQuant:
         _check(_lib.tq_attention(self._h, _ptr(q), _dtype_code(q), n_sets, g, keys.c(), values.c(), n_keys,
                                  float(scale), mode, _ptr(out), _ptr(workspace), wbytes, _stream(stream)),
                "tq_attention")
+        return out
+
+
+class TurboQuantSplit:
+    """Fractional bit widths: channels [0, d_hi) as one instance with b_hi
+    bits per coordinate, channels [d_hi, d) as another with b_lo bits (seeds
+    seed and seed + 1); packed rows come in pairs (part 0, part 1)."""
+
+    def __init__(self, d: int, d_hi: int, b_hi: int, b_lo: int, seed: int = 0):
+        self.d, self.d_hi, self.b_hi, self.b_lo, self.seed = d, d_hi, b_hi, b_lo, seed
+        h = _vp()
+        _check(_lib.tq_split_init(d, d_hi, b_hi, b_lo, seed & (2**64 - 1), ctypes.byref(h)), "tq_split_init")
+        self._h = h
+        self._sizes, self._parts = [], []
+        for p in (0, 1):
+            ph = _vp()
+            _check(_lib.tq_split_part(h, p, ctypes.byref(ph)), "tq_split_part")
+            cb, sb = _sz(), _sz()
+            _check(_lib.tq_packed_sizes(ph, 1, ctypes.byref(cb), ctypes.byref(sb)), "tq_packed_sizes")
+            self._sizes.append((cb.value, sb.value))
+            self._parts.append(ph)
+
+    def sync_status(self, stream=None):
+        """Wait for the stream and raise if a kernel of either part reported an error."""
+        for ph in self._parts:
+            _check(_lib.tq_sync_status(ph, _stream(stream)), "tq_sync_status")
+
+    @property
+    def row_bytes(self) -> int:
+        """Packed bytes per row over both parts (codes, signs, two fp32 norms each)."""
+        return sum(cb + sb + 8 for cb, sb in self._sizes)
+
+    def logits_workspace_bytes(self, n_sets: int, g: int, n_keys: int) -> int:
+        return int(_lib.tq_split_logits_workspace_bytes(self._h, n_sets, g, n_keys))
+
+    @property
+    def bits_per_coordinate(self) -> float:
+        return (self.d_hi * self.b_hi + (self.d - self.d_hi) * self.b_lo) / self.d
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.tq_split_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def empty_packed(self, n_rows: int, device="cuda"):
+        import torch
+        return tuple(Packed(torch.empty((n_rows, cb), dtype=torch.uint8, device=device),
+                            torch.empty((n_rows, sb), dtype=torch.uint8, device=device),
+                            torch.empty((n_rows,), dtype=torch.float32, device=device),
+                            torch.empty((n_rows,), dtype=torch.float32, device=device)) for cb, sb in self._sizes)
+
+    def quantize(self, x, out=None, stream=None):
+        assert x.dim() == 2 and x.stride(1) == 1
+        if out is None:
+            out = self.empty_packed(x.shape[0], x.device)
+        _check(_lib.tq_split_quantize(self._h, _ptr(x), _dtype_code(x), x.shape[0], x.stride(0), out[0].c(),
+                                      out[1].c(), _stream(stream)), "tq_split_quantize")
+        return out
+
+    def logits(self, q, keys, n_sets: int, g: int, n_keys: int, out=None, workspace=None, stream=None):
+        import torch
+        if out is None:
+            out = torch.empty((n_sets, g, n_keys), dtype=torch.float32, device=q.device)
+        need = self.logits_workspace_bytes(n_sets, g, n_keys)
+        if need and workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        _check(_lib.tq_split_logits(self._h, _ptr(q), _dtype_code(q), n_sets, g, keys[0].c(), keys[1].c(), n_keys,
+                                    _ptr(out), _ptr(workspace), wbytes, _stream(stream)), "tq_split_logits")
+        return out
+
+    def dequant(self, packed, n_rows: int | None = None, out_dtype=None, mode: int = TQ_DEQUANT_PROD, out=None,
+                stream=None):
+        import torch
+        n = packed[0].n_rows if n_rows is None else n_rows
+        if out is None:
+            out = torch.empty((n, self.d), dtype=out_dtype or torch.bfloat16, device=packed[0].norm.device)
+        _check(_lib.tq_split_dequant(self._h, packed[0].c(), packed[1].c(), n, _ptr(out), _dtype_code(out), mode,
+                                     _stream(stream)), "tq_split_dequant")
         return out
 
 

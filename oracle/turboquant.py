@@ -278,3 +278,47 @@ def topk(scores: np.ndarray, k: int):
     scores = np.asarray(scores)
     order = np.argsort(-scores, axis=1, kind="stable")[:, :k]
     return order.astype(np.int32), np.take_along_axis(scores, order, axis=1)
+
+
+# --------------------------------------------------------------------------
+# Fractional bit widths by a channel split.  The pages report 2.5- and 3.5-bit
+# results without the split rule [inlevel9 "TurboQuantのメモリ圧縮と半導体需要",
+# section "TurboQuantが実際に行っていること"]; the reading followed here (and by
+# the library): channels [0, d_hi) of every row are one instance with b_hi bits
+# per coordinate and channels [d_hi, d) another with b_lo bits, each with its
+# own D, S and codebook, m = the part's channel count, seeds seed and seed + 1;
+# a part whose channel count is not a power of two is zero-padded like any
+# row.  Inner products add over disjoint channel sets, so the estimate of
+# <q, k> is the sum of the parts' estimates.
+
+def split_parts(d: int, d_hi: int, b_hi: int, b_lo: int, seed: int, params_cls):
+    """[(first channel, channel count, Params of the padded part)] for the two parts."""
+    parts = []
+    for p, (c0, dc, b) in enumerate(((0, d_hi, b_hi), (d_hi, d - d_hi, b_lo))):
+        parts.append((c0, dc, params_cls(padded_dim(dc), b, dc, seed=seed + p)))
+    return parts
+
+
+def split_bits_per_coordinate(parts) -> float:
+    """Stored bits per coordinate of the caller's row, norms aside: b - 1 code
+    bits per (padded) channel plus one sign per projection."""
+    d = sum(dc for _, dc, _ in parts)
+    return sum(P.d * P.B + P.m for _, _, P in parts) / d
+
+
+def split_quantize(x: np.ndarray, parts, **kw):
+    """(packed part 0, packed part 1) of rows x [N, d]."""
+    x = np.asarray(x, dtype=np.float64)
+    return tuple(quantize(pad_rows(x[:, c0:c0 + dc], P.d), P, **kw) for c0, dc, P in parts)
+
+
+def split_logits(q: np.ndarray, packed, parts, n_sets: int, g: int, n_keys: int) -> np.ndarray:
+    """The sum of the two parts' estimates, (n_sets, g, n_keys)."""
+    q = np.asarray(q, dtype=np.float64)
+    return sum(logits(pad_rows(q[:, c0:c0 + dc], P.d), pk, P, n_sets, g, n_keys)
+               for (c0, dc, P), pk in zip(parts, packed))
+
+
+def split_dequant(packed, parts, mode: int = DEQUANT_PROD) -> np.ndarray:
+    """Reconstructed rows [N, d]: each part's channels from its packed rows."""
+    return np.concatenate([dequant(pk, P, mode)[:, :dc] for (_, dc, P), pk in zip(parts, packed)], axis=1)

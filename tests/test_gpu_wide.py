@@ -88,3 +88,55 @@ def test_wide_quantize_then_logits_end_to_end(tq):
     tol = parity.logit_tolerance(q, np.linalg.norm(k, axis=1), 1, g, n_keys)
     ok = (np.abs(got - want) <= tol + 1e-30) | ~same.reshape(1, 1, n_keys)
     assert ok.all()
+
+
+@pytest.mark.parametrize("d,b,m,n_q,n_keys,k,qdtype", [
+    (256, 3, 256, 300, CHUNK + 513, 10, "f32"),     # fused: two chunks, ragged key and query tiles
+    (1024, 4, 1024, 64, 5000, 16, "bf16"),           # fused, k = 16
+    (512, 2, 128, 100, 4096, 1, "f32"),              # fused, k = 1
+    (128, 3, 128, 37, 3000, 10, "bf16"),             # through the scores (d = 128)
+    (256, 3, 256, 10, 5000, 5, "f32"),               # through the scores (fewer than 64 queries)
+])
+def test_search_equals_topk_of_logits(tq, d, b, m, n_q, n_keys, k, qdtype):
+    """tq_search gives exactly tq_topk of the tq_logits scores (same values,
+    same indices, ties to the lower row), and its choices agree with the
+    oracle's estimates."""
+    P = op.Params(d, b, m, seed=0)
+    rng = np.random.default_rng(d + n_q + k)
+    kk = rng.standard_normal((n_keys, d)) * rng.uniform(0.1, 10, size=(n_keys, 1))
+    kk[:3] = edge_rows(d, rng)[:3]
+    pk = ot.quantize(kk, P)
+    qt, q = make_rows(d, n_q, qdtype, seed=5 * n_q + b)
+    T = make_ctx(tq, d, b, m)
+    dpk = tq.Packed.from_numpy(pk)
+    scores = T.logits(qt.cuda(), dpk, 1, n_q, n_keys)
+    i_ref, v_ref = tq.topk(scores[0], k)
+    i_got, v_got = T.search(qt.cuda(), dpk, n_keys, k)
+    T.sync_status()
+    assert torch.equal(i_got.cpu(), i_ref.cpu())
+    assert torch.equal(v_got.cpu(), v_ref.cpu())
+    want = ot.logits(q, pk, P, 1, n_q, n_keys)[0]
+    tol = parity.logit_tolerance(q, np.linalg.norm(kk, axis=1), 1, n_q, n_keys)[0]
+    ig = i_got.cpu().numpy().astype(np.int64)
+    vg = v_got.cpu().numpy().astype(np.float64)
+    rows = np.arange(n_q)[:, None]
+    assert np.all(np.abs(vg - want[rows, ig]) <= tol[rows, ig] + 1e-30)
+    # every chosen row is within the estimate tolerance of the oracle's k-th best
+    kth = -np.sort(-want, axis=1)[:, k - 1]
+    assert np.all(want[rows, ig] >= kth[:, None] - 2 * tol.max(axis=1, keepdims=True))
+
+
+def test_search_argument_errors(tq):
+    d, b, m, n_keys = 256, 3, 256, 4096
+    P = op.Params(d, b, m, seed=0)
+    pk = tq.Packed.from_numpy(ot.quantize(np.random.default_rng(0).standard_normal((n_keys, d)), P))
+    T = make_ctx(tq, d, b, m)
+    q = torch.randn(64, d, device="cuda")
+    for bad in (0, 17):
+        with pytest.raises(tq.TQError):
+            T.search(q, pk, n_keys, bad)
+    with pytest.raises(tq.TQError):
+        T.search(q, pk, 3, 4)                                    # k > n_keys
+    with pytest.raises(tq.TQError):
+        T.search(q, pk, n_keys, 10, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    T.sync_status()

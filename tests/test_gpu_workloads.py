@@ -165,7 +165,9 @@ def test_vector_search_sampled(tq):
     dq = torch.from_numpy(qf).cuda()
     scores = T.logits(dq, pk, 1, qs.n_rows, db.n_rows)
     idx_g, val_g = tq.topk(scores[0], 10)
+    idx_s, val_s = T.search(dq, pk, db.n_rows, 10)     # top-10 fused into the estimates
     T.sync_status()
+    assert torch.equal(idx_s, idx_g) and torch.equal(val_s, val_g)
     rng = np.random.default_rng(5)
     ridx = np.sort(rng.choice(db.n_rows, size=1500, replace=False))
     rep, want = sampled_quantize_check(P, db, pk, ridx)

@@ -342,3 +342,72 @@ def test_padding_to_a_power_of_two():
     assert np.isclose(px @ py, x @ y, rtol=1e-14)
     P = op.Params(128, 3, 128, seed=0)
     assert np.isclose(np.linalg.norm(ot.rotate(px[None, :], P)), np.linalg.norm(x), rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# fractional bit widths by a channel split (the library's reading; see
+# oracle.turboquant.split_parts)
+
+def test_split_bit_budgets():
+    """64 + 64 channels at b = 3 / 2 store 2.5 bits per coordinate, at 4 / 3
+    3.5 bits (codes b - 1 per channel plus one sign per channel, m = d_part)."""
+    p25 = ot.split_parts(128, 64, 3, 2, 0, op.Params)
+    p35 = ot.split_parts(128, 64, 4, 3, 0, op.Params)
+    assert ot.split_bits_per_coordinate(p25) == 2.5
+    assert ot.split_bits_per_coordinate(p35) == 3.5
+    # packed bytes per row: codes + signs of both parts, plus two fp32 norms each
+    assert sum(sum(ot.packed_sizes(P.d, P.b, P.m)[:2]) for _, _, P in p25) == 128 * 2.5 / 8
+    assert [P.seed for _, _, P in p25] == [0, 1] and [c0 for c0, _, _ in p25] == [0, 64]
+
+
+def test_split_query_on_one_part_is_that_parts_estimate():
+    """A query that is zero on one part's channels gets exactly the other
+    part's estimate: catches swapped parts and wrong column offsets."""
+    parts = ot.split_parts(96, 64, 4, 2, 3, op.Params)      # 64 + 32 channels
+    rng = np.random.default_rng(5)
+    k = rng.standard_normal((7, 96)) * 2.0
+    pk = ot.split_quantize(k, parts)
+    q = rng.standard_normal((1, 96))
+    q_hi, q_lo = q.copy(), q.copy()
+    q_hi[:, 64:] = 0.0
+    q_lo[:, :64] = 0.0
+    (c0, dc, P0), (c1, dc1, P1) = parts
+    own_hi = ot.logits(q[:, :64], pk[0], P0, 1, 1, 7)
+    own_lo = ot.logits(ot.pad_rows(q[:, 64:], P1.d), pk[1], P1, 1, 1, 7)
+    assert np.array_equal(ot.split_logits(q_hi, pk, parts, 1, 1, 7), own_hi)
+    assert np.array_equal(ot.split_logits(q_lo, pk, parts, 1, 1, 7), own_lo)
+    assert np.allclose(ot.split_logits(q, pk, parts, 1, 1, 7), own_hi + own_lo, rtol=1e-14, atol=1e-14)
+
+
+def test_split_estimator_unbiased_over_seeds():
+    """E over the two parts' (D, S) of the split estimate equals <q, k>."""
+    rng = np.random.default_rng(41)
+    q = rng.standard_normal((1, 32))
+    k = rng.standard_normal((1, 32)) * 2.0
+    want = float(q[0] @ k[0])
+    vals = []
+    for seed in range(0, 6000, 2):
+        parts = ot.split_parts(32, 16, 3, 2, seed, op.Params)
+        vals.append(ot.split_logits(q, ot.split_quantize(k, parts), parts, 1, 1, 1)[0, 0, 0])
+    v = np.array(vals)
+    se = v.std(ddof=1) / math.sqrt(v.size)
+    assert abs(v.mean() - want) < 3 * se and se > 1e-4
+
+
+def test_split_mse_error_per_part_and_distortion():
+    """On each part's channels, x - x~_MSE has length n_p rho_p (that part's
+    stored residual norm, as for one instance), and E[rho_p^2] is that part's
+    codebook distortion: the higher-width part about 4x below the lower."""
+    parts = ot.split_parts(128, 64, 4, 3, 9, op.Params)
+    x = np.random.default_rng(77).standard_normal((6000, 128))
+    pk = ot.split_quantize(x, parts, keep_intermediates=True)
+    xt = ot.split_dequant(pk, parts, ot.DEQUANT_MSE)
+    dist = []
+    for (c0, dc, P), p in zip(parts, pk):
+        err = np.linalg.norm(x[:, c0:c0 + dc] - xt[:, c0:c0 + dc], axis=1)
+        assert np.allclose(err, p["rnorm"], rtol=2e-6)
+        r2 = p["rho"] ** 2
+        D = op.mse_distortion(P.d, P.centroids64)
+        assert abs(r2.mean() - D) < 3 * r2.std(ddof=1) / math.sqrt(r2.size)
+        dist.append(D)
+    assert 3.0 < dist[1] / dist[0] < 4.5
