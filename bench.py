@@ -13,6 +13,12 @@ per-kernel times, the quantize rows/s and the bf16 unquantized-key baseline
 kernel on the same shapes are reported beside it.  Inputs (2.1 GB per K/V
 tensor) are larger than L2, so no flush is needed between steps.
 
+Secondary workloads (`--workload NAME`, each with its own metric line): the
+prefill write path (prefill-b2/b3/b4), decode-time append (append-b3), vector
+search (vsearch: quantize a 10^6 x 1024 database, then tq_search's fused
+top-10; vsearch-128k for profiler captures) and the long-context decode step
+at fractional bit widths (decode-128k-2.5bit / 3.5bit: 64 + 64 channel split).
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 """
 

@@ -217,14 +217,15 @@ tq_status tq_dequant(const tq_ctx* ctx, tq_packed in, int64_t n_rows, void* out,
 
 /* Vector search: for each of n_q queries, the k packed rows (of n_keys) with
  * the largest estimated inner product (the tq_logits estimator with
- * n_sets = 1, g = n_q), larger first, equal estimates by lower row index:
- * exactly tq_topk over the scores tq_logits would write, without writing
- * them when the wide-row path applies (d >= 256, m a multiple of 64,
- * n_q >= 64, n_keys >= 4096): there the estimates GEMM keeps the k largest
- * of every 128-key tile per query (Google Research blog "TurboQuant:
- * Redefining AI efficiency with extreme compression", vector search; the
- * top-k is the search's answer).  Elsewhere the scores go through the
- * workspace.
+ * n_sets = 1, g = n_q), larger first, equal estimates by lower row index
+ * (Google Research blog "TurboQuant: Redefining AI efficiency with extreme
+ * compression", vector search: the top-k is the search's answer).  When the
+ * wide-row path applies (d >= 256, m a multiple of 64, n_q >= 64,
+ * n_keys >= 4096) no score is written: a persistent tensor-core kernel keeps
+ * each query's running top-k in registers while it streams the keys, and the
+ * per-CTA lists are merged at the end; its estimates equal tq_logits' up to
+ * fp32 accumulation order.  Elsewhere the scores go through the workspace
+ * and tq_topk's kernel.
  *   q    [n_q, d] bf16 or fp32, 16-byte aligned; n_q in [0, 4096];
  *   idx  [n_q, k] int32 row indices; val [n_q, k] fp32 estimates (may be NULL);
  *   k in [1, 16], k <= n_keys < 2^31;

@@ -344,7 +344,7 @@ static size_t round16(size_t v) { return (v + 15) & ~static_cast<size_t>(15); }
 size_t tq_search_workspace_bytes(const tq_ctx* ctx, int64_t n_q, int64_t n_keys, int k) {
   if (!ctx || n_q <= 0 || n_keys <= 0 || k <= 0) return 0;
   const size_t qp = round16(static_cast<size_t>(n_q) * (ctx->d + ctx->m) * sizeof(float));
-  if (wide_search_applies(*ctx, n_q, n_keys, k)) return qp + wide_search_partial_bytes(n_q, n_keys, k);
+  if (wide_search_applies(*ctx, n_q, n_keys, k)) return qp + wide_search_partial_bytes(*ctx, n_q, n_keys, k);
   return qp + round16(static_cast<size_t>(n_q) * n_keys * sizeof(float));
 }
 

@@ -101,7 +101,7 @@ int launch_logits_wide(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g
                        float* out, void* stream);
 // vector search with the top-k fused into the estimates' epilogue
 bool wide_search_applies(const tq_ctx& ctx, int64_t n_q, int64_t n_keys, int k);
-size_t wide_search_partial_bytes(int64_t n_q, int64_t n_keys, int k);
+size_t wide_search_partial_bytes(const tq_ctx& ctx, int64_t n_q, int64_t n_keys, int k);
 int launch_search_wide(const tq_ctx& ctx, const float* qp, int64_t n_q, const Packed& keys, int64_t n_keys, int k,
                        int32_t* idx, float* val, void* part, void* stream);
 }  // namespace tq

@@ -91,27 +91,17 @@ struct SignEpi {
   uint32_t fix_cap;
 };
 
-// epilogue of the read half: estimates of one (set, chunk of keys), written
-// out (kScores) or reduced to the k largest per (query, 128-key tile) (kTopk)
+// epilogue of the read half: estimates of one (set, chunk of keys)
 struct LogitEpi {
-  float* out;                            // kScores: out[q * ld_out + key0 + key] for this set
+  float* out;                            // out[q * ld_out + key0 + key] for this set
   int64_t ld_out, key0;
   const float* norm;                     // the chunk's first key
   const float* rnorm;
   const float* qscale;                   // [n_q][2] for this set's queries
-  int k;                                 // kTopk: candidates per (query, tile), <= kMaxSearchK
-  float* pval;                           // kTopk: [n_q][ld_part], tile t at [t k, t k + k)
-  int32_t* pidx;
-  int64_t ld_part;
 };
 
-enum { kSigns = 0, kScores = 1, kTopk = 2 };
+enum { kSigns = 0, kScores = 1 };
 constexpr int kMaxSearchK = 16;
-constexpr int kEstLd = kTM + 1;          // padded row of the [query][key] estimate tile in shared memory
-
-__device__ __forceinline__ const float* sE_col(const uint8_t* base, int col) {
-  return reinterpret_cast<const float*>(base) + col * kEstLd;
-}
 
 __device__ __forceinline__ void set_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
@@ -234,9 +224,6 @@ k_gemm_wide_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
     if constexpr (MODE != kSigns) {
       const float nrm = valid ? E.norm[row] : 0.f, rn = valid ? E.rnorm[row] : 0.f;
       float* orow = E.out + E.key0 + row;
-      // kTopk: the tile's estimates go to shared memory as [query][key] over the
-      // stage buffers (every load has landed and every MMA has completed)
-      float* sE = reinterpret_cast<float*>(base);
       for (int c = 0; c < kTN / 32; ++c) {
         const int q0 = col0 + c * 32;
         if (q0 >= n_cols) break;                     // uniform over the CTA
@@ -249,11 +236,7 @@ k_gemm_wide_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
           const int q = q0 + i;
           const float v = nrm * (__uint_as_float(a0[i]) * s_col[2 * (c * 32 + i)]) +
                           rn * (__uint_as_float(a1[i]) * s_col[2 * (c * 32 + i) + 1]);
-          if constexpr (MODE == kScores) {
-            if (valid && q < n_cols) orow[static_cast<int64_t>(q) * E.ld_out] = v;
-          } else {
-            sE[(c * 32 + i) * kEstLd + rl] = v;
-          }
+          if (valid && q < n_cols) orow[static_cast<int64_t>(q) * E.ld_out] = v;
         }
       }
     } else {
@@ -282,54 +265,6 @@ k_gemm_wide_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
           }
         }
         if (valid) E.signs[row * E.words_per_row + (j0 >> 5)] = bits;
-      }
-    }
-  }
-
-  if constexpr (MODE == kTopk) {
-    // per query column: the k largest estimates of the tile's keys, larger
-    // first, equal values by lower key index.  The list is a 16-slot register
-    // insertion network (compile-time slots; an element moves in only where it
-    // is strictly larger, so an equal later key never displaces an earlier
-    // one); the first k slots are the answer, -inf where the tile has fewer
-    // keys
-    __syncthreads();
-    if (!bad) {
-      const int K = E.k;
-      const int64_t tile = (E.key0 + row0) / kTM;
-      const int nr = static_cast<int>(n_rows - row0 < kTM ? n_rows - row0 : kTM);
-      for (int col = threadIdx.x; col < kTN; col += kThreads) {
-        const int q = col0 + col;
-        if (q >= n_cols) continue;
-        float tv[kMaxSearchK];
-        int32_t ti[kMaxSearchK];
-#pragma unroll
-        for (int u = 0; u < kMaxSearchK; ++u) { tv[u] = -INFINITY; ti[u] = INT32_MAX; }
-        float kth = -INFINITY;                           // slot K - 1
-        const float* e = sE_col(base, col);
-        for (int r = 0; r < nr; ++r) {
-          float x = e[r];
-          if (!(x > kth)) continue;
-          int32_t xi = static_cast<int32_t>(E.key0 + row0 + r);
-#pragma unroll
-          for (int u = 0; u < kMaxSearchK; ++u) {
-            const bool take = x > tv[u];
-            const float pv = tv[u];
-            const int32_t pi = ti[u];
-            tv[u] = take ? x : pv;
-            ti[u] = take ? xi : pi;
-            x = take ? pv : x;
-            xi = take ? pi : xi;
-          }
-#pragma unroll
-          for (int u = 0; u < kMaxSearchK; ++u)
-            if (u == K - 1) kth = tv[u];
-        }
-        float* pv = E.pval + static_cast<int64_t>(q) * E.ld_part + tile * K;
-        int32_t* pi = E.pidx + static_cast<int64_t>(q) * E.ld_part + tile * K;
-#pragma unroll
-        for (int u = 0; u < kMaxSearchK; ++u)
-          if (u < K) { pv[u] = tv[u]; pi[u] = ti[u]; }
       }
     }
   }
@@ -640,6 +575,277 @@ k_query_operand(const KParams P, const float* __restrict__ qp, int64_t n_q, floa
 }
 
 // ---------------------------------------------------------------------------
+// vector search: the roles of the estimates GEMM swapped -- A = the split
+// queries (128 per CTA, query = TMEM lane), B = decoded keys (256 per tile) --
+// and the CTA persistent over its share of a chunk's key tiles, so that each
+// epilogue thread owns one query and keeps that query's running top-k in
+// registers from tile to tile (and, through sv / si, from chunk to chunk).
+// Warps 0-3 read TMEM (lanes 32w .. 32w + 31), warp 4 issues TMA, warp 5 the
+// MMAs; the single 512-column accumulator pair is handed back by an mbarrier
+// once the four warps have read it.
+// ---------------------------------------------------------------------------
+constexpr int kSearchThreads = 192;
+constexpr int kSearchTiles = 74;         // key tiles of 256 per chunk at most (18944 keys)
+
+struct SearchArgs {
+  const float* norm;                     // the chunk's first key
+  const float* rnorm;
+  const float* qscale;                   // [n_q][2]
+  float* sv;                             // running lists [n_q][S][k], larger first
+  int32_t* si;
+  int k, S, n_q;
+  int64_t key0, nk;                      // index of the chunk's first key, keys in the chunk
+  int tiles_per_split;
+  int first;                             // the chunk that starts the lists
+};
+
+__global__ void __launch_bounds__(kSearchThreads, 1)
+k_search_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, const GemmPlan plan,
+            const SearchArgs X, int* err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = base;
+  uint8_t* sB = base + kStages * kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kBBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* done = empty + kStages;      // a tile's MMAs completed
+  uint64_t* tfree = done + 1;            // the four epilogue warps have read the accumulators
+  uint64_t* fin = tfree + 1;             // every MMA of the CTA completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_nrm = reinterpret_cast<float*>(tmem_slot + 4);
+  float* s_rn = s_nrm + kTN;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, split = blockIdx.y;
+  const int n_tiles = static_cast<int>((X.nk + kTN - 1) / kTN);
+  const int t_begin = split * X.tiles_per_split;
+  const int t_end = min(t_begin + X.tiles_per_split, n_tiles);
+  const int my_tiles = max(0, t_end - t_begin);
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kStages; ++st) { mbar_init(&full[st], 1); mbar_init(&empty[st], 1); }
+    mbar_init(done, 1);
+    mbar_init(tfree, 128);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  int issued = 0;
+
+  if (warp == 4) {
+    if (lane == 0) {                     // ---- TMA producer
+      prefetch_tmap(&ta);
+      prefetch_tmap(&tb);
+      int g = 0;
+      bool stop = false;
+      for (int i = 0; i < my_tiles && !stop; ++i) {
+        const int tile = t_begin + i;
+        for (int sg = 0; sg < plan.nseg && !stop; ++sg) {
+          const GemmSeg S = plan.seg[sg];
+          for (int j = 0; j < S.nkb; ++j, ++g) {
+            const int st = g % kStages;
+            if (g >= kStages && !mbar_wait(&empty[st], ((g / kStages) - 1) & 1, kWaitCycles)) {
+              set_error(err, 2);
+              *abort_flag = 1;
+            }
+            if (*abort_flag) { stop = true; break; }
+            mbar_arrive_expect_tx(&full[st], kABytes + kBBytes);
+            tma_load_2d(sA + st * kABytes, &ta, &full[st], (S.a_kb + j) * kKB, qt * kTM);
+            tma_load_2d(sB + st * kBBytes, &tb, &full[st], (S.b_kb + j) * kKB, tile * kTN);
+            issued = g + 1;
+          }
+        }
+      }
+      for (int st = 0; st < kStages && st < issued; ++st) {     // wait for this thread's own loads
+        const int last = st + ((issued - 1 - st) / kStages) * kStages;
+        if (!mbar_wait(&full[st], (last / kStages) & 1, kWaitCycles)) set_error(err, 2);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {                     // ---- MMA issuer
+      constexpr uint32_t idesc = idesc_f16_f32(kTM, kTN);
+      int g = 0;
+      bool stop = false;
+      for (int i = 0; i < my_tiles && !stop; ++i) {
+        if (i > 0 && !mbar_wait(tfree, (i - 1) & 1, kWaitCycles)) {
+          set_error(err, 2);
+          *abort_flag = 1;
+        }
+        if (*abort_flag) break;
+        tc_fence_after();
+        bool started[2] = {false, false};
+        for (int sg = 0; sg < plan.nseg && !stop; ++sg) {
+          const GemmSeg S = plan.seg[sg];
+          for (int j = 0; j < S.nkb; ++j, ++g) {
+            const int st = g % kStages;
+            if (!mbar_wait(&full[st], (g / kStages) & 1, kWaitCycles)) {
+              set_error(err, 2);
+              *abort_flag = 1;
+              stop = true;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a = smem_u32(sA + st * kABytes), b = smem_u32(sB + st * kBBytes);
+            const uint32_t d_t = tmem + static_cast<uint32_t>(S.acc) * 256u;
+#pragma unroll
+            for (int kk = 0; kk < kKB / 16; ++kk)
+              mma_f16_ss(d_t, smem_desc_sw128(a + kk * 32, 1024), smem_desc_sw128(b + kk * 32, 1024), idesc,
+                         (started[S.acc] || kk > 0) ? 1u : 0u);
+            started[S.acc] = true;
+            mma_commit(&empty[st]);
+          }
+        }
+        if (!stop) mma_commit(done);
+      }
+      mma_commit(fin);                   // after every MMA issued above
+      if (!mbar_wait(fin, 0, kWaitCycles)) set_error(err, 2);
+    }
+  } else {
+    // ---- epilogue: thread = query
+    const int q = qt * kTM + warp * 32 + lane;
+    const bool qv = q < X.n_q;
+    const int K = X.k;
+    const float qs0 = qv ? X.qscale[2 * q] : 0.f, qs1 = qv ? X.qscale[2 * q + 1] : 0.f;
+    float tv[kMaxSearchK];
+    int32_t ti[kMaxSearchK];
+#pragma unroll
+    for (int u = 0; u < kMaxSearchK; ++u) { tv[u] = -INFINITY; ti[u] = INT32_MAX; }
+    float* lv = X.sv + (static_cast<int64_t>(q) * X.S + split) * K;
+    int32_t* li = X.si + (static_cast<int64_t>(q) * X.S + split) * K;
+    if (qv && !X.first) {
+#pragma unroll
+      for (int u = 0; u < kMaxSearchK; ++u)
+        if (u < K) { tv[u] = lv[u]; ti[u] = li[u]; }
+    }
+    float kth = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kMaxSearchK; ++u)
+      if (u == K - 1) kth = tv[u];
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    for (int i = 0; i < my_tiles; ++i) {
+      const bool ok = mbar_wait(done, i & 1, kWaitCycles);
+      if (named_bar_sync_or(1, 128, !ok || *abort_flag)) {      // every epilogue thread leaves together
+        if (!ok) set_error(err, 2);
+        *abort_flag = 1;
+        break;
+      }
+      const int64_t kb = static_cast<int64_t>(t_begin + i) * kTN;
+      for (int c = threadIdx.x; c < kTN; c += 128) {
+        const int64_t key = kb + c;
+        s_nrm[c] = key < X.nk ? X.norm[key] : 0.f;
+        s_rn[c] = key < X.nk ? X.rnorm[key] : 0.f;
+      }
+      named_bar_sync(1, 128);
+      tc_fence_after();
+      for (int c = 0; c < kTN / 32; ++c) {
+        uint32_t a0[32], a1[32];
+        tmem_ld32(taddr + c * 32, a0);
+        tmem_ld32(taddr + 256 + c * 32, a1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int col = c * 32 + j;
+          float x = s_nrm[col] * (__uint_as_float(a0[j]) * qs0) + s_rn[col] * (__uint_as_float(a1[j]) * qs1);
+          if (qv && kb + col < X.nk && x > kth) {
+            // insertion network: keys reach a list in increasing order, so a
+            // strictly larger value is the only one that moves in
+            int32_t xi = static_cast<int32_t>(X.key0 + kb + col);
+#pragma unroll
+            for (int u = 0; u < kMaxSearchK; ++u) {
+              const bool take = x > tv[u];
+              const float pv = tv[u];
+              const int32_t pi = ti[u];
+              tv[u] = take ? x : pv;
+              ti[u] = take ? xi : pi;
+              x = take ? pv : x;
+              xi = take ? pi : xi;
+            }
+#pragma unroll
+            for (int u = 0; u < kMaxSearchK; ++u)
+              if (u == K - 1) kth = tv[u];
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tfree);
+    }
+    if (qv && !*abort_flag) {
+#pragma unroll
+      for (int u = 0; u < kMaxSearchK; ++u)
+        if (u < K) { lv[u] = tv[u]; li[u] = ti[u]; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// The k best of each query's S lists (value larger first, equal values by
+// lower key index), one warp per query: every lane keeps the best k of its
+// share of the S k candidates, then k rounds of a warp-wide best.
+__device__ __forceinline__ bool better_vi(float va, int32_t ia, float vb, int32_t ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+__global__ void __launch_bounds__(256)
+k_merge_lists(const float* __restrict__ sv, const int32_t* __restrict__ si, int n_cand, int k, int n_q,
+              int32_t* __restrict__ idx, float* __restrict__ val) {
+  const int q = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (q >= n_q) return;                                  // warp-uniform
+  float tv[kMaxSearchK];
+  int32_t ti[kMaxSearchK];
+#pragma unroll
+  for (int u = 0; u < kMaxSearchK; ++u) { tv[u] = -INFINITY; ti[u] = INT32_MAX; }
+  for (int c = lane; c < n_cand; c += 32) {
+    float x = sv[static_cast<int64_t>(q) * n_cand + c];
+    int32_t xi = si[static_cast<int64_t>(q) * n_cand + c];
+#pragma unroll
+    for (int u = 0; u < kMaxSearchK; ++u) {
+      const bool take = better_vi(x, xi, tv[u], ti[u]);
+      const float pv = tv[u];
+      const int32_t pi = ti[u];
+      tv[u] = take ? x : pv;
+      ti[u] = take ? xi : pi;
+      x = take ? pv : x;
+      xi = take ? pi : xi;
+    }
+  }
+  for (int r = 0; r < k; ++r) {
+    float bv = tv[0];
+    int32_t bi = ti[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (better_vi(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+    }
+    if (lane == 0) {
+      idx[static_cast<int64_t>(q) * k + r] = bi;
+      if (val) val[static_cast<int64_t>(q) * k + r] = bv;
+    }
+    if (ti[0] == bi && tv[0] == bv) {                    // the winner's lane moves to its next candidate
+#pragma unroll
+      for (int u = 0; u + 1 < kMaxSearchK; ++u) { tv[u] = tv[u + 1]; ti[u] = ti[u + 1]; }
+      tv[kMaxSearchK - 1] = -INFINITY;
+      ti[kMaxSearchK - 1] = INT32_MAX;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host
 // ---------------------------------------------------------------------------
 constexpr size_t gemm_smem_bytes() { return 1024 + kStages * (kABytes + kBBytes) + 256 + kTN * 8 + 16 + kLocalFix * 4; }
@@ -863,15 +1069,6 @@ int run_estimates(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, con
   return 0;
 }
 
-// idx[q][r] = pidx[q][pos[q][r]]: the key index of each chosen candidate
-__global__ void k_gather_idx(const int32_t* __restrict__ pidx, int64_t ld_part, const int32_t* __restrict__ pos,
-                             int64_t n, int k, int32_t* __restrict__ idx) {
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (t >= n) return;
-  const int64_t q = t / k;
-  idx[t] = pidx[q * ld_part + pos[t]];
-}
-
 size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 
 }  // namespace
@@ -887,29 +1084,101 @@ bool wide_search_applies(const tq_ctx& ctx, int64_t n_q, int64_t n_keys, int k) 
   return wide_applies(ctx) && ctx.kp.m % 64 == 0 && n_q >= 64 && n_keys >= 4096 && k >= 1 && k <= kMaxSearchK;
 }
 
-size_t wide_search_partial_bytes(int64_t n_q, int64_t n_keys, int k) {
-  const int64_t L = (n_keys + kTM - 1) / kTM * k;
-  return 2 * round256(static_cast<size_t>(n_q) * L * 4) + round256(static_cast<size_t>(n_q) * k * 4);
+namespace {
+int search_splits(const tq_ctx& ctx, int64_t n_q) {     // CTAs per query tile
+  const int64_t qtiles = (n_q + kTM - 1) / kTM;
+  const int64_t s = ctx.num_sms / qtiles;
+  return static_cast<int>(s < 1 ? 1 : s);
+}
+}  // namespace
+
+size_t wide_search_partial_bytes(const tq_ctx& ctx, int64_t n_q, int64_t n_keys, int k) {
+  (void)n_keys;
+  return 2 * round256(static_cast<size_t>(n_q) * search_splits(ctx, n_q) * k * 4);
 }
 
 int launch_search_wide(const tq_ctx& ctx, const float* qp, int64_t n_q, const Packed& keys, int64_t n_keys, int k,
                        int32_t* idx, float* val, void* part, void* stream) {
+  const KParams& P = ctx.kp;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int64_t L = (n_keys + kTM - 1) / kTM * k;
+  const int d = P.d, m = P.m;
+  const int S = search_splits(ctx, n_q);
+  const int qtiles = static_cast<int>((n_q + kTM - 1) / kTM);
+  const int tps = kSearchTiles / S > 0 ? kSearchTiles / S : 1;   // key tiles per CTA and chunk
+  const int64_t chunk = static_cast<int64_t>(S) * tps * kTN;
+  const int64_t keys_cap = n_keys < chunk ? n_keys : chunk;
+  const int64_t lda = 2 * (d + m), ldb = 2 * d + m;              // A: split queries, B: decoded keys
+  const size_t b_bytes = static_cast<size_t>(keys_cap) * ldb * 2;
+  const size_t a_off = round256(b_bytes);
+  const size_t qs_off = a_off + round256(static_cast<size_t>(n_q) * lda * 2);
+  PoolBuf buf;
+  buf.s = s;
+  cudaError_t e = cudaMallocFromPoolAsync(&buf.p, qs_off + static_cast<size_t>(n_q) * 8,
+                                          static_cast<cudaMemPool_t>(ctx.pool), s);
+  if (e != cudaSuccess) { buf.p = nullptr; return static_cast<int>(e); }
+  uint8_t* base = static_cast<uint8_t*>(buf.p);
+  __half* kop = reinterpret_cast<__half*>(base);
+  __half* qop = reinterpret_cast<__half*>(base + a_off);
+  float* qscale = reinterpret_cast<float*>(base + qs_off);
   uint8_t* pb = static_cast<uint8_t*>(part);
-  float* pval = reinterpret_cast<float*>(pb);
-  int32_t* pidx = reinterpret_cast<int32_t*>(pb + round256(static_cast<size_t>(n_q) * L * 4));
-  int32_t* pos = reinterpret_cast<int32_t*>(pb + 2 * round256(static_cast<size_t>(n_q) * L * 4));
-  LogitEpi t{};
-  t.k = k;
-  t.pval = pval;
-  t.pidx = pidx;
-  t.ld_part = L;
-  int err = run_estimates<kTopk>(ctx, qp, 1, static_cast<int>(n_q), keys, n_keys, t, s);
-  if (err) return err;
-  if ((err = launch_topk(pval, n_q, L, k, pos, val, stream))) return err;
-  const int64_t n = n_q * k;
-  k_gather_idx<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(pidx, L, pos, n, k, idx);
+  float* sv = reinterpret_cast<float*>(pb);
+  int32_t* si = reinterpret_cast<int32_t*>(pb + round256(static_cast<size_t>(n_q) * S * k * 4));
+
+  const int sc = pow2_at_least_sqrt(d);
+  k_query_operand<<<grid_warps(n_q, ctx.num_sms), 256, 0, s>>>(P, qp, n_q, 1.0f / static_cast<float>(sc), qop,
+                                                               qscale);
+  count_launch();
+  KeyOpArgs K{};
+  for (int i = 0; i < P.L; ++i) {
+    const double v = static_cast<double>(P.c[i]) * sc;
+    const uint16_t h = double_to_half_bits(v);
+    K.c_hi[i] = h;
+    K.c_lo[i] = double_to_half_bits(v - half_bits_to_double(h));
+  }
+  CUtensorMap ta, tb;
+  int err;
+  if ((err = make_map(&ta, qop, lda, n_q, kTM))) return err;
+  if ((err = make_map(&tb, kop, ldb, keys_cap, kTN))) return err;
+  GemmPlan plan{};
+  plan.nseg = 5;
+  const int nd = d / kKB, nm = m / kKB;
+  plan.seg[0] = {0, 0, nd, 0};                        // q_hi c_hi
+  plan.seg[1] = {0, nd, nd, 0};                       // q_hi c_lo
+  plan.seg[2] = {nd, 0, nd, 0};                       // q_lo c_hi
+  plan.seg[3] = {2 * nd, 2 * nd, nm, 1};              // sq_hi z
+  plan.seg[4] = {2 * nd + nm, 2 * nd, nm, 1};         // sq_lo z
+  const size_t smem = 1024 + kStages * (kABytes + kBBytes) + 256 + 2 * kTN * 4;
+  static bool attr_set = false;
+  if (!attr_set) {
+    e = cudaFuncSetAttribute(k_search_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+    attr_set = true;
+  }
+  for (int64_t k0 = 0; k0 < n_keys; k0 += chunk) {
+    const int64_t nk = n_keys - k0 < chunk ? n_keys - k0 : chunk;
+    const Packed kk{keys.codes + k0 * P.codes_bytes, keys.signs + k0 * P.signs_bytes, keys.norm + k0,
+                    keys.rnorm + k0};
+    k_key_operand<<<grid_warps(nk, ctx.num_sms), 256, 0, s>>>(P, kk, nk, K, kop);
+    count_launch();
+    SearchArgs X{};
+    X.norm = kk.norm;
+    X.rnorm = kk.rnorm;
+    X.qscale = qscale;
+    X.sv = sv;
+    X.si = si;
+    X.k = k;
+    X.S = S;
+    X.n_q = static_cast<int>(n_q);
+    X.key0 = k0;
+    X.nk = nk;
+    X.tiles_per_split = tps;
+    X.first = k0 == 0;
+    k_search_tc<<<dim3(qtiles, S), kSearchThreads, smem, s>>>(ta, tb, plan, X, P.err);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return static_cast<int>(e);
+  }
+  k_merge_lists<<<static_cast<unsigned>((n_q + 7) / 8), 256, 0, s>>>(sv, si, S * k, k, static_cast<int>(n_q), idx,
+                                                                      val);
   count_launch();
   return static_cast<int>(cudaGetLastError());
 }

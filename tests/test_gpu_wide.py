@@ -98,9 +98,11 @@ def test_wide_quantize_then_logits_end_to_end(tq):
     (256, 3, 256, 10, 5000, 5, "f32"),               # through the scores (fewer than 64 queries)
 ])
 def test_search_equals_topk_of_logits(tq, d, b, m, n_q, n_keys, k, qdtype):
-    """tq_search gives exactly tq_topk of the tq_logits scores (same values,
-    same indices, ties to the lower row), and its choices agree with the
-    oracle's estimates."""
+    """tq_search picks the k best rows by the same estimates tq_logits writes
+    (its own tensor-core pass: values equal to the scores within fp32
+    accumulation-order noise, every pick within that noise of the k-th best,
+    larger first, no repeats), and its choices agree with the oracle's
+    estimates."""
     P = op.Params(d, b, m, seed=0)
     rng = np.random.default_rng(d + n_q + k)
     kk = rng.standard_normal((n_keys, d)) * rng.uniform(0.1, 10, size=(n_keys, 1))
@@ -113,8 +115,16 @@ def test_search_equals_topk_of_logits(tq, d, b, m, n_q, n_keys, k, qdtype):
     i_ref, v_ref = tq.topk(scores[0], k)
     i_got, v_got = T.search(qt.cuda(), dpk, n_keys, k)
     T.sync_status()
-    assert torch.equal(i_got.cpu(), i_ref.cpu())
-    assert torch.equal(v_got.cpu(), v_ref.cpu())
+    sc = scores[0].cpu().numpy().astype(np.float64)
+    ig64 = i_got.cpu().numpy().astype(np.int64)
+    vg64 = v_got.cpu().numpy().astype(np.float64)
+    r_ = np.arange(n_q)[:, None]
+    eps = 1e-5 * np.abs(sc).max(axis=1, keepdims=True)
+    assert np.all(np.abs(vg64 - sc[r_, ig64]) <= eps)
+    assert np.all(sc[r_, ig64] >= -np.sort(-sc, axis=1)[:, k - 1:k] - eps)
+    assert np.all(np.diff(vg64, axis=1) <= 0)
+    assert all(len(set(row)) == k for row in ig64.tolist())
+    assert np.mean(ig64 == i_ref.cpu().numpy()) >= 0.98
     want = ot.logits(q, pk, P, 1, n_q, n_keys)[0]
     tol = parity.logit_tolerance(q, np.linalg.norm(kk, axis=1), 1, n_q, n_keys)[0]
     ig = i_got.cpu().numpy().astype(np.int64)

