@@ -1,6 +1,6 @@
 """Comparison rules between the CUDA path and the oracle (test infrastructure).
 
-Tolerances, from the spec contract and the arithmetic:
+Tolerances, from the stated parity contract and the arithmetic:
   * codes and sign bits: bit-exact, except coordinates whose oracle value lies
     within 1e-6 of a decision boundary (|y_i - t_k| < 1e-6 in the rotated,
     unit-normalised domain for codes; |p_j| < 1e-6 for signs).  Those
