@@ -43,6 +43,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -848,6 +849,20 @@ k_merge_lists(const float* __restrict__ sv, const int32_t* __restrict__ si, int 
 // ---------------------------------------------------------------------------
 // host
 // ---------------------------------------------------------------------------
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per device (bit d of
+// `done`); devices beyond 63 set it on every call
+int set_smem_once(const void* fn, size_t bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return 0;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e != cudaSuccess) return static_cast<int>(e);
+  if (bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return 0;
+}
+
 constexpr size_t gemm_smem_bytes() { return 1024 + kStages * (kABytes + kBBytes) + 256 + kTN * 8 + 16 + kLocalFix * 4; }
 
 int make_map(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows, int box_rows) {
@@ -867,13 +882,9 @@ template <int NACC, int MODE, class Epi>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPlan& plan, int64_t n_rows, int n_cols,
                 const Epi& E, int* err, cudaStream_t s) {
   const size_t smem = gemm_smem_bytes();
-  static bool attr_set = false;                        // once per instantiation (host-side cost per launch)
-  if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(k_gemm_wide_tc<NACC, MODE, Epi>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return static_cast<int>(e);
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_set{0};          // per device, once (a host-side cost per launch otherwise)
+  const int e = set_smem_once(reinterpret_cast<const void*>(k_gemm_wide_tc<NACC, MODE, Epi>), smem, attr_set);
+  if (e) return e;
   const dim3 grid(static_cast<unsigned>((n_cols + kTN - 1) / kTN), static_cast<unsigned>((n_rows + kTM - 1) / kTM));
   k_gemm_wide_tc<NACC, MODE, Epi><<<grid, kThreads, smem, s>>>(ta, tb, plan, n_rows, n_cols, E, err);
   count_launch();
@@ -1148,12 +1159,8 @@ int launch_search_wide(const tq_ctx& ctx, const float* qp, int64_t n_q, const Pa
   plan.seg[3] = {2 * nd, 2 * nd, nm, 1};              // sq_hi z
   plan.seg[4] = {2 * nd + nm, 2 * nd, nm, 1};         // sq_lo z
   const size_t smem = 1024 + kStages * (kABytes + kBBytes) + 256 + 2 * kTN * 4;
-  static bool attr_set = false;
-  if (!attr_set) {
-    e = cudaFuncSetAttribute(k_search_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return static_cast<int>(e);
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_set{0};
+  if ((err = set_smem_once(reinterpret_cast<const void*>(k_search_tc), smem, attr_set))) return err;
   for (int64_t k0 = 0; k0 < n_keys; k0 += chunk) {
     const int64_t nk = n_keys - k0 < chunk ? n_keys - k0 : chunk;
     const Packed kk{keys.codes + k0 * P.codes_bytes, keys.signs + k0 * P.signs_bytes, keys.norm + k0,
