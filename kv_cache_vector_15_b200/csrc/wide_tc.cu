@@ -66,7 +66,8 @@ constexpr uint32_t kABytes = kTM * 128;  // 16 KB
 constexpr uint32_t kBBytes = kTN * 128;  // 32 KB
 constexpr int kThreads = 128;
 constexpr long long kWaitCycles = 2000000000ll;   // ~1 s at 2 GHz
-constexpr int kChunkTiles = 148;         // row tiles per chunk (one wave per column tile at 1 CTA / SM)
+constexpr int kChunkTiles = 148;         // key tiles per chunk of the estimates (one wave per column tile at 1 CTA / SM)
+constexpr int kQuantChunkTiles = 296;    // row tiles per chunk of the write half (two waves per column tile)
 constexpr int kMaxSeg = 6;
 constexpr int kLocalFix = 512;           // ambiguous projections a tile lists in shared memory
 
@@ -327,6 +328,7 @@ struct PrepArgs {
   __half* res;                           // [rows][2d]
   float* rn;                             // [rows]: s ||r||, 0 for zero rows
   float s;                               // residual scale (a power of two)
+  uint32_t* nfix;                        // the chunk's fix-up list counter, reset here
 };
 
 template <int E, bool BF16>
@@ -336,6 +338,8 @@ k_quantize_residual_warp(const KParams P, const void* __restrict__ x, int64_t n_
   __shared__ float thr[kMaxLevels], lut[kMaxLevels];
   __shared__ uint8_t cs_all[8][E * 32];
   if (threadIdx.x < kMaxLevels) { thr[threadIdx.x] = P.t[threadIdx.x]; lut[threadIdx.x] = P.c[threadIdx.x]; }
+  // the previous chunk's fix-up has run (stream order); this chunk's GEMM appends after this kernel
+  if (blockIdx.x == 0 && threadIdx.x == 0 && A.nfix) *A.nfix = 0u;
   __syncthreads();
   const int d = E * 32, B = P.B, half_levels = P.L >> 1;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -586,7 +590,7 @@ k_query_operand(const KParams P, const float* __restrict__ qp, int64_t n_q, floa
 // once the four warps have read it.
 // ---------------------------------------------------------------------------
 constexpr int kSearchThreads = 192;
-constexpr int kSearchTiles = 74;         // key tiles of 256 per chunk at most (18944 keys)
+constexpr int kSearchTiles = 296;        // key tiles of 256 per chunk at most (75776 keys, 450 MB decoded at d = m = 1024)
 
 struct SearchArgs {
   const float* norm;                     // the chunk's first key
@@ -948,7 +952,7 @@ int launch_quantize_wide(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_
   const KParams& P = ctx.kp;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int d = P.d, m = P.m;
-  const int64_t chunk = wide_chunk_rows();
+  const int64_t chunk = static_cast<int64_t>(kQuantChunkTiles) * kTM;
   const int64_t rows_cap = n_rows < chunk ? n_rows : chunk;
   const uint32_t fix_cap = static_cast<uint32_t>(rows_cap * m / 8);
   const size_t res_bytes = static_cast<size_t>(rows_cap) * 2 * d * 2;
@@ -966,6 +970,7 @@ int launch_quantize_wide(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_
   A.s = static_cast<float>(8 * pow2_at_least_sqrt(d));
   uint32_t* fix = reinterpret_cast<uint32_t*>(base + fix_off);
   uint32_t* nfix = reinterpret_cast<uint32_t*>(base + cnt_off);
+  A.nfix = nfix;
 
   CUtensorMap ta, tb;
   int err;
@@ -990,7 +995,6 @@ int launch_quantize_wide(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_
     const int64_t nr = n_rows - r0 < chunk ? n_rows - r0 : chunk;
     const Packed po{out.codes + r0 * P.codes_bytes, out.signs + r0 * P.signs_bytes, out.norm + r0, out.rnorm + r0};
     const void* xr = static_cast<const uint8_t*>(x) + r0 * ld * (x_is_bf16 ? 2 : 4);
-    if ((e = cudaMemsetAsync(nfix, 0, 4, s)) != cudaSuccess) return static_cast<int>(e);
     switch (d / 32) {
       case 8: err = launch_prep_E<8>(P, xr, x_is_bf16, nr, ld, po, A, ctx.num_sms, s); break;
       case 16: err = launch_prep_E<16>(P, xr, x_is_bf16, nr, ld, po, A, ctx.num_sms, s); break;

@@ -3,7 +3,7 @@ QJL projection of the write half as an fp16 GEMM with a listed fp64 fix-up of
 the projections inside its error bound, and the all-pairs estimates as an
 fp16 GEMM over decoded keys and split queries.
 
-Row counts span more than one 18944-row chunk (148 tiles of 128 rows) and end
+Row counts span more than one write-half chunk (296 tiles of 128 rows) and end
 in a ragged tile; query counts end in a ragged 256-column tile.  Codes, signs,
 norms and estimates follow the oracle rules of tests/parity.py.
 """
@@ -30,7 +30,7 @@ def tq():
 
 
 @pytest.mark.parametrize("d,b,m,dtype,n", [
-    (256, 3, 256, "f32", 2 * CHUNK + 1001),
+    (256, 3, 256, "f32", 2 * CHUNK + 1001),     # two write-half chunks (37888 rows each)
     (256, 2, 96, "bf16", CHUNK + 77),
     (512, 4, 128, "bf16", 4096),
     (1024, 4, 1024, "f32", CHUNK + 777),
@@ -91,7 +91,8 @@ def test_wide_quantize_then_logits_end_to_end(tq):
 
 
 @pytest.mark.parametrize("d,b,m,n_q,n_keys,k,qdtype", [
-    (256, 3, 256, 300, CHUNK + 513, 10, "f32"),     # fused: two chunks, ragged key and query tiles
+    (256, 3, 256, 300, CHUNK + 513, 10, "f32"),     # fused: ragged key and query tiles
+    (256, 3, 256, 64, 80000, 10, "f32"),             # fused: lists carried across two key chunks
     (1024, 4, 1024, 64, 5000, 16, "bf16"),           # fused, k = 16
     (512, 2, 128, 100, 4096, 1, "f32"),              # fused, k = 1
     (128, 3, 128, 37, 3000, 10, "bf16"),             # through the scores (d = 128)
