@@ -27,6 +27,11 @@
 // 48 KB TMA stages; one thread issues the loads, one the MMAs, and the four
 // warps read the accumulators back (warp w owns TMEM lanes 32w..32w+31).
 //
+// The vector search (tq_search) runs the read-half product with the roles
+// swapped -- A = the split queries, B = the decoded keys -- in a persistent
+// kernel (k_search_tc) whose epilogue threads each own one query and keep its
+// running top-k in registers across key tiles, so no score is written.
+//
 // A projection is given its sign by the tensor cores only where |p_j|
 // exceeds a bound on the product's error: the split's 2^-22 plus d/8 fp32
 // accumulation steps of at most 2^-22 of sum |S_ji r_i| <= ||S_j|| ||r||
