@@ -80,7 +80,27 @@ def test_host_calls_validate_before_any_launch():
     assert tq.call_status("tq_attention", None, None, 0, 1, 4, P, P, 10, ctypes.c_float(0.1), 0, None, None, 0,
                           None) == tq.TQ_ERR_INVALID_ARG
     assert tq._lib.tq_attention_workspace_bytes(None, 1, 4, 10) == 0
+    # vector search and the channel split: a NULL context is refused before any launch
+    assert tq.call_status("tq_search", None, None, 0, 64, P, 4096, 10, None, None, None, 0,
+                          None) == tq.TQ_ERR_INVALID_ARG
+    assert tq._lib.tq_search_workspace_bytes(None, 64, 4096, 10) == 0
+    assert tq.call_status("tq_split_quantize", None, None, 0, 10, 128, P, P, None) == tq.TQ_ERR_INVALID_ARG
+    assert tq.call_status("tq_split_logits", None, None, 0, 1, 4, P, P, 10, None, None, 0,
+                          None) == tq.TQ_ERR_INVALID_ARG
+    assert tq.call_status("tq_split_dequant", None, P, P, 10, None, 0, 0, None) == tq.TQ_ERR_INVALID_ARG
+    assert tq._lib.tq_split_logits_workspace_bytes(None, 1, 4, 10) == 0
+    assert tq.call_status("tq_split_destroy", None) == tq.TQ_OK
     assert tq.launch_count() == before
+
+
+@pytest.mark.parametrize("d,d_hi", [(128, 48), (128, 128), (64, 16), (128, 0), (96, 100)])
+def test_split_rejects_bad_channel_splits_on_the_host(d, d_hi):
+    """Both parts need a multiple of 32 channels, at least 32: checked before
+    any device call, so it holds without a GPU."""
+    tq = _lib()
+    h = ctypes.c_void_p()
+    assert tq.call_status("tq_split_init", d, d_hi, 3, 2, 0, ctypes.byref(h)) == tq.TQ_ERR_INVALID_ARG
+    assert not h.value
 
 
 def test_init_without_device_fails_cleanly():
