@@ -76,21 +76,26 @@ UNIT = "logits/s"
 KERNEL_OF = {"quantize": "k_quantize_d128_rot_tc", "logits": "k_logits_d128_i8", "dequant": "k_dequant_d128_tc"}
 
 
-def captured_traffic(kernel: str, units: int):
-    """DRAM bytes per launch of `kernel` from the committed ncu capture summary
-    (profiles/traffic.json), scaled by the units one launch processes -- or
-    None when there is no capture or the kernel's source changed since."""
+def captured_traffic(kernel: str, b: int, units: int):
+    """DRAM bytes per launch of `kernel` at bit width `b` from the committed ncu
+    capture summary (profiles/traffic.json: one entry per kernel and bit
+    width, DRAM bytes read + written per unit over one captured launch),
+    scaled by the units one launch processes -- or None when there is no
+    capture of that kernel at that bit width, or the kernel's source changed
+    since it was taken."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    entry = json.load(open(p)).get(KERNEL_OF.get(kernel, ""), None)
-    if not entry:
-        return None
-    src = os.path.join(ROOT, entry["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != entry["source_sha256"]:
-        return None
-    return entry["dram_bytes_per_unit"] * units
+    name = KERNEL_OF.get(kernel, "")
+    for entry in json.load(open(p)).get("entries", []):
+        if entry.get("kernel") != name or int(entry.get("b", -1)) != b:
+            continue
+        src = os.path.join(ROOT, entry["source"])
+        if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != entry["source_sha256"]:
+            return None
+        return entry["dram_bytes_per_unit"] * units
+    return None
 
 
 def peaks():
@@ -289,7 +294,7 @@ def run_ours(args, cfg, ws, rank, local):
     pK, pV = T.empty_packed(N, dev), T.empty_packed(N, dev)
     logits = torch.empty((n_sets, g, n_keys), dtype=torch.float32, device=dev)
     vhat = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
-    wbytes = T.workspace_bytes(n_sets, g)
+    wbytes = T.workspace_bytes(n_sets, g, n_keys)
     work = torch.empty(max(wbytes, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -484,7 +489,7 @@ def run_ours(args, cfg, ws, rank, local):
                                       "no data-path collective)",
                        "l2": "inputs larger than L2 (K, V 2.1 GB each); no flush"},
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dk["gbs"], "peak": hbm,
-                         "unit": "GB/s", "frac": dk["frac_hbm"], "traffic": captured_traffic(dominant, N),
+                         "unit": "GB/s", "frac": dk["frac_hbm"], "traffic": captured_traffic(dominant, cfg["b"], N),
                          "algorithmic_bytes": dk["bytes"], "peak_kind": hbm_kind},
             "quantize_rows_per_s": total_rows / (q_ms * 1e-3),
             "kernels": {k: {"ms_per_launch": v["ms"], "algorithmic_GBps": v["gbs"], "frac_hbm": v["frac_hbm"],
@@ -629,6 +634,7 @@ def run_aux(args, cfg, ws, rank, local):
         idx = torch.empty((nq, kq), dtype=torch.int32, device=dev)
         val = torch.empty((nq, kq), dtype=torch.float32, device=dev)
         work = torch.empty(max(T.search_workspace_bytes(nq, ndb, kq), 16), dtype=torch.uint8, device=dev)
+        qwork = torch.empty(max(T.quantize_workspace_bytes(ndb), 16), dtype=torch.uint8, device=dev)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         split = {"quantize": 0.0, "search": 0.0}
 
@@ -637,7 +643,7 @@ def run_aux(args, cfg, ws, rank, local):
             # inner product (estimates on the tensor cores, top-k fused into
             # their epilogue)
             if timed: ev[0].record(stream)
-            T.quantize(ddb, pk, stream=stream)
+            T.quantize(ddb, pk, workspace=qwork, stream=stream)
             if timed: ev[1].record(stream)
             T.search(dq, pk, ndb, kq, idx=idx, val=val, workspace=work, stream=stream)
             if timed:

@@ -27,12 +27,11 @@
  *   - Tensor pointers are DEVICE pointers owned by the caller, unless a
  *     parameter says "host".  The library never frees them.
  *   - Compute calls are asynchronous on the CUDA stream passed as `stream`
- *     (a cudaStream_t; NULL = legacy default stream) and allocate nothing,
- *     except tq_quantize and tq_logits on wide rows (d >= 256, at least 4096
- *     rows or keys), which take stream-ordered scratch on `stream` from a
- *     memory pool the context owns (cudaMallocFromPoolAsync / cudaFreeAsync;
- *     the pool keeps the memory between calls and is released by tq_destroy);
- *     a failed scratch allocation returns TQ_ERR_CUDA.
+ *     (a cudaStream_t; NULL = legacy default stream) and allocate nothing.
+ *     A call that needs device scratch takes it from a caller-provided
+ *     `workspace` whose size the matching *_workspace_bytes function gives
+ *     (16-byte aligned; used only by that call's kernels on `stream`, so two
+ *     calls in flight at once need two workspaces).
  *   - Arguments are checked on the host before any launch.  A failed check
  *     returns a status and launches nothing; tq_last_error() then gives a
  *     one-line reason (thread-local, valid until the next call on the thread).
@@ -127,12 +126,17 @@ tq_status tq_get_params(const tq_ctx* ctx, float* centroids, float* thresholds, 
  * power of two, x aligned to its element size otherwise) into `out`.
  * Per row: norm, rotation, Lloyd-Max codes, QJL signs of the residual,
  * residual norm (write half above).  One launch at d = 128 and for small
- * batches.  Wide rows (d >= 256, n_rows >= 4096) run per 18944-row chunk: a
+ * batches.  Wide rows (d >= 256, n_rows >= 4096) run per 37888-row chunk: a
  * CUDA-core kernel (norm, rotation, codes, residual halves), a tensor-core
  * GEMM for the projections and their signs, and a fix-up of the rare
- * projections inside the GEMM's error bound (recomputed in fp64). */
+ * projections inside the GEMM's error bound (recomputed in fp64); their
+ * scratch (residual halves, fix-up list) is the workspace.
+ *   workspace: device memory of at least tq_quantize_workspace_bytes(ctx,
+ *   n_rows) bytes, 16-byte aligned (may be NULL when that is 0, which it is
+ *   at d = 128 and for the general kernels). */
+size_t tq_quantize_workspace_bytes(const tq_ctx* ctx, int64_t n_rows);
 tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
-                      tq_packed out, void* stream);
+                      tq_packed out, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ----------------------------------------------------------- read half -- */
 
@@ -149,9 +153,11 @@ tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_
 tq_status tq_quantize_scatter(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
                               const int64_t* dest_rows, int64_t n_cache_rows, tq_packed cache, void* stream);
 
-/* Device workspace that tq_logits needs for n_sets * g queries (bytes; 0 when
- * the call needs none, in which case workspace may be NULL). */
-size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g);
+/* Device workspace that tq_logits needs for n_sets * g queries against
+ * n_keys keys per set (bytes; 0 for an empty call): the query operands
+ * (R q | S R q, fp32, per query), and on wide rows the tensor-core GEMM's
+ * operands (keys decoded to binary16, 18944 at a time, and the split queries). */
+size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g, int64_t n_keys);
 
 /* Estimated logits of queries against packed keys (estimator above; no
  * 1/sqrt(d) softmax scale).
@@ -161,10 +167,10 @@ size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g);
  * For grouped-query attention a set is one (batch, kv head) pair and g the
  * number of query heads sharing it; for vector search n_sets = 1 and g the
  * number of queries.  g in [1, 4096].  workspace: device memory of at least
- * tq_logits_workspace_bytes(ctx, n_sets, g) bytes, 16-byte aligned, not used
- * concurrently by another call.  With d >= 256, m a multiple of 64, g >= 64
- * and n_keys >= 4096 the estimates run as a tensor-core GEMM over keys
- * decoded into binary16 operands, 18944 keys at a time. */
+ * tq_logits_workspace_bytes(ctx, n_sets, g, n_keys) bytes, 16-byte aligned,
+ * not used concurrently by another call.  With d >= 256, m a multiple of 64,
+ * g >= 64 and n_keys >= 4096 the estimates run as a tensor-core GEMM over
+ * keys decoded into binary16 operands, 18944 keys at a time. */
 tq_status tq_logits(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
                     tq_packed keys, int64_t n_keys, float* out, void* workspace, size_t workspace_bytes,
                     void* stream);
@@ -174,14 +180,20 @@ tq_status tq_logits(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t 
  * own the device memory pool, a plug-in barred from the CUDA allocator, a
  * latency-critical path that must not risk the synchronization an allocation
  * can cause).  The pages describe no such call: it is an interface
- * convenience of this library.  Same arguments and results as tq_logits; the
- * per-query operands go to a 4 MiB scratch array compiled into the library
- * (held on every device that loads it until the process exits), so
- * n_sets * g * (d + m) * 4 must be at most 4 MiB (else TQ_ERR_UNSUPPORTED, no
- * launch).  Allocates nothing.  The first call on each device looks up the
- * array's device address (make it before any stream capture).  All calls
- * share the array: calls that may overlap on the GPU race and must be
- * serialized by the caller. */
+ * convenience of this library.  Same arguments, checks and results as
+ * tq_logits, without the workspace: the per-query operands go to a 4 MiB
+ * scratch array compiled into the library (held on every device that loads
+ * it until the process exits), so n_sets * g * (d + m) * 4 must be at most
+ * 4 MiB (else TQ_ERR_UNSUPPORTED, no launch).  On wide rows, where tq_logits
+ * would decode keys into a GEMM operand, this call runs the general logit
+ * kernels on the packed keys instead (results within the logit tolerance of
+ * tq_logits', not bit-identical).  Allocates nothing.  The first call with a
+ * given CUDA context current looks up the array's device address in that
+ * context and caches it (make that call before any stream capture; a context
+ * destroyed by cudaDeviceReset leaves a stale cached address, so processes
+ * that reset the device should not use this call).  All calls share the
+ * array: calls that may overlap on the GPU race and must be serialized by
+ * the caller. */
 tq_status tq_logits_noalloc(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
                             tq_packed keys, int64_t n_keys, float* out, void* stream);
 
@@ -218,8 +230,9 @@ tq_status tq_dequant(const tq_ctx* ctx, tq_packed in, int64_t n_rows, void* out,
 /* Vector search: for each of n_q queries, the k packed rows (of n_keys) with
  * the largest estimated inner product (the tq_logits estimator with
  * n_sets = 1, g = n_q), larger first, equal estimates by lower row index
- * (Google Research blog "TurboQuant: Redefining AI efficiency with extreme
- * compression", vector search: the top-k is the search's answer).  When the
+ * (0h-n0 "ICLR 2026論文解説: TurboQuant", "実験結果 — ベクトル検索（Recall評価）":
+ * Recall@k of a 4-bit database; Qiita TurboQuant explainer, "ベクトル検索への応用").
+ * When the
  * wide-row path applies (d >= 256, m a multiple of 64, n_q >= 64,
  * n_keys >= 4096) no score is written: a persistent tensor-core kernel keeps
  * each query's running top-k in registers while it streams the keys, and the

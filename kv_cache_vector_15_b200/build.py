@@ -31,8 +31,18 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _compile(src: str, verbose: bool) -> str:
+def _headers_mtime() -> float:
+    hs = glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
+        glob.glob(os.path.join(ROOT, "include", "*.h"))
+    return max((os.path.getmtime(h) for h in hs), default=0.0)
+
+
+def _compile(src: str, verbose: bool, force: bool = False) -> str:
     obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+    # objects newer than their source and every header are reused
+    if not force and not verbose and os.path.exists(obj) and \
+            os.path.getmtime(obj) > max(os.path.getmtime(src), _headers_mtime()):
+        return obj
     cmd = [nvcc(), *ARCH, *COMMON, "-c", src, "-o", obj]
     if src.endswith(".cu") and verbose:
         cmd += ["-Xptxas", "-v"]

@@ -1,23 +1,35 @@
 // Kernel selection: the d = 128 hot-path kernels where they apply, then the
-// wide-row tensor-core paths (d >= 256, many rows), the general kernels
-// everywhere else.
+// wide-row tensor-core paths (d >= 256, many rows; only when the caller's
+// workspace holds their scratch), the general kernels everywhere else.
 #include "tq_internal.h"
 
 namespace tq {
 
+size_t quantize_scratch_bytes(const tq_ctx& ctx, int64_t n_rows) {
+  if (quantize_d128_applies(ctx, n_rows)) return 0;
+  return wide_quantize_applies(ctx, n_rows) ? wide_quantize_scratch_bytes(ctx, n_rows) : 0;
+}
+
 int launch_quantize(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x, const Packed& out,
-                    void* stream) {
+                    void* scratch, void* stream) {
   if (quantize_d128_applies(ctx, n_rows))
     return launch_quantize_d128(ctx, x, x_is_bf16, n_rows, ld_x, out, stream);
-  if (wide_quantize_applies(ctx, n_rows)) return launch_quantize_wide(ctx, x, x_is_bf16, n_rows, ld_x, out, stream);
+  if (scratch && wide_quantize_applies(ctx, n_rows))
+    return launch_quantize_wide(ctx, x, x_is_bf16, n_rows, ld_x, out, scratch, stream);
   return launch_quantize_generic(ctx.kp, x, x_is_bf16, n_rows, ld_x, out, stream);
 }
 
+size_t logits_scratch_bytes(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys) {
+  if (logits_d128_applies(ctx, n_sets, g, n_keys)) return 0;
+  return wide_logits_applies(ctx, n_sets, g, n_keys) ? wide_logits_scratch_bytes(ctx, n_sets, g, n_keys) : 0;
+}
+
 int launch_logits(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
-                  float* out, void* stream) {
+                  float* out, void* scratch, void* stream) {
   if (logits_d128_applies(ctx, n_sets, g, n_keys))
     return launch_logits_d128(ctx, qp, n_sets, g, keys, n_keys, out, stream);
-  if (wide_logits_applies(ctx, n_sets, g, n_keys)) return launch_logits_wide(ctx, qp, n_sets, g, keys, n_keys, out, stream);
+  if (scratch && wide_logits_applies(ctx, n_sets, g, n_keys))
+    return launch_logits_wide(ctx, qp, n_sets, g, keys, n_keys, out, scratch, stream);
   return launch_logits_generic(ctx.kp, qp, n_sets, g, keys, n_keys, out, stream);
 }
 

@@ -11,16 +11,24 @@
 // loads the library keeps until the process exits.  Nothing is allocated on
 // any call.
 //
-// The device address of that array is looked up once per device, on the
-// first call made with that device current (cudaGetSymbolAddress), and cached.
-// Make that first call before any stream capture begins.
+// Only the query operands go to the array.  On wide rows, where tq_logits
+// would decode the keys into a binary16 operand for the tensor-core GEMM (a
+// scratch of tens of megabytes), this call runs the general logit kernels
+// instead, which read the packed keys directly; the results agree with
+// tq_logits within the logit tolerance, not bit for bit.
 //
-// All calls share the one array, whatever their context or stream: calls that
-// may overlap on the GPU (different streams, or different host threads) race
-// on it and must be serialized by the caller.  The array keeps the previous
-// call's contents; nothing in it needs to start at zero, because the query
-// preparation kernel writes every byte the logit kernel reads.
+// The device address of that array is looked up once per CUDA context, on
+// the first call made with that context current (cudaGetSymbolAddress), and
+// cached (up to kMaxContexts contexts per process).  Make that first call
+// before any stream capture begins.
+//
+// All calls share the one array of a context, whatever their stream: calls
+// that may overlap on the GPU (different streams, or different host threads)
+// race on it and must be serialized by the caller.  The array keeps the
+// previous call's contents; nothing in it needs to start at zero, because the
+// query preparation kernel writes every byte the logit kernel reads.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -31,39 +39,71 @@
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;    // 4 MiB
-constexpr int kMaxDevices = 64;
+constexpr int kMaxContexts = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+CUcontext g_ctx_key[kMaxContexts] = {};
+void* g_scratch_addr[kMaxContexts] = {};
+int g_n_cached = 0;
+
+// cuCtxGetCurrent through the runtime's driver entry point (no libcuda link)
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  return fn;
+}
 
 }  // namespace
 
 extern "C" tq_status tq_logits_noalloc(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
                                        tq_packed keys, int64_t n_keys, float* out, void* stream) {
-  if (!ctx) return tq::fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
-  if (n_sets < 0 || n_keys < 0) return tq::fail(TQ_ERR_INVALID_ARG, "n_sets and n_keys must be >= 0");
-  if (g < 1 || g > 4096) return tq::fail(TQ_ERR_INVALID_ARG, "g must be in [1, 4096]");
-  const size_t need = tq_logits_workspace_bytes(ctx, n_sets, g);
+  bool empty = false;
+  tq_status st = tq::logits_args(ctx, q, q_dtype, n_sets, g, keys, n_keys, out, &empty);
+  if (st != TQ_OK || empty) return st;
+  const size_t need = tq::qprep_bytes(ctx, n_sets * g);
   if (need > kNoAllocScratchBytes)
     return tq::fail(TQ_ERR_UNSUPPORTED, "n_sets * g * (d + m) * 4 = " + std::to_string(need) +
                                             " bytes exceeds the 4 MiB static scratch of tq_logits_noalloc");
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return tq::fail(TQ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices) return tq::fail(TQ_ERR_UNSUPPORTED, "device ordinal beyond 63");
+  CtxGetCurrentFn get = ctx_get_current();
+  if (!get) return tq::fail(TQ_ERR_CUDA, "cuCtxGetCurrent is not available");
+  CUcontext cu = nullptr;
+  cudaError_t e = cudaSuccess;
+  if (get(&cu) != CUDA_SUCCESS) return tq::fail(TQ_ERR_CUDA, "cuCtxGetCurrent failed");
+  if (!cu) {
+    // no context bound to this thread yet: the runtime binds the device's
+    // primary context on its first call that needs one, as this lookup does
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return tq::fail(TQ_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    if (get(&cu) != CUDA_SUCCESS || !cu) return tq::fail(TQ_ERR_CUDA, "no current CUDA context");
+  }
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
+    for (int i = 0; i < g_n_cached; ++i)
+      if (g_ctx_key[i] == cu) scratch = g_scratch_addr[i];
+    if (!scratch) {
+      if (g_n_cached == kMaxContexts) return tq::fail(TQ_ERR_UNSUPPORTED, "more than 64 CUDA contexts");
       void* p = nullptr;
       e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
       if (e != cudaSuccess || !p)
         return tq::fail(TQ_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
-      g_scratch_addr[dev] = p;
+      g_ctx_key[g_n_cached] = cu;
+      g_scratch_addr[g_n_cached] = p;
+      ++g_n_cached;
+      scratch = p;
     }
-    scratch = g_scratch_addr[dev];
   }
-  return tq_logits(ctx, q, q_dtype, n_sets, g, keys, n_keys, out, scratch, kNoAllocScratchBytes, stream);
+  return tq::logits_checked(ctx, q, q_dtype, n_sets, g, keys, n_keys, out, static_cast<float*>(scratch), nullptr,
+                            stream);
 }

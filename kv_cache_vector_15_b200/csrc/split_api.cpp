@@ -91,15 +91,19 @@ tq_status tq_split_quantize(const tq_split* sp, const void* x, tq_dtype x_dtype,
   if (st != TQ_OK) return st;
   if (x_dtype != TQ_BF16 && x_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "x_dtype must be TQ_BF16 or TQ_F32");
   if (ld_x < sp->d) return fail(TQ_ERR_INVALID_ARG, "ld_x < d");
-  if ((st = tq_quantize(sp->part[0], x, x_dtype, n_rows, ld_x, out_hi, stream)) != TQ_OK) return st;
+  if (n_rows < 0) return fail(TQ_ERR_INVALID_ARG, "n_rows < 0");
+  for (int p = 0; p < 2; ++p)
+    if ((st = check_ctx(sp->part[p])) != TQ_OK) return st;
+  if (n_rows == 0) return TQ_OK;
+  // each part on its own kernels (no workspace: a wide part takes the general path)
+  if ((st = quantize_checked(sp->part[0], x, x_dtype, n_rows, ld_x, out_hi, nullptr, stream)) != TQ_OK) return st;
   const void* x_lo = x ? static_cast<const uint8_t*>(x) + static_cast<size_t>(sp->d_hi) * esize(x_dtype) : nullptr;
-  return tq_quantize(sp->part[1], x_lo, x_dtype, n_rows, ld_x, out_lo, stream);
+  return quantize_checked(sp->part[1], x_lo, x_dtype, n_rows, ld_x, out_lo, nullptr, stream);
 }
 
 size_t tq_split_logits_workspace_bytes(const tq_split* sp, int64_t n_sets, int g, int64_t n_keys) {
   if (!sp || n_sets <= 0 || g <= 0 || n_keys <= 0) return 0;
-  return r16(tq_logits_workspace_bytes(sp->part[0], n_sets, g)) +
-         r16(tq_logits_workspace_bytes(sp->part[1], n_sets, g)) +
+  return r16(qprep_bytes(sp->part[0], n_sets * g)) + r16(qprep_bytes(sp->part[1], n_sets * g)) +
          r16(static_cast<size_t>(n_sets) * g * n_keys * sizeof(float));
 }
 
@@ -123,9 +127,8 @@ tq_status tq_split_logits(const tq_split* sp, const void* q, tq_dtype q_dtype, i
   uint8_t* w = static_cast<uint8_t*>(workspace);
   float* qp[2];
   qp[0] = reinterpret_cast<float*>(w);
-  qp[1] = reinterpret_cast<float*>(w + r16(tq_logits_workspace_bytes(sp->part[0], n_sets, g)));
-  float* half = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(qp[1]) +
-                                         r16(tq_logits_workspace_bytes(sp->part[1], n_sets, g)));
+  qp[1] = reinterpret_cast<float*>(w + r16(qprep_bytes(sp->part[0], n_sets * g)));
+  float* half = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(qp[1]) + r16(qprep_bytes(sp->part[1], n_sets * g)));
   const tq_packed* keys[2] = {&keys_hi, &keys_lo};
   const size_t off[2] = {0, static_cast<size_t>(sp->d_hi) * esize(q_dtype)};
   for (int p = 0; p < 2; ++p) {
@@ -134,7 +137,7 @@ tq_status tq_split_logits(const tq_split* sp, const void* q, tq_dtype q_dtype, i
     int err = launch_qprep(P, static_cast<const uint8_t*>(q) + off[p], q_dtype == TQ_BF16, n_sets * g, qp[p], stream);
     if (err) return cuda_err(err, "tq_split_logits query-prep launch");
     const Packed k{keys[p]->codes, keys[p]->signs, keys[p]->norm, keys[p]->rnorm};
-    err = launch_logits(*sp->part[p], qp[p], n_sets, g, k, n_keys, p == 0 ? out : half, stream);
+    err = launch_logits(*sp->part[p], qp[p], n_sets, g, k, n_keys, p == 0 ? out : half, nullptr, stream);
     if (err) return cuda_err(err, "tq_split_logits launch");
   }
   int err = launch_add(out, half, n_sets * g * n_keys, stream);

@@ -45,7 +45,7 @@ static tq_status cuda_fail(int err, const char* what) {
   return fail(TQ_ERR_CUDA, std::string(what) + ": " + cuda_error_string(err));
 }
 
-static tq_status check_ctx(const tq_ctx* ctx) {
+tq_status check_ctx(const tq_ctx* ctx) {
   if (!ctx) return fail(TQ_ERR_INVALID_ARG, "ctx is NULL");
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(TQ_ERR_CUDA, "cudaGetDevice failed");
@@ -64,6 +64,61 @@ static tq_status check_packed(const tq_ctx* ctx, const tq_packed& p) {
 }
 
 static Packed to_internal(const tq_packed& p) { return Packed{p.codes, p.signs, p.norm, p.rnorm}; }
+
+// tq_quantize after its context, count and workspace checks: the remaining
+// argument checks, then the launch (scratch null: no wide-row path)
+tq_status quantize_checked(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
+                           const tq_packed& out, void* scratch, void* stream) {
+  if (!x) return fail(TQ_ERR_INVALID_ARG, "x is NULL");
+  const size_t esz = x_dtype == TQ_BF16 ? 2 : 4;
+  if (ld_x < ctx->d_in) return fail(TQ_ERR_INVALID_ARG, "ld_x < d");
+  if (ctx->d_in == ctx->d) {
+    if (!aligned(x, 16) || (static_cast<size_t>(ld_x) * esz) % 16)
+      return fail(TQ_ERR_INVALID_ARG, "x and its row stride must be 16-byte aligned");
+  } else if (!aligned(x, esz)) {        // padded rows are read element by element
+    return fail(TQ_ERR_INVALID_ARG, "x must be aligned to its element size");
+  }
+  tq_status st = check_packed(ctx, out);
+  if (st != TQ_OK) return st;
+  int err = launch_quantize(*ctx, x, x_dtype == TQ_BF16, n_rows, ld_x, to_internal(out), scratch, stream);
+  if (err) return cuda_fail(err, "tq_quantize launch");
+  return TQ_OK;
+}
+
+size_t round16(size_t v) { return (v + 15) & ~static_cast<size_t>(15); }
+size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+// bytes of the query operands (R q | S R q per query) at the front of a
+// logits workspace
+size_t qprep_bytes(const tq_ctx* ctx, int64_t n_q) {
+  return static_cast<size_t>(n_q) * (ctx->d + ctx->m) * sizeof(float);
+}
+
+// tq_logits after its argument checks: query prep into qp, then the logit
+// kernels (scratch null: no wide-row path)
+tq_status logits_checked(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
+                         const tq_packed& keys, int64_t n_keys, float* out, float* qp, void* scratch, void* stream) {
+  int err = launch_qprep(ctx->kp, q, q_dtype == TQ_BF16, n_sets * g, qp, stream);
+  if (err) return cuda_fail(err, "tq_logits query-prep launch");
+  err = launch_logits(*ctx, qp, n_sets, g, to_internal(keys), n_keys, out, scratch, stream);
+  if (err) return cuda_fail(err, "tq_logits launch");
+  return TQ_OK;
+}
+
+// the checks tq_logits makes before it looks at the workspace
+tq_status logits_args(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
+                      const tq_packed& keys, int64_t n_keys, const float* out, bool* empty) {
+  *empty = false;
+  tq_status st = check_ctx(ctx);
+  if (st != TQ_OK) return st;
+  if (n_sets < 0 || n_keys < 0) return fail(TQ_ERR_INVALID_ARG, "n_sets and n_keys must be >= 0");
+  if (g < 1 || g > 4096) return fail(TQ_ERR_INVALID_ARG, "g must be in [1, 4096]");
+  if (q_dtype != TQ_BF16 && q_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "q_dtype must be TQ_BF16 or TQ_F32");
+  if (n_sets == 0 || n_keys == 0) { *empty = true; return TQ_OK; }
+  if (!q || !out) return fail(TQ_ERR_INVALID_ARG, "q or out is NULL");
+  if (!aligned(q, 16) || !aligned(out, 4)) return fail(TQ_ERR_INVALID_ARG, "q must be 16-byte and out 4-byte aligned");
+  return check_packed(ctx, keys);
+}
 
 double half_bits_to_double(uint16_t h) {
   const int sign = (h >> 15) & 1, e = (h >> 10) & 31, f = h & 1023;
@@ -220,23 +275,6 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
       ctx->colsum_d128[i] = static_cast<float>(acc);
     }
   }
-  // wide rows: a memory pool for the stream-ordered scratch of the tensor-core
-  // paths, kept (not released to the device) between calls
-  ctx->pool = nullptr;
-  if (d >= 256) {
-    cudaMemPoolProps props{};
-    props.allocType = cudaMemAllocationTypePinned;
-    props.location.type = cudaMemLocationTypeDevice;
-    props.location.id = dev;
-    cudaMemPool_t pool = nullptr;
-    if (cudaMemPoolCreate(&pool, &props) == cudaSuccess) {
-      uint64_t keep = UINT64_MAX;
-      cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-      ctx->pool = pool;
-    } else {
-      cudaGetLastError();                              // the general kernels serve instead
-    }
-  }
   *out = ctx;
   return TQ_OK;
 }
@@ -244,8 +282,6 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
 tq_status tq_destroy(tq_ctx* ctx) {
   if (!ctx) return TQ_OK;
   cudaError_t e = cudaSuccess;
-  // a pool whose stream-ordered frees are still queued is released once they complete
-  if (ctx->pool) cudaMemPoolDestroy(static_cast<cudaMemPool_t>(ctx->pool));
   if (ctx->dev_block) e = cudaFree(ctx->dev_block);
   delete ctx;
   if (e != cudaSuccess) return cuda_fail(e, "cudaFree");
@@ -269,26 +305,24 @@ tq_status tq_get_params(const tq_ctx* ctx, float* centroids, float* thresholds, 
   return TQ_OK;
 }
 
+size_t tq_quantize_workspace_bytes(const tq_ctx* ctx, int64_t n_rows) {
+  if (!ctx || n_rows <= 0) return 0;
+  return quantize_scratch_bytes(*ctx, n_rows);
+}
+
 tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
-                      tq_packed out, void* stream) {
+                      tq_packed out, void* workspace, size_t workspace_bytes, void* stream) {
   tq_status st = check_ctx(ctx);
   if (st != TQ_OK) return st;
   if (n_rows < 0) return fail(TQ_ERR_INVALID_ARG, "n_rows < 0");
   if (x_dtype != TQ_BF16 && x_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "x_dtype must be TQ_BF16 or TQ_F32");
   if (n_rows == 0) return TQ_OK;
-  if (!x) return fail(TQ_ERR_INVALID_ARG, "x is NULL");
-  const size_t esz = x_dtype == TQ_BF16 ? 2 : 4;
-  if (ld_x < ctx->d_in) return fail(TQ_ERR_INVALID_ARG, "ld_x < d");
-  if (ctx->d_in == ctx->d) {
-    if (!aligned(x, 16) || (static_cast<size_t>(ld_x) * esz) % 16)
-      return fail(TQ_ERR_INVALID_ARG, "x and its row stride must be 16-byte aligned");
-  } else if (!aligned(x, esz)) {        // padded rows are read element by element
-    return fail(TQ_ERR_INVALID_ARG, "x must be aligned to its element size");
+  const size_t need = quantize_scratch_bytes(*ctx, n_rows);
+  if (need) {
+    if (!workspace || workspace_bytes < need) return fail(TQ_ERR_INVALID_ARG, "workspace missing or too small");
+    if (!aligned(workspace, 16)) return fail(TQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   }
-  if ((st = check_packed(ctx, out)) != TQ_OK) return st;
-  int err = launch_quantize(*ctx, x, x_dtype == TQ_BF16, n_rows, ld_x, to_internal(out), stream);
-  if (err) return cuda_fail(err, "tq_quantize launch");
-  return TQ_OK;
+  return quantize_checked(ctx, x, x_dtype, n_rows, ld_x, out, need ? workspace : nullptr, stream);
 }
 
 tq_status tq_quantize_scatter(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
@@ -310,40 +344,29 @@ tq_status tq_quantize_scatter(const tq_ctx* ctx, const void* x, tq_dtype x_dtype
   return TQ_OK;
 }
 
-size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g) {
-  if (!ctx || n_sets <= 0 || g <= 0) return 0;
-  return static_cast<size_t>(n_sets) * g * (ctx->d + ctx->m) * sizeof(float);
+size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g, int64_t n_keys) {
+  if (!ctx || n_sets <= 0 || g <= 0 || n_keys <= 0) return 0;
+  const size_t wide = logits_scratch_bytes(*ctx, n_sets, g, n_keys);
+  return wide ? round256(qprep_bytes(ctx, n_sets * g)) + wide : qprep_bytes(ctx, n_sets * g);
 }
 
 tq_status tq_logits(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g, tq_packed keys,
                     int64_t n_keys, float* out, void* workspace, size_t workspace_bytes, void* stream) {
-  tq_status st = check_ctx(ctx);
-  if (st != TQ_OK) return st;
-  if (n_sets < 0 || n_keys < 0) return fail(TQ_ERR_INVALID_ARG, "n_sets and n_keys must be >= 0");
-  if (g < 1 || g > 4096) return fail(TQ_ERR_INVALID_ARG, "g must be in [1, 4096]");
-  if (q_dtype != TQ_BF16 && q_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "q_dtype must be TQ_BF16 or TQ_F32");
-  if (n_sets == 0 || n_keys == 0) return TQ_OK;
-  if (!q || !out) return fail(TQ_ERR_INVALID_ARG, "q or out is NULL");
-  if (!aligned(q, 16) || !aligned(out, 4)) return fail(TQ_ERR_INVALID_ARG, "q must be 16-byte and out 4-byte aligned");
-  if ((st = check_packed(ctx, keys)) != TQ_OK) return st;
-  const size_t need = tq_logits_workspace_bytes(ctx, n_sets, g);
-  if (need) {
-    if (!workspace || workspace_bytes < need) return fail(TQ_ERR_INVALID_ARG, "workspace missing or too small");
-    if (!aligned(workspace, 16)) return fail(TQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
-  }
-  float* qp = static_cast<float*>(workspace);
-  int err = launch_qprep(ctx->kp, q, q_dtype == TQ_BF16, n_sets * g, qp, stream);
-  if (err) return cuda_fail(err, "tq_logits query-prep launch");
-  err = launch_logits(*ctx, qp, n_sets, g, to_internal(keys), n_keys, out, stream);
-  if (err) return cuda_fail(err, "tq_logits launch");
-  return TQ_OK;
+  bool empty = false;
+  tq_status st = logits_args(ctx, q, q_dtype, n_sets, g, keys, n_keys, out, &empty);
+  if (st != TQ_OK || empty) return st;
+  const size_t need = tq_logits_workspace_bytes(ctx, n_sets, g, n_keys);
+  if (!workspace || workspace_bytes < need) return fail(TQ_ERR_INVALID_ARG, "workspace missing or too small");
+  if (!aligned(workspace, 16)) return fail(TQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  const bool wide = logits_scratch_bytes(*ctx, n_sets, g, n_keys) != 0;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  return logits_checked(ctx, q, q_dtype, n_sets, g, keys, n_keys, out, reinterpret_cast<float*>(w),
+                        wide ? w + round256(qprep_bytes(ctx, n_sets * g)) : nullptr, stream);
 }
-
-static size_t round16(size_t v) { return (v + 15) & ~static_cast<size_t>(15); }
 
 size_t tq_search_workspace_bytes(const tq_ctx* ctx, int64_t n_q, int64_t n_keys, int k) {
   if (!ctx || n_q <= 0 || n_keys <= 0 || k <= 0) return 0;
-  const size_t qp = round16(static_cast<size_t>(n_q) * (ctx->d + ctx->m) * sizeof(float));
+  const size_t qp = round256(qprep_bytes(ctx, n_q));
   if (wide_search_applies(*ctx, n_q, n_keys, k)) return qp + wide_search_partial_bytes(*ctx, n_q, n_keys, k);
   return qp + round16(static_cast<size_t>(n_q) * n_keys * sizeof(float));
 }
@@ -368,7 +391,7 @@ tq_status tq_search(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t 
   if (!aligned(workspace, 16)) return fail(TQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   uint8_t* w = static_cast<uint8_t*>(workspace);
   float* qp = reinterpret_cast<float*>(w);
-  void* rest = w + round16(static_cast<size_t>(n_q) * (ctx->d + ctx->m) * sizeof(float));
+  void* rest = w + round256(qprep_bytes(ctx, n_q));
   int err = launch_qprep(ctx->kp, q, q_dtype == TQ_BF16, n_q, qp, stream);
   if (err) return cuda_fail(err, "tq_search query-prep launch");
   if (wide_search_applies(*ctx, n_q, n_keys, k)) {
@@ -377,7 +400,7 @@ tq_status tq_search(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t 
     return TQ_OK;
   }
   float* scores = static_cast<float*>(rest);         // [n_q, n_keys], then the top-k of each row
-  err = launch_logits(*ctx, qp, 1, static_cast<int>(n_q), to_internal(keys), n_keys, scores, stream);
+  err = launch_logits(*ctx, qp, 1, static_cast<int>(n_q), to_internal(keys), n_keys, scores, nullptr, stream);
   if (err) return cuda_fail(err, "tq_search logits launch");
   err = launch_topk(scores, n_q, n_keys, k, idx, val, stream);
   if (err) return cuda_fail(err, "tq_search top-k launch");
@@ -386,7 +409,7 @@ tq_status tq_search(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t 
 
 size_t tq_attention_workspace_bytes(const tq_ctx* ctx, int64_t n_sets, int g, int64_t n_keys) {
   if (!ctx || n_sets <= 0 || g <= 0 || n_keys <= 0) return 0;
-  return round16(tq_logits_workspace_bytes(ctx, n_sets, g)) +
+  return round16(qprep_bytes(ctx, n_sets * g)) +
          round16(static_cast<size_t>(n_sets) * g * n_keys * sizeof(float)) +
          round16(attention_partial_bytes(ctx->kp, n_sets, g, n_keys));
 }
@@ -415,12 +438,12 @@ tq_status tq_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64
   if (!aligned(workspace, 16)) return fail(TQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   uint8_t* w = static_cast<uint8_t*>(workspace);
   float* qp = reinterpret_cast<float*>(w);
-  float* lg = reinterpret_cast<float*>(w + round16(tq_logits_workspace_bytes(ctx, n_sets, g)));
+  float* lg = reinterpret_cast<float*>(w + round16(qprep_bytes(ctx, n_sets * g)));
   float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(lg) +
                                          round16(static_cast<size_t>(n_sets) * g * n_keys * sizeof(float)));
   int err = launch_qprep(ctx->kp, q, q_dtype == TQ_BF16, n_sets * g, qp, stream);
   if (err) return cuda_fail(err, "tq_attention query-prep launch");
-  err = launch_logits(*ctx, qp, n_sets, g, to_internal(keys), n_keys, lg, stream);
+  err = launch_logits(*ctx, qp, n_sets, g, to_internal(keys), n_keys, lg, nullptr, stream);
   if (err) return cuda_fail(err, "tq_attention logits launch");
   err = launch_attention_tail(ctx->kp, lg, to_internal(values), n_sets, g, n_keys, scale,
                               mode == TQ_DEQUANT_PROD ? 1 : 0, part, out, stream);

@@ -39,6 +39,8 @@ struct Packed {
 };
 
 tq_status check_dims(int d, int b, int m);
+size_t round16(size_t v);
+size_t round256(size_t v);
 int padded_dim(int d);                // the next power of two >= d
 tq_status fail(tq_status s, const std::string& why);   // records tq_last_error()
 void count_launch(int n = 1);
@@ -58,13 +60,17 @@ int launch_logits_generic(const KParams& P, const float* qp, int64_t n_sets, int
                           int64_t n_keys, float* out, void* stream);
 int launch_dequant_generic(const KParams& P, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
                            void* stream);
+// scratch: the wide-row path's part of the caller's workspace, or null (the
+// wide-row path is then not taken)
+size_t quantize_scratch_bytes(const tq_ctx& ctx, int64_t n_rows);
 int launch_quantize(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x,
-                    const Packed& out, void* stream);
+                    const Packed& out, void* scratch, void* stream);
 int launch_quantize_scatter(const KParams& P, const void* x, int bf16, int64_t n_rows, int64_t ld,
                             const int64_t* dest, int64_t n_dest, const Packed& out, void* stream);
 int launch_qprep(const KParams& P, const void* q, int q_is_bf16, int64_t n_queries, float* qp, void* stream);
+size_t logits_scratch_bytes(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys);
 int launch_logits(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys,
-                  int64_t n_keys, float* out, void* stream);
+                  int64_t n_keys, float* out, void* scratch, void* stream);
 int launch_dequant(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
                    void* stream);
 // attention.cu: the softmax-weighted value sums after the logits are in place
@@ -92,13 +98,25 @@ int launch_logits_d128(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g
                        float* out, void* stream);
 int launch_dequant_d128(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
                         void* stream);
-// wide rows (d >= 256): tensor-core QJL projection and estimates (wide_tc.cu)
+// wide rows (d >= 256): tensor-core QJL projection and estimates (wide_tc.cu);
+// their scratch is part of the caller's workspace
 bool wide_quantize_applies(const tq_ctx& ctx, int64_t n_rows);
+size_t wide_quantize_scratch_bytes(const tq_ctx& ctx, int64_t n_rows);
 int launch_quantize_wide(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
-                         const Packed& out, void* stream);
+                         const Packed& out, void* scratch, void* stream);
 bool wide_logits_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys);
+size_t wide_logits_scratch_bytes(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys);
 int launch_logits_wide(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
-                       float* out, void* stream);
+                       float* out, void* scratch, void* stream);
+// tq_api.cpp: the compute entry points' shared steps, for the other C-ABI files
+tq_status check_ctx(const tq_ctx* ctx);      // non-null, and made on the current device
+tq_status quantize_checked(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
+                           const tq_packed& out, void* scratch, void* stream);
+size_t qprep_bytes(const tq_ctx* ctx, int64_t n_q);
+tq_status logits_args(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
+                      const tq_packed& keys, int64_t n_keys, const float* out, bool* empty);
+tq_status logits_checked(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int64_t n_sets, int g,
+                         const tq_packed& keys, int64_t n_keys, float* out, float* qp, void* scratch, void* stream);
 // vector search with the top-k fused into the estimates' epilogue
 bool wide_search_applies(const tq_ctx& ctx, int64_t n_q, int64_t n_keys, int k);
 size_t wide_search_partial_bytes(const tq_ctx& ctx, int64_t n_q, int64_t n_keys, int k);
@@ -121,7 +139,6 @@ struct tq_ctx {
   std::vector<uint16_t> S_bits;
   double s1max;                       // max_j ||S_j||_1
   const float* snorm_dev;             // [m] ||S_j||_2 on the device (in dev_block)
-  void* pool;                         // cudaMemPool_t for stream-ordered scratch (wide rows), or null
   void* dev_block;                    // one allocation holding everything below
   tq::KParams kp;
 };

@@ -7,8 +7,12 @@
 //     sqrt(pi/2)/m * rnorm <S R q, z>: Qiita TurboQuant explainer, "Stage 2:
 //     QJL"; ai.spot.hk "Google TurboQuant", "無偏內積估計";
 //   the vector-search use (quantize a database, estimate every query-row inner
-//     product, keep the best): Google Research blog "TurboQuant: Redefining AI
-//     efficiency with extreme compression", "Vector search".
+//     product, keep the best): 0h-n0.github.io "ICLR 2026論文解説: TurboQuant",
+//     "実験結果 — ベクトル検索（Recall評価）"; Qiita TurboQuant explainer,
+//     "ベクトル検索への応用".
+//
+// Scratch (residual halves, decoded keys, split queries, candidate lists)
+// lives in the workspace the caller passes; no call allocates device memory.
 //
 // Both products have an operand that is only exact in fp32, so it enters as
 // two binary16 halves (hi = rn(v), lo = rn(v - hi), |v - hi - lo| <= 2^-22 |v|)
@@ -911,12 +915,6 @@ int grid_warps(int64_t n, int nsm) {     // 8 warps per CTA, at most 16 CTAs per
   return static_cast<int>(want < cap ? want : cap);
 }
 
-struct PoolBuf {                         // stream-ordered scratch from the context's pool
-  void* p = nullptr;
-  cudaStream_t s = nullptr;
-  ~PoolBuf() { if (p) cudaFreeAsync(p, s); }
-};
-
 template <int E, bool BF16>
 int launch_prep(const KParams& P, const void* x, int64_t n_rows, int64_t ld, const Packed& out, const PrepArgs& A,
                 int nsm, cudaStream_t s) {
@@ -936,7 +934,7 @@ int launch_prep_E(const KParams& P, const void* x, int bf16, int64_t n_rows, int
 
 bool wide_applies(const tq_ctx& ctx) {
   const KParams& P = ctx.kp;
-  return ctx.use_tc && ctx.pool != nullptr && P.d >= 256 && P.d <= 4096 && P.m <= 4096 &&
+  return ctx.use_tc && P.d >= 256 && P.d <= 4096 && P.m <= 4096 &&
          tensor_map_encoder() != nullptr;
 }
 
@@ -952,23 +950,46 @@ bool wide_logits_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_key
 int64_t wide_chunk_rows() { return static_cast<int64_t>(kChunkTiles) * kTM; }
 
 
+namespace {
+// Write-half scratch of one call, carved from the caller's workspace:
+// residual halves [rows, 2d] binary16 | s ||r|| [rows] f32 | fix-up list
+// [rows m / 8] u32 | its counter, for one chunk of at most kQuantChunkTiles
+// row tiles.
+struct QuantScratch {
+  int64_t rows_cap;
+  uint32_t fix_cap;
+  size_t rn_off, fix_off, cnt_off, total;
+};
+QuantScratch quant_scratch(const KParams& P, int64_t n_rows) {
+  QuantScratch q{};
+  const int64_t chunk = static_cast<int64_t>(kQuantChunkTiles) * kTM;
+  q.rows_cap = n_rows < chunk ? n_rows : chunk;
+  q.fix_cap = static_cast<uint32_t>(q.rows_cap * P.m / 8);
+  const size_t res_bytes = static_cast<size_t>(q.rows_cap) * 2 * P.d * 2;
+  q.rn_off = (res_bytes + 255) / 256 * 256;
+  q.fix_off = q.rn_off + (static_cast<size_t>(q.rows_cap) * 4 + 255) / 256 * 256;
+  q.cnt_off = q.fix_off + (static_cast<size_t>(q.fix_cap) * 4 + 255) / 256 * 256;
+  q.total = q.cnt_off + 256;
+  return q;
+}
+}  // namespace
+
+size_t wide_quantize_scratch_bytes(const tq_ctx& ctx, int64_t n_rows) {
+  return quant_scratch(ctx.kp, n_rows).total;
+}
+
 int launch_quantize_wide(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
-                         const Packed& out, void* stream) {
+                         const Packed& out, void* scratch, void* stream) {
   const KParams& P = ctx.kp;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int d = P.d, m = P.m;
   const int64_t chunk = static_cast<int64_t>(kQuantChunkTiles) * kTM;
-  const int64_t rows_cap = n_rows < chunk ? n_rows : chunk;
-  const uint32_t fix_cap = static_cast<uint32_t>(rows_cap * m / 8);
-  const size_t res_bytes = static_cast<size_t>(rows_cap) * 2 * d * 2;
-  const size_t rn_off = (res_bytes + 255) / 256 * 256;
-  const size_t fix_off = rn_off + (static_cast<size_t>(rows_cap) * 4 + 255) / 256 * 256;
-  const size_t cnt_off = fix_off + (static_cast<size_t>(fix_cap) * 4 + 255) / 256 * 256;
-  PoolBuf buf;
-  buf.s = s;
-  cudaError_t e = cudaMallocFromPoolAsync(&buf.p, cnt_off + 256, static_cast<cudaMemPool_t>(ctx.pool), s);
-  if (e != cudaSuccess) { buf.p = nullptr; return static_cast<int>(e); }
-  uint8_t* base = static_cast<uint8_t*>(buf.p);
+  const QuantScratch Q = quant_scratch(P, n_rows);
+  const int64_t rows_cap = Q.rows_cap;
+  const uint32_t fix_cap = Q.fix_cap;
+  const size_t rn_off = Q.rn_off, fix_off = Q.fix_off, cnt_off = Q.cnt_off;
+  cudaError_t e = cudaSuccess;
+  uint8_t* base = static_cast<uint8_t*>(scratch);
   PrepArgs A;
   A.res = reinterpret_cast<__half*>(base);
   A.rn = reinterpret_cast<float*>(base + rn_off);
@@ -1022,24 +1043,36 @@ namespace {
 
 // estimates of every query of a set against every key of that set, per
 // 18944-key chunk: key operand, then the GEMM with the MODE epilogue
+// Estimates scratch, carved from the caller's workspace: decoded keys
+// [keys per chunk, 2d + m] binary16 | split queries [n_q, 2(d + m)] binary16 |
+// query scales [n_q, 2] f32.
+struct EstScratch {
+  int64_t keys_cap;
+  size_t b_off, qs_off, total;
+};
+EstScratch est_scratch(const KParams& P, int64_t n_q, int64_t n_keys) {
+  EstScratch q{};
+  const int64_t chunk = wide_chunk_rows();
+  q.keys_cap = n_keys < chunk ? n_keys : chunk;
+  const size_t a_bytes = static_cast<size_t>(q.keys_cap) * (2 * P.d + P.m) * 2;
+  q.b_off = (a_bytes + 255) / 256 * 256;
+  q.qs_off = q.b_off + (static_cast<size_t>(n_q) * 2 * (P.d + P.m) * 2 + 255) / 256 * 256;
+  q.total = q.qs_off + (static_cast<size_t>(n_q) * 8 + 255) / 256 * 256;
+  return q;
+}
+
 template <int MODE>
 int run_estimates(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
-                  const LogitEpi& tmpl, cudaStream_t s) {
+                  const LogitEpi& tmpl, void* scratch, cudaStream_t s) {
   const KParams& P = ctx.kp;
   const int d = P.d, m = P.m;
   const int64_t n_q = n_sets * g;
   const int64_t chunk = wide_chunk_rows();
-  const int64_t keys_cap = n_keys < chunk ? n_keys : chunk;
+  const EstScratch Q = est_scratch(P, n_q, n_keys);
+  const int64_t keys_cap = Q.keys_cap;
   const int64_t lda = 2 * d + m, ldb = 2 * (d + m);
-  const size_t a_bytes = static_cast<size_t>(keys_cap) * lda * 2;
-  const size_t b_off = (a_bytes + 255) / 256 * 256;
-  const size_t qs_off = b_off + (static_cast<size_t>(n_q) * ldb * 2 + 255) / 256 * 256;
-  const size_t total = qs_off + static_cast<size_t>(n_q) * 8;
-  PoolBuf buf;
-  buf.s = s;
-  cudaError_t e = cudaMallocFromPoolAsync(&buf.p, total, static_cast<cudaMemPool_t>(ctx.pool), s);
-  if (e != cudaSuccess) { buf.p = nullptr; return static_cast<int>(e); }
-  uint8_t* base = static_cast<uint8_t*>(buf.p);
+  const size_t b_off = Q.b_off, qs_off = Q.qs_off;
+  uint8_t* base = static_cast<uint8_t*>(scratch);
   __half* a = reinterpret_cast<__half*>(base);
   __half* b = reinterpret_cast<__half*>(base + b_off);
   float* qscale = reinterpret_cast<float*>(base + qs_off);
@@ -1089,15 +1122,18 @@ int run_estimates(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, con
   return 0;
 }
 
-size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 
 }  // namespace
 
+size_t wide_logits_scratch_bytes(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys) {
+  return est_scratch(ctx.kp, n_sets * g, n_keys).total;
+}
+
 int launch_logits_wide(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys,
-                       int64_t n_keys, float* out, void* stream) {
+                       int64_t n_keys, float* out, void* scratch, void* stream) {
   LogitEpi t{};
   t.out = out;
-  return run_estimates<kScores>(ctx, qp, n_sets, g, keys, n_keys, t, static_cast<cudaStream_t>(stream));
+  return run_estimates<kScores>(ctx, qp, n_sets, g, keys, n_keys, t, scratch, static_cast<cudaStream_t>(stream));
 }
 
 bool wide_search_applies(const tq_ctx& ctx, int64_t n_q, int64_t n_keys, int k) {
@@ -1112,9 +1148,34 @@ int search_splits(const tq_ctx& ctx, int64_t n_q) {     // CTAs per query tile
 }
 }  // namespace
 
+namespace {
+// Search scratch, carved from the caller's workspace: per-CTA candidate
+// values and rows [n_q, splits, k] | decoded keys [keys per chunk, 2d + m]
+// binary16 | split queries [n_q, 2(d + m)] binary16 | query scales [n_q, 2] f32.
+struct SearchScratch {
+  int S, tps;
+  int64_t chunk, keys_cap;
+  size_t si_off, kop_off, a_off, qs_off, total;
+};
+SearchScratch search_scratch(const tq_ctx& ctx, int64_t n_q, int64_t n_keys, int k) {
+  const KParams& P = ctx.kp;
+  SearchScratch q{};
+  q.S = search_splits(ctx, n_q);
+  q.tps = kSearchTiles / q.S > 0 ? kSearchTiles / q.S : 1;       // key tiles per CTA and chunk
+  q.chunk = static_cast<int64_t>(q.S) * q.tps * kTN;
+  q.keys_cap = n_keys < q.chunk ? n_keys : q.chunk;
+  const size_t lists = round256(static_cast<size_t>(n_q) * q.S * k * 4);
+  q.si_off = lists;
+  q.kop_off = 2 * lists;
+  q.a_off = q.kop_off + round256(static_cast<size_t>(q.keys_cap) * (2 * P.d + P.m) * 2);
+  q.qs_off = q.a_off + round256(static_cast<size_t>(n_q) * 2 * (P.d + P.m) * 2);
+  q.total = q.qs_off + round256(static_cast<size_t>(n_q) * 8);
+  return q;
+}
+}  // namespace
+
 size_t wide_search_partial_bytes(const tq_ctx& ctx, int64_t n_q, int64_t n_keys, int k) {
-  (void)n_keys;
-  return 2 * round256(static_cast<size_t>(n_q) * search_splits(ctx, n_q) * k * 4);
+  return search_scratch(ctx, n_q, n_keys, k).total;
 }
 
 int launch_search_wide(const tq_ctx& ctx, const float* qp, int64_t n_q, const Packed& keys, int64_t n_keys, int k,
@@ -1122,27 +1183,20 @@ int launch_search_wide(const tq_ctx& ctx, const float* qp, int64_t n_q, const Pa
   const KParams& P = ctx.kp;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int d = P.d, m = P.m;
-  const int S = search_splits(ctx, n_q);
+  const SearchScratch Q = search_scratch(ctx, n_q, n_keys, k);
+  const int S = Q.S;
   const int qtiles = static_cast<int>((n_q + kTM - 1) / kTM);
-  const int tps = kSearchTiles / S > 0 ? kSearchTiles / S : 1;   // key tiles per CTA and chunk
-  const int64_t chunk = static_cast<int64_t>(S) * tps * kTN;
-  const int64_t keys_cap = n_keys < chunk ? n_keys : chunk;
+  const int tps = Q.tps;
+  const int64_t chunk = Q.chunk;
+  const int64_t keys_cap = Q.keys_cap;
   const int64_t lda = 2 * (d + m), ldb = 2 * d + m;              // A: split queries, B: decoded keys
-  const size_t b_bytes = static_cast<size_t>(keys_cap) * ldb * 2;
-  const size_t a_off = round256(b_bytes);
-  const size_t qs_off = a_off + round256(static_cast<size_t>(n_q) * lda * 2);
-  PoolBuf buf;
-  buf.s = s;
-  cudaError_t e = cudaMallocFromPoolAsync(&buf.p, qs_off + static_cast<size_t>(n_q) * 8,
-                                          static_cast<cudaMemPool_t>(ctx.pool), s);
-  if (e != cudaSuccess) { buf.p = nullptr; return static_cast<int>(e); }
-  uint8_t* base = static_cast<uint8_t*>(buf.p);
-  __half* kop = reinterpret_cast<__half*>(base);
-  __half* qop = reinterpret_cast<__half*>(base + a_off);
-  float* qscale = reinterpret_cast<float*>(base + qs_off);
-  uint8_t* pb = static_cast<uint8_t*>(part);
-  float* sv = reinterpret_cast<float*>(pb);
-  int32_t* si = reinterpret_cast<int32_t*>(pb + round256(static_cast<size_t>(n_q) * S * k * 4));
+  cudaError_t e = cudaSuccess;
+  uint8_t* base = static_cast<uint8_t*>(part);
+  float* sv = reinterpret_cast<float*>(base);
+  int32_t* si = reinterpret_cast<int32_t*>(base + Q.si_off);
+  __half* kop = reinterpret_cast<__half*>(base + Q.kop_off);
+  __half* qop = reinterpret_cast<__half*>(base + Q.a_off);
+  float* qscale = reinterpret_cast<float*>(base + Q.qs_off);
 
   const int sc = pow2_at_least_sqrt(d);
   k_query_operand<<<grid_warps(n_q, ctx.num_sms), 256, 0, s>>>(P, qp, n_q, 1.0f / static_cast<float>(sc), qop,

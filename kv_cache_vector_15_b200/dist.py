@@ -3,8 +3,10 @@ of independent units.
 
 TurboQuant's write and read halves are row-local (quantize, dequant) or local
 to one (batch, kv head) set (the logits of a set read only that set's keys and
-queries), as the TurboQuant paper's quantization map and its inner-product
-estimator (Section 3) define them.  A multi-GPU job therefore splits the
+queries): each row is normalised, rotated, bucketed and projected on its own
+(0h-n0 "ICLR 2026論文解説: TurboQuant", "Step 1: PolarQuant" and "Step 2: QJL"),
+and the estimate of <q, k> reads only q and that key's packed row (Qiita
+TurboQuant explainer, "Stage 2: QJL").  A multi-GPU job therefore splits the
 global batch of sequences into contiguous shards, one per rank, and needs no
 collective on the data path: every rank quantizes, scores and dequantizes its
 own sequences.  The collectives here are only for timing (a barrier and the

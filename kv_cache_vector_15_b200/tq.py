@@ -28,8 +28,8 @@ TQ_DEQUANT_PROD, TQ_DEQUANT_MSE = 0, 1
 
 # exported symbols, in header order
 SYMBOLS = [
-    "tq_host_params", "tq_init", "tq_destroy", "tq_packed_sizes", "tq_get_params", "tq_quantize",
-    "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_dequant", "tq_topk", "tq_logits_bf16",
+    "tq_host_params", "tq_init", "tq_destroy", "tq_packed_sizes", "tq_get_params", "tq_quantize_workspace_bytes",
+    "tq_quantize", "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_dequant", "tq_topk", "tq_logits_bf16",
     "tq_status_str", "tq_sync_status", "tq_last_error", "tq_launch_count", "tq_attention_workspace_bytes",
     "tq_attention", "tq_quantize_scatter", "tq_search_workspace_bytes", "tq_search", "tq_split_init",
     "tq_split_destroy", "tq_split_part", "tq_split_quantize", "tq_split_logits_workspace_bytes", "tq_split_logits",
@@ -49,9 +49,10 @@ _sig = {
     "tq_destroy": (_i32, [_vp]),
     "tq_packed_sizes": (_i32, [_vp, _i64, ctypes.POINTER(_sz), ctypes.POINTER(_sz)]),
     "tq_get_params": (_i32, [_vp, _vp, _vp, _vp, _vp]),
-    "tq_quantize": (_i32, [_vp, _vp, _i32, _i64, _i64, _Packed, _vp]),
+    "tq_quantize_workspace_bytes": (_sz, [_vp, _i64]),
+    "tq_quantize": (_i32, [_vp, _vp, _i32, _i64, _i64, _Packed, _vp, _sz, _vp]),
     "tq_quantize_scatter": (_i32, [_vp, _vp, _i32, _i64, _i64, _vp, _i64, _Packed, _vp]),
-    "tq_logits_workspace_bytes": (_sz, [_vp, _i64, _i32]),
+    "tq_logits_workspace_bytes": (_sz, [_vp, _i64, _i32, _i64]),
     "tq_logits": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _i64, _vp, _vp, _sz, _vp]),
     "tq_logits_noalloc": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _i64, _vp, _vp]),
     "tq_dequant": (_i32, [_vp, _Packed, _i64, _vp, _i32, _i32, _vp]),
@@ -214,22 +215,30 @@ class TurboQuant:
                       torch.empty((n_rows,), dtype=torch.float32, device=device),
                       torch.empty((n_rows,), dtype=torch.float32, device=device))
 
-    def quantize(self, x, out: Packed | None = None, stream=None) -> Packed:
+    def quantize_workspace_bytes(self, n_rows: int) -> int:
+        return int(_lib.tq_quantize_workspace_bytes(self._h, n_rows))
+
+    def quantize(self, x, out: Packed | None = None, workspace=None, stream=None) -> Packed:
         """x: [N, d] (or [N, ld] with ld >= d) bf16/fp32 CUDA tensor, unit stride in the last dim."""
+        import torch
         assert x.dim() == 2 and x.stride(1) == 1
         n = x.shape[0]
         if out is None:
             out = self.empty_packed(n, x.device)
-        _check(_lib.tq_quantize(self._h, _ptr(x), _dtype_code(x), n, x.stride(0), out.c(), _stream(stream)),
-               "tq_quantize")
+        need = self.quantize_workspace_bytes(n)
+        if need and workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+        wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        _check(_lib.tq_quantize(self._h, _ptr(x), _dtype_code(x), n, x.stride(0), out.c(), _ptr(workspace), wbytes,
+                                _stream(stream)), "tq_quantize")
         return out
 
     def sync_status(self, stream=None):
         """Wait for the stream and raise if a kernel's bounded wait ran out."""
         _check(_lib.tq_sync_status(self._h, _stream(stream)), "tq_sync_status")
 
-    def workspace_bytes(self, n_sets: int, g: int) -> int:
-        return int(_lib.tq_logits_workspace_bytes(self._h, n_sets, g))
+    def workspace_bytes(self, n_sets: int, g: int, n_keys: int) -> int:
+        return int(_lib.tq_logits_workspace_bytes(self._h, n_sets, g, n_keys))
 
     def logits(self, q, keys: Packed, n_sets: int, g: int, n_keys: int, out=None, workspace=None,
                stream=None):
@@ -237,7 +246,7 @@ class TurboQuant:
         import torch
         if out is None:
             out = torch.empty((n_sets, g, n_keys), dtype=torch.float32, device=q.device)
-        need = self.workspace_bytes(n_sets, g)
+        need = self.workspace_bytes(n_sets, g, n_keys)
         if need and workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

@@ -67,7 +67,9 @@ def test_host_calls_validate_before_any_launch():
     tq = _lib()
     P = tq._Packed(0, 0, 0, 0)
     before = tq.launch_count()
-    assert tq.call_status("tq_quantize", None, None, 0, 10, 128, P, None) == tq.TQ_ERR_INVALID_ARG
+    assert tq.call_status("tq_quantize", None, None, 0, 10, 128, P, None, 0, None) == tq.TQ_ERR_INVALID_ARG
+    assert tq._lib.tq_quantize_workspace_bytes(None, 10) == 0
+    assert tq._lib.tq_logits_workspace_bytes(None, 1, 4, 10) == 0
     assert tq.call_status("tq_dequant", None, P, 10, None, 0, 0, None) == tq.TQ_ERR_INVALID_ARG
     assert tq.call_status("tq_logits", None, None, 0, 1, 4, P, 10, None, None, 0, None) == tq.TQ_ERR_INVALID_ARG
     assert tq.call_status("tq_topk", None, 4, 100, 0, None, None, None) == tq.TQ_ERR_INVALID_ARG

@@ -137,18 +137,34 @@ def test_long_context_decode_sampled(tq, b):
         assert ok.all()
 
 
-def test_prefill_write_path_sampled(tq):
-    """32 layers x 8 heads x 32768 tokens of bf16 keys with 1% of tokens x20,
-    b = 3: quantize all 8.4M rows of K, check 20000 sampled rows."""
+@pytest.fixture(scope="module")
+def prefill_keys():
+    """The prefill workload's K (32 x 8 x 32768 bf16 rows), drawn once and kept
+    on the device for the three bit widths."""
     K, _ = inputs.prefill()
-    P = op.Params(128, 3, 128, seed=0)
-    T = tq.TurboQuant(128, 3, 128, seed=0)
-    pk = T.quantize(to_dev(K))
+    dK = to_dev(K)
+    yield K, dK
+    del dK
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_prefill_write_path_sampled(tq, prefill_keys, b):
+    """32 layers x 8 heads x 32768 tokens of bf16 keys with 1% of tokens x20,
+    b in {2, 3, 4}: quantize all 8.4M rows of K, check 20000 sampled rows (a
+    thousand of them from the x20 tokens)."""
+    K, dK = prefill_keys
+    P = op.Params(128, b, 128, seed=0)
+    T = tq.TurboQuant(128, b, 128, seed=0)
+    pk = T.quantize(dK)
     T.sync_status()
-    rng = np.random.default_rng(4)
-    idx = np.sort(np.concatenate([rng.choice(K.n_rows, size=19000, replace=False),
-                                  np.nonzero(K.token_mask())[0][:1000]]))   # include scaled tokens
+    rng = np.random.default_rng(4 + b)
+    ctx = K.token_mask().size                     # the mask is per token, shared by every (layer, head)
+    scaled = rng.choice(np.nonzero(K.token_mask())[0], size=1000) + ctx * rng.integers(0, K.n_rows // ctx, 1000)
+    idx = np.sort(np.concatenate([rng.choice(K.n_rows, size=19000, replace=False), scaled]))
     sampled_quantize_check(P, K, pk, np.unique(idx))
+    del pk
+    T.close()
 
 
 def test_vector_search_sampled(tq):
