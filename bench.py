@@ -691,6 +691,7 @@ def run_aux(args, cfg, ws, rank, local):
         roof = {"bound": "tensor", "kernel": "search (estimates incl. key / query operands, fused top-10)", "achieved": ach,
                 "peak": tf, "unit": "TFLOP/s", "frac": ach / tf, "traffic": None, "algorithmic_flops": flops,
                 "executed_flops": 2.0 * nq * ndb * (3 * d + 2 * m), "peak_kind": tf_kind}
+        recall = exact_recall(torch, ddb, dq, idx, kq)
     if rank == 0:
         print(json.dumps({
             "metric": metric, "value": total / (ms * 1e-3), "unit": unit, "n_gpus": ws, "steps": args.steps,
@@ -698,10 +699,36 @@ def run_aux(args, cfg, ws, rank, local):
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": args.workload, "d": d, "b": b, "m": m, "l2": "inputs larger than L2; no flush"},
             "roofline": roof, "phases_ms": phases,
+            "recall_at_10": recall if cfg["kind"] == "vsearch" else None,
             "cuda_graph_ms_per_step": graph_ms,
             "gpu_launches": launches, "clocks": clk.summary()}), flush=True)
     T.close()
 
+
+
+def exact_recall(torch, ddb, dq, idx, k):
+    """Recall@k of the search's answers against the exact top-k by fp32 inner
+    product (the synthetic stand-in for the pages' Recall@k study; 0h-n0
+    "ICLR 2026論文解説: TurboQuant", "実験結果 — ベクトル検索（Recall評価）").
+    Reporting only, outside the timed region: a plain fp32 product (TF32
+    off) per block of database rows, and torch's top-k."""
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        best_v = torch.full((dq.shape[0], k), -float("inf"), device=dq.device)
+        best_i = torch.zeros((dq.shape[0], k), dtype=torch.int64, device=dq.device)
+        blk = 131072
+        for r0 in range(0, ddb.shape[0], blk):
+            s = dq @ ddb[r0:r0 + blk].T
+            v, i = torch.topk(s, k, dim=1)
+            cat_v, cat_i = torch.cat([best_v, v], 1), torch.cat([best_i, i + r0], 1)
+            top = torch.topk(cat_v, k, dim=1)
+            best_v, best_i = top.values, torch.gather(cat_i, 1, top.indices)
+        got = idx.to(torch.int64)
+        hits = (got[:, :, None] == best_i[:, None, :]).any(dim=2).sum().item()
+        return hits / float(got.numel())
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
 
 
 def main():

@@ -296,6 +296,30 @@ tq_status tq_split_logits(const tq_split* sp, const void* q, tq_dtype q_dtype, i
 tq_status tq_split_dequant(const tq_split* sp, tq_packed in_hi, tq_packed in_lo, int64_t n_rows, void* out,
                            tq_dtype out_dtype, tq_dequant_mode mode, void* stream);
 
+/* ------------------------------------------------------------- testing -- */
+
+/* Process-wide test settings (no counterpart on the pages; for the library's
+ * own failure tests, not for production use).  Injected failures happen on
+ * the host: no GPU fault is provoked.
+ *   TQ_TEST_WAIT_LIMIT   limit, in SM clock cycles, of the bounded mbarrier
+ *                        waits in the tile loop of the d = 128 tensor-core
+ *                        quantize kernel (0 restores the default, about one
+ *                        second).  A limit shorter than the work makes the
+ *                        kernel give up: it stops, waits (with the default
+ *                        limit) for its own MMAs and stage loads, frees its
+ *                        tensor memory, writes no results and leaves an
+ *                        error that tq_sync_status reports as TQ_ERR_CUDA.
+ *                        Applies to launches made after the call.
+ *   TQ_TEST_FAIL_ALLOC   the next `value` device allocations of tq_init fail
+ *                        as if the device were out of memory (TQ_ERR_NOMEM,
+ *                        nothing leaked).
+ *   TQ_TEST_FAIL_LAUNCH  the next `value` calls that would launch quantize,
+ *                        logit or dequant kernels fail with TQ_ERR_CUDA
+ *                        before launching anything.
+ * value >= 0, else TQ_ERR_INVALID_ARG. */
+typedef enum { TQ_TEST_WAIT_LIMIT = 0, TQ_TEST_FAIL_ALLOC = 1, TQ_TEST_FAIL_LAUNCH = 2 } tq_test_knob;
+tq_status tq_test_set(tq_test_knob knob, int64_t value);
+
 /* ----------------------------------------------------------- reporting -- */
 
 const char* tq_status_str(tq_status s);

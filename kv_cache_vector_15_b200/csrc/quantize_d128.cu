@@ -79,6 +79,7 @@ struct QuantD128Args {
   float eps_scale;                   // see header comment
   float eps_abs;                     // binary16 underflow term of the bound (normalised units)
   int* err;                          // device error word
+  long long wait_cycles;             // limit of the bounded waits in the tile loop (SM clocks)
 };
 
 // The residual enters the MMA multiplied by 64 (exact), which keeps its
@@ -492,9 +493,115 @@ k_quantize_d128_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, co
 // (the 128-byte-swizzled layout the TMA writes is the MMA's K-major operand
 // layout) and B = D H as bf16 +-1 values (exact products, fp32 accumulation),
 // so no widening, no butterflies and no cross-thread exchange run on the CUDA
-// cores.  Each thread reads its row's 128 rotated values from TMEM (the norm
-// is ||y'|| / sqrt(d)), keeps its 64, and the rest follows the fp32 kernel:
-// codes, residual hi | lo into TMEM, the projection MMA, signs, stores.
+// cores.  Each thread reads its 64 rotated values from TMEM, the two halves of
+// a row add their sums of squares through shared memory (||y'|| = sqrt(d) n),
+// and the codes, residual and projection follow.
+//
+// Codes from the symmetric codebook (c[L-1-k] = -c[k], t[L/2-1] = 0, exact
+// in fp32): with u = |y'|, the code's top bit is s = [y' > 0] and the rest is
+// the magnitude index k = #{j : T_j < u} over the positive thresholds
+// T_j = t[L/2 + j] n sqrt(d), complemented when s = 0 (code = L/2 + k or
+// L/2 - 1 - k).  Each decision is the sign of an exact difference (T - u,
+// 0 - y'), funnel-shifted into the packed words; the complement is applied
+// to whole words afterwards.  The residual is r = +-(u 64 / (n sqrt(d)) -
+// 64 c[L/2 + k]) with the centroid picked by bit masks from those signs.
+// A value exactly equal (in fp32) to a negative scaled threshold lands in
+// the upper of its two cells, every other value where the definition puts
+// it; such ties lie inside the 1e-6 band in which a code may differ from the
+// fp64 decision.
+template <int B>
+struct SymConsts {
+  static constexpr int kMag = B - 1;                       // magnitude bits
+  static constexpr int kNT = (1 << kMag) - 1;              // positive thresholds
+  static constexpr int kNC = 1 << kMag;                    // centroid magnitudes
+};
+
+// one coordinate: pushes its B code bits (top bit s, then the magnitude bits
+// from the highest, not yet complemented) into the running words and returns
+// the residual x 64.  POS = B e, the position of the code's lowest bit (a
+// constant once the caller's loops are unrolled, so cw stays in registers).
+template <int B>
+__device__ __forceinline__ float quant_coord(float y, const float* T, const uint32_t* nc, float sc,
+                                             uint32_t* cw, const int POS) {
+  const float sp = 0.f - y;                                  // negative iff y > 0 (0 - 0 = +0)
+  const float u = fabsf(y);
+  uint32_t negc;                                             // -64 c[L/2 + k] as fp32 bits
+  cw[(POS + B - 1) >> 5] = __funnelshift_l(__float_as_uint(sp), cw[(POS + B - 1) >> 5], 1);
+  if constexpr (B == 1) {
+    negc = nc[0];
+  } else if constexpr (B == 2) {
+    const float d = T[0] - u;                                // negative iff u > T
+    cw[POS >> 5] = __funnelshift_l(__float_as_uint(d), cw[POS >> 5], 1);
+    const uint32_t m = static_cast<uint32_t>(static_cast<int>(__float_as_uint(d)) >> 31);
+    negc = (m & (nc[0] ^ nc[1])) ^ nc[0];
+  } else if constexpr (B == 3) {
+    const float d2 = T[1] - u;
+    cw[(POS + 1) >> 5] = __funnelshift_l(__float_as_uint(d2), cw[(POS + 1) >> 5], 1);
+    const uint32_t m2 = static_cast<uint32_t>(static_cast<int>(__float_as_uint(d2)) >> 31);
+    const uint32_t tb = (m2 & __float_as_uint(T[2])) | (~m2 & __float_as_uint(T[0]));
+    const float d0 = __uint_as_float(tb) - u;
+    cw[POS >> 5] = __funnelshift_l(__float_as_uint(d0), cw[POS >> 5], 1);
+    const uint32_t m0 = static_cast<uint32_t>(static_cast<int>(__float_as_uint(d0)) >> 31);
+    const uint32_t ca = (m2 & nc[2]) | (~m2 & nc[0]);
+    const uint32_t cb = (m2 & nc[3]) | (~m2 & nc[1]);
+    negc = (m0 & cb) | (~m0 & ca);
+  } else {
+    // three magnitude bits: binary search T[3], then T[1] / T[5], then T[0..6 even]
+    const float d2 = T[3] - u;
+    cw[(POS + 2) >> 5] = __funnelshift_l(__float_as_uint(d2), cw[(POS + 2) >> 5], 1);
+    const uint32_t m2 = static_cast<uint32_t>(static_cast<int>(__float_as_uint(d2)) >> 31);
+    const uint32_t t1 = (m2 & __float_as_uint(T[5])) | (~m2 & __float_as_uint(T[1]));
+    const float d1 = __uint_as_float(t1) - u;
+    cw[(POS + 1) >> 5] = __funnelshift_l(__float_as_uint(d1), cw[(POS + 1) >> 5], 1);
+    const uint32_t m1 = static_cast<uint32_t>(static_cast<int>(__float_as_uint(d1)) >> 31);
+    const uint32_t lo = (m2 & __float_as_uint(T[4])) | (~m2 & __float_as_uint(T[0]));
+    const uint32_t hi = (m2 & __float_as_uint(T[6])) | (~m2 & __float_as_uint(T[2]));
+    const float d0 = __uint_as_float((m1 & hi) | (~m1 & lo)) - u;
+    cw[POS >> 5] = __funnelshift_l(__float_as_uint(d0), cw[POS >> 5], 1);
+    const uint32_t m0 = static_cast<uint32_t>(static_cast<int>(__float_as_uint(d0)) >> 31);
+    uint32_t c4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) c4[q] = (m2 & nc[4 + q]) | (~m2 & nc[q]);
+    const uint32_t c2a = (m1 & c4[2]) | (~m1 & c4[0]);
+    const uint32_t c2b = (m1 & c4[3]) | (~m1 & c4[1]);
+    negc = (m0 & c2b) | (~m0 & c2a);
+  }
+  const float rm = fmaf(u, sc, __uint_as_float(negc));
+  return __uint_as_float(__float_as_uint(rm) ^ (~__float_as_uint(sp) & 0x80000000u));
+}
+
+// Mask of the stream positions p in [32 w, 32 w + 32) with p mod B == j
+// (B in 2..4).
+__device__ __forceinline__ uint32_t residue_mask(int B, int w, int j) {
+  if (B == 3) {
+    const int r = ((j - 2 * w) % 3 + 3) % 3;                  // 32 = 2 (mod 3)
+    return r == 0 ? 0x49249249u : (r == 1 ? 0x92492492u : 0x24924924u);
+  }
+  return (B == 2 ? 0x55555555u : 0x11111111u) << j;
+}
+
+// Complement the magnitude bits of every code whose top bit (s) is 0: bit j
+// of code i (position B i + j, j < B - 1) ^= !s_i (position B i + B - 1).
+template <int B>
+__device__ __forceinline__ void complement_negative_codes(uint32_t (&cw)[2 * B]) {
+  if constexpr (B > 1) {
+    uint32_t fix[2 * B];
+#pragma unroll
+    for (int w = 0; w < 2 * B; ++w) fix[w] = 0u;
+#pragma unroll
+    for (int j = 0; j < B - 1; ++j) {
+      const int o = B - 1 - j;
+#pragma unroll
+      for (int w = 0; w < 2 * B; ++w) {
+        const uint32_t above = w + 1 < 2 * B ? ~cw[w + 1] : 0u;
+        fix[w] |= __funnelshift_r(~cw[w], above, o) & residue_mask(B, w, j);
+      }
+    }
+#pragma unroll
+    for (int w = 0; w < 2 * B; ++w) cw[w] ^= fix[w];
+  }
+}
+
 template <int B>
 __global__ void __launch_bounds__(kThreads, 1)
 k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, const QuantD128Args X,
@@ -503,29 +610,31 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
   constexpr int kStage = XStage<true>::kBytes;                  // 32 KB: two 64-column boxes
   constexpr int NS = XStage<true>::kStages;                     // two stages per pair
   constexpr int kH = kD / 2;
+  constexpr int kNT = SymConsts<B>::kNT > 0 ? SymConsts<B>::kNT : 1;
+  constexpr int kNC = SymConsts<B>::kNC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sS = smem;                                            // projection B operand
   uint8_t* sHD = smem + kSmemS;                                  // rotation B operand (D H, bf16 +-1)
   uint8_t* sX = sHD + kSmemS;                                    // [pair][NS] stages
-  float* sR2 = reinterpret_cast<float*>(sX + NS * kPairs * kStage);      // [pair][half][row] partial ||r||^2
+  float* sN2 = reinterpret_cast<float*>(sX + NS * kPairs * kStage);      // [pair][half][row] partial ||y'||^2
+  float* sR2 = sN2 + kPairs * 2 * kTile;                         // [pair][half][row] partial ||r||^2
   uint64_t* full = reinterpret_cast<uint64_t*>(sR2 + kPairs * 2 * kTile);   // [pair][2]
   uint64_t* ydone = full + 2 * kPairs;                           // [pair]
   uint64_t* mdone = ydone + kPairs;                              // [pair]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kPairs);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  float* lut = reinterpret_cast<float*>(tmem_slot + 2);          // L centroids (scaled by 64), then L zeros
-  int* loads_issued = reinterpret_cast<int*>(lut + 2 * L);       // [pair][stage]
+  int* loads_issued = abort_flag + 1;                            // [pair][stage]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
+  const long long wait_cycles = X.wait_cycles;
   if (tid == 0) {
     for (int i = 0; i < 2 * kPairs; ++i) mbar_init(&full[i], 1);
     for (int i = 0; i < kPairs; ++i) { mbar_init(&ydone[i], 1); mbar_init(&mdone[i], 1); }
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (tid < 2 * L) lut[tid] = tid < L ? P.c[tid] * kResScale : 0.f;
   for (int e = tid; e < kM * 16; e += kThreads) {
     const int j = e >> 4, c = e & 15, kb = c >> 3, cc = c & 7;
     const uint4 v = *reinterpret_cast<const uint4*>(P.S + j * kD + c * 8);
@@ -559,6 +668,8 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
   const uint32_t bar_id = 1 + pair;
   uint8_t* stages = sX + pair * NS * kStage;
   uint64_t* pfull = full + 2 * pair;
+  float* myN2 = sN2 + (pair * 2 + half) * kTile;
+  const float* otN2 = sN2 + (pair * 2 + (half ^ 1)) * kTile;
   float* myR2 = sR2 + (pair * 2 + half) * kTile;
   const float* otR2 = sR2 + (pair * 2 + (half ^ 1)) * kTile;
   const int64_t t_first = blockIdx.x + static_cast<int64_t>(pair) * gridDim.x;
@@ -570,18 +681,26 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
       tma_load_2d(stages + buf * kStage + bx * (kTile * 128), &tmap, &pfull[buf], bx * 64,
                   static_cast<int>(tile * kTile));
   };
-  int issued[2] = {0, 0}, waited[2] = {0, 0};
+  int issued[2] = {0, 0}, waited[2] = {0, 0};                    // stage loads (loader / leader)
+  int y_issued = 0, y_seen = 0, m_issued = 0, m_seen = 0;       // MMA commits (leader)
   if (loader) {
     prefetch_tmap(&tmap);
     if (t_first < n_tiles) { issue_load(t_first, 0); ++issued[0]; }
     if (t_first + t_step < n_tiles) { issue_load(t_first + t_step, 1); ++issued[1]; }
   }
 
-  // the rotation MMA of this pair's k-th tile (leader only): waits for its stage
+  // the rotation MMA of this pair's k-th tile (leader only): waits for its
+  // stage; if that wait runs out no MMA is issued and the phase is completed
+  // by hand, so the others reach the abort check
   auto issue_rotation = [&](int k) {
     const int b = k & 1;
-    if (mbar_wait(&pfull[b], (k >> 1) & 1, kWaitCycles)) ++waited[b];
-    else flag_error(X.err, abort_flag, 2);
+    ++y_issued;
+    if (!mbar_wait(&pfull[b], (k >> 1) & 1, wait_cycles)) {
+      flag_error(X.err, abort_flag, 2);
+      mbar_arrive(&ydone[pair]);
+      return;
+    }
+    ++waited[b];
     tc_fence_after();
     const uint32_t xbase = smem_u32(stages + b * kStage), hbase = smem_u32(sHD);
     const uint32_t idesc = idesc_bf16_f32(kTile, kD);
@@ -598,123 +717,102 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
   // has been read (below), so it runs under that tile's stores
   if (leader && t_first < n_tiles) issue_rotation(0);
 
+  // magnitude thresholds and centroids of the symmetric codebook (x 64 for
+  // the centroids, as negated fp32 bit patterns)
+  float tpos[kNT];
+  uint32_t ncen[kNC];
+#pragma unroll
+  for (int j = 0; j < kNT; ++j) tpos[j] = (B > 1) ? P.t[L / 2 + j] : 0.f;
+#pragma unroll
+  for (int k = 0; k < kNC; ++k) ncen[k] = __float_as_uint(-kResScale * P.c[L / 2 + k]);
+
   int mine = 0;
   for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
     const int buf = mine & 1;
-    if (!mbar_wait(&ydone[pair], mine & 1, kWaitCycles)) flag_error(X.err, abort_flag, 5);
+    if (mbar_wait(&ydone[pair], mine & 1, wait_cycles)) {
+      if (leader) ++y_seen;
+    } else {
+      flag_error(X.err, abort_flag, 5);
+    }
     tc_fence_after();
 
-    // ---- the row's rotated values: all 128 for the norm, my 64 kept ----------------
-    // (four loads in flight per wait: the other half's columns, then my own)
-    uint32_t u[kH];
-    float2 ss2 = make_float2(0.f, 0.f);
+    // ---- the row's ||y'||^2 from both halves' sums of squares -------------------
     {
-      uint32_t w[4][16];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(t_acc + (half ^ 1) * 64 + c * 16, w[c]);
+      uint32_t u[kH];
+      tmem_ld32(t_acc + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+      tmem_ld32(t_acc + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
       tmem_wait_ld();
+      float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int k = 0; k < 16; k += 2) {
-          const float2 a = make_float2(__uint_as_float(w[c][k]), __uint_as_float(w[c][k + 1]));
-          ss2 = __ffma2_rn(a, a, ss2);
-        }
+      for (int k = 0; k < kH; k += 4) {
+        const float2 a = make_float2(__uint_as_float(u[k]), __uint_as_float(u[k + 1]));
+        const float2 b2 = make_float2(__uint_as_float(u[k + 2]), __uint_as_float(u[k + 3]));
+        s0 = __ffma2_rn(a, a, s0);
+        s1 = __ffma2_rn(b2, b2, s1);
+      }
+      myN2[trow] = (s0.x + s0.y) + (s1.x + s1.y);
     }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld16(t_acc + half * 64 + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&u[c * 16]));
-    tmem_wait_ld();
-#pragma unroll
-    for (int k = 0; k < kH; k += 2) {
-      const float2 a = make_float2(__uint_as_float(u[k]), __uint_as_float(u[k + 1]));
-      ss2 = __ffma2_rn(a, a, ss2);
-    }
-    const float nsd = sqrtf(ss2.x + ss2.y);                      // ||H D x|| = sqrt(d) ||x||
+    named_bar_sync(bar_id, 256);                                 // #X: both partial sums written
+    const float ss = half == 0 ? myN2[trow] + otN2[trow] : otN2[trow] + myN2[trow];
+    const float nsd = sqrtf(ss);                                 // ||H D x|| = sqrt(d) ||x||
     const float n = nsd * 0.08838834764831845f;                  // / sqrt(128)
     const bool zero_row = !(n >= kZeroNorm);
     const float nsd_t = zero_row ? 1.f : nsd;
-    const float sc64 = zero_row ? 0.f : kResScale / nsd_t;
-    // a zero row reads an all-zero table: y = 0, scale 0, residual 0
-    const float* tab = zero_row ? lut + L : lut;
-    float tq[L - 1];
+    const float sc = zero_row ? 0.f : kResScale / nsd_t;
+    float T[kNT];
+    uint32_t nc[kNC];
 #pragma unroll
-    for (int k = 0; k < L - 1; ++k) tq[k] = P.t[k] * nsd_t;
+    for (int j = 0; j < kNT; ++j) T[j] = tpos[j] * nsd_t;
+#pragma unroll
+    for (int k = 0; k < kNC; ++k) nc[k] = zero_row ? 0u : ncen[k];   // a zero row's residual is 0
+
+    // ---- codes and the residual (x 64), hi | lo into TMEM -----------------------
+    // (the 64 values come back from TMEM 32 at a time; coordinates 63 .. 0 in
+    // order, so each packed word receives its bits from the top down)
     uint32_t cw[B * 2];
 #pragma unroll
     for (int w = 0; w < B * 2; ++w) cw[w] = 0u;
-    float2 r2 = make_float2(0.f, 0.f);
-    // 2-bit codes: bit 1 = [y > t1], bit 0 = [y > (bit 1 ? t2 : t0)], each the
-    // sign of an exact difference (t - y < 0 iff y > t; t - t = +0), funnel-
-    // shifted into the packed word from the word's last code down
-    float cc[4] = {0.f, 0.f, 0.f, 0.f};
-    if constexpr (B == 2) {
+    float2 r2a = make_float2(0.f, 0.f), r2b = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) cc[k] = tab[k];
-    }
+    for (int ch = 1; ch >= 0; --ch) {
+      uint32_t u[32];
+      tmem_ld32(t_acc + half * 64 + ch * 32, u);
+      tmem_wait_ld();
 #pragma unroll
-    for (int ch = 0; ch < 2; ++ch) {
-      uint32_t hw[16], lw[16];
-      float rb[32];
-      if constexpr (B == 2) {
+      for (int g8 = 1; g8 >= 0; --g8) {                         // 16 coordinates -> 8 hi and 8 lo columns
+        uint32_t hw[8], lw[8];
 #pragma unroll
-        for (int e = ch * 32 + 31; e >= ch * 32; --e) {
-          const float y = __uint_as_float(u[e]);
-          const float d1 = tq[1] - y;
-          const bool b1 = d1 < 0.f;
-          const float d0 = (b1 ? tq[2] : tq[0]) - y;
-          const bool b0 = d0 < 0.f;
-          cw[e >> 4] = __funnelshift_l(__float_as_uint(d1), cw[e >> 4], 1);
-          cw[e >> 4] = __funnelshift_l(__float_as_uint(d0), cw[e >> 4], 1);
-          const float c = b1 ? (b0 ? cc[3] : cc[2]) : (b0 ? cc[1] : cc[0]);
-          rb[e - ch * 32] = fmaf(y, sc64, -c);
+        for (int q = 7; q >= 0; --q) {
+          const int l1 = g8 * 16 + 2 * q + 1, l0 = l1 - 1;        // within the chunk
+          const int e1 = ch * 32 + l1, e0 = e1 - 1;               // within my 64
+          const float r1 = quant_coord<B>(__uint_as_float(u[l1]), T, nc, sc, cw, B * e1);
+          const float r0 = quant_coord<B>(__uint_as_float(u[l0]), T, nc, sc, cw, B * e0);
+          const float2 rv = make_float2(r0, r1);
+          if (q & 1) r2a = __ffma2_rn(rv, rv, r2a); else r2b = __ffma2_rn(rv, rv, r2b);
+          const __half2 h = __floats2half2_rn(r0, r1);
+          const float2 hf = __half22float2(h);
+          const float2 lf = __fadd2_rn(rv, make_float2(-hf.x, -hf.y));
+          const __half2 l = __floats2half2_rn(lf.x, lf.y);
+          hw[q] = *reinterpret_cast<const uint32_t*>(&h);
+          lw[q] = *reinterpret_cast<const uint32_t*>(&l);
         }
+        tmem_st8(t_a + half * 32 + ch * 16 + g8 * 8, hw);
+        tmem_st8(t_a + 64 + half * 32 + ch * 16 + g8 * 8, lw);
       }
-#pragma unroll
-      for (int e = ch * 32; e < ch * 32 + 32; e += 2) {
-        float rr[2];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          if constexpr (B == 2) {
-            rr[q] = rb[e + q - ch * 32];
-          } else {
-            const float y = __uint_as_float(u[e + q]);
-            uint32_t code = 0u;
-#pragma unroll
-            for (int lev = B - 1; lev >= 0; --lev) {
-              const int base = (1 << lev) - 1;
-              float thr = tq[base];
-#pragma unroll
-              for (int k = 1; k < (1 << (B - 1 - lev)); ++k)
-                if (code == static_cast<uint32_t>(k << (lev + 1))) thr = tq[base + (k << (lev + 1))];
-              if (y > thr) code |= (1u << lev);
-            }
-            rr[q] = fmaf(y, sc64, -tab[code]);
-            const int bit = B * (e + q), wi = bit >> 5, sh = bit & 31;
-            cw[wi] |= code << sh;
-            if (sh + B > 32) cw[wi + 1] |= code >> (32 - sh);
-          }
-        }
-        const float2 rv = make_float2(rr[0], rr[1]);
-        r2 = __ffma2_rn(rv, rv, r2);
-        const __half2 h = __floats2half2_rn(rr[0], rr[1]);
-        const float2 hf = __half22float2(h);
-        const __half2 l = __floats2half2_rn(rr[0] - hf.x, rr[1] - hf.y);
-        hw[(e - ch * 32) >> 1] = *reinterpret_cast<const uint32_t*>(&h);
-        lw[(e - ch * 32) >> 1] = *reinterpret_cast<const uint32_t*>(&l);
-      }
-      tmem_st16(t_a + half * 32 + ch * 16, hw);
-      tmem_st16(t_a + 64 + half * 32 + ch * 16, lw);
     }
+    complement_negative_codes<B>(cw);
     if (zero_row) {
 #pragma unroll
       for (int w = 0; w < B * 2; ++w) cw[w] = 0u;
     }
-    myR2[trow] = r2.x + r2.y;
+    myR2[trow] = (r2a.x + r2a.y) + (r2b.x + r2b.y);
     tmem_wait_st();
     tc_fence_before();
-    // #B: A complete and every y' read done (the projection overwrites them)
+    // #B: A complete and every y' read done (the projection overwrites them);
+    // the abort flag ORed over the pair so that all take the same decision
     if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
-    const float rho = zero_row ? 0.f : sqrtf(myR2[trow] + otR2[trow]) * (1.0f / kResScale);
+    const float rho = zero_row ? 0.f : sqrtf(half == 0 ? myR2[trow] + otR2[trow] : otR2[trow] + myR2[trow]) *
+                                           (1.0f / kResScale);
     if (leader) {
       tc_fence_after();
       const uint32_t sbase = smem_u32(sS);
@@ -727,8 +825,13 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
         mma_f16_ts(d_tmem, d_tmem + 128 + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
       }
       mma_commit(&mdone[pair]);
+      ++m_issued;
     }
-    if (!mbar_wait(&mdone[pair], mine & 1, kWaitCycles)) flag_error(X.err, abort_flag, 3);
+    if (mbar_wait(&mdone[pair], mine & 1, wait_cycles)) {
+      if (leader) ++m_seen;
+    } else {
+      flag_error(X.err, abort_flag, 3);
+    }
     tc_fence_after();
 
     // ---- my 64 signs, exact recomputation within the error bound of zero ------------
@@ -736,37 +839,31 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
     uint32_t s0 = 0, s1 = 0, f0 = 0, f1 = 0;
     float pmin = INFINITY;
     {
-      uint32_t p[4][16];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(t_acc + half * 64 + c * 16, p[c]);
+      uint32_t p[kH];
+      tmem_ld32(t_acc + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
+      tmem_ld32(t_acc + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t bits = 0u;
-#pragma unroll
-        for (int j = 15; j >= 0; --j) {
-          bits = (bits << 1) | (p[c][j] >> 31);
-          pmin = fminf(pmin, fabsf(__uint_as_float(p[c][j])));
-        }
-        if (c == 0) s0 = bits;
-        if (c == 1) s0 |= bits << 16;
-        if (c == 2) s1 = bits;
-        if (c == 3) s1 |= bits << 16;
+      for (int j = 31; j >= 0; --j) {
+        s0 = __funnelshift_l(p[j], s0, 1);
+        s1 = __funnelshift_l(p[32 + j], s1, 1);
       }
+#pragma unroll
+      for (int j = 0; j < kH; j += 2)
+        pmin = fminf(pmin, fminf(fabsf(__uint_as_float(p[j])), fabsf(__uint_as_float(p[j + 1]))));
     }
+    // rare: find which projections are within the bound.  The TMEM loads are
+    // warp-collective, so the whole warp takes this branch when any lane needs it.
     if (__any_sync(0xffffffffu, pmin < eps)) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t p[16];
-        tmem_ld16(t_acc + half * 64 + c * 16, p);
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t p[32];
+        tmem_ld32(t_acc + half * 64 + hh * 32, p);
         tmem_wait_ld();
-        uint32_t flags = 0u;
+        uint32_t f = 0u;
 #pragma unroll
-        for (int j = 15; j >= 0; --j) flags = (flags << 1) | (fabsf(__uint_as_float(p[j])) < eps ? 1u : 0u);
-        if (c == 0) f0 = flags;
-        if (c == 1) f0 |= flags << 16;
-        if (c == 2) f1 = flags;
-        if (c == 3) f1 |= flags << 16;
+        for (int j = 31; j >= 0; --j) f = (f << 1) | (fabsf(__uint_as_float(p[j])) < eps ? 1u : 0u);
+        if (hh == 0) f0 = f; else f1 = f;
       }
     }
     const int nflag = __popc(f0) + __popc(f1);
@@ -779,24 +876,22 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
       }
       const int jg = half * 64 + (j < 0 ? 0 : j);
       float acc = 0.f;
-      // S_j . hi, then S_j . lo: 32 columns per load batch, one wait each
+      // S_j . hi, then S_j . lo: 16 columns (32 coordinates) per load
 #pragma unroll 1
-      for (int part = 0; part < 4; ++part) {
-        uint32_t a[2][16];
-        tmem_ld16(t_a + part * 32, a[0]);
-        tmem_ld16(t_a + part * 32 + 16, a[1]);
+      for (int part = 0; part < 8; ++part) {
+        uint32_t a[16];
+        tmem_ld16(t_a + part * 16, a);
         tmem_wait_ld();
         if (j >= 0) {
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const int chunk = (part & 1) * 8 + ch, kb = chunk >> 3, cc = chunk & 7;
+          for (int ch = 0; ch < 4; ++ch) {
+            const int chunk = (part & 3) * 4 + ch, kb = chunk >> 3, cc = chunk & 7;
             const uint4 sv = *reinterpret_cast<const uint4*>(sS + kb * 16384 + jg * 128 + ((cc ^ (jg & 7)) << 4));
             const uint32_t sws[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int w = ch * 4 + u;                              // column part * 32 + w
-              const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sws[u]));
-              const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&a[w >> 4][w & 15]));
+            for (int uu = 0; uu < 4; ++uu) {
+              const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sws[uu]));
+              const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&a[ch * 4 + uu]));
               acc = fmaf(sf.x, hf.x, acc);
               acc = fmaf(sf.y, hf.y, acc);
             }
@@ -845,7 +940,15 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
     // the other half than the one that issues the MMAs)
     if (loader && t + NS * t_step < n_tiles) { issue_load(t + NS * t_step, buf); ++issued[buf]; }
   }
-  // let every issued stage load land before the shared memory is released
+  // Wind-down, with the full wait limit whatever limit the loop ran with: no
+  // MMA of ours may still be running and no stage load still landing when the
+  // TMEM and the shared memory are released.
+  if (leader) {
+    for (; y_seen < y_issued; ++y_seen)
+      if (!mbar_wait(&ydone[pair], y_seen & 1, kWaitCycles)) { flag_error(X.err, abort_flag, 4); break; }
+    for (; m_seen < m_issued; ++m_seen)
+      if (!mbar_wait(&mdone[pair], m_seen & 1, kWaitCycles)) { flag_error(X.err, abort_flag, 4); break; }
+  }
   if (loader) { loads_issued[2 * pair] = issued[0]; loads_issued[2 * pair + 1] = issued[1]; }
   __syncthreads();
   if (leader) {
@@ -868,7 +971,7 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() { return tensor_map_encoder(); }
 
 constexpr size_t quant_rot_smem_bytes() {
-  return 1024 + 2 * kSmemS + 2 * kPairs * XStage<true>::kBytes + kPairs * 2 * kTile * 4 + 256;
+  return 1024 + 2 * kSmemS + 2 * kPairs * XStage<true>::kBytes + 2 * kPairs * 2 * kTile * 4 + 256;
 }
 
 template <int B, bool BF16IN>
@@ -891,6 +994,7 @@ int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, cons
   X.eps_scale = ctx.qjl_eps_scale;
   X.eps_abs = ctx.qjl_eps_abs;
   X.err = P.err;
+  X.wait_cycles = wait_limit_cycles();
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
   const int grid = static_cast<int>(n_tiles < ctx.num_sms ? n_tiles : ctx.num_sms);
   if constexpr (BF16IN) {                // bf16 rows: the rotation on the tensor cores

@@ -26,6 +26,21 @@ tq_status fail(tq_status s, const std::string& why) {
 
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
+constexpr long long kDefaultWaitCycles = 2000000000ll;         // about one second at 2 GHz
+static std::atomic<long long> g_wait_limit{kDefaultWaitCycles};
+static std::atomic<int64_t> g_fail_alloc{0}, g_fail_launch{0};
+
+long long wait_limit_cycles() { return g_wait_limit.load(std::memory_order_relaxed); }
+
+static bool take_one(std::atomic<int64_t>& n) {
+  int64_t v = n.load(std::memory_order_relaxed);
+  while (v > 0)
+    if (n.compare_exchange_weak(v, v - 1, std::memory_order_relaxed)) return true;
+  return false;
+}
+bool take_injected_alloc_failure() { return take_one(g_fail_alloc); }
+bool take_injected_launch_failure() { return take_one(g_fail_launch); }
+
 int padded_dim(int d) {
   int p = 1;
   while (p < d) p <<= 1;
@@ -208,7 +223,7 @@ tq_status tq_init(int d, int b, int m, uint64_t seed, tq_ctx** out) {
   const size_t off_sn = off_St + round256(sz_S);
   const size_t total = off_sn + round256(static_cast<size_t>(m) * 4);
   void* blk = nullptr;
-  e = cudaMalloc(&blk, total);
+  e = take_injected_alloc_failure() ? cudaErrorMemoryAllocation : cudaMalloc(&blk, total);
   if (e != cudaSuccess) { delete ctx; return fail(TQ_ERR_NOMEM, std::string("cudaMalloc: ") + cudaGetErrorString(e)); }
   ctx->dev_block = blk;
 
@@ -479,6 +494,18 @@ tq_status tq_topk(const float* scores, int64_t rows, int64_t cols, int k, int32_
   int err = launch_topk(scores, rows, cols, k, idx, val, stream);
   if (err) return cuda_fail(err, "tq_topk launch");
   return TQ_OK;
+}
+
+tq_status tq_test_set(tq_test_knob knob, int64_t value) {
+  if (value < 0) return fail(TQ_ERR_INVALID_ARG, "value must be >= 0");
+  switch (knob) {
+    case TQ_TEST_WAIT_LIMIT:
+      g_wait_limit.store(value == 0 ? kDefaultWaitCycles : value, std::memory_order_relaxed);
+      return TQ_OK;
+    case TQ_TEST_FAIL_ALLOC: g_fail_alloc.store(value, std::memory_order_relaxed); return TQ_OK;
+    case TQ_TEST_FAIL_LAUNCH: g_fail_launch.store(value, std::memory_order_relaxed); return TQ_OK;
+  }
+  return fail(TQ_ERR_INVALID_ARG, "unknown test setting");
 }
 
 tq_status tq_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, int d, float* out,

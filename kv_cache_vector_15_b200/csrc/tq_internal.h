@@ -44,6 +44,11 @@ size_t round256(size_t v);
 int padded_dim(int d);                // the next power of two >= d
 tq_status fail(tq_status s, const std::string& why);   // records tq_last_error()
 void count_launch(int n = 1);
+// test settings (tq_test_set): the bounded-wait limit the tensor-core
+// quantize kernel's tile loop runs with, and injected host-side failures
+long long wait_limit_cycles();
+bool take_injected_alloc_failure();
+bool take_injected_launch_failure();
 
 // host_params.cpp
 uint16_t double_to_half_bits(double v);

@@ -25,6 +25,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_NOMEM, TQ_ERR_CUDA = range(5)
 TQ_BF16, TQ_F32 = 0, 1
 TQ_DEQUANT_PROD, TQ_DEQUANT_MSE = 0, 1
+TQ_TEST_WAIT_LIMIT, TQ_TEST_FAIL_ALLOC, TQ_TEST_FAIL_LAUNCH = 0, 1, 2
 
 # exported symbols, in header order
 SYMBOLS = [
@@ -33,7 +34,7 @@ SYMBOLS = [
     "tq_status_str", "tq_sync_status", "tq_last_error", "tq_launch_count", "tq_attention_workspace_bytes",
     "tq_attention", "tq_quantize_scatter", "tq_search_workspace_bytes", "tq_search", "tq_split_init",
     "tq_split_destroy", "tq_split_part", "tq_split_quantize", "tq_split_logits_workspace_bytes", "tq_split_logits",
-    "tq_split_dequant",
+    "tq_split_dequant", "tq_test_set",
 ]
 
 
@@ -74,6 +75,7 @@ _sig = {
     "tq_sync_status": (_i32, [_vp, _vp]),
     "tq_last_error": (ctypes.c_char_p, []),
     "tq_launch_count": (_u64, []),
+    "tq_test_set": (_i32, [_i32, _i64]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -91,6 +93,12 @@ class TQError(RuntimeError):
 def _check(status: int, where: str):
     if status != TQ_OK:
         raise TQError(status, where)
+
+
+def test_set(knob: int, value: int):
+    """Process-wide test setting (tq_test_set): wait limit of the d = 128
+    quantize kernel, or injected host-side allocation / launch failures."""
+    _check(_lib.tq_test_set(knob, value), "tq_test_set")
 
 
 def launch_count() -> int:

@@ -92,6 +92,9 @@ def test_host_calls_validate_before_any_launch():
     assert tq.call_status("tq_split_dequant", None, P, P, 10, None, 0, 0, None) == tq.TQ_ERR_INVALID_ARG
     assert tq._lib.tq_split_logits_workspace_bytes(None, 1, 4, 10) == 0
     assert tq.call_status("tq_split_destroy", None) == tq.TQ_OK
+    assert tq.call_status("tq_test_set", 0, -1) == tq.TQ_ERR_INVALID_ARG
+    assert tq.call_status("tq_test_set", 7, 0) == tq.TQ_ERR_INVALID_ARG
+    assert tq.call_status("tq_test_set", tq.TQ_TEST_FAIL_LAUNCH, 0) == tq.TQ_OK
     assert tq.launch_count() == before
 
 

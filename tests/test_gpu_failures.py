@@ -1,0 +1,86 @@
+"""Failure paths, provoked on the host (no GPU fault, no hang):
+
+* a bounded device-side wait that runs out: a test setting shortens the wait
+  limit of the d = 128 quantize kernel's tile loop to 100 SM clocks, so its
+  first wait gives up; the kernel must wind down (drain its own MMAs and stage
+  loads, free its tensor memory), write no results and leave an error that
+  tq_sync_status reports; the next launch with the normal limit must run (it
+  allocates all of the SM's tensor memory, so a leak would show) and match
+  the oracle;
+* an injected device-allocation failure in tq_init (TQ_ERR_NOMEM, then a
+  normal tq_init works);
+* an injected launch failure (TQ_ERR_CUDA before anything is launched).
+"""
+
+import numpy as np
+import pytest
+
+from oracle import params as op
+from oracle import turboquant as ot
+from tests import parity
+from tests.test_gpu_parity import make_rows
+
+torch = pytest.importorskip("torch")
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+
+@pytest.fixture(scope="module")
+def tq():
+    from kv_cache_vector_15_b200 import tq as _tq
+    yield _tq
+    _tq.test_set(_tq.TQ_TEST_WAIT_LIMIT, 0)
+    _tq.test_set(_tq.TQ_TEST_FAIL_ALLOC, 0)
+    _tq.test_set(_tq.TQ_TEST_FAIL_LAUNCH, 0)
+
+
+@pytest.mark.parametrize("b", [3, 4])
+def test_quantize_wait_runs_out_then_recovers(tq, b):
+    d, m, n = 128, 128, 40000                       # 313 tiles: every CTA has several
+    P = op.Params(d, b, m, seed=0)
+    xt, x = make_rows(d, n, "bf16", seed=31)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    xd = xt.cuda()
+    out = T.empty_packed(n, "cuda")
+    out.norm.fill_(-1.0)
+    tq.test_set(tq.TQ_TEST_WAIT_LIMIT, 100)
+    try:
+        T.quantize(xd, out)
+        with pytest.raises(tq.TQError) as e:
+            T.sync_status()
+        assert e.value.status == tq.TQ_ERR_CUDA
+    finally:
+        tq.test_set(tq.TQ_TEST_WAIT_LIMIT, 0)
+    assert bool(torch.all(out.norm == -1.0)), "a CTA that gave up wrote results"
+    T.sync_status()                                  # the error was reported once and cleared
+    for _ in range(2):                               # normal limit: runs, frees and allocates TMEM again
+        got = T.quantize(xd).to_numpy()
+        T.sync_status()
+    parity.assert_quantize_ok(parity.compare_quantize(P, got, ot.quantize(x, P, keep_intermediates=True)))
+    T.close()
+
+
+def test_injected_allocation_failure(tq):
+    tq.test_set(tq.TQ_TEST_FAIL_ALLOC, 1)
+    with pytest.raises(tq.TQError) as e:
+        tq.TurboQuant(128, 3, 128, seed=0)
+    assert e.value.status == tq.TQ_ERR_NOMEM
+    T = tq.TurboQuant(128, 3, 128, seed=0)           # the injection was used up
+    T.close()
+
+
+def test_injected_launch_failure(tq):
+    T = tq.TurboQuant(128, 3, 128, seed=0)
+    xt, x = make_rows(128, 300, "bf16", seed=3)
+    xd = xt.cuda()
+    tq.test_set(tq.TQ_TEST_FAIL_LAUNCH, 1)
+    before = tq.launch_count()
+    with pytest.raises(tq.TQError) as e:
+        T.quantize(xd)
+    assert e.value.status == tq.TQ_ERR_CUDA
+    assert tq.launch_count() == before
+    P = op.Params(128, 3, 128, seed=0)
+    got = T.quantize(xd).to_numpy()
+    T.sync_status()
+    parity.assert_quantize_ok(parity.compare_quantize(P, got, ot.quantize(x, P, keep_intermediates=True)))
+    T.close()
