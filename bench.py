@@ -296,15 +296,16 @@ def run_ours(args, cfg, ws, rank, local):
     vhat = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
     wbytes = T.workspace_bytes(n_sets, g, n_keys)
     work = torch.empty(max(wbytes, 16), dtype=torch.uint8, device=dev)
+    qwork = torch.empty(max(T.quantize_workspace_bytes(N), 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        T.quantize(dK, pK, stream=stream)
+        T.quantize(dK, pK, workspace=qwork, stream=stream)
         if ev:
             ev[1].record(stream)
-        T.quantize(dV, pV, stream=stream)
+        T.quantize(dV, pV, workspace=qwork, stream=stream)
         if ev:
             ev[2].record(stream)
         T.logits(dQ, pK, n_sets, g, n_keys, out=logits, workspace=work, stream=stream)
@@ -439,8 +440,8 @@ def run_ours(args, cfg, ws, rank, local):
             if downloaded[i] is not None:
                 stream.wait_event(downloaded[i])
             pk, pv = pK.rows(r0, r1), pV.rows(r0, r1)
-            T.quantize(dK[r0:r1], pk, stream=stream)
-            T.quantize(dV[r0:r1], pv, stream=stream)
+            T.quantize(dK[r0:r1], pk, workspace=qwork, stream=stream)
+            T.quantize(dV[r0:r1], pv, workspace=qwork, stream=stream)
             T.logits(dQ[q0:q1], pk, sets_per, g, n_keys, out=logits[s0:s1], workspace=work, stream=stream)
             T.dequant(pv, kv_per, out=vhat[r0:r1], stream=stream)
             done = torch.cuda.Event()
@@ -596,10 +597,11 @@ def run_aux(args, cfg, ws, rank, local):
         dK, dV = hK.to(dev), hV.to(dev)
         del hK, hV
         pK, pV = T.empty_packed(n, dev), T.empty_packed(n, dev)
+        qwork = torch.empty(max(T.quantize_workspace_bytes(n), 16), dtype=torch.uint8, device=dev)
 
         def step():
-            T.quantize(dK, pK, stream=stream)
-            T.quantize(dV, pV, stream=stream)
+            T.quantize(dK, pK, workspace=qwork, stream=stream)
+            T.quantize(dV, pV, workspace=qwork, stream=stream)
         units, unit, metric = 2 * n, "rows/s", f"tq_quantize rows/s, prefill write path (b={b})"
         alg = 2 * n * (2 * d + P)
         kern = "quantize"

@@ -125,15 +125,18 @@ tq_status tq_get_params(const tq_ctx* ctx, float* centroids, float* thresholds, 
  * fp32, ld_x >= d; x and ld_x * element size 16-byte aligned when d is a
  * power of two, x aligned to its element size otherwise) into `out`.
  * Per row: norm, rotation, Lloyd-Max codes, QJL signs of the residual,
- * residual norm (write half above).  One launch at d = 128 and for small
- * batches.  Wide rows (d >= 256, n_rows >= 4096) run per 37888-row chunk: a
- * CUDA-core kernel (norm, rotation, codes, residual halves), a tensor-core
- * GEMM for the projections and their signs, and a fix-up of the rare
- * projections inside the GEMM's error bound (recomputed in fp64); their
- * scratch (residual halves, fix-up list) is the workspace.
+ * residual norm (write half above).  At d = m = 128 a tensor-core kernel
+ * does it all and marks the rows in which a projection fell inside the
+ * tensor cores' error bound (one bit per row in the workspace); a second
+ * kernel recomputes those rows' signs exactly (fp64).  Wide rows (d >= 256,
+ * n_rows >= 4096) run per 37888-row chunk: a CUDA-core kernel (norm,
+ * rotation, codes, residual halves), a tensor-core GEMM for the projections
+ * and their signs, and a fix-up of the rare projections inside the GEMM's
+ * error bound (recomputed in fp64); their scratch (residual halves, fix-up
+ * list) is the workspace.  Other shapes run on general CUDA-core kernels.
  *   workspace: device memory of at least tq_quantize_workspace_bytes(ctx,
- *   n_rows) bytes, 16-byte aligned (may be NULL when that is 0, which it is
- *   at d = 128 and for the general kernels). */
+ *   n_rows) bytes, 16-byte aligned (may be NULL when that is 0, as it is for
+ *   the general kernels). */
 size_t tq_quantize_workspace_bytes(const tq_ctx* ctx, int64_t n_rows);
 tq_status tq_quantize(const tq_ctx* ctx, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
                       tq_packed out, void* workspace, size_t workspace_bytes, void* stream);
@@ -316,8 +319,18 @@ tq_status tq_split_dequant(const tq_split* sp, tq_packed in_hi, tq_packed in_lo,
  *   TQ_TEST_FAIL_LAUNCH  the next `value` calls that would launch quantize,
  *                        logit or dequant kernels fail with TQ_ERR_CUDA
  *                        before launching anything.
+ *   TQ_TEST_FIXUP_CAP    caps the list of projections that the d = 128
+ *                        quantize kernel hands to its exact fix-up at `value`
+ *                        entries (0 restores the default, two per 128-row
+ *                        tile): rows beyond the list take the overflow path,
+ *                        which recomputes all their signs.
  * value >= 0, else TQ_ERR_INVALID_ARG. */
-typedef enum { TQ_TEST_WAIT_LIMIT = 0, TQ_TEST_FAIL_ALLOC = 1, TQ_TEST_FAIL_LAUNCH = 2 } tq_test_knob;
+typedef enum {
+  TQ_TEST_WAIT_LIMIT = 0,
+  TQ_TEST_FAIL_ALLOC = 1,
+  TQ_TEST_FAIL_LAUNCH = 2,
+  TQ_TEST_FIXUP_CAP = 3
+} tq_test_knob;
 tq_status tq_test_set(tq_test_knob knob, int64_t value);
 
 /* ----------------------------------------------------------- reporting -- */

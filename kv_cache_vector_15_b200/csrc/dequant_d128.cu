@@ -48,6 +48,7 @@ constexpr float kUnit = 64.0f;          // scale of the unit-norm domain the rot
 struct DequantD128Args {
   uint32_t Dneg[kD / 32];               // bit i of word i / 32: D_i = -1
   int* err;
+  long long wait_cycles;                // limit of the bounded waits in the tile loop (SM clocks)
 };
 
 template <bool BF16OUT>
@@ -60,6 +61,10 @@ struct OutStage {
 template <bool BF16OUT>
 constexpr size_t dequant_smem_bytes() {
   return 1024 + 32768 /*St*/ + 32768 /*D H*/ + kPairs * OutStage<BF16OUT>::kBytes + 512;
+}
+constexpr size_t dequant_ovl_smem_bytes() {
+  return 1024 + 32768 /*St*/ + 32768 /*D H*/ + kPairs * 32768 /*sign operands*/ + kPairs * OutStage<true>::kBytes +
+         512;
 }
 
 __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* smem_src, int x, int y) {
@@ -361,6 +366,334 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
   }
 }
 
+// bf16 output, overlapped: the same two products per tile, arranged so that
+// the tensor cores never wait for the CUDA cores of the same pair.
+//   * The sign operand of S^T z lives in shared memory (A of an ss MMA, z_j
+//     as binary16 +-1 in the K-major 128-byte-swizzled layout), written for
+//     the NEXT tile while the current tile's rotation runs.
+//   * Each pair has two 128-column TMEM regions with alternating roles: tile
+//     k's S^T z and then its rotated output in region k mod 2, its v hi | lo
+//     in the other; so the next tile's S^T z product can run into the region
+//     of this tile's v as soon as the rotation has read it, under this tile's
+//     output stores.
+// Per tile (pair): wait S^T z -> v = yhat + w S^T z -> v hi | lo into TMEM,
+// the next tile's signs into shared memory -> barrier -> rotation MMA; while
+// it runs, decode the next tile's yhat -> wait -> the next tile's S^T z MMA
+// -> read, scale, round and stage the output -> barrier -> TMA store.
+template <int B, bool PROD>
+__global__ void __launch_bounds__(kThreads, 1)
+k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P, const DequantD128Args X,
+                   const Packed in, int64_t n_rows) {
+  constexpr int L = 1 << B;
+  constexpr int kStage = OutStage<true>::kBytes;          // 32 KB
+  constexpr int kH = kD / 2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sSt = smem;                                   // B of S^T z: row i, K position j holds S[j][i]
+  uint8_t* sDH = smem + 32768;                           // B of the rotation (N = n, K = k)
+  uint8_t* sZ = smem + 65536;                            // [pair] A of S^T z: row r, K position j holds z_j
+  uint8_t* sOut = sZ + kPairs * 32768;                   // [pair] output stages
+  uint64_t* m1 = reinterpret_cast<uint64_t*>(sOut + kPairs * kStage);   // [pair] S^T z done
+  uint64_t* m2 = m1 + kPairs;                                            // [pair] rotation done
+  uint64_t* fdone = m2 + kPairs;                                         // [pair] wind-down commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fdone + kPairs);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* lut = reinterpret_cast<float*>(tmem_slot + 2);                 // L centroids x kUnit
+  float2* lut2 = reinterpret_cast<float2*>(lut + 16);                   // 2-bit codes: pairs (4 bits)
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
+  const long long wait_cycles = X.wait_cycles;
+  if (tid == 0) {
+    for (int i = 0; i < kPairs; ++i) { mbar_init(&m1[i], 1); mbar_init(&m2[i], 1); mbar_init(&fdone[i], 1); }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (tid < L) lut[tid] = P.c[tid] * kUnit;
+  if (B == 2 && tid < 16) lut2[tid] = make_float2(P.c[tid & 3] * kUnit, P.c[tid >> 2] * kUnit);
+  if (PROD) {
+    uint16_t* st16 = reinterpret_cast<uint16_t*>(sSt);
+    for (int e = tid; e < kD * kM; e += kThreads) {
+      const int i = e >> 7, j = e & 127;
+      const int kb = j >> 6, chunk = (j & 63) >> 3, within = j & 7;
+      st16[(kb * 16384 + i * 128 + ((chunk ^ (i & 7)) << 4)) / 2 + within] = P.St[i * kM + j];
+    }
+  }
+  {
+    // (D H)[n][k] = D_n (-1)^popcount(n & k), binary16 +-1, same swizzled layout
+    uint16_t* h16 = reinterpret_cast<uint16_t*>(sDH);
+    for (int e = tid; e < kD * kD; e += kThreads) {
+      const int n = e >> 7, k = e & 127;
+      const bool neg = ((__popc(n & k) & 1) != 0) != (((X.Dneg[n >> 5] >> (n & 31)) & 1u) != 0);
+      const int kb = k >> 6, chunk = (k & 63) >> 3, within = k & 7;
+      h16[(kb * 16384 + n * 128 + ((chunk ^ (n & 7)) << 4)) / 2 + within] = neg ? 0xBC00u : 0x3C00u;
+    }
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int wgi = warp >> 2, pair = wgi >> 1, half = wgi & 1, lb = warp & 3;
+  const bool leader = (half == 0 && lb == 0 && lane == 0);        // issues the pair's MMAs
+  const bool storer = (half == 1 && lb == 0 && lane == 0);        // issues the pair's TMA stores
+  const int trow = lb * 32 + lane;
+  const uint32_t lane_base = static_cast<uint32_t>(lb * 32) << 16;
+  const uint32_t t_reg0 = tmem + lane_base + pair * 256;  // region k mod 2: S^T z, then the output of tile k
+  const uint32_t bar_id = 1 + pair;
+  uint8_t* stage = sOut + pair * kStage;
+  uint8_t* zbuf = sZ + pair * 32768;
+  const float inv_sqrt_d = 0.08838834764831845f;
+  const float qjl = P.qjl_scale * kUnit;                  // S^T z in unit-norm x kUnit
+  const int64_t t_first = blockIdx.x + static_cast<int64_t>(pair) * gridDim.x;
+  const int64_t t_step = static_cast<int64_t>(kPairs) * gridDim.x;
+  bool store_pending = false, mma_issued = false;
+
+  // my part of a packed row: codes of my 64 coordinates, my two sign words, norms
+  struct Part {
+    uint32_t cw[B * 2];
+    uint32_t sg0, sg1;
+    float nrm, rn;
+  };
+  auto load_packed = [&](int64_t tile, Part& pt) {
+    const int64_t row = tile * kTile + trow;
+    if (tile < n_tiles && row < n_rows) {
+      const uint8_t* cp = in.codes + row * (B * 16) + half * (B * 8);
+      if constexpr (B == 1) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(cp));
+        pt.cw[0] = u.x; pt.cw[1] = u.y;
+      } else if constexpr (B == 2) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(cp));
+        pt.cw[0] = u.x; pt.cw[1] = u.y; pt.cw[2] = u.z; pt.cw[3] = u.w;
+      } else if constexpr (B == 3) {
+        if (half == 0) {
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(cp));
+          const uint2 w = __ldg(reinterpret_cast<const uint2*>(cp + 16));
+          pt.cw[0] = u.x; pt.cw[1] = u.y; pt.cw[2] = u.z; pt.cw[3] = u.w; pt.cw[4] = w.x; pt.cw[5] = w.y;
+        } else {
+          const uint2 w = __ldg(reinterpret_cast<const uint2*>(cp));
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(cp + 8));
+          pt.cw[0] = w.x; pt.cw[1] = w.y; pt.cw[2] = u.x; pt.cw[3] = u.y; pt.cw[4] = u.z; pt.cw[5] = u.w;
+        }
+      } else {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(cp));
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(cp + 16));
+        pt.cw[0] = u.x; pt.cw[1] = u.y; pt.cw[2] = u.z; pt.cw[3] = u.w;
+        pt.cw[4] = w.x; pt.cw[5] = w.y; pt.cw[6] = w.z; pt.cw[7] = w.w;
+      }
+      if (PROD) {
+        const uint2 sg = __ldg(reinterpret_cast<const uint2*>(in.signs + row * 16 + half * 8));
+        pt.sg0 = sg.x; pt.sg1 = sg.y;
+      } else {
+        pt.sg0 = pt.sg1 = 0u;
+      }
+      pt.nrm = __ldg(in.norm + row);
+      pt.rn = __ldg(in.rnorm + row);
+    } else {
+#pragma unroll
+      for (int w = 0; w < B * 2; ++w) pt.cw[w] = 0u;
+      pt.sg0 = pt.sg1 = 0u;
+      pt.nrm = 0.f;
+      pt.rn = 0.f;
+    }
+  };
+  // yhat x kUnit of my 64 coordinates
+  auto decode = [&](const Part& pt, float (&v)[kH]) {
+    if constexpr (B == 2) {
+#pragma unroll
+      for (int e = 0; e < kH; e += 2) {                    // two codes per lookup
+        const float2 c2 = lut2[(pt.cw[e >> 4] >> ((2 * e) & 31)) & 15u];
+        v[e] = c2.x;
+        v[e + 1] = c2.y;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < kH; ++e) {
+        const int bit = B * e, wi = bit >> 5, sh = bit & 31;
+        uint32_t code = pt.cw[wi] >> sh;
+        if (sh + B > 32) code |= pt.cw[wi + 1] << (32 - sh);
+        code &= (1u << B) - 1u;
+        v[e] = lut[code];
+      }
+    }
+  };
+  // my 64 sign bits as binary16 z_j = +-1 into row trow of the sign operand:
+  // K block `half`, 16-byte chunk c (projections 64 half + 8 c ..) at chunk c ^ (trow & 7)
+  auto write_signs = [&](const Part& pt) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t sgw = (c < 4 ? pt.sg0 : pt.sg1) >> ((c & 3) * 8);   // projections 8 c .. 8 c + 7 (of mine)
+      uint32_t w4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t b2 = sgw >> (2 * u);                 // bits of projections 2u, 2u + 1
+        w4[u] = 0x3C003C00u | ((b2 & 1u) << 15) | ((b2 & 2u) << 30);
+      }
+      *reinterpret_cast<uint4*>(zbuf + half * 16384 + trow * 128 + ((c ^ (trow & 7)) << 4)) =
+          make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+  };
+  auto issue_stz = [&](int k) {                            // S^T z of this pair's k-th tile
+    tc_fence_after();
+    const uint32_t zbase = smem_u32(zbuf), sbase = smem_u32(sSt);
+    const uint32_t idesc = idesc_f16_f32(kTile, kD);
+    const uint32_t d_tmem = tmem + pair * 256 + (k & 1) * 128;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+      mma_f16_ss(d_tmem, smem_desc_sw128(zbase + off, 1024), smem_desc_sw128(sbase + off, 1024), idesc,
+                 kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&m1[pair]);
+    mma_issued = true;
+  };
+
+  Part cur, nxt;
+  float v[kH];
+  load_packed(t_first, cur);
+  load_packed(t_first + t_step, nxt);
+  if (PROD) write_signs(cur);
+  decode(cur, v);
+  fence_proxy_async_smem();
+  named_bar_sync(bar_id, 256);                             // the first tile's sign operand is complete
+  if (PROD && leader && t_first < n_tiles) issue_stz(0);
+
+  int mine = 0;
+  for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
+    const uint32_t t_acc = t_reg0 + (mine & 1) * 128;      // S^T z, then the output
+    const uint32_t t_a = t_reg0 + ((mine + 1) & 1) * 128;   // v hi | lo
+    // v in the unit-norm domain times kUnit; norm / sqrt(d) / kUnit is applied to the output
+    const float wq = cur.nrm > 0.f ? (cur.rn / cur.nrm) * qjl : 0.f;
+    const float oscale = cur.nrm * (inv_sqrt_d / kUnit);
+    if (PROD) {
+      if (!mbar_wait(&m1[pair], mine & 1, wait_cycles)) {
+        if (X.err) atomicCAS(X.err, 0, 5);
+        atomicExch(abort_flag, 1);
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int g2 = 0; g2 < 2; ++g2) {
+        uint32_t acc[32];
+        tmem_ld32(t_acc + half * 64 + g2 * 32, acc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[g2 * 32 + k] = fmaf(wq, __uint_as_float(acc[k]), v[g2 * 32 + k]);
+      }
+      // S^T z of this tile has been read and its operand consumed: the next
+      // tile's signs may take the operand's place
+      write_signs(nxt);
+    }
+    // ---- v = hi + lo (binary16) into TMEM: the rotation's A operand ------------------
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+      for (int g8 = 0; g8 < 2; ++g8) {
+        uint32_t hw[8], lw[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int e = ch * 32 + g8 * 16 + 2 * k;
+          const __half2 h = __floats2half2_rn(v[e], v[e + 1]);
+          const float2 hf = __half22float2(h);
+          const float2 lf = __fadd2_rn(make_float2(v[e], v[e + 1]), make_float2(-hf.x, -hf.y));
+          const __half2 l = __floats2half2_rn(lf.x, lf.y);
+          hw[k] = *reinterpret_cast<const uint32_t*>(&h);
+          lw[k] = *reinterpret_cast<const uint32_t*>(&l);
+        }
+        tmem_st8(t_a + half * 32 + ch * 16 + g8 * 8, hw);
+        tmem_st8(t_a + 64 + half * 32 + ch * 16 + g8 * 8, lw);
+      }
+    }
+    tmem_wait_st();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    // #2: v complete in TMEM, every S^T z read done (the rotation overwrites
+    // them), the next tile's sign operand written
+    if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
+    if (leader) {
+      tc_fence_after();
+      const uint32_t sbase = smem_u32(sDH);
+      const uint32_t idesc = idesc_f16_f32(kTile, kD);
+      const uint32_t d_tmem = tmem + pair * 256 + (mine & 1) * 128;
+      const uint32_t a_tmem = tmem + pair * 256 + ((mine + 1) & 1) * 128;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int kk = k & 7;
+        const uint64_t bdesc = smem_desc_sw128(sbase + (kk >> 2) * 16384 + (kk & 3) * 32, 1024);
+        mma_f16_ts(d_tmem, a_tmem + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
+      }
+      mma_commit(&m2[pair]);
+      mma_issued = true;
+    }
+    // ---- while the rotation runs: the next tile's yhat, and the packed row after it --
+    cur = nxt;
+    decode(cur, v);
+    load_packed(t + 2 * t_step, nxt);
+    if (!mbar_wait(&m2[pair], mine & 1, wait_cycles)) {
+      if (X.err) atomicCAS(X.err, 0, 8);
+      atomicExch(abort_flag, 1);
+    }
+    tc_fence_after();
+    // the rotation has read v: the next tile's S^T z may run into its region
+    if (PROD && leader && t + t_step < n_tiles && *reinterpret_cast<volatile int*>(abort_flag) == 0)
+      issue_stz(mine + 1);
+    // ---- my 64 output columns, staged (swizzled) for the TMA store, 32 at a time -------
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t o[32];
+      tmem_ld32(t_acc + half * 64 + hh * 32, o);
+      tmem_wait_ld();
+      if (hh == 0) {
+        if (storer && store_pending) bulk_wait_read0();     // previous tile's store has read the stage
+        named_bar_sync(bar_id, 256);
+      }
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {                      // box `half`: my 64 columns, 8 per chunk
+        const int cc = hh * 4 + c4;
+        uint32_t wv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = c4 * 8 + 2 * u;
+          const __nv_bfloat162 p2 =
+              __floats2bfloat162_rn(__uint_as_float(o[e]) * oscale, __uint_as_float(o[e + 1]) * oscale);
+          wv[u] = *reinterpret_cast<const uint32_t*>(&p2);
+        }
+        *reinterpret_cast<uint4*>(stage + half * (kTile * 128) + trow * 128 + ((cc ^ (trow & 7)) << 4)) =
+            make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      }
+    }
+    tc_fence_before();
+    fence_proxy_async_smem();
+    // #3: the stage is complete, and every read of this tile's output region is
+    // done (the next tile's v goes there)
+    named_bar_sync(bar_id, 256);
+    if (storer) {
+#pragma unroll
+      for (int bx = 0; bx < OutStage<true>::kBoxes; ++bx)
+        tma_store_2d(&tmap_out, stage + bx * (kTile * 128), bx * OutStage<true>::kColsPerBox,
+                     static_cast<int>(t * kTile));
+      bulk_commit();
+      store_pending = true;
+    }
+  }
+  // wind-down (full wait limit): our MMAs and stores complete before the TMEM
+  // and the shared memory are released
+  if (leader && mma_issued) {
+    mma_commit(&fdone[pair]);
+    if (!mbar_wait(&fdone[pair], 0, kWaitCycles) && X.err) atomicCAS(X.err, 0, 4);
+  }
+  if (storer && store_pending) bulk_wait0();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 template <int B, bool PROD, bool BF16OUT>
 int launch(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, cudaStream_t s) {
   const KParams& P = ctx.kp;
@@ -380,13 +713,22 @@ int launch(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, cudaS
   for (int i = 0; i < kD; ++i)
     if (ctx.D[i] < 0) X.Dneg[i >> 5] |= 1u << (i & 31);
   X.err = P.err;
-  const size_t smem = dequant_smem_bytes<BF16OUT>();
-  cudaError_t e = cudaFuncSetAttribute(k_dequant_d128_tc<B, PROD, BF16OUT>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return static_cast<int>(e);
+  X.wait_cycles = wait_limit_cycles();
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
   const int grid = static_cast<int>(n_tiles < ctx.num_sms ? n_tiles : ctx.num_sms);
-  k_dequant_d128_tc<B, PROD, BF16OUT><<<grid, kThreads, smem, s>>>(tmap, P, X, in, n_rows);
+  if constexpr (BF16OUT) {                 // the overlapped kernel (bf16 output)
+    const size_t smem = dequant_ovl_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(k_dequant_d128_ovl<B, PROD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+    k_dequant_d128_ovl<B, PROD><<<grid, kThreads, smem, s>>>(tmap, P, X, in, n_rows);
+  } else {
+    const size_t smem = dequant_smem_bytes<BF16OUT>();
+    cudaError_t e = cudaFuncSetAttribute(k_dequant_d128_tc<B, PROD, BF16OUT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+    k_dequant_d128_tc<B, PROD, BF16OUT><<<grid, kThreads, smem, s>>>(tmap, P, X, in, n_rows);
+  }
   count_launch();
   return static_cast<int>(cudaGetLastError());
 }

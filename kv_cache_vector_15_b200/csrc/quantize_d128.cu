@@ -80,6 +80,15 @@ struct QuantD128Args {
   float eps_abs;                     // binary16 underflow term of the bound (normalised units)
   int* err;                          // device error word
   long long wait_cycles;             // limit of the bounded waits in the tile loop (SM clocks)
+  // bf16 kernel: projections inside the bound go to the exact fix-up kernel
+  // that runs after it, as (row << 8) | j entries of fix_list (fix_count
+  // claims slots, zeroed before the launch); a row whose entries do not fit
+  // gets its bit in fix_rows instead (zeroed too), and all its signs are
+  // recomputed
+  unsigned long long* fix_list;
+  unsigned int* fix_count;
+  unsigned int fix_cap;
+  unsigned int* fix_rows;
 };
 
 // The residual enters the MMA multiplied by 64 (exact), which keeps its
@@ -622,7 +631,8 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
   uint64_t* full = reinterpret_cast<uint64_t*>(sR2 + kPairs * 2 * kTile);   // [pair][2]
   uint64_t* ydone = full + 2 * kPairs;                           // [pair]
   uint64_t* mdone = ydone + kPairs;                              // [pair]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kPairs);
+  uint64_t* fdone = mdone + kPairs;                              // [pair] wind-down commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fdone + kPairs);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* loads_issued = abort_flag + 1;                            // [pair][stage]
 
@@ -631,7 +641,7 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
   const long long wait_cycles = X.wait_cycles;
   if (tid == 0) {
     for (int i = 0; i < 2 * kPairs; ++i) mbar_init(&full[i], 1);
-    for (int i = 0; i < kPairs; ++i) { mbar_init(&ydone[i], 1); mbar_init(&mdone[i], 1); }
+    for (int i = 0; i < kPairs; ++i) { mbar_init(&ydone[i], 1); mbar_init(&mdone[i], 1); mbar_init(&fdone[i], 1); }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -659,12 +669,17 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
   const uint32_t tmem = *tmem_slot;
 
   const int wgi = warp >> 2, pair = wgi >> 1, half = wgi & 1, lb = warp & 3;
-  const bool leader = (half == 0 && lb == 0 && lane == 0);       // waits for stages, issues MMAs
-  const bool loader = (half == 1 && lb == 0 && lane == 0);       // issues the stage loads (TMA)
+  // the leader issues the pair's MMAs, the loader (a warp of the other half)
+  // its stage loads
+  const bool leader = (half == 0 && lb == 0 && lane == 0);
+  const bool loader = (half == 1 && lb == 0 && lane == 0);
   const int trow = lb * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>(lb * 32) << 16;
-  const uint32_t t_acc = tmem + lane_base + pair * 256;          // y', then the projections
-  const uint32_t t_a = t_acc + 128;                              // residual hi | lo
+  // two 128-column regions per pair, alternating roles from tile to tile: the
+  // k-th tile's y' (then its projections) in region k mod 2, its residual
+  // hi | lo in the other, so the next tile's rotation can run into the region
+  // of this tile's residual while this tile's projections are still read
+  const uint32_t t_reg0 = tmem + lane_base + pair * 256;
   const uint32_t bar_id = 1 + pair;
   uint8_t* stages = sX + pair * NS * kStage;
   uint64_t* pfull = full + 2 * pair;
@@ -682,7 +697,7 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
                   static_cast<int>(tile * kTile));
   };
   int issued[2] = {0, 0}, waited[2] = {0, 0};                    // stage loads (loader / leader)
-  int y_issued = 0, y_seen = 0, m_issued = 0, m_seen = 0;       // MMA commits (leader)
+  bool mma_issued = false;                                       // leader: any MMA of ours in flight
   if (loader) {
     prefetch_tmap(&tmap);
     if (t_first < n_tiles) { issue_load(t_first, 0); ++issued[0]; }
@@ -694,17 +709,17 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
   // by hand, so the others reach the abort check
   auto issue_rotation = [&](int k) {
     const int b = k & 1;
-    ++y_issued;
     if (!mbar_wait(&pfull[b], (k >> 1) & 1, wait_cycles)) {
       flag_error(X.err, abort_flag, 2);
       mbar_arrive(&ydone[pair]);
       return;
     }
     ++waited[b];
+    mma_issued = true;
     tc_fence_after();
     const uint32_t xbase = smem_u32(stages + b * kStage), hbase = smem_u32(sHD);
     const uint32_t idesc = idesc_bf16_f32(kTile, kD);
-    const uint32_t d_tmem = tmem + pair * 256;
+    const uint32_t d_tmem = tmem + pair * 256 + (k & 1) * 128;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -713,8 +728,9 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
     }
     mma_commit(&ydone[pair]);
   };
-  // each tile's rotation is issued as soon as the previous tile's accumulator
-  // has been read (below), so it runs under that tile's stores
+  // each later tile's rotation is issued as soon as the previous tile's
+  // projection has completed (below), so it runs under that tile's sign
+  // extraction and stores
   if (leader && t_first < n_tiles) issue_rotation(0);
 
   // magnitude thresholds and centroids of the symmetric codebook (x 64 for
@@ -728,13 +744,12 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
 
   int mine = 0;
   for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
-    const int buf = mine & 1;
-    if (mbar_wait(&ydone[pair], mine & 1, wait_cycles)) {
-      if (leader) ++y_seen;
-    } else {
-      flag_error(X.err, abort_flag, 5);
-    }
+    const uint32_t t_acc = t_reg0 + (mine & 1) * 128;            // y', then the projections
+    const uint32_t t_a = t_reg0 + ((mine + 1) & 1) * 128;         // residual hi | lo
+    if (!mbar_wait(&ydone[pair], mine & 1, wait_cycles)) flag_error(X.err, abort_flag, 5);
     tc_fence_after();
+    // the stage has been read by this tile's rotation: refill it two tiles ahead
+    if (loader && t + NS * t_step < n_tiles) { issue_load(t + NS * t_step, mine & 1); ++issued[mine & 1]; }
 
     // ---- the row's ||y'||^2 from both halves' sums of squares -------------------
     {
@@ -817,91 +832,70 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
       tc_fence_after();
       const uint32_t sbase = smem_u32(sS);
       const uint32_t idesc = idesc_f16_f32(kTile, kM);
-      const uint32_t d_tmem = tmem + pair * 256;
+      const uint32_t d_tmem = tmem + pair * 256 + (mine & 1) * 128;
+      const uint32_t a_tmem = tmem + pair * 256 + ((mine + 1) & 1) * 128;
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         const int kk = k & 7;
         const uint64_t bdesc = smem_desc_sw128(sbase + (kk >> 2) * 16384 + (kk & 3) * 32, 1024);
-        mma_f16_ts(d_tmem, d_tmem + 128 + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
+        mma_f16_ts(d_tmem, a_tmem + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
       }
       mma_commit(&mdone[pair]);
-      ++m_issued;
+      mma_issued = true;
     }
-    if (mbar_wait(&mdone[pair], mine & 1, wait_cycles)) {
-      if (leader) ++m_seen;
-    } else {
-      flag_error(X.err, abort_flag, 3);
-    }
+    if (!mbar_wait(&mdone[pair], mine & 1, wait_cycles)) flag_error(X.err, abort_flag, 3);
     tc_fence_after();
+    // the projection has read this tile's residual region: the next tile's
+    // rotation may write it
+    if (leader && t + t_step < n_tiles && *reinterpret_cast<volatile int*>(abort_flag) == 0) issue_rotation(mine + 1);
 
     // ---- my 64 signs, exact recomputation within the error bound of zero ------------
     const float eps = kResScale * fmaf(X.eps_scale, rho, X.eps_abs);
-    uint32_t s0 = 0, s1 = 0, f0 = 0, f1 = 0;
+    uint32_t s0 = 0, s1 = 0;
     float pmin = INFINITY;
-    {
-      uint32_t p[kH];
-      tmem_ld32(t_acc + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
-      tmem_ld32(t_acc + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t p[32];
+      tmem_ld32(t_acc + half * 64 + hh * 32, p);
       tmem_wait_ld();
+      uint32_t sw = 0u;
 #pragma unroll
-      for (int j = 31; j >= 0; --j) {
-        s0 = __funnelshift_l(p[j], s0, 1);
-        s1 = __funnelshift_l(p[32 + j], s1, 1);
-      }
+      for (int j = 31; j >= 0; --j) sw = __funnelshift_l(p[j], sw, 1);
+      if (hh == 0) s0 = sw; else s1 = sw;
 #pragma unroll
-      for (int j = 0; j < kH; j += 2)
+      for (int j = 0; j < 32; j += 2)
         pmin = fminf(pmin, fminf(fabsf(__uint_as_float(p[j])), fabsf(__uint_as_float(p[j + 1]))));
     }
-    // rare: find which projections are within the bound.  The TMEM loads are
-    // warp-collective, so the whole warp takes this branch when any lane needs it.
-    if (__any_sync(0xffffffffu, pmin < eps)) {
+    // rare: projections inside the bound.  They are listed for the exact
+    // fix-up kernel that runs after this one (this tile's residual region is
+    // already being overwritten by the next tile's rotation); the tensor-core
+    // signs stay in place until then.  The TMEM loads are warp-collective, so
+    // the whole warp reloads when any lane needs it.
+    const int64_t row = t * kTile + trow;
+    const bool mine_flagged = pmin < eps && !zero_row && rho != 0.f && row < n_rows;
+    if (__any_sync(0xffffffffu, mine_flagged)) {
 #pragma unroll 1
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t p[32];
         tmem_ld32(t_acc + half * 64 + hh * 32, p);
         tmem_wait_ld();
-        uint32_t f = 0u;
+        if (mine_flagged) {
+          uint32_t f = 0u;
 #pragma unroll
-        for (int j = 31; j >= 0; --j) f = (f << 1) | (fabsf(__uint_as_float(p[j])) < eps ? 1u : 0u);
-        if (hh == 0) f0 = f; else f1 = f;
-      }
-    }
-    const int nflag = __popc(f0) + __popc(f1);
-    const int passes = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(nflag));
-    for (int q = 0; q < passes; ++q) {
-      int j = -1;
-      if (q < nflag) {
-        if (f1) j = 32 + __ffs(f1) - 1;
-        if (f0) j = __ffs(f0) - 1;
-      }
-      const int jg = half * 64 + (j < 0 ? 0 : j);
-      float acc = 0.f;
-      // S_j . hi, then S_j . lo: 16 columns (32 coordinates) per load
-#pragma unroll 1
-      for (int part = 0; part < 8; ++part) {
-        uint32_t a[16];
-        tmem_ld16(t_a + part * 16, a);
-        tmem_wait_ld();
-        if (j >= 0) {
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int chunk = (part & 3) * 4 + ch, kb = chunk >> 3, cc = chunk & 7;
-            const uint4 sv = *reinterpret_cast<const uint4*>(sS + kb * 16384 + jg * 128 + ((cc ^ (jg & 7)) << 4));
-            const uint32_t sws[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-            for (int uu = 0; uu < 4; ++uu) {
-              const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sws[uu]));
-              const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&a[ch * 4 + uu]));
-              acc = fmaf(sf.x, hf.x, acc);
-              acc = fmaf(sf.y, hf.y, acc);
-            }
+          for (int j = 31; j >= 0; --j) f = (f << 1) | (fabsf(__uint_as_float(p[j])) < eps ? 1u : 0u);
+          const unsigned int nf = __popc(f);
+          unsigned int slot = nf ? atomicAdd(X.fix_count, nf) : 0u;
+          // every claimed slot below the capacity is written; a row with an
+          // entry beyond it is marked for the recomputation of all its signs
+          while (f) {
+            const int j = half * 64 + hh * 32 + __ffs(f) - 1;
+            if (slot < X.fix_cap)
+              X.fix_list[slot] = (static_cast<unsigned long long>(row) << 8) | static_cast<unsigned>(j);
+            ++slot;
+            f &= f - 1;
           }
+          if (slot > X.fix_cap) atomicOr(X.fix_rows + (row >> 5), 1u << (row & 31));
         }
-      }
-      if (j >= 0) {
-        const uint32_t m = 1u << (j & 31), nb = acc < 0.f ? m : 0u;
-        if (j < 32) { s0 = (s0 & ~m) | nb; f0 &= ~m; }
-        else { s1 = (s1 & ~m) | nb; f1 &= ~m; }
       }
     }
     if (zero_row || rho == 0.f) s0 = s1 = 0u;
@@ -909,8 +903,6 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
     // #A: every read of this tile's accumulator and operand columns is done
     // (and a uniform abort check): the next tile's rotation may start
     if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
-    if (leader && t + t_step < n_tiles) issue_rotation(mine + 1);
-    const int64_t row = t * kTile + trow;
     if (row < n_rows) {
       uint32_t* co = reinterpret_cast<uint32_t*>(out.codes + row * (B * 16) + half * (B * 8));
       if constexpr (B == 1) {
@@ -935,19 +927,14 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
         out.rnorm[row] = zero_row ? 0.f : n * rho;
       }
     }
-    // the stage was read by this tile's rotation MMA: refill it two tiles ahead
-    // (a TMA issue can hold its thread for a while, so it comes from a warp of
-    // the other half than the one that issues the MMAs)
-    if (loader && t + NS * t_step < n_tiles) { issue_load(t + NS * t_step, buf); ++issued[buf]; }
   }
   // Wind-down, with the full wait limit whatever limit the loop ran with: no
   // MMA of ours may still be running and no stage load still landing when the
-  // TMEM and the shared memory are released.
-  if (leader) {
-    for (; y_seen < y_issued; ++y_seen)
-      if (!mbar_wait(&ydone[pair], y_seen & 1, kWaitCycles)) { flag_error(X.err, abort_flag, 4); break; }
-    for (; m_seen < m_issued; ++m_seen)
-      if (!mbar_wait(&mdone[pair], m_seen & 1, kWaitCycles)) { flag_error(X.err, abort_flag, 4); break; }
+  // TMEM and the shared memory are released.  One more commit tracks every
+  // MMA this thread has issued.
+  if (leader && mma_issued) {
+    mma_commit(&fdone[pair]);
+    if (!mbar_wait(&fdone[pair], 0, kWaitCycles)) flag_error(X.err, abort_flag, 4);
   }
   if (loader) { loads_issued[2 * pair] = issued[0]; loads_issued[2 * pair + 1] = issued[1]; }
   __syncthreads();
@@ -967,6 +954,128 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
   }
 }
 
+// Exact signs of the projections the tensor-core kernel left inside its
+// error bound, in fp64 from the input row and the codes the kernel stored for
+// it: norm, D, the Walsh-Hadamard butterflies, r = y - c[code], p_j = S_j . r,
+// and the sign bit set or cleared in place (1 = negative; p_j = 0 counts as
+// positive).  Listed (row, j) entries first, one warp each; then the rows
+// marked in the overflow bitmap, all of whose m = 128 signs are recomputed.
+// Lane l holds coordinates 4 l .. 4 l + 3 of the row.
+template <int B, bool BF16IN>
+__device__ __forceinline__ void fixup_residual(const KParams& P, const void* __restrict__ x, int64_t ld, int64_t row,
+                                               const Packed& out, int lane, double (&r)[4]) {
+  double v[4];
+  if constexpr (BF16IN) {
+    const uint2 xw = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(x) + row * ld + 4 * lane);
+    v[0] = __uint_as_float(xw.x << 16); v[1] = __uint_as_float(xw.x & 0xffff0000u);
+    v[2] = __uint_as_float(xw.y << 16); v[3] = __uint_as_float(xw.y & 0xffff0000u);
+  } else {
+    const float4 xw = *reinterpret_cast<const float4*>(static_cast<const float*>(x) + row * ld + 4 * lane);
+    v[0] = xw.x; v[1] = xw.y; v[2] = xw.z; v[3] = xw.w;
+  }
+  // codes of coordinates 4 lane .. 4 lane + 3: bits [4 B lane, 4 B lane + 4 B) of the row
+  const uint8_t* cb = out.codes + row * (B * 16);
+  const int bit0 = 4 * B * lane;
+  uint32_t win = 0;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const int byte = (bit0 >> 3) + k;
+    if (byte < B * 16) win |= static_cast<uint32_t>(cb[byte]) << (8 * k);
+  }
+  win >>= (bit0 & 7);
+  const uint32_t dm = P.Dmask[lane >> 3] >> (4 * (lane & 7));
+  double ss = 0.0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if ((dm >> q) & 1u) v[q] = -v[q];
+    ss = fma(v[q], v[q], ss);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  // butterflies over coordinate bits 0, 1 (in the lane), then 2 .. 6 (across lanes)
+#pragma unroll
+  for (int h = 1; h < 4; h <<= 1)
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if ((q & h) == 0) {
+        const double a = v[q], c2 = v[q + h];
+        v[q] = a + c2;
+        v[q + h] = a - c2;
+      }
+#pragma unroll
+  for (int lh = 1; lh < 32; lh <<= 1)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const double o = __shfl_xor_sync(0xffffffffu, v[q], lh);
+      v[q] = (lane & lh) ? o - v[q] : v[q] + o;
+    }
+  const double inv = 1.0 / (sqrt(ss) * sqrt(static_cast<double>(kD)));
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t code = (win >> (B * q)) & ((1u << B) - 1u);
+    r[q] = v[q] * inv - static_cast<double>(P.c[code]);
+  }
+}
+
+// S_j . r over the warp (lane l: coordinates 4 l .. 4 l + 3), all lanes get it
+__device__ __forceinline__ double fixup_project(const KParams& P, int j, int lane, const double (&r)[4]) {
+  const uint2 sw = __ldg(reinterpret_cast<const uint2*>(P.S + j * kD + 4 * lane));
+  const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sw.x));
+  const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sw.y));
+  double p = static_cast<double>(s01.x) * r[0];
+  p = fma(static_cast<double>(s01.y), r[1], p);
+  p = fma(static_cast<double>(s23.x), r[2], p);
+  p = fma(static_cast<double>(s23.y), r[3], p);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+  return p;
+}
+
+template <int B, bool BF16IN>
+__global__ void __launch_bounds__(256)
+k_qjl_fixup_d128(const KParams P, const void* __restrict__ x, int64_t ld, int64_t n_rows, const Packed out,
+                 const unsigned long long* __restrict__ fix_list, const unsigned int* __restrict__ fix_count,
+                 unsigned int fix_cap, const unsigned int* __restrict__ fix_rows) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const unsigned int claimed = *fix_count;
+  const int64_t n_list = claimed < fix_cap ? claimed : fix_cap;
+  for (int64_t e = warp; e < n_list; e += nwarps) {
+    const unsigned long long ent = fix_list[e];
+    const int64_t row = static_cast<int64_t>(ent >> 8);
+    const int j = static_cast<int>(ent & 0xffu);
+    if (row >= n_rows || j >= kM) continue;                      // never listed; kept in bounds regardless
+    double r[4];
+    fixup_residual<B, BF16IN>(P, x, ld, row, out, lane, r);
+    const double p = fixup_project(P, j, lane, r);
+    if (lane == 0) {
+      unsigned int* word = reinterpret_cast<unsigned int*>(out.signs + row * 16) + (j >> 5);
+      const unsigned int m = 1u << (j & 31);
+      if (p < 0.0) atomicOr(word, m); else atomicAnd(word, ~m);
+    }
+  }
+  if (claimed <= fix_cap) return;                                // no overflow: the bitmap is empty
+  const int64_t n_words = (n_rows + 31) >> 5;
+  for (int64_t w = warp; w < n_words; w += nwarps) {
+    uint32_t bits = fix_rows[w];
+    while (bits) {
+      const int b = __ffs(bits) - 1;
+      bits &= bits - 1;
+      const int64_t row = w * 32 + b;
+      double r[4];
+      fixup_residual<B, BF16IN>(P, x, ld, row, out, lane, r);
+      uint32_t word = 0u;                                        // lane l keeps sign word l / 8... built below
+#pragma unroll 1
+      for (int j = 0; j < kM; ++j) {
+        const double p = fixup_project(P, j, lane, r);
+        if (lane == (j >> 5) && p < 0.0) word |= 1u << (j & 31);
+      }
+      if (lane < kM / 32) reinterpret_cast<uint32_t*>(out.signs + row * 16)[lane] = word;
+    }
+  }
+}
+
 // -------------------------------------------------------------------------- host
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() { return tensor_map_encoder(); }
 
@@ -974,8 +1083,19 @@ constexpr size_t quant_rot_smem_bytes() {
   return 1024 + 2 * kSmemS + 2 * kPairs * XStage<true>::kBytes + 2 * kPairs * 2 * kTile * 4 + 256;
 }
 
+// The bf16 kernel's fix-up scratch in the caller's workspace: the overflow
+// bitmap (one bit per row), the list counter (both zeroed before each
+// launch), then the list.  Two entries per tile is about three times what the
+// error bound flags on Gaussian-like rows.
+size_t fix_bitmap_bytes(int64_t n_rows) { return (static_cast<size_t>((n_rows + 31) / 32) * 4 + 255) / 256 * 256; }
+int64_t fix_cap_for(int64_t n_rows) { return 2 * ((n_rows + kTile - 1) / kTile) + 4096; }
+size_t fix_scratch_bytes(int64_t n_rows) {
+  return fix_bitmap_bytes(n_rows) + 256 + static_cast<size_t>(fix_cap_for(n_rows)) * sizeof(unsigned long long);
+}
+
 template <int B, bool BF16IN>
-int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, const Packed& out, cudaStream_t s) {
+int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, const Packed& out, void* scratch,
+              cudaStream_t s) {
   const KParams& P = ctx.kp;
   auto encode = get_encode();
   if (!encode) return static_cast<int>(cudaErrorNotSupported);
@@ -995,14 +1115,31 @@ int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, cons
   X.eps_abs = ctx.qjl_eps_abs;
   X.err = P.err;
   X.wait_cycles = wait_limit_cycles();
+  X.fix_rows = nullptr;
+  X.fix_list = nullptr;
+  X.fix_count = nullptr;
+  X.fix_cap = 0;
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
   const int grid = static_cast<int>(n_tiles < ctx.num_sms ? n_tiles : ctx.num_sms);
   if constexpr (BF16IN) {                // bf16 rows: the rotation on the tensor cores
+    if (!scratch) return static_cast<int>(cudaErrorInvalidValue);   // the fix-up scratch lives there
+    uint8_t* sc = static_cast<uint8_t*>(scratch);
+    X.fix_rows = reinterpret_cast<unsigned int*>(sc);
+    X.fix_count = reinterpret_cast<unsigned int*>(sc + fix_bitmap_bytes(n_rows));
+    X.fix_list = reinterpret_cast<unsigned long long*>(sc + fix_bitmap_bytes(n_rows) + 256);
+    const int64_t cap = fix_cap_for(n_rows), forced = fixup_cap_override();
+    X.fix_cap = static_cast<unsigned int>(forced > 0 && forced < cap ? forced : cap);
+    cudaError_t e = cudaMemsetAsync(sc, 0, fix_bitmap_bytes(n_rows) + 256, s);
+    if (e != cudaSuccess) return static_cast<int>(e);
     const size_t smem = quant_rot_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(k_quantize_d128_rot_tc<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    e = cudaFuncSetAttribute(k_quantize_d128_rot_tc<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
     k_quantize_d128_rot_tc<B><<<grid, kThreads, smem, s>>>(tmap, P, X, n_rows, out);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return static_cast<int>(e);
+    k_qjl_fixup_d128<B, true><<<ctx.num_sms * 8, 256, 0, s>>>(P, x, ld, n_rows, out, X.fix_list, X.fix_count,
+                                                                 X.fix_cap, X.fix_rows);
   } else {                                // fp32 rows: the rotation in registers
     const size_t smem = quant_smem_bytes<false>();
     cudaError_t e = cudaFuncSetAttribute(k_quantize_d128_tc<B, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1016,6 +1153,11 @@ int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, cons
 
 }  // namespace
 
+size_t quantize_d128_scratch_bytes(const tq_ctx& ctx, int64_t n_rows) {
+  (void)ctx;
+  return fix_scratch_bytes(n_rows);
+}
+
 bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows) {
   if (ctx.d_in != ctx.d) return false;                   // padded rows use the general kernel
   const KParams& P = ctx.kp;
@@ -1024,22 +1166,22 @@ bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows) {
 }
 
 int launch_quantize_d128(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
-                         const Packed& out, void* stream) {
+                         const Packed& out, void* scratch, void* stream) {
   const KParams& P = ctx.kp;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (x_is_bf16) {
     switch (P.B) {
-      case 1: return launch_tc<1, true>(ctx, x, n_rows, ld, out, s);
-      case 2: return launch_tc<2, true>(ctx, x, n_rows, ld, out, s);
-      case 3: return launch_tc<3, true>(ctx, x, n_rows, ld, out, s);
-      default: return launch_tc<4, true>(ctx, x, n_rows, ld, out, s);
+      case 1: return launch_tc<1, true>(ctx, x, n_rows, ld, out, scratch, s);
+      case 2: return launch_tc<2, true>(ctx, x, n_rows, ld, out, scratch, s);
+      case 3: return launch_tc<3, true>(ctx, x, n_rows, ld, out, scratch, s);
+      default: return launch_tc<4, true>(ctx, x, n_rows, ld, out, scratch, s);
     }
   }
   switch (P.B) {
-    case 1: return launch_tc<1, false>(ctx, x, n_rows, ld, out, s);
-    case 2: return launch_tc<2, false>(ctx, x, n_rows, ld, out, s);
-    case 3: return launch_tc<3, false>(ctx, x, n_rows, ld, out, s);
-    default: return launch_tc<4, false>(ctx, x, n_rows, ld, out, s);
+    case 1: return launch_tc<1, false>(ctx, x, n_rows, ld, out, scratch, s);
+    case 2: return launch_tc<2, false>(ctx, x, n_rows, ld, out, scratch, s);
+    case 3: return launch_tc<3, false>(ctx, x, n_rows, ld, out, scratch, s);
+    default: return launch_tc<4, false>(ctx, x, n_rows, ld, out, scratch, s);
   }
 }
 

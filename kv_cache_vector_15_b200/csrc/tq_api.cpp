@@ -28,9 +28,10 @@ void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::m
 
 constexpr long long kDefaultWaitCycles = 2000000000ll;         // about one second at 2 GHz
 static std::atomic<long long> g_wait_limit{kDefaultWaitCycles};
-static std::atomic<int64_t> g_fail_alloc{0}, g_fail_launch{0};
+static std::atomic<int64_t> g_fail_alloc{0}, g_fail_launch{0}, g_fixup_cap{0};
 
 long long wait_limit_cycles() { return g_wait_limit.load(std::memory_order_relaxed); }
+int64_t fixup_cap_override() { return g_fixup_cap.load(std::memory_order_relaxed); }
 
 static bool take_one(std::atomic<int64_t>& n) {
   int64_t v = n.load(std::memory_order_relaxed);
@@ -504,6 +505,7 @@ tq_status tq_test_set(tq_test_knob knob, int64_t value) {
       return TQ_OK;
     case TQ_TEST_FAIL_ALLOC: g_fail_alloc.store(value, std::memory_order_relaxed); return TQ_OK;
     case TQ_TEST_FAIL_LAUNCH: g_fail_launch.store(value, std::memory_order_relaxed); return TQ_OK;
+    case TQ_TEST_FIXUP_CAP: g_fixup_cap.store(value, std::memory_order_relaxed); return TQ_OK;
   }
   return fail(TQ_ERR_INVALID_ARG, "unknown test setting");
 }

@@ -47,6 +47,7 @@ void count_launch(int n = 1);
 // test settings (tq_test_set): the bounded-wait limit the tensor-core
 // quantize kernel's tile loop runs with, and injected host-side failures
 long long wait_limit_cycles();
+int64_t fixup_cap_override();          // 0: the default capacity of the quantize fix-up list
 bool take_injected_alloc_failure();
 bool take_injected_launch_failure();
 
@@ -95,8 +96,9 @@ struct tq_ctx;
 namespace tq {
 // d = 128 hot-path kernels (quantize_d128.cu, ...)
 bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows);
+size_t quantize_d128_scratch_bytes(const tq_ctx& ctx, int64_t n_rows);   // deferred sign fix-up list
 int launch_quantize_d128(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
-                         const Packed& out, void* stream);
+                         const Packed& out, void* scratch, void* stream);
 bool dequant_d128_applies(const tq_ctx& ctx, int64_t n_rows);
 bool logits_d128_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys);
 int launch_logits_d128(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,

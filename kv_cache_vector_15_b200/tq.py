@@ -25,7 +25,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_NOMEM, TQ_ERR_CUDA = range(5)
 TQ_BF16, TQ_F32 = 0, 1
 TQ_DEQUANT_PROD, TQ_DEQUANT_MSE = 0, 1
-TQ_TEST_WAIT_LIMIT, TQ_TEST_FAIL_ALLOC, TQ_TEST_FAIL_LAUNCH = 0, 1, 2
+TQ_TEST_WAIT_LIMIT, TQ_TEST_FAIL_ALLOC, TQ_TEST_FAIL_LAUNCH, TQ_TEST_FIXUP_CAP = 0, 1, 2, 3
 
 # exported symbols, in header order
 SYMBOLS = [

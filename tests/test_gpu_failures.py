@@ -32,6 +32,7 @@ def tq():
     _tq.test_set(_tq.TQ_TEST_WAIT_LIMIT, 0)
     _tq.test_set(_tq.TQ_TEST_FAIL_ALLOC, 0)
     _tq.test_set(_tq.TQ_TEST_FAIL_LAUNCH, 0)
+    _tq.test_set(_tq.TQ_TEST_FIXUP_CAP, 0)
 
 
 @pytest.mark.parametrize("b", [3, 4])
@@ -83,4 +84,30 @@ def test_injected_launch_failure(tq):
     got = T.quantize(xd).to_numpy()
     T.sync_status()
     parity.assert_quantize_ok(parity.compare_quantize(P, got, ot.quantize(x, P, keep_intermediates=True)))
+    T.close()
+
+
+@pytest.mark.parametrize("b", [3, 4])
+def test_quantize_fixup_overflow_path(tq, b):
+    """The d = 128 quantize kernel lists projections inside its tensor-core
+    error bound for an exact fp64 fix-up; with the list capped at one entry
+    almost every such row takes the overflow path (all its signs recomputed).
+    Both paths must give the oracle's signs."""
+    d, m, n = 128, 128, 60000
+    P = op.Params(d, b, m, seed=0)
+    xt, x = make_rows(d, n, "bf16", seed=41 + b)
+    T = tq.TurboQuant(d, b, m, seed=0)
+    xd = xt.cuda()
+    want = ot.quantize(x, P, keep_intermediates=True)
+    tq.test_set(tq.TQ_TEST_FIXUP_CAP, 1)
+    try:
+        got = T.quantize(xd).to_numpy()
+        T.sync_status()
+    finally:
+        tq.test_set(tq.TQ_TEST_FIXUP_CAP, 0)
+    parity.assert_quantize_ok(parity.compare_quantize(P, got, want))
+    got2 = T.quantize(xd).to_numpy()
+    T.sync_status()
+    parity.assert_quantize_ok(parity.compare_quantize(P, got2, want))
+    assert all(np.array_equal(got[k], got2[k]) for k in ("codes", "signs"))
     T.close()
