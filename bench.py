@@ -575,10 +575,11 @@ def run_aux(args, cfg, ws, rank, local):
         lg = torch.empty((n_sets, g, n_keys), dtype=torch.float32, device=dev)
         vhat = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
         work = torch.empty(max(T.logits_workspace_bytes(n_sets, g, n_keys), 16), dtype=torch.uint8, device=dev)
+        qwork = torch.empty(max(T.quantize_workspace_bytes(N), 16), dtype=torch.uint8, device=dev)
 
         def step():
-            T.quantize(dK, pK, stream=stream)
-            T.quantize(dV, pV, stream=stream)
+            T.quantize(dK, pK, workspace=qwork, stream=stream)
+            T.quantize(dV, pV, workspace=qwork, stream=stream)
             T.logits(dQ, pK, n_sets, g, n_keys, out=lg, workspace=work, stream=stream)
             T.dequant(pV, N, out=vhat, stream=stream)
         units, unit = n_sets * g * n_keys, "logits/s"

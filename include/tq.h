@@ -286,9 +286,17 @@ tq_status tq_split_init(int d, int d_hi, int b_hi, int b_lo, uint64_t seed, tq_s
 tq_status tq_split_destroy(tq_split* sp);
 /* part 0 (channels [0, d_hi)) or 1 (channels [d_hi, d)); owned by sp */
 tq_status tq_split_part(const tq_split* sp, int part, const tq_ctx** out);
-/* x [n_rows, ld_x >= d] as tq_quantize; each part's columns into its packed rows. */
+/* Workspace bytes of tq_split_quantize for n_rows rows: the larger of the
+ * two parts' tq_quantize_workspace_bytes (the parts run one after the other
+ * on the caller's stream and share it); 0 when neither part needs one. */
+size_t tq_split_quantize_workspace_bytes(const tq_split* sp, int64_t n_rows);
+/* x [n_rows, ld_x >= d] as tq_quantize; each part's columns into its packed
+ * rows.  workspace: device memory, 16-byte aligned, at least
+ * tq_split_quantize_workspace_bytes(sp, n_rows) bytes (NULL when that is 0);
+ * TQ_ERR_INVALID_ARG when missing or too small. */
 tq_status tq_split_quantize(const tq_split* sp, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
-                            tq_packed out_hi, tq_packed out_lo, void* stream);
+                            tq_packed out_hi, tq_packed out_lo, void* workspace, size_t workspace_bytes,
+                            void* stream);
 size_t tq_split_logits_workspace_bytes(const tq_split* sp, int64_t n_sets, int g, int64_t n_keys);
 /* As tq_logits, with q [n_sets, g, d] and each part's packed keys; out is the
  * sum of the two parts' estimates. */

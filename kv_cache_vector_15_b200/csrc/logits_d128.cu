@@ -46,7 +46,6 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128, kM = 128, kTile = 128;
-constexpr long long kWaitCycles = 2000000000ll;
 constexpr uint32_t kTmemCols = 512;          // split evenly between the warpgroups (A columns, then D)
 
 __host__ __device__ constexpr uint32_t idesc_i8(uint32_t M, uint32_t N) {
@@ -82,11 +81,35 @@ struct Shape {
 };
 
 constexpr int kStages = 4;                   // packed tiles in flight per warpgroup
+constexpr int kScalFloats = 160;             // per-warpgroup partial maxima / sums, constants, scales
+
+// Four signed 8-bit limbs of v (|v| < 2^31): v = l0 + 2^8 l1 + 2^16 l2 + 2^24 l3.
+__device__ __forceinline__ void split_limbs(int v, int8_t* l) {
+  const int l0 = static_cast<int8_t>(v & 0xff);
+  const int r1 = (v - l0) >> 8;
+  const int l1 = static_cast<int8_t>(r1 & 0xff);
+  const int r2 = (r1 - l1) >> 8;
+  const int l2 = static_cast<int8_t>(r2 & 0xff);
+  l[0] = static_cast<int8_t>(l0);
+  l[1] = static_cast<int8_t>(l1);
+  l[2] = static_cast<int8_t>(l2);
+  l[3] = static_cast<int8_t>((r2 - l2) >> 8);
+}
+
+// Recombined limb sums.  Each accumulator is at most 128 * (255 / 8) * K < 2^22 in
+// magnitude (K <= 640 operand bytes), so the two
+// low limbs join exactly in 32-bit integers; the rest is two fp32 FMAs.
+__device__ __forceinline__ float join_limbs(const uint32_t* a) {
+  const int lo = static_cast<int>(a[0]) + static_cast<int>(a[1] << 8);
+  return fmaf(static_cast<float>(static_cast<int>(a[3])), 16777216.f,
+              fmaf(static_cast<float>(static_cast<int>(a[2])), 65536.f, static_cast<float>(lo)));
+}
 
 struct LogitsArgs {
   float wbit[3];                  // weight of code bit 0 / 1 / 2 in the centroid
   float wpar;                     // weight of the code's parity bit (3-bit codes)
   float cconst;                   // centroid constant term
+  long long wait_cycles;          // bound of every wait
   int* err;
 };
 
@@ -123,8 +146,8 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
   const int wg = warp >> 2, wl = warp & 3;
   uint8_t* sB = smem + wg * kBBytes;
   uint8_t* stages = smem + kWG * kBBytes + wg * kStages * S::kStageBytes;
-  float* sScal = reinterpret_cast<float*>(smem + kWG * (kBBytes + kStages * S::kStageBytes)) + wg * 64;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWG * (kBBytes + kStages * S::kStageBytes) + kWG * 64 * 4);
+  float* sScal = reinterpret_cast<float*>(smem + kWG * (kBBytes + kStages * S::kStageBytes)) + wg * kScalFloats;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWG * (kBBytes + kStages * S::kStageBytes) + kWG * kScalFloats * 4);
   uint64_t* full = bars + wg * kStages;                     // [wg][stage]
   uint64_t* mdone = bars + kWG * kStages;                   // [wg]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kWG);
@@ -200,45 +223,59 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
       // ---- build the query operand of this set --------------------------------
       cur_set = set;
       named_bar_sync(1 + wg, 128);                      // previous tile's MMA inputs no longer in use
-      // thread trow owns coordinate/projection trow; per query maxima for scaling
-      float* sMax = sScal;                              // [0..G): mse max, [G..2G): qjl max
-      if (trow < 2 * G) sMax[trow] = 0.f;
-      named_bar_sync(1 + wg, 128);
+      // per-warp maxima and sums of every query's two halves, combined below in a
+      // fixed order (thread trow owns coordinate / projection trow)
+      float* sPM = sScal;                               // [warp][2G] partial maxima
+      float* sPS = sScal + 64;                          // [warp][2G] partial sums
+      float* sC = sScal + 128;                          // [2G] constant terms
+      float* sInv = sScal + 144;                        // [2G] inverse fixed-point scales
       const float* qs = qp + set * G * (kD + kM);
 #pragma unroll
       for (int q = 0; q < G; ++q) {
-        float a = fabsf(qs[q * (kD + kM) + trow]);
-        float b = fabsf(qs[q * (kD + kM) + kD + trow]);
+        const float va = qs[q * (kD + kM) + trow], vb = qs[q * (kD + kM) + kD + trow];
+        float a = fabsf(va), b = fabsf(vb), sa = va, sb = vb;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
           a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
           b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
+          sa += __shfl_xor_sync(0xffffffffu, sa, o);
+          sb += __shfl_xor_sync(0xffffffffu, sb, o);
         }
         if (lane == 0) {
-          atomicMax(reinterpret_cast<int*>(&sMax[q]), __float_as_int(a));
-          atomicMax(reinterpret_cast<int*>(&sMax[G + q]), __float_as_int(b));
+          sPM[wl * 16 + q] = a;
+          sPM[wl * 16 + G + q] = b;
+          sPS[wl * 16 + q] = sa;
+          sPS[wl * 16 + G + q] = sb;
         }
       }
       named_bar_sync(1 + wg, 128);
-      // fixed-point scales: |value| * 2^F <= 2^22
-      float scale[2 * G];
       float wmax = fabsf(X.wbit[0]);
       if (B >= 2) wmax = fmaxf(wmax, fabsf(X.wbit[1]));
       if (B == 3) wmax = fmaxf(wmax, fmaxf(fabsf(X.wbit[2]), fabsf(X.wpar)));
+      // fixed-point exponent of half h of query q: |value| * 2^F <= 2^22
+      auto fp_exp = [&](int h, int q) {
+        const int i = h * G + q;
+        const float m = fmaxf(fmaxf(sPM[i], sPM[16 + i]), fmaxf(sPM[32 + i], sPM[48 + i]));
+        const float v = h == 0 ? m * wmax : m * 2.f;
+        int e = 0;
+        frexpf(v > 0.f ? v : 1.f, &e);
+        return 22 - e;
+      };
+      int fe[2 * G];
 #pragma unroll
       for (int q = 0; q < G; ++q) {
-        const float vm = sMax[q] * wmax, vq = sMax[G + q] * 2.f;
-        int e1 = 0, e2 = 0;
-        frexpf(vm > 0.f ? vm : 1.f, &e1);
-        frexpf(vq > 0.f ? vq : 1.f, &e2);
-        scale[q] = ldexpf(1.f, 22 - e1);
-        scale[G + q] = ldexpf(1.f, 22 - e2);
+        fe[q] = fp_exp(0, q);
+        fe[G + q] = fp_exp(1, q);
       }
-      // operand bytes: K position kappa (byte t of A column o) of this thread
+      // operand bytes: K position kappa (byte t of A column o) of this thread.  Column
+      // o holds bit t * 8 + (o & 7) of a packed word at bit (o & 7) of each byte, so
+      // the byte is bit * 2^(o & 7); the query value is scaled by 2^(7 - (o & 7)) and
+      // every product carries the common factor 2^7.
 #pragma unroll
       for (int r = 0; r < S::kK / 128; ++r) {
         const int kappa = trow + 128 * r;
         const int o = kappa >> 2, tb = kappa & 3;
+        const int up = 7 - (o & 7);
         int8_t limb[N];
 #pragma unroll
         for (int n = 0; n < N; ++n) limb[n] = 0;
@@ -257,28 +294,16 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
           }
 #pragma unroll
           for (int q = 0; q < G; ++q) {
-            const int v = __float2int_rn(w * qs[q * (kD + kM) + coord] * scale[q]);
-            const int l0 = static_cast<int8_t>(v & 0xff);
-            const int r1 = (v - l0) >> 8;
-            const int l1 = static_cast<int8_t>(r1 & 0xff);
-            const int l2 = (r1 - l1) >> 8;
-            limb[3 * q] = static_cast<int8_t>(l0);
-            limb[3 * q + 1] = static_cast<int8_t>(l1);
-            limb[3 * q + 2] = static_cast<int8_t>(l2);
+            const int v = __float2int_rn(ldexpf(w * qs[q * (kD + kM) + coord], fe[q])) * (1 << up);
+            split_limbs(v, &limb[4 * q]);
           }
         } else {
           const int c = (o - 8 * (S::kCodeWords + S::kParWords)) >> 3, k = o & 7;
           const int j = 32 * c + k + 8 * tb;           // projection
 #pragma unroll
           for (int q = 0; q < G; ++q) {
-            const int v = __float2int_rn(-2.f * qs[q * (kD + kM) + kD + j] * scale[G + q]);
-            const int l0 = static_cast<int8_t>(v & 0xff);
-            const int r1 = (v - l0) >> 8;
-            const int l1 = static_cast<int8_t>(r1 & 0xff);
-            const int l2 = (r1 - l1) >> 8;
-            limb[NG + 3 * q] = static_cast<int8_t>(l0);
-            limb[NG + 3 * q + 1] = static_cast<int8_t>(l1);
-            limb[NG + 3 * q + 2] = static_cast<int8_t>(l2);
+            const int v = __float2int_rn(ldexpf(-2.f * qs[q * (kD + kM) + kD + j], fe[G + q])) * (1 << up);
+            split_limbs(v, &limb[NG + 4 * q]);
           }
         }
         const int kb = kappa >> 7, chunk = (kappa & 127) >> 4, within = kappa & 15;
@@ -286,21 +311,19 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
         for (int n = 0; n < N; ++n)
           sB[kb * (N * 128) + n * 128 + ((chunk ^ (n & 7)) << 4) + within] = static_cast<uint8_t>(limb[n]);
       }
-      // per-query constants: c_const * sum q_rot, sum sq, and the inverse scales
-      named_bar_sync(1 + wg, 128);
+      // per-query constants (c_const * sum q_rot, sum sq) and the inverse scales
+      // with the 2^-7 of the shifted bits
       if (trow < 2 * G) {
-        const int q = trow % G;
-        const bool isq = trow >= G;
-        float acc = 0.f;
-        for (int i2 = 0; i2 < 128; ++i2) acc += qs[q * (kD + kM) + (isq ? kD : 0) + i2];
-        sScal[2 * G + trow] = isq ? acc : X.cconst * acc;
-        sScal[4 * G + trow] = 1.f / scale[trow];
+        const float sum = (sPS[trow] + sPS[16 + trow]) + (sPS[32 + trow] + sPS[48 + trow]);
+        const int h = trow >= G ? 1 : 0;
+        sC[trow] = h ? sum : X.cconst * sum;
+        sInv[trow] = ldexpf(1.f, -fp_exp(h, trow - h * G) - 7);
       }
       fence_proxy_async_smem();
       named_bar_sync(1 + wg, 128);
     }
     // ---- this thread's key from the stage, decoded into TMEM -----------------------
-    if (mbar_wait(&full[stage], parity, kWaitCycles)) {
+    if (mbar_wait(&full[stage], parity, X.wait_cycles)) {
       if (leader) ++consumed;
     } else {
       if (X.err) atomicCAS(X.err, 0, 7);
@@ -333,7 +356,7 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
       for (int c = 0; c < S::kCodeWords + S::kParWords + 4; ++c) {
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          a[n++] = (cw[c] >> k) & 0x01010101u;
+          a[n++] = cw[c] & (0x01010101u << k);
           if (n == 32) {
             tmem_st32(t_a + col, a);
             col += 32;
@@ -359,7 +382,7 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
       }
       mma_commit(&mdone[wg]);
     }
-    if (!mbar_wait(&mdone[wg], static_cast<uint32_t>(i & 1), kWaitCycles)) {
+    if (!mbar_wait(&mdone[wg], static_cast<uint32_t>(i & 1), X.wait_cycles)) {
       if (X.err) atomicCAS(X.err, 0, 6);
       atomicExch(abort_flag, 1);
     }
@@ -379,14 +402,14 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
     tc_fence_before();
     if (valid) {
       float* o = out + set * G * n_keys + key;
+      const float* sC = sScal + 128;
+      const float* sInv = sScal + 144;
 #pragma unroll
       for (int q = 0; q < G; ++q) {
-        const int mse_i = static_cast<int>(acc[3 * q]) + (static_cast<int>(acc[3 * q + 1]) << 8) +
-                          (static_cast<int>(acc[3 * q + 2]) << 16);
-        const int qjl_i = static_cast<int>(acc[NG + 3 * q]) + (static_cast<int>(acc[NG + 3 * q + 1]) << 8) +
-                          (static_cast<int>(acc[NG + 3 * q + 2]) << 16);
-        const float mse = fmaf(static_cast<float>(mse_i), sScal[4 * G + q], sScal[2 * G + q]);
-        const float qjl = fmaf(static_cast<float>(qjl_i), sScal[4 * G + G + q], sScal[2 * G + G + q]);
+        const float mse_f = join_limbs(&acc[4 * q]);
+        const float qjl_f = join_limbs(&acc[NG + 4 * q]);
+        const float mse = fmaf(mse_f, sInv[q], sC[q]);
+        const float qjl = fmaf(qjl_f, sInv[G + q], sC[G + q]);
         o[q * n_keys] = fmaf(nrm, mse, rn * qjl);
       }
     }
@@ -397,7 +420,7 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
     // copies still in flight (only after an abort): let them land before exit
     for (; consumed < issued; ++consumed) {
       const int64_t j = consumed;
-      if (!mbar_wait(&full[j % kStages], static_cast<uint32_t>((j / kStages) & 1), kWaitCycles)) break;
+      if (!mbar_wait(&full[j % kStages], static_cast<uint32_t>((j / kStages) & 1), X.wait_cycles)) break;
     }
   }
   __syncthreads();
@@ -432,7 +455,7 @@ double odd_fit3(const float* c, double a[4]) {
 template <int B, int G>
 int launch_G(const tq_ctx& ctx, const float* qp, int64_t n_sets, int64_t n_keys, const Packed& keys, float* out,
              cudaStream_t s) {
-  constexpr int NG = (3 * G <= 16) ? 16 : 32;
+  constexpr int NG = (4 * G <= 16) ? 16 : 32;
   using Sh = Shape<B>;
   constexpr int kWG = Sh::kWG;
   const KParams& P = ctx.kp;
@@ -457,8 +480,9 @@ int launch_G(const tq_ctx& ctx, const float* qp, int64_t n_sets, int64_t n_keys,
     X.cconst = -P.c[1];
   }
   X.err = P.err;
+  X.wait_cycles = wait_limit_cycles();
   const size_t smem = 1024 + static_cast<size_t>(kWG) * (Sh::kKBlocks * (2 * NG) * 128 + kStages * Sh::kStageBytes) +
-                      kWG * 64 * 4 + (kWG * kStages + kWG) * 8 + 16;
+                      kWG * kScalFloats * 4 + (kWG * kStages + kWG) * 8 + 16;
   cudaError_t e = cudaFuncSetAttribute(k_logits_d128_i8<B, G, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return static_cast<int>(e);
@@ -493,7 +517,7 @@ bool logits_d128_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_key
         ctx.use_tc))
     return false;
   // the A operand and the accumulator share a warpgroup's TMEM columns
-  const int a_cols = 8 * (P.B * 4 + (P.B == 3 ? 4 : 0) + 4), n_cols = (3 * g <= 16) ? 32 : 64;
+  const int a_cols = 8 * (P.B * 4 + (P.B == 3 ? 4 : 0) + 4), n_cols = (4 * g <= 16) ? 32 : 64;
   const int cols = P.B == 3 ? 256 : 128;
   if (a_cols + n_cols > cols) return false;
   if (P.B == 3) {                       // the bit-plane form needs a symmetric codebook

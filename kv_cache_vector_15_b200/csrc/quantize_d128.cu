@@ -9,19 +9,19 @@
 //                                             "Stage 1: PolarQuant" (Lloyd-Max)
 //   bit_j = [ (S r)_j < 0 ], rnorm = n ||r||    Qiita explainer, "Stage 2: QJL"
 //
-// CTA layout (persistent, one CTA per SM): two pairs of warpgroups, each pair
-// on one 128-row tile at a time; thread t of warp w in half h of a pair owns
-// coordinates [64h, 64h + 64) (and projections [64h, 64h + 64)) of row
-// 32 (w % 4) + t, which is also the row's TMEM lane, so tensor-core results
-// come back to the threads that own the row.  Rows arrive by TMA, a tile or
-// two ahead.  Two kernels:
-//   k_quantize_d128_rot_tc  bf16 rows: the rotation itself is an MMA whose A
-//                           operand is the TMA stage and B = D H (+-1), then
-//                           codes / residual on the CUDA cores, then the
-//                           projection MMA;
-//   k_quantize_d128_tc      fp32 rows: the rotation in registers (five FWHT
-//                           stages, the stride-64 stage through the TMEM lane),
-//                           then the same codes and projection MMA.
+// Two kernels, persistent (one CTA per SM), rows arriving by TMA:
+//   k_quantize_d128_ws  bf16 rows, warp-specialized: sixteen compute warps
+//                       share each 128-row tile (four threads per row, 32
+//                       coordinates each, the row in its TMEM lane) and a
+//                       seventeenth warp issues the TMA loads and the
+//                       tensor-core work: the rotation itself as an MMA
+//                       (A = the TMA stage, B = D H as bf16 +-1) and the
+//                       projection MMA, into four rotating TMEM regions so
+//                       both run under the CUDA-core work on the tile before;
+//   k_quantize_d128_tc  fp32 rows: two pairs of warpgroups, the rotation in
+//                       registers (five FWHT stages, the stride-64 stage
+//                       through the TMEM lane), then the same codes and
+//                       projection MMA.
 //
 // Projection precision: S is binary16 by definition (exact in the MMA).  The
 // residual, scaled by 64, is split r = hi + lo into two binary16 parts
@@ -31,7 +31,12 @@
 // with eps_scale = 16 * 2^-22 * max_j ||S_j||_2 (the split's 2^-22 plus 16
 // accumulation steps of at most 2^-23 each, with margin) and eps_abs =
 // max_j ||S_j||_1 * 2^-25 / 64 (binary16 underflow); the rare projections
-// below it are recomputed in fp32 on the CUDA cores from hi + lo.
+// below it are recomputed: by the fp32 kernel in fp32 on the CUDA cores from
+// hi + lo, and for the bf16 kernel in fp64 from the input row by the fix-up
+// kernel that runs after it.  The bf16 kernel splits r by Veltkamp's method
+// (hi = r rounded to 11 bits, lo = r - hi exactly, both then binary16), which
+// keeps the same bound, and decides each code bit from the sign of T^2 - y^2
+// computed with one rounding (the threshold moves by at most about one ulp).
 //
 // Every mbarrier wait is bounded (about one second); a wait that runs out
 // sets the context's error word, the CTA stops issuing work, waits for its
@@ -579,6 +584,83 @@ __device__ __forceinline__ float quant_coord(float y, const float* T, const uint
   return __uint_as_float(__float_as_uint(rm) ^ (~__float_as_uint(sp) & 0x80000000u));
 }
 
+// Two coordinates at once (e0 and e1 = e0 + 1, stream positions POS0 = B e0
+// and POS0 + B) with packed fp32 arithmetic.  Decisions are the signs of
+// T^2 - y^2 (one rounding, so a decision can differ from the exact one only
+// for |y| within about one ulp of a threshold), the code bits are pushed
+// from the highest stream position down, and the residual x 64 comes back
+// as y sc - (+-64 c[L/2 + k]) in one packed FMA.  T2: squared magnitude
+// thresholds; nc: -64 c[L/2 + k] as fp32 bits.
+__device__ __forceinline__ uint32_t sel_neg(uint32_t m, uint32_t a, uint32_t b) {   // m all-ones: a, else b
+  return (m & a) | (~m & b);
+}
+__device__ __forceinline__ uint32_t sign_mask(float v) {
+  return static_cast<uint32_t>(static_cast<int>(__float_as_uint(v)) >> 31);
+}
+template <int B>
+__device__ __forceinline__ float2 quant_pair(float y0, float y1, const float* T2, const uint32_t* nc, float sc,
+                                             uint32_t* cw, const int POS0) {
+  const float2 y = make_float2(y0, y1);
+  const float2 sp = __ffma2_rn(y, make_float2(-1.f, -1.f), make_float2(0.f, 0.f));   // negative iff y > 0
+  const int P1 = POS0 + B;
+  auto push = [&](int pos, float v) { cw[pos >> 5] = __funnelshift_l(__float_as_uint(v), cw[pos >> 5], 1); };
+  uint32_t n0, n1;                                         // -64 c[L/2 + k] of each coordinate
+  if constexpr (B == 1) {
+    push(P1, sp.y);
+    push(POS0, sp.x);
+    n0 = n1 = nc[0];
+  } else if constexpr (B == 2) {
+    const float2 d = __ffma2_rn(sp, y, make_float2(T2[0], T2[0]));
+    push(P1 + 1, sp.y); push(P1, d.y);
+    push(POS0 + 1, sp.x); push(POS0, d.x);
+    // k = [d < 0] as 0.0 / 1.0 (|d| is 0 or far above 2^-126 for any row above
+    // the zero-norm cut), then -64 c[L/2 + k] = k (-c1) + (1 - k) (-c0) with one
+    // of the two terms exactly zero, so the centroid is exact
+    const float2 kk = make_float2(__saturatef(d.x * -8.507059e37f), __saturatef(d.y * -8.507059e37f));
+    const float c0 = __uint_as_float(nc[0]), c1 = __uint_as_float(nc[1]);
+    const float2 lo = __ffma2_rn(kk, make_float2(-c0, -c0), make_float2(c0, c0));
+    const float2 nv = __ffma2_rn(kk, make_float2(c1, c1), lo);
+    n0 = __float_as_uint(nv.x);
+    n1 = __float_as_uint(nv.y);
+  } else if constexpr (B == 3) {
+    const float2 d2 = __ffma2_rn(sp, y, make_float2(T2[1], T2[1]));
+    const uint32_t m2a = sign_mask(d2.x), m2b = sign_mask(d2.y);
+    const uint32_t t2 = __float_as_uint(T2[2]), t0 = __float_as_uint(T2[0]);
+    const float2 d0 = __ffma2_rn(sp, y, make_float2(__uint_as_float(sel_neg(m2a, t2, t0)),
+                                                    __uint_as_float(sel_neg(m2b, t2, t0))));
+    push(P1 + 2, sp.y); push(P1 + 1, d2.y); push(P1, d0.y);
+    push(POS0 + 2, sp.x); push(POS0 + 1, d2.x); push(POS0, d0.x);
+    n0 = sel_neg(sign_mask(d0.x), sel_neg(m2a, nc[3], nc[1]), sel_neg(m2a, nc[2], nc[0]));
+    n1 = sel_neg(sign_mask(d0.y), sel_neg(m2b, nc[3], nc[1]), sel_neg(m2b, nc[2], nc[0]));
+  } else {
+    // three magnitude bits: T[3], then T[1] / T[5], then T[0..6 even]
+    const float2 d2 = __ffma2_rn(sp, y, make_float2(T2[3], T2[3]));
+    const uint32_t m2a = sign_mask(d2.x), m2b = sign_mask(d2.y);
+    const uint32_t t5 = __float_as_uint(T2[5]), t1 = __float_as_uint(T2[1]);
+    const float2 d1 = __ffma2_rn(sp, y, make_float2(__uint_as_float(sel_neg(m2a, t5, t1)),
+                                                    __uint_as_float(sel_neg(m2b, t5, t1))));
+    const uint32_t m1a = sign_mask(d1.x), m1b = sign_mask(d1.y);
+    const uint32_t t4 = __float_as_uint(T2[4]), t0 = __float_as_uint(T2[0]);
+    const uint32_t t6 = __float_as_uint(T2[6]), t2 = __float_as_uint(T2[2]);
+    const uint32_t ta = sel_neg(m1a, sel_neg(m2a, t6, t2), sel_neg(m2a, t4, t0));
+    const uint32_t tb = sel_neg(m1b, sel_neg(m2b, t6, t2), sel_neg(m2b, t4, t0));
+    const float2 d0 = __ffma2_rn(sp, y, make_float2(__uint_as_float(ta), __uint_as_float(tb)));
+    push(P1 + 3, sp.y); push(P1 + 2, d2.y); push(P1 + 1, d1.y); push(P1, d0.y);
+    push(POS0 + 3, sp.x); push(POS0 + 2, d2.x); push(POS0 + 1, d1.x); push(POS0, d0.x);
+    auto pick = [&](uint32_t m2, uint32_t m1, uint32_t m0) {
+      const uint32_t c0 = sel_neg(m2, nc[4], nc[0]), c1 = sel_neg(m2, nc[5], nc[1]);
+      const uint32_t c2 = sel_neg(m2, nc[6], nc[2]), c3 = sel_neg(m2, nc[7], nc[3]);
+      return sel_neg(m0, sel_neg(m1, c3, c1), sel_neg(m1, c2, c0));
+    };
+    n0 = pick(m2a, m1a, sign_mask(d0.x));
+    n1 = pick(m2b, m1b, sign_mask(d0.y));
+  }
+  // +-64 c: the sign of the cell's centroid follows the code's top bit
+  const uint32_t q0 = n0 ^ (~__float_as_uint(sp.x) & 0x80000000u);
+  const uint32_t q1 = n1 ^ (~__float_as_uint(sp.y) & 0x80000000u);
+  return __ffma2_rn(y, make_float2(sc, sc), make_float2(__uint_as_float(q0), __uint_as_float(q1)));
+}
+
 // Mask of the stream positions p in [32 w, 32 w + 32) with p mod B == j
 // (B in 2..4).
 __device__ __forceinline__ uint32_t residue_mask(int B, int w, int j) {
@@ -611,48 +693,129 @@ __device__ __forceinline__ void complement_negative_codes(uint32_t (&cw)[2 * B])
   }
 }
 
+// Complement the magnitude bits of every negative code (as above) in a run
+// of NW words that starts on a word boundary of the code stream where no code
+// straddles the run's ends (NW = B: 32 coordinates).
+template <int B, int NW>
+__device__ __forceinline__ void complement_negative_codes_run(uint32_t (&cw)[NW]) {
+  if constexpr (B > 1) {
+    uint32_t fix[NW];
+#pragma unroll
+    for (int w = 0; w < NW; ++w) fix[w] = 0u;
+#pragma unroll
+    for (int j = 0; j < B - 1; ++j) {
+      const int o = B - 1 - j;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const uint32_t above = w + 1 < NW ? ~cw[w + 1] : 0u;
+        fix[w] |= __funnelshift_r(~cw[w], above, o) & residue_mask(B, w, j);
+      }
+    }
+#pragma unroll
+    for (int w = 0; w < NW; ++w) cw[w] ^= fix[w];
+  }
+}
+
+// mbarrier phase test that may suspend the thread until the phase completes
+// (or about 20 us pass)
+__device__ __forceinline__ bool try_wait_suspend(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 20000;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// min(|a|, |b|, c) in one three-input minimum
+__device__ __forceinline__ float min3_abs(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(c));
+  return d;
+}
+
+// bf16 rows, warp-specialized.  Sixteen compute warps share every 128-row
+// tile: warp w owns coordinates (and projections) [32 g, 32 g + 32), g = w / 4,
+// of rows 32 (w % 4) .. + 31, each row in the TMEM lane of its index, so the
+// four threads of a row sit in the four warps of one lane quadrant.  A
+// seventeenth warp issues everything asynchronous: the TMA loads of the row
+// tiles (a ring of four stages), the rotation y' = x (D H)^T (A = the TMA
+// stage, B = D H as bf16 +-1, exact products, fp32 sums) and the projection
+// p = (64 r) S^T from the residual's binary16 hi | lo parts (K = 256).
+//
+// TMEM holds four 128-column regions.  Tile k reads y' from region Y(k),
+// writes its residual to Z(k), and gets p back in Y(k); the next tile of the
+// same parity uses the regions the other way round (Y(k + 2) = Z(k)), so the
+// rotation of tile k + 2 runs as soon as the projection of tile k has read
+// its residual, and two tiles are always in flight: the compute warps turn
+// tile k into codes while the tensor cores finish the projection of tile
+// k - 1, whose signs are taken next.  A thread reads and writes the same
+// 32 columns of every region: y' and p of its coordinates / projections and,
+// in Z, the hi parts (16 columns) then the lo parts of its 32 residuals, so
+// no thread ever overwrites a column another thread still has to read.  The
+// projection's K order is hi(0..31) lo(0..31) hi(32..63) ..., and its B
+// operand (S) is addressed to match.
+//
+// Codes, residual and the tensor-core error bound are those of the kernel
+// above; projections inside the bound go to the exact fix-up kernel.
+constexpr int kWsCompute = 16;                 // compute warps
+constexpr int kWsThreads = (kWsCompute + 1) * 32;
+constexpr int kWsStages = 4;                   // row tiles in shared memory
+
+constexpr size_t quant_ws_smem_bytes() {
+  return 1024 + 2 * kSmemS + kWsStages * XStage<true>::kBytes + 2 * 4 * kTile * 4 /*norm partials*/ +
+         2 * 4 * kTile * 4 /*residual partials*/ + 256;
+}
+
 template <int B>
-__global__ void __launch_bounds__(kThreads, 1)
-k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P, const QuantD128Args X,
-                       int64_t n_rows, const Packed out) {
+__global__ void __launch_bounds__(kWsThreads, 1)
+k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, const QuantD128Args X,
+                   int64_t n_rows, const Packed out) {
   constexpr int L = 1 << B;
   constexpr int kStage = XStage<true>::kBytes;                  // 32 KB: two 64-column boxes
-  constexpr int NS = XStage<true>::kStages;                     // two stages per pair
-  constexpr int kH = kD / 2;
   constexpr int kNT = SymConsts<B>::kNT > 0 ? SymConsts<B>::kNT : 1;
   constexpr int kNC = SymConsts<B>::kNC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sS = smem;                                            // projection B operand
+  uint8_t* sS = smem;                                            // projection B operand (S, fp16)
   uint8_t* sHD = smem + kSmemS;                                  // rotation B operand (D H, bf16 +-1)
-  uint8_t* sX = sHD + kSmemS;                                    // [pair][NS] stages
-  float* sN2 = reinterpret_cast<float*>(sX + NS * kPairs * kStage);      // [pair][half][row] partial ||y'||^2
-  float* sR2 = sN2 + kPairs * 2 * kTile;                         // [pair][half][row] partial ||r||^2
-  uint64_t* full = reinterpret_cast<uint64_t*>(sR2 + kPairs * 2 * kTile);   // [pair][2]
-  uint64_t* ydone = full + 2 * kPairs;                           // [pair]
-  uint64_t* mdone = ydone + kPairs;                              // [pair]
-  uint64_t* fdone = mdone + kPairs;                              // [pair] wind-down commit
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fdone + kPairs);
+  uint8_t* stages = sHD + kSmemS;                                // [kWsStages] row tiles
+  float* sN2 = reinterpret_cast<float*>(stages + kWsStages * kStage);   // [2][4][row] partial ||y'||^2
+  float* sR2 = sN2 + 2 * 4 * kTile;                              // [2][4][row] partial ||64 r||^2
+  uint64_t* full = reinterpret_cast<uint64_t*>(sR2 + 2 * 4 * kTile);    // [kWsStages]
+  uint64_t* yrdy = full + kWsStages;                             // [2] rotation done
+  uint64_t* prdy = yrdy + 2;                                     // [2] projection done
+  uint64_t* rrdy = prdy + 2;                                     // [2] residual written (16 arrivals)
+  uint64_t* fdone = rrdy + 2;                                    // wind-down commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fdone + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  int* loads_issued = abort_flag + 1;                            // [pair][stage]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
+  const int64_t n_mine = n_tiles > blockIdx.x ? (n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
   const long long wait_cycles = X.wait_cycles;
   if (tid == 0) {
-    for (int i = 0; i < 2 * kPairs; ++i) mbar_init(&full[i], 1);
-    for (int i = 0; i < kPairs; ++i) { mbar_init(&ydone[i], 1); mbar_init(&mdone[i], 1); mbar_init(&fdone[i], 1); }
+    for (int i = 0; i < kWsStages; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&yrdy[i], 1);
+      mbar_init(&prdy[i], 1);
+      mbar_init(&rrdy[i], kWsCompute);
+    }
+    mbar_init(fdone, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  for (int e = tid; e < kM * 16; e += kThreads) {
+  for (int e = tid; e < kM * 16; e += kWsThreads) {
     const int j = e >> 4, c = e & 15, kb = c >> 3, cc = c & 7;
     const uint4 v = *reinterpret_cast<const uint4*>(P.S + j * kD + c * 8);
     *reinterpret_cast<uint4*>(sS + kb * 16384 + j * 128 + ((cc ^ (j & 7)) << 4)) = v;
   }
   // (D H)[n][k] = H[n][k] D_k = (-1)^popcount(n & k) D_k, as bf16 +-1.0, same swizzled layout
   uint16_t* hd16 = reinterpret_cast<uint16_t*>(sHD);
-  for (int e = tid; e < kD * kD; e += kThreads) {
+  for (int e = tid; e < kD * kD; e += kWsThreads) {
     const int n = e >> 7, k = e & 127;
     const bool neg = ((__popc(n & k) & 1) != 0) != (X.Dsign[k] != 0u);
     const int kb = k >> 6, chunk = (k & 63) >> 3, within = k & 7;
@@ -660,297 +823,275 @@ k_quantize_d128_rot_tc(const __grid_constant__ CUtensorMap tmap, const KParams P
   }
   fence_proxy_async_smem();
   if (warp == 0) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  const int wgi = warp >> 2, pair = wgi >> 1, half = wgi & 1, lb = warp & 3;
-  // the leader issues the pair's MMAs, the loader (a warp of the other half)
-  // its stage loads
-  const bool leader = (half == 0 && lb == 0 && lane == 0);
-  const bool loader = (half == 1 && lb == 0 && lane == 0);
-  const int trow = lb * 32 + lane;
-  const uint32_t lane_base = static_cast<uint32_t>(lb * 32) << 16;
-  // two 128-column regions per pair, alternating roles from tile to tile: the
-  // k-th tile's y' (then its projections) in region k mod 2, its residual
-  // hi | lo in the other, so the next tile's rotation can run into the region
-  // of this tile's residual while this tile's projections are still read
-  const uint32_t t_reg0 = tmem + lane_base + pair * 256;
-  const uint32_t bar_id = 1 + pair;
-  uint8_t* stages = sX + pair * NS * kStage;
-  uint64_t* pfull = full + 2 * pair;
-  float* myN2 = sN2 + (pair * 2 + half) * kTile;
-  const float* otN2 = sN2 + (pair * 2 + (half ^ 1)) * kTile;
-  float* myR2 = sR2 + (pair * 2 + half) * kTile;
-  const float* otR2 = sR2 + (pair * 2 + (half ^ 1)) * kTile;
-  const int64_t t_first = blockIdx.x + static_cast<int64_t>(pair) * gridDim.x;
-  const int64_t t_step = static_cast<int64_t>(kPairs) * gridDim.x;
-  auto issue_load = [&](int64_t tile, int buf) {
-    mbar_arrive_expect_tx(&pfull[buf], kStage);
-#pragma unroll
-    for (int bx = 0; bx < 2; ++bx)
-      tma_load_2d(stages + buf * kStage + bx * (kTile * 128), &tmap, &pfull[buf], bx * 64,
-                  static_cast<int>(tile * kTile));
-  };
-  int issued[2] = {0, 0}, waited[2] = {0, 0};                    // stage loads (loader / leader)
-  bool mma_issued = false;                                       // leader: any MMA of ours in flight
-  if (loader) {
-    prefetch_tmap(&tmap);
-    if (t_first < n_tiles) { issue_load(t_first, 0); ++issued[0]; }
-    if (t_first + t_step < n_tiles) { issue_load(t_first + t_step, 1); ++issued[1]; }
-  }
-
-  // the rotation MMA of this pair's k-th tile (leader only): waits for its
-  // stage; if that wait runs out no MMA is issued and the phase is completed
-  // by hand, so the others reach the abort check
-  auto issue_rotation = [&](int k) {
-    const int b = k & 1;
-    if (!mbar_wait(&pfull[b], (k >> 1) & 1, wait_cycles)) {
-      flag_error(X.err, abort_flag, 2);
-      mbar_arrive(&ydone[pair]);
-      return;
+  // regions of local tile k: Y (y', then p) and Z (residual hi | lo)
+  auto region_y = [](int64_t k) { return static_cast<uint32_t>(2 * (k & 1) + ((k >> 1) & 1)) * 128u; };
+  auto region_z = [](int64_t k) { return static_cast<uint32_t>(2 * (k & 1) + 1 - ((k >> 1) & 1)) * 128u; };
+  // a bounded wait that also gives up once another thread has flagged an
+  // abort; with a limit of a second or so a waiting thread is suspended
+  // between polls (so the waiting warps leave the issue slots to the others),
+  // with a short limit it polls and keeps to the cycle count
+  const bool suspend = wait_cycles >= (1ll << 24);
+  auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!(suspend ? try_wait_suspend(bar, parity) : mbar_try_wait(bar, parity))) {
+      if (*reinterpret_cast<volatile int*>(abort_flag) != 0) return false;
+      if (clock64() - t0 > wait_cycles) return false;
     }
-    ++waited[b];
-    mma_issued = true;
-    tc_fence_after();
-    const uint32_t xbase = smem_u32(stages + b * kStage), hbase = smem_u32(sHD);
-    const uint32_t idesc = idesc_bf16_f32(kTile, kD);
-    const uint32_t d_tmem = tmem + pair * 256 + (k & 1) * 128;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-      mma_f16_ss(d_tmem, smem_desc_sw128(xbase + off, 1024), smem_desc_sw128(hbase + off, 1024), idesc,
-                 kk > 0 ? 1u : 0u);
-    }
-    mma_commit(&ydone[pair]);
+    return true;
   };
-  // each later tile's rotation is issued as soon as the previous tile's
-  // projection has completed (below), so it runs under that tile's sign
-  // extraction and stores
-  if (leader && t_first < n_tiles) issue_rotation(0);
 
-  // magnitude thresholds and centroids of the symmetric codebook (x 64 for
-  // the centroids, as negated fp32 bit patterns)
-  float tpos[kNT];
-  uint32_t ncen[kNC];
+  if (warp == kWsCompute) {
+    // ================================ control warp ================================
+    if (lane == 0) {
+      prefetch_tmap(&tmap);
+      int64_t loads = 0, landed = 0;                             // stage loads issued / waited for
+      bool mma_issued = false;
+      auto tile_of = [&](int64_t k) { return static_cast<int64_t>(blockIdx.x) + k * gridDim.x; };
+      auto issue_load = [&](int64_t k) {
+        const int st = static_cast<int>(k % kWsStages);
+        mbar_arrive_expect_tx(&full[st], kStage);
 #pragma unroll
-  for (int j = 0; j < kNT; ++j) tpos[j] = (B > 1) ? P.t[L / 2 + j] : 0.f;
+        for (int bx = 0; bx < 2; ++bx)
+          tma_load_2d(stages + st * kStage + bx * (kTile * 128), &tmap, &full[st], bx * 64,
+                      static_cast<int>(tile_of(k) * kTile));
+        ++loads;
+      };
+      // rotation of local tile k into Y(k); false if its stage never arrived
+      auto rotate = [&](int64_t k) -> bool {
+        const int st = static_cast<int>(k % kWsStages);
+        if (!wait_or_abort(&full[st], static_cast<uint32_t>((k / kWsStages) & 1))) return false;
+        ++landed;
+        tc_fence_after();
+        const uint32_t xbase = smem_u32(stages + st * kStage), hbase = smem_u32(sHD);
+        const uint32_t idesc = idesc_bf16_f32(kTile, kD);
+        const uint32_t d_tmem = tmem + region_y(k);
 #pragma unroll
-  for (int k = 0; k < kNC; ++k) ncen[k] = __float_as_uint(-kResScale * P.c[L / 2 + k]);
-
-  int mine = 0;
-  for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
-    const uint32_t t_acc = t_reg0 + (mine & 1) * 128;            // y', then the projections
-    const uint32_t t_a = t_reg0 + ((mine + 1) & 1) * 128;         // residual hi | lo
-    if (!mbar_wait(&ydone[pair], mine & 1, wait_cycles)) flag_error(X.err, abort_flag, 5);
-    tc_fence_after();
-    // the stage has been read by this tile's rotation: refill it two tiles ahead
-    if (loader && t + NS * t_step < n_tiles) { issue_load(t + NS * t_step, mine & 1); ++issued[mine & 1]; }
-
-    // ---- the row's ||y'||^2 from both halves' sums of squares -------------------
-    {
-      uint32_t u[kH];
-      tmem_ld32(t_acc + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-      tmem_ld32(t_acc + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-      tmem_wait_ld();
-      float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_f16_ss(d_tmem, smem_desc_sw128(xbase + off, 1024), smem_desc_sw128(hbase + off, 1024), idesc,
+                     kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&yrdy[k & 1]);
+        mma_issued = true;
+        return true;
+      };
+      bool ok = true;
+      for (int64_t k = 0; k < kWsStages && k < n_mine; ++k) issue_load(k);
+      for (int64_t k = 0; k < 2 && k < n_mine && ok; ++k) ok = rotate(k);
+      for (int64_t k = 0; k < n_mine && ok; ++k) {
+        const uint32_t ph = static_cast<uint32_t>((k >> 1) & 1);
+        if (!wait_or_abort(&rrdy[k & 1], ph)) { ok = false; break; }
+        tc_fence_after();
+        // tile k's stage was read by its rotation (the compute warps waited for it)
+        if (k + kWsStages < n_mine) issue_load(k + kWsStages);
+        {
+          const uint32_t sbase = smem_u32(sS);
+          const uint32_t idesc = idesc_f16_f32(kTile, kM);
+          const uint32_t d_tmem = tmem + region_y(k), a_tmem = tmem + region_z(k);
 #pragma unroll
-      for (int k = 0; k < kH; k += 4) {
-        const float2 a = make_float2(__uint_as_float(u[k]), __uint_as_float(u[k + 1]));
-        const float2 b2 = make_float2(__uint_as_float(u[k + 2]), __uint_as_float(u[k + 3]));
-        s0 = __ffma2_rn(a, a, s0);
-        s1 = __ffma2_rn(b2, b2, s1);
+          for (int kk = 0; kk < 16; ++kk) {
+            // A step kk: hi (kk & 2 == 0) or lo parts of coordinates 32 (kk >> 2) + 16 (kk & 1) .. + 15
+            const int sk = 2 * (kk >> 2) + (kk & 1);
+            const uint64_t bdesc = smem_desc_sw128(sbase + (sk >> 2) * 16384 + (sk & 3) * 32, 1024);
+            mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&prdy[k & 1]);
+        }
+        if (k + 2 < n_mine) {
+          // Y(k + 2) = Z(k): free once this projection has read it
+          if (!wait_or_abort(&prdy[k & 1], ph)) { ok = false; break; }
+          ok = rotate(k + 2);
+        }
       }
-      myN2[trow] = (s0.x + s0.y) + (s1.x + s1.y);
+      if (!ok) {
+        if (X.err) atomicCAS(X.err, 0, 2);
+        atomicExch(abort_flag, 1);
+      }
+      // wind-down with the full limit: no MMA of ours still running, no stage load still landing
+      if (mma_issued) {
+        mma_commit(fdone);
+        if (!mbar_wait(fdone, 0, kWaitCycles)) flag_error(X.err, abort_flag, 4);
+      }
+      for (; landed < loads; ++landed)
+        if (!mbar_wait(&full[landed % kWsStages], static_cast<uint32_t>((landed / kWsStages) & 1), kWaitCycles)) {
+          flag_error(X.err, abort_flag, 4);
+          break;
+        }
     }
-    named_bar_sync(bar_id, 256);                                 // #X: both partial sums written
-    const float ss = half == 0 ? myN2[trow] + otN2[trow] : otN2[trow] + myN2[trow];
-    const float nsd = sqrtf(ss);                                 // ||H D x|| = sqrt(d) ||x||
-    const float n = nsd * 0.08838834764831845f;                  // / sqrt(128)
-    const bool zero_row = !(n >= kZeroNorm);
-    const float nsd_t = zero_row ? 1.f : nsd;
-    const float sc = zero_row ? 0.f : kResScale / nsd_t;
-    float T[kNT];
-    uint32_t nc[kNC];
-#pragma unroll
-    for (int j = 0; j < kNT; ++j) T[j] = tpos[j] * nsd_t;
-#pragma unroll
-    for (int k = 0; k < kNC; ++k) nc[k] = zero_row ? 0u : ncen[k];   // a zero row's residual is 0
-
-    // ---- codes and the residual (x 64), hi | lo into TMEM -----------------------
-    // (the 64 values come back from TMEM 32 at a time; coordinates 63 .. 0 in
-    // order, so each packed word receives its bits from the top down)
-    uint32_t cw[B * 2];
-#pragma unroll
-    for (int w = 0; w < B * 2; ++w) cw[w] = 0u;
-    float2 r2a = make_float2(0.f, 0.f), r2b = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int ch = 1; ch >= 0; --ch) {
-      uint32_t u[32];
-      tmem_ld32(t_acc + half * 64 + ch * 32, u);
+  } else {
+    // ================================ compute warps ================================
+    const int quad = warp & 3, g = warp >> 2;
+    const int trow = quad * 32 + lane;
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 32 * g;   // my lane, my columns
+    const int n_k = static_cast<int>(n_mine);
+    // this thread's row of local tile k is row0 + k * row_step (below 2^31:
+    // the kernel takes fewer than 2^31 - 256 rows)
+    const int row0 = static_cast<int>(blockIdx.x) * kTile + trow;
+    const int row_step = static_cast<int>(gridDim.x) * kTile;
+    const int nr = static_cast<int>(n_rows);
+    // the previous tile's row state, for its signs
+    bool prev_zero = true;
+    float prev_n = 0.f;
+    int prev_row = 0;
+    // region offsets of local tile k: Y = 256 (k & 1) + 128 ((k >> 1) & 1), Z = Y ^ 128
+    auto off_y = [](int k) { return static_cast<uint32_t>(((k & 1) << 8) | ((k & 2) << 6)); };
+    // signs of local tile k (its projection), exact recomputation listed within the error bound
+    auto signs = [&](int k) {
+      if (!wait_or_abort(&prdy[k & 1], static_cast<uint32_t>((k >> 1) & 1))) {
+        flag_error(X.err, abort_flag, 3);
+        return;
+      }
+      tc_fence_after();
+      const float* r2 = sR2 + (k & 1) * 4 * kTile + trow;
+      const float rr = (r2[0] + r2[kTile]) + (r2[2 * kTile] + r2[3 * kTile]);
+      const float rho = prev_zero ? 0.f : sqrtf(rr) * (1.0f / kResScale);
+      const float eps = kResScale * fmaf(X.eps_scale, rho, X.eps_abs);
+      uint32_t p[32];
+      tmem_ld32(tbase + off_y(k), p);
       tmem_wait_ld();
+      uint32_t sw = 0u;
+#pragma unroll
+      for (int j = 31; j >= 0; --j) sw = __funnelshift_l(p[j], sw, 1);
+      float pmin = INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) pmin = min3_abs(__uint_as_float(p[j]), __uint_as_float(p[j + 1]), pmin);
+      const int row = prev_row;
+      const bool live = row < nr;
+      if (pmin < eps && !prev_zero && rho != 0.f && live) {
+        // rare: list each projection inside the bound for the fix-up kernel;
+        // a row whose entries do not all fit is marked for a full recomputation
+        uint32_t f = 0u;
+#pragma unroll
+        for (int j = 31; j >= 0; --j) f = (f << 1) | (fabsf(__uint_as_float(p[j])) < eps ? 1u : 0u);
+        unsigned int slot = atomicAdd(X.fix_count, static_cast<unsigned int>(__popc(f)));
+        while (f) {
+          const int j = 32 * g + __ffs(f) - 1;
+          if (slot < X.fix_cap)
+            X.fix_list[slot] = (static_cast<unsigned long long>(row) << 8) | static_cast<unsigned>(j);
+          ++slot;
+          f &= f - 1;
+        }
+        if (slot > X.fix_cap) atomicOr(X.fix_rows + (row >> 5), 1u << (row & 31));
+      }
+      if (prev_zero || rho == 0.f) sw = 0u;
+      if (live) {
+        reinterpret_cast<uint32_t*>(out.signs + static_cast<size_t>(row) * 16)[g] = sw;
+        if (g == 0) out.rnorm[row] = prev_zero ? 0.f : prev_n * rho;
+      }
+    };
+
+    int k = 0;
+    for (; k < n_k; ++k) {
+      const int row = row0 + k * row_step;
+      const uint32_t oy = off_y(k);
+      const bool got = wait_or_abort(&yrdy[k & 1], static_cast<uint32_t>((k >> 1) & 1));
+      if (!got) flag_error(X.err, abort_flag, 5);
+      tc_fence_after();
+      uint32_t u[32];
+      tmem_ld32(tbase + oy, u);
+      tmem_wait_ld();
+      {
+        float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float2 a = make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1]));
+          const float2 b2 = make_float2(__uint_as_float(u[j + 2]), __uint_as_float(u[j + 3]));
+          s0 = __ffma2_rn(a, a, s0);
+          s1 = __ffma2_rn(b2, b2, s1);
+        }
+        sN2[(k & 1) * 4 * kTile + g * kTile + trow] = (s0.x + s0.y) + (s1.x + s1.y);
+      }
+      // all four partial sums of every row written; one abort decision for all
+      if (named_bar_sync_or(1, kWsCompute * 32, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
+      const float* n2 = sN2 + (k & 1) * 4 * kTile + trow;
+      const float ss = (n2[0] + n2[kTile]) + (n2[2 * kTile] + n2[3 * kTile]);
+      const float nsd = sqrtf(ss);                               // ||H D x|| = sqrt(d) ||x||
+      const float n = nsd * 0.08838834764831845f;                // / sqrt(128)
+      const bool zero_row = !(n >= kZeroNorm);
+      const float nsd_t = zero_row ? 1.f : nsd;
+      const float sc = zero_row ? 0.f : kResScale * __frcp_rn(nsd_t);   // = RN(64 / nsd)
+      // squared thresholds and the centroids (x 64, as negated fp32 bit
+      // patterns) straight from the parameter space
+      float T2[kNT];
+      uint32_t nc[kNC];
+#pragma unroll
+      for (int j = 0; j < kNT; ++j) {
+        const float tj = (B > 1 ? P.t[L / 2 + j] : 0.f) * nsd_t;
+        T2[j] = tj * tj;
+      }
+#pragma unroll
+      for (int c = 0; c < kNC; ++c) nc[c] = zero_row ? 0u : __float_as_uint(-kResScale * P.c[L / 2 + c]);
+
+      // ---- codes and the residual (x 64): hi parts to Z + 32 g, lo parts to Z + 32 g + 16 ----
+      uint32_t cw[B];
+#pragma unroll
+      for (int w = 0; w < B; ++w) cw[w] = 0u;
+      float2 r2a = make_float2(0.f, 0.f), r2b = make_float2(0.f, 0.f);
+      const uint32_t zb = tbase + (oy ^ 128u);
 #pragma unroll
       for (int g8 = 1; g8 >= 0; --g8) {                         // 16 coordinates -> 8 hi and 8 lo columns
         uint32_t hw[8], lw[8];
 #pragma unroll
         for (int q = 7; q >= 0; --q) {
-          const int l1 = g8 * 16 + 2 * q + 1, l0 = l1 - 1;        // within the chunk
-          const int e1 = ch * 32 + l1, e0 = e1 - 1;               // within my 64
-          const float r1 = quant_coord<B>(__uint_as_float(u[l1]), T, nc, sc, cw, B * e1);
-          const float r0 = quant_coord<B>(__uint_as_float(u[l0]), T, nc, sc, cw, B * e0);
-          const float2 rv = make_float2(r0, r1);
+          const int e0 = g8 * 16 + 2 * q;
+          const float2 rv = quant_pair<B>(__uint_as_float(u[e0]), __uint_as_float(u[e0 + 1]), T2, nc, sc, cw, B * e0);
           if (q & 1) r2a = __ffma2_rn(rv, rv, r2a); else r2b = __ffma2_rn(rv, rv, r2b);
-          const __half2 h = __floats2half2_rn(r0, r1);
-          const float2 hf = __half22float2(h);
-          const float2 lf = __fadd2_rn(rv, make_float2(-hf.x, -hf.y));
+          // hi = r rounded to 11 significant bits by Veltkamp's split (c = (2^13 + 1) r,
+          // hi = c - (c - r)), exact in binary16 in its normal range; lo = r - hi exactly
+          const float2 c = __fmul2_rn(rv, make_float2(8193.f, 8193.f));
+          const float2 hv = __ffma2_rn(__ffma2_rn(rv, make_float2(-1.f, -1.f), c), make_float2(-1.f, -1.f), c);
+          const float2 lf = __ffma2_rn(hv, make_float2(-1.f, -1.f), rv);
+          const __half2 h = __floats2half2_rn(hv.x, hv.y);
           const __half2 l = __floats2half2_rn(lf.x, lf.y);
           hw[q] = *reinterpret_cast<const uint32_t*>(&h);
           lw[q] = *reinterpret_cast<const uint32_t*>(&l);
         }
-        tmem_st8(t_a + half * 32 + ch * 16 + g8 * 8, hw);
-        tmem_st8(t_a + 64 + half * 32 + ch * 16 + g8 * 8, lw);
+        tmem_st8(zb + g8 * 8, hw);
+        tmem_st8(zb + 16 + g8 * 8, lw);
       }
-    }
-    complement_negative_codes<B>(cw);
-    if (zero_row) {
+      complement_negative_codes_run<B, B>(cw);
+      if (zero_row) {
 #pragma unroll
-      for (int w = 0; w < B * 2; ++w) cw[w] = 0u;
-    }
-    myR2[trow] = (r2a.x + r2a.y) + (r2b.x + r2b.y);
-    tmem_wait_st();
-    tc_fence_before();
-    // #B: A complete and every y' read done (the projection overwrites them);
-    // the abort flag ORed over the pair so that all take the same decision
-    if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
-    const float rho = zero_row ? 0.f : sqrtf(half == 0 ? myR2[trow] + otR2[trow] : otR2[trow] + myR2[trow]) *
-                                           (1.0f / kResScale);
-    if (leader) {
-      tc_fence_after();
-      const uint32_t sbase = smem_u32(sS);
-      const uint32_t idesc = idesc_f16_f32(kTile, kM);
-      const uint32_t d_tmem = tmem + pair * 256 + (mine & 1) * 128;
-      const uint32_t a_tmem = tmem + pair * 256 + ((mine + 1) & 1) * 128;
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int kk = k & 7;
-        const uint64_t bdesc = smem_desc_sw128(sbase + (kk >> 2) * 16384 + (kk & 3) * 32, 1024);
-        mma_f16_ts(d_tmem, a_tmem + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
+        for (int w = 0; w < B; ++w) cw[w] = 0u;
       }
-      mma_commit(&mdone[pair]);
-      mma_issued = true;
-    }
-    if (!mbar_wait(&mdone[pair], mine & 1, wait_cycles)) flag_error(X.err, abort_flag, 3);
-    tc_fence_after();
-    // the projection has read this tile's residual region: the next tile's
-    // rotation may write it
-    if (leader && t + t_step < n_tiles && *reinterpret_cast<volatile int*>(abort_flag) == 0) issue_rotation(mine + 1);
-
-    // ---- my 64 signs, exact recomputation within the error bound of zero ------------
-    const float eps = kResScale * fmaf(X.eps_scale, rho, X.eps_abs);
-    uint32_t s0 = 0, s1 = 0;
-    float pmin = INFINITY;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      uint32_t p[32];
-      tmem_ld32(t_acc + half * 64 + hh * 32, p);
-      tmem_wait_ld();
-      uint32_t sw = 0u;
-#pragma unroll
-      for (int j = 31; j >= 0; --j) sw = __funnelshift_l(p[j], sw, 1);
-      if (hh == 0) s0 = sw; else s1 = sw;
-#pragma unroll
-      for (int j = 0; j < 32; j += 2)
-        pmin = fminf(pmin, fminf(fabsf(__uint_as_float(p[j])), fabsf(__uint_as_float(p[j + 1]))));
-    }
-    // rare: projections inside the bound.  They are listed for the exact
-    // fix-up kernel that runs after this one (this tile's residual region is
-    // already being overwritten by the next tile's rotation); the tensor-core
-    // signs stay in place until then.  The TMEM loads are warp-collective, so
-    // the whole warp reloads when any lane needs it.
-    const int64_t row = t * kTile + trow;
-    const bool mine_flagged = pmin < eps && !zero_row && rho != 0.f && row < n_rows;
-    if (__any_sync(0xffffffffu, mine_flagged)) {
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t p[32];
-        tmem_ld32(t_acc + half * 64 + hh * 32, p);
-        tmem_wait_ld();
-        if (mine_flagged) {
-          uint32_t f = 0u;
-#pragma unroll
-          for (int j = 31; j >= 0; --j) f = (f << 1) | (fabsf(__uint_as_float(p[j])) < eps ? 1u : 0u);
-          const unsigned int nf = __popc(f);
-          unsigned int slot = nf ? atomicAdd(X.fix_count, nf) : 0u;
-          // every claimed slot below the capacity is written; a row with an
-          // entry beyond it is marked for the recomputation of all its signs
-          while (f) {
-            const int j = half * 64 + hh * 32 + __ffs(f) - 1;
-            if (slot < X.fix_cap)
-              X.fix_list[slot] = (static_cast<unsigned long long>(row) << 8) | static_cast<unsigned>(j);
-            ++slot;
-            f &= f - 1;
-          }
-          if (slot > X.fix_cap) atomicOr(X.fix_rows + (row >> 5), 1u << (row & 31));
-        }
-      }
-    }
-    if (zero_row || rho == 0.f) s0 = s1 = 0u;
-    tc_fence_before();
-    // #A: every read of this tile's accumulator and operand columns is done
-    // (and a uniform abort check): the next tile's rotation may start
-    if (named_bar_sync_or(bar_id, 256, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
-    if (row < n_rows) {
-      uint32_t* co = reinterpret_cast<uint32_t*>(out.codes + row * (B * 16) + half * (B * 8));
-      if constexpr (B == 1) {
-        *reinterpret_cast<uint2*>(co) = make_uint2(cw[0], cw[1]);
-      } else if constexpr (B == 2) {
-        *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      } else if constexpr (B == 3) {
-        if (half == 0) {
-          *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-          *reinterpret_cast<uint2*>(co + 4) = make_uint2(cw[4], cw[5]);
-        } else {
+      sR2[(k & 1) * 4 * kTile + g * kTile + trow] = (r2a.x + r2a.y) + (r2b.x + r2b.y);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rrdy[k & 1]);
+      if (row < nr) {
+        uint32_t* co = reinterpret_cast<uint32_t*>(out.codes + static_cast<size_t>(row) * (B * 16)) + B * g;
+        if constexpr (B == 1) {
+          co[0] = cw[0];
+        } else if constexpr (B == 2) {
           *reinterpret_cast<uint2*>(co) = make_uint2(cw[0], cw[1]);
-          *reinterpret_cast<uint4*>(co + 2) = make_uint4(cw[2], cw[3], cw[4], cw[5]);
+        } else if constexpr (B == 3) {
+          co[0] = cw[0]; co[1] = cw[1]; co[2] = cw[2];
+        } else {
+          *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
         }
-      } else {
-        *reinterpret_cast<uint4*>(co) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        *reinterpret_cast<uint4*>(co + 4) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        if (g == 0) out.norm[row] = zero_row ? 0.f : n;
       }
-      *reinterpret_cast<uint2*>(out.signs + row * 16 + half * 8) = make_uint2(s0, s1);
-      if (half == 0) {
-        out.norm[row] = zero_row ? 0.f : n;
-        out.rnorm[row] = zero_row ? 0.f : n * rho;
-      }
+      // the previous tile's signs, while this tile's projection runs
+      if (k > 0) signs(k - 1);
+      prev_zero = zero_row;
+      prev_n = n;
+      prev_row = row;
     }
-  }
-  // Wind-down, with the full wait limit whatever limit the loop ran with: no
-  // MMA of ours may still be running and no stage load still landing when the
-  // TMEM and the shared memory are released.  One more commit tracks every
-  // MMA this thread has issued.
-  if (leader && mma_issued) {
-    mma_commit(&fdone[pair]);
-    if (!mbar_wait(&fdone[pair], 0, kWaitCycles)) flag_error(X.err, abort_flag, 4);
-  }
-  if (loader) { loads_issued[2 * pair] = issued[0]; loads_issued[2 * pair + 1] = issued[1]; }
-  __syncthreads();
-  if (leader) {
-    issued[0] = loads_issued[2 * pair];
-    issued[1] = loads_issued[2 * pair + 1];
-    for (int b2 = 0; b2 < 2; ++b2)
-      while (waited[b2] < issued[b2]) {
-        if (!mbar_wait(&pfull[b2], waited[b2] & 1, kWaitCycles)) { flag_error(X.err, abort_flag, 4); break; }
-        ++waited[b2];
-      }
+    if (k == n_k && n_k > 0) signs(n_k - 1);
   }
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -1079,10 +1220,6 @@ k_qjl_fixup_d128(const KParams P, const void* __restrict__ x, int64_t ld, int64_
 // -------------------------------------------------------------------------- host
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() { return tensor_map_encoder(); }
 
-constexpr size_t quant_rot_smem_bytes() {
-  return 1024 + 2 * kSmemS + 2 * kPairs * XStage<true>::kBytes + 2 * kPairs * 2 * kTile * 4 + 256;
-}
-
 // The bf16 kernel's fix-up scratch in the caller's workspace: the overflow
 // bitmap (one bit per row), the list counter (both zeroed before each
 // launch), then the list.  Two entries per tile is about three times what the
@@ -1131,11 +1268,11 @@ int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, cons
     X.fix_cap = static_cast<unsigned int>(forced > 0 && forced < cap ? forced : cap);
     cudaError_t e = cudaMemsetAsync(sc, 0, fix_bitmap_bytes(n_rows) + 256, s);
     if (e != cudaSuccess) return static_cast<int>(e);
-    const size_t smem = quant_rot_smem_bytes();
-    e = cudaFuncSetAttribute(k_quantize_d128_rot_tc<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const size_t smem = quant_ws_smem_bytes();
+    e = cudaFuncSetAttribute(k_quantize_d128_ws<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
-    k_quantize_d128_rot_tc<B><<<grid, kThreads, smem, s>>>(tmap, P, X, n_rows, out);
+    k_quantize_d128_ws<B><<<grid, kWsThreads, smem, s>>>(tmap, P, X, n_rows, out);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return static_cast<int>(e);
     k_qjl_fixup_d128<B, true><<<ctx.num_sms * 8, 256, 0, s>>>(P, x, ld, n_rows, out, X.fix_list, X.fix_count,
@@ -1161,7 +1298,7 @@ size_t quantize_d128_scratch_bytes(const tq_ctx& ctx, int64_t n_rows) {
 bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows) {
   if (ctx.d_in != ctx.d) return false;                   // padded rows use the general kernel
   const KParams& P = ctx.kp;
-  return P.d == kD && P.m == kM && P.B >= 1 && P.B <= 4 && n_rows > 0 && n_rows < (int64_t(1) << 31) &&
+  return P.d == kD && P.m == kM && P.B >= 1 && P.B <= 4 && n_rows > 0 && n_rows < (int64_t(1) << 31) - 256 &&
          ctx.use_tc && get_encode() != nullptr;
 }
 

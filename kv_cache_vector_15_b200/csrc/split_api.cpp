@@ -17,6 +17,7 @@
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <new>
 #include <string>
@@ -85,8 +86,14 @@ tq_status tq_split_part(const tq_split* sp, int part, const tq_ctx** out) {
   return TQ_OK;
 }
 
+size_t tq_split_quantize_workspace_bytes(const tq_split* sp, int64_t n_rows) {
+  if (!sp || n_rows <= 0) return 0;
+  return std::max(tq_quantize_workspace_bytes(sp->part[0], n_rows), tq_quantize_workspace_bytes(sp->part[1], n_rows));
+}
+
 tq_status tq_split_quantize(const tq_split* sp, const void* x, tq_dtype x_dtype, int64_t n_rows, int64_t ld_x,
-                            tq_packed out_hi, tq_packed out_lo, void* stream) {
+                            tq_packed out_hi, tq_packed out_lo, void* workspace, size_t workspace_bytes,
+                            void* stream) {
   tq_status st = check_split(sp);
   if (st != TQ_OK) return st;
   if (x_dtype != TQ_BF16 && x_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "x_dtype must be TQ_BF16 or TQ_F32");
@@ -95,10 +102,17 @@ tq_status tq_split_quantize(const tq_split* sp, const void* x, tq_dtype x_dtype,
   for (int p = 0; p < 2; ++p)
     if ((st = check_ctx(sp->part[p])) != TQ_OK) return st;
   if (n_rows == 0) return TQ_OK;
-  // each part on its own kernels (no workspace: a wide part takes the general path)
-  if ((st = quantize_checked(sp->part[0], x, x_dtype, n_rows, ld_x, out_hi, nullptr, stream)) != TQ_OK) return st;
+  const size_t need = tq_split_quantize_workspace_bytes(sp, n_rows);
+  if (need) {
+    if (!workspace || workspace_bytes < need) return fail(TQ_ERR_INVALID_ARG, "workspace missing or too small");
+    if (reinterpret_cast<uintptr_t>(workspace) & 15) return fail(TQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  }
+  // the parts in turn on the caller's stream, each with the workspace its kernels need
+  void* w[2];
+  for (int p = 0; p < 2; ++p) w[p] = tq_quantize_workspace_bytes(sp->part[p], n_rows) ? workspace : nullptr;
+  if ((st = quantize_checked(sp->part[0], x, x_dtype, n_rows, ld_x, out_hi, w[0], stream)) != TQ_OK) return st;
   const void* x_lo = x ? static_cast<const uint8_t*>(x) + static_cast<size_t>(sp->d_hi) * esize(x_dtype) : nullptr;
-  return quantize_checked(sp->part[1], x_lo, x_dtype, n_rows, ld_x, out_lo, nullptr, stream);
+  return quantize_checked(sp->part[1], x_lo, x_dtype, n_rows, ld_x, out_lo, w[1], stream);
 }
 
 size_t tq_split_logits_workspace_bytes(const tq_split* sp, int64_t n_sets, int g, int64_t n_keys) {

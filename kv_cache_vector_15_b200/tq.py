@@ -33,7 +33,8 @@ SYMBOLS = [
     "tq_quantize", "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_dequant", "tq_topk", "tq_logits_bf16",
     "tq_status_str", "tq_sync_status", "tq_last_error", "tq_launch_count", "tq_attention_workspace_bytes",
     "tq_attention", "tq_quantize_scatter", "tq_search_workspace_bytes", "tq_search", "tq_split_init",
-    "tq_split_destroy", "tq_split_part", "tq_split_quantize", "tq_split_logits_workspace_bytes", "tq_split_logits",
+    "tq_split_destroy", "tq_split_part", "tq_split_quantize_workspace_bytes", "tq_split_quantize",
+    "tq_split_logits_workspace_bytes", "tq_split_logits",
     "tq_split_dequant", "tq_test_set",
 ]
 
@@ -65,7 +66,8 @@ _sig = {
     "tq_split_init": (_i32, [_i32, _i32, _i32, _i32, _u64, ctypes.POINTER(_vp)]),
     "tq_split_destroy": (_i32, [_vp]),
     "tq_split_part": (_i32, [_vp, _i32, ctypes.POINTER(_vp)]),
-    "tq_split_quantize": (_i32, [_vp, _vp, _i32, _i64, _i64, _Packed, _Packed, _vp]),
+    "tq_split_quantize_workspace_bytes": (_sz, [_vp, _i64]),
+    "tq_split_quantize": (_i32, [_vp, _vp, _i32, _i64, _i64, _Packed, _Packed, _vp, _sz, _vp]),
     "tq_split_logits_workspace_bytes": (_sz, [_vp, _i64, _i32, _i64]),
     "tq_split_logits": (_i32, [_vp, _vp, _i32, _i64, _i32, _Packed, _Packed, _i64, _vp, _vp, _sz, _vp]),
     "tq_split_dequant": (_i32, [_vp, _Packed, _Packed, _i64, _vp, _i32, _i32, _vp]),
@@ -388,12 +390,21 @@ class TurboQuantSplit:
                             torch.empty((n_rows,), dtype=torch.float32, device=device),
                             torch.empty((n_rows,), dtype=torch.float32, device=device)) for cb, sb in self._sizes)
 
-    def quantize(self, x, out=None, stream=None):
+    def quantize_workspace_bytes(self, n_rows: int) -> int:
+        return int(_lib.tq_split_quantize_workspace_bytes(self._h, n_rows))
+
+    def quantize(self, x, out=None, workspace=None, stream=None):
+        import torch
         assert x.dim() == 2 and x.stride(1) == 1
+        n = x.shape[0]
         if out is None:
-            out = self.empty_packed(x.shape[0], x.device)
-        _check(_lib.tq_split_quantize(self._h, _ptr(x), _dtype_code(x), x.shape[0], x.stride(0), out[0].c(),
-                                      out[1].c(), _stream(stream)), "tq_split_quantize")
+            out = self.empty_packed(n, x.device)
+        need = self.quantize_workspace_bytes(n)
+        if need and workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+        wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        _check(_lib.tq_split_quantize(self._h, _ptr(x), _dtype_code(x), n, x.stride(0), out[0].c(), out[1].c(),
+                                      _ptr(workspace), wbytes, _stream(stream)), "tq_split_quantize")
         return out
 
     def logits(self, q, keys, n_sets: int, g: int, n_keys: int, out=None, workspace=None, stream=None):

@@ -86,7 +86,8 @@ def test_host_calls_validate_before_any_launch():
     assert tq.call_status("tq_search", None, None, 0, 64, P, 4096, 10, None, None, None, 0,
                           None) == tq.TQ_ERR_INVALID_ARG
     assert tq._lib.tq_search_workspace_bytes(None, 64, 4096, 10) == 0
-    assert tq.call_status("tq_split_quantize", None, None, 0, 10, 128, P, P, None) == tq.TQ_ERR_INVALID_ARG
+    assert tq.call_status("tq_split_quantize", None, None, 0, 10, 128, P, P, None, 0, None) == tq.TQ_ERR_INVALID_ARG
+    assert tq._lib.tq_split_quantize_workspace_bytes(None, 10) == 0
     assert tq.call_status("tq_split_logits", None, None, 0, 1, 4, P, P, 10, None, None, 0,
                           None) == tq.TQ_ERR_INVALID_ARG
     assert tq.call_status("tq_split_dequant", None, P, P, 10, None, 0, 0, None) == tq.TQ_ERR_INVALID_ARG
