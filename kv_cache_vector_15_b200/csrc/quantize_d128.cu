@@ -767,7 +767,7 @@ constexpr int kWsStages = 4;                   // row tiles in shared memory
 
 constexpr size_t quant_ws_smem_bytes() {
   return 1024 + 2 * kSmemS + kWsStages * XStage<true>::kBytes + 2 * 4 * kTile * 4 /*norm partials*/ +
-         2 * 4 * kTile * 4 /*residual partials*/ + 256;
+         2 * 4 * kTile * 4 /*residual partials*/ + 2 * kWsCompute * 32 * 4 /*norms*/ + 256;
 }
 
 template <int B>
@@ -785,11 +785,13 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
   uint8_t* stages = sHD + kSmemS;                                // [kWsStages] row tiles
   float* sN2 = reinterpret_cast<float*>(stages + kWsStages * kStage);   // [2][4][row] partial ||y'||^2
   float* sR2 = sN2 + 2 * 4 * kTile;                              // [2][4][row] partial ||64 r||^2
-  uint64_t* full = reinterpret_cast<uint64_t*>(sR2 + 2 * 4 * kTile);    // [kWsStages]
+  float* sNrm = sR2 + 2 * 4 * kTile;                             // [2][compute thread] norms awaiting signs
+  uint64_t* full = reinterpret_cast<uint64_t*>(sNrm + 2 * kWsCompute * 32);   // [kWsStages]
   uint64_t* yrdy = full + kWsStages;                             // [2] rotation done
   uint64_t* prdy = yrdy + 2;                                     // [2] projection done
   uint64_t* rrdy = prdy + 2;                                     // [2] residual written (16 arrivals)
-  uint64_t* fdone = rrdy + 2;                                    // wind-down commit
+  uint64_t* nrdy = rrdy + 2;                                     // [2] norm partials written (16 arrivals)
+  uint64_t* fdone = nrdy + 2;                                    // wind-down commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fdone + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -803,6 +805,7 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
       mbar_init(&yrdy[i], 1);
       mbar_init(&prdy[i], 1);
       mbar_init(&rrdy[i], kWsCompute);
+      mbar_init(&nrdy[i], kWsCompute);
     }
     mbar_init(fdone, 1);
     *abort_flag = 0;
@@ -937,22 +940,25 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
     const int row0 = static_cast<int>(blockIdx.x) * kTile + trow;
     const int row_step = static_cast<int>(gridDim.x) * kTile;
     const int nr = static_cast<int>(n_rows);
-    // the previous tile's row state, for its signs
-    bool prev_zero = true;
-    float prev_n = 0.f;
-    int prev_row = 0;
+    // each tile's norm (0 for a zero row) waits in shared memory for its signs
+    float* my_norm = sNrm + tid;                                 // [2][512]
     // region offsets of local tile k: Y = 256 (k & 1) + 128 ((k >> 1) & 1), Z = Y ^ 128
     auto off_y = [](int k) { return static_cast<uint32_t>(((k & 1) << 8) | ((k & 2) << 6)); };
+    // the sum of the four partial ||64 r||^2 of tile k (written before rrdy(k))
+    auto resid2 = [&](int k) {
+      const float* r2 = sR2 + (k & 1) * 4 * kTile + trow;
+      return (r2[0] + r2[kTile]) + (r2[2 * kTile] + r2[3 * kTile]);
+    };
     // signs of local tile k (its projection), exact recomputation listed within the error bound
-    auto signs = [&](int k) {
+    auto signs = [&](int k, float rr) {
       if (!wait_or_abort(&prdy[k & 1], static_cast<uint32_t>((k >> 1) & 1))) {
         flag_error(X.err, abort_flag, 3);
         return;
       }
       tc_fence_after();
-      const float* r2 = sR2 + (k & 1) * 4 * kTile + trow;
-      const float rr = (r2[0] + r2[kTile]) + (r2[2 * kTile] + r2[3 * kTile]);
-      const float rho = prev_zero ? 0.f : sqrtf(rr) * (1.0f / kResScale);
+      const float nk = my_norm[(k & 1) * 512];
+      const bool zero = nk == 0.f;
+      const float rho = zero ? 0.f : sqrtf(rr) * (1.0f / kResScale);
       const float eps = kResScale * fmaf(X.eps_scale, rho, X.eps_abs);
       uint32_t p[32];
       tmem_ld32(tbase + off_y(k), p);
@@ -963,9 +969,9 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
       float pmin = INFINITY;
 #pragma unroll
       for (int j = 0; j < 32; j += 2) pmin = min3_abs(__uint_as_float(p[j]), __uint_as_float(p[j + 1]), pmin);
-      const int row = prev_row;
+      const int row = row0 + k * row_step;
       const bool live = row < nr;
-      if (pmin < eps && !prev_zero && rho != 0.f && live) {
+      if (pmin < eps && !zero && rho != 0.f && live) {
         // rare: list each projection inside the bound for the fix-up kernel;
         // a row whose entries do not all fit is marked for a full recomputation
         uint32_t f = 0u;
@@ -981,19 +987,22 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
         }
         if (slot > X.fix_cap) atomicOr(X.fix_rows + (row >> 5), 1u << (row & 31));
       }
-      if (prev_zero || rho == 0.f) sw = 0u;
+      if (zero || rho == 0.f) sw = 0u;
       if (live) {
         reinterpret_cast<uint32_t*>(out.signs + static_cast<size_t>(row) * 16)[g] = sw;
-        if (g == 0) out.rnorm[row] = prev_zero ? 0.f : prev_n * rho;
+        if (g == 0) out.rnorm[row] = zero ? 0.f : nk * rho;
       }
     };
 
+    // Per tile k: y' -> partial ||y'||^2 -> arrive -> the signs of tile k - 2
+    // (its projection finished long ago) while the other warps' partial sums
+    // come in -> wait -> codes and residual -> arrive for the projection.
     int k = 0;
     for (; k < n_k; ++k) {
       const int row = row0 + k * row_step;
       const uint32_t oy = off_y(k);
-      const bool got = wait_or_abort(&yrdy[k & 1], static_cast<uint32_t>((k >> 1) & 1));
-      if (!got) flag_error(X.err, abort_flag, 5);
+      const uint32_t ph = static_cast<uint32_t>((k >> 1) & 1);
+      if (!wait_or_abort(&yrdy[k & 1], ph)) { flag_error(X.err, abort_flag, 5); break; }
       tc_fence_after();
       uint32_t u[32];
       tmem_ld32(tbase + oy, u);
@@ -1009,8 +1018,13 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
         }
         sN2[(k & 1) * 4 * kTile + g * kTile + trow] = (s0.x + s0.y) + (s1.x + s1.y);
       }
-      // all four partial sums of every row written; one abort decision for all
-      if (named_bar_sync_or(1, kWsCompute * 32, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
+      // tile k - 2's residual partials share a buffer with this tile's: read
+      // them before this warp's arrival lets the others write this tile's
+      const float rr_old = k >= 2 ? resid2(k) : 0.f;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&nrdy[k & 1]);
+      if (k >= 2) signs(k - 2, rr_old);
+      if (!wait_or_abort(&nrdy[k & 1], ph)) { flag_error(X.err, abort_flag, 5); break; }
       const float* n2 = sN2 + (k & 1) * 4 * kTile + trow;
       const float ss = (n2[0] + n2[kTile]) + (n2[2 * kTile] + n2[3 * kTile]);
       const float nsd = sqrtf(ss);                               // ||H D x|| = sqrt(d) ||x||
@@ -1080,13 +1094,18 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
         }
         if (g == 0) out.norm[row] = zero_row ? 0.f : n;
       }
-      // the previous tile's signs, while this tile's projection runs
-      if (k > 0) signs(k - 1);
-      prev_zero = zero_row;
-      prev_n = n;
-      prev_row = row;
+      my_norm[(k & 1) * 512] = zero_row ? 0.f : n;
     }
-    if (k == n_k && n_k > 0) signs(n_k - 1);
+    if (k == n_k) {
+      // the last two tiles' signs, once every warp has written its residual partials
+      for (int j = n_k >= 2 ? n_k - 2 : 0; j < n_k; ++j) {
+        if (!wait_or_abort(&rrdy[j & 1], static_cast<uint32_t>((j >> 1) & 1))) {
+          flag_error(X.err, abort_flag, 3);
+          break;
+        }
+        signs(j, resid2(j));
+      }
+    }
   }
   __syncthreads();
   if (warp == 0) {
