@@ -8,14 +8,14 @@
 namespace tq {
 
 size_t quantize_scratch_bytes(const tq_ctx& ctx, int64_t n_rows) {
-  if (quantize_d128_applies(ctx, n_rows)) return quantize_d128_scratch_bytes(ctx, n_rows);
+  if (quantize_d128_applies(ctx, n_rows, -1)) return quantize_d128_scratch_bytes(ctx, n_rows);
   return wide_quantize_applies(ctx, n_rows) ? wide_quantize_scratch_bytes(ctx, n_rows) : 0;
 }
 
 int launch_quantize(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld_x, const Packed& out,
                     void* scratch, void* stream) {
   if (take_injected_launch_failure()) return static_cast<int>(cudaErrorLaunchFailure);
-  if (quantize_d128_applies(ctx, n_rows))
+  if (quantize_d128_applies(ctx, n_rows, x_is_bf16))
     return launch_quantize_d128(ctx, x, x_is_bf16, n_rows, ld_x, out, scratch, stream);
   if (scratch && wide_quantize_applies(ctx, n_rows))
     return launch_quantize_wide(ctx, x, x_is_bf16, n_rows, ld_x, out, scratch, stream);

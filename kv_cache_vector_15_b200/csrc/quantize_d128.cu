@@ -761,36 +761,55 @@ __device__ __forceinline__ float min3_abs(float a, float b, float c) {
 //
 // Codes, residual and the tensor-core error bound are those of the kernel
 // above; projections inside the bound go to the exact fix-up kernel.
-constexpr int kWsCompute = 16;                 // compute warps
-constexpr int kWsThreads = (kWsCompute + 1) * 32;
-constexpr int kWsStages = 4;                   // row tiles in shared memory
+// Shape of the kernel for rows of KD coordinates (m = KD projections): KD / 32
+// threads per row, 32 coordinates each, so KD / 8 compute warps; TMEM regions
+// of KD columns (four of them); the row-tile stages hold KD / 64 boxes of 64
+// bf16 columns.  At KD = 64 two CTAs share an SM (256 TMEM columns each).
+template <int KD>
+struct WsShape {
+  static constexpr int kG = KD / 32;                 // threads per row
+  static constexpr int kCompute = KD / 8;            // compute warps
+  static constexpr int kThreads = (kCompute + 1) * 32;
+  static constexpr int kStages = 4;                  // row tiles in shared memory
+  static constexpr int kStage = (KD / 64) * kTile * 128;
+  static constexpr int kOpBytes = KD * KD * 2;       // S or D H as a 16-bit MMA operand
+  static constexpr uint32_t kTmemCols = 4 * KD;
+  static constexpr int kCtasPerSm = KD == 64 ? 2 : 1;
+};
 
+template <int KD>
 constexpr size_t quant_ws_smem_bytes() {
-  return 1024 + 2 * kSmemS + kWsStages * XStage<true>::kBytes + 2 * 4 * kTile * 4 /*norm partials*/ +
-         2 * 4 * kTile * 4 /*residual partials*/ + 2 * kWsCompute * 32 * 4 /*norms*/ + 256;
+  using W = WsShape<KD>;
+  return 1024 + 2 * W::kOpBytes + W::kStages * W::kStage + 2 * W::kG * kTile * 4 /*norm partials*/ +
+         2 * W::kG * kTile * 4 /*residual partials*/ + 2 * W::kCompute * 32 * 4 /*norms*/ + 256;
 }
 
-template <int B>
-__global__ void __launch_bounds__(kWsThreads, 1)
+template <int B, int KD>
+__global__ void __launch_bounds__(WsShape<KD>::kThreads, WsShape<KD>::kCtasPerSm)
 k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, const QuantD128Args X,
                    int64_t n_rows, const Packed out) {
+  using W = WsShape<KD>;
   constexpr int L = 1 << B;
-  constexpr int kStage = XStage<true>::kBytes;                  // 32 KB: two 64-column boxes
+  constexpr int kStage = W::kStage;
+  constexpr int kWsStages = W::kStages;
+  constexpr int kWsCompute = W::kCompute;
+  constexpr int kWsThreads = W::kThreads;
+  constexpr int kG = W::kG;
   constexpr int kNT = SymConsts<B>::kNT > 0 ? SymConsts<B>::kNT : 1;
   constexpr int kNC = SymConsts<B>::kNC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sS = smem;                                            // projection B operand (S, fp16)
-  uint8_t* sHD = smem + kSmemS;                                  // rotation B operand (D H, bf16 +-1)
-  uint8_t* stages = sHD + kSmemS;                                // [kWsStages] row tiles
-  float* sN2 = reinterpret_cast<float*>(stages + kWsStages * kStage);   // [2][4][row] partial ||y'||^2
-  float* sR2 = sN2 + 2 * 4 * kTile;                              // [2][4][row] partial ||64 r||^2
-  float* sNrm = sR2 + 2 * 4 * kTile;                             // [2][compute thread] norms awaiting signs
+  uint8_t* sHD = smem + W::kOpBytes;                             // rotation B operand (D H, bf16 +-1)
+  uint8_t* stages = sHD + W::kOpBytes;                           // [kWsStages] row tiles
+  float* sN2 = reinterpret_cast<float*>(stages + kWsStages * kStage);   // [2][kG][row] partial ||y'||^2
+  float* sR2 = sN2 + 2 * kG * kTile;                             // [2][kG][row] partial ||64 r||^2
+  float* sNrm = sR2 + 2 * kG * kTile;                            // [2][compute thread] norms awaiting signs
   uint64_t* full = reinterpret_cast<uint64_t*>(sNrm + 2 * kWsCompute * 32);   // [kWsStages]
   uint64_t* yrdy = full + kWsStages;                             // [2] rotation done
   uint64_t* prdy = yrdy + 2;                                     // [2] projection done
-  uint64_t* rrdy = prdy + 2;                                     // [2] residual written (16 arrivals)
-  uint64_t* nrdy = rrdy + 2;                                     // [2] norm partials written (16 arrivals)
+  uint64_t* rrdy = prdy + 2;                                     // [2] residual written (one arrival per compute warp)
+  uint64_t* nrdy = rrdy + 2;                                     // [2] norm partials written (likewise)
   uint64_t* fdone = nrdy + 2;                                    // wind-down commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fdone + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
@@ -811,22 +830,23 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
     *abort_flag = 0;
     mbar_fence_init();
   }
-  for (int e = tid; e < kM * 16; e += kWsThreads) {
-    const int j = e >> 4, c = e & 15, kb = c >> 3, cc = c & 7;
-    const uint4 v = *reinterpret_cast<const uint4*>(P.S + j * kD + c * 8);
-    *reinterpret_cast<uint4*>(sS + kb * 16384 + j * 128 + ((cc ^ (j & 7)) << 4)) = v;
+  // S (m = KD rows of KD coordinates) and D H, K-major, 64-coordinate atoms of KD rows
+  for (int e = tid; e < KD * (KD / 8); e += kWsThreads) {
+    const int j = e / (KD / 8), c = e % (KD / 8), kb = c >> 3, cc = c & 7;
+    const uint4 v = *reinterpret_cast<const uint4*>(P.S + j * KD + c * 8);
+    *reinterpret_cast<uint4*>(sS + kb * (KD * 128) + j * 128 + ((cc ^ (j & 7)) << 4)) = v;
   }
   // (D H)[n][k] = H[n][k] D_k = (-1)^popcount(n & k) D_k, as bf16 +-1.0, same swizzled layout
   uint16_t* hd16 = reinterpret_cast<uint16_t*>(sHD);
-  for (int e = tid; e < kD * kD; e += kWsThreads) {
-    const int n = e >> 7, k = e & 127;
+  for (int e = tid; e < KD * KD; e += kWsThreads) {
+    const int n = e / KD, k = e % KD;
     const bool neg = ((__popc(n & k) & 1) != 0) != (X.Dsign[k] != 0u);
     const int kb = k >> 6, chunk = (k & 63) >> 3, within = k & 7;
-    hd16[(kb * 16384 + n * 128 + ((chunk ^ (n & 7)) << 4)) / 2 + within] = neg ? 0xBF80u : 0x3F80u;
+    hd16[(kb * (KD * 128) + n * 128 + ((chunk ^ (n & 7)) << 4)) / 2 + within] = neg ? 0xBF80u : 0x3F80u;
   }
   fence_proxy_async_smem();
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, W::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -834,8 +854,8 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // regions of local tile k: Y (y', then p) and Z (residual hi | lo)
-  auto region_y = [](int64_t k) { return static_cast<uint32_t>(2 * (k & 1) + ((k >> 1) & 1)) * 128u; };
-  auto region_z = [](int64_t k) { return static_cast<uint32_t>(2 * (k & 1) + 1 - ((k >> 1) & 1)) * 128u; };
+  auto region_y = [](int64_t k) { return static_cast<uint32_t>(2 * (k & 1) + ((k >> 1) & 1)) * KD; };
+  auto region_z = [](int64_t k) { return static_cast<uint32_t>(2 * (k & 1) + 1 - ((k >> 1) & 1)) * KD; };
   // a bounded wait that also gives up once another thread has flagged an
   // abort; with a limit of a second or so a waiting thread is suspended
   // between polls (so the waiting warps leave the issue slots to the others),
@@ -862,7 +882,7 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
         const int st = static_cast<int>(k % kWsStages);
         mbar_arrive_expect_tx(&full[st], kStage);
 #pragma unroll
-        for (int bx = 0; bx < 2; ++bx)
+        for (int bx = 0; bx < KD / 64; ++bx)
           tma_load_2d(stages + st * kStage + bx * (kTile * 128), &tmap, &full[st], bx * 64,
                       static_cast<int>(tile_of(k) * kTile));
         ++loads;
@@ -874,12 +894,13 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
         ++landed;
         tc_fence_after();
         const uint32_t xbase = smem_u32(stages + st * kStage), hbase = smem_u32(sHD);
-        const uint32_t idesc = idesc_bf16_f32(kTile, kD);
+        const uint32_t idesc = idesc_bf16_f32(kTile, KD);
         const uint32_t d_tmem = tmem + region_y(k);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_f16_ss(d_tmem, smem_desc_sw128(xbase + off, 1024), smem_desc_sw128(hbase + off, 1024), idesc,
+        for (int kk = 0; kk < KD / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (kTile * 128) + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * (KD * 128) + (kk & 3) * 32;
+          mma_f16_ss(d_tmem, smem_desc_sw128(xbase + aoff, 1024), smem_desc_sw128(hbase + boff, 1024), idesc,
                      kk > 0 ? 1u : 0u);
         }
         mma_commit(&yrdy[k & 1]);
@@ -897,13 +918,13 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
         if (k + kWsStages < n_mine) issue_load(k + kWsStages);
         {
           const uint32_t sbase = smem_u32(sS);
-          const uint32_t idesc = idesc_f16_f32(kTile, kM);
+          const uint32_t idesc = idesc_f16_f32(kTile, KD);
           const uint32_t d_tmem = tmem + region_y(k), a_tmem = tmem + region_z(k);
 #pragma unroll
-          for (int kk = 0; kk < 16; ++kk) {
+          for (int kk = 0; kk < 2 * KD / 16; ++kk) {
             // A step kk: hi (kk & 2 == 0) or lo parts of coordinates 32 (kk >> 2) + 16 (kk & 1) .. + 15
             const int sk = 2 * (kk >> 2) + (kk & 1);
-            const uint64_t bdesc = smem_desc_sw128(sbase + (sk >> 2) * 16384 + (sk & 3) * 32, 1024);
+            const uint64_t bdesc = smem_desc_sw128(sbase + (sk >> 2) * (KD * 128) + (sk & 3) * 32, 1024);
             mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk > 0 ? 1u : 0u);
           }
           mma_commit(&prdy[k & 1]);
@@ -931,7 +952,7 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
     }
   } else {
     // ================================ compute warps ================================
-    const int quad = warp & 3, g = warp >> 2;
+    const int quad = warp & 3, g = warp >> 2;                    // g < kG
     const int trow = quad * 32 + lane;
     const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 32 * g;   // my lane, my columns
     const int n_k = static_cast<int>(n_mine);
@@ -941,13 +962,14 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
     const int row_step = static_cast<int>(gridDim.x) * kTile;
     const int nr = static_cast<int>(n_rows);
     // each tile's norm (0 for a zero row) waits in shared memory for its signs
-    float* my_norm = sNrm + tid;                                 // [2][512]
-    // region offsets of local tile k: Y = 256 (k & 1) + 128 ((k >> 1) & 1), Z = Y ^ 128
-    auto off_y = [](int k) { return static_cast<uint32_t>(((k & 1) << 8) | ((k & 2) << 6)); };
-    // the sum of the four partial ||64 r||^2 of tile k (written before rrdy(k))
+    float* my_norm = sNrm + tid;                                 // [2][compute threads]
+    // region offsets of local tile k: Y = 2 KD (k & 1) + KD ((k >> 1) & 1), Z = Y ^ KD
+    constexpr int kLog = KD == 128 ? 7 : 6;
+    auto off_y = [](int k) { return static_cast<uint32_t>(((k & 1) << (kLog + 1)) | ((k & 2) << (kLog - 1))); };
+    // the sum of the kG partial ||64 r||^2 of tile k (written before rrdy(k))
     auto resid2 = [&](int k) {
-      const float* r2 = sR2 + (k & 1) * 4 * kTile + trow;
-      return (r2[0] + r2[kTile]) + (r2[2 * kTile] + r2[3 * kTile]);
+      const float* r2 = sR2 + (k & 1) * kG * kTile + trow;
+      return kG == 4 ? (r2[0] + r2[kTile]) + (r2[2 * kTile] + r2[3 * kTile]) : r2[0] + r2[kTile];
     };
     // signs of local tile k (its projection), exact recomputation listed within the error bound
     auto signs = [&](int k, float rr) {
@@ -956,7 +978,7 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
         return;
       }
       tc_fence_after();
-      const float nk = my_norm[(k & 1) * 512];
+      const float nk = my_norm[(k & 1) * (kWsCompute * 32)];
       const bool zero = nk == 0.f;
       const float rho = zero ? 0.f : sqrtf(rr) * (1.0f / kResScale);
       const float eps = kResScale * fmaf(X.eps_scale, rho, X.eps_abs);
@@ -989,7 +1011,7 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
       }
       if (zero || rho == 0.f) sw = 0u;
       if (live) {
-        reinterpret_cast<uint32_t*>(out.signs + static_cast<size_t>(row) * 16)[g] = sw;
+        reinterpret_cast<uint32_t*>(out.signs + static_cast<size_t>(row) * (KD / 8))[g] = sw;
         if (g == 0) out.rnorm[row] = zero ? 0.f : nk * rho;
       }
     };
@@ -1016,7 +1038,7 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
           s0 = __ffma2_rn(a, a, s0);
           s1 = __ffma2_rn(b2, b2, s1);
         }
-        sN2[(k & 1) * 4 * kTile + g * kTile + trow] = (s0.x + s0.y) + (s1.x + s1.y);
+        sN2[(k & 1) * kG * kTile + g * kTile + trow] = (s0.x + s0.y) + (s1.x + s1.y);
       }
       // tile k - 2's residual partials share a buffer with this tile's: read
       // them before this warp's arrival lets the others write this tile's
@@ -1025,10 +1047,10 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
       if (lane == 0) mbar_arrive(&nrdy[k & 1]);
       if (k >= 2) signs(k - 2, rr_old);
       if (!wait_or_abort(&nrdy[k & 1], ph)) { flag_error(X.err, abort_flag, 5); break; }
-      const float* n2 = sN2 + (k & 1) * 4 * kTile + trow;
-      const float ss = (n2[0] + n2[kTile]) + (n2[2 * kTile] + n2[3 * kTile]);
+      const float* n2 = sN2 + (k & 1) * kG * kTile + trow;
+      const float ss = kG == 4 ? (n2[0] + n2[kTile]) + (n2[2 * kTile] + n2[3 * kTile]) : n2[0] + n2[kTile];
       const float nsd = sqrtf(ss);                               // ||H D x|| = sqrt(d) ||x||
-      const float n = nsd * 0.08838834764831845f;                // / sqrt(128)
+      const float n = nsd * (KD == 128 ? 0.08838834764831845f : 0.125f);   // / sqrt(KD)
       const bool zero_row = !(n >= kZeroNorm);
       const float nsd_t = zero_row ? 1.f : nsd;
       const float sc = zero_row ? 0.f : kResScale * __frcp_rn(nsd_t);   // = RN(64 / nsd)
@@ -1049,7 +1071,7 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
 #pragma unroll
       for (int w = 0; w < B; ++w) cw[w] = 0u;
       float2 r2a = make_float2(0.f, 0.f), r2b = make_float2(0.f, 0.f);
-      const uint32_t zb = tbase + (oy ^ 128u);
+      const uint32_t zb = tbase + (oy ^ static_cast<uint32_t>(KD));
 #pragma unroll
       for (int g8 = 1; g8 >= 0; --g8) {                         // 16 coordinates -> 8 hi and 8 lo columns
         uint32_t hw[8], lw[8];
@@ -1076,13 +1098,13 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
 #pragma unroll
         for (int w = 0; w < B; ++w) cw[w] = 0u;
       }
-      sR2[(k & 1) * 4 * kTile + g * kTile + trow] = (r2a.x + r2a.y) + (r2b.x + r2b.y);
+      sR2[(k & 1) * kG * kTile + g * kTile + trow] = (r2a.x + r2a.y) + (r2b.x + r2b.y);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&rrdy[k & 1]);
       if (row < nr) {
-        uint32_t* co = reinterpret_cast<uint32_t*>(out.codes + static_cast<size_t>(row) * (B * 16)) + B * g;
+        uint32_t* co = reinterpret_cast<uint32_t*>(out.codes + static_cast<size_t>(row) * (B * KD / 8)) + B * g;
         if constexpr (B == 1) {
           co[0] = cw[0];
         } else if constexpr (B == 2) {
@@ -1094,7 +1116,7 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
         }
         if (g == 0) out.norm[row] = zero_row ? 0.f : n;
       }
-      my_norm[(k & 1) * 512] = zero_row ? 0.f : n;
+      my_norm[(k & 1) * (kWsCompute * 32)] = zero_row ? 0.f : n;
     }
     if (k == n_k) {
       // the last two tiles' signs, once every warp has written its residual partials
@@ -1110,7 +1132,7 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, W::kTmemCols);
   }
 }
 
@@ -1119,44 +1141,52 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
 // it: norm, D, the Walsh-Hadamard butterflies, r = y - c[code], p_j = S_j . r,
 // and the sign bit set or cleared in place (1 = negative; p_j = 0 counts as
 // positive).  Listed (row, j) entries first, one warp each; then the rows
-// marked in the overflow bitmap, all of whose m = 128 signs are recomputed.
-// Lane l holds coordinates 4 l .. 4 l + 3 of the row.
-template <int B, bool BF16IN>
+// marked in the overflow bitmap, all of whose m = KD signs are recomputed.
+// Lane l holds coordinates V l .. V l + V - 1, V = KD / 32.
+template <int B, bool BF16IN, int KD>
 __device__ __forceinline__ void fixup_residual(const KParams& P, const void* __restrict__ x, int64_t ld, int64_t row,
-                                               const Packed& out, int lane, double (&r)[4]) {
-  double v[4];
+                                               const Packed& out, int lane, double (&r)[KD / 32]) {
+  constexpr int V = KD / 32;
+  double v[V];
   if constexpr (BF16IN) {
-    const uint2 xw = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(x) + row * ld + 4 * lane);
-    v[0] = __uint_as_float(xw.x << 16); v[1] = __uint_as_float(xw.x & 0xffff0000u);
-    v[2] = __uint_as_float(xw.y << 16); v[3] = __uint_as_float(xw.y & 0xffff0000u);
+    const uint16_t* xr = static_cast<const uint16_t*>(x) + row * ld + V * lane;
+    if constexpr (V == 4) {
+      const uint2 xw = *reinterpret_cast<const uint2*>(xr);
+      v[0] = __uint_as_float(xw.x << 16); v[1] = __uint_as_float(xw.x & 0xffff0000u);
+      v[2] = __uint_as_float(xw.y << 16); v[3] = __uint_as_float(xw.y & 0xffff0000u);
+    } else {
+      const uint32_t xw = *reinterpret_cast<const uint32_t*>(xr);
+      v[0] = __uint_as_float(xw << 16); v[1] = __uint_as_float(xw & 0xffff0000u);
+    }
   } else {
-    const float4 xw = *reinterpret_cast<const float4*>(static_cast<const float*>(x) + row * ld + 4 * lane);
-    v[0] = xw.x; v[1] = xw.y; v[2] = xw.z; v[3] = xw.w;
+    const float* xr = static_cast<const float*>(x) + row * ld + V * lane;
+#pragma unroll
+    for (int q = 0; q < V; ++q) v[q] = xr[q];
   }
-  // codes of coordinates 4 lane .. 4 lane + 3: bits [4 B lane, 4 B lane + 4 B) of the row
-  const uint8_t* cb = out.codes + row * (B * 16);
-  const int bit0 = 4 * B * lane;
+  // codes of coordinates V lane .. V lane + V - 1: bits [V B lane, V B lane + V B) of the row
+  const uint8_t* cb = out.codes + row * (B * KD / 8);
+  const int bit0 = V * B * lane;
   uint32_t win = 0;
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
     const int byte = (bit0 >> 3) + k;
-    if (byte < B * 16) win |= static_cast<uint32_t>(cb[byte]) << (8 * k);
+    if (byte < B * KD / 8) win |= static_cast<uint32_t>(cb[byte]) << (8 * k);
   }
   win >>= (bit0 & 7);
-  const uint32_t dm = P.Dmask[lane >> 3] >> (4 * (lane & 7));
+  const uint32_t dm = P.Dmask[(V * lane) >> 5] >> ((V * lane) & 31);
   double ss = 0.0;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < V; ++q) {
     if ((dm >> q) & 1u) v[q] = -v[q];
     ss = fma(v[q], v[q], ss);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  // butterflies over coordinate bits 0, 1 (in the lane), then 2 .. 6 (across lanes)
+  // butterflies over the coordinate bits inside the lane, then across lanes
 #pragma unroll
-  for (int h = 1; h < 4; h <<= 1)
+  for (int h = 1; h < V; h <<= 1)
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+    for (int q = 0; q < V; ++q)
       if ((q & h) == 0) {
         const double a = v[q], c2 = v[q + h];
         v[q] = a + c2;
@@ -1165,33 +1195,43 @@ __device__ __forceinline__ void fixup_residual(const KParams& P, const void* __r
 #pragma unroll
   for (int lh = 1; lh < 32; lh <<= 1)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < V; ++q) {
       const double o = __shfl_xor_sync(0xffffffffu, v[q], lh);
       v[q] = (lane & lh) ? o - v[q] : v[q] + o;
     }
-  const double inv = 1.0 / (sqrt(ss) * sqrt(static_cast<double>(kD)));
+  const double inv = 1.0 / (sqrt(ss) * sqrt(static_cast<double>(KD)));
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < V; ++q) {
     const uint32_t code = (win >> (B * q)) & ((1u << B) - 1u);
     r[q] = v[q] * inv - static_cast<double>(P.c[code]);
   }
 }
 
-// S_j . r over the warp (lane l: coordinates 4 l .. 4 l + 3), all lanes get it
-__device__ __forceinline__ double fixup_project(const KParams& P, int j, int lane, const double (&r)[4]) {
-  const uint2 sw = __ldg(reinterpret_cast<const uint2*>(P.S + j * kD + 4 * lane));
-  const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sw.x));
-  const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sw.y));
-  double p = static_cast<double>(s01.x) * r[0];
-  p = fma(static_cast<double>(s01.y), r[1], p);
-  p = fma(static_cast<double>(s23.x), r[2], p);
-  p = fma(static_cast<double>(s23.y), r[3], p);
+// S_j . r over the warp (lane l: coordinates V l .. V l + V - 1), all lanes get it
+template <int KD>
+__device__ __forceinline__ double fixup_project(const KParams& P, int j, int lane, const double (&r)[KD / 32]) {
+  constexpr int V = KD / 32;
+  double p = 0.0;
+  if constexpr (V == 4) {
+    const uint2 sw = __ldg(reinterpret_cast<const uint2*>(P.S + j * KD + 4 * lane));
+    const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sw.x));
+    const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sw.y));
+    p = static_cast<double>(s01.x) * r[0];
+    p = fma(static_cast<double>(s01.y), r[1], p);
+    p = fma(static_cast<double>(s23.x), r[2], p);
+    p = fma(static_cast<double>(s23.y), r[3], p);
+  } else {
+    const uint32_t sw = __ldg(reinterpret_cast<const uint32_t*>(P.S + j * KD + 2 * lane));
+    const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sw));
+    p = static_cast<double>(s01.x) * r[0];
+    p = fma(static_cast<double>(s01.y), r[1], p);
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
   return p;
 }
 
-template <int B, bool BF16IN>
+template <int B, bool BF16IN, int KD>
 __global__ void __launch_bounds__(256)
 k_qjl_fixup_d128(const KParams P, const void* __restrict__ x, int64_t ld, int64_t n_rows, const Packed out,
                  const unsigned long long* __restrict__ fix_list, const unsigned int* __restrict__ fix_count,
@@ -1205,12 +1245,12 @@ k_qjl_fixup_d128(const KParams P, const void* __restrict__ x, int64_t ld, int64_
     const unsigned long long ent = fix_list[e];
     const int64_t row = static_cast<int64_t>(ent >> 8);
     const int j = static_cast<int>(ent & 0xffu);
-    if (row >= n_rows || j >= kM) continue;                      // never listed; kept in bounds regardless
-    double r[4];
-    fixup_residual<B, BF16IN>(P, x, ld, row, out, lane, r);
-    const double p = fixup_project(P, j, lane, r);
+    if (row >= n_rows || j >= KD) continue;                      // never listed; kept in bounds regardless
+    double r[KD / 32];
+    fixup_residual<B, BF16IN, KD>(P, x, ld, row, out, lane, r);
+    const double p = fixup_project<KD>(P, j, lane, r);
     if (lane == 0) {
-      unsigned int* word = reinterpret_cast<unsigned int*>(out.signs + row * 16) + (j >> 5);
+      unsigned int* word = reinterpret_cast<unsigned int*>(out.signs + row * (KD / 8)) + (j >> 5);
       const unsigned int m = 1u << (j & 31);
       if (p < 0.0) atomicOr(word, m); else atomicAnd(word, ~m);
     }
@@ -1223,15 +1263,15 @@ k_qjl_fixup_d128(const KParams P, const void* __restrict__ x, int64_t ld, int64_
       const int b = __ffs(bits) - 1;
       bits &= bits - 1;
       const int64_t row = w * 32 + b;
-      double r[4];
-      fixup_residual<B, BF16IN>(P, x, ld, row, out, lane, r);
-      uint32_t word = 0u;                                        // lane l keeps sign word l / 8... built below
+      double r[KD / 32];
+      fixup_residual<B, BF16IN, KD>(P, x, ld, row, out, lane, r);
+      uint32_t word = 0u;                                        // lane l builds sign word l
 #pragma unroll 1
-      for (int j = 0; j < kM; ++j) {
-        const double p = fixup_project(P, j, lane, r);
+      for (int j = 0; j < KD; ++j) {
+        const double p = fixup_project<KD>(P, j, lane, r);
         if (lane == (j >> 5) && p < 0.0) word |= 1u << (j & 31);
       }
-      if (lane < kM / 32) reinterpret_cast<uint32_t*>(out.signs + row * 16)[lane] = word;
+      if (lane < KD / 32) reinterpret_cast<uint32_t*>(out.signs + row * (KD / 8))[lane] = word;
     }
   }
 }
@@ -1249,14 +1289,15 @@ size_t fix_scratch_bytes(int64_t n_rows) {
   return fix_bitmap_bytes(n_rows) + 256 + static_cast<size_t>(fix_cap_for(n_rows)) * sizeof(unsigned long long);
 }
 
-template <int B, bool BF16IN>
+template <int B, bool BF16IN, int KD>
 int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, const Packed& out, void* scratch,
               cudaStream_t s) {
+  static_assert(BF16IN || KD == 128, "fp32 rows: d = 128 only");
   const KParams& P = ctx.kp;
   auto encode = get_encode();
   if (!encode) return static_cast<int>(cudaErrorNotSupported);
   CUtensorMap tmap;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(n_rows)};
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(KD), static_cast<cuuint64_t>(n_rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * (BF16IN ? 2 : 4)};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(XStage<BF16IN>::kColsPerBox), static_cast<cuuint32_t>(kTile)};
   const cuuint32_t estr[2] = {1, 1};
@@ -1266,7 +1307,7 @@ int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, cons
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return static_cast<int>(cudaErrorInvalidValue);
   QuantD128Args X;
-  for (int i = 0; i < kD; ++i) X.Dsign[i] = ctx.D[i] < 0 ? 0x80000000u : 0u;
+  for (int i = 0; i < kD; ++i) X.Dsign[i] = (i < KD && ctx.D[i] < 0) ? 0x80000000u : 0u;
   X.eps_scale = ctx.qjl_eps_scale;
   X.eps_abs = ctx.qjl_eps_abs;
   X.err = P.err;
@@ -1276,7 +1317,6 @@ int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, cons
   X.fix_count = nullptr;
   X.fix_cap = 0;
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
-  const int grid = static_cast<int>(n_tiles < ctx.num_sms ? n_tiles : ctx.num_sms);
   if constexpr (BF16IN) {                // bf16 rows: the rotation on the tensor cores
     if (!scratch) return static_cast<int>(cudaErrorInvalidValue);   // the fix-up scratch lives there
     uint8_t* sc = static_cast<uint8_t*>(scratch);
@@ -1287,16 +1327,19 @@ int launch_tc(const tq_ctx& ctx, const void* x, int64_t n_rows, int64_t ld, cons
     X.fix_cap = static_cast<unsigned int>(forced > 0 && forced < cap ? forced : cap);
     cudaError_t e = cudaMemsetAsync(sc, 0, fix_bitmap_bytes(n_rows) + 256, s);
     if (e != cudaSuccess) return static_cast<int>(e);
-    const size_t smem = quant_ws_smem_bytes();
-    e = cudaFuncSetAttribute(k_quantize_d128_ws<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const size_t smem = quant_ws_smem_bytes<KD>();
+    e = cudaFuncSetAttribute(k_quantize_d128_ws<B, KD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
-    k_quantize_d128_ws<B><<<grid, kWsThreads, smem, s>>>(tmap, P, X, n_rows, out);
+    const int64_t slots = static_cast<int64_t>(ctx.num_sms) * WsShape<KD>::kCtasPerSm;
+    const int grid = static_cast<int>(n_tiles < slots ? n_tiles : slots);
+    k_quantize_d128_ws<B, KD><<<grid, WsShape<KD>::kThreads, smem, s>>>(tmap, P, X, n_rows, out);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return static_cast<int>(e);
-    k_qjl_fixup_d128<B, true><<<ctx.num_sms * 8, 256, 0, s>>>(P, x, ld, n_rows, out, X.fix_list, X.fix_count,
-                                                                 X.fix_cap, X.fix_rows);
+    k_qjl_fixup_d128<B, true, KD><<<ctx.num_sms * 8, 256, 0, s>>>(P, x, ld, n_rows, out, X.fix_list, X.fix_count,
+                                                                     X.fix_cap, X.fix_rows);
   } else {                                // fp32 rows: the rotation in registers
+    const int grid = static_cast<int>(n_tiles < ctx.num_sms ? n_tiles : ctx.num_sms);
     const size_t smem = quant_smem_bytes<false>();
     cudaError_t e = cudaFuncSetAttribute(k_quantize_d128_tc<B, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -1314,30 +1357,41 @@ size_t quantize_d128_scratch_bytes(const tq_ctx& ctx, int64_t n_rows) {
   return fix_scratch_bytes(n_rows);
 }
 
-bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows) {
+bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows, int x_is_bf16) {
   if (ctx.d_in != ctx.d) return false;                   // padded rows use the general kernel
   const KParams& P = ctx.kp;
-  return P.d == kD && P.m == kM && P.B >= 1 && P.B <= 4 && n_rows > 0 && n_rows < (int64_t(1) << 31) - 256 &&
-         ctx.use_tc && get_encode() != nullptr;
+  // d = m = 128 (bf16 or fp32 rows), or d = m = 64 for bf16 rows (the
+  // 64-channel parts of a split row); x_is_bf16 < 0: either input type
+  const bool shape = (P.d == 128 && P.m == 128) || (P.d == 64 && P.m == 64 && x_is_bf16 != 0);
+  return shape && P.B >= 1 && P.B <= 4 && n_rows > 0 && n_rows < (int64_t(1) << 31) - 256 && ctx.use_tc &&
+         get_encode() != nullptr;
 }
 
 int launch_quantize_d128(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
                          const Packed& out, void* scratch, void* stream) {
   const KParams& P = ctx.kp;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (P.d == 64) {
+    switch (P.B) {
+      case 1: return launch_tc<1, true, 64>(ctx, x, n_rows, ld, out, scratch, s);
+      case 2: return launch_tc<2, true, 64>(ctx, x, n_rows, ld, out, scratch, s);
+      case 3: return launch_tc<3, true, 64>(ctx, x, n_rows, ld, out, scratch, s);
+      default: return launch_tc<4, true, 64>(ctx, x, n_rows, ld, out, scratch, s);
+    }
+  }
   if (x_is_bf16) {
     switch (P.B) {
-      case 1: return launch_tc<1, true>(ctx, x, n_rows, ld, out, scratch, s);
-      case 2: return launch_tc<2, true>(ctx, x, n_rows, ld, out, scratch, s);
-      case 3: return launch_tc<3, true>(ctx, x, n_rows, ld, out, scratch, s);
-      default: return launch_tc<4, true>(ctx, x, n_rows, ld, out, scratch, s);
+      case 1: return launch_tc<1, true, 128>(ctx, x, n_rows, ld, out, scratch, s);
+      case 2: return launch_tc<2, true, 128>(ctx, x, n_rows, ld, out, scratch, s);
+      case 3: return launch_tc<3, true, 128>(ctx, x, n_rows, ld, out, scratch, s);
+      default: return launch_tc<4, true, 128>(ctx, x, n_rows, ld, out, scratch, s);
     }
   }
   switch (P.B) {
-    case 1: return launch_tc<1, false>(ctx, x, n_rows, ld, out, scratch, s);
-    case 2: return launch_tc<2, false>(ctx, x, n_rows, ld, out, scratch, s);
-    case 3: return launch_tc<3, false>(ctx, x, n_rows, ld, out, scratch, s);
-    default: return launch_tc<4, false>(ctx, x, n_rows, ld, out, scratch, s);
+    case 1: return launch_tc<1, false, 128>(ctx, x, n_rows, ld, out, scratch, s);
+    case 2: return launch_tc<2, false, 128>(ctx, x, n_rows, ld, out, scratch, s);
+    case 3: return launch_tc<3, false, 128>(ctx, x, n_rows, ld, out, scratch, s);
+    default: return launch_tc<4, false, 128>(ctx, x, n_rows, ld, out, scratch, s);
   }
 }
 

@@ -95,7 +95,7 @@ struct tq_ctx;
 
 namespace tq {
 // d = 128 hot-path kernels (quantize_d128.cu, ...)
-bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows);
+bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows, int x_is_bf16);   // x_is_bf16 < 0: either
 size_t quantize_d128_scratch_bytes(const tq_ctx& ctx, int64_t n_rows);   // deferred sign fix-up list
 int launch_quantize_d128(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
                          const Packed& out, void* scratch, void* stream);

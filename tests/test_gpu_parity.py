@@ -78,11 +78,12 @@ def test_quantize_d128_tensor_core_small_first(tq, b):
 
 
 @pytest.mark.parametrize("b", [2, 3, 4, 5])
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_quantize_d128_many_tiles(tq, b, dtype):
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 128), ("bf16", 64)])
+def test_quantize_d128_many_tiles(tq, b, dtype, d):
     """Enough rows that every CTA loops over several tiles (phase flips of
-    every barrier), with a ragged last tile."""
-    d, m, n = 128, 128, 100003
+    every barrier), with a ragged last tile; d = 64 bf16 rows take the same
+    tensor-core kernel at half width (two CTAs per SM)."""
+    m, n = d, 100003
     xt, x = make_rows(d, n, dtype, seed=100 + b)
     P = op.Params(d, b, m, seed=0)
     T = make_ctx(tq, d, b, m)
