@@ -62,9 +62,10 @@ template <bool BF16OUT>
 constexpr size_t dequant_smem_bytes() {
   return 1024 + 32768 /*St*/ + 32768 /*D H*/ + kPairs * OutStage<BF16OUT>::kBytes + 512;
 }
+template <int KD>
 constexpr size_t dequant_ovl_smem_bytes() {
-  return 1024 + 32768 /*St*/ + 32768 /*D H*/ + kPairs * 32768 /*sign operands*/ + kPairs * OutStage<true>::kBytes +
-         512;
+  return 1024 + 2 * (KD * KD * 2) /*S^T, D H*/ + kPairs * (kTile * KD * 2) /*sign operands*/ +
+         kPairs * (kTile * KD * 2) /*output stages*/ + 512;
 }
 
 __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* smem_src, int x, int y) {
@@ -380,19 +381,21 @@ k_dequant_d128_tc(const __grid_constant__ CUtensorMap tmap_out, const KParams P,
 // the next tile's signs into shared memory -> barrier -> rotation MMA; while
 // it runs, decode the next tile's yhat -> wait -> the next tile's S^T z MMA
 // -> read, scale, round and stage the output -> barrier -> TMA store.
-template <int B, bool PROD>
+template <int B, bool PROD, int KD>
 __global__ void __launch_bounds__(kThreads, 1)
 k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P, const DequantD128Args X,
                    const Packed in, int64_t n_rows) {
   constexpr int L = 1 << B;
-  constexpr int kStage = OutStage<true>::kBytes;          // 32 KB
-  constexpr int kH = kD / 2;
+  constexpr int kStage = kTile * KD * 2;                  // bf16 output tile (KD / 64 boxes)
+  constexpr int kH = KD / 2;                               // coordinates (and projections) per thread
+  constexpr int kNW = B * kH / 32;                         // packed code words per thread
+  constexpr int kOp = KD * KD * 2;                         // S^T or D H as a binary16 operand
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sSt = smem;                                   // B of S^T z: row i, K position j holds S[j][i]
-  uint8_t* sDH = smem + 32768;                           // B of the rotation (N = n, K = k)
-  uint8_t* sZ = smem + 65536;                            // [pair] A of S^T z: row r, K position j holds z_j
-  uint8_t* sOut = sZ + kPairs * 32768;                   // [pair] output stages
+  uint8_t* sDH = smem + kOp;                             // B of the rotation (N = n, K = k)
+  uint8_t* sZ = sDH + kOp;                               // [pair] A of S^T z: row r, K position j holds z_j
+  uint8_t* sOut = sZ + kPairs * kStage;                  // [pair] output stages
   uint64_t* m1 = reinterpret_cast<uint64_t*>(sOut + kPairs * kStage);   // [pair] S^T z done
   uint64_t* m2 = m1 + kPairs;                                            // [pair] rotation done
   uint64_t* fdone = m2 + kPairs;                                         // [pair] wind-down commit
@@ -413,25 +416,25 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
   if (B == 2 && tid < 16) lut2[tid] = make_float2(P.c[tid & 3] * kUnit, P.c[tid >> 2] * kUnit);
   if (PROD) {
     uint16_t* st16 = reinterpret_cast<uint16_t*>(sSt);
-    for (int e = tid; e < kD * kM; e += kThreads) {
-      const int i = e >> 7, j = e & 127;
+    for (int e = tid; e < KD * KD; e += kThreads) {
+      const int i = e / KD, j = e % KD;
       const int kb = j >> 6, chunk = (j & 63) >> 3, within = j & 7;
-      st16[(kb * 16384 + i * 128 + ((chunk ^ (i & 7)) << 4)) / 2 + within] = P.St[i * kM + j];
+      st16[(kb * (KD * 128) + i * 128 + ((chunk ^ (i & 7)) << 4)) / 2 + within] = P.St[i * KD + j];
     }
   }
   {
     // (D H)[n][k] = D_n (-1)^popcount(n & k), binary16 +-1, same swizzled layout
     uint16_t* h16 = reinterpret_cast<uint16_t*>(sDH);
-    for (int e = tid; e < kD * kD; e += kThreads) {
-      const int n = e >> 7, k = e & 127;
+    for (int e = tid; e < KD * KD; e += kThreads) {
+      const int n = e / KD, k = e % KD;
       const bool neg = ((__popc(n & k) & 1) != 0) != (((X.Dneg[n >> 5] >> (n & 31)) & 1u) != 0);
       const int kb = k >> 6, chunk = (k & 63) >> 3, within = k & 7;
-      h16[(kb * 16384 + n * 128 + ((chunk ^ (n & 7)) << 4)) / 2 + within] = neg ? 0xBC00u : 0x3C00u;
+      h16[(kb * (KD * 128) + n * 128 + ((chunk ^ (n & 7)) << 4)) / 2 + within] = neg ? 0xBC00u : 0x3C00u;
     }
   }
   fence_proxy_async_smem();
   if (warp == 0) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(tmem_slot, 4 * KD);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -444,11 +447,11 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
   const bool storer = (half == 1 && lb == 0 && lane == 0);        // issues the pair's TMA stores
   const int trow = lb * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>(lb * 32) << 16;
-  const uint32_t t_reg0 = tmem + lane_base + pair * 256;  // region k mod 2: S^T z, then the output of tile k
+  const uint32_t t_reg0 = tmem + lane_base + pair * (2 * KD);   // region k mod 2: S^T z, then the output of tile k
   const uint32_t bar_id = 1 + pair;
   uint8_t* stage = sOut + pair * kStage;
-  uint8_t* zbuf = sZ + pair * 32768;
-  const float inv_sqrt_d = 0.08838834764831845f;
+  uint8_t* zbuf = sZ + pair * kStage;
+  const float inv_sqrt_d = KD == 128 ? 0.08838834764831845f : 0.125f;
   const float qjl = P.qjl_scale * kUnit;                  // S^T z in unit-norm x kUnit
   const int64_t t_first = blockIdx.x + static_cast<int64_t>(pair) * gridDim.x;
   const int64_t t_step = static_cast<int64_t>(kPairs) * gridDim.x;
@@ -456,13 +459,31 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
 
   // my part of a packed row: codes of my 64 coordinates, my two sign words, norms
   struct Part {
-    uint32_t cw[B * 2];
+    uint32_t cw[kNW];
     uint32_t sg0, sg1;
     float nrm, rn;
   };
   auto load_packed = [&](int64_t tile, Part& pt) {
     const int64_t row = tile * kTile + trow;
-    if (tile < n_tiles && row < n_rows) {
+    if (tile < n_tiles && row < n_rows && KD == 64) {
+      const uint8_t* cp = in.codes + row * (B * 8) + half * (B * 4);
+      if constexpr (B == 1) {
+        pt.cw[0] = __ldg(reinterpret_cast<const uint32_t*>(cp));
+      } else if constexpr (B == 2) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(cp));
+        pt.cw[0] = u.x; pt.cw[1] = u.y;
+      } else if constexpr (B == 3) {
+#pragma unroll
+        for (int w = 0; w < 3; ++w) pt.cw[w] = __ldg(reinterpret_cast<const uint32_t*>(cp) + w);
+      } else {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(cp));
+        pt.cw[0] = u.x; pt.cw[1] = u.y; pt.cw[2] = u.z; pt.cw[3] = u.w;
+      }
+      pt.sg0 = PROD ? __ldg(reinterpret_cast<const uint32_t*>(in.signs + row * 8 + half * 4)) : 0u;
+      pt.sg1 = 0u;
+      pt.nrm = __ldg(in.norm + row);
+      pt.rn = __ldg(in.rnorm + row);
+    } else if (tile < n_tiles && row < n_rows) {
       const uint8_t* cp = in.codes + row * (B * 16) + half * (B * 8);
       if constexpr (B == 1) {
         const uint2 u = __ldg(reinterpret_cast<const uint2*>(cp));
@@ -496,7 +517,7 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
       pt.rn = __ldg(in.rnorm + row);
     } else {
 #pragma unroll
-      for (int w = 0; w < B * 2; ++w) pt.cw[w] = 0u;
+      for (int w = 0; w < kNW; ++w) pt.cw[w] = 0u;
       pt.sg0 = pt.sg1 = 0u;
       pt.nrm = 0.f;
       pt.rn = 0.f;
@@ -526,7 +547,7 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
   // K block `half`, 16-byte chunk c (projections 64 half + 8 c ..) at chunk c ^ (trow & 7)
   auto write_signs = [&](const Part& pt) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < kH / 8; ++c) {
       const uint32_t sgw = (c < 4 ? pt.sg0 : pt.sg1) >> ((c & 3) * 8);   // projections 8 c .. 8 c + 7 (of mine)
       uint32_t w4[4];
 #pragma unroll
@@ -534,19 +555,22 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
         const uint32_t b2 = sgw >> (2 * u);                 // bits of projections 2u, 2u + 1
         w4[u] = 0x3C003C00u | ((b2 & 1u) << 15) | ((b2 & 2u) << 30);
       }
-      *reinterpret_cast<uint4*>(zbuf + half * 16384 + trow * 128 + ((c ^ (trow & 7)) << 4)) =
+      // K atom and 16-byte chunk of projections half kH + 8 c .. + 7
+      const int atom = KD == 128 ? half : 0, chunk = KD == 128 ? c : 4 * half + c;
+      *reinterpret_cast<uint4*>(zbuf + atom * 16384 + trow * 128 + ((chunk ^ (trow & 7)) << 4)) =
           make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
   };
   auto issue_stz = [&](int k) {                            // S^T z of this pair's k-th tile
     tc_fence_after();
     const uint32_t zbase = smem_u32(zbuf), sbase = smem_u32(sSt);
-    const uint32_t idesc = idesc_f16_f32(kTile, kD);
-    const uint32_t d_tmem = tmem + pair * 256 + (k & 1) * 128;
+    const uint32_t idesc = idesc_f16_f32(kTile, KD);
+    const uint32_t d_tmem = tmem + pair * (2 * KD) + (k & 1) * KD;
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-      mma_f16_ss(d_tmem, smem_desc_sw128(zbase + off, 1024), smem_desc_sw128(sbase + off, 1024), idesc,
+    for (int kk = 0; kk < KD / 16; ++kk) {
+      const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+      const uint32_t boff = (kk >> 2) * (KD * 128) + (kk & 3) * 32;
+      mma_f16_ss(d_tmem, smem_desc_sw128(zbase + aoff, 1024), smem_desc_sw128(sbase + boff, 1024), idesc,
                  kk > 0 ? 1u : 0u);
     }
     mma_commit(&m1[pair]);
@@ -565,8 +589,8 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
 
   int mine = 0;
   for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
-    const uint32_t t_acc = t_reg0 + (mine & 1) * 128;      // S^T z, then the output
-    const uint32_t t_a = t_reg0 + ((mine + 1) & 1) * 128;   // v hi | lo
+    const uint32_t t_acc = t_reg0 + (mine & 1) * KD;       // S^T z, then the output
+    const uint32_t t_a = t_reg0 + ((mine + 1) & 1) * KD;    // v hi | lo
     // v in the unit-norm domain times kUnit; norm / sqrt(d) / kUnit is applied to the output
     const float wq = cur.nrm > 0.f ? (cur.rn / cur.nrm) * qjl : 0.f;
     const float oscale = cur.nrm * (inv_sqrt_d / kUnit);
@@ -577,9 +601,9 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
       }
       tc_fence_after();
 #pragma unroll
-      for (int g2 = 0; g2 < 2; ++g2) {
+      for (int g2 = 0; g2 < kH / 32; ++g2) {
         uint32_t acc[32];
-        tmem_ld32(t_acc + half * 64 + g2 * 32, acc);
+        tmem_ld32(t_acc + half * kH + g2 * 32, acc);
         tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 32; ++k) v[g2 * 32 + k] = fmaf(wq, __uint_as_float(acc[k]), v[g2 * 32 + k]);
@@ -590,7 +614,7 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
     }
     // ---- v = hi + lo (binary16) into TMEM: the rotation's A operand ------------------
 #pragma unroll
-    for (int ch = 0; ch < 2; ++ch) {
+    for (int ch = 0; ch < kH / 32; ++ch) {
 #pragma unroll
       for (int g8 = 0; g8 < 2; ++g8) {
         uint32_t hw[8], lw[8];
@@ -604,8 +628,8 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
           hw[k] = *reinterpret_cast<const uint32_t*>(&h);
           lw[k] = *reinterpret_cast<const uint32_t*>(&l);
         }
-        tmem_st8(t_a + half * 32 + ch * 16 + g8 * 8, hw);
-        tmem_st8(t_a + 64 + half * 32 + ch * 16 + g8 * 8, lw);
+        tmem_st8(t_a + half * (KD / 4) + ch * 16 + g8 * 8, hw);
+        tmem_st8(t_a + KD / 2 + half * (KD / 4) + ch * 16 + g8 * 8, lw);
       }
     }
     tmem_wait_st();
@@ -617,13 +641,13 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
     if (leader) {
       tc_fence_after();
       const uint32_t sbase = smem_u32(sDH);
-      const uint32_t idesc = idesc_f16_f32(kTile, kD);
-      const uint32_t d_tmem = tmem + pair * 256 + (mine & 1) * 128;
-      const uint32_t a_tmem = tmem + pair * 256 + ((mine + 1) & 1) * 128;
+      const uint32_t idesc = idesc_f16_f32(kTile, KD);
+      const uint32_t d_tmem = tmem + pair * (2 * KD) + (mine & 1) * KD;
+      const uint32_t a_tmem = tmem + pair * (2 * KD) + ((mine + 1) & 1) * KD;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int kk = k & 7;
-        const uint64_t bdesc = smem_desc_sw128(sbase + (kk >> 2) * 16384 + (kk & 3) * 32, 1024);
+      for (int k = 0; k < 2 * KD / 16; ++k) {
+        const int kk = k % (KD / 16);
+        const uint64_t bdesc = smem_desc_sw128(sbase + (kk >> 2) * (KD * 128) + (kk & 3) * 32, 1024);
         mma_f16_ts(d_tmem, a_tmem + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
       }
       mma_commit(&m2[pair]);
@@ -641,18 +665,18 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
     // the rotation has read v: the next tile's S^T z may run into its region
     if (PROD && leader && t + t_step < n_tiles && *reinterpret_cast<volatile int*>(abort_flag) == 0)
       issue_stz(mine + 1);
-    // ---- my 64 output columns, staged (swizzled) for the TMA store, 32 at a time -------
+    // ---- my kH output columns, staged (swizzled) for the TMA store, 32 at a time -------
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
+    for (int hh = 0; hh < kH / 32; ++hh) {
       uint32_t o[32];
-      tmem_ld32(t_acc + half * 64 + hh * 32, o);
+      tmem_ld32(t_acc + half * kH + hh * 32, o);
       tmem_wait_ld();
       if (hh == 0) {
         if (storer && store_pending) bulk_wait_read0();     // previous tile's store has read the stage
         named_bar_sync(bar_id, 256);
       }
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {                      // box `half`: my 64 columns, 8 per chunk
+      for (int c4 = 0; c4 < 4; ++c4) {                      // 8 columns per 16-byte chunk
         const int cc = hh * 4 + c4;
         uint32_t wv[4];
 #pragma unroll
@@ -662,7 +686,9 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
               __floats2bfloat162_rn(__uint_as_float(o[e]) * oscale, __uint_as_float(o[e + 1]) * oscale);
           wv[u] = *reinterpret_cast<const uint32_t*>(&p2);
         }
-        *reinterpret_cast<uint4*>(stage + half * (kTile * 128) + trow * 128 + ((cc ^ (trow & 7)) << 4)) =
+        // box and 16-byte chunk of output columns half kH + 8 cc .. + 7
+        const int box = KD == 128 ? half : 0, chunk = KD == 128 ? cc : 4 * half + cc;
+        *reinterpret_cast<uint4*>(stage + box * (kTile * 128) + trow * 128 + ((chunk ^ (trow & 7)) << 4)) =
             make_uint4(wv[0], wv[1], wv[2], wv[3]);
       }
     }
@@ -673,9 +699,8 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
     named_bar_sync(bar_id, 256);
     if (storer) {
 #pragma unroll
-      for (int bx = 0; bx < OutStage<true>::kBoxes; ++bx)
-        tma_store_2d(&tmap_out, stage + bx * (kTile * 128), bx * OutStage<true>::kColsPerBox,
-                     static_cast<int>(t * kTile));
+      for (int bx = 0; bx < KD / 64; ++bx)
+        tma_store_2d(&tmap_out, stage + bx * (kTile * 128), bx * 64, static_cast<int>(t * kTile));
       bulk_commit();
       store_pending = true;
     }
@@ -690,18 +715,19 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, 4 * KD);
   }
 }
 
-template <int B, bool PROD, bool BF16OUT>
-int launch(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, cudaStream_t s) {
+template <int B, bool PROD, bool BF16OUT, int KD>
+int launch(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int64_t ld_out, cudaStream_t s) {
+  static_assert(BF16OUT || KD == 128, "fp32 output: d = 128 only");
   const KParams& P = ctx.kp;
   auto encode = tensor_map_encoder();
   if (!encode) return static_cast<int>(cudaErrorNotSupported);
   CUtensorMap tmap;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(n_rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * (BF16OUT ? 2 : 4)};
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(KD), static_cast<cuuint64_t>(n_rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_out) * (BF16OUT ? 2 : 4)};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(OutStage<BF16OUT>::kColsPerBox), static_cast<cuuint32_t>(kTile)};
   const cuuint32_t estr[2] = {1, 1};
   if (encode(&tmap, BF16OUT ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, out, dims,
@@ -710,18 +736,18 @@ int launch(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, cudaS
     return static_cast<int>(cudaErrorInvalidValue);
   DequantD128Args X;
   for (int w = 0; w < kD / 32; ++w) X.Dneg[w] = 0u;
-  for (int i = 0; i < kD; ++i)
+  for (int i = 0; i < KD; ++i)
     if (ctx.D[i] < 0) X.Dneg[i >> 5] |= 1u << (i & 31);
   X.err = P.err;
   X.wait_cycles = wait_limit_cycles();
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
   const int grid = static_cast<int>(n_tiles < ctx.num_sms ? n_tiles : ctx.num_sms);
   if constexpr (BF16OUT) {                 // the overlapped kernel (bf16 output)
-    const size_t smem = dequant_ovl_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(k_dequant_d128_ovl<B, PROD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    const size_t smem = dequant_ovl_smem_bytes<KD>();
+    cudaError_t e = cudaFuncSetAttribute(k_dequant_d128_ovl<B, PROD, KD>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
-    k_dequant_d128_ovl<B, PROD><<<grid, kThreads, smem, s>>>(tmap, P, X, in, n_rows);
+    k_dequant_d128_ovl<B, PROD, KD><<<grid, kThreads, smem, s>>>(tmap, P, X, in, n_rows);
   } else {
     const size_t smem = dequant_smem_bytes<BF16OUT>();
     cudaError_t e = cudaFuncSetAttribute(k_dequant_d128_tc<B, PROD, BF16OUT>,
@@ -734,28 +760,39 @@ int launch(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, cudaS
 }
 
 template <int B>
-int launch_B(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int bf16, int prod, cudaStream_t s) {
-  if (prod) return bf16 ? launch<B, true, true>(ctx, in, n_rows, out, s) : launch<B, true, false>(ctx, in, n_rows, out, s);
-  return bf16 ? launch<B, false, true>(ctx, in, n_rows, out, s) : launch<B, false, false>(ctx, in, n_rows, out, s);
+int launch_B(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int64_t ld_out, int bf16, int prod,
+             cudaStream_t s) {
+  if (ctx.kp.d == 64) {                    // bf16 output only (see dequant_d128_applies)
+    return prod ? launch<B, true, true, 64>(ctx, in, n_rows, out, ld_out, s)
+                : launch<B, false, true, 64>(ctx, in, n_rows, out, ld_out, s);
+  }
+  if (prod)
+    return bf16 ? launch<B, true, true, 128>(ctx, in, n_rows, out, ld_out, s)
+                : launch<B, true, false, 128>(ctx, in, n_rows, out, ld_out, s);
+  return bf16 ? launch<B, false, true, 128>(ctx, in, n_rows, out, ld_out, s)
+              : launch<B, false, false, 128>(ctx, in, n_rows, out, ld_out, s);
 }
 
 }  // namespace
 
-bool dequant_d128_applies(const tq_ctx& ctx, int64_t n_rows) {
+bool dequant_d128_applies(const tq_ctx& ctx, int64_t n_rows, int out_is_bf16) {
   if (ctx.d_in != ctx.d) return false;                   // padded rows use the general kernel
   const KParams& P = ctx.kp;
-  return P.d == kD && P.m == kM && P.B >= 1 && P.B <= 4 && n_rows > 0 && n_rows < (int64_t(1) << 31) &&
-         ctx.use_tc && tensor_map_encoder() != nullptr;
+  // d = m = 128 (bf16 or fp32 output), or d = m = 64 with bf16 output (the
+  // 64-channel parts of a split row)
+  const bool shape = (P.d == 128 && P.m == 128) || (P.d == 64 && P.m == 64 && out_is_bf16);
+  return shape && P.B >= 1 && P.B <= 4 && n_rows > 0 && n_rows < (int64_t(1) << 31) && ctx.use_tc &&
+         tensor_map_encoder() != nullptr;
 }
 
-int launch_dequant_d128(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
-                        void* stream) {
+int launch_dequant_d128(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int64_t ld_out,
+                        int out_is_bf16, int prod, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (ctx.kp.B) {
-    case 1: return launch_B<1>(ctx, in, n_rows, out, out_is_bf16, prod, s);
-    case 2: return launch_B<2>(ctx, in, n_rows, out, out_is_bf16, prod, s);
-    case 3: return launch_B<3>(ctx, in, n_rows, out, out_is_bf16, prod, s);
-    default: return launch_B<4>(ctx, in, n_rows, out, out_is_bf16, prod, s);
+    case 1: return launch_B<1>(ctx, in, n_rows, out, ld_out, out_is_bf16, prod, s);
+    case 2: return launch_B<2>(ctx, in, n_rows, out, ld_out, out_is_bf16, prod, s);
+    case 3: return launch_B<3>(ctx, in, n_rows, out, ld_out, out_is_bf16, prod, s);
+    default: return launch_B<4>(ctx, in, n_rows, out, ld_out, out_is_bf16, prod, s);
   }
 }
 

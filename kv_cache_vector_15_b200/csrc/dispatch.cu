@@ -40,8 +40,8 @@ int launch_logits(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, con
 int launch_dequant(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
                    void* stream) {
   if (take_injected_launch_failure()) return static_cast<int>(cudaErrorLaunchFailure);
-  if (dequant_d128_applies(ctx, n_rows))
-    return launch_dequant_d128(ctx, in, n_rows, out, out_is_bf16, prod, stream);
+  if (dequant_d128_applies(ctx, n_rows, out_is_bf16))
+    return launch_dequant_d128(ctx, in, n_rows, out, ctx.d, out_is_bf16, prod, stream);
   return launch_dequant_generic(ctx.kp, in, n_rows, out, out_is_bf16, prod, stream);
 }
 

@@ -178,7 +178,14 @@ tq_status tq_split_dequant(const tq_split* sp, tq_packed in_hi, tq_packed in_lo,
     P.ld_out = sp->d;                                  // into the part's columns of [n_rows, d]
     const Packed pk{in[p]->codes, in[p]->signs, in[p]->norm, in[p]->rnorm};
     void* o = static_cast<uint8_t*>(out) + (p == 0 ? 0 : static_cast<size_t>(sp->d_hi) * esize(out_dtype));
-    const int err = launch_dequant_generic(P, pk, n_rows, o, out_dtype == TQ_BF16, mode == TQ_DEQUANT_PROD, stream);
+    const bool bf16 = out_dtype == TQ_BF16, prod = mode == TQ_DEQUANT_PROD;
+    // the tensor-core kernel stores through TMA: the part's columns start on a
+    // 16-byte boundary and the row stride is a multiple of 16 bytes
+    const size_t esz = esize(out_dtype);
+    const bool tc = dequant_d128_applies(*sp->part[p], n_rows, bf16) &&
+                    (reinterpret_cast<uintptr_t>(o) & 15) == 0 && (static_cast<size_t>(sp->d) * esz) % 16 == 0;
+    const int err = tc ? launch_dequant_d128(*sp->part[p], pk, n_rows, o, sp->d, bf16, prod, stream)
+                       : launch_dequant_generic(P, pk, n_rows, o, bf16, prod, stream);
     if (err) return cuda_err(err, "tq_split_dequant launch");
   }
   return TQ_OK;

@@ -99,12 +99,14 @@ bool quantize_d128_applies(const tq_ctx& ctx, int64_t n_rows, int x_is_bf16);   
 size_t quantize_d128_scratch_bytes(const tq_ctx& ctx, int64_t n_rows);   // deferred sign fix-up list
 int launch_quantize_d128(const tq_ctx& ctx, const void* x, int x_is_bf16, int64_t n_rows, int64_t ld,
                          const Packed& out, void* scratch, void* stream);
-bool dequant_d128_applies(const tq_ctx& ctx, int64_t n_rows);
+bool dequant_d128_applies(const tq_ctx& ctx, int64_t n_rows, int out_is_bf16);
 bool logits_d128_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_keys);
 int launch_logits_d128(const tq_ctx& ctx, const float* qp, int64_t n_sets, int g, const Packed& keys, int64_t n_keys,
                        float* out, void* stream);
-int launch_dequant_d128(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int out_is_bf16, int prod,
-                        void* stream);
+// out: rows of ld_out elements (ld_out >= d; the parts of a split row write
+// into their columns of the full row)
+int launch_dequant_d128(const tq_ctx& ctx, const Packed& in, int64_t n_rows, void* out, int64_t ld_out,
+                        int out_is_bf16, int prod, void* stream);
 // wide rows (d >= 256): tensor-core QJL projection and estimates (wide_tc.cu);
 // their scratch is part of the caller's workspace
 bool wide_quantize_applies(const tq_ctx& ctx, int64_t n_rows);

@@ -183,7 +183,9 @@ def test_end_to_end_quantize_then_logits(tq, d, b, m):
 
 @pytest.mark.parametrize("d,b,m,n", [(128, 3, 128, 1029), (128, 4, 128, 1029), (128, 2, 128, 1029),
                                      (64, 5, 32, 1029), (1024, 4, 1024, 1029), (4096, 3, 64, 130),
-                                     (128, 3, 128, 77777), (128, 5, 128, 40001)])
+                                     (128, 3, 128, 77777), (128, 5, 128, 40001),
+                                     (64, 2, 64, 1029), (64, 3, 64, 40001), (64, 4, 64, 40001),
+                                     (64, 5, 64, 1029)])
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 def test_dequant_parity_on_oracle_packed_rows(tq, d, b, m, n, mode, out):

@@ -72,9 +72,14 @@ def test_split_end_to_end(tq, d, d_hi, b_hi, b_lo, dtype, n):
     tol = parity.logit_tolerance(q, np.linalg.norm(x[:n_sets * n_keys], axis=1), n_sets, g, n_keys)
     assert np.all(np.abs(lg - lw) <= tol + 1e-30), float(np.max(np.abs(lg - lw) / (tol + 1e-30)))
     for mode in (tq.TQ_DEQUANT_PROD, tq.TQ_DEQUANT_MSE):
+        want_dq = ot.split_dequant(po, parts, mode)
         dq = T.dequant(keys, out_dtype=torch.float32, mode=mode).cpu().numpy()
         assert dq.shape == (n_sets * n_keys, d)
-        parity.assert_dequant_ok(dq, ot.split_dequant(po, parts, mode), bf16=False)
+        parity.assert_dequant_ok(dq, want_dq, bf16=False)
+        # bf16 rows: 64-channel parts go through the tensor-core kernel, each
+        # storing into its columns of the full rows
+        dqb = T.dequant(keys, out_dtype=torch.bfloat16, mode=mode).float().cpu().numpy()
+        parity.assert_dequant_ok(dqb, want_dq, bf16=True)
 
 
 def test_split_argument_errors(tq):
