@@ -33,9 +33,7 @@
 // max_j ||S_j||_1 * 2^-25 / 64 (binary16 underflow); the rare projections
 // below it are recomputed: by the fp32 kernel in fp32 on the CUDA cores from
 // hi + lo, and for the bf16 kernel in fp64 from the input row by the fix-up
-// kernel that runs after it.  The bf16 kernel splits r by Veltkamp's method
-// (hi = r rounded to 11 bits, lo = r - hi exactly, both then binary16), which
-// keeps the same bound, and decides each code bit from the sign of T^2 - y^2
+// kernel that runs after it.  The bf16 kernel decides each code bit from the sign of T^2 - y^2
 // computed with one rounding (the threshold moves by at most about one ulp).
 //
 // Every mbarrier wait is bounded (about one second); a wait that runs out
@@ -1080,12 +1078,9 @@ k_quantize_d128_ws(const __grid_constant__ CUtensorMap tmap, const KParams P, co
           const int e0 = g8 * 16 + 2 * q;
           const float2 rv = quant_pair<B>(__uint_as_float(u[e0]), __uint_as_float(u[e0 + 1]), T2, nc, sc, cw, B * e0);
           if (q & 1) r2a = __ffma2_rn(rv, rv, r2a); else r2b = __ffma2_rn(rv, rv, r2b);
-          // hi = r rounded to 11 significant bits by Veltkamp's split (c = (2^13 + 1) r,
-          // hi = c - (c - r)), exact in binary16 in its normal range; lo = r - hi exactly
-          const float2 c = __fmul2_rn(rv, make_float2(8193.f, 8193.f));
-          const float2 hv = __ffma2_rn(__ffma2_rn(rv, make_float2(-1.f, -1.f), c), make_float2(-1.f, -1.f), c);
-          const float2 lf = __ffma2_rn(hv, make_float2(-1.f, -1.f), rv);
-          const __half2 h = __floats2half2_rn(hv.x, hv.y);
+          // hi = r rounded to binary16, lo = r - hi (exact in fp32), then rounded to binary16
+          const __half2 h = __floats2half2_rn(rv.x, rv.y);
+          const float2 lf = __ffma2_rn(__half22float2(h), make_float2(-1.f, -1.f), rv);
           const __half2 l = __floats2half2_rn(lf.x, lf.y);
           hw[q] = *reinterpret_cast<const uint32_t*>(&h);
           lw[q] = *reinterpret_cast<const uint32_t*>(&l);
