@@ -554,51 +554,138 @@ k_topk_row(const float* __restrict__ scores, int64_t cols, int k, int32_t* __res
 }
 
 // ---------------------------------------------------------------------------
-// bf16 unquantized-key logits: 8 lanes per key, fp32 accumulation
+// bf16 unquantized-key logits (the comparison kernel).  L = d / 8 lanes share a
+// key, each holding 8 of its coordinates; a warp covers 32 / L keys per step and
+// kBfSteps steps per chunk.  Every lane prefetches its own 16-byte pieces of the
+// next kBfStages - 1 chunks into shared memory with cp.async, so the bytes in
+// flight cost no registers and no lane waits on another; the kBfSteps * G partial
+// dot products of a chunk are then summed across the L lanes by transposing
+// butterflies (each level halves the number of values a lane holds).
 // ---------------------------------------------------------------------------
-template <int DL, int G>     // DL = d / 8 elements per lane
-__global__ void __launch_bounds__(256)
-k_logits_bf16(const uint16_t* __restrict__ q, const uint16_t* __restrict__ keys, int64_t n_keys,
-              float* __restrict__ out) {
-  const int d = DL * 8;
-  const int sub = threadIdx.x & 7;
-  const int64_t set = blockIdx.y;
-  float qr[G][DL];
+constexpr int kBfWarps = 8, kBfStages = 4, kBfSteps = 4;
+constexpr int kBfSmem = kBfWarps * kBfStages * kBfSteps * 32 * 16;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// C values per lane, lane-mask level M.  Lanes with bit M set keep the upper half
+// of their values and send the lower half, the others the reverse; once a lane holds
+// one value the remaining levels are plain butterflies (recorded in plain).
+template <int C, int M>
+struct XposeSum {
+  static __device__ __forceinline__ void run(float* a, int r, int& jbase, int& plain) {
+    if constexpr (M > 0) {
+      if constexpr (C > 1) {
+        const bool hi = (r & M) != 0;
 #pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < DL; ++e)
-      qr[g][e] = __uint_as_float(static_cast<uint32_t>(__ldg(q + (set * G + g) * d + sub * DL + e)) << 16);
-  const int64_t keys_per_iter = static_cast<int64_t>(gridDim.x) * (blockDim.x / 8);
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 8) + (threadIdx.x >> 3); t < n_keys;
-       t += keys_per_iter) {
-    const uint4* kp = reinterpret_cast<const uint4*>(keys + (set * n_keys + t) * d + sub * DL);
-    float acc[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) acc[g] = 0.f;
-#pragma unroll
-    for (int v = 0; v < DL / 8; ++v) {
-      const uint4 u = __ldg(kp + v);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float lo = __uint_as_float(w[h] << 16), hi = __uint_as_float(w[h] & 0xffff0000u);
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          acc[g] = fmaf(qr[g][v * 8 + 2 * h], lo, acc[g]);
-          acc[g] = fmaf(qr[g][v * 8 + 2 * h + 1], hi, acc[g]);
+        for (int i = 0; i < C / 2; ++i) {
+          const float keep = hi ? a[i + C / 2] : a[i];
+          const float send = hi ? a[i] : a[i + C / 2];
+          a[i] = keep + __shfl_xor_sync(0xffffffffu, send, M);
         }
+        if (hi) jbase += C / 2;
+        XposeSum<C / 2, M / 2>::run(a, r, jbase, plain);
+      } else {
+        a[0] += __shfl_xor_sync(0xffffffffu, a[0], M);
+        plain |= M;
+        XposeSum<1, M / 2>::run(a, r, jbase, plain);
+      }
+    }
+  }
+};
+
+template <int L, int G>
+__global__ void __launch_bounds__(kBfWarps * 32, 2)
+k_logits_bf16(const uint16_t* __restrict__ q, const uint16_t* __restrict__ keys, int64_t n_sets, int64_t n_keys,
+              int64_t per_warp, float* __restrict__ out) {
+  constexpr int d = 8 * L, KPS = 32 / L, KW = kBfSteps * KPS;
+  constexpr int V = kBfSteps * G, VP = V <= 4 ? 4 : V <= 8 ? 8 : V <= 16 ? 16 : 32;
+  constexpr int kLeft = VP >= L ? VP / L : 1;       // values a lane holds after the sums
+  extern __shared__ uint4 bf_sbuf[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane % L, ks = lane / L;
+  // [warp][stage][step][lane]: each lane reads back only the pieces it copied itself
+  const uint4* mine = bf_sbuf + warp * (kBfStages * kBfSteps * 32) + lane;
+  const uint32_t mine_s = static_cast<uint32_t>(__cvta_generic_to_shared(mine));
+  // the warp takes chunks [c0, c0 + n_mine) of the (set, key chunk) order; chunks do not
+  // cross sets, the last chunk of a set may be ragged
+  const int64_t cps = (n_keys + KW - 1) / KW, total = n_sets * cps;
+  const int64_t c0 = (static_cast<int64_t>(blockIdx.x) * kBfWarps + warp) * per_warp;
+  if (c0 >= total) return;                           // uniform over the warp
+  const int n_mine = static_cast<int>(c0 + per_warp < total ? per_warp : total - c0);
+  // copy cursor: key ikb of the current set, at row ip (set rows are contiguous, so the
+  // row pointer runs on across a set boundary); compute cursor: key ckb of set cset
+  const int64_t set0 = c0 / cps;
+  int64_t ikb = (c0 - set0 * cps) * KW, ckb = ikb, cset = set0;
+  const uint16_t* ip = keys + (set0 * n_keys + ikb) * d + r * 8;
+  float* op = out + set0 * G * n_keys;
+
+  auto issue = [&](int i, int stage) {
+    if (i < n_mine) {
+#pragma unroll
+      for (int u = 0; u < kBfSteps; ++u) {
+        const bool ok = ikb + u * KPS + ks < n_keys;   // else zero-fill, nothing read
+        cp_async16(mine_s + (stage * kBfSteps + u) * 512, ip + (ok ? (u * KPS + ks) * d : 0), ok ? 16u : 0u);
+      }
+      if (ikb + KW >= n_keys) { ip += (n_keys - ikb) * d; ikb = 0; } else { ip += KW * d; ikb += KW; }
+    }
+    cp_async_commit();                               // one group per chunk slot, empty past the end
+  };
+
+#pragma unroll
+  for (int i = 0; i < kBfStages - 1; ++i) issue(i, i);
+  float2 q2[G][4];
+  int64_t qset = -1;
+  int stage = 0;
+  for (int i = 0; i < n_mine; ++i) {
+    issue(i + kBfStages - 1, stage == 0 ? kBfStages - 1 : stage - 1);
+    cp_async_wait<kBfStages - 1>();                  // this lane's copies of chunk i have landed
+    if (cset != qset) {
+      qset = cset;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const uint4 qq = __ldg(reinterpret_cast<const uint4*>(q + (cset * G + g) * d + r * 8));
+        const uint32_t w[4] = {qq.x, qq.y, qq.z, qq.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+          q2[g][h] = make_float2(__uint_as_float(w[h] << 16), __uint_as_float(w[h] & 0xffff0000u));
+      }
+    }
+    float a[VP];
+#pragma unroll
+    for (int u = 0; u < kBfSteps; ++u) {
+      const uint4 kk = mine[(stage * kBfSteps + u) * 32];
+      const uint32_t w[4] = {kk.x, kk.y, kk.z, kk.w};
+      float2 kf[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) kf[h] = make_float2(__uint_as_float(w[h] << 16), __uint_as_float(w[h] & 0xffff0000u));
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float2 acc = __fmul2_rn(q2[g][0], kf[0]);
+#pragma unroll
+        for (int h = 1; h < 4; ++h) acc = __ffma2_rn(q2[g][h], kf[h], acc);
+        a[u * G + g] = acc.x + acc.y;
       }
     }
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float a = acc[g];
-      a += __shfl_xor_sync(0xffffffffu, a, 1);
-      a += __shfl_xor_sync(0xffffffffu, a, 2);
-      a += __shfl_xor_sync(0xffffffffu, a, 4);
-      if (sub == g) out[(set * G + g) * n_keys + t] = a;
+    for (int j = V; j < VP; ++j) a[j] = 0.f;
+    int jbase = 0, plain = 0;
+    XposeSum<VP, L / 2>::run(a, r, jbase, plain);
+    if ((r & plain) == 0) {
+#pragma unroll
+      for (int k = 0; k < kLeft; ++k) {
+        const int j = jbase + k;                     // value j: step j / G, query j % G
+        const int64_t t = ckb + (j / G) * KPS + ks;
+        if (j < V && t < n_keys) op[(j % G) * n_keys + t] = a[k];
+      }
     }
+    if (ckb + KW >= n_keys) { ckb = 0; ++cset; op += G * n_keys; } else { ckb += KW; }
+    stage = stage == kBfStages - 1 ? 0 : stage + 1;
   }
+  cp_async_wait<0>();
 }
 
 int sm_count() {
@@ -710,28 +797,35 @@ int launch_rowkey_B(const KParams& P, const float* qp, int64_t n_sets, int g, in
   }
 }
 
-template <int DL>
-int launch_bf16_DL(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, float* out,
-                   cudaStream_t s) {
-  const int64_t blocks_per_set_want = (n_keys + 31) / 32;
-  int64_t cap = (static_cast<int64_t>(sm_count()) * 8 + n_sets - 1) / n_sets;
-  if (cap < 1) cap = 1;
-  dim3 grid(static_cast<unsigned>(blocks_per_set_want < cap ? blocks_per_set_want : cap),
-            static_cast<unsigned>(n_sets));
-  const uint16_t* qq = static_cast<const uint16_t*>(q);
-  const uint16_t* kk = static_cast<const uint16_t*>(keys);
-  switch (g) {
-    case 1: k_logits_bf16<DL, 1><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
-    case 2: k_logits_bf16<DL, 2><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
-    case 3: k_logits_bf16<DL, 3><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
-    case 4: k_logits_bf16<DL, 4><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
-    case 5: k_logits_bf16<DL, 5><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
-    case 6: k_logits_bf16<DL, 6><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
-    case 7: k_logits_bf16<DL, 7><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
-    default: k_logits_bf16<DL, 8><<<grid, 256, 0, s>>>(qq, kk, n_keys, out); break;
-  }
+template <int L, int G>
+int launch_bf16_LG(const void* q, const void* keys, int64_t n_sets, int64_t n_keys, float* out, cudaStream_t s) {
+  constexpr int64_t KW = kBfSteps * (32 / L);
+  const int64_t total = n_sets * ((n_keys + KW - 1) / KW);
+  int64_t warps = static_cast<int64_t>(sm_count()) * 2 * kBfWarps;
+  if (warps > total) warps = total;
+  const int64_t per_warp = (total + warps - 1) / warps;
+  const int64_t blocks = ((total + per_warp - 1) / per_warp + kBfWarps - 1) / kBfWarps;
+  int err = set_smem(k_logits_bf16<L, G>, kBfSmem);
+  if (err) return err;
+  k_logits_bf16<L, G><<<static_cast<unsigned>(blocks), kBfWarps * 32, kBfSmem, s>>>(
+      static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(keys), n_sets, n_keys, per_warp, out);
   count_launch();
   return static_cast<int>(cudaGetLastError());
+}
+
+template <int L>
+int launch_bf16_L(const void* q, const void* keys, int64_t n_sets, int g, int64_t n_keys, float* out,
+                  cudaStream_t s) {
+  switch (g) {
+    case 1: return launch_bf16_LG<L, 1>(q, keys, n_sets, n_keys, out, s);
+    case 2: return launch_bf16_LG<L, 2>(q, keys, n_sets, n_keys, out, s);
+    case 3: return launch_bf16_LG<L, 3>(q, keys, n_sets, n_keys, out, s);
+    case 4: return launch_bf16_LG<L, 4>(q, keys, n_sets, n_keys, out, s);
+    case 5: return launch_bf16_LG<L, 5>(q, keys, n_sets, n_keys, out, s);
+    case 6: return launch_bf16_LG<L, 6>(q, keys, n_sets, n_keys, out, s);
+    case 7: return launch_bf16_LG<L, 7>(q, keys, n_sets, n_keys, out, s);
+    default: return launch_bf16_LG<L, 8>(q, keys, n_sets, n_keys, out, s);
+  }
 }
 
 }  // namespace
@@ -859,9 +953,9 @@ int launch_logits_bf16(const void* q, const void* keys, int64_t n_sets, int g, i
                        void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d) {
-    case 64: return launch_bf16_DL<8>(q, keys, n_sets, g, n_keys, out, s);
-    case 128: return launch_bf16_DL<16>(q, keys, n_sets, g, n_keys, out, s);
-    case 256: return launch_bf16_DL<32>(q, keys, n_sets, g, n_keys, out, s);
+    case 64: return launch_bf16_L<8>(q, keys, n_sets, g, n_keys, out, s);
+    case 128: return launch_bf16_L<16>(q, keys, n_sets, g, n_keys, out, s);
+    case 256: return launch_bf16_L<32>(q, keys, n_sets, g, n_keys, out, s);
   }
   return static_cast<int>(cudaErrorInvalidValue);
 }

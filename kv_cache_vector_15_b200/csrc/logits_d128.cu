@@ -65,6 +65,17 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// K-steps [K0, K1) of a 128-key tile into one accumulator: A (0/1 bytes) from the
+// tile's TMEM columns, B from rows of the query operand (N rows per 128-byte K atom)
+template <int K0, int K1, int N>
+__device__ __forceinline__ void mma_chain(uint32_t d_tmem, uint32_t a_tmem, uint32_t sbase, uint32_t idesc) {
+#pragma unroll
+  for (int k = K0; k < K1; ++k) {
+    const uint64_t bdesc = smem_desc_sw128(sbase + (k >> 2) * (N * 128) + (k & 3) * 32, 1024);
+    mma_i8_ts(d_tmem, a_tmem + k * 8, bdesc, idesc, k > K0 ? 1u : 0u);
+  }
+}
+
 template <int B>
 struct Shape {
   static constexpr int kCodeWords = B * 4;                  // 32-bit words of codes per key
@@ -78,6 +89,13 @@ struct Shape {
   static constexpr int kKBlocks = kK / 128;                 // 128-byte swizzle atoms along K
   static constexpr int kKSteps = kK / 32;
   static constexpr int kStageBytes = kTile * (kCodeBytes + 16);   // one tile's codes | signs
+  // K-steps of the code (and parity) planes, then 4 of the sign plane.  They run as
+  // separate MMA chains issued by different warps (one thread issues an MMA only every
+  // few dozen cycles): the code steps against the N / 2 code-limb rows of the query
+  // operand, the sign steps against the sign-limb rows, and for 3-bit codes the code
+  // steps split once more into a second accumulator of their own.
+  static constexpr int kMseSteps = kCodeWords + kParWords;
+  static constexpr int kChains = B == 3 ? 3 : 2;
 };
 
 constexpr int kStages = 4;                   // packed tiles in flight per warpgroup
@@ -155,7 +173,7 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
 
   if (tid == 0) {
     for (int i = 0; i < kWG * kStages; ++i) mbar_init(&bars[i], 1);
-    for (int i = 0; i < kWG; ++i) mbar_init(&mdone[i], 1);
+    for (int i = 0; i < kWG; ++i) mbar_init(&mdone[i], S::kChains);   // one commit per chain
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -170,6 +188,8 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
   const bool leader = (wl == 0 && lane == 0);
   const int trow = wl * 32 + lane;
   const uint32_t t_base = tmem + (static_cast<uint32_t>(wl * 32) << 16) + wg * S::kColsPerWG;   // my lane
+  // A columns, then the accumulator: N columns (code limbs | sign limbs), and for
+  // 3-bit codes NG more for the second half of the code steps
   const uint32_t t_a = t_base, t_d = t_base + S::kAWords;
 
   // contiguous tile range of this warpgroup; (set, key tile) advance incrementally
@@ -369,17 +389,16 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
     tc_fence_before();
     // every thread has read its key from the stage and written its TMEM row
     if (named_bar_sync_or(1 + wg, 128, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
-    if (leader) {
-      if (issued < n_mine) issue(stage);
+    if (leader && issued < n_mine) issue(stage);
+    if (lane == 0 && wl < S::kChains) {
+      // chain wl: 0 = code steps [0, h), 1 = sign steps, 2 = code steps [h, kMseSteps)
+      constexpr int h = S::kChains == 3 ? S::kMseSteps / 2 : S::kMseSteps;
       tc_fence_after();
-      const uint32_t sbase = smem_u32(sB);
-      const uint32_t idesc = idesc_i8(kTile, N);
-      const uint32_t d_tmem = tmem + wg * S::kColsPerWG + S::kAWords;
-#pragma unroll
-      for (int k = 0; k < S::kKSteps; ++k) {
-        const uint64_t bdesc = smem_desc_sw128(sbase + (k >> 2) * (N * 128) + (k & 3) * 32, 1024);
-        mma_i8_ts(d_tmem, tmem + wg * S::kColsPerWG + k * 8, bdesc, idesc, k > 0 ? 1u : 0u);
-      }
+      const uint32_t a_tmem = tmem + wg * S::kColsPerWG, d_tmem = a_tmem + S::kAWords;
+      const uint32_t sbase = smem_u32(sB), idesc = idesc_i8(kTile, NG);
+      if (wl == 0) mma_chain<0, h, N>(d_tmem, a_tmem, sbase, idesc);
+      else if (wl == 1) mma_chain<S::kMseSteps, S::kKSteps, N>(d_tmem + NG, a_tmem, sbase + NG * 128, idesc);
+      else mma_chain<h, S::kMseSteps, N>(d_tmem + N, a_tmem, sbase, idesc);
       mma_commit(&mdone[wg]);
     }
     if (!mbar_wait(&mdone[wg], static_cast<uint32_t>(i & 1), X.wait_cycles)) {
@@ -397,6 +416,21 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
         tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 32; ++k) acc[32 * c + k] = part[k];
+      }
+      if constexpr (S::kChains == 3) {
+        // the second code accumulator joins the first exactly (integer limbs)
+        if constexpr (NG == 16) {
+          uint32_t p16[16];
+          tmem_ld16(t_d + N, p16);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 16; ++k) acc[k] += p16[k];
+        } else {
+          tmem_ld32(t_d + N, part);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) acc[k] += part[k];
+        }
       }
     }
     tc_fence_before();
@@ -517,7 +551,8 @@ bool logits_d128_applies(const tq_ctx& ctx, int64_t n_sets, int g, int64_t n_key
         ctx.use_tc))
     return false;
   // the A operand and the accumulator share a warpgroup's TMEM columns
-  const int a_cols = 8 * (P.B * 4 + (P.B == 3 ? 4 : 0) + 4), n_cols = (4 * g <= 16) ? 32 : 64;
+  const int ng = (4 * g <= 16) ? 16 : 32;
+  const int a_cols = 8 * (P.B * 4 + (P.B == 3 ? 4 : 0) + 4), n_cols = (P.B == 3 ? 3 : 2) * ng;
   const int cols = P.B == 3 ? 256 : 128;
   if (a_cols + n_cols > cols) return false;
   if (P.B == 3) {                       // the bit-plane form needs a symmetric codebook

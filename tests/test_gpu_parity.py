@@ -213,9 +213,11 @@ def test_topk_parity_with_ties(tq, rows, cols, k):
     assert np.array_equal(val.cpu().numpy(), wv)
 
 
-@pytest.mark.parametrize("d,g", [(128, 4), (64, 1), (256, 8), (128, 3)])
-def test_bf16_baseline_logits(tq, d, g):
-    n_sets, n_keys = 3, 2049
+@pytest.mark.parametrize("d,g,n_sets,n_keys", [(128, 4, 3, 2049), (64, 1, 3, 2049), (256, 8, 3, 2049),
+                                               (128, 3, 3, 2049), (128, 2, 700, 5), (64, 8, 50, 3001),
+                                               (256, 5, 9, 77), (128, 4, 1, 1)])
+def test_bf16_baseline_logits(tq, d, g, n_sets, n_keys):
+    """Ragged key chunks: n_keys below one chunk (set boundaries inside one warp's range), one key."""
     kt, k = make_rows(d, n_sets * n_keys, "bf16", seed=d + g)
     qt, q = make_rows(d, n_sets * g, "bf16", seed=d * g)
     got = tq.logits_bf16(qt.cuda(), kt.cuda(), n_sets, g, n_keys).cpu().numpy()
