@@ -73,7 +73,7 @@ METRIC = "compressed-key logits/s and % HBM roofline (d=128,b=3); quantize rows/
 UNIT = "logits/s"
 
 
-KERNEL_OF = {"quantize": "k_quantize_d128_ws", "logits": "k_logits_d128_i8", "dequant": "k_dequant_d128_ovl"}
+KERNEL_OF = {"quantize": "k_quantize_d128_ws", "logits": "k_logits_d128_ws", "dequant": "k_dequant_d128_ovl"}
 
 
 def captured_traffic(kernel: str, b: int, units: int):

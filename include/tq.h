@@ -313,14 +313,17 @@ tq_status tq_split_dequant(const tq_split* sp, tq_packed in_hi, tq_packed in_lo,
  * own failure tests, not for production use).  Injected failures happen on
  * the host: no GPU fault is provoked.
  *   TQ_TEST_WAIT_LIMIT   limit, in SM clock cycles, of the bounded mbarrier
- *                        waits in the tile loop of the d = 128 tensor-core
- *                        quantize kernel (0 restores the default, about one
- *                        second).  A limit shorter than the work makes the
- *                        kernel give up: it stops, waits (with the default
- *                        limit) for its own MMAs and stage loads, frees its
- *                        tensor memory, writes no results and leaves an
- *                        error that tq_sync_status reports as TQ_ERR_CUDA.
- *                        Applies to launches made after the call.
+ *                        waits in the tile loops of the d = 128 tensor-core
+ *                        kernels (quantize, logits, dequant; 0 restores the
+ *                        default, about one second).  A limit shorter than the
+ *                        work makes a kernel give up: it stops, waits (with
+ *                        the default limit) for its own MMAs and stage loads,
+ *                        frees its tensor memory and leaves an error that
+ *                        tq_sync_status reports as TQ_ERR_CUDA (the quantize
+ *                        kernel, whose first wait gives up, writes no
+ *                        results; the logits and dequant kernels may have
+ *                        written some before they gave up).  Applies to
+ *                        launches made after the call.
  *   TQ_TEST_FAIL_ALLOC   the next `value` device allocations of tq_init fail
  *                        as if the device were out of memory (TQ_ERR_NOMEM,
  *                        nothing leaked).

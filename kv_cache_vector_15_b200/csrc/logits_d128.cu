@@ -23,11 +23,15 @@
 // 8-bit limbs of a fixed-point value per (bit, query).  The epilogue recombines
 // the limbs, adds the constants and applies norm and rnorm.
 //
-// Work split: persistent CTAs of four warpgroups (two for 3-bit codes, whose
-// wider operand takes 160 of a warpgroup's TMEM columns); each warpgroup walks
-// a contiguous range of 128-key tiles (so the set, and with it the query
-// operand it builds in its own shared-memory slot, changes rarely), one thread
-// per key.
+// Work split, two forms.  Warp-specialized (k_logits_d128_ws, used whenever
+// every CTA's contiguous range of 128-key tiles spans at most two sets):
+// decode, MMA-issue and epilogue warps pass tiles through four (two for 3-bit
+// codes) TMEM slots.  General (k_logits_d128_i8): persistent CTAs of four
+// warpgroups (two for 3-bit codes, whose wider operand takes 160 of a
+// warpgroup's TMEM columns); each warpgroup walks a contiguous range of tiles
+// (so the set, and with it the query operand it builds in its own
+// shared-memory slot, changes rarely), one thread per key, decode, MMAs and
+// epilogue in turn.
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -150,6 +154,117 @@ __device__ __forceinline__ uint32_t code_parities(uint32_t w0, uint32_t w1, uint
   return every_third_bit(x0) | (every_third_bit(x1 >> 1) << 11) | ((every_third_bit(x2 >> 2) & 0x3FFu) << 22);
 }
 
+// The query operand of one set in shared memory, built by the 128 threads of
+// a warpgroup (thread trow = 32 wl + lane owns coordinate / projection trow):
+// per (K position, query) the fixed-point value as four signed 8-bit limbs in
+// the MMA's B layout (N rows of 128-byte K atoms, swizzled), plus the per-query
+// constants and inverse scales in sScal (partial maxima at 0, partial sums at
+// 64, constants at 128, inverse scales at 144).  Ends with the operand visible
+// to the tensor cores and a barrier of the 128 threads.
+template <int B, int G, int NG>
+__device__ __forceinline__ void build_query_operand(const LogitsArgs& X, const float* __restrict__ qs, int trow,
+                                                    int wl, int lane, float* sScal, uint8_t* sB, uint32_t bar_id) {
+  using S = Shape<B>;
+  constexpr int N = 2 * NG;
+  // per-warp maxima and sums of every query's two halves, combined below in a
+  // fixed order (thread trow owns coordinate / projection trow)
+  float* sPM = sScal;                               // [warp][2G] partial maxima
+  float* sPS = sScal + 64;                          // [warp][2G] partial sums
+  float* sC = sScal + 128;                          // [2G] constant terms
+  float* sInv = sScal + 144;                        // [2G] inverse fixed-point scales
+#pragma unroll
+  for (int q = 0; q < G; ++q) {
+    const float va = qs[q * (kD + kM) + trow], vb = qs[q * (kD + kM) + kD + trow];
+    float a = fabsf(va), b = fabsf(vb), sa = va, sb = vb;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
+      sa += __shfl_xor_sync(0xffffffffu, sa, o);
+      sb += __shfl_xor_sync(0xffffffffu, sb, o);
+    }
+    if (lane == 0) {
+      sPM[wl * 16 + q] = a;
+      sPM[wl * 16 + G + q] = b;
+      sPS[wl * 16 + q] = sa;
+      sPS[wl * 16 + G + q] = sb;
+    }
+  }
+  named_bar_sync(bar_id, 128);
+  float wmax = fabsf(X.wbit[0]);
+  if (B >= 2) wmax = fmaxf(wmax, fabsf(X.wbit[1]));
+  if (B == 3) wmax = fmaxf(wmax, fmaxf(fabsf(X.wbit[2]), fabsf(X.wpar)));
+  // fixed-point exponent of half h of query q: |value| * 2^F <= 2^22
+  auto fp_exp = [&](int h, int q) {
+    const int i = h * G + q;
+    const float m = fmaxf(fmaxf(sPM[i], sPM[16 + i]), fmaxf(sPM[32 + i], sPM[48 + i]));
+    const float v = h == 0 ? m * wmax : m * 2.f;
+    int e = 0;
+    frexpf(v > 0.f ? v : 1.f, &e);
+    return 22 - e;
+  };
+  int fe[2 * G];
+#pragma unroll
+  for (int q = 0; q < G; ++q) {
+    fe[q] = fp_exp(0, q);
+    fe[G + q] = fp_exp(1, q);
+  }
+  // operand bytes: K position kappa (byte t of A column o) of this thread.  Column
+  // o holds bit t * 8 + (o & 7) of a packed word at bit (o & 7) of each byte, so
+  // the byte is bit * 2^(o & 7); the query value is scaled by 2^(7 - (o & 7)) and
+  // every product carries the common factor 2^7.
+#pragma unroll
+  for (int r = 0; r < S::kK / 128; ++r) {
+    const int kappa = trow + 128 * r;
+    const int o = kappa >> 2, tb = kappa & 3;
+    const int up = 7 - (o & 7);
+    int8_t limb[N];
+#pragma unroll
+    for (int n = 0; n < N; ++n) limb[n] = 0;
+    if (o < 8 * (S::kCodeWords + S::kParWords)) {
+      int coord;
+      float w;
+      if (o < 8 * S::kCodeWords) {
+        const int c = o >> 3, k = o & 7;
+        const int s = 32 * c + k + 8 * tb;        // bit position in the code stream
+        coord = s / B;
+        w = X.wbit[s % B];
+      } else {
+        const int c = (o - 8 * S::kCodeWords) >> 3, k = o & 7;
+        coord = 32 * c + k + 8 * tb;              // parity bit of this code
+        w = X.wpar;
+      }
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        const int v = __float2int_rn(ldexpf(w * qs[q * (kD + kM) + coord], fe[q])) * (1 << up);
+        split_limbs(v, &limb[4 * q]);
+      }
+    } else {
+      const int c = (o - 8 * (S::kCodeWords + S::kParWords)) >> 3, k = o & 7;
+      const int j = 32 * c + k + 8 * tb;           // projection
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        const int v = __float2int_rn(ldexpf(-2.f * qs[q * (kD + kM) + kD + j], fe[G + q])) * (1 << up);
+        split_limbs(v, &limb[NG + 4 * q]);
+      }
+    }
+    const int kb = kappa >> 7, chunk = (kappa & 127) >> 4, within = kappa & 15;
+#pragma unroll
+    for (int n = 0; n < N; ++n)
+      sB[kb * (N * 128) + n * 128 + ((chunk ^ (n & 7)) << 4) + within] = static_cast<uint8_t>(limb[n]);
+  }
+  // per-query constants (c_const * sum q_rot, sum sq) and the inverse scales
+  // with the 2^-7 of the shifted bits
+  if (trow < 2 * G) {
+    const float sum = (sPS[trow] + sPS[16 + trow]) + (sPS[32 + trow] + sPS[48 + trow]);
+    const int h = trow >= G ? 1 : 0;
+    sC[trow] = h ? sum : X.cconst * sum;
+    sInv[trow] = ldexpf(1.f, -fp_exp(h, trow - h * G) - 7);
+  }
+  fence_proxy_async_smem();
+  named_bar_sync(bar_id, 128);
+}
+
 template <int B, int G, int NG>
 __global__ void __launch_bounds__(Shape<B>::kThreads, 1)
 k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ qp, int64_t n_sets,
@@ -243,104 +358,7 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
       // ---- build the query operand of this set --------------------------------
       cur_set = set;
       named_bar_sync(1 + wg, 128);                      // previous tile's MMA inputs no longer in use
-      // per-warp maxima and sums of every query's two halves, combined below in a
-      // fixed order (thread trow owns coordinate / projection trow)
-      float* sPM = sScal;                               // [warp][2G] partial maxima
-      float* sPS = sScal + 64;                          // [warp][2G] partial sums
-      float* sC = sScal + 128;                          // [2G] constant terms
-      float* sInv = sScal + 144;                        // [2G] inverse fixed-point scales
-      const float* qs = qp + set * G * (kD + kM);
-#pragma unroll
-      for (int q = 0; q < G; ++q) {
-        const float va = qs[q * (kD + kM) + trow], vb = qs[q * (kD + kM) + kD + trow];
-        float a = fabsf(va), b = fabsf(vb), sa = va, sb = vb;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-          b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
-          sa += __shfl_xor_sync(0xffffffffu, sa, o);
-          sb += __shfl_xor_sync(0xffffffffu, sb, o);
-        }
-        if (lane == 0) {
-          sPM[wl * 16 + q] = a;
-          sPM[wl * 16 + G + q] = b;
-          sPS[wl * 16 + q] = sa;
-          sPS[wl * 16 + G + q] = sb;
-        }
-      }
-      named_bar_sync(1 + wg, 128);
-      float wmax = fabsf(X.wbit[0]);
-      if (B >= 2) wmax = fmaxf(wmax, fabsf(X.wbit[1]));
-      if (B == 3) wmax = fmaxf(wmax, fmaxf(fabsf(X.wbit[2]), fabsf(X.wpar)));
-      // fixed-point exponent of half h of query q: |value| * 2^F <= 2^22
-      auto fp_exp = [&](int h, int q) {
-        const int i = h * G + q;
-        const float m = fmaxf(fmaxf(sPM[i], sPM[16 + i]), fmaxf(sPM[32 + i], sPM[48 + i]));
-        const float v = h == 0 ? m * wmax : m * 2.f;
-        int e = 0;
-        frexpf(v > 0.f ? v : 1.f, &e);
-        return 22 - e;
-      };
-      int fe[2 * G];
-#pragma unroll
-      for (int q = 0; q < G; ++q) {
-        fe[q] = fp_exp(0, q);
-        fe[G + q] = fp_exp(1, q);
-      }
-      // operand bytes: K position kappa (byte t of A column o) of this thread.  Column
-      // o holds bit t * 8 + (o & 7) of a packed word at bit (o & 7) of each byte, so
-      // the byte is bit * 2^(o & 7); the query value is scaled by 2^(7 - (o & 7)) and
-      // every product carries the common factor 2^7.
-#pragma unroll
-      for (int r = 0; r < S::kK / 128; ++r) {
-        const int kappa = trow + 128 * r;
-        const int o = kappa >> 2, tb = kappa & 3;
-        const int up = 7 - (o & 7);
-        int8_t limb[N];
-#pragma unroll
-        for (int n = 0; n < N; ++n) limb[n] = 0;
-        if (o < 8 * (S::kCodeWords + S::kParWords)) {
-          int coord;
-          float w;
-          if (o < 8 * S::kCodeWords) {
-            const int c = o >> 3, k = o & 7;
-            const int s = 32 * c + k + 8 * tb;        // bit position in the code stream
-            coord = s / B;
-            w = X.wbit[s % B];
-          } else {
-            const int c = (o - 8 * S::kCodeWords) >> 3, k = o & 7;
-            coord = 32 * c + k + 8 * tb;              // parity bit of this code
-            w = X.wpar;
-          }
-#pragma unroll
-          for (int q = 0; q < G; ++q) {
-            const int v = __float2int_rn(ldexpf(w * qs[q * (kD + kM) + coord], fe[q])) * (1 << up);
-            split_limbs(v, &limb[4 * q]);
-          }
-        } else {
-          const int c = (o - 8 * (S::kCodeWords + S::kParWords)) >> 3, k = o & 7;
-          const int j = 32 * c + k + 8 * tb;           // projection
-#pragma unroll
-          for (int q = 0; q < G; ++q) {
-            const int v = __float2int_rn(ldexpf(-2.f * qs[q * (kD + kM) + kD + j], fe[G + q])) * (1 << up);
-            split_limbs(v, &limb[NG + 4 * q]);
-          }
-        }
-        const int kb = kappa >> 7, chunk = (kappa & 127) >> 4, within = kappa & 15;
-#pragma unroll
-        for (int n = 0; n < N; ++n)
-          sB[kb * (N * 128) + n * 128 + ((chunk ^ (n & 7)) << 4) + within] = static_cast<uint8_t>(limb[n]);
-      }
-      // per-query constants (c_const * sum q_rot, sum sq) and the inverse scales
-      // with the 2^-7 of the shifted bits
-      if (trow < 2 * G) {
-        const float sum = (sPS[trow] + sPS[16 + trow]) + (sPS[32 + trow] + sPS[48 + trow]);
-        const int h = trow >= G ? 1 : 0;
-        sC[trow] = h ? sum : X.cconst * sum;
-        sInv[trow] = ldexpf(1.f, -fp_exp(h, trow - h * G) - 7);
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(1 + wg, 128);
+      build_query_operand<B, G, NG>(X, qp + set * G * (kD + kM), trow, wl, lane, sScal, sB, 1 + wg);
     }
     // ---- this thread's key from the stage, decoded into TMEM -----------------------
     if (mbar_wait(&full[stage], parity, X.wait_cycles)) {
@@ -464,6 +482,364 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Warp-specialized form: one CTA per SM walks a contiguous range of 128-key
+// tiles, spanning at most two sets, through kSlots TMEM slots (A columns, then
+// the accumulators), so the decode of later tiles runs while the tensor cores
+// and the epilogue work on earlier ones.  Warps, in pairs of groups that take
+// the tiles of even / odd local index:
+//   0 .. 7    two epilogue groups: accumulators -> limbs joined, constants,
+//             norms, stores; first, group e builds the query operand of the
+//             range's set e (one buffer each);
+//   8 .. 15   two decode groups: the group's leader keeps bulk copies of the
+//             group's next tiles (codes and signs) in flight in its own stages;
+//             the packed words go from the stage into TMEM 0/1 bytes;
+//   16 .. 19  MMA issuers, one thread each (a thread issues an MMA only every
+//             60 to 100 cycles, so the four issue side by side), one or two
+//             per slot: the code steps against the code-limb rows of the query
+//             operand, the sign steps against the sign-limb rows.
+// Barriers per slot: a_ready (decode -> issuers), mma_done (issuers ->
+// epilogue), slot_free (epilogue -> decode); per stage: full, stage_free; per
+// query buffer: q_ready.  Every wait is bounded and gives up once another
+// thread has flagged an abort.
+// ---------------------------------------------------------------------------
+template <int B, int NG>
+struct WsLog {
+  using S = Shape<B>;
+  static constexpr int N = 2 * NG;                                  // code limbs | sign limbs
+  // a slot: A, then the code | sign accumulators; four slots of 128 columns
+  // (one issuer each) or two of 256, each with two issuers, the code steps split
+  // between them into a second code accumulator
+  static constexpr int kSlots = S::kAWords + N <= 128 ? 4 : 2;
+  static constexpr int kSlotCols = 512 / kSlots;
+  static constexpr int kIssuersPerSlot = 4 / kSlots;
+  static constexpr int kChains = kSlots == 2 ? 3 : 2;
+  static constexpr int kStages = 6;                                 // three per decode group
+  static constexpr int kBBytes = S::kKBlocks * N * 128;
+  static constexpr int kThreads = 20 * 32;
+};
+
+template <int B, int NG>
+constexpr size_t logits_ws_smem_bytes() {
+  using W = WsLog<B, NG>;
+  return 1024 + 2 * W::kBBytes + W::kStages * Shape<B>::kStageBytes + 2 * kScalFloats * 4 +
+         (3 * W::kSlots + 2 * W::kStages + 2 + 4) * 8 + 16;
+}
+
+// bounded wait that also gives up once the abort flag is set; a long limit lets
+// the waiting thread be suspended between polls (leaving the issue slots to the
+// other warps), a short one polls and keeps to the cycle count
+__device__ __forceinline__ bool ws_wait(uint64_t* bar, uint32_t parity, long long limit, const int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const bool suspend = limit >= (1ll << 24);
+  const long long t0 = clock64();
+  for (;;) {
+    bool ok;
+    if (suspend) {
+      uint32_t r;
+      asm volatile(
+          "{\n\t.reg .pred p;\n\t"
+          "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 20000;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(r)
+          : "r"(smem_u32(bar)), "r"(parity)
+          : "memory");
+      ok = r != 0;
+    } else {
+      ok = mbar_try_wait(bar, parity);
+    }
+    if (ok) return true;
+    if (*reinterpret_cast<volatile const int*>(abort_flag) != 0) return false;
+    if (clock64() - t0 > limit) return false;
+  }
+}
+
+// (set, key tile) of local tile i, stepped forward by a few tiles at a time
+struct TileCursor {
+  int64_t set, kt, tps;
+  __device__ __forceinline__ void step(int by) {
+    kt += by;
+    while (kt >= tps) {
+      kt -= tps;
+      ++set;
+    }
+  }
+};
+
+template <int B, int G, int NG>
+__global__ void __launch_bounds__(WsLog<B, NG>::kThreads, 1)
+k_logits_d128_ws(const KParams P, const LogitsArgs X, const float* __restrict__ qp, int64_t n_sets, int64_t n_keys,
+                 const Packed keys, float* __restrict__ out) {
+  using S = Shape<B>;
+  using W = WsLog<B, NG>;
+  constexpr int N = W::N, kSlots = W::kSlots, kSt = W::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sBq = smem;                                                // [2] query operands
+  uint8_t* stages = smem + 2 * W::kBBytes;                            // [kSt] codes | signs of a tile
+  float* sScal = reinterpret_cast<float*>(stages + kSt * S::kStageBytes);   // [2][kScalFloats]
+  uint64_t* a_ready = reinterpret_cast<uint64_t*>(sScal + 2 * kScalFloats);
+  uint64_t* mma_done = a_ready + kSlots;
+  uint64_t* slot_free = mma_done + kSlots;
+  uint64_t* full = slot_free + kSlots;
+  uint64_t* stage_free = full + kSt;
+  uint64_t* q_ready = stage_free + kSt;                               // [2]
+  uint64_t* fdone = q_ready + 2;                                      // [4] issuers' wind-down
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fdone + 4);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long lim = X.wait_cycles;
+  if (tid == 0) {
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&a_ready[s], 4);
+      mbar_init(&mma_done[s], W::kIssuersPerSlot);
+      mbar_init(&slot_free[s], 4);
+    }
+    for (int i = 0; i < kSt; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&stage_free[i], 4);
+    }
+    mbar_init(&q_ready[0], 1);
+    mbar_init(&q_ready[1], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&fdone[i], 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto fail = [&](int code) {
+    if (X.err) atomicCAS(X.err, 0, code);
+    atomicExch(abort_flag, 1);
+  };
+
+  // this CTA's contiguous tile range
+  const int64_t tps = (n_keys + kTile - 1) / kTile;
+  const int64_t n_tiles = tps * n_sets;
+  const int64_t t0 = n_tiles * blockIdx.x / gridDim.x, t1 = n_tiles * (blockIdx.x + 1) / gridDim.x;
+  const int64_t set0 = t0 / tps;
+  const int64_t kt0 = t0 - set0 * tps;
+  const int64_t last_set = t1 > t0 ? (t1 - 1) / tps : set0;
+  // the launch keeps every range within two sets (one query buffer each)
+  const bool span_ok = last_set <= set0 + 1;
+  if (!span_ok && tid == 0) fail(9);
+  const int n_mine = span_ok ? static_cast<int>(t1 - t0) : 0;
+
+  if (warp < 8) {
+    // ================================ epilogue groups ================================
+    const int eg = warp >> 2, wl = warp & 3;
+    const int trow = wl * 32 + lane;
+    const uint32_t bar = 1 + eg;                                      // this group's named barrier
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wl * 32) << 16);
+    if (n_mine > 0 && set0 + eg <= last_set) {
+      build_query_operand<B, G, NG>(X, qp + (set0 + eg) * G * (kD + kM), trow, wl, lane, sScal + eg * kScalFloats,
+                                    sBq + eg * W::kBBytes, bar);
+      if (wl == 0 && lane == 0) mbar_arrive(&q_ready[eg]);
+    }
+    TileCursor c{set0, kt0, tps};
+    c.step(eg);
+    float nnrm = 0.f, nrn = 0.f;
+    auto load_norms = [&](const TileCursor& cc) {
+      const int64_t key = cc.kt * kTile + trow;
+      nnrm = nrn = 0.f;
+      if (key < n_keys) {
+        nnrm = __ldg(keys.norm + cc.set * n_keys + key);
+        nrn = __ldg(keys.rnorm + cc.set * n_keys + key);
+      }
+    };
+    if (eg < n_mine) load_norms(c);
+    for (int i = eg; i < n_mine; i += 2) {
+      const int s = i % kSlots;
+      const float nrm = nnrm, rn = nrn * P.qjl_scale;
+      TileCursor nx = c;
+      nx.step(2);
+      if (i + 2 < n_mine) load_norms(nx);
+      // the group's four warps leave together (they share a named barrier)
+      const bool ok = ws_wait(&mma_done[s], static_cast<uint32_t>((i / kSlots) & 1), lim, abort_flag);
+      if (!ok) fail(9);
+      if (named_bar_sync_or(bar, 128, !ok)) break;
+      tc_fence_after();
+      const uint32_t t_d = t_lane + s * W::kSlotCols + S::kAWords;
+      uint32_t acc[N];
+      {
+        uint32_t part[32];
+#pragma unroll
+        for (int cc = 0; cc < N / 32; ++cc) {
+          tmem_ld32(t_d + 32 * cc, part);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) acc[32 * cc + k] = part[k];
+        }
+        if constexpr (W::kChains == 3) {
+          // the second code accumulator joins the first exactly (integer limbs)
+#pragma unroll
+          for (int h = 0; h < NG / 16; ++h) {
+            uint32_t p16[16];
+            tmem_ld16(t_d + N + 16 * h, p16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) acc[16 * h + k] += p16[k];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&slot_free[s]);
+      const int64_t key = c.kt * kTile + trow;
+      if (key < n_keys) {
+        const float* sc = sScal + static_cast<int>(c.set - set0) * kScalFloats;
+        float* o = out + c.set * G * n_keys + key;
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+          const float mse = fmaf(join_limbs(&acc[4 * q]), sc[144 + q], sc[128 + q]);
+          const float qjl = fmaf(join_limbs(&acc[NG + 4 * q]), sc[144 + G + q], sc[128 + G + q]);
+          o[q * n_keys] = fmaf(nrm, mse, rn * qjl);
+        }
+      }
+      c = nx;
+    }
+  } else if (warp < 16) {
+    // ================================ decode groups ================================
+    const int grp = (warp - 8) >> 2, wl = warp & 3;
+    const int trow = wl * 32 + lane;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wl * 32) << 16);
+    const bool leader = wl == 0 && lane == 0;
+    constexpr int kGS = kSt / 2;                                      // stages of this group
+    // the leader's bulk copies of local tile m (global local index grp + 2 m) into stage grp kGS + m % kGS
+    TileCursor cl{set0, kt0, tps};
+    cl.step(grp);
+    int loads = 0;
+    auto issue_load = [&]() {
+      const int st = grp * kGS + loads % kGS;
+      const int64_t row0 = cl.set * n_keys + cl.kt * kTile;
+      const int64_t left = n_keys - cl.kt * kTile;
+      const uint32_t valid = static_cast<uint32_t>(left < kTile ? left : kTile);
+      uint8_t* sg = stages + st * S::kStageBytes;
+      mbar_arrive_expect_tx(&full[st], valid * (S::kCodeBytes + 16));
+      bulk_load(sg, keys.codes + row0 * S::kCodeBytes, valid * S::kCodeBytes, &full[st]);
+      bulk_load(sg + kTile * S::kCodeBytes, keys.signs + row0 * 16, valid * 16, &full[st]);
+      ++loads;
+      cl.step(2);
+    };
+    const int n_grp = n_mine > grp ? (n_mine - grp + 1) / 2 : 0;       // tiles of this group
+    if (leader)
+      while (loads < kGS && loads < n_grp) issue_load();
+    TileCursor c{set0, kt0, tps};
+    c.step(grp);
+    int m = 0;
+    for (int i = grp; i < n_mine; i += 2, c.step(2), ++m) {
+      const int s = i % kSlots, n = i / kSlots, st = grp * kGS + m % kGS;
+      const uint32_t sph = static_cast<uint32_t>((m / kGS) & 1);
+      if (n >= 1 && !ws_wait(&slot_free[s], static_cast<uint32_t>((n - 1) & 1), lim, abort_flag)) { fail(9); break; }
+      if (!ws_wait(&full[st], sph, lim, abort_flag)) { fail(9); break; }
+      const bool valid = c.kt * kTile + trow < n_keys;
+      uint32_t cw[S::kCodeWords + S::kParWords + 4];
+      const uint8_t* sg = stages + st * S::kStageBytes;
+      if (valid) {
+#pragma unroll
+        for (int q = 0; q < B; ++q) {
+          const uint4 u = *reinterpret_cast<const uint4*>(sg + trow * S::kCodeBytes + 16 * q);
+          cw[4 * q] = u.x; cw[4 * q + 1] = u.y; cw[4 * q + 2] = u.z; cw[4 * q + 3] = u.w;
+        }
+        const uint4 u = *reinterpret_cast<const uint4*>(sg + kTile * S::kCodeBytes + trow * 16);
+        constexpr int so = S::kCodeWords + S::kParWords;
+        cw[so] = u.x; cw[so + 1] = u.y; cw[so + 2] = u.z; cw[so + 3] = u.w;
+      } else {
+#pragma unroll
+        for (int w = 0; w < S::kCodeWords + S::kParWords + 4; ++w) cw[w] = 0u;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&stage_free[st]);
+      if constexpr (B == 3) {
+#pragma unroll
+        for (int g2 = 0; g2 < 4; ++g2)
+          cw[S::kCodeWords + g2] = code_parities(cw[3 * g2], cw[3 * g2 + 1], cw[3 * g2 + 2]);
+      }
+      const uint32_t t_a = t_lane + s * W::kSlotCols;
+      uint32_t a[32];
+      int na = 0, col = 0;
+#pragma unroll
+      for (int cc = 0; cc < S::kCodeWords + S::kParWords + 4; ++cc) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          a[na++] = cw[cc] & (0x01010101u << k);
+          if (na == 32) {
+            tmem_st32(t_a + col, a);
+            col += 32;
+            na = 0;
+          }
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_ready[s]);
+      if (leader && loads < n_grp) {
+        // refill the stage (the group's four warps read it long before their
+        // TMEM rows were written)
+        if (!ws_wait(&stage_free[st], sph, lim, abort_flag)) { fail(9); break; }
+        issue_load();
+      }
+    }
+    if (leader) {
+      // copies still in flight (only after an abort): let them land before exit
+      for (int k = loads > kGS ? loads - kGS : 0; k < loads; ++k)
+        if (!mbar_wait(&full[grp * kGS + k % kGS], static_cast<uint32_t>((k / kGS) & 1), 2000000000ll)) break;
+    }
+  } else {
+    // ================================ MMA issuers ================================
+    const int j = warp - 16, slot = j / W::kIssuersPerSlot, part = j % W::kIssuersPerSlot;
+    if (lane == 0) {
+      bool issued = false;
+      int64_t q_set = -1;
+      TileCursor c{set0, kt0, tps};
+      c.step(slot);
+      const uint32_t idesc = idesc_i8(kTile, NG);
+      const uint32_t a_tmem = tmem + slot * W::kSlotCols, d_tmem = a_tmem + S::kAWords;
+      // every use of the slot, in order (the slot's barriers complete once per use)
+      for (int i = slot; i < n_mine; i += kSlots, c.step(kSlots)) {
+        if (c.set != q_set) {
+          q_set = c.set;
+          if (!ws_wait(&q_ready[c.set - set0], 0u, lim, abort_flag)) { fail(9); break; }
+        }
+        if (!ws_wait(&a_ready[slot], static_cast<uint32_t>((i / kSlots) & 1), lim, abort_flag)) { fail(9); break; }
+        tc_fence_after();
+        const uint32_t sbase = smem_u32(sBq + static_cast<int>(c.set - set0) * W::kBBytes);
+        if constexpr (W::kIssuersPerSlot == 1) {
+          mma_chain<0, S::kMseSteps, N>(d_tmem, a_tmem, sbase, idesc);
+          mma_chain<S::kMseSteps, S::kKSteps, N>(d_tmem + NG, a_tmem, sbase + NG * 128, idesc);
+        } else {
+          constexpr int h = S::kMseSteps / 2;
+          if (part == 0) {
+            mma_chain<0, h, N>(d_tmem, a_tmem, sbase, idesc);
+          } else {
+            mma_chain<h, S::kMseSteps, N>(d_tmem + N, a_tmem, sbase, idesc);
+            mma_chain<S::kMseSteps, S::kKSteps, N>(d_tmem + NG, a_tmem, sbase + NG * 128, idesc);
+          }
+        }
+        mma_commit(&mma_done[slot]);
+        issued = true;
+      }
+      // wind-down with the full limit: no MMA of ours still running
+      if (issued) {
+        mma_commit(&fdone[j]);
+        if (!mbar_wait(&fdone[j], 0, 2000000000ll)) fail(9);
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // The 3-bit codebook as an odd function of x_i = 2 b_i - 1: coefficients of
 // x0, x1, x2 and x0 x1 x2 (a Walsh transform of the eight centroids), and the
 // largest deviation of that fit from the centroids (zero for a symmetric book).
@@ -515,15 +891,27 @@ int launch_G(const tq_ctx& ctx, const float* qp, int64_t n_sets, int64_t n_keys,
   }
   X.err = P.err;
   X.wait_cycles = wait_limit_cycles();
-  const size_t smem = 1024 + static_cast<size_t>(kWG) * (Sh::kKBlocks * (2 * NG) * 128 + kStages * Sh::kStageBytes) +
-                      kWG * kScalFloats * 4 + (kWG * kStages + kWG) * 8 + 16;
-  cudaError_t e = cudaFuncSetAttribute(k_logits_d128_i8<B, G, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return static_cast<int>(e);
-  const int64_t n_tiles = ((n_keys + kTile - 1) / kTile) * n_sets;
-  int64_t grid = (n_tiles + kWG - 1) / kWG;
-  if (grid > ctx.num_sms) grid = ctx.num_sms;
-  k_logits_d128_i8<B, G, NG><<<static_cast<int>(grid), Sh::kThreads, smem, s>>>(P, X, qp, n_sets, n_keys, keys, out);
+  const int64_t tps = (n_keys + kTile - 1) / kTile, n_tiles = tps * n_sets;
+  // warp-specialized form when every CTA's contiguous tile range spans at most
+  // two sets: ranges of at most tps + 1 tiles
+  const int64_t ws_grid = n_tiles < ctx.num_sms ? n_tiles : ctx.num_sms;
+  if ((n_tiles + ws_grid - 1) / ws_grid <= tps + 1) {
+    const size_t smem = logits_ws_smem_bytes<B, NG>();
+    cudaError_t e = cudaFuncSetAttribute(k_logits_d128_ws<B, G, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+    k_logits_d128_ws<B, G, NG><<<static_cast<int>(ws_grid), WsLog<B, NG>::kThreads, smem, s>>>(P, X, qp, n_sets,
+                                                                                              n_keys, keys, out);
+  } else {
+    const size_t smem = 1024 + static_cast<size_t>(kWG) * (Sh::kKBlocks * (2 * NG) * 128 + kStages * Sh::kStageBytes) +
+                        kWG * kScalFloats * 4 + (kWG * kStages + kWG) * 8 + 16;
+    cudaError_t e = cudaFuncSetAttribute(k_logits_d128_i8<B, G, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+    int64_t grid = (n_tiles + kWG - 1) / kWG;
+    if (grid > ctx.num_sms) grid = ctx.num_sms;
+    k_logits_d128_i8<B, G, NG><<<static_cast<int>(grid), Sh::kThreads, smem, s>>>(P, X, qp, n_sets, n_keys, keys, out);
+  }
   count_launch();
   return static_cast<int>(cudaGetLastError());
 }

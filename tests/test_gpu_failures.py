@@ -7,6 +7,8 @@
   tq_sync_status reports; the next launch with the normal limit must run (it
   allocates all of the SM's tensor memory, so a leak would show) and match
   the oracle;
+* the same for the warp-specialized logits kernel (every role gives up and
+  winds down; the next launches reproduce the logits exactly);
 * an injected device-allocation failure in tq_init (TQ_ERR_NOMEM, then a
   normal tq_init works);
 * an injected launch failure (TQ_ERR_CUDA before anything is launched).
@@ -58,6 +60,37 @@ def test_quantize_wait_runs_out_then_recovers(tq, b):
         got = T.quantize(xd).to_numpy()
         T.sync_status()
     parity.assert_quantize_ok(parity.compare_quantize(P, got, ot.quantize(x, P, keep_intermediates=True)))
+    T.close()
+
+
+@pytest.mark.parametrize("b", [3, 4])
+def test_logits_wait_runs_out_then_recovers(tq, b):
+    """The warp-specialized logits kernel (2 sets x 313 key tiles: every CTA's
+    range within two sets) under the 100-clock limit: every role gives up,
+    drains its own MMAs and copies, and the kernel frees its tensor memory; the
+    error is reported once, and the next launches reproduce the logits bit for
+    bit."""
+    d, m, n_sets, g, n_keys = 128, 128, 2, 4, 40000
+    T = tq.TurboQuant(d, b, m, seed=0)
+    kt, _ = make_rows(d, n_sets * n_keys, "bf16", seed=41)
+    qt, _ = make_rows(d, n_sets * g, "bf16", seed=42)
+    keys = T.quantize(kt.cuda())
+    qd = qt.cuda()
+    want = T.logits(qd, keys, n_sets, g, n_keys).clone()
+    T.sync_status()
+    tq.test_set(tq.TQ_TEST_WAIT_LIMIT, 100)
+    try:
+        T.logits(qd, keys, n_sets, g, n_keys)
+        with pytest.raises(tq.TQError) as e:
+            T.sync_status()
+        assert e.value.status == tq.TQ_ERR_CUDA
+    finally:
+        tq.test_set(tq.TQ_TEST_WAIT_LIMIT, 0)
+    T.sync_status()
+    for _ in range(2):
+        got = T.logits(qd, keys, n_sets, g, n_keys)
+        T.sync_status()
+        assert torch.equal(got, want)
     T.close()
 
 
