@@ -398,8 +398,8 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
   uint8_t* sOut = sZ + kPairs * kStage;                  // [pair] output stages
   uint64_t* m1 = reinterpret_cast<uint64_t*>(sOut + kPairs * kStage);   // [pair] S^T z done
   uint64_t* m2 = m1 + kPairs;                                            // [pair] rotation done
-  uint64_t* fdone = m2 + kPairs;                                         // [pair] wind-down commit
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fdone + kPairs);
+  uint64_t* fdone = m2 + kPairs;                                         // [2][pair] wind-down commits
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fdone + 2 * kPairs);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   float* lut = reinterpret_cast<float*>(tmem_slot + 2);                 // L centroids x kUnit
   float2* lut2 = reinterpret_cast<float2*>(lut + 16);                   // 2-bit codes: pairs (4 bits)
@@ -408,7 +408,12 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
   const int64_t n_tiles = (n_rows + kTile - 1) / kTile;
   const long long wait_cycles = X.wait_cycles;
   if (tid == 0) {
-    for (int i = 0; i < kPairs; ++i) { mbar_init(&m1[i], 1); mbar_init(&m2[i], 1); mbar_init(&fdone[i], 1); }
+    for (int i = 0; i < kPairs; ++i) {
+      mbar_init(&m1[i], 1);
+      mbar_init(&m2[i], 1);
+      mbar_init(&fdone[i], 1);
+      mbar_init(&fdone[kPairs + i], 1);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -445,6 +450,12 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
   const int wgi = warp >> 2, pair = wgi >> 1, half = wgi & 1, lb = warp & 3;
   const bool leader = (half == 0 && lb == 0 && lane == 0);        // issues the pair's MMAs
   const bool storer = (half == 1 && lb == 0 && lane == 0);        // issues the pair's TMA stores
+  // issues the pair's S^T z products: for 3-bit codes a second thread, so that
+  // the leader's warp spends no issue time on them (one thread issues an MMA
+  // only every few dozen cycles); 10 % faster there, while for the other code
+  // widths the extra live state costs register spills and the leader keeps them
+  constexpr bool kSplitIssue = B == 3;
+  const bool zissuer = kSplitIssue ? (half == 1 && lb == 1 && lane == 0) : leader;
   const int trow = lb * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>(lb * 32) << 16;
   const uint32_t t_reg0 = tmem + lane_base + pair * (2 * KD);   // region k mod 2: S^T z, then the output of tile k
@@ -455,7 +466,7 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
   const float qjl = P.qjl_scale * kUnit;                  // S^T z in unit-norm x kUnit
   const int64_t t_first = blockIdx.x + static_cast<int64_t>(pair) * gridDim.x;
   const int64_t t_step = static_cast<int64_t>(kPairs) * gridDim.x;
-  bool store_pending = false, mma_issued = false;
+  bool store_pending = false, mma_issued = false, stz_issued = false;
 
   // my part of a packed row: codes of my 64 coordinates, my two sign words, norms
   struct Part {
@@ -574,7 +585,7 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
                  kk > 0 ? 1u : 0u);
     }
     mma_commit(&m1[pair]);
-    mma_issued = true;
+    (kSplitIssue ? stz_issued : mma_issued) = true;
   };
 
   Part cur, nxt;
@@ -585,7 +596,7 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
   decode(cur, v);
   fence_proxy_async_smem();
   named_bar_sync(bar_id, 256);                             // the first tile's sign operand is complete
-  if (PROD && leader && t_first < n_tiles) issue_stz(0);
+  if (PROD && zissuer && t_first < n_tiles) issue_stz(0);
 
   int mine = 0;
   for (int64_t t = t_first; t < n_tiles; t += t_step, ++mine) {
@@ -663,7 +674,7 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
     }
     tc_fence_after();
     // the rotation has read v: the next tile's S^T z may run into its region
-    if (PROD && leader && t + t_step < n_tiles && *reinterpret_cast<volatile int*>(abort_flag) == 0)
+    if (PROD && zissuer && t + t_step < n_tiles && *reinterpret_cast<volatile int*>(abort_flag) == 0)
       issue_stz(mine + 1);
     // ---- my kH output columns, staged (swizzled) for the TMA store, 32 at a time -------
 #pragma unroll
@@ -710,6 +721,10 @@ k_dequant_d128_ovl(const __grid_constant__ CUtensorMap tmap_out, const KParams P
   if (leader && mma_issued) {
     mma_commit(&fdone[pair]);
     if (!mbar_wait(&fdone[pair], 0, kWaitCycles) && X.err) atomicCAS(X.err, 0, 4);
+  }
+  if (kSplitIssue && zissuer && stz_issued) {
+    mma_commit(&fdone[kPairs + pair]);
+    if (!mbar_wait(&fdone[kPairs + pair], 0, kWaitCycles) && X.err) atomicCAS(X.err, 0, 4);
   }
   if (storer && store_pending) bulk_wait0();
   __syncthreads();
