@@ -59,6 +59,9 @@ __host__ __device__ constexpr uint32_t idesc_i8(uint32_t M, uint32_t N) {
          | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// the same with a signed 8-bit A
+__host__ __device__ constexpr uint32_t idesc_s8(uint32_t M, uint32_t N) { return idesc_i8(M, N) | (1u << 7); }
+
 __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
   asm volatile(
@@ -71,12 +74,13 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
 
 // K-steps [K0, K1) of a 128-key tile into one accumulator: A (0/1 bytes) from the
 // tile's TMEM columns, B from rows of the query operand (N rows per 128-byte K atom)
-template <int K0, int K1, int N>
+// (ACC: the first step accumulates onto what the accumulator holds)
+template <int K0, int K1, int N, bool ACC = false>
 __device__ __forceinline__ void mma_chain(uint32_t d_tmem, uint32_t a_tmem, uint32_t sbase, uint32_t idesc) {
 #pragma unroll
   for (int k = K0; k < K1; ++k) {
     const uint64_t bdesc = smem_desc_sw128(sbase + (k >> 2) * (N * 128) + (k & 3) * 32, 1024);
-    mma_i8_ts(d_tmem, a_tmem + k * 8, bdesc, idesc, k > K0 ? 1u : 0u);
+    mma_i8_ts(d_tmem, a_tmem + k * 8, bdesc, idesc, (ACC || k > K0) ? 1u : 0u);
   }
 }
 
@@ -127,10 +131,25 @@ __device__ __forceinline__ float join_limbs(const uint32_t* a) {
               fmaf(static_cast<float>(static_cast<int>(a[2])), 65536.f, static_cast<float>(lo)));
 }
 
+// The same for accumulators up to 2^23 in magnitude (centroid byte planes):
+// the two low limbs join in 64-bit integers.
+__device__ __forceinline__ float join_limbs_wide(const uint32_t* a) {
+  const long long lo = static_cast<long long>(static_cast<int>(a[0])) +
+                       static_cast<long long>(static_cast<int>(a[1])) * 256ll;
+  return fmaf(static_cast<float>(static_cast<int>(a[3])), 16777216.f,
+              fmaf(static_cast<float>(static_cast<int>(a[2])), 65536.f, static_cast<float>(lo)));
+}
+
 struct LogitsArgs {
   float wbit[3];                  // weight of code bit 0 / 1 / 2 in the centroid
   float wpar;                     // weight of the code's parity bit (3-bit codes)
   float cconst;                   // centroid constant term
+  // 3-bit codes in the warp-specialized kernel: each centroid as a 16-bit fixed
+  // point value round(c s), s = 32767 / max |c|, split into a signed high byte
+  // and an unsigned low byte (lut8: high bytes of codes 0..3, 4..7, low bytes
+  // likewise, for byte permutes), and 1 / s
+  uint32_t lut8[4];
+  float cinv;
   long long wait_cycles;          // bound of every wait
   int* err;
 };
@@ -161,11 +180,19 @@ __device__ __forceinline__ uint32_t code_parities(uint32_t w0, uint32_t w1, uint
 // constants and inverse scales in sScal (partial maxima at 0, partial sums at
 // 64, constants at 128, inverse scales at 144).  Ends with the operand visible
 // to the tensor cores and a barrier of the 128 threads.
-template <int B, int G, int NG>
+//
+// BYTES: the byte-plane operand of 3-bit codes (warp-specialized kernel): K
+// positions 0..127 the centroids' high bytes of coordinates 0..127, 128..255
+// their low bytes, 256..383 the sign bits as in the bit-plane form; the query
+// value of a coordinate, at 2^fe, times 256 against the high byte; no constant
+// term, and the inverse scale carries 1 / s instead of 2^-7.
+template <int B, int G, int NG, bool BYTES = false>
 __device__ __forceinline__ void build_query_operand(const LogitsArgs& X, const float* __restrict__ qs, int trow,
                                                     int wl, int lane, float* sScal, uint8_t* sB, uint32_t bar_id) {
   using S = Shape<B>;
   constexpr int N = 2 * NG;
+  constexpr int kK = BYTES ? 384 : S::kK;
+  constexpr int kSignCol = BYTES ? 64 : 8 * (S::kCodeWords + S::kParWords);   // first column of the sign plane
   // per-warp maxima and sums of every query's two halves, combined below in a
   // fixed order (thread trow owns coordinate / projection trow)
   float* sPM = sScal;                               // [warp][2G] partial maxima
@@ -194,6 +221,7 @@ __device__ __forceinline__ void build_query_operand(const LogitsArgs& X, const f
   float wmax = fabsf(X.wbit[0]);
   if (B >= 2) wmax = fmaxf(wmax, fabsf(X.wbit[1]));
   if (B == 3) wmax = fmaxf(wmax, fmaxf(fabsf(X.wbit[2]), fabsf(X.wpar)));
+  if (BYTES) wmax = 1.f;
   // fixed-point exponent of half h of query q: |value| * 2^F <= 2^22
   auto fp_exp = [&](int h, int q) {
     const int i = h * G + q;
@@ -214,14 +242,21 @@ __device__ __forceinline__ void build_query_operand(const LogitsArgs& X, const f
   // the byte is bit * 2^(o & 7); the query value is scaled by 2^(7 - (o & 7)) and
   // every product carries the common factor 2^7.
 #pragma unroll
-  for (int r = 0; r < S::kK / 128; ++r) {
+  for (int r = 0; r < kK / 128; ++r) {
     const int kappa = trow + 128 * r;
     const int o = kappa >> 2, tb = kappa & 3;
     const int up = 7 - (o & 7);
     int8_t limb[N];
 #pragma unroll
     for (int n = 0; n < N; ++n) limb[n] = 0;
-    if (o < 8 * (S::kCodeWords + S::kParWords)) {
+    if (BYTES && r < 2) {
+      // centroid byte plane r of coordinate trow
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        const int v = __float2int_rn(ldexpf(qs[q * (kD + kM) + trow], fe[q])) * (r == 0 ? 256 : 1);
+        split_limbs(v, &limb[4 * q]);
+      }
+    } else if (!BYTES && o < kSignCol) {
       int coord;
       float w;
       if (o < 8 * S::kCodeWords) {
@@ -240,7 +275,7 @@ __device__ __forceinline__ void build_query_operand(const LogitsArgs& X, const f
         split_limbs(v, &limb[4 * q]);
       }
     } else {
-      const int c = (o - 8 * (S::kCodeWords + S::kParWords)) >> 3, k = o & 7;
+      const int c = (o - kSignCol) >> 3, k = o & 7;
       const int j = 32 * c + k + 8 * tb;           // projection
 #pragma unroll
       for (int q = 0; q < G; ++q) {
@@ -258,8 +293,8 @@ __device__ __forceinline__ void build_query_operand(const LogitsArgs& X, const f
   if (trow < 2 * G) {
     const float sum = (sPS[trow] + sPS[16 + trow]) + (sPS[32 + trow] + sPS[48 + trow]);
     const int h = trow >= G ? 1 : 0;
-    sC[trow] = h ? sum : X.cconst * sum;
-    sInv[trow] = ldexpf(1.f, -fp_exp(h, trow - h * G) - 7);
+    sC[trow] = h ? sum : (BYTES ? 0.f : X.cconst * sum);
+    sInv[trow] = (BYTES && h == 0) ? ldexpf(X.cinv, -fp_exp(h, trow)) : ldexpf(1.f, -fp_exp(h, trow - h * G) - 7);
   }
   fence_proxy_async_smem();
   named_bar_sync(bar_id, 128);
@@ -498,6 +533,12 @@ k_logits_d128_i8(const KParams P, const LogitsArgs X, const float* __restrict__ 
 //             60 to 100 cycles, so the four issue side by side), one or two
 //             per slot: the code steps against the code-limb rows of the query
 //             operand, the sign steps against the sign-limb rows.
+// 3-bit codes take their centroids as two byte planes here, the high and low
+// byte of round(c s) with s = 32767 / max |c| (a byte permute per four
+// coordinates from an eight-entry table; the high bytes signed), so a slot
+// has the 96 operand columns of b = 3 and the TMEM holds four: the centroid
+// error is at most max |c| / 65534 per coordinate, a logit error of at most
+// 3.3e-5 |q| |k| at d = 128 (the bit-plane form of the general kernel is exact).
 // Barriers per slot: a_ready (decode -> issuers), mma_done (issuers ->
 // epilogue), slot_free (epilogue -> decode); per stage: full, stage_free; per
 // query buffer: q_ready.  Every wait is bounded and gives up once another
@@ -507,15 +548,22 @@ template <int B, int NG>
 struct WsLog {
   using S = Shape<B>;
   static constexpr int N = 2 * NG;                                  // code limbs | sign limbs
+  // 3-bit codes as two centroid byte planes (high, low) instead of four bit
+  // planes (three code bits and the parity): 96 operand columns, as at b = 3
+  static constexpr bool kBytes = B == 3;
+  static constexpr int kAWords = kBytes ? 96 : S::kAWords;
+  static constexpr int kKSteps = kBytes ? 12 : S::kKSteps;
+  static constexpr int kMseSteps = kBytes ? 8 : S::kMseSteps;
+  static constexpr int kKBlocks = kBytes ? 3 : S::kKBlocks;
   // a slot: A, then the code | sign accumulators; four slots of 128 columns
   // (one issuer each) or two of 256, each with two issuers, the code steps split
   // between them into a second code accumulator
-  static constexpr int kSlots = S::kAWords + N <= 128 ? 4 : 2;
+  static constexpr int kSlots = kAWords + N <= 128 ? 4 : 2;
   static constexpr int kSlotCols = 512 / kSlots;
   static constexpr int kIssuersPerSlot = 4 / kSlots;
   static constexpr int kChains = kSlots == 2 ? 3 : 2;
   static constexpr int kStages = 6;                                 // three per decode group
-  static constexpr int kBBytes = S::kKBlocks * N * 128;
+  static constexpr int kBBytes = kKBlocks * N * 128;
   static constexpr int kThreads = 20 * 32;
 };
 
@@ -638,8 +686,8 @@ k_logits_d128_ws(const KParams P, const LogitsArgs X, const float* __restrict__ 
     const uint32_t bar = 1 + eg;                                      // this group's named barrier
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wl * 32) << 16);
     if (n_mine > 0 && set0 + eg <= last_set) {
-      build_query_operand<B, G, NG>(X, qp + (set0 + eg) * G * (kD + kM), trow, wl, lane, sScal + eg * kScalFloats,
-                                    sBq + eg * W::kBBytes, bar);
+      build_query_operand<B, G, NG, W::kBytes>(X, qp + (set0 + eg) * G * (kD + kM), trow, wl, lane,
+                                               sScal + eg * kScalFloats, sBq + eg * W::kBBytes, bar);
       if (wl == 0 && lane == 0) mbar_arrive(&q_ready[eg]);
     }
     TileCursor c{set0, kt0, tps};
@@ -665,7 +713,7 @@ k_logits_d128_ws(const KParams P, const LogitsArgs X, const float* __restrict__ 
       if (!ok) fail(9);
       if (named_bar_sync_or(bar, 128, !ok)) break;
       tc_fence_after();
-      const uint32_t t_d = t_lane + s * W::kSlotCols + S::kAWords;
+      const uint32_t t_d = t_lane + s * W::kSlotCols + W::kAWords;
       uint32_t acc[N];
       {
         uint32_t part[32];
@@ -697,7 +745,8 @@ k_logits_d128_ws(const KParams P, const LogitsArgs X, const float* __restrict__ 
         float* o = out + c.set * G * n_keys + key;
 #pragma unroll
         for (int q = 0; q < G; ++q) {
-          const float mse = fmaf(join_limbs(&acc[4 * q]), sc[144 + q], sc[128 + q]);
+          const float mse = fmaf(W::kBytes ? join_limbs_wide(&acc[4 * q]) : join_limbs(&acc[4 * q]), sc[144 + q],
+                                 sc[128 + q]);
           const float qjl = fmaf(join_limbs(&acc[NG + 4 * q]), sc[144 + G + q], sc[128 + G + q]);
           o[q * n_keys] = fmaf(nrm, mse, rn * qjl);
         }
@@ -756,23 +805,48 @@ k_logits_d128_ws(const KParams P, const LogitsArgs X, const float* __restrict__ 
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&stage_free[st]);
-      if constexpr (B == 3) {
-#pragma unroll
-        for (int g2 = 0; g2 < 4; ++g2)
-          cw[S::kCodeWords + g2] = code_parities(cw[3 * g2], cw[3 * g2 + 1], cw[3 * g2 + 2]);
-      }
       const uint32_t t_a = t_lane + s * W::kSlotCols;
-      uint32_t a[32];
-      int na = 0, col = 0;
+      if constexpr (W::kBytes) {
+        // the centroid bytes of four coordinates per byte permute: the four
+        // 3-bit codes of a 12-bit group spread to the selector's nibbles
 #pragma unroll
-      for (int cc = 0; cc < S::kCodeWords + S::kParWords + 4; ++cc) {
+        for (int j8 = 0; j8 < 4; ++j8) {
+          uint32_t hw[8], lw[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          a[na++] = cw[cc] & (0x01010101u << k);
-          if (na == 32) {
-            tmem_st32(t_a + col, a);
-            col += 32;
-            na = 0;
+          for (int jj = 0; jj < 8; ++jj) {
+            const int j = 8 * j8 + jj, bit = 12 * j, w = bit >> 5, sh = bit & 31;
+            const uint32_t x = sh + 12 <= 32 ? cw[w] >> sh : __funnelshift_r(cw[w], cw[w + 1], sh);
+            const uint32_t sel = (x & 0x7u) | ((x << 1) & 0x70u) | ((x << 2) & 0x700u) | ((x << 3) & 0x7000u);
+            hw[jj] = __byte_perm(X.lut8[0], X.lut8[1], sel);
+            lw[jj] = __byte_perm(X.lut8[2], X.lut8[3], sel);
+          }
+          tmem_st8(t_a + 8 * j8, hw);
+          tmem_st8(t_a + 32 + 8 * j8, lw);
+        }
+        uint32_t a[32];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) a[8 * cc + k] = cw[S::kCodeWords + S::kParWords + cc] & (0x01010101u << k);
+        tmem_st32(t_a + 64, a);
+      } else {
+        if constexpr (B == 3) {
+#pragma unroll
+          for (int g2 = 0; g2 < 4; ++g2)
+            cw[S::kCodeWords + g2] = code_parities(cw[3 * g2], cw[3 * g2 + 1], cw[3 * g2 + 2]);
+        }
+        uint32_t a[32];
+        int na = 0, col = 0;
+#pragma unroll
+        for (int cc = 0; cc < S::kCodeWords + S::kParWords + 4; ++cc) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            a[na++] = cw[cc] & (0x01010101u << k);
+            if (na == 32) {
+              tmem_st32(t_a + col, a);
+              col += 32;
+              na = 0;
+            }
           }
         }
       }
@@ -801,7 +875,7 @@ k_logits_d128_ws(const KParams P, const LogitsArgs X, const float* __restrict__ 
       TileCursor c{set0, kt0, tps};
       c.step(slot);
       const uint32_t idesc = idesc_i8(kTile, NG);
-      const uint32_t a_tmem = tmem + slot * W::kSlotCols, d_tmem = a_tmem + S::kAWords;
+      const uint32_t a_tmem = tmem + slot * W::kSlotCols, d_tmem = a_tmem + W::kAWords;
       // every use of the slot, in order (the slot's barriers complete once per use)
       for (int i = slot; i < n_mine; i += kSlots, c.step(kSlots)) {
         if (c.set != q_set) {
@@ -811,16 +885,20 @@ k_logits_d128_ws(const KParams P, const LogitsArgs X, const float* __restrict__ 
         if (!ws_wait(&a_ready[slot], static_cast<uint32_t>((i / kSlots) & 1), lim, abort_flag)) { fail(9); break; }
         tc_fence_after();
         const uint32_t sbase = smem_u32(sBq + static_cast<int>(c.set - set0) * W::kBBytes);
+        // code steps [0, h) and [h, kMseSteps): with centroid byte planes the high
+        // bytes (steps 0..3) are signed, the low bytes (4..7) unsigned
+        constexpr int h = W::kBytes ? 4 : W::kMseSteps / 2;
+        const uint32_t idesc_a = W::kBytes ? idesc_s8(kTile, NG) : idesc;
         if constexpr (W::kIssuersPerSlot == 1) {
-          mma_chain<0, S::kMseSteps, N>(d_tmem, a_tmem, sbase, idesc);
-          mma_chain<S::kMseSteps, S::kKSteps, N>(d_tmem + NG, a_tmem, sbase + NG * 128, idesc);
+          mma_chain<0, h, N>(d_tmem, a_tmem, sbase, idesc_a);
+          mma_chain<h, W::kMseSteps, N, true>(d_tmem, a_tmem, sbase, idesc);
+          mma_chain<W::kMseSteps, W::kKSteps, N>(d_tmem + NG, a_tmem, sbase + NG * 128, idesc);
         } else {
-          constexpr int h = S::kMseSteps / 2;
           if (part == 0) {
-            mma_chain<0, h, N>(d_tmem, a_tmem, sbase, idesc);
+            mma_chain<0, h, N>(d_tmem, a_tmem, sbase, idesc_a);
           } else {
-            mma_chain<h, S::kMseSteps, N>(d_tmem + N, a_tmem, sbase, idesc);
-            mma_chain<S::kMseSteps, S::kKSteps, N>(d_tmem + NG, a_tmem, sbase + NG * 128, idesc);
+            mma_chain<h, W::kMseSteps, N>(d_tmem + N, a_tmem, sbase, idesc);
+            mma_chain<W::kMseSteps, W::kKSteps, N>(d_tmem + NG, a_tmem, sbase + NG * 128, idesc);
           }
         }
         mma_commit(&mma_done[slot]);
@@ -888,6 +966,23 @@ int launch_G(const tq_ctx& ctx, const float* qp, int64_t n_sets, int64_t n_keys,
     X.wbit[0] = 2.f * P.c[1];
     X.wbit[1] = 0.f;
     X.cconst = -P.c[1];
+  }
+  // centroid byte planes (warp-specialized kernel, 3-bit codes): round(c s) as a
+  // signed high byte and an unsigned low byte, |error| <= max |c| / 65534
+  for (int i = 0; i < 4; ++i) X.lut8[i] = 0u;
+  X.cinv = 1.f;
+  if (B == 3) {
+    float cmax = 0.f;
+    for (int k = 0; k < 8; ++k) cmax = std::max(cmax, std::fabs(P.c[k]));
+    const double sc = cmax > 0.f ? 32767.0 / cmax : 1.0;
+    for (int k = 0; k < 8; ++k) {
+      long v = std::lrint(static_cast<double>(P.c[k]) * sc);
+      v = std::min(32767l, std::max(-32767l, v));
+      const uint32_t hi = static_cast<uint32_t>((v >> 8) & 0xFF), lo = static_cast<uint32_t>(v & 0xFF);
+      X.lut8[k >> 2] |= hi << (8 * (k & 3));
+      X.lut8[2 + (k >> 2)] |= lo << (8 * (k & 3));
+    }
+    X.cinv = static_cast<float>(1.0 / sc);
   }
   X.err = P.err;
   X.wait_cycles = wait_limit_cycles();
