@@ -807,18 +807,23 @@ k_logits_d128_ws(const KParams P, const LogitsArgs X, const float* __restrict__ 
       if (lane == 0) mbar_arrive(&stage_free[st]);
       const uint32_t t_a = t_lane + s * W::kSlotCols;
       if constexpr (W::kBytes) {
-        // the centroid bytes of four coordinates per byte permute: the four
-        // 3-bit codes of a 12-bit group spread to the selector's nibbles
+        // the centroid bytes of four coordinates per byte permute: the eight
+        // 3-bit codes of a 24-bit group spread to the nibbles of two selectors
+        // (three shift-and-merge steps)
 #pragma unroll
         for (int j8 = 0; j8 < 4; ++j8) {
           uint32_t hw[8], lw[8];
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int j = 8 * j8 + jj, bit = 12 * j, w = bit >> 5, sh = bit & 31;
-            const uint32_t x = sh + 12 <= 32 ? cw[w] >> sh : __funnelshift_r(cw[w], cw[w + 1], sh);
-            const uint32_t sel = (x & 0x7u) | ((x << 1) & 0x70u) | ((x << 2) & 0x700u) | ((x << 3) & 0x7000u);
-            hw[jj] = __byte_perm(X.lut8[0], X.lut8[1], sel);
-            lw[jj] = __byte_perm(X.lut8[2], X.lut8[3], sel);
+          for (int jj = 0; jj < 4; ++jj) {
+            const int j = 4 * j8 + jj, bit = 24 * j, w = bit >> 5, sh = bit & 31;
+            uint32_t x = sh + 24 <= 32 ? cw[w] >> sh : __funnelshift_r(cw[w], cw[w + 1], sh);
+            x = (x & 0xFFFu) | ((x << 4) & 0x0FFF0000u);               // codes 4..7 to bits 16..
+            x = (x & 0x003F003Fu) | ((x << 2) & 0x3F003F00u);          // codes 2, 3 (and 6, 7) up by 2
+            x = (x & 0x07070707u) | ((x << 1) & 0x70707070u);          // codes 1, 3, 5, 7 up by 1
+            hw[2 * jj] = __byte_perm(X.lut8[0], X.lut8[1], x);
+            lw[2 * jj] = __byte_perm(X.lut8[2], X.lut8[3], x);
+            hw[2 * jj + 1] = __byte_perm(X.lut8[0], X.lut8[1], x >> 16);
+            lw[2 * jj + 1] = __byte_perm(X.lut8[2], X.lut8[3], x >> 16);
           }
           tmem_st8(t_a + 8 * j8, hw);
           tmem_st8(t_a + 32 + 8 * j8, lw);
