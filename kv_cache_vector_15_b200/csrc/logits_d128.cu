@@ -708,10 +708,9 @@ k_logits_d128_ws(const KParams P, const LogitsArgs X, const float* __restrict__ 
       TileCursor nx = c;
       nx.step(2);
       if (i + 2 < n_mine) load_norms(nx);
-      // the group's four warps leave together (they share a named barrier)
-      const bool ok = ws_wait(&mma_done[s], static_cast<uint32_t>((i / kSlots) & 1), lim, abort_flag);
-      if (!ok) fail(9);
-      if (named_bar_sync_or(bar, 128, !ok)) break;
+      // (the group's warps meet in no barrier after the operand build: each
+      // waits for the accumulators on its own)
+      if (!ws_wait(&mma_done[s], static_cast<uint32_t>((i / kSlots) & 1), lim, abort_flag)) { fail(9); break; }
       tc_fence_after();
       const uint32_t t_d = t_lane + s * W::kSlotCols + W::kAWords;
       uint32_t acc[N];
