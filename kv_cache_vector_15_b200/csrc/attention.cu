@@ -15,6 +15,8 @@
 // so no value row is ever reconstructed in memory.
 //
 // Kernels (after qprep + logits into the workspace):
+//   k_attn_chunk128  d = m = 128, 2- and 3-bit codes: as below, with a pair of
+//                    coordinates / projections per thread and packed FMAs;
 //   k_attn_chunk     one CTA per (key chunk, set): the chunk's softmax maximum
 //                    and normaliser per query, and its partial a, b (weights
 //                    exp(scale (s - max_chunk))), one thread per coordinate /
@@ -185,6 +187,182 @@ k_attn_chunk(const KParams P, const float* __restrict__ logits, const Packed val
   }
 }
 
+// The d = m = 128 form of the chunk kernel (code widths of 2 and 3 bits): a
+// thread owns a pair of coordinates (threads 0..127) or of projections
+// (128..255) for one half of each staged batch of keys, with every query's
+// accumulators as packed fp32 pairs, so a key costs it one table lookup (both
+// centroids of the pair from the pair's 2B code bits) or two sign bits, one
+// weight load per four queries and G packed FMAs.  The two key halves are
+// summed at the end; the record is that of the general kernel.
+template <int B, int G>
+__global__ void __launch_bounds__(kAttnThreads)
+k_attn_chunk128(const KParams P, const float* __restrict__ logits, const Packed values, int64_t n_keys, int chunk,
+                float scale_log2, int prod, float* __restrict__ partial) {
+  constexpr int d = 128, m = 128;
+  constexpr int cw32 = B * 4, sw32 = 4;                         // words per packed row
+  constexpr int GP = (G + 3) / 4 * 4;
+  constexpr int L = 1 << B;
+  const int set = blockIdx.y, c = blockIdx.x, n_chunks = gridDim.x;
+  const int64_t k0 = static_cast<int64_t>(c) * chunk;
+  const int64_t k1 = k0 + chunk < n_keys ? k0 + chunk : n_keys;
+  const int tid = threadIdx.x;
+  __shared__ uint32_t sCodes[kAttnBatch][cw32 + 1];             // + a zero word for pairs that straddle words
+  __shared__ uint32_t sSigns[kAttnBatch][sw32];
+  __shared__ __align__(16) float sWn[kAttnBatch][GP];           // weight * norm
+  __shared__ __align__(16) float sWr[kAttnBatch][GP];           // weight * rnorm
+  __shared__ float sMax[G];
+  __shared__ float sRed[kAttnThreads];
+  __shared__ float2 lut2[L * L];                                // (c[i mod L], c[i / L])
+  __shared__ float2 sHalf[128][G];                              // the odd key half's sums
+  for (int i = tid; i < L * L; i += kAttnThreads) lut2[i] = make_float2(P.c[i & (L - 1)], P.c[i >> B]);
+
+  const float* lg = logits + static_cast<int64_t>(set) * G * n_keys;
+  // ---- the chunk's maximum of scale * logit per query (log2 units) -------------
+  float mx[G];
+#pragma unroll
+  for (int q = 0; q < G; ++q) mx[q] = -INFINITY;
+  for (int64_t k = k0 + tid; k < k1; k += kAttnThreads)
+#pragma unroll
+    for (int q = 0; q < G; ++q) mx[q] = fmaxf(mx[q], lg[q * n_keys + k] * scale_log2);
+#pragma unroll
+  for (int q = 0; q < G; ++q) {
+    float v = mx[q];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if ((tid & 31) == 0) sRed[(tid >> 5) * G + q] = v;
+  }
+  __syncthreads();
+  if (tid < G) {
+    float v = -INFINITY;
+    for (int w = 0; w < kAttnThreads / 32; ++w) v = fmaxf(v, sRed[w * G + tid]);
+    sMax[tid] = v;
+  }
+  __syncthreads();
+  float cm[G];
+#pragma unroll
+  for (int q = 0; q < G; ++q) cm[q] = sMax[q];
+
+  const int role = tid >> 7, pair = tid & 63, khalf = (tid >> 6) & 1;
+  const bool active = role == 0 || prod;
+  float2 acc[G];
+#pragma unroll
+  for (int q = 0; q < G; ++q) acc[q] = make_float2(0.f, 0.f);
+  float lsum = 0.f;                                             // thread tid < batch*G: its (key, query)
+  // my pair's bits: code bits 2 B pair .. + 2 B - 1, or sign bits 2 pair, 2 pair + 1
+  const int cbit = 2 * B * pair, cw = cbit >> 5, csh = cbit & 31;
+  const int sw = pair >> 4, ssh = (2 * pair) & 31;
+  // staging of a batch: the next batch's words are loaded into registers while
+  // the current one is summed, then stored once every thread is done with it
+  struct Pref {
+    uint32_t c0, c1, sg;
+    float lgv, nrm, rnm;
+  };
+  auto load_batch = [&](int64_t kb, int nb, Pref& p) {
+    const int64_t row0 = static_cast<int64_t>(set) * n_keys + kb;
+    const uint32_t* cwp = reinterpret_cast<const uint32_t*>(values.codes) + row0 * cw32;
+    p.c0 = tid < nb * cw32 ? __ldg(cwp + tid) : 0u;
+    p.c1 = tid + kAttnThreads < nb * cw32 ? __ldg(cwp + tid + kAttnThreads) : 0u;
+    p.sg = prod && tid < nb * sw32 ? __ldg(reinterpret_cast<const uint32_t*>(values.signs) + row0 * sw32 + tid) : 0u;
+    if (tid < nb * G) {                                         // one (key, query) per thread
+      const int r = tid / G, q = tid - r * G;
+      p.lgv = lg[q * n_keys + kb + r];
+      p.nrm = __ldg(values.norm + row0 + r);
+      p.rnm = __ldg(values.rnorm + row0 + r);
+    }
+  };
+  auto store_batch = [&](int nb, const Pref& p) {
+    if (tid < nb * cw32) sCodes[tid / cw32][tid % cw32] = p.c0;
+    if (tid + kAttnThreads < nb * cw32) sCodes[(tid + kAttnThreads) / cw32][(tid + kAttnThreads) % cw32] = p.c1;
+    if (tid < nb) sCodes[tid][cw32] = 0u;
+    if (prod && tid < nb * sw32) sSigns[tid / sw32][tid % sw32] = p.sg;
+    if (tid < nb * G) {
+      const int r = tid / G, q = tid - r * G;
+      float cq = cm[0];
+#pragma unroll
+      for (int qq = 1; qq < G; ++qq) cq = q == qq ? cm[qq] : cq;
+      const float w = exp2f(p.lgv * scale_log2 - cq);
+      sWn[r][q] = w * p.nrm;
+      sWr[r][q] = w * p.rnm;
+      lsum += w;
+    }
+  };
+  Pref pf;
+  int64_t kb = k0;
+  int nb = static_cast<int>(k1 - kb < kAttnBatch ? k1 - kb : kAttnBatch);
+  if (nb > 0) {
+    load_batch(kb, nb, pf);
+    store_batch(nb, pf);
+  }
+  for (; nb > 0;) {
+    const int64_t kn = kb + kAttnBatch;
+    const int nbn = kn < k1 ? static_cast<int>(k1 - kn < kAttnBatch ? k1 - kn : kAttnBatch) : 0;
+    if (nbn > 0) load_batch(kn, nbn, pf);
+    __syncthreads();
+    if (active) {
+      if (role == 0) {
+#pragma unroll 4
+        for (int r = khalf; r < nb; r += 2) {
+          uint32_t idx;
+          if ((csh + 2 * B) <= 32) idx = sCodes[r][cw] >> csh;
+          else idx = __funnelshift_r(sCodes[r][cw], sCodes[r][cw + 1], csh);
+          const float2 c2 = lut2[idx & (L * L - 1)];
+#pragma unroll
+          for (int q4 = 0; q4 < GP; q4 += 4) {
+            const float4 w = *reinterpret_cast<const float4*>(&sWn[r][q4]);
+            if (q4 + 0 < G) acc[q4 + 0] = __ffma2_rn(make_float2(w.x, w.x), c2, acc[q4 + 0]);
+            if (q4 + 1 < G) acc[q4 + 1] = __ffma2_rn(make_float2(w.y, w.y), c2, acc[q4 + 1]);
+            if (q4 + 2 < G) acc[q4 + 2] = __ffma2_rn(make_float2(w.z, w.z), c2, acc[q4 + 2]);
+            if (q4 + 3 < G) acc[q4 + 3] = __ffma2_rn(make_float2(w.w, w.w), c2, acc[q4 + 3]);
+          }
+        }
+      } else {
+#pragma unroll 4
+        for (int r = khalf; r < nb; r += 2) {
+          const uint32_t bits = sSigns[r][sw] >> ssh;           // z = 1 - 2 bit
+          const float2 z2 = make_float2(__uint_as_float(0x3F800000u | (bits << 31)),
+                                        __uint_as_float(0x3F800000u | ((bits & 2u) << 30)));
+#pragma unroll
+          for (int q4 = 0; q4 < GP; q4 += 4) {
+            const float4 w = *reinterpret_cast<const float4*>(&sWr[r][q4]);
+            if (q4 + 0 < G) acc[q4 + 0] = __ffma2_rn(make_float2(w.x, w.x), z2, acc[q4 + 0]);
+            if (q4 + 1 < G) acc[q4 + 1] = __ffma2_rn(make_float2(w.y, w.y), z2, acc[q4 + 1]);
+            if (q4 + 2 < G) acc[q4 + 2] = __ffma2_rn(make_float2(w.z, w.z), z2, acc[q4 + 2]);
+            if (q4 + 3 < G) acc[q4 + 3] = __ffma2_rn(make_float2(w.w, w.w), z2, acc[q4 + 3]);
+          }
+        }
+      }
+    }
+    __syncthreads();                                            // the batch is consumed
+    if (nbn > 0) store_batch(nbn, pf);
+    kb = kn;
+    nb = nbn;
+  }
+  // ---- the two key halves, the chunk's normaliser per query, the partial record --------
+  __syncthreads();
+  if (khalf == 1) {
+#pragma unroll
+    for (int q = 0; q < G; ++q) sHalf[role * 64 + pair][q] = acc[q];
+  }
+  sRed[tid] = lsum;                                             // thread tid accumulated (key tid / G, query tid % G)
+  __syncthreads();
+  float* rec = partial + ((static_cast<int64_t>(set) * G) * n_chunks + c) * partial_floats(d, m);
+  const int64_t qstride = static_cast<int64_t>(n_chunks) * partial_floats(d, m);
+  if (tid < G) {
+    float l = 0.f;
+    for (int t = tid; t < kAttnBatch * G && t < kAttnThreads; t += G) l += sRed[t];
+    rec[tid * qstride + 0] = cm[tid];
+    rec[tid * qstride + 1] = l;
+  }
+  if (khalf == 0 && active) {
+    const int x = role * d + 2 * pair;                          // coordinate, or d + projection
+#pragma unroll
+    for (int q = 0; q < G; ++q) {
+      const float2 o = sHalf[role * 64 + pair][q];
+      *reinterpret_cast<float2*>(rec + q * qstride + 2 + x) = make_float2(acc[q].x + o.x, acc[q].y + o.y);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kAttnThreads)
 k_attn_finalize(const KParams P, const float* __restrict__ partial, int n_chunks, int prod, float* __restrict__ out) {
   const int d = P.d, m = P.m, tid = threadIdx.x;
@@ -262,6 +440,15 @@ int launch_chunk(const KParams& P, const float* logits, const Packed& values, in
 template <int G>
 int launch_chunk_g(const KParams& P, const float* logits, const Packed& values, int64_t n_sets, int64_t n_keys,
                    int chunk, int n_chunks, float scale_log2, int prod, float* partial, cudaStream_t s) {
+  if (P.d == 128 && P.m == 128 && (P.B == 2 || P.B == 3) && P.codes_bytes == P.B * 16 && P.signs_bytes == 16) {
+    dim3 grid(static_cast<unsigned>(n_chunks), static_cast<unsigned>(n_sets));
+    if (P.B == 2)
+      k_attn_chunk128<2, G><<<grid, kAttnThreads, 0, s>>>(P, logits, values, n_keys, chunk, scale_log2, prod, partial);
+    else
+      k_attn_chunk128<3, G><<<grid, kAttnThreads, 0, s>>>(P, logits, values, n_keys, chunk, scale_log2, prod, partial);
+    count_launch();
+    return static_cast<int>(cudaGetLastError());
+  }
   const int nx = P.d + (prod ? P.m : 0);
   const int slots = (nx + kAttnThreads - 1) / kAttnThreads;
   if (slots <= 1) return launch_chunk<G, 1>(P, logits, values, n_sets, n_keys, chunk, n_chunks, scale_log2, prod, partial, s);

@@ -249,6 +249,7 @@ def test_gpu_api_errors_and_empty_calls(tq):
 
 @pytest.mark.parametrize("d,b,m,n_sets,g,n_keys", [
     (128, 3, 128, 3, 4, 5000), (128, 4, 128, 2, 8, 2049), (128, 2, 128, 2, 1, 77), (64, 3, 96, 2, 3, 4100),
+    (128, 3, 128, 2, 3, 4099), (128, 4, 128, 1, 5, 2100),
     (256, 4, 128, 1, 5, 1500), (1024, 4, 1024, 1, 2, 300)])
 @pytest.mark.parametrize("mode", [0, 1])
 def test_attention_parity(tq, d, b, m, n_sets, g, n_keys, mode):
