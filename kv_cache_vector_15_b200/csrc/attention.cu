@@ -202,14 +202,16 @@ k_attn_chunk128(const KParams P, const float* __restrict__ logits, const Packed 
   constexpr int cw32 = B * 4, sw32 = 4;                         // words per packed row
   constexpr int GP = (G + 3) / 4 * 4;
   constexpr int L = 1 << B;
+  constexpr int KB = G <= 4 ? 2 * kAttnBatch : kAttnBatch;     // keys per staged batch (KB * G <= threads)
+  constexpr int kCW = (KB * cw32 + kAttnThreads - 1) / kAttnThreads;   // code words staged per thread
   const int set = blockIdx.y, c = blockIdx.x, n_chunks = gridDim.x;
   const int64_t k0 = static_cast<int64_t>(c) * chunk;
   const int64_t k1 = k0 + chunk < n_keys ? k0 + chunk : n_keys;
   const int tid = threadIdx.x;
-  __shared__ uint32_t sCodes[kAttnBatch][cw32 + 1];             // + a zero word for pairs that straddle words
-  __shared__ uint32_t sSigns[kAttnBatch][sw32];
-  __shared__ __align__(16) float sWn[kAttnBatch][GP];           // weight * norm
-  __shared__ __align__(16) float sWr[kAttnBatch][GP];           // weight * rnorm
+  __shared__ uint32_t sCodes[KB][cw32 + 1];                     // + a zero word for pairs that straddle words
+  __shared__ uint32_t sSigns[KB][sw32];
+  __shared__ __align__(16) float sWn[KB][GP];                   // weight * norm
+  __shared__ __align__(16) float sWr[KB][GP];                   // weight * rnorm
   __shared__ float sMax[G];
   __shared__ float sRed[kAttnThreads];
   __shared__ float2 lut2[L * L];                                // (c[i mod L], c[i / L])
@@ -254,14 +256,17 @@ k_attn_chunk128(const KParams P, const float* __restrict__ logits, const Packed 
   // staging of a batch: the next batch's words are loaded into registers while
   // the current one is summed, then stored once every thread is done with it
   struct Pref {
-    uint32_t c0, c1, sg;
+    uint32_t cw[kCW], sg;
     float lgv, nrm, rnm;
   };
   auto load_batch = [&](int64_t kb, int nb, Pref& p) {
     const int64_t row0 = static_cast<int64_t>(set) * n_keys + kb;
     const uint32_t* cwp = reinterpret_cast<const uint32_t*>(values.codes) + row0 * cw32;
-    p.c0 = tid < nb * cw32 ? __ldg(cwp + tid) : 0u;
-    p.c1 = tid + kAttnThreads < nb * cw32 ? __ldg(cwp + tid + kAttnThreads) : 0u;
+#pragma unroll
+    for (int i = 0; i < kCW; ++i) {
+      const int e = tid + i * kAttnThreads;
+      p.cw[i] = e < nb * cw32 ? __ldg(cwp + e) : 0u;
+    }
     p.sg = prod && tid < nb * sw32 ? __ldg(reinterpret_cast<const uint32_t*>(values.signs) + row0 * sw32 + tid) : 0u;
     if (tid < nb * G) {                                         // one (key, query) per thread
       const int r = tid / G, q = tid - r * G;
@@ -271,8 +276,11 @@ k_attn_chunk128(const KParams P, const float* __restrict__ logits, const Packed 
     }
   };
   auto store_batch = [&](int nb, const Pref& p) {
-    if (tid < nb * cw32) sCodes[tid / cw32][tid % cw32] = p.c0;
-    if (tid + kAttnThreads < nb * cw32) sCodes[(tid + kAttnThreads) / cw32][(tid + kAttnThreads) % cw32] = p.c1;
+#pragma unroll
+    for (int i = 0; i < kCW; ++i) {
+      const int e = tid + i * kAttnThreads;
+      if (e < nb * cw32) sCodes[e / cw32][e % cw32] = p.cw[i];
+    }
     if (tid < nb) sCodes[tid][cw32] = 0u;
     if (prod && tid < nb * sw32) sSigns[tid / sw32][tid % sw32] = p.sg;
     if (tid < nb * G) {
@@ -288,14 +296,14 @@ k_attn_chunk128(const KParams P, const float* __restrict__ logits, const Packed 
   };
   Pref pf;
   int64_t kb = k0;
-  int nb = static_cast<int>(k1 - kb < kAttnBatch ? k1 - kb : kAttnBatch);
+  int nb = static_cast<int>(k1 - kb < KB ? k1 - kb : KB);
   if (nb > 0) {
     load_batch(kb, nb, pf);
     store_batch(nb, pf);
   }
   for (; nb > 0;) {
-    const int64_t kn = kb + kAttnBatch;
-    const int nbn = kn < k1 ? static_cast<int>(k1 - kn < kAttnBatch ? k1 - kn : kAttnBatch) : 0;
+    const int64_t kn = kb + KB;
+    const int nbn = kn < k1 ? static_cast<int>(k1 - kn < KB ? k1 - kn : KB) : 0;
     if (nbn > 0) load_batch(kn, nbn, pf);
     __syncthreads();
     if (active) {
@@ -349,7 +357,7 @@ k_attn_chunk128(const KParams P, const float* __restrict__ logits, const Packed 
   const int64_t qstride = static_cast<int64_t>(n_chunks) * partial_floats(d, m);
   if (tid < G) {
     float l = 0.f;
-    for (int t = tid; t < kAttnBatch * G && t < kAttnThreads; t += G) l += sRed[t];
+    for (int t = tid; t < KB * G && t < kAttnThreads; t += G) l += sRed[t];
     rec[tid * qstride + 0] = cm[tid];
     rec[tid * qstride + 1] = l;
   }
