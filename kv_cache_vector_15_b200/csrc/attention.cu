@@ -202,8 +202,12 @@ k_attn_chunk128(const KParams P, const float* __restrict__ logits, const Packed 
   constexpr int cw32 = B * 4, sw32 = 4;                         // words per packed row
   constexpr int GP = (G + 3) / 4 * 4;
   constexpr int L = 1 << B;
-  constexpr int KB = G <= 4 ? 2 * kAttnBatch : kAttnBatch;     // keys per staged batch (KB * G <= threads)
+  // keys per staged batch: 128 when the threads' (key, query) weight entries
+  // keep one query per thread (G divides the thread count), else 32 G <= 256
+  constexpr int KB = (kAttnThreads % G == 0 && G <= 4) ? 4 * kAttnBatch : kAttnBatch;
   constexpr int kCW = (KB * cw32 + kAttnThreads - 1) / kAttnThreads;   // code words staged per thread
+  constexpr int kSP = (KB * sw32 + kAttnThreads - 1) / kAttnThreads;   // sign words staged per thread
+  constexpr int kWP = (KB * G + kAttnThreads - 1) / kAttnThreads;      // weight entries per thread
   const int set = blockIdx.y, c = blockIdx.x, n_chunks = gridDim.x;
   const int64_t k0 = static_cast<int64_t>(c) * chunk;
   const int64_t k1 = k0 + chunk < n_keys ? k0 + chunk : n_keys;
@@ -256,8 +260,8 @@ k_attn_chunk128(const KParams P, const float* __restrict__ logits, const Packed 
   // staging of a batch: the next batch's words are loaded into registers while
   // the current one is summed, then stored once every thread is done with it
   struct Pref {
-    uint32_t cw[kCW], sg;
-    float lgv, nrm, rnm;
+    uint32_t cw[kCW], sg[kSP];
+    float lgv[kWP], nrm[kWP], rnm[kWP];
   };
   auto load_batch = [&](int64_t kb, int nb, Pref& p) {
     const int64_t row0 = static_cast<int64_t>(set) * n_keys + kb;
@@ -267,12 +271,20 @@ k_attn_chunk128(const KParams P, const float* __restrict__ logits, const Packed 
       const int e = tid + i * kAttnThreads;
       p.cw[i] = e < nb * cw32 ? __ldg(cwp + e) : 0u;
     }
-    p.sg = prod && tid < nb * sw32 ? __ldg(reinterpret_cast<const uint32_t*>(values.signs) + row0 * sw32 + tid) : 0u;
-    if (tid < nb * G) {                                         // one (key, query) per thread
-      const int r = tid / G, q = tid - r * G;
-      p.lgv = lg[q * n_keys + kb + r];
-      p.nrm = __ldg(values.norm + row0 + r);
-      p.rnm = __ldg(values.rnorm + row0 + r);
+#pragma unroll
+    for (int i = 0; i < kSP; ++i) {
+      const int e = tid + i * kAttnThreads;
+      p.sg[i] = prod && e < nb * sw32 ? __ldg(reinterpret_cast<const uint32_t*>(values.signs) + row0 * sw32 + e) : 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < kWP; ++i) {                             // (key, query) entries e = tid + 256 i
+      const int e = tid + i * kAttnThreads;
+      if (e < nb * G) {
+        const int r = e / G, q = e - r * G;
+        p.lgv[i] = lg[q * n_keys + kb + r];
+        p.nrm[i] = __ldg(values.norm + row0 + r);
+        p.rnm[i] = __ldg(values.rnorm + row0 + r);
+      }
     }
   };
   auto store_batch = [&](int nb, const Pref& p) {
@@ -282,16 +294,26 @@ k_attn_chunk128(const KParams P, const float* __restrict__ logits, const Packed 
       if (e < nb * cw32) sCodes[e / cw32][e % cw32] = p.cw[i];
     }
     if (tid < nb) sCodes[tid][cw32] = 0u;
-    if (prod && tid < nb * sw32) sSigns[tid / sw32][tid % sw32] = p.sg;
-    if (tid < nb * G) {
-      const int r = tid / G, q = tid - r * G;
-      float cq = cm[0];
 #pragma unroll
-      for (int qq = 1; qq < G; ++qq) cq = q == qq ? cm[qq] : cq;
-      const float w = exp2f(p.lgv * scale_log2 - cq);
-      sWn[r][q] = w * p.nrm;
-      sWr[r][q] = w * p.rnm;
-      lsum += w;
+    for (int i = 0; i < kSP; ++i) {
+      const int e = tid + i * kAttnThreads;
+      if (prod && e < nb * sw32) sSigns[e / sw32][e % sw32] = p.sg[i];
+    }
+    // every entry of a thread has the query tid % G (G divides 256 when kWP > 1)
+    const int q = tid % G;
+    float cq = cm[0];
+#pragma unroll
+    for (int qq = 1; qq < G; ++qq) cq = q == qq ? cm[qq] : cq;
+#pragma unroll
+    for (int i = 0; i < kWP; ++i) {
+      const int e = tid + i * kAttnThreads;
+      if (e < nb * G) {
+        const int r = e / G;
+        const float w = exp2f(p.lgv[i] * scale_log2 - cq);
+        sWn[r][q] = w * p.nrm[i];
+        sWr[r][q] = w * p.rnm[i];
+        lsum += w;
+      }
     }
   };
   Pref pf;
@@ -351,13 +373,13 @@ k_attn_chunk128(const KParams P, const float* __restrict__ logits, const Packed 
 #pragma unroll
     for (int q = 0; q < G; ++q) sHalf[role * 64 + pair][q] = acc[q];
   }
-  sRed[tid] = lsum;                                             // thread tid accumulated (key tid / G, query tid % G)
+  sRed[tid] = lsum;                                             // thread tid accumulated query tid % G
   __syncthreads();
   float* rec = partial + ((static_cast<int64_t>(set) * G) * n_chunks + c) * partial_floats(d, m);
   const int64_t qstride = static_cast<int64_t>(n_chunks) * partial_floats(d, m);
   if (tid < G) {
     float l = 0.f;
-    for (int t = tid; t < KB * G && t < kAttnThreads; t += G) l += sRed[t];
+    for (int t = tid; t < kAttnThreads; t += G) l += sRed[t];
     rec[tid * qstride + 0] = cm[tid];
     rec[tid * qstride + 1] = l;
   }
