@@ -11,6 +11,8 @@ claims the kernels rest on against the oracle:
   * the estimates from [c_hi | c_lo | z] x [q_hi | q_lo | sq_hi | sq_lo] with
     the three MSE products c_hi q_hi + c_lo q_hi + c_hi q_lo stay far inside
     the 1e-4 |q| |k| logit tolerance.
+A third check covers the d = 128 logits kernel's centroid byte planes for
+3-bit codes (16-bit fixed point, high and low byte).
 The emulation is independent of the CUDA sources: it restates the operand
 construction from its definition, not from the kernels.
 """
@@ -89,3 +91,34 @@ def test_estimate_decomposition_within_the_logit_tolerance(d, b, m):
     want = ot.logits(qq, pk, P, 1, 40, 200)[0]
     tol = parity.logit_tolerance(qq, np.linalg.norm(k, axis=1), 1, 40, 200)[0]
     assert np.all(np.abs(est - want) <= 1e-2 * tol)
+
+
+def test_centroid_byte_planes_within_the_logit_tolerance():
+    """The d = 128 warp-specialized logits kernel takes 3-bit codes' centroids as
+    the high and low byte of round(c s), s = 32767 / max |c| (a signed high byte
+    and an unsigned low byte).  Restated from that definition: the two bytes
+    recompose the fixed-point value exactly, each centroid moves by at most
+    max |c| / 65534, and the MSE term of the estimator moves by far less than
+    the 1e-4 |q| |k| logit tolerance -- also in the worst case, max |delta| times
+    ||q||_1 <= max |delta| sqrt(d) |q|."""
+    d, b, m = 128, 4, 128
+    P = op.Params(d, b, m, seed=0)
+    c = P.centroids
+    s = 32767.0 / np.abs(c).max()
+    fx = np.clip(np.rint(c * s), -32767, 32767).astype(np.int64)
+    hi, lo = fx >> 8, fx & 0xFF
+    assert np.all((-128 <= hi) & (hi <= 127)) and np.all((0 <= lo) & (lo <= 255))
+    assert np.array_equal(256 * hi + lo, fx)
+    delta = fx / s - c
+    assert np.abs(delta).max() <= np.abs(c).max() / 65534 * (1 + 1e-12)
+    worst = np.abs(delta).max() * np.sqrt(d)          # per unit |q| |k| (unit-norm rotated keys)
+    assert worst < 3.4e-5 < 1e-4
+    rng = np.random.default_rng(11)
+    k = rng.standard_normal((500, d)) * rng.uniform(0.1, 10, size=(500, 1))
+    pk = ot.quantize(k, P)
+    code = ot.unpack_codes(pk["codes"], d, P.B)
+    qq = rng.standard_normal((64, d))
+    q_rot, _ = ot.query_prep(qq, P)
+    moved = (q_rot @ delta[code].T) * pk["norm"][None, :]    # change of the MSE term
+    tol = 1e-4 * np.linalg.norm(qq, axis=1)[:, None] * np.linalg.norm(k, axis=1)[None, :]
+    assert np.all(np.abs(moved) <= 0.34 * tol)
